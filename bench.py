@@ -1,0 +1,321 @@
+#!/usr/bin/env python
+"""Benchmark of the routed-MoE layer stack: 30-layer batch-1 decode.
+
+Workload (decode_30L_b1): 30 independent layers of H=2816, E=128 routed
+experts (top 8), expert I=704, shared expert Is=2112; MLX-style affine 4-bit
+group-64 experts (12.85 GB of routed weights resident in HBM), 8-bit router,
+Zipf(1.1) per-layer routing skew.  One step = one fresh token through all 30
+layers (RMS norm, router + top-8, routed experts, shared expert, combine,
+residual add).  Synthetic seeded weights and inputs.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs one process per GPU (torchrun), each an independent replica on its
+own token stream (no collective on the data path); `value` sums all ranks.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import gen  # noqa: E402
+
+CFG = gen.CONFIGS["decode_30L_b1"]
+METRIC = "MoE tokens/s (30-layer decode b=1)"
+FALLBACK_HBM = 6650.0
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM, "fallback"
+
+
+def step_bytes(cfg, distinct_per_layer: float) -> float:
+    """Algorithmic weight bytes of one step: per layer the router, the shared
+    expert and every distinct routed expert touched, read once."""
+    router = cfg.E * cfg.H + 2 * 2 * cfg.E * (cfg.H // 64)
+    blob = gen.blob_bytes(cfg.H, cfg.I)
+    shared = sum(gen.qmat_bytes(o, i) for o, i in ((cfg.Is, cfg.H), (cfg.Is, cfg.H), (cfg.H, cfg.Is)))
+    return cfg.layers * (router + shared) + distinct_per_layer * cfg.layers * blob
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm = [float(r[1]) for r in rows if len(r) >= 9 and r[1].strip().replace(".", "").isdigit()]
+        if not sm:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.strip() == "Active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def load_stack(cfg, device, rank):
+    import torch
+    from quantized_moe_bit_b200.weights import upload_layer
+    layers = []
+    t0 = time.time()
+    stride = gen.synth.default_blob_stride(cfg.H, cfg.I)
+    host = np.empty((cfg.E, stride), dtype=np.uint8)
+    for l in range(cfg.layers):
+        router = gen.router_weights(cfg.seed, l, cfg.E, cfg.H)
+        bias = gen.zipf_bias(cfg.seed, l, cfg.E) if cfg.zipf else None
+        shared = gen.shared_weights(cfg.seed, l, cfg.H, cfg.Is)
+        gen.layer_blobs(cfg.seed, l, cfg.E, cfg.H, cfg.I, stride, out=host, threads=16)
+        layers.append(upload_layer(router, bias, shared, host, device))
+    torch.cuda.synchronize()
+    log(f"[rank {rank}] weights: {cfg.layers} layers in {time.time() - t0:.1f}s")
+    return layers
+
+
+def cpu_baseline_oracle(cfg, n_layers: int, stream: int):
+    """Time the fp64 oracle on one token through the first n_layers layers."""
+    from oracle import moe_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    z = gen.rows(cfg.seed, stream, 1, cfg.H).astype(np.float64)
+    layers = []
+    for l in range(n_layers):
+        layers.append((gen.router_weights(cfg.seed, l, cfg.E, cfg.H),
+                       gen.zipf_bias(cfg.seed, l, cfg.E) if cfg.zipf else None,
+                       (lambda l_: (lambda e: gen.expert_weights(cfg.seed, l_, e, cfg.H, cfg.I)))(l),
+                       gen.shared_weights(cfg.seed, l, cfg.H, cfg.Is)))
+    t0 = time.perf_counter()
+    O.stack_forward(z, layers, cfg.k, cfg.E)
+    dt = time.perf_counter() - t0
+    tok_s = 1.0 / (dt * cfg.layers / n_layers)
+    return tok_s, cores, dt
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    per_step_layers = 1
+    times = []
+    cores = None
+    for i in range(args.warmup + args.steps):
+        tok_s, cores, dt = cpu_baseline_oracle(CFG, per_step_layers, 1000 + i)
+        if i >= args.warmup:
+            times.append(dt)
+    tot = sum(times)
+    value = args.steps / (tot * CFG.layers / per_step_layers)
+    sample = (f"each step: one token through the first {per_step_layers} of 30 layers (oracle, fp64 numpy, "
+              f"expert weights generated inside the timed call), time scaled by 30/{per_step_layers}")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps * CFG.layers / per_step_layers,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "decode_30L_b1", "layers": 30, "batch": 1, "H": CFG.H, "E": CFG.E, "k": CFG.k,
+                       "I": CFG.I, "Is": CFG.Is},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import quantized_moe_bit_b200 as M
+
+    cfg = CFG
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    layers = load_stack(cfg, device, rank)
+    stack = M.DecodeStack(layers)
+    H = cfg.H
+    n_in = args.warmup + args.steps
+    base_stream = 1000 + rank * 100000
+    z = np.concatenate([gen.rows(cfg.seed, base_stream + s, 1, H) for s in range(n_in)])  # [n_in, H]
+    z_dev = torch.from_numpy(z).to(device).view(n_in, 1, H)
+    ws = torch.empty(M.moe_decode_workspace_size(1, H, cfg.I, cfg.Is, cfg.E, cfg.k), dtype=torch.uint8,
+                     device=device)
+    h = torch.empty((1, H), dtype=torch.float32, device=device)
+    idx_tr = torch.empty((cfg.layers, 1, cfg.k), dtype=torch.int32, device=device)
+
+    def step():
+        M.moe_decode_forward(h, cfg.I, cfg.Is, cfg.E, cfg.k, stack, ws, idx_trace=idx_tr)
+
+    # eager warm-up (sets kernel attributes), then capture one step in a graph
+    h.copy_(z_dev[0])
+    step()
+    torch.cuda.synchronize()
+    M.moe_sync()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            step()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+
+    distinct = []
+    for i in range(args.warmup):
+        h.copy_(z_dev[i])
+        g.replay()
+    torch.cuda.synchronize()
+    M.moe_sync()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        h.copy_(z_dev[args.warmup + i])
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    idx_last = idx_tr.cpu().numpy()
+    distinct = float(np.mean([len(set(idx_last[l, 0].tolist())) for l in range(cfg.layers)]))
+
+    # end to end through the public call: pinned host input -> step -> host result
+    zh = torch.from_numpy(z[args.warmup:]).pin_memory().view(args.steps, 1, H)
+    out_h = torch.empty((args.steps, 1, H), dtype=torch.float32).pin_memory()
+    torch.cuda.synchronize()
+    barrier()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record()
+    for i in range(args.steps):
+        h.copy_(zh[i], non_blocking=True)
+        g.replay()
+        out_h[i].copy_(h, non_blocking=True)
+    e3.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = e2.elapsed_time(e3)
+    M.moe_sync()
+
+    t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms, ms_e2e = float(t[0]), float(t[1])
+    del g
+    if rank != 0:
+        return
+    tokens = args.steps * world
+    value = tokens / (ms / 1e3)
+    e2e_val = tokens / (ms_e2e / 1e3)
+    hbm, src = peaks()
+    bytes_step = step_bytes(cfg, distinct)
+    achieved = bytes_step / (ms / args.steps / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16xf16->f32", "data": "synthetic",
+        "config": {"workload": "decode_30L_b1", "layers": cfg.layers, "batch": 1, "H": cfg.H, "E": cfg.E,
+                   "k": cfg.k, "I": cfg.I, "Is": cfg.Is, "weights": "4-bit affine g64 experts, 8-bit router",
+                   "routing": "Zipf(1.1) per-layer bias", "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (1.1 GB of weights per step)"},
+        "roofline": {"bound": "hbm", "kernel": "decode step: all kernels of moe_decode_forward",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "peak_source": src, "traffic": None, "bytes_per_step": bytes_step,
+                     "distinct_experts_per_layer": distinct},
+        "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": H * 4, "d2h_bytes_per_step": H * 4},
+        "gpu_launches": M.moe_decode_launches(1, cfg.layers) * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        tok_s, cores, dt = cpu_baseline_oracle(cfg, 6, 999)
+        line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": f"one token through the first 6 of 30 layers ({dt:.1f} s), scaled by 5"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

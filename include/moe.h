@@ -1,0 +1,207 @@
+/*
+ * libmoe — routed Mixture-of-Experts layer with MLX-style affine 4-bit experts
+ * and an 8-bit router, for NVIDIA B200 (sm_100a).
+ *
+ * The layer (one step of a routed-MoE transformer block):
+ *   A0  x = bf16( h / sqrt(mean(h^2) + eps) )            layer-input RMS norm
+ *   A1  logits = W_r x + beta                             8-bit affine router
+ *   A2  idx = top-k(logits), gates = softmax(logits[idx])
+ *   A3  pairs (t, j) grouped by expert
+ *   A4  act = gelu_tanh(W_g x) * (W_u x)                  per (token, expert) pair
+ *   A5  y_pair = W_d act
+ *   A6  ysh = W_sd (gelu_tanh(W_sg x) * (W_su x))         always-on shared expert
+ *   A7  y = sum_j gates_j * y_pair_j + ysh                (then h += y between layers)
+ *
+ * Passages defining the operations:
+ *   "TurboFieldfare: Gemma 4 26B on an 8 GB MacBook, in ~2 GB of RAM"
+ *   (blog-mushroom.pages.dev), section "Why 26B Fits in 2 GB": 8 of 128 experts
+ *   per token and layer; the shared-expert branch runs while expert blobs are
+ *   fetched and the two outputs are merged; a 16-slot LFU per layer; prefill in
+ *   chunks of up to 128 rows so that one expert blob serves the chunk.
+ *   "TurboFieldfareとは｜26BのGemma 4を約2GBのRAMで動かすSwift製ランタイムの実像"
+ *   (ai-heartland.com), section "TurboFieldfareとは": MLX affine 4-bit, group 64,
+ *   bf16 scale and bias; 8-bit router; 4-bit shared and routed experts.
+ *   The softmax over the top-k logits, the gelu_tanh GeGLU, the ungated
+ *   shared expert and the eps = 1e-6 norm without weight are this library's
+ *   definition of the layer; the pages do not state them.
+ *
+ * Conventions (every call):
+ *   - Return an int status (moe_status).  No call aborts or exits.
+ *     moe_last_error_string() gives detail for the calling thread.
+ *   - Pointers documented "device" are CUDA device pointers owned by the
+ *     caller; the library never allocates device memory in these calls.
+ *     Scratch comes from caller workspaces sized by the *_workspace_size calls.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous on it; errors of a kernel surface at a later call or at
+ *     moe_sync().
+ *   - bf16 / fp16 values are passed as uint16_t bit patterns.
+ *   - Dimensions: H, I, Is multiples of 64; E a multiple of 8, E <= 1024;
+ *     1 <= k <= 8 and k <= E.  Device pointers 16-byte aligned.
+ *
+ * Quantised matrix [out, in] (moe_qmat): w[r,c] = S[r,c/64] * q[r,c] + B[r,c/64]
+ *   q  uint32 [out, in*bits/32], element c at bit bits*(c % (32/bits)) of word
+ *      c / (32/bits) (low bits first)
+ *   s  bf16   [out, in/64]    b  bf16 [out, in/64]
+ *   bits = 4 for experts, 8 for the router.
+ *
+ * Expert blob (routed expert, bytes, contiguous, 16-byte aligned):
+ *   gate.q gate.s gate.b | up.q up.s up.b | down.q down.s down.b
+ *   with gate, up = [I, H] and down = [H, I], 4-bit; blob_bytes = 3*(I*H/2 + 4*I*H/64).
+ *   A routed layer is given as a device array of E blob pointers, so blobs may
+ *   live anywhere (one allocation with a fixed stride, or cache slots).
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* bad size, NULL pointer or misalignment; nothing launched */
+  MOE_ERR_CUDA = 2,          /* a CUDA runtime call or launch failed */
+  MOE_ERR_TIMEOUT = 3,       /* a bounded host wait ran out */
+  MOE_ERR_DEVICE_CHECK = 4,  /* a kernel found an out-of-range index and skipped it */
+  MOE_ERR_UNSUPPORTED = 5    /* valid request this build does not serve */
+} moe_status;
+
+typedef struct moe_qmat {
+  const uint32_t* q;   /* device */
+  const uint16_t* s;   /* device, bf16 */
+  const uint16_t* b;   /* device, bf16 */
+  int32_t out;
+  int32_t in;
+  int32_t bits;        /* 4 or 8 */
+} moe_qmat;
+
+/* Detail of the last non-OK status on this thread (static storage). */
+MOE_API const char* moe_last_error_string(void);
+/* Library version (major*10000 + minor*100 + patch). */
+MOE_API int moe_version(void);
+/* Synchronise `stream`, then report CUDA errors and the device check word
+ * (MOE_ERR_DEVICE_CHECK if a kernel skipped an out-of-range index since the
+ * last moe_sync; the word is cleared). */
+MOE_API int moe_sync(void* stream);
+
+/* Bytes of one expert blob and its offsets: offsets[9] receives the byte
+ * offsets of gate.q gate.s gate.b up.q up.s up.b down.q down.s down.b. */
+MOE_API size_t moe_blob_bytes(int H, int I, size_t* offsets9);
+
+/* A0 — layer-input RMS norm.  h fp32 [T,H] (device) -> x bf16 [T,H] (device):
+ * x = bf16_rn(h / sqrt(mean(h^2) + eps)), sum of squares in fp32, fixed order. */
+MOE_API int moe_rmsnorm(const float* h, int T, int H, float eps, uint16_t* x, void* stream);
+
+/* A1 + A2 — router and top-k.
+ *   x       bf16 [T,H] (device)
+ *   router  8-bit q-matrix [E,H] (host struct of device pointers)
+ *   bias    fp32 [E] (bias_per_row = 0) or [T,E] (bias_per_row = 1) or NULL (device)
+ *   idx     int32 [T,k] (device): the k largest logits, descending; an exact
+ *           tie goes to the lower expert id
+ *   gates   fp32 [T,k] (device): softmax over the k selected logits
+ *   logits_opt fp32 [T,E] (device) or NULL: logits including the bias
+ * Logits are accumulated in fp32.  Runs as clusters of 8 CTAs per block of
+ * rows; the top-k reads the logits through distributed shared memory. */
+MOE_API int moe_router_topk(const uint16_t* x, int T, int H, const moe_qmat* router,
+                    const float* bias, int bias_per_row, int E, int k,
+                    int32_t* idx, float* gates, float* logits_opt, void* stream);
+
+/* A3 — bucketing (stable counting sort of the T*k pairs by expert).
+ *   idx      int32 [T,k] (device)
+ *   offsets  int32 [E+1] (device): bucket e is pairs[offsets[e] .. offsets[e+1])
+ *   pairs    int32 [T*k] (device): value t*k + j, t then j ascending inside a bucket
+ *   active   int32 [E]   (device): experts with a non-empty bucket, ascending
+ *   n_active int32 [1]   (device)
+ * Requires T*k <= 65536.  Out-of-range ids are skipped and flagged. */
+MOE_API int moe_bucket(const int32_t* idx, int T, int k, int E, int32_t* offsets,
+               int32_t* pairs, int32_t* active, int32_t* n_active, void* stream);
+
+/* A4 + A5 — routed experts for every pair.
+ *   x          bf16 [T,H] (device)
+ *   blob_ptrs  device array [E] of device pointers to expert blobs
+ *   offsets, pairs, active, n_active   from moe_bucket (device)
+ *   y_pairs    fp32 [T*k, H] (device): row t*k + j = expert idx[t,j] applied to x[t]
+ *   ws         device workspace of at least moe_expert_workspace_size(T,H,I,k) bytes
+ * Each expert runs on the decode GEMV kernels (CUDA cores) when its bucket has
+ * at most gemv_max_rows rows (moe_set_gemv_max_rows; default 2) and on the
+ * tcgen05 grouped GEMM otherwise.  The choice depends only on the bucket's
+ * row count.  The activation between the two projections is held in fp16. */
+MOE_API size_t moe_expert_workspace_size(int T, int H, int I, int k);
+MOE_API int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, int k,
+                       const void* const* blob_ptrs, const int32_t* offsets,
+                       const int32_t* pairs, const int32_t* active,
+                       const int32_t* n_active, float* y_pairs,
+                       void* ws, size_t ws_bytes, void* stream);
+/* Bucket-size threshold between the GEMV and the tensor-core path (>= 0). */
+MOE_API int moe_set_gemv_max_rows(int rows);
+
+/* A6 — shared expert on every row.
+ *   shared  host array of 3 q-matrices: gate [Is,H], up [Is,H], down [H,Is]
+ *   ysh     fp32 [T,H] (device)
+ *   ws      device workspace of at least moe_shared_workspace_size(T,H,Is) bytes */
+MOE_API size_t moe_shared_workspace_size(int T, int H, int Is);
+MOE_API int moe_shared_forward(const uint16_t* x, int T, int H, int Is, const moe_qmat* shared,
+                       float* ysh, void* ws, size_t ws_bytes, void* stream);
+
+/* A7 — combine.  y[t] = sum_{j=0..k-1} gates[t,j] * y_pairs[t*k+j] + ysh[t],
+ * summed in fp32 in that order; y bf16 [T,H] (device, may be NULL);
+ * residual_inout fp32 [T,H] (device) or NULL: residual += the fp32 sum. */
+MOE_API int moe_combine(const float* y_pairs, const float* gates, const float* ysh,
+                int T, int H, int k, uint16_t* y, float* residual_inout, void* stream);
+
+/* One whole layer, A0 (optional) to A7, through the calls above.
+ *   h_in     fp32 [T,H] (device) residual stream or NULL; when x_in is NULL the
+ *            layer input is its RMS norm (A0, eps = 1e-6)
+ *   h_out    fp32 [T,H] (device) or NULL: receives h_in + y (fp32, before the
+ *            bf16 rounding of y); may equal h_in
+ *   x_in     bf16 [T,H] (device) layer input used instead of the norm of h_in
+ *            when non-NULL
+ *   x_out    bf16 [T,H] (device) or NULL: the layer input actually used
+ *   y        bf16 [T,H] (device) or NULL: the layer output
+ *   idx, gates  int32/fp32 [T,k] (device) or NULL: the routing used
+ *   blob_ptrs   device array [E] of blob pointers
+ *   ws       device workspace of at least moe_layer_workspace_size(...) bytes */
+MOE_API size_t moe_layer_workspace_size(int T, int H, int I, int Is, int E, int k);
+MOE_API int moe_layer_forward(const float* h_in, float* h_out, const uint16_t* x_in, int T, int H,
+                      int I, int Is, int E, int k, const moe_qmat* router,
+                      const float* bias, int bias_per_row, const void* const* blob_ptrs,
+                      const moe_qmat* shared, uint16_t* x_out, uint16_t* y,
+                      int32_t* idx, float* gates, void* ws, size_t ws_bytes, void* stream);
+
+/* A whole decode/prefill step through L stacked layers (A0 .. A7 per layer,
+ * residual add between layers): for l = 0 .. L-1
+ *   x_l = rmsnorm(h); h += layer_l(x_l)
+ *   h          fp32 [T,H] (device), updated in place (the step input on entry,
+ *              the residual stream after the last layer on return)
+ *   routers    host array [L] of 8-bit router q-matrices [E,H]
+ *   biases     host array [L] of device fp32 pointers ([E] or, with
+ *              bias_per_row, [T,E]) or NULL entries / NULL array for none
+ *   blob_tables host array [L] of device arrays [E] of expert-blob pointers
+ *   shared     host array [L*3] of shared-expert q-matrices
+ *   x_trace, y_trace   bf16 [L,T,H] (device) or NULL: every layer's input/output
+ *   idx_trace, gates_trace  int32/fp32 [L,T,k] (device) or NULL
+ *   ws         device workspace of at least moe_decode_workspace_size(...) bytes
+ * Layers run in order on `stream`. */
+MOE_API size_t moe_decode_workspace_size(int T, int H, int I, int Is, int E, int k);
+/* Number of kernels one moe_decode_forward(T, L) call launches. */
+MOE_API int moe_decode_launches(int T, int L);
+MOE_API int moe_decode_forward(float* h, int T, int H, int I, int Is, int E, int k, int L,
+                               const moe_qmat* routers, const float* const* biases,
+                               int bias_per_row, const void* const* const* blob_tables,
+                               const moe_qmat* shared, uint16_t* x_trace, uint16_t* y_trace,
+                               int32_t* idx_trace, float* gates_trace, void* ws,
+                               size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

@@ -1,0 +1,355 @@
+// C-ABI of libmoe: argument checks, workspace carving and kernel launches.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "gemv.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+static thread_local char g_err[512] = "";
+static int g_gemv_max_rows = 2;
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_check(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return MOE_OK;
+}
+
+int launch_check(const char* what) { return cuda_check(cudaGetLastError(), what); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static size_t align_up(size_t n, size_t a = 256) { return (n + a - 1) / a * a; }
+
+static void blob_offsets(int H, int I, size_t off[9]) {
+  const size_t q = static_cast<size_t>(I) * H / 2, s = static_cast<size_t>(I) * (H / 64) * 2;
+  size_t o = 0;
+  for (int m = 0; m < 3; ++m) {
+    off[3 * m + 0] = o; o += q;
+    off[3 * m + 1] = o; o += s;
+    off[3 * m + 2] = o; o += s;
+  }
+}
+
+static int check_dims(int T, int H, int I, int E, int k) {
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0 (got %d)", T);
+  if (H <= 0 || H % 64) return fail(MOE_ERR_INVALID_ARG, "H must be a positive multiple of 64 (got %d)", H);
+  if (I <= 0 || I % 64) return fail(MOE_ERR_INVALID_ARG, "I must be a positive multiple of 64 (got %d)", I);
+  if (E <= 0 || E % 8 || E > 1024) return fail(MOE_ERR_INVALID_ARG, "E must be a multiple of 8 in [8, 1024] (got %d)", E);
+  if (k < 1 || k > 8 || k > E) return fail(MOE_ERR_INVALID_ARG, "k must be in [1, min(8, E)] (got %d)", k);
+  return MOE_OK;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per (device, kernel);
+// later calls (also inside stream capture) find it done and make no API call.
+static int set_smem(const void* fn, size_t bytes) {
+  if (bytes <= 48 * 1024) return MOE_OK;
+  struct Entry { const void* fn; int dev; size_t bytes; };
+  static Entry table[64];
+  static int n = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  for (int i = 0; i < n; ++i)
+    if (table[i].fn == fn && table[i].dev == dev && table[i].bytes >= bytes) return MOE_OK;
+  int st = cuda_check(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(bytes)),
+                      "cudaFuncSetAttribute(smem)");
+  if (st) return st;
+  for (int i = 0; i < n; ++i)
+    if (table[i].fn == fn && table[i].dev == dev) { table[i].bytes = bytes; return MOE_OK; }
+  if (n < 64) table[n++] = Entry{fn, dev, bytes};
+  return MOE_OK;
+}
+
+static size_t gemv_smem(int K) {
+  return GEMV_RG * staged_row_bytes(K) + static_cast<size_t>(GEMV_RG) * (K / 8) * sizeof(float2);
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_last_error_string(void) { return g_err; }
+
+int moe_version(void) { return 100; }
+
+int moe_sync(void* stream) {
+  int st = cuda_check(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)), "moe_sync");
+  if (st) return st;
+  unsigned int w = 0;
+  st = cuda_check(cudaMemcpyFromSymbol(&w, g_check_word, sizeof(w)), "read check word");
+  if (st) return st;
+  if (w != 0) {
+    unsigned int z = 0;
+    cudaMemcpyToSymbol(g_check_word, &z, sizeof(z));
+    return fail(MOE_ERR_DEVICE_CHECK, "device check word 0x%x (1: expert id, 2: pair id, 4: wait)", w);
+  }
+  return MOE_OK;
+}
+
+size_t moe_blob_bytes(int H, int I, size_t* offsets9) {
+  if (H <= 0 || I <= 0 || H % 64 || I % 64) return 0;
+  size_t off[9];
+  blob_offsets(H, I, off);
+  if (offsets9) memcpy(offsets9, off, sizeof(off));
+  return 3 * (static_cast<size_t>(I) * H / 2 + static_cast<size_t>(I) * (H / 64) * 4);
+}
+
+int moe_set_gemv_max_rows(int rows) {
+  if (rows < 0) return fail(MOE_ERR_INVALID_ARG, "gemv_max_rows must be >= 0");
+  g_gemv_max_rows = rows;
+  return MOE_OK;
+}
+
+int moe_rmsnorm(const float* h, int T, int H, float eps, uint16_t* x, void* stream) {
+  if (T < 0 || H <= 0 || H % 64) return fail(MOE_ERR_INVALID_ARG, "moe_rmsnorm: bad T/H");
+  if (T == 0) return MOE_OK;
+  if (!h || !x || !aligned16(h) || !aligned16(x)) return fail(MOE_ERR_INVALID_ARG, "moe_rmsnorm: bad pointer");
+  k_rmsnorm<<<T, 256, 0, static_cast<cudaStream_t>(stream)>>>(h, H, eps, x);
+  return launch_check("k_rmsnorm");
+}
+
+int moe_router_topk(const uint16_t* x, int T, int H, const moe_qmat* router, const float* bias,
+                    int bias_per_row, int E, int k, int32_t* idx, float* gates, float* logits_opt,
+                    void* stream) {
+  int st = check_dims(T, H, 64, E, k);
+  if (st) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !router || !idx || !gates || !router->q || !router->s || !router->b)
+    return fail(MOE_ERR_INVALID_ARG, "moe_router_topk: NULL pointer");
+  if (router->bits != 8 || router->out != E || router->in != H)
+    return fail(MOE_ERR_INVALID_ARG, "moe_router_topk: router must be 8-bit [E=%d, H=%d]", E, H);
+  if (!aligned16(x) || !aligned16(router->q)) return fail(MOE_ERR_INVALID_ARG, "moe_router_topk: misaligned");
+  const size_t smem = router_smem_bytes(H, E);
+  if (smem > 227 * 1024) return fail(MOE_ERR_UNSUPPORTED, "moe_router_topk: H=%d E=%d too large", H, E);
+  st = set_smem(reinterpret_cast<const void*>(k_router_topk), smem);
+  if (st) return st;
+  const int nblk = (T + ROUTER_TB - 1) / ROUTER_TB;
+  k_router_topk<<<nblk * 8, 256, smem, static_cast<cudaStream_t>(stream)>>>(
+      x, T, H, router->q, router->s, router->b, bias, bias_per_row, E, k, idx, gates, logits_opt);
+  return launch_check("k_router_topk");
+}
+
+int moe_bucket(const int32_t* idx, int T, int k, int E, int32_t* offsets, int32_t* pairs,
+               int32_t* active, int32_t* n_active, void* stream) {
+  int st = check_dims(T, 64, 64, E, k);
+  if (st) return st;
+  if (static_cast<long>(T) * k > 65536) return fail(MOE_ERR_UNSUPPORTED, "moe_bucket: T*k > 65536");
+  if (!idx || !offsets || !pairs || !active || !n_active) return fail(MOE_ERR_INVALID_ARG, "moe_bucket: NULL pointer");
+  k_bucket<<<1, 256, 2 * E * sizeof(int), static_cast<cudaStream_t>(stream)>>>(idx, T * k, E, offsets, pairs,
+                                                                              active, n_active);
+  return launch_check("k_bucket");
+}
+
+size_t moe_expert_workspace_size(int T, int H, int I, int k) {
+  (void)H;
+  return align_up(static_cast<size_t>(T) * k * I * sizeof(__half));
+}
+
+int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, int k, const void* const* blob_ptrs,
+                       const int32_t* offsets, const int32_t* pairs, const int32_t* active,
+                       const int32_t* n_active, float* y_pairs, void* ws, size_t ws_bytes, void* stream) {
+  int st = check_dims(T, H, I, E, k);
+  if (st) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !blob_ptrs || !offsets || !pairs || !active || !n_active || !y_pairs || !ws)
+    return fail(MOE_ERR_INVALID_ARG, "moe_expert_forward: NULL pointer");
+  if (ws_bytes < moe_expert_workspace_size(T, H, I, k))
+    return fail(MOE_ERR_INVALID_ARG, "moe_expert_forward: workspace too small");
+  if (!aligned16(x) || !aligned16(ws) || !aligned16(y_pairs))
+    return fail(MOE_ERR_INVALID_ARG, "moe_expert_forward: misaligned pointer");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  __half* act = static_cast<__half*>(ws);
+  const int maxA = T * k < E ? T * k : E;
+
+  GateUpArgs g{};
+  g.x = x; g.T = T; g.H = H; g.I = I; g.E = E; g.k = k;
+  g.blob_ptrs = blob_ptrs; g.offsets = offsets; g.pairs = pairs; g.active = active; g.n_active = n_active;
+  g.max_rows = 1 << 30;
+  blob_offsets(H, I, g.off);
+  g.act = act;
+  size_t sm = gemv_smem(H);
+  if ((st = set_smem(reinterpret_cast<const void*>(k_gateup_gemv), sm))) return st;
+  k_gateup_gemv<<<dim3((I + GEMV_ROWS - 1) / GEMV_ROWS, maxA), 256, sm, s>>>(g);
+  if ((st = launch_check("k_gateup_gemv"))) return st;
+
+  DownArgs d{};
+  d.act = act; d.T = T; d.H = H; d.I = I; d.E = E; d.k = k;
+  d.blob_ptrs = blob_ptrs; d.offsets = offsets; d.pairs = pairs; d.active = active; d.n_active = n_active;
+  d.max_rows = 1 << 30;
+  blob_offsets(H, I, d.off);
+  d.y = y_pairs;
+  sm = gemv_smem(I);
+  if ((st = set_smem(reinterpret_cast<const void*>(k_down_gemv), sm))) return st;
+  k_down_gemv<<<dim3((H + GEMV_ROWS - 1) / GEMV_ROWS, maxA), 256, sm, s>>>(d);
+  return launch_check("k_down_gemv");
+}
+
+size_t moe_shared_workspace_size(int T, int H, int Is) {
+  (void)H;
+  return align_up(static_cast<size_t>(T) * Is * sizeof(__half));
+}
+
+int moe_shared_forward(const uint16_t* x, int T, int H, int Is, const moe_qmat* sh, float* ysh, void* ws,
+                       size_t ws_bytes, void* stream) {
+  int st = check_dims(T, H, Is, 8, 1);
+  if (st) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !sh || !ysh || !ws) return fail(MOE_ERR_INVALID_ARG, "moe_shared_forward: NULL pointer");
+  for (int m = 0; m < 3; ++m) {
+    const int out = m < 2 ? Is : H, in = m < 2 ? H : Is;
+    if (!sh[m].q || !sh[m].s || !sh[m].b || sh[m].bits != 4 || sh[m].out != out || sh[m].in != in)
+      return fail(MOE_ERR_INVALID_ARG, "moe_shared_forward: matrix %d must be 4-bit [%d, %d]", m, out, in);
+    if (!aligned16(sh[m].q)) return fail(MOE_ERR_INVALID_ARG, "moe_shared_forward: misaligned weights");
+  }
+  if (ws_bytes < moe_shared_workspace_size(T, H, Is))
+    return fail(MOE_ERR_INVALID_ARG, "moe_shared_forward: workspace too small");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  __half* act = static_cast<__half*>(ws);
+  GateUpArgs g{};
+  g.x = x; g.T = T; g.H = H; g.I = Is; g.E = 1; g.k = 1; g.max_rows = 1 << 30;
+  g.gq = sh[0].q; g.gs = sh[0].s; g.gb = sh[0].b;
+  g.uq = sh[1].q; g.us = sh[1].s; g.ub = sh[1].b;
+  g.act = act;
+  size_t sm = gemv_smem(H);
+  if ((st = set_smem(reinterpret_cast<const void*>(k_gateup_gemv), sm))) return st;
+  k_gateup_gemv<<<dim3((Is + GEMV_ROWS - 1) / GEMV_ROWS, 1), 256, sm, s>>>(g);
+  if ((st = launch_check("k_gateup_gemv(shared)"))) return st;
+  DownArgs d{};
+  d.act = act; d.T = T; d.H = H; d.I = Is; d.E = 1; d.k = 1; d.max_rows = 1 << 30;
+  d.dq = sh[2].q; d.ds = sh[2].s; d.db = sh[2].b;
+  d.y = ysh;
+  sm = gemv_smem(Is);
+  if ((st = set_smem(reinterpret_cast<const void*>(k_down_gemv), sm))) return st;
+  k_down_gemv<<<dim3((H + GEMV_ROWS - 1) / GEMV_ROWS, 1), 256, sm, s>>>(d);
+  return launch_check("k_down_gemv(shared)");
+}
+
+int moe_combine(const float* y_pairs, const float* gates, const float* ysh, int T, int H, int k, uint16_t* y,
+                float* residual_inout, void* stream) {
+  if (T < 0 || H <= 0 || k < 1 || k > 8) return fail(MOE_ERR_INVALID_ARG, "moe_combine: bad T/H/k");
+  if (T == 0) return MOE_OK;
+  if (!y_pairs || !gates) return fail(MOE_ERR_INVALID_ARG, "moe_combine: NULL pointer");
+  k_combine<<<dim3((H + 255) / 256, T), 256, 0, static_cast<cudaStream_t>(stream)>>>(y_pairs, gates, ysh, H, k, y,
+                                                                                 residual_inout);
+  return launch_check("k_combine");
+}
+
+size_t moe_layer_workspace_size(int T, int H, int I, int Is, int E, int k) {
+  size_t n = 0;
+  n += align_up(static_cast<size_t>(T) * H * 2);        // x
+  n += align_up(static_cast<size_t>(T) * k * 4) * 2;    // idx, gates
+  n += align_up(static_cast<size_t>(E + 1) * 4);        // offsets
+  n += align_up(static_cast<size_t>(T) * k * 4);        // pairs
+  n += align_up(static_cast<size_t>(E) * 4);            // active
+  n += align_up(4);                                     // n_active
+  n += align_up(static_cast<size_t>(T) * k * H * 4);    // y_pairs
+  n += align_up(static_cast<size_t>(T) * H * 4);        // ysh
+  n += moe_expert_workspace_size(T, H, I, k);
+  n += moe_shared_workspace_size(T, H, Is);
+  return n;
+}
+
+int moe_layer_forward(const float* h_in, float* h_out, const uint16_t* x_in, int T, int H, int I, int Is, int E,
+                      int k, const moe_qmat* router, const float* bias, int bias_per_row,
+                      const void* const* blob_ptrs, const moe_qmat* shared, uint16_t* x_out, uint16_t* y,
+                      int32_t* idx_out, float* gates_out, void* ws, size_t ws_bytes, void* stream) {
+  int st = check_dims(T, H, I, E, k);
+  if (st) return st;
+  if (T == 0) return MOE_OK;
+  if (!x_in && !h_in) return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward: need h_in or x_in");
+  if (h_out && !h_in) return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward: h_out needs h_in");
+  if (!ws || ws_bytes < moe_layer_workspace_size(T, H, I, Is, E, k))
+    return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward: workspace too small");
+  char* p = static_cast<char*>(ws);
+  auto take = [&](size_t n) { char* q = p; p += align_up(n); return q; };
+  uint16_t* x = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(T) * H * 2));
+  int32_t* idx = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * k * 4));
+  float* gates = reinterpret_cast<float*>(take(static_cast<size_t>(T) * k * 4));
+  int32_t* offsets = reinterpret_cast<int32_t*>(take(static_cast<size_t>(E + 1) * 4));
+  int32_t* pairs = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * k * 4));
+  int32_t* active = reinterpret_cast<int32_t*>(take(static_cast<size_t>(E) * 4));
+  int32_t* n_active = reinterpret_cast<int32_t*>(take(4));
+  float* y_pairs = reinterpret_cast<float*>(take(static_cast<size_t>(T) * k * H * 4));
+  float* ysh = reinterpret_cast<float*>(take(static_cast<size_t>(T) * H * 4));
+  const size_t ews = moe_expert_workspace_size(T, H, I, k);
+  void* ew = take(ews);
+  const size_t sws = moe_shared_workspace_size(T, H, Is);
+  void* sw = take(sws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  const uint16_t* xin = x_in;
+  if (!xin) {
+    if ((st = moe_rmsnorm(h_in, T, H, 1e-6f, x, stream))) return st;
+    xin = x;
+  }
+  if (x_out && (st = cuda_check(cudaMemcpyAsync(x_out, xin, static_cast<size_t>(T) * H * 2,
+                                                cudaMemcpyDeviceToDevice, s), "copy x_out")))
+    return st;
+  if ((st = moe_router_topk(xin, T, H, router, bias, bias_per_row, E, k, idx, gates, nullptr, stream))) return st;
+  if ((st = moe_bucket(idx, T, k, E, offsets, pairs, active, n_active, stream))) return st;
+  if ((st = moe_shared_forward(xin, T, H, Is, shared, ysh, sw, sws, stream))) return st;
+  if ((st = moe_expert_forward(xin, T, H, I, E, k, blob_ptrs, offsets, pairs, active, n_active, y_pairs, ew, ews,
+                               stream)))
+    return st;
+  float* resid = nullptr;
+  if (h_out) {
+    if (h_out != h_in &&
+        (st = cuda_check(cudaMemcpyAsync(h_out, h_in, static_cast<size_t>(T) * H * 4, cudaMemcpyDeviceToDevice, s),
+                         "copy h")))
+      return st;
+    resid = h_out;
+  }
+  if ((st = moe_combine(y_pairs, gates, ysh, T, H, k, y, resid, stream))) return st;
+  if (idx_out && (st = cuda_check(cudaMemcpyAsync(idx_out, idx, static_cast<size_t>(T) * k * 4,
+                                                  cudaMemcpyDeviceToDevice, s), "copy idx")))
+    return st;
+  if (gates_out && (st = cuda_check(cudaMemcpyAsync(gates_out, gates, static_cast<size_t>(T) * k * 4,
+                                                    cudaMemcpyDeviceToDevice, s), "copy gates")))
+    return st;
+  return MOE_OK;
+}
+
+int moe_decode_launches(int T, int L) {
+  // rmsnorm, router, bucket, shared gate/up, shared down, expert gate/up,
+  // expert down, combine per layer
+  return (T > 0 && L > 0) ? 8 * L : 0;
+}
+
+size_t moe_decode_workspace_size(int T, int H, int I, int Is, int E, int k) {
+  return moe_layer_workspace_size(T, H, I, Is, E, k);
+}
+
+int moe_decode_forward(float* h, int T, int H, int I, int Is, int E, int k, int L, const moe_qmat* routers,
+                       const float* const* biases, int bias_per_row, const void* const* const* blob_tables,
+                       const moe_qmat* shared, uint16_t* x_trace, uint16_t* y_trace, int32_t* idx_trace,
+                       float* gates_trace, void* ws, size_t ws_bytes, void* stream) {
+  int st = check_dims(T, H, I, E, k);
+  if (st) return st;
+  if (L < 0) return fail(MOE_ERR_INVALID_ARG, "moe_decode_forward: L < 0");
+  if (T == 0 || L == 0) return MOE_OK;
+  if (!h || !routers || !blob_tables || !shared) return fail(MOE_ERR_INVALID_ARG, "moe_decode_forward: NULL pointer");
+  const size_t TH = static_cast<size_t>(T) * H, Tk = static_cast<size_t>(T) * k;
+  for (int l = 0; l < L; ++l) {
+    const float* b = biases ? biases[l] : nullptr;
+    st = moe_layer_forward(h, h, nullptr, T, H, I, Is, E, k, &routers[l], b, bias_per_row, blob_tables[l],
+                           &shared[3 * l], x_trace ? x_trace + l * TH : nullptr, y_trace ? y_trace + l * TH : nullptr,
+                           idx_trace ? idx_trace + l * Tk : nullptr, gates_trace ? gates_trace + l * Tk : nullptr, ws,
+                           ws_bytes, stream);
+    if (st) return st;
+  }
+  return MOE_OK;
+}
+
+}  // extern "C"

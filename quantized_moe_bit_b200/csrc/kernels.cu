@@ -1,0 +1,355 @@
+// CUDA-core kernels of the routed-MoE layer: RMS norm (A0), router + top-k
+// (A1, A2), bucketing (A3), expert and shared-expert GEMVs (A4 - A6) and the
+// combine (A7).
+#include <cooperative_groups.h>
+
+#include "gemv.cuh"
+#include "kernels.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace moe {
+
+
+// ------------------------------------------------------------------------ A0
+// One block per row; fixed-order fp32 sum of squares; x = bf16_rn(h / r).
+__global__ void k_rmsnorm(const float* __restrict__ h, int H, float eps, uint16_t* __restrict__ x) {
+  const int t = blockIdx.x;
+  const float* row = h + static_cast<size_t>(t) * H;
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < H; c += blockDim.x) ss = fmaf(row[c], row[c], ss);
+  __shared__ float red[32];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float r = sqrtf(red[0] / static_cast<float>(H) + eps);
+  for (int c = threadIdx.x; c < H; c += blockDim.x)
+    x[static_cast<size_t>(t) * H + c] = f32_to_bf16(__fdiv_rn(row[c], r));
+}
+
+// --------------------------------------------------------------------- A1+A2
+// Cluster of 8 CTAs per block of ROUTER_TB rows.  CTA rank r computes the
+// logits of experts [r*E/8, (r+1)*E/8) for those rows and writes them into
+// rank 0's shared memory; after the cluster barrier rank 0 selects the top k
+// per row (one warp per row) and applies the softmax.
+//
+// x is staged as "byte-paired" half2: word m of a row holds elements 4m..4m+3
+// as P0 = (v0, v2), P1 = (v1, v3), stored word-pair-major per 16-element
+// chunk so lane c reads consecutive bytes.  Chunk stats per 16 elements:
+// (1024 * sum of stored halves, plain sum).
+__global__ void __cluster_dims__(8, 1, 1) __launch_bounds__(256)
+k_router_topk(const uint16_t* __restrict__ x, int T, int H, const uint32_t* __restrict__ rq,
+              const uint16_t* __restrict__ rs, const uint16_t* __restrict__ rb,
+              const float* __restrict__ bias, int bias_per_row, int E, int k,
+              int32_t* __restrict__ idx, float* __restrict__ gates, float* __restrict__ logits_out) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int row0 = (blockIdx.x / 8) * ROUTER_TB;
+  const int nrows = min(ROUTER_TB, T - row0);
+  const int nch = H / 16;                      // 16-element chunks (one uint4 of 8-bit codes)
+  // smem: logits [TB][E] | per row: P uint2 [nch*4] (word-major), st float2 [nch]
+  float* lg = reinterpret_cast<float*>(smem);
+  unsigned char* xs = smem + ROUTER_TB * E * sizeof(float);
+  const size_t row_bytes = static_cast<size_t>(nch) * 4 * sizeof(uint2) + nch * sizeof(float2);
+
+  // stage x rows
+  for (int i = threadIdx.x; i < nrows * nch; i += blockDim.x) {
+    const int r = i / nch, c = i - r * nch;
+    const uint16_t* src = x + static_cast<size_t>(row0 + r) * H + 16 * c;
+    uint2* P = reinterpret_cast<uint2*>(xs + r * row_bytes);
+    float2* st = reinterpret_cast<float2*>(xs + r * row_bytes + static_cast<size_t>(nch) * 4 * sizeof(uint2));
+    float off = 0.f, sum = 0.f;
+    const uint4 u0 = *reinterpret_cast<const uint4*>(src);
+    const uint4 u1 = *reinterpret_cast<const uint4*>(src + 8);
+    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {          // word m covers elements 4m..4m+3
+      const float v0 = __uint_as_float(w[2 * m] << 16), v1 = __uint_as_float(w[2 * m] & 0xFFFF0000u);
+      const float v2 = __uint_as_float(w[2 * m + 1] << 16), v3 = __uint_as_float(w[2 * m + 1] & 0xFFFF0000u);
+      const uint32_t p0 = pack_half2(v0, v2), p1 = pack_half2(v1, v3);
+      P[m * nch + c] = make_uint2(p0, p1);
+      const float2 f0 = unpack_half2(p0), f1 = unpack_half2(p1);
+      off += (f0.x + f0.y) + (f1.x + f1.y);
+    }
+    sum = off;
+    st[c] = make_float2(1024.f * off, sum);
+  }
+  __syncthreads();
+
+  float* lg0 = cluster.map_shared_rank(lg, 0);
+  const int epc = E / 8;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarp = blockDim.x >> 5;
+  const int hb = H / 4;                       // bytes... words per router row
+  for (int el = warp; el < epc; el += nwarp) {
+    const int e = rank * epc + el;
+    const uint8_t* qrow = reinterpret_cast<const uint8_t*>(rq + static_cast<size_t>(e) * hb);
+    float acc[ROUTER_TB];
+#pragma unroll
+    for (int r = 0; r < ROUTER_TB; ++r) acc[r] = 0.f;
+    for (int c = lane; c < nch; c += 32) {
+      const uint4 q = ldg_nc_v4(qrow + static_cast<size_t>(c) * 16);
+      const float sc = bf16_to_f32(ldg_u16(rs + static_cast<size_t>(e) * (H / 64) + (c >> 2)));
+      const float bi = bf16_to_f32(ldg_u16(rb + static_cast<size_t>(e) * (H / 64) + (c >> 2)));
+#pragma unroll
+      for (int r = 0; r < ROUTER_TB; ++r) {
+        if (r < nrows) {
+          const uint2* P = reinterpret_cast<const uint2*>(xs + r * row_bytes);
+          const float2* st = reinterpret_cast<const float2*>(xs + r * row_bytes + static_cast<size_t>(nch) * 4 * sizeof(uint2));
+          float a0 = 0.f, a1 = 0.f;
+          uint2 p;
+          p = P[0 * nch + c]; { uint32_t pp[2] = {p.x, p.y}; dot_word8(q.x, pp, a0, a1); }
+          p = P[1 * nch + c]; { uint32_t pp[2] = {p.x, p.y}; dot_word8(q.y, pp, a0, a1); }
+          p = P[2 * nch + c]; { uint32_t pp[2] = {p.x, p.y}; dot_word8(q.z, pp, a0, a1); }
+          p = P[3 * nch + c]; { uint32_t pp[2] = {p.x, p.y}; dot_word8(q.w, pp, a0, a1); }
+          const float2 s2 = st[c];
+          acc[r] += sc * ((a0 + a1) - s2.x) + bi * s2.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < ROUTER_TB; ++r) {
+      const float v = warp_sum(acc[r]);
+      if (lane == 0 && r < nrows) {
+        float bb = 0.f;
+        if (bias != nullptr) bb = bias_per_row ? bias[static_cast<size_t>(row0 + r) * E + e] : bias[e];
+        lg0[r * E + e] = v + bb;
+      }
+    }
+  }
+  cluster.sync();
+  if (rank != 0) return;
+
+  // top-k + softmax, one warp per row
+  for (int r = warp; r < nrows; r += nwarp) {
+    const int t = row0 + r;
+    const float* L = lg + r * E;
+    if (logits_out != nullptr)
+      for (int e = lane; e < E; e += 32) logits_out[static_cast<size_t>(t) * E + e] = L[e];
+    // each lane holds experts lane, lane+32, ...; taken experts are marked in a bit mask
+    unsigned taken = 0u;
+    float sel[8];
+    int sid[8];
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int s = 0, e = lane; e < E; ++s, e += 32) {
+        if (taken & (1u << s)) continue;
+        const float v = L[e];
+        if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      sel[j] = bv;
+      sid[j] = bi;
+    }
+    if (lane == 0) {
+      float z[8], den = 0.f;
+      for (int j = 0; j < k; ++j) { z[j] = expf(sel[j] - sel[0]); den += z[j]; }
+      for (int j = 0; j < k; ++j) {
+        idx[static_cast<size_t>(t) * k + j] = sid[j];
+        gates[static_cast<size_t>(t) * k + j] = z[j] / den;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------ A3
+// One block.  Counts with shared atomics (order-free), exclusive scan, then a
+// single warp places the pairs chunk by chunk in index order (stable).
+__global__ void k_bucket(const int32_t* __restrict__ idx, int n, int E, int32_t* __restrict__ offsets,
+                         int32_t* __restrict__ pairs, int32_t* __restrict__ active,
+                         int32_t* __restrict__ n_active) {
+  extern __shared__ int sh[];
+  int* cnt = sh;          // [E]
+  int* cur = sh + E;      // [E]
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  for (int p = threadIdx.x; p < n; p += blockDim.x) {
+    const int e = idx[p];
+    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+    else flag_check(CHECK_EXPERT_ID);
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    // warp scan over E in chunks of 32
+    const int lane = threadIdx.x;
+    int base = 0, abase = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const int v = e < E ? cnt[e] : 0;
+      const int a = v > 0 ? 1 : 0;
+      int incl = v, ainc = a;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t1 = __shfl_up_sync(0xffffffffu, incl, o);
+        const int t2 = __shfl_up_sync(0xffffffffu, ainc, o);
+        if (lane >= o) { incl += t1; ainc += t2; }
+      }
+      if (e < E) {
+        offsets[e] = base + incl - v;
+        cur[e] = base + incl - v;
+        if (a) active[abase + ainc - 1] = e;
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+      abase += __shfl_sync(0xffffffffu, ainc, 31);
+    }
+    if (lane == 0) {
+      offsets[E] = base;
+      *n_active = abase;
+    }
+    __syncwarp();
+    for (int p0 = 0; p0 < n; p0 += 32) {
+      const int p = p0 + lane;
+      const int e = p < n ? idx[p] : -1;
+      const bool ok = (e >= 0 && e < E);
+      const unsigned m = __match_any_sync(0xffffffffu, ok ? e : -1);
+      if (ok) {
+        const int rk = __popc(m & ((1u << lane) - 1u));
+        pairs[cur[e] + rk] = p;
+      }
+      __syncwarp();
+      if (ok && (__ffs(m) - 1) == lane) cur[e] += __popc(m);
+      __syncwarp();
+    }
+  }
+}
+
+// ---------------------------------------------------------------- A4 / A6 up
+// Gate/up projections + GeGLU for bucket rows, GEMV form.
+// blockIdx.y = active-expert slot (routed) or 0 (shared); blockIdx.x = block
+// of GEMV_ROWS intermediate rows.  Bucket rows are processed RG at a time from
+// shared memory.  act[row] (fp16) is written at the bucket position.
+__global__ void __launch_bounds__(256)
+k_gateup_gemv(GateUpArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  int e = 0, pos0 = 0, cnt = a.T;
+  const uint8_t *gq, *uq;
+  const uint16_t *gs, *gb, *us, *ub;
+  if (a.blob_ptrs != nullptr) {
+    if (static_cast<int>(blockIdx.y) >= *a.n_active) return;
+    e = a.active[blockIdx.y];
+    if (e < 0 || e >= a.E) { flag_check(CHECK_EXPERT_ID); return; }
+    pos0 = a.offsets[e];
+    cnt = a.offsets[e + 1] - pos0;
+    if (cnt > a.max_rows) return;
+    const uint8_t* blob = static_cast<const uint8_t*>(a.blob_ptrs[e]);
+    gq = blob + a.off[0]; gs = reinterpret_cast<const uint16_t*>(blob + a.off[1]);
+    gb = reinterpret_cast<const uint16_t*>(blob + a.off[2]);
+    uq = blob + a.off[3]; us = reinterpret_cast<const uint16_t*>(blob + a.off[4]);
+    ub = reinterpret_cast<const uint16_t*>(blob + a.off[5]);
+  } else {
+    gq = reinterpret_cast<const uint8_t*>(a.gq); gs = a.gs; gb = a.gb;
+    uq = reinterpret_cast<const uint8_t*>(a.uq); us = a.us; ub = a.ub;
+  }
+  const int K = a.H, nch = K / 32, N = a.I;
+  float2* scratch = reinterpret_cast<float2*>(smem + GEMV_RG * staged_row_bytes(K));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarp = blockDim.x >> 5;
+  const int i0 = blockIdx.x * GEMV_ROWS;
+  for (int g0 = 0; g0 < cnt; g0 += GEMV_RG) {
+    const int nr = min(GEMV_RG, cnt - g0);
+    if (g0 > 0) __syncthreads();
+    stage_rows4<uint16_t>(smem, scratch, K, nr, [&](int r) -> const uint16_t* {
+      int tok;
+      if (a.pairs != nullptr) {
+        const int p = a.pairs[pos0 + g0 + r];
+        tok = p / a.k;
+      } else {
+        tok = g0 + r;
+      }
+      if (tok < 0 || tok >= a.T) { flag_check(CHECK_PAIR_ID); return nullptr; }
+      return a.x + static_cast<size_t>(tok) * K;
+    });
+    for (int i = i0 + warp; i < min(i0 + GEMV_ROWS, N); i += nwarp) {
+      float av[GEMV_RG], uv[GEMV_RG];
+      row_dot4<GEMV_RG>(gq + static_cast<size_t>(i) * (K / 2), gs + static_cast<size_t>(i) * (K / 64),
+                        gb + static_cast<size_t>(i) * (K / 64), nch, smem, K, nr, av);
+      row_dot4<GEMV_RG>(uq + static_cast<size_t>(i) * (K / 2), us + static_cast<size_t>(i) * (K / 64),
+                        ub + static_cast<size_t>(i) * (K / 64), nch, smem, K, nr, uv);
+      if (lane < nr) {
+        float va = 0.f, vu = 0.f;
+#pragma unroll
+        for (int r = 0; r < GEMV_RG; ++r) if (r == lane) { va = av[r]; vu = uv[r]; }
+        const float h = gelu_tanh(va) * vu;
+        a.act[static_cast<size_t>(pos0 + g0 + lane) * N + i] = __float2half_rn(h);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- A5 / A6 down
+// Down projection, GEMV form: y[dest(row)][o] = sum_i Wd[o, i] act[row][i].
+// Routed: dest = pairs[pos] (row of y_pairs); shared: dest = row (ysh).
+__global__ void __launch_bounds__(256)
+k_down_gemv(DownArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  int e = 0, pos0 = 0, cnt = a.T;
+  const uint8_t* dq;
+  const uint16_t *ds, *db;
+  if (a.blob_ptrs != nullptr) {
+    if (static_cast<int>(blockIdx.y) >= *a.n_active) return;
+    e = a.active[blockIdx.y];
+    if (e < 0 || e >= a.E) { flag_check(CHECK_EXPERT_ID); return; }
+    pos0 = a.offsets[e];
+    cnt = a.offsets[e + 1] - pos0;
+    if (cnt > a.max_rows) return;
+    const uint8_t* blob = static_cast<const uint8_t*>(a.blob_ptrs[e]);
+    dq = blob + a.off[6]; ds = reinterpret_cast<const uint16_t*>(blob + a.off[7]);
+    db = reinterpret_cast<const uint16_t*>(blob + a.off[8]);
+  } else {
+    dq = reinterpret_cast<const uint8_t*>(a.dq); ds = a.ds; db = a.db;
+  }
+  const int K = a.I, nch = K / 32, N = a.H;
+  float2* scratch = reinterpret_cast<float2*>(smem + GEMV_RG * staged_row_bytes(K));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarp = blockDim.x >> 5;
+  const int o0 = blockIdx.x * GEMV_ROWS;
+  for (int g0 = 0; g0 < cnt; g0 += GEMV_RG) {
+    const int nr = min(GEMV_RG, cnt - g0);
+    if (g0 > 0) __syncthreads();
+    stage_rows4<__half>(smem, scratch, K, nr, [&](int r) -> const __half* {
+      return a.act + static_cast<size_t>(pos0 + g0 + r) * K;
+    });
+    for (int o = o0 + warp; o < min(o0 + GEMV_ROWS, N); o += nwarp) {
+      float yv[GEMV_RG];
+      row_dot4<GEMV_RG>(dq + static_cast<size_t>(o) * (K / 2), ds + static_cast<size_t>(o) * (K / 64),
+                        db + static_cast<size_t>(o) * (K / 64), nch, smem, K, nr, yv);
+      if (lane < nr) {
+        float v = 0.f;
+#pragma unroll
+        for (int r = 0; r < GEMV_RG; ++r) if (r == lane) v = yv[r];
+        int dest = pos0 + g0 + lane;
+        if (a.pairs != nullptr) dest = a.pairs[dest];
+        a.y[static_cast<size_t>(dest) * N + o] = v;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------ A7
+__global__ void k_combine(const float* __restrict__ yp, const float* __restrict__ gates,
+                          const float* __restrict__ ysh, int H, int k, uint16_t* __restrict__ y,
+                          float* __restrict__ resid) {
+  const int t = blockIdx.y;
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= H) return;
+  float g[8];
+  for (int j = 0; j < k; ++j) g[j] = gates[static_cast<size_t>(t) * k + j];
+  float acc = 0.f;
+  for (int j = 0; j < k; ++j) acc = fmaf(g[j], yp[(static_cast<size_t>(t) * k + j) * H + c], acc);
+  if (ysh != nullptr) acc += ysh[static_cast<size_t>(t) * H + c];
+  if (y != nullptr) y[static_cast<size_t>(t) * H + c] = f32_to_bf16(acc);
+  if (resid != nullptr) resid[static_cast<size_t>(t) * H + c] += acc;
+}
+
+}  // namespace moe
