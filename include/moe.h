@@ -141,6 +141,29 @@ MOE_API int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, in
                        const int32_t* pairs, const int32_t* active,
                        const int32_t* n_active, float* y_pairs,
                        void* ws, size_t ws_bytes, void* stream);
+/* moe_expert_forward without a workspace argument, for callers that cannot
+ * allocate device memory where they run the experts (inside a CUDA graph
+ * being captured, under a memory pool that must not be re-entered, or in an
+ * embedder whose device memory is reserved up front).  The pages describe no
+ * counterpart of this call; it is a convenience of this library.
+ *   Arguments and results are those of moe_expert_forward.
+ *   Scratch: a static device array of MOE_NOALLOC_SCRATCH_BYTES (4 MiB) in
+ *   the library image, one per GPU that loads the library, kept until exit.
+ *   It must hold moe_expert_workspace_size(T,H,I,k) bytes (T*k*I fp16
+ *   values; with I = 704 and k = 8 that is T <= 372); larger requests return
+ *   MOE_ERR_INVALID_ARG and launch nothing.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) and caches it; make that first call before any
+ *   stream capture.
+ *   Every call on a device shares the one array and leaves its contents
+ *   behind; two calls whose kernels overlap on the GPU (different streams,
+ *   no ordering between them) race on it.  Nothing in it needs to start at
+ *   zero.  The call allocates no device memory. */
+#define MOE_NOALLOC_SCRATCH_BYTES (4 * 1024 * 1024)
+MOE_API int moe_expert_forward_noalloc(const uint16_t* x, int T, int H, int I, int E, int k,
+                                       const void* const* blob_ptrs, const int32_t* offsets,
+                                       const int32_t* pairs, const int32_t* active,
+                                       const int32_t* n_active, float* y_pairs, void* stream);
 /* Bucket-size threshold between the GEMV and the tensor-core path (>= 0). */
 MOE_API int moe_set_gemv_max_rows(int rows);
 

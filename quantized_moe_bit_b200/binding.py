@@ -58,6 +58,15 @@ def moe_expert_forward(x, I: int, E: int, k: int, blob_ptrs, offsets, pairs, act
                                    stream_ptr(stream)))
 
 
+def moe_expert_forward_noalloc(x, I: int, E: int, k: int, blob_ptrs, offsets, pairs, active, n_active,
+                               y_pairs, stream=None):
+    """moe_expert_forward with its scratch in the library's static device
+    array (no workspace argument; see include/moe.h for the size limit)."""
+    T, H = x.shape
+    check(lib().moe_expert_forward_noalloc(ptr(x), T, H, I, E, k, ptr(blob_ptrs), ptr(offsets), ptr(pairs),
+                                           ptr(active), ptr(n_active), ptr(y_pairs), stream_ptr(stream)))
+
+
 def moe_shared_workspace_size(T: int, H: int, Is: int) -> int:
     return lib().moe_shared_workspace_size(T, H, Is)
 

@@ -2,3 +2,4 @@
 // device symbols such as the check word without relocatable device code).
 #include "kernels.cu"
 #include "api.cu"
+#include "expert_noalloc.cu"
