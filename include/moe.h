@@ -150,7 +150,8 @@ MOE_API int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, in
  *   Scratch: a static device array of MOE_NOALLOC_SCRATCH_BYTES (4 MiB) in
  *   the library image, one per GPU that loads the library, kept until exit.
  *   It must hold moe_expert_workspace_size(T,H,I,k) bytes (T*k*I fp16
- *   values; with I = 704 and k = 8 that is T <= 372); larger requests return
+ *   values plus a T*H fp16 copy of x; at H = 2816, I = 704, k = 8 that is
+ *   T <= 248); larger requests return
  *   MOE_ERR_INVALID_ARG and launch nothing.
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress) and caches it; make that first call before any

@@ -5,6 +5,7 @@
 
 #include "gemv.cuh"
 #include "kernels.cuh"
+#include "tc_gemm.cu"
 
 namespace moe {
 
@@ -153,8 +154,8 @@ int moe_bucket(const int32_t* idx, int T, int k, int E, int32_t* offsets, int32_
 }
 
 size_t moe_expert_workspace_size(int T, int H, int I, int k) {
-  (void)H;
-  return align_up(static_cast<size_t>(T) * k * I * sizeof(__half));
+  // fp16 activation between the projections + fp16 copy of x for the tensor-core path
+  return align_up(static_cast<size_t>(T) * k * I * sizeof(__half)) + align_up(static_cast<size_t>(T) * H * sizeof(__half));
 }
 
 int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, int k, const void* const* blob_ptrs,
@@ -171,12 +172,17 @@ int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, int k, con
     return fail(MOE_ERR_INVALID_ARG, "moe_expert_forward: misaligned pointer");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   __half* act = static_cast<__half*>(ws);
+  __half* xh = reinterpret_cast<__half*>(static_cast<char*>(ws) + align_up(static_cast<size_t>(T) * k * I * sizeof(__half)));
   const int maxA = T * k < E ? T * k : E;
+  // Buckets of at most gemv_max_rows rows go to the GEMV kernels, larger ones
+  // to the tensor-core kernel (shapes it supports: H % 128 == 0, H, I <= 4096).
+  const bool tc = T > g_gemv_max_rows && H % 128 == 0 && H <= 4096 && I <= 4096;
+  const int gemv_rows = tc ? g_gemv_max_rows : (1 << 30);
 
   GateUpArgs g{};
   g.x = x; g.T = T; g.H = H; g.I = I; g.E = E; g.k = k;
   g.blob_ptrs = blob_ptrs; g.offsets = offsets; g.pairs = pairs; g.active = active; g.n_active = n_active;
-  g.max_rows = 1 << 30;
+  g.max_rows = gemv_rows;
   blob_offsets(H, I, g.off);
   g.act = act;
   size_t sm = gemv_smem(H);
@@ -184,16 +190,37 @@ int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, int k, con
   k_gateup_gemv<<<dim3((I + GEMV_ROWS - 1) / GEMV_ROWS, maxA), 256, sm, s>>>(g);
   if ((st = launch_check("k_gateup_gemv"))) return st;
 
+  TcArgs ta{};
+  if (tc) {
+    const size_t n8 = static_cast<size_t>(T) * H / 8;
+    k_to_f16<<<static_cast<int>((n8 + 255) / 256 < 1024 ? (n8 + 255) / 256 : 1024), 256, 0, s>>>(x, n8, xh);
+    if ((st = launch_check("k_to_f16"))) return st;
+    ta.mode = 0; ta.xh = xh; ta.T = T; ta.H = H; ta.I = I; ta.E = E; ta.k = k;
+    ta.blob_ptrs = blob_ptrs; ta.offsets = offsets; ta.pairs = pairs; ta.active = active; ta.n_active = n_active;
+    ta.max_rows = g_gemv_max_rows;
+    blob_offsets(H, I, ta.off);
+    ta.act_out = act; ta.act_in = act; ta.y_out = y_pairs;
+    if ((st = set_smem(reinterpret_cast<const void*>(k_expert_tc), TC_SMEM))) return st;
+    k_expert_tc<<<dim3(I / 64, maxA), TC_THREADS, TC_SMEM, s>>>(ta);
+    if ((st = launch_check("k_expert_tc(gate/up)"))) return st;
+  }
+
   DownArgs d{};
   d.act = act; d.T = T; d.H = H; d.I = I; d.E = E; d.k = k;
   d.blob_ptrs = blob_ptrs; d.offsets = offsets; d.pairs = pairs; d.active = active; d.n_active = n_active;
-  d.max_rows = 1 << 30;
+  d.max_rows = gemv_rows;
   blob_offsets(H, I, d.off);
   d.y = y_pairs;
   sm = gemv_smem(I);
   if ((st = set_smem(reinterpret_cast<const void*>(k_down_gemv), sm))) return st;
   k_down_gemv<<<dim3((H + GEMV_ROWS - 1) / GEMV_ROWS, maxA), 256, sm, s>>>(d);
-  return launch_check("k_down_gemv");
+  if ((st = launch_check("k_down_gemv"))) return st;
+  if (tc) {
+    ta.mode = 1;
+    k_expert_tc<<<dim3(H / 128, maxA), TC_THREADS, TC_SMEM, s>>>(ta);
+    if ((st = launch_check("k_expert_tc(down)"))) return st;
+  }
+  return MOE_OK;
 }
 
 size_t moe_shared_workspace_size(int T, int H, int Is) {

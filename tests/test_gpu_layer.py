@@ -142,3 +142,35 @@ def test_empty_and_invalid(M):
     with pytest.raises(M.MoeError):
         M.moe_rmsnorm(torch.empty((1, 100), device="cuda"), bad)
     M.moe_sync()
+
+
+@pytest.fixture
+def gemv_rows(M):
+    def set_(n):
+        M.moe_set_gemv_max_rows(n)
+    yield set_
+    M.moe_set_gemv_max_rows(2)
+
+
+@pytest.mark.parametrize("max_rows", [0, 2, 1 << 30])
+@pytest.mark.parametrize("T", [37, 130])
+def test_expert_paths_tiny(M, gemv_rows, T, max_rows):
+    """Tensor-core path (buckets > max_rows) and GEMV path against the oracle;
+    T = 130 gives buckets above 128 rows (two N tiles on the tensor cores)."""
+    gemv_rows(max_rows)
+    cfg = tiny_config("prefill_1L_128tok", T=T)
+    hl = HostLayer(cfg, 0)
+    z = gen.rows(cfg.seed, 1000, T, cfg.H, accept=gap_ok_predicate(hl))
+    g = _run_calls(M, hl, hl.upload(), z)
+    _check_all(hl, z, g)
+
+
+@pytest.mark.parametrize("max_rows", [2, 1 << 30])
+def test_prefill_128_full(M, gemv_rows, max_rows):
+    """The 128-row prefill chunk at full size (H=2816, E=128, I=704)."""
+    gemv_rows(max_rows)
+    cfg = CONFIGS["prefill_1L_128tok"]
+    hl = HostLayer(cfg, 0)
+    z = gen.rows(cfg.seed, 1000, cfg.T, cfg.H, accept=gap_ok_predicate(hl))
+    g = _run_calls(M, hl, hl.upload(), z)
+    _check_all(hl, z, g)
