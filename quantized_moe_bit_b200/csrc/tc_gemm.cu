@@ -271,8 +271,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_expert_tc(TcArgs a) {
     }
 
     // ------------------------------------------------------------ epilogue
+    if (warp < 4) ok = __all_sync(0xffffffffu, ok);        // .aligned tcgen05.ld below: warp-uniform
     if (warp < 4 && ok) {
-      ok = tc::mbar_wait(done_bar, ntile & 1);
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(done_bar, ntile & 1));
       if (ok) {
         tc::tc_fence_after();
         const int row = 32 * warp + lane;
