@@ -89,3 +89,33 @@ def check_close(a: np.ndarray, ref: np.ndarray, max_rel: float, mean_rel: float,
     mx, mean = float(err.max()) / rms, float(err.mean()) / rms
     assert mx <= max_rel and mean <= mean_rel, f"{what}: max {mx:.3e} mean {mean:.3e} (x rms)"
     return mx, mean
+
+
+class HostStack:
+    """Per-layer host weights of a multi-layer workload, generated on demand
+    (router, bias, shared expert, expert lookup) for the oracle side."""
+
+    def __init__(self, cfg):
+        self.cfg = cfg
+        self._layers = {}
+
+    def layer(self, l: int) -> HostLayer:
+        if l not in self._layers:
+            self._layers[l] = HostLayer(self.cfg, l, with_blobs=False)
+        return self._layers[l]
+
+
+def upload_stack(cfg, device="cuda"):
+    """All layers of a workload on the device (one layer of host blobs at a time)."""
+    import gen as G
+    from quantized_moe_bit_b200.weights import upload_layer
+    stride = G.synth.default_blob_stride(cfg.H, cfg.I)
+    host = np.empty((cfg.E, stride), dtype=np.uint8)
+    out = []
+    for l in range(cfg.layers):
+        router = G.router_weights(cfg.seed, l, cfg.E, cfg.H)
+        bias = G.zipf_bias(cfg.seed, l, cfg.E) if cfg.zipf else None
+        shared = G.shared_weights(cfg.seed, l, cfg.H, cfg.Is)
+        G.layer_blobs(cfg.seed, l, cfg.E, cfg.H, cfg.I, stride, out=host, threads=16)
+        out.append(upload_layer(router, bias, shared, host, device))
+    return out

@@ -1,0 +1,99 @@
+"""Multi-layer workloads on the GPU against the oracle, teacher-forced per layer.
+
+The GPU runs the whole stack (moe_decode_forward) and traces every layer's
+bf16 input x_l, output y_l and routing.  The oracle recomputes each sampled
+layer from the GPU's own x_l (so rounding drift over 30 layers does not
+decide a comparison), checks the selection (bit-exact where the logits have
+no near tie), the gates and the output against the tolerance, and checks the
+residual stream: x_l must be the RMS norm of h_0 + sum of earlier outputs.
+"""
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+import gen
+from gen import CONFIGS, tiny_config
+from oracle import moe_oracle as O
+from tests._support import HostStack, check_close, check_output, check_routing, upload_stack
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_stack(M, cfg, layers, z, traces=True):
+    T, H, L = z.shape[0], cfg.H, cfg.layers
+    stack = M.DecodeStack(layers)
+    h = torch.from_numpy(z).cuda()
+    ws = torch.empty(M.moe_decode_workspace_size(T, H, cfg.I, cfg.Is, cfg.E, cfg.k), dtype=torch.uint8, device="cuda")
+    xt = torch.empty((L, T, H), dtype=torch.int16, device="cuda")
+    yt = torch.empty((L, T, H), dtype=torch.int16, device="cuda")
+    it = torch.empty((L, T, cfg.k), dtype=torch.int32, device="cuda")
+    gt = torch.empty((L, T, cfg.k), dtype=torch.float32, device="cuda")
+    M.moe_decode_forward(h, cfg.I, cfg.Is, cfg.E, cfg.k, stack, ws, x_trace=xt, y_trace=yt, idx_trace=it,
+                         gates_trace=gt)
+    M.moe_sync()
+    u16 = lambda t: t.cpu().numpy().view(np.uint16)
+    return dict(h=h.cpu().numpy(), x=u16(xt), y=u16(yt), idx=it.cpu().numpy(), gates=gt.cpu().numpy())
+
+
+def _check_stack(cfg, hs, z, g, sample_layers):
+    ties = 0
+    h = z.astype(np.float64)
+    outs = {}
+    for l in range(cfg.layers):
+        hl = hs.layer(l) if l in sample_layers else None
+        x = O.bf16_to_f64(g["x"][l])
+        if l in sample_layers:
+            lg = O.router_logits(x, hl.router, hl.bias)
+            ties += check_routing(g["idx"][l], lg, cfg.k)
+            assert np.abs(g["gates"][l] - O.softmax_gates(lg, g["idx"][l])).max() < 2e-6
+            r = O.layer_forward(x, hl.router, hl.bias, hl.expert, hl.shared, cfg.k, cfg.E, idx=g["idx"][l])
+            check_output(g["y"][l], r["out"], f"layer {l}")
+            outs[l] = r["out"]
+        # residual stream: the GPU's x_l is the norm of h_0 + the earlier outputs (the
+        # oracle's where sampled, the GPU's bf16 outputs elsewhere), within the output tolerance
+        _, xr = O.rmsnorm(h)
+        check_close(x, xr, 2e-2, 2e-3, f"layer {l} input")
+        h = h + (outs[l] if l in outs else O.bf16_to_f64(g["y"][l]))
+    rms = np.sqrt(np.mean(h * h))
+    assert np.abs(g["h"] - h).max() < 2e-2 * rms
+    return ties
+
+
+@pytest.fixture(scope="module")
+def M():
+    import quantized_moe_bit_b200 as M
+    return M
+
+
+def test_stack_tiny_all_layers(M):
+    cfg = tiny_config("decode_30L_b64", layers=6, T=24)
+    layers = upload_stack(cfg)
+    z = gen.rows(cfg.seed, 1000, cfg.T, cfg.H)
+    g = _run_stack(M, cfg, layers, z)
+    _check_stack(cfg, HostStack(cfg), z, g, set(range(cfg.layers)))
+    g2 = _run_stack(M, cfg, layers, z)
+    for key in ("h", "x", "y", "idx", "gates"):
+        assert np.array_equal(g[key], g2[key]), key          # bitwise deterministic
+
+
+def test_decode_30L_b1_full(M):
+    """30 layers, batch 1, all resident (12.9 GB): two steps, every layer checked."""
+    cfg = CONFIGS["decode_30L_b1"]
+    layers = upload_stack(cfg)
+    hs = HostStack(cfg)
+    for step in (0, 1):
+        z = gen.rows(cfg.seed, cfg.row_stream + step, 1, cfg.H)
+        g = _run_stack(M, cfg, layers, z)
+        _check_stack(cfg, hs, z, g, set(range(cfg.layers)))
+
+
+def test_decode_30L_b64_full(M):
+    """30 layers, 64 rows per step: one step, layers 0, 14 and 29 checked against
+    the oracle, the residual stream checked at every layer."""
+    cfg = CONFIGS["decode_30L_b64"]
+    layers = upload_stack(cfg)
+    z = gen.rows(cfg.seed, cfg.row_stream, cfg.T, cfg.H)
+    g = _run_stack(M, cfg, layers, z)
+    _check_stack(cfg, HostStack(cfg), z, g, {0, 14, 29})
