@@ -216,6 +216,13 @@ MOE_API int moe_layer_forward(const float* h_in, float* h_out, const uint16_t* x
  *   ws         device workspace of at least moe_decode_workspace_size(...) bytes
  * Layers run in order on `stream`. */
 MOE_API size_t moe_decode_workspace_size(int T, int H, int I, int Is, int E, int k);
+/* Batch-1 steps (T = 1, per-expert or no bias) run as one persistent kernel
+ * per up to 48 layers (8-CTA clusters, cooperative launch); other shapes run
+ * the per-layer calls.  enable = 0 forces the per-layer path.  spec_experts
+ * (0..8, default 2): per layer, the experts with the largest router bias are
+ * prefetched into L2 while the layer waits for its routing (their bytes are
+ * read again, from L2, only if they are chosen). */
+MOE_API int moe_set_decode_fused(int enable, int spec_experts);
 /* Number of kernels one moe_decode_forward(T, L) call launches. */
 MOE_API int moe_decode_launches(int T, int L);
 MOE_API int moe_decode_forward(float* h, int T, int H, int I, int Is, int E, int k, int L,

@@ -6,11 +6,14 @@
 #include "gemv.cuh"
 #include "kernels.cuh"
 #include "tc_gemm.cu"
+#include "decode_fused.cu"
 
 namespace moe {
 
 static thread_local char g_err[512] = "";
 static int g_gemv_max_rows = 2;
+static int g_decode_fused = 1;
+static int g_decode_spec = 2;
 
 int fail(int code, const char* fmt, ...) {
   va_list ap;
@@ -348,14 +351,112 @@ int moe_layer_forward(const float* h_in, float* h_out, const uint16_t* x_in, int
   return MOE_OK;
 }
 
+// Shapes the fused batch-1 kernel serves.
+static bool fused_ok(int T, int H, int I, int Is, int E, int k, int bias_per_row, int G) {
+  if (!g_decode_fused || T != 1 || bias_per_row) return false;
+  if (H % 64 || H > 4096 || I % 64 || Is % 64 || E % 8 || E > 1024 || k > 8) return false;
+  if (k * I + Is > DF_MAX_ACT || k + (Is + I - 1) / I > DF_MAX_UNITS) return false;
+  if (G <= 0 || (H + G - 1) / G > DF_MAX_ROWS) return false;
+  return true;
+}
+
+// Clusters of the fused kernel that fit at once on this device (cached).
+static int fused_grid(int H) {
+  static int cached[64][2];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  const int which = H > 3072 ? 1 : 0;
+  if (cached[dev][which]) return cached[dev][which];
+  const size_t smem = decode_fused_smem(H, 0);
+  const void* fn = which ? reinterpret_cast<const void*>(k_decode_b1<4>) : reinterpret_cast<const void*>(k_decode_b1<3>);
+  if (set_smem(fn, smem)) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(DF_CLUSTER * 148, 1, 1);
+  cfg.blockDim = dim3(DF_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = DF_CLUSTER; at[0].val.clusterDim.y = 1; at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n <= 0) { cudaGetLastError(); return 0; }
+  cached[dev][which] = n * DF_CLUSTER;
+  return cached[dev][which];
+}
+
+static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, const moe_qmat* routers,
+                        const float* const* biases, const void* const* const* blob_tables, const moe_qmat* shared,
+                        uint16_t* x_trace, uint16_t* y_trace, int32_t* idx_trace, float* gates_trace, void* ws,
+                        int G, cudaStream_t s) {
+  __half* act = static_cast<__half*>(ws);
+  unsigned* ctr = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + align_up(static_cast<size_t>(k * I + Is) * 2));
+  const size_t smem = decode_fused_smem(H, k * I + Is);
+  const bool big = H > 3072;
+  const void* fn = big ? reinterpret_cast<const void*>(k_decode_b1<4>) : reinterpret_cast<const void*>(k_decode_b1<3>);
+  int st;
+  if ((st = set_smem(fn, smem))) return st;
+  for (int l0 = 0; l0 < L; l0 += DF_MAX_LAYERS) {
+    const int nl = L - l0 < DF_MAX_LAYERS ? L - l0 : DF_MAX_LAYERS;
+    static DfArgs args;   // large parameter block; copied into the launch
+    memset(&args, 0, sizeof(args));
+    args.h = h; args.H = H; args.I = I; args.Is = Is; args.E = E; args.k = k; args.L = nl;
+    blob_offsets(H, I, args.off);
+    args.act = act; args.counter = ctr;
+    const size_t TH = static_cast<size_t>(H), Tk = static_cast<size_t>(k);
+    args.x_trace = x_trace ? x_trace + l0 * TH : nullptr;
+    args.y_trace = y_trace ? y_trace + l0 * TH : nullptr;
+    args.idx_trace = idx_trace ? idx_trace + l0 * Tk : nullptr;
+    args.gates_trace = gates_trace ? gates_trace + l0 * Tk : nullptr;
+    args.spec = g_decode_spec;
+    for (int l = 0; l < nl; ++l) {
+      const moe_qmat& R = routers[l0 + l];
+      DfLayer& d = args.layer[l];
+      d.rq = R.q; d.rs = R.s; d.rb = R.b;
+      d.bias = biases ? biases[l0 + l] : nullptr;
+      d.blobs = blob_tables[l0 + l];
+      for (int m = 0; m < 3; ++m) {
+        const moe_qmat& S = shared[3 * (l0 + l) + m];
+        d.sq[m] = S.q; d.ss[m] = S.s; d.sb[m] = S.b;
+      }
+    }
+    if ((st = cuda_check(cudaMemsetAsync(ctr, 0, sizeof(unsigned), s), "zero barrier counter"))) return st;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(G, 1, 1);
+    cfg.blockDim = dim3(DF_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeCooperative;
+    at[0].val.cooperative = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cudaError_t e = big ? cudaLaunchKernelEx(&cfg, k_decode_b1<4>, args) : cudaLaunchKernelEx(&cfg, k_decode_b1<3>, args);
+    if ((st = cuda_check(e, "k_decode_b1 launch"))) return st;
+  }
+  return MOE_OK;
+}
+
+int moe_set_decode_fused(int enable, int spec_experts) {
+  if (spec_experts < 0 || spec_experts > 8) return fail(MOE_ERR_INVALID_ARG, "spec_experts must be in [0, 8]");
+  g_decode_fused = enable ? 1 : 0;
+  g_decode_spec = spec_experts;
+  return MOE_OK;
+}
+
 int moe_decode_launches(int T, int L) {
-  // rmsnorm, router, bucket, shared gate/up, shared down, expert gate/up,
-  // expert down, combine per layer
-  return (T > 0 && L > 0) ? 8 * L : 0;
+  if (T <= 0 || L <= 0) return 0;
+  // fused batch-1 path: one kernel per DF_MAX_LAYERS layers; otherwise rmsnorm,
+  // router, bucket, shared gate/up, shared down, expert gate/up, expert down and
+  // combine per layer (plus the tensor-core kernels for multi-row buckets)
+  if (T == 1 && g_decode_fused) return (L + DF_MAX_LAYERS - 1) / DF_MAX_LAYERS;
+  return 8 * L;
 }
 
 size_t moe_decode_workspace_size(int T, int H, int I, int Is, int E, int k) {
-  return moe_layer_workspace_size(T, H, I, Is, E, k);
+  const size_t layered = moe_layer_workspace_size(T, H, I, Is, E, k);
+  const size_t fused = align_up(static_cast<size_t>(k * I + Is) * 2) + 256;
+  return layered > fused ? layered : fused;
 }
 
 int moe_decode_forward(float* h, int T, int H, int I, int Is, int E, int k, int L, const moe_qmat* routers,
@@ -367,6 +468,12 @@ int moe_decode_forward(float* h, int T, int H, int I, int Is, int E, int k, int 
   if (L < 0) return fail(MOE_ERR_INVALID_ARG, "moe_decode_forward: L < 0");
   if (T == 0 || L == 0) return MOE_OK;
   if (!h || !routers || !blob_tables || !shared) return fail(MOE_ERR_INVALID_ARG, "moe_decode_forward: NULL pointer");
+  if (ws_bytes < moe_decode_workspace_size(T, H, I, Is, E, k))
+    return fail(MOE_ERR_INVALID_ARG, "moe_decode_forward: workspace too small");
+  const int G = (T == 1 && g_decode_fused) ? fused_grid(H) : 0;
+  if (fused_ok(T, H, I, Is, E, k, bias_per_row, G))
+    return launch_fused(h, H, I, Is, E, k, L, routers, biases, blob_tables, shared, x_trace, y_trace, idx_trace,
+                        gates_trace, ws, G, static_cast<cudaStream_t>(stream));
   const size_t TH = static_cast<size_t>(T) * H, Tk = static_cast<size_t>(T) * k;
   for (int l = 0; l < L; ++l) {
     const float* b = biases ? biases[l] : nullptr;

@@ -101,3 +101,32 @@ def test_decode_30L_b64_full(M):
     z = gen.rows(cfg.seed, cfg.row_stream, cfg.T, cfg.H)
     g = _run_stack(M, cfg, layers, z)
     _check_stack(cfg, HostStack(cfg), z, g, {0, 14, 29}, chain=False)
+
+
+@pytest.mark.parametrize("spec", [0, 2])
+def test_stack_tiny_b1_fused_and_layered(M, spec):
+    """Batch 1: the persistent fused kernel and the per-layer path, both against
+    the oracle on every layer; the fused result does not depend on the
+    speculative prefetch setting and is bitwise repeatable."""
+    cfg = tiny_config("decode_30L_b1", layers=5, T=1)
+    layers = upload_stack(cfg)
+    hs = HostStack(cfg)
+    z = gen.rows(cfg.seed, 1000, 1, cfg.H)
+    try:
+        M.moe_set_decode_fused(True, spec)
+        gf = _run_stack(M, cfg, layers, z)
+        gf2 = _run_stack(M, cfg, layers, z)
+        M.moe_set_decode_fused(False, spec)
+        gl = _run_stack(M, cfg, layers, z)
+    finally:
+        M.moe_set_decode_fused(True, 2)
+    for g in (gf, gl):
+        _check_stack(cfg, hs, z, g, set(range(cfg.layers)))
+    for key in ("h", "x", "y", "idx", "gates"):
+        assert np.array_equal(gf[key], gf2[key]), key
+    assert np.array_equal(gf["idx"], gl["idx"])
+
+
+def test_fused_launch_count(M):
+    assert M.moe_decode_launches(1, 30) == 1
+    assert M.moe_decode_launches(2, 30) == 240
