@@ -271,7 +271,7 @@ def run_ours(args, rank, world, local_rank):
                    "k": cfg.k, "I": cfg.I, "Is": cfg.Is, "weights": "4-bit affine g64 experts, 8-bit router",
                    "routing": "Zipf(1.1) per-layer bias", "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (1.1 GB of weights per step)"},
-        "roofline": {"bound": "hbm", "kernel": "decode step: all kernels of moe_decode_forward",
+        "roofline": {"bound": "hbm", "kernel": "k_decode_b1 (one persistent launch per step)",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "peak_source": src, "traffic": None, "bytes_per_step": bytes_step,
                      "distinct_experts_per_layer": distinct},

@@ -337,10 +337,8 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
           if (j >= k) break;
           sel_idx[j] = si[j];
           sel_g[j] = z[j] / den;
-          if (c == 0 && a.idx_trace) {
-            a.idx_trace[static_cast<size_t>(l) * k + j] = si[j];
-            a.gates_trace[static_cast<size_t>(l) * k + j] = z[j] / den;
-          }
+          if (c == 0 && a.idx_trace) a.idx_trace[static_cast<size_t>(l) * k + j] = si[j];
+          if (c == 0 && a.gates_trace) a.gates_trace[static_cast<size_t>(l) * k + j] = z[j] / den;
         }
       }
     }

@@ -26,6 +26,15 @@ def _run_stack(M, cfg, layers, z, traces=True):
     stack = M.DecodeStack(layers)
     h = torch.from_numpy(z).cuda()
     ws = torch.empty(M.moe_decode_workspace_size(T, H, cfg.I, cfg.Is, cfg.E, cfg.k), dtype=torch.uint8, device="cuda")
+    if traces == "idx":          # only the routing trace, as the benchmark asks
+        it = torch.empty((L, T, cfg.k), dtype=torch.int32, device="cuda")
+        M.moe_decode_forward(h, cfg.I, cfg.Is, cfg.E, cfg.k, stack, ws, idx_trace=it)
+        M.moe_sync()
+        return dict(h=h.cpu().numpy(), idx=it.cpu().numpy())
+    if not traces:
+        M.moe_decode_forward(h, cfg.I, cfg.Is, cfg.E, cfg.k, stack, ws)
+        M.moe_sync()
+        return dict(h=h.cpu().numpy())
     xt = torch.empty((L, T, H), dtype=torch.int16, device="cuda")
     yt = torch.empty((L, T, H), dtype=torch.int16, device="cuda")
     it = torch.empty((L, T, cfg.k), dtype=torch.int32, device="cuda")
@@ -125,6 +134,15 @@ def test_stack_tiny_b1_fused_and_layered(M, spec):
     for key in ("h", "x", "y", "idx", "gates"):
         assert np.array_equal(gf[key], gf2[key]), key
     assert np.array_equal(gf["idx"], gl["idx"])
+    # traces are optional, each on its own; the result does not depend on them
+    M.moe_set_decode_fused(True, spec)
+    try:
+        g_none = _run_stack(M, cfg, layers, z, traces=False)
+        g_idx = _run_stack(M, cfg, layers, z, traces="idx")
+    finally:
+        M.moe_set_decode_fused(True, 2)
+    assert np.array_equal(g_none["h"], gf["h"]) and np.array_equal(g_idx["h"], gf["h"])
+    assert np.array_equal(g_idx["idx"], gf["idx"])
 
 
 def test_fused_launch_count(M):
