@@ -354,24 +354,28 @@ int moe_layer_forward(const float* h_in, float* h_out, const uint16_t* x_in, int
 // Shapes the fused batch-1 kernel serves.
 static bool fused_ok(int T, int H, int I, int Is, int E, int k, int bias_per_row, int G) {
   if (!g_decode_fused || T != 1 || bias_per_row) return false;
-  if (H % 64 || H > 4096 || I % 64 || Is % 64 || E % 8 || E > 1024 || k > 8) return false;
-  if (k * I + Is > DF_MAX_ACT || k + (Is + I - 1) / I > DF_MAX_UNITS) return false;
-  if (G <= 0 || (H + G - 1) / G > DF_MAX_ROWS) return false;
+  if (H % 64 || H > DF_MAX_H || I % 64 || Is % 64 || E % 8 || E > DF_MAX_E || k > 8) return false;
+  if (k * I + Is > DF_MAX_ACT) return false;
+  if (G <= 0 || G % DF_CLUSTER || (H + G - 1) / G > DF_MAX_ROWS) return false;
+  if (df_rows_fit(1, H, 2, 2 * (H / 64)) < 2) return false;                       // router jobs: 2 rows
+  if (df_rows_fit(2, H / 2, 4, 2 * (H / 64)) < 1) return false;                   // gate/up row pairs
+  if (df_rows_fit(1, I / 2, 2, 2 * (I / 64)) < 1 || df_rows_fit(1, Is / 2, 2, 2 * (Is / 64)) < 1) return false;
   return true;
 }
 
-// Clusters of the fused kernel that fit at once on this device (cached).
-static int fused_grid(int H) {
-  static int cached[64][2];
+// CTAs of the fused kernel that fit at once on this device (whole clusters; cached).
+static int fused_grid() {
+  static int cached[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  const int which = H > 3072 ? 1 : 0;
-  if (cached[dev][which]) return cached[dev][which];
-  const size_t smem = decode_fused_smem(H, 0);
-  const void* fn = which ? reinterpret_cast<const void*>(k_decode_b1<4>) : reinterpret_cast<const void*>(k_decode_b1<3>);
+  if (cached[dev]) return cached[dev];
+  const size_t smem = decode_fused_smem();
+  const void* fn = reinterpret_cast<const void*>(k_decode_b1);
   if (set_smem(fn, smem)) return 0;
+  int nsm = 0;
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(DF_CLUSTER * 148, 1, 1);
+  cfg.gridDim = dim3(DF_CLUSTER * ((nsm + DF_CLUSTER - 1) / DF_CLUSTER), 1, 1);
   cfg.blockDim = dim3(DF_THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute at[1];
@@ -381,24 +385,23 @@ static int fused_grid(int H) {
   cfg.numAttrs = 1;
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n <= 0) { cudaGetLastError(); return 0; }
-  cached[dev][which] = n * DF_CLUSTER;
-  return cached[dev][which];
+  cached[dev] = n * DF_CLUSTER;
+  return cached[dev];
 }
 
 static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, const moe_qmat* routers,
                         const float* const* biases, const void* const* const* blob_tables, const moe_qmat* shared,
                         uint16_t* x_trace, uint16_t* y_trace, int32_t* idx_trace, float* gates_trace, void* ws,
                         int G, cudaStream_t s) {
+  if (!aligned16(h)) return fail(MOE_ERR_INVALID_ARG, "moe_decode_forward: h must be 16-byte aligned");
   __half* act = static_cast<__half*>(ws);
   unsigned* ctr = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + align_up(static_cast<size_t>(k * I + Is) * 2));
-  const size_t smem = decode_fused_smem(H, k * I + Is);
-  const bool big = H > 3072;
-  const void* fn = big ? reinterpret_cast<const void*>(k_decode_b1<4>) : reinterpret_cast<const void*>(k_decode_b1<3>);
+  const size_t smem = decode_fused_smem();
   int st;
-  if ((st = set_smem(fn, smem))) return st;
+  if ((st = set_smem(reinterpret_cast<const void*>(k_decode_b1), smem))) return st;
   for (int l0 = 0; l0 < L; l0 += DF_MAX_LAYERS) {
     const int nl = L - l0 < DF_MAX_LAYERS ? L - l0 : DF_MAX_LAYERS;
-    static DfArgs args;   // large parameter block; copied into the launch
+    static DfArgs args;   // large parameter block; the launch copies it
     memset(&args, 0, sizeof(args));
     args.h = h; args.H = H; args.I = I; args.Is = Is; args.E = E; args.k = k; args.L = nl;
     blob_offsets(H, I, args.off);
@@ -409,6 +412,9 @@ static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, con
     args.idx_trace = idx_trace ? idx_trace + l0 * Tk : nullptr;
     args.gates_trace = gates_trace ? gates_trace + l0 * Tk : nullptr;
     args.spec = g_decode_spec;
+    args.rg_rows = df_rows_fit(2, H / 2, 4, 2 * (H / 64));
+    args.d_rows = df_rows_fit(1, I / 2, 2, 2 * (I / 64));
+    args.ds_rows = df_rows_fit(1, Is / 2, 2, 2 * (Is / 64));
     for (int l = 0; l < nl; ++l) {
       const moe_qmat& R = routers[l0 + l];
       DfLayer& d = args.layer[l];
@@ -431,8 +437,7 @@ static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, con
     at[0].val.cooperative = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    cudaError_t e = big ? cudaLaunchKernelEx(&cfg, k_decode_b1<4>, args) : cudaLaunchKernelEx(&cfg, k_decode_b1<3>, args);
-    if ((st = cuda_check(e, "k_decode_b1 launch"))) return st;
+    if ((st = cuda_check(cudaLaunchKernelEx(&cfg, k_decode_b1, args), "k_decode_b1 launch"))) return st;
   }
   return MOE_OK;
 }
@@ -470,7 +475,7 @@ int moe_decode_forward(float* h, int T, int H, int I, int Is, int E, int k, int 
   if (!h || !routers || !blob_tables || !shared) return fail(MOE_ERR_INVALID_ARG, "moe_decode_forward: NULL pointer");
   if (ws_bytes < moe_decode_workspace_size(T, H, I, Is, E, k))
     return fail(MOE_ERR_INVALID_ARG, "moe_decode_forward: workspace too small");
-  const int G = (T == 1 && g_decode_fused) ? fused_grid(H) : 0;
+  const int G = (T == 1 && g_decode_fused) ? fused_grid() : 0;
   if (fused_ok(T, H, I, Is, E, k, bias_per_row, G))
     return launch_fused(h, H, I, Is, E, k, L, routers, biases, blob_tables, shared, x_trace, y_trace, idx_trace,
                         gates_trace, ws, G, static_cast<cudaStream_t>(stream));

@@ -1,44 +1,56 @@
 // Batch-1 decode of a stack of routed-MoE layers in one persistent kernel.
 //
 // One launch runs every layer of the step.  The grid is a set of 8-CTA
-// clusters, one CTA per SM, launched cooperatively (all CTAs resident).  Per
-// layer:
-//   phase A  every CTA computes the RMS norm of the residual h (redundantly,
-//            same order, same result); its share of the shared expert's
-//            gate/up rows; then the router: CTA rank r of each cluster
-//            computes the logits of experts [r*E/8, (r+1)*E/8), the cluster
-//            exchanges them through distributed shared memory, and every CTA
-//            selects the top k itself -- no grid-wide step for routing.  Each
-//            CTA then computes its share of the routed experts' gate/up rows
-//            (a contiguous slice of the k*I (slot, row) pairs) and writes the
-//            fp16 activations.
-//   barrier  hierarchical grid barrier (cluster barrier, one atomic per
-//            cluster, cluster barrier).
-//   phase C  every CTA stages all activations (k*I + Is fp16) in shared
-//            memory and computes its slice of output rows: per row the k
-//            routed down dots and the shared down dot, combined in a fixed
-//            order, y = sum_j g_j y_j + ysh; h += y.
-//   barrier
-// Memory traffic is driven by bulk L2 prefetches issued as soon as the
-// addresses are known: after the top-k, a CTA prefetches its routed gate/up
-// rows and its phase-C down rows; at the start of phase C it prefetches the
-// next layer's routing-independent data (router slice, shared-expert rows)
-// and slices of the experts most likely to be chosen (largest router bias),
-// so HBM stays busy while the next layer waits for its routing.
+// clusters, one CTA per SM, launched cooperatively (all CTAs resident).  Each
+// CTA has one loader warp and DF_CW compute warps.
+//
+// Work of one layer, split statically over the G CTAs (CTA c, cluster rank r):
+//   R   router rows [r*E/8, (r+1)*E/8)
+//   SG  shared-expert gate/up row pairs [c*Is/G, (c+1)*Is/G)
+//   RG  routed gate/up (slot, row) pairs [c*k*I/G, (c+1)*k*I/G) of the k*I list
+//   D   output rows [c*H/G, (c+1)*H/G): per routed slot its down rows, then
+//       the shared expert's down rows (DS)
+// Each part is cut into jobs that fit one ring slot.  The loader warp walks
+// the job list in order and copies each job's bytes (weight rows and the
+// 16-byte-aligned windows of their scales and biases) into the next slot of a
+// shared-memory ring with 1-D bulk copies (cp.async.bulk) that complete on
+// the slot's mbarrier; it waits only for a free slot and, before the routed
+// jobs of a layer, for that layer's routing.  The compute warps take the jobs
+// round-robin (job q -> warp q % DF_CW) and read only shared memory:
+//   rms norm of h (every CTA, same order, same result)
+//   R jobs -> logits, broadcast to the 8 CTAs of the cluster with remote
+//     shared-memory stores and remote mbarrier arrivals; every CTA selects
+//     the top k itself, so routing needs no grid-wide step, and hands it to
+//     its loader
+//   SG, RG jobs -> fp16 activations act = gelu_tanh(gate) * up (global)
+//   grid barrier (compute warps: named barrier, cluster mbarriers, one
+//     atomic per cluster)
+//   all activations staged in shared memory; D, DS jobs -> per-row dots;
+//     y = sum_j g_j y_j + ysh in a fixed order; h += y
+//   grid barrier
+// HBM is kept busy with bulk L2 prefetches: when a layer's routing is known
+// the loader prefetches all of its routed rows; when it starts a layer it
+// prefetches the next layer's routing-independent rows and slices of the
+// experts with the largest router bias (the likeliest choices).
 // Every wait is bounded (about two seconds); a wait that runs out sets the
-// device check word and the kernel runs on to its end.
+// device check word and the thread runs on to the end.
 #include <cooperative_groups.h>
 
 namespace moe {
 
-constexpr int DF_THREADS = 384;
-constexpr int DF_WARPS = DF_THREADS / 32;
+constexpr int DF_CW = 15;                       // compute warps
+constexpr int DF_THREADS = (DF_CW + 1) * 32;    // + loader warp (warp DF_CW)
 constexpr int DF_CLUSTER = 8;
 constexpr int DF_MAX_LAYERS = 48;
-constexpr int DF_MAX_H = 4096;
-constexpr int DF_MAX_ACT = 16384;      // k*I + Is
-constexpr int DF_MAX_ROWS = 64;        // output rows per CTA in phase C
-constexpr int DF_MAX_UNITS = 16;       // down dots per output row (k + shared pieces)
+constexpr int DF_MAX_H = 3072;
+constexpr int DF_CPL = 3;                       // uint4 chunks per lane of a gate/up row (H <= 3072)
+constexpr int DF_MAX_ACT = 8192;                // k*I + Is
+constexpr int DF_MAX_ROWS = 32;                 // output rows per CTA
+constexpr int DF_NS = 16;                       // ring slots
+constexpr int DF_SLOT_Q = 8192;                 // weight bytes per slot
+constexpr int DF_SLOT_S = 1024;                 // scale/bias window bytes per slot
+constexpr int DF_SLOT = DF_SLOT_Q + DF_SLOT_S;
+constexpr int DF_MAX_E = 256;
 
 struct DfLayer {
   const uint32_t* rq; const uint16_t* rs; const uint16_t* rb;   // router [E, H], 8-bit
@@ -55,9 +67,11 @@ struct DfArgs {
   unsigned* counter;                // workspace: grid barrier counter (zeroed before launch)
   uint16_t* x_trace; uint16_t* y_trace; int32_t* idx_trace; float* gates_trace;
   int spec;                         // experts speculatively prefetched per layer
+  int rg_rows, d_rows, ds_rows;     // row pairs per SG/RG job, rows per D / DS job
   DfLayer layer[DF_MAX_LAYERS];
 };
 
+// ------------------------------------------------------------------ PTX bits
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -71,187 +85,406 @@ __device__ __forceinline__ uint64_t df_clock() {
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
   return t;
 }
-
-// L2 prefetch of [p, p + bytes): the 16-byte-aligned window around it (arrays
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void df_mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void df_mbar_arrive(uint32_t bar) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void df_mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
+               "r"(bytes)
+               : "memory");
+}
+// arrive on the mbarrier at the same shared-memory offset in CTA `rank` of the cluster
+__device__ __forceinline__ void df_mbar_arrive_remote(uint32_t bar, uint32_t rank) {
+  asm volatile(
+      "{\n\t.reg .b32 ra;\n\tmapa.shared::cluster.u32 ra, %0, %1;\n\t"
+      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(bar),
+      "r"(rank)
+      : "memory");
+}
+__device__ __forceinline__ void df_st_remote_f32(uint32_t addr, uint32_t rank, float v) {
+  asm volatile(
+      "{\n\t.reg .b32 ra;\n\tmapa.shared::cluster.u32 ra, %0, %1;\n\tst.shared::cluster.f32 [ra], %2;\n\t}" ::"r"(
+          addr),
+      "r"(rank), "f"(v)
+      : "memory");
+}
+// bounded wait on a phase parity; `cluster` acquires at cluster scope
+__device__ __forceinline__ bool df_mbar_wait(uint32_t bar, uint32_t parity, bool cluster = false) {
+  uint64_t t0 = 0;
+  for (uint32_t i = 0;; ++i) {
+    uint32_t ok;
+    if (cluster)
+      asm volatile(
+          "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+          "selp.u32 %0, 1, 0, p;\n\t}"
+          : "=r"(ok)
+          : "r"(bar), "r"(parity)
+          : "memory");
+    else
+      asm volatile(
+          "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+          "selp.u32 %0, 1, 0, p;\n\t}"
+          : "=r"(ok)
+          : "r"(bar), "r"(parity)
+          : "memory");
+    if (ok) return true;
+    if ((i & 255u) == 0) {
+      const uint64_t now = df_clock();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > 2000000000ull) break;
+    }
+  }
+  flag_check(CHECK_WAIT);
+  return false;
+}
+__device__ __forceinline__ void df_bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+// L2 prefetch of the 16-byte-aligned window around [p, p + bytes).  Arrays
 // handed to this kernel are 16-byte aligned with sizes that are multiples of
-// 16, so the window stays inside them).
+// 16, so the window stays inside them.
 __device__ __forceinline__ void prefetch_l2(const void* p, size_t bytes) {
   if (bytes == 0) return;
   uintptr_t a = reinterpret_cast<uintptr_t>(p) & ~uintptr_t(15);
-  uintptr_t e = (reinterpret_cast<uintptr_t>(p) + bytes + 15) & ~uintptr_t(15);
+  const uintptr_t e = (reinterpret_cast<uintptr_t>(p) + bytes + 15) & ~uintptr_t(15);
   while (a < e) {
     const uint32_t n = static_cast<uint32_t>((e - a) < 65536 ? (e - a) : 65536);
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(n) : "memory");
     a += n;
   }
 }
-
-// Slice c of G of an array of `total` bytes (total a multiple of 16).
 __device__ __forceinline__ void prefetch_slice(const void* base, size_t total, int c, int G) {
   const size_t b0 = total * c / G, b1 = total * (c + 1) / G;
   prefetch_l2(static_cast<const uint8_t*>(base) + b0, b1 - b0);
 }
-
 __device__ __forceinline__ uint4 ldcg_v4(const void* p) {
   uint4 r;
   asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
 }
-__device__ __forceinline__ uint32_t ldg_nc_u32(const void* p) {
-  uint32_t r;
-  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
-  return r;
+__device__ __forceinline__ void df_named_sync() {   // the compute warps of this CTA
+  asm volatile("bar.sync 1, %0;" ::"n"(DF_CW * 32) : "memory");
 }
 
-// Hierarchical grid barrier: cluster barrier; one thread per cluster adds to
-// the counter and waits for all clusters; cluster barrier.  `target` grows by
-// the number of clusters at every barrier of the launch.
-__device__ void df_grid_sync(cooperative_groups::cluster_group& cl, unsigned* ctr, unsigned target) {
-  cl.sync();
-  if (cl.block_rank() == 0 && threadIdx.x == 0) {
-    __threadfence();
-    red_release_gpu(ctr, 1u);
-    const uint64_t t0 = df_clock();
-    while (ld_acquire_gpu(ctr) < target) {
-      if (df_clock() - t0 > 2000000000ull) { flag_check(CHECK_WAIT); break; }
-    }
-    __threadfence();
+// ---------------------------------------------------------------- job list
+enum : int { JOB_R = 0, JOB_SG = 1, JOB_RG = 2, JOB_D = 3, JOB_DS = 4 };
+
+struct DfJob {
+  int kind;
+  int slot;      // routed slot (RG, D)
+  int r0, n;     // first row (or row pair) and count
+};
+
+struct DfShape {
+  int H, I, Is, E, k, G, c, rank;
+  int epc, s0, s1, r0, r1, o0, o1;
+  int rgn, dn, dsn;
+  int nR, nSG, nRG, nD, nDS;
+};
+
+__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+__device__ inline int df_rg_jobs(const DfShape& s) {
+  if (s.r1 <= s.r0) return 0;
+  int n = 0;
+  for (int j = s.r0 / s.I; j <= (s.r1 - 1) / s.I; ++j) {
+    const int a = max(s.r0, j * s.I), b = min(s.r1, (j + 1) * s.I);
+    n += ceil_div(b - a, s.rgn);
   }
-  cl.sync();
-  if (threadIdx.x == 0) __threadfence();
-  __syncthreads();
+  return n;
 }
 
-// One row-pair (gate row i, up row i) against the register x; returns
-// act = gelu_tanh(gate . x) * (up . x) in every lane.
-template <int DF_CPL>
-__device__ __forceinline__ float df_gateup_row(const uint8_t* gq, const uint16_t* gs, const uint16_t* gb,
-                                               const uint8_t* uq, const uint16_t* us, const uint16_t* ub,
-                                               int i, int K, int nch, const uint32_t (&xp)[DF_CPL][16],
-                                               const float2 (&xst)[DF_CPL]) {
-  const int lane = threadIdx.x & 31;
-  const size_t rq = static_cast<size_t>(i) * (K / 2), rsb = static_cast<size_t>(i) * (K / 64);
-  uint4 qg[DF_CPL], qu[DF_CPL];
-  float sg[DF_CPL], bg[DF_CPL], su[DF_CPL], bu[DF_CPL];
-#pragma unroll
-  for (int j = 0; j < DF_CPL; ++j) {
-    const int c = lane + 32 * j;
-    if (c < nch) {
-      qg[j] = ldg_nc_v4(gq + rq + 16 * c);
-      qu[j] = ldg_nc_v4(uq + rq + 16 * c);
-      sg[j] = bf16_to_f32(ldg_u16(gs + rsb + (c >> 1)));
-      bg[j] = bf16_to_f32(ldg_u16(gb + rsb + (c >> 1)));
-      su[j] = bf16_to_f32(ldg_u16(us + rsb + (c >> 1)));
-      bu[j] = bf16_to_f32(ldg_u16(ub + rsb + (c >> 1)));
+__device__ inline DfJob df_job(const DfShape& s, int q) {
+  DfJob J{};
+  if (q < s.nR) {
+    J.kind = JOB_R; J.r0 = s.rank * s.epc + q * 2; J.n = min(2, s.epc - q * 2);
+    return J;
+  }
+  q -= s.nR;
+  if (q < s.nSG) {
+    J.kind = JOB_SG; J.r0 = s.s0 + q * s.rgn; J.n = min(s.rgn, s.s1 - J.r0);
+    return J;
+  }
+  q -= s.nSG;
+  if (q < s.nRG) {
+    for (int j = s.r0 / s.I; j <= (s.r1 - 1) / s.I; ++j) {
+      const int a = max(s.r0, j * s.I), b = min(s.r1, (j + 1) * s.I);
+      const int nj = ceil_div(b - a, s.rgn);
+      if (q < nj) {
+        J.kind = JOB_RG; J.slot = j; J.r0 = a - j * s.I + q * s.rgn; J.n = min(s.rgn, b - a - q * s.rgn);
+        return J;
+      }
+      q -= nj;
     }
   }
-  float a = 0.f, u = 0.f;
-#pragma unroll
-  for (int j = 0; j < DF_CPL; ++j) {
-    const int c = lane + 32 * j;
-    if (c < nch) {
-      const float dg = dot_chunk4(qg[j], xp[j]);
-      const float du = dot_chunk4(qu[j], xp[j]);
-      a += sg[j] * (dg - xst[j].x) + bg[j] * xst[j].y;
-      u += su[j] * (du - xst[j].x) + bu[j] * xst[j].y;
-    }
+  q -= s.nRG;
+  if (q < s.nD) {
+    const int per = ceil_div(s.o1 - s.o0, s.dn);
+    J.kind = JOB_D; J.slot = q / per; J.r0 = s.o0 + (q % per) * s.dn; J.n = min(s.dn, s.o1 - J.r0);
+    return J;
   }
-  a = warp_sum(a);
-  u = warp_sum(u);
-  return gelu_tanh(a) * u;
+  q -= s.nD;
+  J.kind = JOB_DS; J.r0 = s.o0 + q * s.dsn; J.n = min(s.dsn, s.o1 - J.r0);
+  return J;
 }
 
-template <int DF_CPL>
+// 16-byte-aligned window covering rows [r0, r0+n) of a bf16 array with `per`
+// values per row; skew = offset of row r0 inside the window.
+__device__ __forceinline__ void sb_window(const uint16_t* base, int per, int r0, int n, const uint8_t*& src,
+                                          uint32_t& bytes, uint32_t& skew) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(base) + static_cast<size_t>(r0) * per * 2;
+  const uintptr_t e = a + static_cast<size_t>(n) * per * 2;
+  const uintptr_t a16 = a & ~uintptr_t(15), e16 = (e + 15) & ~uintptr_t(15);
+  src = reinterpret_cast<const uint8_t*>(a16);
+  bytes = static_cast<uint32_t>(e16 - a16);
+  skew = static_cast<uint32_t>(a - a16);
+}
+
+// The copies of one job: weight runs at the start of the slot (run i at
+// i * qbytes), then the scale/bias windows in the slot's scale area; sk[i]
+// is the offset of window i's first row inside that area.
+struct DfJobCopies {
+  const uint8_t* src[6];
+  uint32_t dst[6];
+  uint32_t len[6];
+  int n;
+  uint32_t qbytes;
+  uint32_t sk[4];
+  uint32_t bytes;
+};
+
+__device__ inline DfJobCopies df_job_copies(const DfShape& s, const DfJob& J, const DfArgs& a, const DfLayer& W,
+                                            const int* sel) {
+  DfJobCopies C{};
+  const int H = s.H, I = s.I, Is = s.Is;
+  const uint8_t* q[2] = {nullptr, nullptr};
+  const uint16_t* sc[4] = {nullptr, nullptr, nullptr, nullptr};
+  int per = 0, nq = 0, ns = 0;
+  if (J.kind == JOB_R) {
+    q[0] = reinterpret_cast<const uint8_t*>(W.rq) + static_cast<size_t>(J.r0) * H;
+    C.qbytes = static_cast<uint32_t>(J.n) * H; nq = 1;
+    sc[0] = W.rs; sc[1] = W.rb; ns = 2; per = H / 64;
+  } else if (J.kind == JOB_SG || J.kind == JOB_RG) {
+    const uint8_t *gq, *uq;
+    const uint16_t *gs, *gb, *us, *ub;
+    if (J.kind == JOB_SG) {
+      gq = reinterpret_cast<const uint8_t*>(W.sq[0]); uq = reinterpret_cast<const uint8_t*>(W.sq[1]);
+      gs = W.ss[0]; gb = W.sb[0]; us = W.ss[1]; ub = W.sb[1];
+    } else {
+      const uint8_t* blob = static_cast<const uint8_t*>(W.blobs[sel[J.slot]]);
+      gq = blob + a.off[0]; uq = blob + a.off[3];
+      gs = reinterpret_cast<const uint16_t*>(blob + a.off[1]); gb = reinterpret_cast<const uint16_t*>(blob + a.off[2]);
+      us = reinterpret_cast<const uint16_t*>(blob + a.off[4]); ub = reinterpret_cast<const uint16_t*>(blob + a.off[5]);
+    }
+    q[0] = gq + static_cast<size_t>(J.r0) * (H / 2);
+    q[1] = uq + static_cast<size_t>(J.r0) * (H / 2);
+    C.qbytes = static_cast<uint32_t>(J.n) * (H / 2); nq = 2;
+    sc[0] = gs; sc[1] = gb; sc[2] = us; sc[3] = ub; ns = 4; per = H / 64;
+  } else if (J.kind == JOB_D) {
+    const uint8_t* blob = static_cast<const uint8_t*>(W.blobs[sel[J.slot]]);
+    q[0] = blob + a.off[6] + static_cast<size_t>(J.r0) * (I / 2);
+    C.qbytes = static_cast<uint32_t>(J.n) * (I / 2); nq = 1;
+    sc[0] = reinterpret_cast<const uint16_t*>(blob + a.off[7]);
+    sc[1] = reinterpret_cast<const uint16_t*>(blob + a.off[8]);
+    ns = 2; per = I / 64;
+  } else {
+    q[0] = reinterpret_cast<const uint8_t*>(W.sq[2]) + static_cast<size_t>(J.r0) * (Is / 2);
+    C.qbytes = static_cast<uint32_t>(J.n) * (Is / 2); nq = 1;
+    sc[0] = W.ss[2]; sc[1] = W.sb[2]; ns = 2; per = Is / 64;
+  }
+  uint32_t total = 0;
+  for (int i = 0; i < nq; ++i) {
+    C.src[C.n] = q[i]; C.dst[C.n] = static_cast<uint32_t>(i) * C.qbytes; C.len[C.n] = C.qbytes; ++C.n;
+    total += C.qbytes;
+  }
+  uint32_t so = 0;
+  for (int i = 0; i < ns; ++i) {
+    const uint8_t* src; uint32_t bytes, skew;
+    sb_window(sc[i], per, J.r0, J.n, src, bytes, skew);
+    C.src[C.n] = src; C.dst[C.n] = DF_SLOT_Q + so; C.len[C.n] = bytes; ++C.n;
+    C.sk[i] = so + skew;
+    so += bytes;
+    total += bytes;
+  }
+  C.bytes = total;
+  return C;
+}
+
+// --------------------------------------------------------------- the kernel
 __global__ void __cluster_dims__(DF_CLUSTER, 1, 1) __launch_bounds__(DF_THREADS, 1)
 k_decode_b1(const __grid_constant__ DfArgs a) {
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
-  extern __shared__ __align__(16) unsigned char smem[];
-  const int H = a.H, I = a.I, Is = a.Is, E = a.E, k = a.k;
-  const int G = gridDim.x, c = blockIdx.x;
-  const int rank = static_cast<int>(cl.block_rank());
-  const unsigned nclusters = G / DF_CLUSTER;
+  extern __shared__ __align__(128) unsigned char smem[];
+  DfShape s;
+  s.H = a.H; s.I = a.I; s.Is = a.Is; s.E = a.E; s.k = a.k;
+  s.G = gridDim.x; s.c = blockIdx.x; s.rank = static_cast<int>(cl.block_rank());
+  s.epc = s.E / DF_CLUSTER;
+  const int kI = s.k * s.I, nact = kI + s.Is;
+  s.s0 = (int)((long)s.c * s.Is / s.G); s.s1 = (int)((long)(s.c + 1) * s.Is / s.G);
+  s.r0 = (int)((long)s.c * kI / s.G); s.r1 = (int)((long)(s.c + 1) * kI / s.G);
+  s.o0 = (int)((long)s.c * s.H / s.G); s.o1 = (int)((long)(s.c + 1) * s.H / s.G);
+  s.rgn = a.rg_rows; s.dn = a.d_rows; s.dsn = a.ds_rows;
+  s.nR = ceil_div(s.epc, 2);
+  s.nSG = ceil_div(s.s1 - s.s0, s.rgn);
+  s.nRG = df_rg_jobs(s);
+  s.nD = s.k * ceil_div(s.o1 - s.o0, s.dn);
+  s.nDS = ceil_div(s.o1 - s.o0, s.dsn);
+  const int njobs = s.nR + s.nSG + s.nRG + s.nD + s.nDS;
+  const int H = s.H, I = s.I, Is = s.Is, E = s.E, k = s.k;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kI = k * I, nact = kI + Is;
+  const unsigned nclusters = s.G / DF_CLUSTER;
 
   // shared memory
-  float* xs = reinterpret_cast<float*>(smem);                          // [H] layer input (bf16 values)
-  float* red = xs + DF_MAX_H;                                          // [32] reduction scratch
-  float* lg_part = red + 32;                                           // [E/8] this CTA's logits
-  float* lg_all = lg_part + 128;                                       // [E]
-  int* sel_idx = reinterpret_cast<int*>(lg_all + 1024);                // [8]
-  float* sel_g = reinterpret_cast<float*>(sel_idx + 8);                // [8]
-  int* spec_ids = reinterpret_cast<int*>(sel_g + 8);                   // [8]
-  float* part = reinterpret_cast<float*>(spec_ids + 8);                // [DF_MAX_ROWS][DF_MAX_UNITS]
-  uint4* actP = reinterpret_cast<uint4*>(part + DF_MAX_ROWS * DF_MAX_UNITS);  // [nact/8] paired words
+  unsigned char* ring = smem;                                          // [NS][DF_SLOT]
+  float* xs = reinterpret_cast<float*>(ring + DF_NS * DF_SLOT);        // [H] layer input (bf16 values)
+  uint4* actP = reinterpret_cast<uint4*>(xs + DF_MAX_H);               // [nact/8] paired activations
   float2* actS = reinterpret_cast<float2*>(actP + DF_MAX_ACT / 8);     // [nact/8] (off, sum) per word
+  float* part = reinterpret_cast<float*>(actS + DF_MAX_ACT / 8);       // [MAX_ROWS][9]
+  float* lg_all = part + DF_MAX_ROWS * 9;                              // [E]
+  float* red = lg_all + DF_MAX_E;                                      // [32]
+  int* sel = reinterpret_cast<int*>(red + 32);                         // [2][8]
+  float* selg = reinterpret_cast<float*>(sel + 16);                    // [8]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(selg + 8);
+  const uint32_t bar0 = smem_addr(bars);
+  auto full_bar = [&](int i) { return bar0 + 8u * i; };
+  auto empty_bar = [&](int i) { return bar0 + 8u * (DF_NS + i); };
+  const uint32_t route_bar = bar0 + 8u * (2 * DF_NS);
+  const uint32_t lg_bar = route_bar + 8u;
+  const uint32_t clA_bar = route_bar + 16u;     // in rank 0: all CTAs of the cluster arrived
+  const uint32_t clR_bar = route_bar + 24u;     // every CTA: released
 
-  // static work split
-  const int s0 = (int)((long)c * Is / G), s1 = (int)((long)(c + 1) * Is / G);        // shared gate/up pairs
-  const int r0 = (int)((long)c * kI / G), r1 = (int)((long)(c + 1) * kI / G);        // routed (slot, row)
-  const int o0 = (int)((long)c * H / G), o1 = (int)((long)(c + 1) * H / G);          // output rows
-  const int nsub = (Is + I - 1) / I;                                                 // shared down pieces
-  const int upr = k + nsub;                                                          // units per row
-  const int nch = H / 32;
-  const int epc = E / DF_CLUSTER;
-  unsigned bar_target = 0;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < DF_NS; ++i) {
+      df_mbar_init(full_bar(i), 1);
+      df_mbar_init(empty_bar(i), 1);
+    }
+    df_mbar_init(route_bar, 1);
+    df_mbar_init(lg_bar, DF_CLUSTER * s.epc);
+    df_mbar_init(clA_bar, DF_CLUSTER);
+    df_mbar_init(clR_bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  cl.sync();        // every CTA's barriers initialised before any remote arrival
 
-  // prefetch the routing-independent data of layer l (and likely experts)
-  auto prefetch_independent = [&](int l) {
-    const DfLayer& W = a.layer[l];
-    if (threadIdx.x == 0) {
-      // router: 1/G slice of the whole matrix (every cluster reads all of it)
-      prefetch_slice(W.rq, static_cast<size_t>(E) * H, c, G);
-    } else if (threadIdx.x == 32) {
-      prefetch_slice(W.rs, static_cast<size_t>(E) * (H / 64) * 2, c, G);
-      prefetch_slice(W.rb, static_cast<size_t>(E) * (H / 64) * 2, c, G);
-    } else if (threadIdx.x == 64) {
-      for (int m = 0; m < 2; ++m) {
-        prefetch_l2(reinterpret_cast<const uint8_t*>(W.sq[m]) + static_cast<size_t>(s0) * (H / 2),
-                    static_cast<size_t>(s1 - s0) * (H / 2));
-        prefetch_l2(W.ss[m] + static_cast<size_t>(s0) * (H / 64), static_cast<size_t>(s1 - s0) * (H / 64) * 2);
-        prefetch_l2(W.sb[m] + static_cast<size_t>(s0) * (H / 64), static_cast<size_t>(s1 - s0) * (H / 64) * 2);
-      }
-    } else if (threadIdx.x == 96) {
-      prefetch_l2(reinterpret_cast<const uint8_t*>(W.sq[2]) + static_cast<size_t>(o0) * (Is / 2),
-                  static_cast<size_t>(o1 - o0) * (Is / 2));
-      prefetch_l2(W.ss[2] + static_cast<size_t>(o0) * (Is / 64), static_cast<size_t>(o1 - o0) * (Is / 64) * 2);
-      prefetch_l2(W.sb[2] + static_cast<size_t>(o0) * (Is / 64), static_cast<size_t>(o1 - o0) * (Is / 64) * 2);
-    } else if (warp == 4 && W.bias != nullptr && a.spec > 0) {
-      // the experts with the largest router bias, 1/G of each blob
-      int bi[8];
-      for (int j = 0; j < 8; ++j) bi[j] = 0;
-      unsigned taken = 0;
-      for (int r = 0; r < a.spec; ++r) {
-        float v = -INFINITY;
-        int id = 0x7fffffff;
-        for (int s = 0, e = lane; e < E; ++s, e += 32) {
-          if (taken & (1u << s)) continue;
-          const float b = W.bias[e];
-          if (b > v || (b == v && e < id)) { v = b; id = e; }
+  if (warp == DF_CW) {
+    // ================================================================ loader
+    uint32_t g = 0;   // job sequence over the launch
+    for (int l = 0; l < a.L; ++l) {
+      const DfLayer& W = a.layer[l];
+      if (lane == 0) {
+        // routing-independent rows of this layer (layer 0) and of the next one
+        for (int ll = (l == 0 ? 0 : l + 1); ll <= l + 1 && ll < a.L; ++ll) {
+          const DfLayer& V = a.layer[ll];
+          prefetch_l2(reinterpret_cast<const uint8_t*>(V.rq) + static_cast<size_t>(s.rank * s.epc) * H,
+                      static_cast<size_t>(s.epc) * H);
+          for (int m = 0; m < 2; ++m)
+            prefetch_l2(reinterpret_cast<const uint8_t*>(V.sq[m]) + static_cast<size_t>(s.s0) * (H / 2),
+                        static_cast<size_t>(s.s1 - s.s0) * (H / 2));
+          prefetch_l2(reinterpret_cast<const uint8_t*>(V.sq[2]) + static_cast<size_t>(s.o0) * (Is / 2),
+                      static_cast<size_t>(s.o1 - s.o0) * (Is / 2));
         }
-        for (int o = 16; o > 0; o >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, v, o);
-          const int oi = __shfl_xor_sync(0xffffffffu, id, o);
-          if (ov > v || (ov == v && oi < id)) { v = ov; id = oi; }
-        }
-        if ((id & 31) == lane) taken |= 1u << (id >> 5);
-        bi[r] = id;
       }
-      if (lane < a.spec) {
-        const size_t bb = a.off[8] + static_cast<size_t>(H) * (I / 64) * 2;   // blob bytes
-        prefetch_slice(W.blobs[bi[lane]], bb, c, G);
+      if (l + 1 < a.L && a.spec > 0 && a.layer[l + 1].bias != nullptr) {
+        // the experts of the next layer with the largest bias: slice c of G of each blob
+        const DfLayer& V = a.layer[l + 1];
+        unsigned taken = 0;
+        int my_id = -1;
+        for (int r = 0; r < a.spec && r < 8; ++r) {
+          float v = -INFINITY;
+          int id = 0x7fffffff;
+          for (int t = 0, e = lane; e < E; ++t, e += 32) {
+            if (taken & (1u << t)) continue;
+            const float b = V.bias[e];
+            if (b > v || (b == v && e < id)) { v = b; id = e; }
+          }
+          for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, id, o);
+            if (ov > v || (ov == v && oi < id)) { v = ov; id = oi; }
+          }
+          if ((id & 31) == lane) taken |= 1u << (id >> 5);
+          if (lane == r) my_id = id;
+        }
+        if (my_id >= 0 && my_id < E) {
+          const size_t bb = a.off[8] + static_cast<size_t>(H) * (I / 64) * 2;
+          prefetch_slice(V.blobs[my_id], bb, s.c, s.G);
+        }
+      }
+      const int* sl = sel + 8 * (l & 1);
+      for (int q = 0; q < njobs; ++q, ++g) {
+        if (q == s.nR + s.nSG) {
+          // routed jobs need this layer's routing; then all routed rows into L2 at once
+          df_mbar_wait(route_bar, l & 1);
+          for (int qq = q + lane; qq < njobs; qq += 32) {
+            const DfJobCopies C2 = df_job_copies(s, df_job(s, qq), a, W, sl);
+            for (int i = 0; i < C2.n; ++i) prefetch_l2(C2.src[i], C2.len[i]);
+          }
+        }
+        const int slot = g % DF_NS;
+        if (g >= DF_NS) df_mbar_wait(empty_bar(slot), ((g / DF_NS) + 1) & 1);
+        const DfJobCopies C = df_job_copies(s, df_job(s, q), a, W, sl);
+        if (lane == 0) df_mbar_expect_tx(full_bar(slot), C.bytes);
+        __syncwarp();
+        if (lane < C.n)
+          df_bulk_g2s(smem_addr(ring + slot * DF_SLOT + C.dst[lane]), C.src[lane], C.len[lane], full_bar(slot));
+        __syncwarp();
       }
     }
-  };
+    return;
+  }
 
-  prefetch_independent(0);
+  // ================================================================== compute
+  const int nch = H / 32;
+  uint32_t g = 0;            // job sequence (same numbering as the loader)
+  unsigned bar_target = 0;
+  unsigned gen = 0;          // grid barriers passed
+  auto grid_sync = [&]() {
+    df_named_sync();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      df_mbar_arrive_remote(clA_bar, 0);
+      if (s.rank == 0) {
+        df_mbar_wait(clA_bar, gen & 1, true);
+        bar_target += nclusters;
+        red_release_gpu(a.counter, 1u);
+        const uint64_t t0 = df_clock();
+        while (ld_acquire_gpu(a.counter) < bar_target) {
+          if (df_clock() - t0 > 2000000000ull) { flag_check(CHECK_WAIT); break; }
+        }
+        for (int r = 0; r < DF_CLUSTER; ++r) df_mbar_arrive_remote(clR_bar, r);
+      }
+      df_mbar_wait(clR_bar, gen & 1, true);
+      __threadfence();
+    }
+    ++gen;
+    df_named_sync();
+  };
+  auto slot_of = [&](int q) { return static_cast<int>((g + q) % DF_NS); };
+  auto wait_full = [&](int q) {
+    const uint32_t gg = g + q;
+    df_mbar_wait(full_bar(gg % DF_NS), (gg / DF_NS) & 1);
+  };
+  auto release = [&](int q) {
+    __syncwarp();
+    if (lane == 0) df_mbar_arrive(empty_bar(slot_of(q)));
+  };
 
   for (int l = 0; l < a.L; ++l) {
     const DfLayer& W = a.layer[l];
-    // ------------------------------------------------------------- A0: rms norm
+    int* sl_sel = sel + 8 * (l & 1);
+    // ------------------------------------------------------ A0: rms norm
     float ss = 0.f;
-    for (int i = threadIdx.x * 4; i < H; i += DF_THREADS * 4) {
+    for (int i = threadIdx.x * 4; i < H; i += DF_CW * 32 * 4) {
       const uint4 u = ldcg_v4(a.h + i);
       const float v0 = __uint_as_float(u.x), v1 = __uint_as_float(u.y), v2 = __uint_as_float(u.z),
                   v3 = __uint_as_float(u.w);
@@ -260,111 +493,58 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
     }
     ss = warp_sum(ss);
     if (lane == 0) red[warp] = ss;
-    __syncthreads();
+    df_named_sync();
     if (warp == 0) {
-      float v = lane < DF_WARPS ? red[lane] : 0.f;
+      float v = lane < DF_CW ? red[lane] : 0.f;
       v = warp_sum(v);
-      if (lane == 0) red[DF_WARPS] = v;
+      if (lane == 0) red[DF_CW] = v;
     }
-    __syncthreads();
-    const float rr = sqrtf(red[DF_WARPS] / static_cast<float>(H) + 1e-6f);
-    for (int i = threadIdx.x; i < H; i += DF_THREADS) {
+    df_named_sync();
+    const float rr = sqrtf(red[DF_CW] / static_cast<float>(H) + 1e-6f);
+    for (int i = threadIdx.x; i < H; i += DF_CW * 32) {
       const uint16_t b = f32_to_bf16(__fdiv_rn(xs[i], rr));
       xs[i] = bf16_to_f32(b);
-      if (c == 0 && a.x_trace) a.x_trace[static_cast<size_t>(l) * H + i] = b;
+      if (s.c == 0 && a.x_trace) a.x_trace[static_cast<size_t>(l) * H + i] = b;
     }
-    __syncthreads();
+    df_named_sync();
 
-    // ------------------------------------------------------ router (cluster)
-    for (int el = warp; el < epc; el += DF_WARPS) {
-      const int e = rank * epc + el;
-      const uint8_t* qrow = reinterpret_cast<const uint8_t*>(W.rq) + static_cast<size_t>(e) * H;
-      float acc = 0.f;
-      for (int cc = lane; cc < H / 16; cc += 32) {
-        const uint4 q = ldg_nc_v4(qrow + 16 * cc);
-        const float sc = bf16_to_f32(ldg_u16(W.rs + static_cast<size_t>(e) * (H / 64) + (cc >> 2)));
-        const float bi = bf16_to_f32(ldg_u16(W.rb + static_cast<size_t>(e) * (H / 64) + (cc >> 2)));
-        const float* xv = xs + 16 * cc;
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-        float a0 = 0.f, a1 = 0.f, off = 0.f;
+    // ------------------------------------------------------------- R jobs
+    for (int q = warp; q < s.nR; q += DF_CW) {
+      const DfJob J = df_job(s, q);
+      const DfJobCopies C = df_job_copies(s, J, a, W, sl_sel);
+      wait_full(q);
+      const unsigned char* slp = ring + slot_of(q) * DF_SLOT;
+      for (int r = 0; r < J.n; ++r) {
+        const int e = J.r0 + r;
+        const uint8_t* qrow = slp + static_cast<size_t>(r) * H;
+        const uint16_t* S = reinterpret_cast<const uint16_t*>(slp + DF_SLOT_Q + C.sk[0]) + r * (H / 64);
+        const uint16_t* B = reinterpret_cast<const uint16_t*>(slp + DF_SLOT_Q + C.sk[1]) + r * (H / 64);
+        float acc = 0.f;
+        for (int cc = lane; cc < H / 16; cc += 32) {
+          const uint4 q4 = *reinterpret_cast<const uint4*>(qrow + 16 * cc);
+          const float sc = bf16_to_f32(S[cc >> 2]), bi = bf16_to_f32(B[cc >> 2]);
+          const float* xv = xs + 16 * cc;
+          const uint32_t w[4] = {q4.x, q4.y, q4.z, q4.w};
+          float a0 = 0.f, a1 = 0.f, off = 0.f;
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const uint32_t p[2] = {pack_half2(xv[4 * m], xv[4 * m + 2]), pack_half2(xv[4 * m + 1], xv[4 * m + 3])};
-          dot_word8(w[m], p, a0, a1);
-          const float2 f0 = unpack_half2(p[0]), f1 = unpack_half2(p[1]);
-          off += (f0.x + f0.y) + (f1.x + f1.y);
+          for (int m = 0; m < 4; ++m) {
+            const uint32_t p[2] = {pack_half2(xv[4 * m], xv[4 * m + 2]), pack_half2(xv[4 * m + 1], xv[4 * m + 3])};
+            dot_word8(w[m], p, a0, a1);
+            const float2 f0 = unpack_half2(p[0]), f1 = unpack_half2(p[1]);
+            off += (f0.x + f0.y) + (f1.x + f1.y);
+          }
+          acc += sc * ((a0 + a1) - 1024.f * off) + bi * off;
         }
-        acc += sc * ((a0 + a1) - 1024.f * off) + bi * off;
-      }
-      acc = warp_sum(acc);
-      if (lane == 0) lg_part[el] = acc + (W.bias ? W.bias[e] : 0.f);
-    }
-    cl.sync();
-    for (int e = threadIdx.x; e < E; e += DF_THREADS) {
-      const float* src = cl.map_shared_rank(lg_part, e / epc);
-      lg_all[e] = src[e % epc];
-    }
-    cl.sync();
-    if (warp == 0) {
-      unsigned taken = 0u;
-      float sv[8];
-      int si[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j >= k) break;
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
-        for (int s = 0, e = lane; e < E; ++s, e += 32) {
-          if (taken & (1u << s)) continue;
-          const float v = lg_all[e];
-          if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; }
-        }
-        for (int o = 16; o > 0; o >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-          if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-        }
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-        sv[j] = bv;
-        si[j] = bi;
-      }
-      if (lane == 0) {
-        float z[8], den = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) { z[j] = j < k ? expf(sv[j] - sv[0]) : 0.f; den += z[j]; }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (j >= k) break;
-          sel_idx[j] = si[j];
-          sel_g[j] = z[j] / den;
-          if (c == 0 && a.idx_trace) a.idx_trace[static_cast<size_t>(l) * k + j] = si[j];
-          if (c == 0 && a.gates_trace) a.gates_trace[static_cast<size_t>(l) * k + j] = z[j] / den;
+        acc = warp_sum(acc) + (W.bias ? W.bias[e] : 0.f);
+        if (lane < DF_CLUSTER) {          // broadcast the logit to every CTA of the cluster
+          df_st_remote_f32(smem_addr(lg_all + e), lane, acc);
+          df_mbar_arrive_remote(lg_bar, lane);
         }
       }
-    }
-    __syncthreads();
-
-    // prefetch this CTA's routed rows (gate/up slice and phase-C down rows)
-    if (warp == 1) {
-      for (int j = lane; j < k; j += 32) {
-        const uint8_t* blob = static_cast<const uint8_t*>(W.blobs[sel_idx[j]]);
-        prefetch_l2(blob + a.off[6] + static_cast<size_t>(o0) * (I / 2), static_cast<size_t>(o1 - o0) * (I / 2));
-        prefetch_l2(blob + a.off[7] + static_cast<size_t>(o0) * (I / 64) * 2, static_cast<size_t>(o1 - o0) * (I / 64) * 2);
-        prefetch_l2(blob + a.off[8] + static_cast<size_t>(o0) * (I / 64) * 2, static_cast<size_t>(o1 - o0) * (I / 64) * 2);
-      }
-    } else if (warp == 2 && lane < 2) {
-      // gate/up slice [r0, r1) of the flattened (slot, row) list: at most a few slots
-      for (int j = r0 / I; j <= (r1 - 1) / I && j < k; ++j) {
-        const int i0 = max(r0 - j * I, 0), i1 = min(r1 - j * I, I);
-        const uint8_t* blob = static_cast<const uint8_t*>(W.blobs[sel_idx[j]]);
-        const int m = lane;   // 0 gate, 1 up
-        prefetch_l2(blob + a.off[3 * m] + static_cast<size_t>(i0) * (H / 2), static_cast<size_t>(i1 - i0) * (H / 2));
-        prefetch_l2(blob + a.off[3 * m + 1] + static_cast<size_t>(i0) * (H / 64) * 2, static_cast<size_t>(i1 - i0) * (H / 64) * 2);
-        prefetch_l2(blob + a.off[3 * m + 2] + static_cast<size_t>(i0) * (H / 64) * 2, static_cast<size_t>(i1 - i0) * (H / 64) * 2);
-      }
+      release(q);
     }
 
-    // register copy of x in the nibble-paired layout for this lane's chunks
+    // ----------------------------------------- register x for gate/up rows
     uint32_t xp[DF_CPL][16];
     float2 xst[DF_CPL];
 #pragma unroll
@@ -385,7 +565,8 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
             const float2 f = unpack_half2(p[t]);
             off += f.x + f.y;
           }
-          const float2 f0 = unpack_half2(p[0]), f1 = unpack_half2(p[1]), f2 = unpack_half2(p[2]), f3 = unpack_half2(p[3]);
+          const float2 f0 = unpack_half2(p[0]), f1 = unpack_half2(p[1]), f2 = unpack_half2(p[2]),
+                       f3 = unpack_half2(p[3]);
           sum += (f0.x + f0.y + f2.x + f2.y) + 16.f * (f1.x + f1.y + f3.x + f3.y);
         }
       } else {
@@ -395,31 +576,95 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
       xst[j] = make_float2(1024.f * off, sum);
     }
 
-    // ---------------------------------------------- shared-expert gate/up share
-    for (int i = s0 + warp; i < s1; i += DF_WARPS) {
-      const float v = df_gateup_row<DF_CPL>(reinterpret_cast<const uint8_t*>(W.sq[0]), W.ss[0], W.sb[0],
-                                    reinterpret_cast<const uint8_t*>(W.sq[1]), W.ss[1], W.sb[1], i, H, nch, xp, xst);
-      if (lane == 0) a.act[kI + i] = __float2half_rn(v);
+    // -------------------------------------------------- routing (cluster)
+    df_mbar_wait(lg_bar, l & 1, true);
+    if (warp == 0) {
+      unsigned taken = 0u;
+      float sv[8];
+      int si[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        sv[j] = 0.f;
+        si[j] = 0;
+        if (j < k) {
+          float bv = -INFINITY;
+          int bi = 0x7fffffff;
+          for (int t = 0, e = lane; e < E; ++t, e += 32) {
+            if (taken & (1u << t)) continue;
+            const float v = lg_all[e];
+            if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; }
+          }
+          for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+          }
+          if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+          sv[j] = bv;
+          si[j] = bi;
+        }
+      }
+      if (lane == 0) {
+        float z[8], den = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          z[j] = j < k ? expf(sv[j] - sv[0]) : 0.f;
+          den += z[j];
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j < k) {
+            sl_sel[j] = si[j];
+            selg[j] = z[j] / den;
+            if (s.c == 0 && a.idx_trace) a.idx_trace[static_cast<size_t>(l) * k + j] = si[j];
+            if (s.c == 0 && a.gates_trace) a.gates_trace[static_cast<size_t>(l) * k + j] = z[j] / den;
+          }
+        }
+        df_mbar_arrive(route_bar);      // hand the routing to the loader
+      }
+    }
+    df_named_sync();                    // sl_sel visible to every compute warp
+
+    // ---------------------------------------------------- SG and RG jobs
+    for (int q = s.nR + warp; q < s.nR + s.nSG + s.nRG; q += DF_CW) {
+      const DfJob J = df_job(s, q);
+      const DfJobCopies C = df_job_copies(s, J, a, W, sl_sel);
+      wait_full(q);
+      const unsigned char* slp = ring + slot_of(q) * DF_SLOT;
+      for (int r = 0; r < J.n; ++r) {
+        const uint8_t* gqr = slp + static_cast<size_t>(r) * (H / 2);
+        const uint8_t* uqr = slp + C.qbytes + static_cast<size_t>(r) * (H / 2);
+        const uint16_t* Sg = reinterpret_cast<const uint16_t*>(slp + DF_SLOT_Q + C.sk[0]) + r * (H / 64);
+        const uint16_t* Bg = reinterpret_cast<const uint16_t*>(slp + DF_SLOT_Q + C.sk[1]) + r * (H / 64);
+        const uint16_t* Su = reinterpret_cast<const uint16_t*>(slp + DF_SLOT_Q + C.sk[2]) + r * (H / 64);
+        const uint16_t* Bu = reinterpret_cast<const uint16_t*>(slp + DF_SLOT_Q + C.sk[3]) + r * (H / 64);
+        float ga = 0.f, ua = 0.f;
+#pragma unroll
+        for (int j = 0; j < DF_CPL; ++j) {
+          const int cc = lane + 32 * j;
+          if (cc < nch) {
+            const uint4 q4g = *reinterpret_cast<const uint4*>(gqr + 16 * cc);
+            const uint4 q4u = *reinterpret_cast<const uint4*>(uqr + 16 * cc);
+            const float dg = dot_chunk4(q4g, xp[j]);
+            const float du = dot_chunk4(q4u, xp[j]);
+            ga += bf16_to_f32(Sg[cc >> 1]) * (dg - xst[j].x) + bf16_to_f32(Bg[cc >> 1]) * xst[j].y;
+            ua += bf16_to_f32(Su[cc >> 1]) * (du - xst[j].x) + bf16_to_f32(Bu[cc >> 1]) * xst[j].y;
+          }
+        }
+        ga = warp_sum(ga);
+        ua = warp_sum(ua);
+        if (lane == 0) {
+          const int dst = J.kind == JOB_SG ? kI + J.r0 + r : J.slot * I + J.r0 + r;
+          a.act[dst] = __float2half_rn(gelu_tanh(ga) * ua);
+        }
+      }
+      release(q);
     }
 
-    // ------------------------------------------------- routed gate/up share
-    for (int rr2 = r0 + warp; rr2 < r1; rr2 += DF_WARPS) {
-      const int j = rr2 / I, i = rr2 - j * I;
-      const uint8_t* blob = static_cast<const uint8_t*>(W.blobs[sel_idx[j]]);
-      const float v = df_gateup_row<DF_CPL>(blob + a.off[0], reinterpret_cast<const uint16_t*>(blob + a.off[1]),
-                                    reinterpret_cast<const uint16_t*>(blob + a.off[2]), blob + a.off[3],
-                                    reinterpret_cast<const uint16_t*>(blob + a.off[4]),
-                                    reinterpret_cast<const uint16_t*>(blob + a.off[5]), i, H, nch, xp, xst);
-      if (lane == 0) a.act[rr2] = __float2half_rn(v);
-    }
-
-    bar_target += nclusters;
-    df_grid_sync(cl, a.counter, bar_target);
+    grid_sync();
 
     // ------------------------------------------------------------- phase C
-    if (l + 1 < a.L) prefetch_independent(l + 1);
-    // stage all activations (written by every CTA) in the nibble-paired layout
-    for (int w = threadIdx.x; w < nact / 8; w += DF_THREADS) {
+    for (int w = threadIdx.x; w < nact / 8; w += DF_CW * 32) {
       const uint4 u = ldcg_v4(a.act + 8 * w);
       float v[8];
       const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
@@ -434,71 +679,73 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
       actP[w] = make_uint4(p[0], p[1], p[2], p[3]);
       float off = 0.f;
 #pragma unroll
-      for (int t = 0; t < 4; ++t) { const float2 f = unpack_half2(p[t]); off += f.x + f.y; }
+      for (int t = 0; t < 4; ++t) {
+        const float2 f = unpack_half2(p[t]);
+        off += f.x + f.y;
+      }
       const float2 f0 = unpack_half2(p[0]), f1 = unpack_half2(p[1]), f2 = unpack_half2(p[2]), f3 = unpack_half2(p[3]);
       actS[w] = make_float2(1024.f * off, (f0.x + f0.y + f2.x + f2.y) + 16.f * (f1.x + f1.y + f3.x + f3.y));
     }
-    __syncthreads();
-    // units: (row o, piece u): u < k routed slot u (K = I); u >= k shared piece u-k
-    const int nrow = o1 - o0;
-    for (int un = warp; un < nrow * upr; un += DF_WARPS) {
-      const int ro = un / upr, u = un - ro * upr, o = o0 + ro;
-      const uint8_t* q;
-      const uint16_t *sp, *bp;
-      int wbase, nw;                   // first act word, words in this piece
-      if (u < k) {
-        const uint8_t* blob = static_cast<const uint8_t*>(W.blobs[sel_idx[u]]);
-        q = blob + a.off[6] + static_cast<size_t>(o) * (I / 2);
-        sp = reinterpret_cast<const uint16_t*>(blob + a.off[7]) + static_cast<size_t>(o) * (I / 64);
-        bp = reinterpret_cast<const uint16_t*>(blob + a.off[8]) + static_cast<size_t>(o) * (I / 64);
-        wbase = u * (I / 8);
-        nw = I / 8;
-      } else {
-        const int pc = u - k;
-        const int c0 = pc * I, c1 = min(Is, c0 + I);
-        q = reinterpret_cast<const uint8_t*>(W.sq[2]) + static_cast<size_t>(o) * (Is / 2) + c0 / 2;
-        sp = W.ss[2] + static_cast<size_t>(o) * (Is / 64) + c0 / 64;
-        bp = W.sb[2] + static_cast<size_t>(o) * (Is / 64) + c0 / 64;
-        wbase = (kI + c0) / 8;
-        nw = (c1 - c0) / 8;
+    df_named_sync();
+    const int qD0 = s.nR + s.nSG + s.nRG;
+    for (int q = qD0 + warp; q < njobs; q += DF_CW) {
+      const DfJob J = df_job(s, q);
+      const DfJobCopies C = df_job_copies(s, J, a, W, sl_sel);
+      wait_full(q);
+      const unsigned char* slp = ring + slot_of(q) * DF_SLOT;
+      const int K = J.kind == JOB_D ? I : Is;
+      const int wbase = J.kind == JOB_D ? J.slot * (I / 8) : kI / 8;
+      const int unit = J.kind == JOB_D ? J.slot : k;
+      const int nw = K / 8;
+      for (int r = 0; r < J.n; ++r) {
+        const uint8_t* qrow = slp + static_cast<size_t>(r) * (K / 2);
+        const uint16_t* S = reinterpret_cast<const uint16_t*>(slp + DF_SLOT_Q + C.sk[0]) + r * (K / 64);
+        const uint16_t* B = reinterpret_cast<const uint16_t*>(slp + DF_SLOT_Q + C.sk[1]) + r * (K / 64);
+        float acc = 0.f;
+        for (int w = lane; w < nw; w += 32) {
+          const uint32_t qw = *reinterpret_cast<const uint32_t*>(qrow + 4 * w);
+          const uint4 pp = actP[wbase + w];
+          const uint32_t p[4] = {pp.x, pp.y, pp.z, pp.w};
+          float a0 = 0.f, a1 = 0.f;
+          dot_word4(qw, p, a0, a1);
+          const float2 st = actS[wbase + w];
+          acc += bf16_to_f32(S[w >> 3]) * ((a0 + a1) - st.x) + bf16_to_f32(B[w >> 3]) * st.y;
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) part[(J.r0 + r - s.o0) * 9 + unit] = acc;
       }
-      float acc = 0.f;
-      for (int w = lane; w < nw; w += 32) {
-        const uint32_t qw = ldg_nc_u32(q + 4 * w);
-        const float sc = bf16_to_f32(ldg_u16(sp + (w >> 3)));
-        const float bi = bf16_to_f32(ldg_u16(bp + (w >> 3)));
-        const uint4 pp = actP[wbase + w];
-        const uint32_t p[4] = {pp.x, pp.y, pp.z, pp.w};
-        float a0 = 0.f, a1 = 0.f;
-        dot_word4(qw, p, a0, a1);
-        const float2 st = actS[wbase + w];
-        acc += sc * ((a0 + a1) - st.x) + bi * st.y;
-      }
-      acc = warp_sum(acc);
-      if (lane == 0) part[ro * DF_MAX_UNITS + u] = acc;
+      release(q);
     }
-    __syncthreads();
-    for (int ro = threadIdx.x; ro < nrow; ro += DF_THREADS) {
+    df_named_sync();
+    for (int ro = threadIdx.x; ro < s.o1 - s.o0; ro += DF_CW * 32) {
       float y = 0.f;
-      for (int j = 0; j < k; ++j) y = fmaf(sel_g[j], part[ro * DF_MAX_UNITS + j], y);
-      float ys = 0.f;
-      for (int pc = 0; pc < nsub; ++pc) ys += part[ro * DF_MAX_UNITS + k + pc];
-      y += ys;
-      const int o = o0 + ro;
+      for (int j = 0; j < k; ++j) y = fmaf(selg[j], part[ro * 9 + j], y);
+      y += part[ro * 9 + k];
+      const int o = s.o0 + ro;
       a.h[o] = __ldcg(a.h + o) + y;
       if (a.y_trace) a.y_trace[static_cast<size_t>(l) * H + o] = f32_to_bf16(y);
     }
-    if (l + 1 < a.L) {
-      bar_target += nclusters;
-      df_grid_sync(cl, a.counter, bar_target);
-    }
+    g += njobs;
+    if (l + 1 < a.L) grid_sync();
   }
 }
 
-size_t decode_fused_smem(int H, int nact) {
-  (void)H; (void)nact;
-  return (DF_MAX_H + 32 + 128 + 1024 + 24) * 4 + DF_MAX_ROWS * DF_MAX_UNITS * 4 +
-         static_cast<size_t>(DF_MAX_ACT / 8) * (16 + 8) + 64;
+size_t decode_fused_smem() {
+  return static_cast<size_t>(DF_NS) * DF_SLOT + DF_MAX_H * 4 + static_cast<size_t>(DF_MAX_ACT / 8) * (16 + 8) +
+         DF_MAX_ROWS * 9 * 4 + DF_MAX_E * 4 + 32 * 4 + 16 * 4 + 8 * 4 + (2 * DF_NS + 8) * 8 + 128;
+}
+
+// Rows per job so that one job fits a ring slot (0 if even one row does not).
+inline int df_rows_fit(int runs, int qbytes_per_row, int windows, int sbytes_per_row) {
+  int n = 0;
+  while (true) {
+    const int m = n + 1;
+    if (runs * m * qbytes_per_row > DF_SLOT_Q) break;
+    if (windows * (m * sbytes_per_row + 32) > DF_SLOT_S) break;
+    n = m;
+    if (n >= 64) break;
+  }
+  return n;
 }
 
 }  // namespace moe
