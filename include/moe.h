@@ -223,6 +223,15 @@ MOE_API size_t moe_decode_workspace_size(int T, int H, int I, int Is, int E, int
  * prefetched into L2 while the layer waits for its routing (their bytes are
  * read again, from L2, only if they are chosen). */
 MOE_API int moe_set_decode_fused(int enable, int spec_experts);
+/* Phase timestamps of the fused batch-1 kernel (a tracing aid): when
+ * `stamps` (device, [L][G][8] uint64, G = moe_decode_grid()) is non-NULL,
+ * thread 0 of every CTA writes %globaltimer (ns) at the phase boundaries of
+ * each layer: 0 layer start, 1 router done, 2 routing known, 3 gate/up done,
+ * 4 after the first grid barrier, 5 down/combine done, 6 after the second
+ * grid barrier.  NULL turns it off (default). */
+MOE_API int moe_set_decode_profile(unsigned long long* stamps);
+/* CTAs of the fused batch-1 kernel on the current device (0: not available). */
+MOE_API int moe_decode_grid(void);
 /* Number of kernels one moe_decode_forward(T, L) call launches. */
 MOE_API int moe_decode_launches(int T, int L);
 MOE_API int moe_decode_forward(float* h, int T, int H, int I, int Is, int E, int k, int L,

@@ -107,6 +107,14 @@ def moe_set_decode_fused(enable: bool, spec_experts: int = 2):
     check(lib().moe_set_decode_fused(1 if enable else 0, spec_experts))
 
 
+def moe_set_decode_profile(stamps=None):
+    check(lib().moe_set_decode_profile(ptr(stamps)))
+
+
+def moe_decode_grid() -> int:
+    return lib().moe_decode_grid()
+
+
 def moe_decode_launches(T: int, L: int) -> int:
     return lib().moe_decode_launches(T, L)
 

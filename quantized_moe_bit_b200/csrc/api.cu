@@ -14,6 +14,7 @@ static thread_local char g_err[512] = "";
 static int g_gemv_max_rows = 2;
 static int g_decode_fused = 1;
 static int g_decode_spec = 2;
+static unsigned long long* g_decode_stamps = nullptr;
 
 int fail(int code, const char* fmt, ...) {
   va_list ap;
@@ -357,6 +358,15 @@ static bool fused_ok(int T, int H, int I, int Is, int E, int k, int bias_per_row
   if (H % 64 || H > DF_MAX_H || I % 64 || Is % 64 || E % 8 || E > DF_MAX_E || k > 8) return false;
   if (k * I + Is > DF_MAX_ACT) return false;
   if (G <= 0 || G % DF_CLUSTER || (H + G - 1) / G > DF_MAX_ROWS) return false;
+  {  // jobs per layer per CTA (upper bound) must fit the descriptor table
+    const int rg = df_rows_fit(2, H / 2, 4, 2 * (H / 64));
+    const int dn = df_rows_fit(1, I / 2, 2, 2 * (I / 64)), dsn = df_rows_fit(1, Is / 2, 2, 2 * (Is / 64));
+    if (rg < 1 || dn < 1 || dsn < 1) return false;
+    const int rows = (H + G - 1) / G;
+    const int jobs = (E / DF_CLUSTER + 1) / 2 + ((Is + G - 1) / G + rg - 1) / rg + 1 +
+                     ((k * I + G - 1) / G + rg - 1) / rg + 2 + k * ((rows + dn - 1) / dn) + (rows + dsn - 1) / dsn;
+    if (jobs > DF_MAX_JOBS) return false;
+  }
   if (df_rows_fit(1, H, 2, 2 * (H / 64)) < 2) return false;                       // router jobs: 2 rows
   if (df_rows_fit(2, H / 2, 4, 2 * (H / 64)) < 1) return false;                   // gate/up row pairs
   if (df_rows_fit(1, I / 2, 2, 2 * (I / 64)) < 1 || df_rows_fit(1, Is / 2, 2, 2 * (Is / 64)) < 1) return false;
@@ -412,6 +422,7 @@ static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, con
     args.idx_trace = idx_trace ? idx_trace + l0 * Tk : nullptr;
     args.gates_trace = gates_trace ? gates_trace + l0 * Tk : nullptr;
     args.spec = g_decode_spec;
+    args.stamps = g_decode_stamps ? g_decode_stamps + static_cast<size_t>(l0) * G * 8 : nullptr;
     args.rg_rows = df_rows_fit(2, H / 2, 4, 2 * (H / 64));
     args.d_rows = df_rows_fit(1, I / 2, 2, 2 * (I / 64));
     args.ds_rows = df_rows_fit(1, Is / 2, 2, 2 * (Is / 64));
@@ -441,6 +452,13 @@ static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, con
   }
   return MOE_OK;
 }
+
+int moe_set_decode_profile(unsigned long long* stamps) {
+  g_decode_stamps = stamps;
+  return MOE_OK;
+}
+
+int moe_decode_grid(void) { return fused_grid(); }
 
 int moe_set_decode_fused(int enable, int spec_experts) {
   if (spec_experts < 0 || spec_experts > 8) return fail(MOE_ERR_INVALID_ARG, "spec_experts must be in [0, 8]");

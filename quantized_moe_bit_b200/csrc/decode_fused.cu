@@ -51,6 +51,7 @@ constexpr int DF_SLOT_Q = 8192;                 // weight bytes per slot
 constexpr int DF_SLOT_S = 1024;                 // scale/bias window bytes per slot
 constexpr int DF_SLOT = DF_SLOT_Q + DF_SLOT_S;
 constexpr int DF_MAX_E = 256;
+constexpr int DF_MAX_JOBS = 80;                 // jobs per layer per CTA
 
 struct DfLayer {
   const uint32_t* rq; const uint16_t* rs; const uint16_t* rb;   // router [E, H], 8-bit
@@ -68,6 +69,7 @@ struct DfArgs {
   uint16_t* x_trace; uint16_t* y_trace; int32_t* idx_trace; float* gates_trace;
   int spec;                         // experts speculatively prefetched per layer
   int rg_rows, d_rows, ds_rows;     // row pairs per SG/RG job, rows per D / DS job
+  unsigned long long* stamps;       // optional phase timestamps [L][G][8] (ns), or null
   DfLayer layer[DF_MAX_LAYERS];
 };
 
@@ -174,6 +176,12 @@ __device__ __forceinline__ void df_named_sync() {   // the compute warps of this
   asm volatile("bar.sync 1, %0;" ::"n"(DF_CW * 32) : "memory");
 }
 
+// phase timestamps (when requested): layer l, CTA c, phase p
+__device__ __forceinline__ void df_stamp(const DfArgs& a, int l, int p) {
+  if (a.stamps != nullptr && threadIdx.x == 0)
+    a.stamps[(static_cast<size_t>(l) * gridDim.x + blockIdx.x) * 8 + p] = df_clock();
+}
+
 // ---------------------------------------------------------------- job list
 enum : int { JOB_R = 0, JOB_SG = 1, JOB_RG = 2, JOB_D = 3, JOB_DS = 4 };
 
@@ -259,6 +267,7 @@ struct DfJobCopies {
   uint32_t qbytes;
   uint32_t sk[4];
   uint32_t bytes;
+  int kind, slot, r0, rows;       // the job itself
 };
 
 __device__ inline DfJobCopies df_job_copies(const DfShape& s, const DfJob& J, const DfArgs& a, const DfLayer& W,
@@ -315,6 +324,7 @@ __device__ inline DfJobCopies df_job_copies(const DfShape& s, const DfJob& J, co
     total += bytes;
   }
   C.bytes = total;
+  C.kind = J.kind; C.slot = J.slot; C.r0 = J.r0; C.rows = J.n;
   return C;
 }
 
@@ -339,14 +349,21 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
   s.nD = s.k * ceil_div(s.o1 - s.o0, s.dn);
   s.nDS = ceil_div(s.o1 - s.o0, s.dsn);
   const int njobs = s.nR + s.nSG + s.nRG + s.nD + s.nDS;
+  const int nhead = s.nR + s.nSG;            // jobs that do not depend on the routing
   const int H = s.H, I = s.I, Is = s.Is, E = s.E, k = s.k;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned nclusters = s.G / DF_CLUSTER;
+  const int nch = H / 32, nch16 = H / 16;
 
   // shared memory
   unsigned char* ring = smem;                                          // [NS][DF_SLOT]
-  float* xs = reinterpret_cast<float*>(ring + DF_NS * DF_SLOT);        // [H] layer input (bf16 values)
-  uint4* actP = reinterpret_cast<uint4*>(xs + DF_MAX_H);               // [nact/8] paired activations
+  DfJobCopies* tab = reinterpret_cast<DfJobCopies*>(ring + DF_NS * DF_SLOT);   // [2][MAX_JOBS]
+  float* xs = reinterpret_cast<float*>(tab + 2 * DF_MAX_JOBS);         // [H] layer input (bf16 values)
+  uint4* xP4 = reinterpret_cast<uint4*>(xs + DF_MAX_H);                // [4][nch] nibble-paired x
+  float2* xS4 = reinterpret_cast<float2*>(xP4 + DF_MAX_H / 8);         // [nch] (off, sum)
+  uint2* xP8 = reinterpret_cast<uint2*>(xS4 + DF_MAX_H / 32);          // [4][nch16] byte-paired x
+  float* xS8 = reinterpret_cast<float*>(xP8 + DF_MAX_H / 4);           // [nch16] sum
+  uint4* actP = reinterpret_cast<uint4*>(xS8 + DF_MAX_H / 16);         // [nact/8] paired activations
   float2* actS = reinterpret_cast<float2*>(actP + DF_MAX_ACT / 8);     // [nact/8] (off, sum) per word
   float* part = reinterpret_cast<float*>(actS + DF_MAX_ACT / 8);       // [MAX_ROWS][9]
   float* lg_all = part + DF_MAX_ROWS * 9;                              // [E]
@@ -379,10 +396,28 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
   if (warp == DF_CW) {
     // ================================================================ loader
     uint32_t g = 0;   // job sequence over the launch
+    auto issue = [&](const DfJobCopies& C) {
+      const int slot = g % DF_NS;
+      if (g >= DF_NS) df_mbar_wait(empty_bar(slot), ((g / DF_NS) + 1) & 1);
+      if (lane == 0) df_mbar_expect_tx(full_bar(slot), C.bytes);
+      __syncwarp();
+      if (lane < C.n)
+        df_bulk_g2s(smem_addr(ring + slot * DF_SLOT + C.dst[lane]), C.src[lane], C.len[lane], full_bar(slot));
+      __syncwarp();
+      ++g;
+    };
     for (int l = 0; l < a.L; ++l) {
       const DfLayer& W = a.layer[l];
+      DfJobCopies* T = tab + (l & 1) * DF_MAX_JOBS;
+      const int* sl = sel + 8 * (l & 1);
+      // descriptors of the routing-independent jobs, one job per lane
+      for (int q = lane; q < njobs; q += 32) {
+        const DfJob J = df_job(s, q);
+        if (J.kind == JOB_R || J.kind == JOB_SG || J.kind == JOB_DS) T[q] = df_job_copies(s, J, a, W, sl);
+      }
+      __syncwarp();
       if (lane == 0) {
-        // routing-independent rows of this layer (layer 0) and of the next one
+        // routing-independent rows of this layer (layer 0) and of the next one into L2
         for (int ll = (l == 0 ? 0 : l + 1); ll <= l + 1 && ll < a.L; ++ll) {
           const DfLayer& V = a.layer[ll];
           prefetch_l2(reinterpret_cast<const uint8_t*>(V.rq) + static_cast<size_t>(s.rank * s.epc) * H,
@@ -420,31 +455,23 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
           prefetch_slice(V.blobs[my_id], bb, s.c, s.G);
         }
       }
-      const int* sl = sel + 8 * (l & 1);
-      for (int q = 0; q < njobs; ++q, ++g) {
-        if (q == s.nR + s.nSG) {
-          // routed jobs need this layer's routing; then all routed rows into L2 at once
-          df_mbar_wait(route_bar, l & 1);
-          for (int qq = q + lane; qq < njobs; qq += 32) {
-            const DfJobCopies C2 = df_job_copies(s, df_job(s, qq), a, W, sl);
-            for (int i = 0; i < C2.n; ++i) prefetch_l2(C2.src[i], C2.len[i]);
-          }
+      for (int q = 0; q < nhead; ++q) issue(T[q]);
+      // the routed jobs need this layer's routing
+      df_mbar_wait(route_bar, l & 1);
+      for (int q = nhead + lane; q < njobs; q += 32) {
+        const DfJob J = df_job(s, q);
+        if (J.kind == JOB_RG || J.kind == JOB_D) {
+          T[q] = df_job_copies(s, J, a, W, sl);
+          for (int i = 0; i < T[q].n; ++i) prefetch_l2(T[q].src[i], T[q].len[i]);   // all routed rows into L2
         }
-        const int slot = g % DF_NS;
-        if (g >= DF_NS) df_mbar_wait(empty_bar(slot), ((g / DF_NS) + 1) & 1);
-        const DfJobCopies C = df_job_copies(s, df_job(s, q), a, W, sl);
-        if (lane == 0) df_mbar_expect_tx(full_bar(slot), C.bytes);
-        __syncwarp();
-        if (lane < C.n)
-          df_bulk_g2s(smem_addr(ring + slot * DF_SLOT + C.dst[lane]), C.src[lane], C.len[lane], full_bar(slot));
-        __syncwarp();
       }
+      __syncwarp();
+      for (int q = nhead; q < njobs; ++q) issue(T[q]);
     }
     return;
   }
 
   // ================================================================== compute
-  const int nch = H / 32;
   uint32_t g = 0;            // job sequence (same numbering as the loader)
   unsigned bar_target = 0;
   unsigned gen = 0;          // grid barriers passed
@@ -481,7 +508,9 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
 
   for (int l = 0; l < a.L; ++l) {
     const DfLayer& W = a.layer[l];
+    const DfJobCopies* T = tab + (l & 1) * DF_MAX_JOBS;
     int* sl_sel = sel + 8 * (l & 1);
+    df_stamp(a, l, 0);
     // ------------------------------------------------------ A0: rms norm
     float ss = 0.f;
     for (int i = threadIdx.x * 4; i < H; i += DF_CW * 32 * 4) {
@@ -507,35 +536,70 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
       if (s.c == 0 && a.x_trace) a.x_trace[static_cast<size_t>(l) * H + i] = b;
     }
     df_named_sync();
+    // paired copies of x: nibble-paired per 8-element word (4-bit rows) and
+    // byte-paired per 4-element word (8-bit router), stored word-major
+    for (int w = threadIdx.x; w < H / 8; w += DF_CW * 32) {
+      float v[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) v[t] = xs[8 * w + t];
+      uint32_t p[4];
+      pair_word4(v, p);
+      xP4[(w & 3) * nch + (w >> 2)] = make_uint4(p[0], p[1], p[2], p[3]);
+    }
+    for (int w = threadIdx.x; w < H / 4; w += DF_CW * 32) {
+      const float* v = xs + 4 * w;
+      xP8[(w & 3) * nch16 + (w >> 2)] = make_uint2(pack_half2(v[0], v[2]), pack_half2(v[1], v[3]));
+    }
+    df_named_sync();
+    for (int cc = threadIdx.x; cc < nch; cc += DF_CW * 32) {
+      float off = 0.f, sum = 0.f;
+      for (int m = 0; m < 4; ++m) {
+        const uint4 u = xP4[m * nch + cc];
+        const float2 f0 = unpack_half2(u.x), f1 = unpack_half2(u.y), f2 = unpack_half2(u.z), f3 = unpack_half2(u.w);
+        off += (f0.x + f0.y) + (f1.x + f1.y) + (f2.x + f2.y) + (f3.x + f3.y);
+        sum += (f0.x + f0.y + f2.x + f2.y) + 16.f * (f1.x + f1.y + f3.x + f3.y);
+      }
+      xS4[cc] = make_float2(1024.f * off, sum);
+    }
+    for (int cc = threadIdx.x; cc < nch16; cc += DF_CW * 32) {
+      float sum = 0.f;
+      for (int m = 0; m < 4; ++m) {
+        const uint2 u = xP8[m * nch16 + cc];
+        const float2 f0 = unpack_half2(u.x), f1 = unpack_half2(u.y);
+        sum += (f0.x + f0.y) + (f1.x + f1.y);
+      }
+      xS8[cc] = sum;
+    }
+    df_named_sync();
 
     // ------------------------------------------------------------- R jobs
     for (int q = warp; q < s.nR; q += DF_CW) {
-      const DfJob J = df_job(s, q);
-      const DfJobCopies C = df_job_copies(s, J, a, W, sl_sel);
+      const DfJob J = df_job(s, q);      // (the descriptor is read only after the data landed)
+      float bias_r[2] = {0.f, 0.f};
+      for (int r = 0; r < J.n; ++r) bias_r[r] = W.bias ? W.bias[J.r0 + r] : 0.f;
       wait_full(q);
+      const DfJobCopies& C = T[q];
       const unsigned char* slp = ring + slot_of(q) * DF_SLOT;
-      for (int r = 0; r < J.n; ++r) {
-        const int e = J.r0 + r;
+      for (int r = 0; r < C.rows; ++r) {
+        const int e = C.r0 + r;
         const uint8_t* qrow = slp + static_cast<size_t>(r) * H;
         const uint16_t* S = reinterpret_cast<const uint16_t*>(slp + DF_SLOT_Q + C.sk[0]) + r * (H / 64);
         const uint16_t* B = reinterpret_cast<const uint16_t*>(slp + DF_SLOT_Q + C.sk[1]) + r * (H / 64);
         float acc = 0.f;
-        for (int cc = lane; cc < H / 16; cc += 32) {
+        for (int cc = lane; cc < nch16; cc += 32) {
           const uint4 q4 = *reinterpret_cast<const uint4*>(qrow + 16 * cc);
-          const float sc = bf16_to_f32(S[cc >> 2]), bi = bf16_to_f32(B[cc >> 2]);
-          const float* xv = xs + 16 * cc;
           const uint32_t w[4] = {q4.x, q4.y, q4.z, q4.w};
-          float a0 = 0.f, a1 = 0.f, off = 0.f;
+          float a0 = 0.f, a1 = 0.f;
 #pragma unroll
           for (int m = 0; m < 4; ++m) {
-            const uint32_t p[2] = {pack_half2(xv[4 * m], xv[4 * m + 2]), pack_half2(xv[4 * m + 1], xv[4 * m + 3])};
+            const uint2 pp = xP8[m * nch16 + cc];
+            const uint32_t p[2] = {pp.x, pp.y};
             dot_word8(w[m], p, a0, a1);
-            const float2 f0 = unpack_half2(p[0]), f1 = unpack_half2(p[1]);
-            off += (f0.x + f0.y) + (f1.x + f1.y);
           }
-          acc += sc * ((a0 + a1) - 1024.f * off) + bi * off;
+          const float sm = xS8[cc];
+          acc += bf16_to_f32(S[cc >> 2]) * ((a0 + a1) - 1024.f * sm) + bf16_to_f32(B[cc >> 2]) * sm;
         }
-        acc = warp_sum(acc) + (W.bias ? W.bias[e] : 0.f);
+        acc = warp_sum(acc) + (r == 0 ? bias_r[0] : bias_r[1]);
         if (lane < DF_CLUSTER) {          // broadcast the logit to every CTA of the cluster
           df_st_remote_f32(smem_addr(lg_all + e), lane, acc);
           df_mbar_arrive_remote(lg_bar, lane);
@@ -543,6 +607,7 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
       }
       release(q);
     }
+    df_stamp(a, l, 1);
 
     // ----------------------------------------- register x for gate/up rows
     uint32_t xp[DF_CPL][16];
@@ -550,30 +615,18 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
 #pragma unroll
     for (int j = 0; j < DF_CPL; ++j) {
       const int cc = lane + 32 * j;
-      float off = 0.f, sum = 0.f;
       if (cc < nch) {
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-          float v[8];
-#pragma unroll
-          for (int t = 0; t < 8; ++t) v[t] = xs[32 * cc + 8 * m + t];
-          uint32_t p[4];
-          pair_word4(v, p);
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            xp[j][4 * m + t] = p[t];
-            const float2 f = unpack_half2(p[t]);
-            off += f.x + f.y;
-          }
-          const float2 f0 = unpack_half2(p[0]), f1 = unpack_half2(p[1]), f2 = unpack_half2(p[2]),
-                       f3 = unpack_half2(p[3]);
-          sum += (f0.x + f0.y + f2.x + f2.y) + 16.f * (f1.x + f1.y + f3.x + f3.y);
+          const uint4 u = xP4[m * nch + cc];
+          xp[j][4 * m + 0] = u.x; xp[j][4 * m + 1] = u.y; xp[j][4 * m + 2] = u.z; xp[j][4 * m + 3] = u.w;
         }
+        xst[j] = xS4[cc];
       } else {
 #pragma unroll
         for (int t = 0; t < 16; ++t) xp[j][t] = 0u;
+        xst[j] = make_float2(0.f, 0.f);
       }
-      xst[j] = make_float2(1024.f * off, sum);
     }
 
     // -------------------------------------------------- routing (cluster)
@@ -624,14 +677,14 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
       }
     }
     df_named_sync();                    // sl_sel visible to every compute warp
+    df_stamp(a, l, 2);
 
     // ---------------------------------------------------- SG and RG jobs
     for (int q = s.nR + warp; q < s.nR + s.nSG + s.nRG; q += DF_CW) {
-      const DfJob J = df_job(s, q);
-      const DfJobCopies C = df_job_copies(s, J, a, W, sl_sel);
-      wait_full(q);
+      wait_full(q);                     // (also orders the loader's descriptor writes)
+      const DfJobCopies& C = T[q];
       const unsigned char* slp = ring + slot_of(q) * DF_SLOT;
-      for (int r = 0; r < J.n; ++r) {
+      for (int r = 0; r < C.rows; ++r) {
         const uint8_t* gqr = slp + static_cast<size_t>(r) * (H / 2);
         const uint8_t* uqr = slp + C.qbytes + static_cast<size_t>(r) * (H / 2);
         const uint16_t* Sg = reinterpret_cast<const uint16_t*>(slp + DF_SLOT_Q + C.sk[0]) + r * (H / 64);
@@ -654,14 +707,16 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
         ga = warp_sum(ga);
         ua = warp_sum(ua);
         if (lane == 0) {
-          const int dst = J.kind == JOB_SG ? kI + J.r0 + r : J.slot * I + J.r0 + r;
+          const int dst = C.kind == JOB_SG ? kI + C.r0 + r : C.slot * I + C.r0 + r;
           a.act[dst] = __float2half_rn(gelu_tanh(ga) * ua);
         }
       }
       release(q);
     }
 
+    df_stamp(a, l, 3);
     grid_sync();
+    df_stamp(a, l, 4);
 
     // ------------------------------------------------------------- phase C
     for (int w = threadIdx.x; w < nact / 8; w += DF_CW * 32) {
@@ -687,17 +742,15 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
       actS[w] = make_float2(1024.f * off, (f0.x + f0.y + f2.x + f2.y) + 16.f * (f1.x + f1.y + f3.x + f3.y));
     }
     df_named_sync();
-    const int qD0 = s.nR + s.nSG + s.nRG;
-    for (int q = qD0 + warp; q < njobs; q += DF_CW) {
-      const DfJob J = df_job(s, q);
-      const DfJobCopies C = df_job_copies(s, J, a, W, sl_sel);
+    for (int q = nhead + s.nRG + warp; q < njobs; q += DF_CW) {
       wait_full(q);
+      const DfJobCopies& C = T[q];
       const unsigned char* slp = ring + slot_of(q) * DF_SLOT;
-      const int K = J.kind == JOB_D ? I : Is;
-      const int wbase = J.kind == JOB_D ? J.slot * (I / 8) : kI / 8;
-      const int unit = J.kind == JOB_D ? J.slot : k;
+      const int K = C.kind == JOB_D ? I : Is;
+      const int wbase = C.kind == JOB_D ? C.slot * (I / 8) : kI / 8;
+      const int unit = C.kind == JOB_D ? C.slot : k;
       const int nw = K / 8;
-      for (int r = 0; r < J.n; ++r) {
+      for (int r = 0; r < C.rows; ++r) {
         const uint8_t* qrow = slp + static_cast<size_t>(r) * (K / 2);
         const uint16_t* S = reinterpret_cast<const uint16_t*>(slp + DF_SLOT_Q + C.sk[0]) + r * (K / 64);
         const uint16_t* B = reinterpret_cast<const uint16_t*>(slp + DF_SLOT_Q + C.sk[1]) + r * (K / 64);
@@ -712,7 +765,7 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
           acc += bf16_to_f32(S[w >> 3]) * ((a0 + a1) - st.x) + bf16_to_f32(B[w >> 3]) * st.y;
         }
         acc = warp_sum(acc);
-        if (lane == 0) part[(J.r0 + r - s.o0) * 9 + unit] = acc;
+        if (lane == 0) part[(C.r0 + r - s.o0) * 9 + unit] = acc;
       }
       release(q);
     }
@@ -726,13 +779,17 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
       if (a.y_trace) a.y_trace[static_cast<size_t>(l) * H + o] = f32_to_bf16(y);
     }
     g += njobs;
+    df_stamp(a, l, 5);
     if (l + 1 < a.L) grid_sync();
+    df_stamp(a, l, 6);
   }
 }
 
 size_t decode_fused_smem() {
-  return static_cast<size_t>(DF_NS) * DF_SLOT + DF_MAX_H * 4 + static_cast<size_t>(DF_MAX_ACT / 8) * (16 + 8) +
-         DF_MAX_ROWS * 9 * 4 + DF_MAX_E * 4 + 32 * 4 + 16 * 4 + 8 * 4 + (2 * DF_NS + 8) * 8 + 128;
+  return static_cast<size_t>(DF_NS) * DF_SLOT + 2 * DF_MAX_JOBS * sizeof(DfJobCopies) + DF_MAX_H * 4 +
+         DF_MAX_H / 8 * 16 + DF_MAX_H / 32 * 8 + DF_MAX_H / 4 * 8 + DF_MAX_H / 16 * 4 +
+         static_cast<size_t>(DF_MAX_ACT / 8) * (16 + 8) + DF_MAX_ROWS * 9 * 4 + DF_MAX_E * 4 + 32 * 4 + 16 * 4 +
+         8 * 4 + (2 * DF_NS + 8) * 8 + 128;
 }
 
 // Rows per job so that one job fits a ring slot (0 if even one row does not).
