@@ -223,6 +223,10 @@ MOE_API size_t moe_decode_workspace_size(int T, int H, int I, int Is, int E, int
  * prefetched into L2 while the layer waits for its routing (their bytes are
  * read again, from L2, only if they are chosen). */
 MOE_API int moe_set_decode_fused(int enable, int spec_experts);
+/* L2 prefetch policy of the fused batch-1 kernel (bit flags, default 3):
+ * 1 = once a layer's routing is known, prefetch all of its routed rows;
+ * 2 = prefetch the next layer's routing-independent rows ahead of time. */
+MOE_API int moe_set_decode_prefetch(int flags);
 /* Phase timestamps of the fused batch-1 kernel (a tracing aid): when
  * `stamps` (device, [L][G][8] uint64, G = moe_decode_grid()) is non-NULL,
  * thread 0 of every CTA writes %globaltimer (ns) at the phase boundaries of

@@ -56,6 +56,7 @@ SIGNATURES = {
     "moe_decode_launches": (_I, [_I, _I]),
     "moe_set_decode_fused": (_I, [_I, _I]),
     "moe_set_decode_profile": (_I, [_P]),
+    "moe_set_decode_prefetch": (_I, [_I]),
     "moe_decode_grid": (_I, []),
     "moe_decode_forward": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, C.POINTER(moe_qmat), C.POINTER(C.c_void_p), _I,
                                 C.POINTER(C.c_void_p), C.POINTER(moe_qmat), _P, _P, _P, _P, _P, _Z, _P]),

@@ -111,6 +111,10 @@ def moe_set_decode_profile(stamps=None):
     check(lib().moe_set_decode_profile(ptr(stamps)))
 
 
+def moe_set_decode_prefetch(flags: int):
+    check(lib().moe_set_decode_prefetch(flags))
+
+
 def moe_decode_grid() -> int:
     return lib().moe_decode_grid()
 

@@ -14,6 +14,7 @@ static thread_local char g_err[512] = "";
 static int g_gemv_max_rows = 2;
 static int g_decode_fused = 1;
 static int g_decode_spec = 2;
+static int g_decode_prefetch = 3;
 static unsigned long long* g_decode_stamps = nullptr;
 
 int fail(int code, const char* fmt, ...) {
@@ -422,6 +423,7 @@ static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, con
     args.idx_trace = idx_trace ? idx_trace + l0 * Tk : nullptr;
     args.gates_trace = gates_trace ? gates_trace + l0 * Tk : nullptr;
     args.spec = g_decode_spec;
+    args.prefetch = g_decode_prefetch;
     args.stamps = g_decode_stamps ? g_decode_stamps + static_cast<size_t>(l0) * G * 8 : nullptr;
     args.rg_rows = df_rows_fit(2, H / 2, 4, 2 * (H / 64));
     args.d_rows = df_rows_fit(1, I / 2, 2, 2 * (I / 64));
@@ -459,6 +461,12 @@ int moe_set_decode_profile(unsigned long long* stamps) {
 }
 
 int moe_decode_grid(void) { return fused_grid(); }
+
+int moe_set_decode_prefetch(int flags) {
+  if (flags < 0 || flags > 3) return fail(MOE_ERR_INVALID_ARG, "prefetch flags must be in [0, 3]");
+  g_decode_prefetch = flags;
+  return MOE_OK;
+}
 
 int moe_set_decode_fused(int enable, int spec_experts) {
   if (spec_experts < 0 || spec_experts > 8) return fail(MOE_ERR_INVALID_ARG, "spec_experts must be in [0, 8]");

@@ -68,6 +68,7 @@ struct DfArgs {
   unsigned* counter;                // workspace: grid barrier counter (zeroed before launch)
   uint16_t* x_trace; uint16_t* y_trace; int32_t* idx_trace; float* gates_trace;
   int spec;                         // experts speculatively prefetched per layer
+  int prefetch;                     // bit 0: routed rows into L2 once routed; bit 1: independent rows
   int rg_rows, d_rows, ds_rows;     // row pairs per SG/RG job, rows per D / DS job
   unsigned long long* stamps;       // optional phase timestamps [L][G][8] (ns), or null
   DfLayer layer[DF_MAX_LAYERS];
@@ -352,7 +353,6 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
   const int nhead = s.nR + s.nSG;            // jobs that do not depend on the routing
   const int H = s.H, I = s.I, Is = s.Is, E = s.E, k = s.k;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const unsigned nclusters = s.G / DF_CLUSTER;
   const int nch = H / 32, nch16 = H / 16;
 
   // shared memory
@@ -416,7 +416,7 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
         if (J.kind == JOB_R || J.kind == JOB_SG || J.kind == JOB_DS) T[q] = df_job_copies(s, J, a, W, sl);
       }
       __syncwarp();
-      if (lane == 0) {
+      if (lane == 0 && (a.prefetch & 2)) {
         // routing-independent rows of this layer (layer 0) and of the next one into L2
         for (int ll = (l == 0 ? 0 : l + 1); ll <= l + 1 && ll < a.L; ++ll) {
           const DfLayer& V = a.layer[ll];
@@ -462,7 +462,8 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
         const DfJob J = df_job(s, q);
         if (J.kind == JOB_RG || J.kind == JOB_D) {
           T[q] = df_job_copies(s, J, a, W, sl);
-          for (int i = 0; i < T[q].n; ++i) prefetch_l2(T[q].src[i], T[q].len[i]);   // all routed rows into L2
+          if (a.prefetch & 1)
+            for (int i = 0; i < T[q].n; ++i) prefetch_l2(T[q].src[i], T[q].len[i]);   // all routed rows into L2
         }
       }
       __syncwarp();
@@ -475,31 +476,30 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
   uint32_t g = 0;            // job sequence (same numbering as the loader)
   unsigned bar_target = 0;
   unsigned gen = 0;          // grid barriers passed
+  // grid barrier among the compute warps of all CTAs: named barrier, one
+  // atomic per CTA on a counter that grows by G per barrier, named barrier
   auto grid_sync = [&]() {
     df_named_sync();
     if (threadIdx.x == 0) {
       __threadfence();
-      df_mbar_arrive_remote(clA_bar, 0);
-      if (s.rank == 0) {
-        df_mbar_wait(clA_bar, gen & 1, true);
-        bar_target += nclusters;
-        red_release_gpu(a.counter, 1u);
-        const uint64_t t0 = df_clock();
-        while (ld_acquire_gpu(a.counter) < bar_target) {
-          if (df_clock() - t0 > 2000000000ull) { flag_check(CHECK_WAIT); break; }
-        }
-        for (int r = 0; r < DF_CLUSTER; ++r) df_mbar_arrive_remote(clR_bar, r);
+      bar_target += static_cast<unsigned>(s.G);
+      red_release_gpu(a.counter, 1u);
+      const uint64_t t0 = df_clock();
+      while (ld_acquire_gpu(a.counter) < bar_target) {
+        if (df_clock() - t0 > 2000000000ull) { flag_check(CHECK_WAIT); break; }
       }
-      df_mbar_wait(clR_bar, gen & 1, true);
       __threadfence();
     }
     ++gen;
     df_named_sync();
   };
   auto slot_of = [&](int q) { return static_cast<int>((g + q) % DF_NS); };
+  unsigned long long waited = 0;
   auto wait_full = [&](int q) {
     const uint32_t gg = g + q;
+    const unsigned long long t0 = (a.stamps && warp == 0 && lane == 0) ? df_clock() : 0ull;
     df_mbar_wait(full_bar(gg % DF_NS), (gg / DF_NS) & 1);
+    if (t0) waited += df_clock() - t0;
   };
   auto release = [&](int q) {
     __syncwarp();
@@ -715,6 +715,9 @@ k_decode_b1(const __grid_constant__ DfArgs a) {
     }
 
     df_stamp(a, l, 3);
+    if (a.stamps && threadIdx.x == 0)
+      a.stamps[(static_cast<size_t>(l) * gridDim.x + blockIdx.x) * 8 + 7] = waited;
+    waited = 0;
     grid_sync();
     df_stamp(a, l, 4);
 
