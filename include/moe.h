@@ -217,22 +217,23 @@ MOE_API int moe_layer_forward(const float* h_in, float* h_out, const uint16_t* x
  * Layers run in order on `stream`. */
 MOE_API size_t moe_decode_workspace_size(int T, int H, int I, int Is, int E, int k);
 /* Batch-1 steps (T = 1, per-expert or no bias) run as one persistent kernel
- * per up to 48 layers (8-CTA clusters, cooperative launch); other shapes run
+ * per up to 48 layers (one CTA per SM, cooperative launch); other shapes run
  * the per-layer calls.  enable = 0 forces the per-layer path.  spec_experts
  * (0..8, default 2): per layer, the experts with the largest router bias are
  * prefetched into L2 while the layer waits for its routing (their bytes are
  * read again, from L2, only if they are chosen). */
 MOE_API int moe_set_decode_fused(int enable, int spec_experts);
 /* L2 prefetch policy of the fused batch-1 kernel (bit flags, default 3):
- * 1 = once a layer's routing is known, prefetch all of its routed rows;
- * 2 = prefetch the next layer's routing-independent rows ahead of time. */
+ * 2 = prefetch the next layer's routing-independent rows ahead of time;
+ * 1 is reserved (no effect). */
 MOE_API int moe_set_decode_prefetch(int flags);
 /* Phase timestamps of the fused batch-1 kernel (a tracing aid): when
  * `stamps` (device, [L][G][8] uint64, G = moe_decode_grid()) is non-NULL,
  * thread 0 of every CTA writes %globaltimer (ns) at the phase boundaries of
- * each layer: 0 layer start, 1 router done, 2 routing known, 3 gate/up done,
- * 4 after the first grid barrier, 5 down/combine done, 6 after the second
- * grid barrier.  NULL turns it off (default). */
+ * each layer: 0 layer start, 1 router logit and shared gate/up done, 2 after
+ * the first grid barrier, 3 routed bytes issued, 4 routed gate/up done, 5
+ * after the second grid barrier, 6 down/combine done, 7 after the third grid
+ * barrier.  NULL turns it off (default). */
 MOE_API int moe_set_decode_profile(unsigned long long* stamps);
 /* CTAs of the fused batch-1 kernel on the current device (0: not available). */
 MOE_API int moe_decode_grid(void);

@@ -358,23 +358,12 @@ static bool fused_ok(int T, int H, int I, int Is, int E, int k, int bias_per_row
   if (!g_decode_fused || T != 1 || bias_per_row) return false;
   if (H % 64 || H > DF_MAX_H || I % 64 || Is % 64 || E % 8 || E > DF_MAX_E || k > 8) return false;
   if (k * I + Is > DF_MAX_ACT) return false;
-  if (G <= 0 || G % DF_CLUSTER || (H + G - 1) / G > DF_MAX_ROWS) return false;
-  {  // jobs per layer per CTA (upper bound) must fit the descriptor table
-    const int rg = df_rows_fit(2, H / 2, 4, 2 * (H / 64));
-    const int dn = df_rows_fit(1, I / 2, 2, 2 * (I / 64)), dsn = df_rows_fit(1, Is / 2, 2, 2 * (Is / 64));
-    if (rg < 1 || dn < 1 || dsn < 1) return false;
-    const int rows = (H + G - 1) / G;
-    const int jobs = (E / DF_CLUSTER + 1) / 2 + ((Is + G - 1) / G + rg - 1) / rg + 1 +
-                     ((k * I + G - 1) / G + rg - 1) / rg + 2 + k * ((rows + dn - 1) / dn) + (rows + dsn - 1) / dsn;
-    if (jobs > DF_MAX_JOBS) return false;
-  }
-  if (df_rows_fit(1, H, 2, 2 * (H / 64)) < 2) return false;                       // router jobs: 2 rows
-  if (df_rows_fit(2, H / 2, 4, 2 * (H / 64)) < 1) return false;                   // gate/up row pairs
-  if (df_rows_fit(1, I / 2, 2, 2 * (I / 64)) < 1 || df_rows_fit(1, Is / 2, 2, 2 * (Is / 64)) < 1) return false;
-  return true;
+  if (G <= 0 || (H + G - 1) / G > DF_MAX_ROWS) return false;
+  const long need = df_staging_need(H, I, Is, k, G);
+  return need >= 0 && need <= DF_RS;
 }
 
-// CTAs of the fused kernel that fit at once on this device (whole clusters; cached).
+// CTAs of the fused kernel: one per SM when that many fit at once (cached).
 static int fused_grid() {
   static int cached[64];
   int dev = 0;
@@ -383,21 +372,18 @@ static int fused_grid() {
   const size_t smem = decode_fused_smem();
   const void* fn = reinterpret_cast<const void*>(k_decode_b1);
   if (set_smem(fn, smem)) return 0;
-  int nsm = 0;
-  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(DF_CLUSTER * ((nsm + DF_CLUSTER - 1) / DF_CLUSTER), 1, 1);
-  cfg.blockDim = dim3(DF_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = DF_CLUSTER; at[0].val.clusterDim.y = 1; at[0].val.clusterDim.z = 1;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n <= 0) { cudaGetLastError(); return 0; }
-  cached[dev] = n * DF_CLUSTER;
+  int nsm = 0, per = 0;
+  if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, DF_THREADS, smem) != cudaSuccess || per < 1) {
+    cudaGetLastError();
+    return 0;
+  }
+  cached[dev] = nsm;
   return cached[dev];
+}
+
+static size_t fused_ws(int I, int Is, int E, int k) {
+  return align_up(static_cast<size_t>(k * I + Is) * 2) + align_up(static_cast<size_t>(E) * 4) + 256;
 }
 
 static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, const moe_qmat* routers,
@@ -405,8 +391,11 @@ static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, con
                         uint16_t* x_trace, uint16_t* y_trace, int32_t* idx_trace, float* gates_trace, void* ws,
                         int G, cudaStream_t s) {
   if (!aligned16(h)) return fail(MOE_ERR_INVALID_ARG, "moe_decode_forward: h must be 16-byte aligned");
-  __half* act = static_cast<__half*>(ws);
-  unsigned* ctr = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + align_up(static_cast<size_t>(k * I + Is) * 2));
+  char* w = static_cast<char*>(ws);
+  __half* act = reinterpret_cast<__half*>(w);
+  float* logits = reinterpret_cast<float*>(w + align_up(static_cast<size_t>(k * I + Is) * 2));
+  unsigned* ctr = reinterpret_cast<unsigned*>(w + align_up(static_cast<size_t>(k * I + Is) * 2) +
+                                              align_up(static_cast<size_t>(E) * 4));
   const size_t smem = decode_fused_smem();
   int st;
   if ((st = set_smem(reinterpret_cast<const void*>(k_decode_b1), smem))) return st;
@@ -416,7 +405,7 @@ static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, con
     memset(&args, 0, sizeof(args));
     args.h = h; args.H = H; args.I = I; args.Is = Is; args.E = E; args.k = k; args.L = nl;
     blob_offsets(H, I, args.off);
-    args.act = act; args.counter = ctr;
+    args.act = act; args.logits = logits; args.counter = ctr;
     const size_t TH = static_cast<size_t>(H), Tk = static_cast<size_t>(k);
     args.x_trace = x_trace ? x_trace + l0 * TH : nullptr;
     args.y_trace = y_trace ? y_trace + l0 * TH : nullptr;
@@ -425,9 +414,6 @@ static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, con
     args.spec = g_decode_spec;
     args.prefetch = g_decode_prefetch;
     args.stamps = g_decode_stamps ? g_decode_stamps + static_cast<size_t>(l0) * G * 8 : nullptr;
-    args.rg_rows = df_rows_fit(2, H / 2, 4, 2 * (H / 64));
-    args.d_rows = df_rows_fit(1, I / 2, 2, 2 * (I / 64));
-    args.ds_rows = df_rows_fit(1, Is / 2, 2, 2 * (Is / 64));
     for (int l = 0; l < nl; ++l) {
       const moe_qmat& R = routers[l0 + l];
       DfLayer& d = args.layer[l];
@@ -455,13 +441,6 @@ static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, con
   return MOE_OK;
 }
 
-int moe_set_decode_profile(unsigned long long* stamps) {
-  g_decode_stamps = stamps;
-  return MOE_OK;
-}
-
-int moe_decode_grid(void) { return fused_grid(); }
-
 int moe_set_decode_prefetch(int flags) {
   if (flags < 0 || flags > 3) return fail(MOE_ERR_INVALID_ARG, "prefetch flags must be in [0, 3]");
   g_decode_prefetch = flags;
@@ -486,7 +465,7 @@ int moe_decode_launches(int T, int L) {
 
 size_t moe_decode_workspace_size(int T, int H, int I, int Is, int E, int k) {
   const size_t layered = moe_layer_workspace_size(T, H, I, Is, E, k);
-  const size_t fused = align_up(static_cast<size_t>(k * I + Is) * 2) + 256;
+  const size_t fused = fused_ws(I, Is, E, k);
   return layered > fused ? layered : fused;
 }
 
