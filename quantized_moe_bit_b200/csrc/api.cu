@@ -441,6 +441,13 @@ static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, con
   return MOE_OK;
 }
 
+int moe_set_decode_profile(unsigned long long* stamps) {
+  g_decode_stamps = stamps;
+  return MOE_OK;
+}
+
+int moe_decode_grid(void) { return fused_grid(); }
+
 int moe_set_decode_prefetch(int flags) {
   if (flags < 0 || flags > 3) return fail(MOE_ERR_INVALID_ARG, "prefetch flags must be in [0, 3]");
   g_decode_prefetch = flags;
