@@ -358,7 +358,7 @@ static bool fused_ok(int T, int H, int I, int Is, int E, int k, int bias_per_row
   if (!g_decode_fused || T != 1 || bias_per_row) return false;
   if (H % 64 || H > DF_MAX_H || I % 64 || Is % 64 || E % 8 || E > DF_MAX_E || k > 8) return false;
   if (k * I + Is > DF_MAX_ACT) return false;
-  if (G <= 0 || (H + G - 1) / G > DF_MAX_ROWS) return false;
+  if (G <= 0 || (H + G - 1) / G > DF_MAX_ROWS || E > G) return false;
   const long need = df_staging_need(H, I, Is, k, G);
   return need >= 0 && need <= DF_RS;
 }

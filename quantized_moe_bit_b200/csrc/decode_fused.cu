@@ -42,7 +42,7 @@ constexpr int DF_MAX_ROWS = 32;                 // output rows per CTA
 constexpr int DF_MAX_E = 256;
 constexpr int DF_RGC = 2;                       // row pairs per routed gate/up chunk
 constexpr int DF_MAX_CHUNKS = 32;               // routed chunks per CTA and layer (one per lane)
-constexpr int DF_RS = 194048;                   // shared-memory staging for a CTA's routed bytes
+constexpr int DF_RS = 193536;                   // shared-memory staging for a CTA's routed bytes
 
 struct DfLayer {
   const uint32_t* rq; const uint16_t* rs; const uint16_t* rb;   // router [E, H], 8-bit
@@ -186,7 +186,7 @@ __device__ __forceinline__ void sb_window(const uint16_t* base, int per, int r0,
   skew = static_cast<uint32_t>(a - a16);
 }
 
-enum : int { CH_RG = 0, CH_D = 1, CH_DS = 2 };
+enum : int { CH_RG = 0, CH_D = 1, CH_DS = 2, CH_SG = 3, CH_R = 4 };
 
 // One chunk of staged bytes: weight runs (run i at i * qbytes from the chunk
 // start), then scale/bias windows; sk[i] = offset of window i's first row
@@ -222,10 +222,19 @@ __device__ inline DfChunk df_chunk(int kind, int slot, int r0, int rows, int H, 
     C.qbytes = static_cast<uint32_t>(rows) * (I / 2); nq = 1;
     sc[0] = reinterpret_cast<const uint16_t*>(blob + a.off[7]); sc[1] = reinterpret_cast<const uint16_t*>(blob + a.off[8]);
     ns = 2; per = I / 64;
-  } else {
+  } else if (kind == CH_DS) {
     q[0] = reinterpret_cast<const uint8_t*>(W.sq[2]) + static_cast<size_t>(r0) * (Is / 2);
     C.qbytes = static_cast<uint32_t>(rows) * (Is / 2); nq = 1;
     sc[0] = W.ss[2]; sc[1] = W.sb[2]; ns = 2; per = Is / 64;
+  } else if (kind == CH_SG) {
+    q[0] = reinterpret_cast<const uint8_t*>(W.sq[0]) + static_cast<size_t>(r0) * (H / 2);
+    q[1] = reinterpret_cast<const uint8_t*>(W.sq[1]) + static_cast<size_t>(r0) * (H / 2);
+    C.qbytes = static_cast<uint32_t>(rows) * (H / 2); nq = 2;
+    sc[0] = W.ss[0]; sc[1] = W.sb[0]; sc[2] = W.ss[1]; sc[3] = W.sb[1]; ns = 4; per = H / 64;
+  } else {   // CH_R: router rows (8-bit, H bytes each)
+    q[0] = reinterpret_cast<const uint8_t*>(W.rq) + static_cast<size_t>(r0) * H;
+    C.qbytes = static_cast<uint32_t>(rows) * H; nq = 1;
+    sc[0] = W.rs; sc[1] = W.rb; ns = 2; per = H / 64;
   }
   uint32_t o = 0;
   for (int i = 0; i < nq; ++i) {
@@ -325,12 +334,13 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
   float* red = part + DF_MAX_ROWS * 9;                                 // [32]
   int* sel = reinterpret_cast<int*>(red + 32);                         // [8]
   float* selg = reinterpret_cast<float*>(sel + 8);                     // [8]
-  DfChunk* tab = reinterpret_cast<DfChunk*>(selg + 8);                 // [DF_MAX_CHUNKS + 1]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(tab + DF_MAX_CHUNKS + 1);   // [DF_MAX_CHUNKS + 1]
+  DfChunk* tab = reinterpret_cast<DfChunk*>(selg + 8);                 // [DF_MAX_CHUNKS + 3]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(tab + DF_MAX_CHUNKS + 3);   // [DF_MAX_CHUNKS + 3]
+  const int IDX_DS = DF_MAX_CHUNKS, IDX_SG = DF_MAX_CHUNKS + 1, IDX_R = DF_MAX_CHUNKS + 2;
   const uint32_t bar0 = smem_addr(bars);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i <= DF_MAX_CHUNKS; ++i) df_mbar_init(bar0 + 8u * i, 1);
+    for (int i = 0; i < DF_MAX_CHUNKS + 3; ++i) df_mbar_init(bar0 + 8u * i, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -395,7 +405,30 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       }
     }
   };
+  // warp 0: chunk `idx` at `off` in the staging area, completing on its mbarrier
+  auto issue_chunk = [&](int idx, const DfChunk& C0, uint32_t off) {
+    if (lane == 0) {
+      tab[idx] = C0;
+      tab[idx].off = off;
+      df_mbar_expect_tx(bar0 + 8u * idx, C0.bytes);
+    }
+    __syncwarp();
+    const DfChunk& T = tab[idx];
+    if (lane < T.n) df_bulk_g2s(smem_addr(rs + T.off + T.dst[lane]), T.src[lane], T.len[lane], bar0 + 8u * idx);
+    __syncwarp();
+  };
+  // routing-independent rows of layer l's phase A: shared gate/up rows, router row c
+  auto issue_phase_a = [&](int l) {
+    const DfLayer& V = a.layer[l];
+    DfChunk sg = df_chunk(CH_SG, 0, s0, s1 - s0, H, I, Is, a, V, sel);
+    issue_chunk(IDX_SG, sg, 0u);
+    if (c < E) {
+      DfChunk rc = df_chunk(CH_R, 0, c, 1, H, I, Is, a, V, sel);
+      issue_chunk(IDX_R, rc, (sg.bytes + 127u) & ~127u);
+    }
+  };
   prefetch_layer(0);
+  if (warp == 0) issue_phase_a(0);
 
   for (int l = 0; l < a.L; ++l) {
     const DfLayer& W = a.layer[l];
@@ -465,16 +498,18 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       }
     }
 
-    // --------------------------------- router logit(s) and shared gate/up rows
+    // --------------------------------- router logit and shared gate/up rows
     if (warp == DF_WARPS - 1) {
-      for (int e = c; e < E; e += G) {
-        const uint8_t* qrow = reinterpret_cast<const uint8_t*>(W.rq) + static_cast<size_t>(e) * H;
-        const uint16_t* S = W.rs + static_cast<size_t>(e) * (H / 64);
-        const uint16_t* B = W.rb + static_cast<size_t>(e) * (H / 64);
+      if (c < E) {
+        const DfChunk& C = tab[IDX_R];
+        df_mbar_wait(bar0 + 8u * IDX_R, par);
+        const uint8_t* qrow = rs + C.off;
+        const uint16_t* S = reinterpret_cast<const uint16_t*>(rs + C.off + C.sk[0]);
+        const uint16_t* B = reinterpret_cast<const uint16_t*>(rs + C.off + C.sk[1]);
         float acc = 0.f;
         for (int cc = lane; cc < H / 16; cc += 32) {
-          const uint4 q4 = ldg_nc_v4(qrow + 16 * cc);
-          const float sc = bf16_to_f32(ldg_u16(S + (cc >> 2))), bi = bf16_to_f32(ldg_u16(B + (cc >> 2)));
+          const uint4 q4 = *reinterpret_cast<const uint4*>(qrow + 16 * cc);
+          const float sc = bf16_to_f32(S[cc >> 2]), bi = bf16_to_f32(B[cc >> 2]);
           const float* xv = xs + 16 * cc;
           const uint32_t w[4] = {q4.x, q4.y, q4.z, q4.w};
           float a0 = 0.f, a1 = 0.f, sm = 0.f;
@@ -488,15 +523,19 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
           acc += sc * ((a0 + a1) - 1024.f * sm) + bi * sm;
         }
         acc = warp_sum(acc);
-        if (lane == 0) a.logits[e] = acc + (W.bias ? W.bias[e] : 0.f);
+        if (lane == 0) a.logits[c] = acc + (W.bias ? W.bias[c] : 0.f);
       }
-    } else {
-      for (int i = s0 + warp; i < s1; i += DF_WARPS - 1) {
-        const size_t rq = static_cast<size_t>(i) * (H / 2), rsb = static_cast<size_t>(i) * (H / 64);
-        const float2 gu = df_pair(reinterpret_cast<const uint8_t*>(W.sq[0]) + rq,
-                                  reinterpret_cast<const uint8_t*>(W.sq[1]) + rq, W.ss[0] + rsb, W.sb[0] + rsb,
-                                  W.ss[1] + rsb, W.sb[1] + rsb, nch, xp, xst, true);
-        if (lane == 0) a.act[kI + i] = __float2half_rn(gelu_tanh(gu.x) * gu.y);
+    } else if (s1 > s0) {
+      const DfChunk& C = tab[IDX_SG];
+      df_mbar_wait(bar0 + 8u * IDX_SG, par);
+      const unsigned char* base = rs + C.off;
+      for (int r = warp; r < s1 - s0; r += DF_WARPS - 1) {
+        const float2 gu = df_pair(base + r * (H / 2), base + C.qbytes + r * (H / 2),
+                                  reinterpret_cast<const uint16_t*>(base + C.sk[0]) + r * (H / 64),
+                                  reinterpret_cast<const uint16_t*>(base + C.sk[1]) + r * (H / 64),
+                                  reinterpret_cast<const uint16_t*>(base + C.sk[2]) + r * (H / 64),
+                                  reinterpret_cast<const uint16_t*>(base + C.sk[3]) + r * (H / 64), nch, xp, xst, false);
+        if (lane == 0) a.act[kI + s0 + r] = __float2half_rn(gelu_tanh(gu.x) * gu.y);
       }
     }
     df_stamp(a, l, 1);
@@ -508,6 +547,9 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       unsigned taken = 0u;
       float sv[8];
       int si[8];
+      float lv[DF_MAX_E / 32];            // this lane's logits, read once
+#pragma unroll
+      for (int t = 0; t < DF_MAX_E / 32; ++t) lv[t] = (lane + 32 * t < E) ? __ldcg(a.logits + lane + 32 * t) : 0.f;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         sv[j] = 0.f;
@@ -515,9 +557,11 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
         if (j < k) {
           float bv = -INFINITY;
           int bi = 0x7fffffff;
-          for (int t = 0, e = lane; e < E; ++t, e += 32) {
-            if (taken & (1u << t)) continue;
-            const float v = __ldcg(a.logits + e);
+#pragma unroll
+          for (int t = 0; t < DF_MAX_E / 32; ++t) {
+            const int e = lane + 32 * t;
+            if (e >= E || (taken & (1u << t))) continue;
+            const float v = lv[t];
             if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; }
           }
           for (int o = 16; o > 0; o >>= 1) {
@@ -601,26 +645,20 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       }
     }
     df_stamp(a, l, 4);
+    // shared down rows of phase C into the gate/up part of the staging area
+    // (free now) when it is large enough, else after the down chunks
+    const int dsc = IDX_DS;
+    __syncthreads();
+    if (warp == 0) {
+      const DfChunk C = df_chunk(CH_DS, 0, o0, nrow, H, I, Is, a, W, sel);
+      const uint32_t rg_bytes = tab[nrg].off;
+      const uint32_t used = tab[nchunk - 1].off + tab[nchunk - 1].bytes;
+      issue_chunk(dsc, C, C.bytes <= rg_bytes ? 0u : ((used + 127u) & ~127u));
+    }
     grid_sync();
     df_stamp(a, l, 5);
 
     // ------------------------------------------------------------- phase C
-    // shared down rows into the (now free) gate/up part of the staging area
-    const int dsc = DF_MAX_CHUNKS;               // its mbarrier
-    if (warp == 0) {
-      if (lane == 0) {
-        DfChunk C = df_chunk(CH_DS, 0, o0, nrow, H, I, Is, a, W, sel);
-        // over the gate/up chunks when they are large enough, else after the down chunks
-        const uint32_t rg_bytes = tab[nrg].off;
-        const uint32_t used = tab[nchunk - 1].off + tab[nchunk - 1].bytes;
-        C.off = C.bytes <= rg_bytes ? 0u : ((used + 127u) & ~127u);
-        tab[DF_MAX_CHUNKS] = C;
-        df_mbar_expect_tx(bar0 + 8u * dsc, C.bytes);
-      }
-      __syncwarp();
-      const DfChunk& T = tab[DF_MAX_CHUNKS];
-      if (lane < T.n) df_bulk_g2s(smem_addr(rs + T.off + T.dst[lane]), T.src[lane], T.len[lane], bar0 + 8u * dsc);
-    }
     if (l + 1 < a.L) prefetch_layer(l + 1);
     for (int w = threadIdx.x; w < nact / 8; w += DF_THREADS) {
       const uint4 u = ldcg_v4(a.act + 8 * w);
@@ -679,6 +717,10 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       a.h[o] = __ldcg(a.h + o) + y;
       if (a.y_trace) a.y_trace[static_cast<size_t>(l) * H + o] = f32_to_bf16(y);
     }
+    if (l + 1 < a.L) {
+      __syncthreads();                     // staging area read out
+      if (warp == 0) issue_phase_a(l + 1);
+    }
     df_stamp(a, l, 6);
     if (l + 1 < a.L) grid_sync();
     df_stamp(a, l, 7);
@@ -688,13 +730,13 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
 size_t decode_fused_smem() {
   return static_cast<size_t>(DF_RS) + static_cast<size_t>(DF_MAX_ACT / 8) * 24 + DF_MAX_H / 8 * 16 +
          DF_MAX_H / 32 * 8 + DF_MAX_ROWS * 9 * 4 + 32 * 4 + 8 * 4 + 8 * 4 +
-         (DF_MAX_CHUNKS + 1) * sizeof(DfChunk) + (DF_MAX_CHUNKS + 1) * 8 + 128;
+         (DF_MAX_CHUNKS + 3) * sizeof(DfChunk) + (DF_MAX_CHUNKS + 3) * 8 + 128;
 }
 
 // Staging bytes a CTA needs for its routed chunks (worst case over CTAs), or
 // -1 if more chunks than DF_MAX_CHUNKS.
 inline long df_staging_need(int H, int I, int Is, int k, int G) {
-  const int pairs = (k * I + G - 1) / G + 1, rows = (H + G - 1) / G;
+  const int pairs = (k * I + G - 1) / G, rows = (H + G - 1) / G;
   const int nrg = (pairs + DF_RGC - 1) / DF_RGC + 1;
   if (nrg + k > DF_MAX_CHUNKS) return -1;
   const long rg = static_cast<long>(pairs) * H + static_cast<long>(nrg) * 4 * (DF_RGC * 2 * (H / 64) + 32);
