@@ -40,7 +40,7 @@ constexpr int DF_CPL = 3;                       // uint4 chunks per lane of a ga
 constexpr int DF_MAX_ACT = 8192;                // k*I + Is
 constexpr int DF_MAX_ROWS = 32;                 // output rows per CTA
 constexpr int DF_MAX_E = 256;
-constexpr int DF_RGC = 2;                       // row pairs per routed gate/up chunk
+constexpr int DF_RGC = 10;                      // row pairs per routed gate/up chunk
 constexpr int DF_MAX_CHUNKS = 32;               // routed chunks per CTA and layer (one per lane)
 constexpr int DF_RS = 193536;                   // shared-memory staging for a CTA's routed bytes
 
@@ -683,30 +683,46 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       actS[w] = make_float2(1024.f * off, (f0.x + f0.y + f2.x + f2.y) + 16.f * (f1.x + f1.y + f3.x + f3.y));
     }
     __syncthreads();
-    // units (row r, piece u): u < k routed slot u, u == k the shared expert
-    for (int un = warp; un < nrow * (k + 1); un += DF_WARPS) {
-      const int r = un / (k + 1), u = un - r * (k + 1);
+    // units (piece u, block of DF_RB rows): u < k routed slot u (K = I),
+    // u == k the shared expert (K = Is); the activation word is loaded once
+    // and applied to the block's rows (independent accumulators)
+    constexpr int DF_RB = 4;
+    const int nblk = (nrow + DF_RB - 1) / DF_RB;
+    for (int un = warp; un < nblk * (k + 1); un += DF_WARPS) {
+      const int u = un % (k + 1), rb = un / (k + 1);
       const int ch = u < k ? nrg + u : dsc;
       const DfChunk& C = tab[ch];
       df_mbar_wait(bar0 + 8u * ch, par);
       const int K = u < k ? I : Is;
       const int wbase = u < k ? u * (I / 8) : kI / 8;
+      const int rbeg = rb * DF_RB, nr = min(DF_RB, nrow - rbeg);
       const unsigned char* base = rs + C.off;
-      const uint8_t* qrow = base + static_cast<size_t>(r) * (K / 2);
-      const uint16_t* S = reinterpret_cast<const uint16_t*>(base + C.sk[0]) + r * (K / 64);
-      const uint16_t* B = reinterpret_cast<const uint16_t*>(base + C.sk[1]) + r * (K / 64);
-      float acc = 0.f;
+      const uint8_t* q0 = base + static_cast<size_t>(rbeg) * (K / 2);
+      const uint16_t* S0 = reinterpret_cast<const uint16_t*>(base + C.sk[0]) + rbeg * (K / 64);
+      const uint16_t* B0 = reinterpret_cast<const uint16_t*>(base + C.sk[1]) + rbeg * (K / 64);
+      float acc[DF_RB];
+#pragma unroll
+      for (int t = 0; t < DF_RB; ++t) acc[t] = 0.f;
       for (int w = lane; w < K / 8; w += 32) {
-        const uint32_t qw = *reinterpret_cast<const uint32_t*>(qrow + 4 * w);
         const uint4 pp = actP[wbase + w];
         const uint32_t p[4] = {pp.x, pp.y, pp.z, pp.w};
-        float a0 = 0.f, a1 = 0.f;
-        dot_word4(qw, p, a0, a1);
         const float2 st = actS[wbase + w];
-        acc += bf16_to_f32(S[w >> 3]) * ((a0 + a1) - st.x) + bf16_to_f32(B[w >> 3]) * st.y;
+#pragma unroll
+        for (int t = 0; t < DF_RB; ++t) {
+          if (t < nr) {
+            const uint32_t qw = *reinterpret_cast<const uint32_t*>(q0 + t * (K / 2) + 4 * w);
+            float a0 = 0.f, a1 = 0.f;
+            dot_word4(qw, p, a0, a1);
+            acc[t] += bf16_to_f32(S0[t * (K / 64) + (w >> 3)]) * ((a0 + a1) - st.x) +
+                      bf16_to_f32(B0[t * (K / 64) + (w >> 3)]) * st.y;
+          }
+        }
       }
-      acc = warp_sum(acc);
-      if (lane == 0) part[r * 9 + u] = acc;
+#pragma unroll
+      for (int t = 0; t < DF_RB; ++t) {
+        const float v = warp_sum(acc[t]);
+        if (lane == 0 && t < nr) part[(rbeg + t) * 9 + u] = v;
+      }
     }
     __syncthreads();
     for (int r = threadIdx.x; r < nrow; r += DF_THREADS) {
