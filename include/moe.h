@@ -219,21 +219,23 @@ MOE_API size_t moe_decode_workspace_size(int T, int H, int I, int Is, int E, int
 /* Batch-1 steps (T = 1, per-expert or no bias) run as one persistent kernel
  * per up to 48 layers (one CTA per SM, cooperative launch); other shapes run
  * the per-layer calls.  enable = 0 forces the per-layer path.  spec_experts
- * (0..8, default 2): per layer, the experts with the largest router bias are
+ * (0..8, default 0): per layer, the experts with the largest router bias are
  * prefetched into L2 while the layer waits for its routing (their bytes are
  * read again, from L2, only if they are chosen). */
 MOE_API int moe_set_decode_fused(int enable, int spec_experts);
-/* L2 prefetch policy of the fused batch-1 kernel (bit flags, default 3):
+/* L2 prefetch policy of the fused batch-1 kernel (bit flags, default 0):
  * 2 = prefetch the next layer's routing-independent rows ahead of time;
  * 1 is reserved (no effect). */
 MOE_API int moe_set_decode_prefetch(int flags);
 /* Phase timestamps of the fused batch-1 kernel (a tracing aid): when
- * `stamps` (device, [L][G][8] uint64, G = moe_decode_grid()) is non-NULL,
+ * `stamps` (device, [L][G][16] uint64, G = moe_decode_grid()) is non-NULL,
  * thread 0 of every CTA writes %globaltimer (ns) at the phase boundaries of
- * each layer: 0 layer start, 1 router logit and shared gate/up done, 2 after
- * the first grid barrier, 3 routed bytes issued, 4 routed gate/up done, 5
- * after the second grid barrier, 6 down/combine done, 7 after the third grid
- * barrier.  NULL turns it off (default). */
+ * each layer: 0 start, 1 norm done, 2 router/shared gate-up done, 3 after the
+ * first grid barrier, 4 top-k done, 5 routed copies issued, 6 routed gate/up
+ * done, 7 shared-down copies issued, 8 after the second grid barrier, 9 L2
+ * prefetch issued, 10 activations staged, 11 down dots done, 12 combine done,
+ * 13 next layer's copies issued, 14 after the third grid barrier.  NULL turns
+ * it off (default). */
 MOE_API int moe_set_decode_profile(unsigned long long* stamps);
 /* CTAs of the fused batch-1 kernel on the current device (0: not available). */
 MOE_API int moe_decode_grid(void);

@@ -103,7 +103,7 @@ def moe_layer_forward(T: int, H: int, I: int, Is: int, E: int, k: int, router: m
                                   ptr(gates), ptr(ws), ws.numel() * ws.element_size(), stream_ptr(stream)))
 
 
-def moe_set_decode_fused(enable: bool, spec_experts: int = 2):
+def moe_set_decode_fused(enable: bool, spec_experts: int = 0):
     check(lib().moe_set_decode_fused(1 if enable else 0, spec_experts))
 
 

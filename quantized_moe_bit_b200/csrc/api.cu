@@ -13,8 +13,8 @@ namespace moe {
 static thread_local char g_err[512] = "";
 static int g_gemv_max_rows = 2;
 static int g_decode_fused = 1;
-static int g_decode_spec = 2;
-static int g_decode_prefetch = 3;
+static int g_decode_spec = 0;
+static int g_decode_prefetch = 0;
 static unsigned long long* g_decode_stamps = nullptr;
 
 int fail(int code, const char* fmt, ...) {
@@ -413,7 +413,7 @@ static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, con
     args.gates_trace = gates_trace ? gates_trace + l0 * Tk : nullptr;
     args.spec = g_decode_spec;
     args.prefetch = g_decode_prefetch;
-    args.stamps = g_decode_stamps ? g_decode_stamps + static_cast<size_t>(l0) * G * 8 : nullptr;
+    args.stamps = g_decode_stamps ? g_decode_stamps + static_cast<size_t>(l0) * G * 16 : nullptr;
     for (int l = 0; l < nl; ++l) {
       const moe_qmat& R = routers[l0 + l];
       DfLayer& d = args.layer[l];

@@ -61,7 +61,7 @@ struct DfArgs {
   uint16_t* x_trace; uint16_t* y_trace; int32_t* idx_trace; float* gates_trace;
   int spec;                         // experts speculatively prefetched per layer
   int prefetch;                     // bit 1: routing-independent rows of the next layer into L2
-  unsigned long long* stamps;       // optional phase timestamps [L][G][8] (ns), or null
+  unsigned long long* stamps;       // optional phase timestamps [L][G][16] (ns), or null
   DfLayer layer[DF_MAX_LAYERS];
 };
 
@@ -168,7 +168,7 @@ __device__ __forceinline__ uint4 ldcg_v4(const void* p) {
 // phase timestamps (when requested): layer l, CTA c, phase p
 __device__ __forceinline__ void df_stamp(const DfArgs& a, int l, int p) {
   if (a.stamps != nullptr && threadIdx.x == 0)
-    a.stamps[(static_cast<size_t>(l) * gridDim.x + blockIdx.x) * 8 + p] = df_clock();
+    a.stamps[(static_cast<size_t>(l) * gridDim.x + blockIdx.x) * 16 + p] = df_clock();
 }
 
 
@@ -498,6 +498,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       }
     }
 
+    df_stamp(a, l, 1);
     // --------------------------------- router logit and shared gate/up rows
     if (warp == DF_WARPS - 1) {
       if (c < E) {
@@ -538,9 +539,9 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
         if (lane == 0) a.act[kI + s0 + r] = __float2half_rn(gelu_tanh(gu.x) * gu.y);
       }
     }
-    df_stamp(a, l, 1);
-    grid_sync();
     df_stamp(a, l, 2);
+    grid_sync();
+    df_stamp(a, l, 3);
 
     // ------------------------------------------------ top-k, issue routed bytes
     if (warp == 0) {
@@ -591,6 +592,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
         if (c == 0 && a.gates_trace) a.gates_trace[static_cast<size_t>(l) * k + lane] = zl / den;
       }
       __syncwarp();
+      if (lane == 0) df_stamp(a, l, 4);
       // chunk `lane`: its bytes, its place in the staging area (exclusive scan)
       DfChunk C{};
       if (lane < nchunk) {
@@ -617,7 +619,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       }
     }
     __syncthreads();
-    df_stamp(a, l, 3);
+    df_stamp(a, l, 5);
 
     // ------------------------------------------------------ routed gate/up
     {
@@ -644,7 +646,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
         if (lane == 0) a.act[C.slot * I + C.r0 + r] = __float2half_rn(gelu_tanh(gu.x) * gu.y);
       }
     }
-    df_stamp(a, l, 4);
+    df_stamp(a, l, 6);
     // shared down rows of phase C into the gate/up part of the staging area
     // (free now) when it is large enough, else after the down chunks
     const int dsc = IDX_DS;
@@ -655,11 +657,13 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       const uint32_t used = tab[nchunk - 1].off + tab[nchunk - 1].bytes;
       issue_chunk(dsc, C, C.bytes <= rg_bytes ? 0u : ((used + 127u) & ~127u));
     }
+    df_stamp(a, l, 7);
     grid_sync();
-    df_stamp(a, l, 5);
+    df_stamp(a, l, 8);
 
     // ------------------------------------------------------------- phase C
     if (l + 1 < a.L) prefetch_layer(l + 1);
+    df_stamp(a, l, 9);
     for (int w = threadIdx.x; w < nact / 8; w += DF_THREADS) {
       const uint4 u = ldcg_v4(a.act + 8 * w);
       float v[8];
@@ -683,6 +687,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       actS[w] = make_float2(1024.f * off, (f0.x + f0.y + f2.x + f2.y) + 16.f * (f1.x + f1.y + f3.x + f3.y));
     }
     __syncthreads();
+    df_stamp(a, l, 10);
     // units (piece u, block of DF_RB rows): u < k routed slot u (K = I),
     // u == k the shared expert (K = Is); the activation word is loaded once
     // and applied to the block's rows (independent accumulators)
@@ -725,6 +730,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       }
     }
     __syncthreads();
+    df_stamp(a, l, 11);
     for (int r = threadIdx.x; r < nrow; r += DF_THREADS) {
       float y = 0.f;
       for (int j = 0; j < k; ++j) y = fmaf(selg[j], part[r * 9 + j], y);
@@ -733,13 +739,14 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       a.h[o] = __ldcg(a.h + o) + y;
       if (a.y_trace) a.y_trace[static_cast<size_t>(l) * H + o] = f32_to_bf16(y);
     }
+    df_stamp(a, l, 12);
     if (l + 1 < a.L) {
       __syncthreads();                     // staging area read out
       if (warp == 0) issue_phase_a(l + 1);
     }
-    df_stamp(a, l, 6);
+    df_stamp(a, l, 13);
     if (l + 1 < a.L) grid_sync();
-    df_stamp(a, l, 7);
+    df_stamp(a, l, 14);
   }
 }
 

@@ -128,7 +128,7 @@ def test_stack_tiny_b1_fused_and_layered(M, spec):
         M.moe_set_decode_fused(False, spec)
         gl = _run_stack(M, cfg, layers, z)
     finally:
-        M.moe_set_decode_fused(True, 2)
+        M.moe_set_decode_fused(True, 0)
     for g in (gf, gl):
         _check_stack(cfg, hs, z, g, set(range(cfg.layers)))
     for key in ("h", "x", "y", "idx", "gates"):
@@ -140,7 +140,7 @@ def test_stack_tiny_b1_fused_and_layered(M, spec):
         g_none = _run_stack(M, cfg, layers, z, traces=False)
         g_idx = _run_stack(M, cfg, layers, z, traces="idx")
     finally:
-        M.moe_set_decode_fused(True, 2)
+        M.moe_set_decode_fused(True, 0)
     assert np.array_equal(g_none["h"], gf["h"]) and np.array_equal(g_idx["h"], gf["h"])
     assert np.array_equal(g_idx["idx"], gf["idx"])
 
