@@ -248,6 +248,74 @@ MOE_API int moe_decode_forward(float* h, int T, int H, int I, int Is, int E, int
                                int32_t* idx_trace, float* gates_trace, void* ws,
                                size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Per-layer LFU expert-slot cache (routed experts streamed from pinned host
+ * memory).  "TurboFieldfare: Gemma 4 26B on an 8 GB MacBook, in ~2 GB of
+ * RAM" (blog-mushroom.pages.dev), section "Why 26B Fits in 2 GB": per token
+ * the host checks the 8 selected ids against a 16-slot LFU cache of the
+ * layer; hits reuse the resident copy, misses fetch the blob; the shared
+ * expert runs while the fetches complete.
+ * Policy (the pages say only "16-slot LFU"): counts live while an expert is
+ * resident (insert 1, hit +1); in a step hits are taken first, then misses,
+ * each in the step's order; a global tick advances per access; a miss fills
+ * the lowest empty slot, else evicts, among slots not used by the step, the
+ * smallest (count, last tick, slot index).  Every access is logged as
+ * (layer, step, expert, hit, slot), `step` counting that layer's steps.
+ * A handle is not thread-safe: one handle per pair of streams.
+ */
+typedef struct moe_lfu moe_lfu;
+enum { MOE_LFU_FAULT_NONE = 0, MOE_LFU_FAULT_COPY_FAILS = 1, MOE_LFU_FAULT_SLOW_COPY = 2 };
+/* host_blobs: host array [L*E] of pinned host pointers (blob of expert e of
+ * layer l at index l*E + e), slot_pool: device memory of L*n_slots*slot_stride
+ * bytes (caller-owned; slot s of layer l at (l*n_slots + s)*slot_stride).
+ * Both NULL: a planning-only handle (moe_lfu_plan, moe_lfu_get_log). */
+MOE_API int moe_lfu_create(int n_layers, int n_experts, int n_slots, size_t blob_bytes,
+                           const void* const* host_blobs, void* slot_pool, size_t slot_stride,
+                           moe_lfu** out);
+/* Plan one step without copying: slots_out[i], hit_out[i] for ids[i]
+ * (distinct, at most n_slots of them).  Updates the cache state and log. */
+MOE_API int moe_lfu_plan(moe_lfu* h, int layer, const int32_t* ids, int n, int32_t* slots_out,
+                         int32_t* hit_out);
+/* One step: plan; on `side_stream` wait for `wait_event` (recorded by the
+ * caller after the kernels that read this layer's slots; may be NULL), copy
+ * each missed blob into its slot (one cudaMemcpyAsync per miss), update the
+ * layer's device pointer table dev_table [E] for the step's ids, and record
+ * `done_event`; the caller's compute stream waits on done_event before the
+ * expert kernels.  Host waits are bounded by timeout_ms (MOE_ERR_TIMEOUT). */
+MOE_API int moe_lfu_step(moe_lfu* h, int layer, const int32_t* ids, int n, void* side_stream,
+                         void* wait_event, void* done_event, void** dev_table, int timeout_ms);
+/* Poll an event until it completes or timeout_ms passes (MOE_ERR_TIMEOUT). */
+MOE_API int moe_lfu_wait(void* event, int timeout_ms);
+/* The access log: n_records records of 5 int32 (layer, step, expert, hit,
+ * slot); up to cap_records are copied into buf (may be NULL). */
+MOE_API int moe_lfu_get_log(moe_lfu* h, int32_t* buf, size_t cap_records, size_t* n_records);
+MOE_API int moe_lfu_stats(moe_lfu* h, int64_t* hits, int64_t* misses, int64_t* bytes_copied);
+/* Test hook: after `after_n` copies, every further copy fails (kind 1) or is
+ * delayed by 50 ms on the host (kind 2); kind 0 clears it. */
+MOE_API int moe_lfu_set_fault(moe_lfu* h, int kind, int after_n);
+MOE_API int moe_lfu_destroy(moe_lfu* h);
+
+/* One routed-MoE layer whose routed experts are streamed through the LFU
+ * slots of layer `layer` (A0 .. A7 with the residual update of hres):
+ * rms norm, router + top-k and bucketing on main_stream; the routing goes to
+ * the host (bounded wait); the shared expert is queued on main_stream so it
+ * runs while the misses are copied on side_stream; the layer's accesses are
+ * cut into steps (T = 1: the token's k ids in selection order; T > 1: the
+ * chunk's distinct experts, resident ones first, each group ascending, k per
+ * step); per step moe_lfu_step stages the blobs and main_stream runs the
+ * expert kernels for that step's experts through dev_table; then the combine
+ * adds y into hres.  The per-pair arithmetic is that of moe_layer_forward,
+ * so the result equals the all-resident layer bit for bit.
+ *   dev_table  device [E] pointer table of this layer (updated per step)
+ *   ws         device workspace >= moe_streamed_workspace_size(...) */
+MOE_API size_t moe_streamed_workspace_size(int T, int H, int I, int Is, int E, int k);
+MOE_API int moe_streamed_layer_forward(moe_lfu* h, int layer, float* hres, int T, int H, int I, int Is,
+                                       int E, int k, const moe_qmat* router, const float* bias,
+                                       int bias_per_row, const moe_qmat* shared, void** dev_table,
+                                       uint16_t* x_out, uint16_t* y_out, int32_t* idx_out, void* ws,
+                                       size_t ws_bytes, void* main_stream, void* side_stream,
+                                       int timeout_ms);
+
 #ifdef __cplusplus
 }
 #endif

@@ -11,7 +11,7 @@ LIB = os.path.join(HERE, "libmoe.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 CU_MAIN = ["libmoe.cu"]
-CPP = []
+CPP = ["lfu.cpp"]
 
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

@@ -60,6 +60,17 @@ SIGNATURES = {
     "moe_decode_grid": (_I, []),
     "moe_decode_forward": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, C.POINTER(moe_qmat), C.POINTER(C.c_void_p), _I,
                                 C.POINTER(C.c_void_p), C.POINTER(moe_qmat), _P, _P, _P, _P, _P, _Z, _P]),
+    "moe_lfu_create": (_I, [_I, _I, _I, _Z, _P, _P, _Z, C.POINTER(C.c_void_p)]),
+    "moe_lfu_plan": (_I, [_P, _I, _P, _I, _P, _P]),
+    "moe_lfu_step": (_I, [_P, _I, _P, _I, _P, _P, _P, _P, _I]),
+    "moe_lfu_wait": (_I, [_P, _I]),
+    "moe_lfu_get_log": (_I, [_P, _P, _Z, C.POINTER(C.c_size_t)]),
+    "moe_lfu_stats": (_I, [_P, C.POINTER(C.c_int64), C.POINTER(C.c_int64), C.POINTER(C.c_int64)]),
+    "moe_lfu_set_fault": (_I, [_P, _I, _I]),
+    "moe_lfu_destroy": (_I, [_P]),
+    "moe_streamed_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "moe_streamed_layer_forward": (_I, [_P, _I, _P, _I, _I, _I, _I, _I, _I, C.POINTER(moe_qmat), _P, _I,
+                                        C.POINTER(moe_qmat), _P, _P, _P, _P, _P, _Z, _P, _P, _I]),
 }
 
 

@@ -152,3 +152,83 @@ def moe_decode_forward(h, I: int, Is: int, E: int, k: int, stack: "DecodeStack",
                                    stack.bias_per_row, stack.tables, stack.shared, ptr(x_trace), ptr(y_trace),
                                    ptr(idx_trace), ptr(gates_trace), ptr(ws), ws.numel() * ws.element_size(),
                                    stream_ptr(stream)))
+
+
+# ------------------------------------------------------------------ LFU cache
+class MoeLfu:
+    """Handle of the per-layer LFU expert-slot cache (moe_lfu_* calls)."""
+
+    def __init__(self, n_layers: int, n_experts: int, n_slots: int, blob_bytes: int = 0, host_blob_ptrs=None,
+                 slot_pool=None, slot_stride: int = 0):
+        self._h = C.c_void_p()
+        self._blobs = None
+        if host_blob_ptrs is not None:
+            self._blobs = (C.c_void_p * len(host_blob_ptrs))(*host_blob_ptrs)
+        check(lib().moe_lfu_create(n_layers, n_experts, n_slots, blob_bytes, self._blobs, ptr(slot_pool),
+                                   slot_stride, C.byref(self._h)))
+        self.n_slots = n_slots
+
+    @property
+    def handle(self):
+        return self._h
+
+    def plan(self, layer: int, ids):
+        n = len(ids)
+        a = (C.c_int32 * max(n, 1))(*ids)
+        so = (C.c_int32 * max(n, 1))()
+        ho = (C.c_int32 * max(n, 1))()
+        check(lib().moe_lfu_plan(self._h, layer, a, n, so, ho))
+        return list(so)[:n], list(ho)[:n]
+
+    def step(self, layer: int, ids, side_stream, wait_event, done_event, dev_table, timeout_ms: int = 2000):
+        n = len(ids)
+        a = (C.c_int32 * max(n, 1))(*ids)
+        check(lib().moe_lfu_step(self._h, layer, a, n, stream_ptr(side_stream),
+                                 None if wait_event is None else wait_event.cuda_event,
+                                 done_event.cuda_event, ptr(dev_table), timeout_ms))
+
+    def log(self):
+        n = C.c_size_t()
+        check(lib().moe_lfu_get_log(self._h, None, 0, C.byref(n)))
+        buf = (C.c_int32 * (5 * max(n.value, 1)))()
+        check(lib().moe_lfu_get_log(self._h, buf, n.value, C.byref(n)))
+        v = list(buf)[:5 * n.value]
+        return [tuple(v[i:i + 5]) for i in range(0, len(v), 5)]
+
+    def stats(self):
+        h, m, b = C.c_int64(), C.c_int64(), C.c_int64()
+        check(lib().moe_lfu_stats(self._h, C.byref(h), C.byref(m), C.byref(b)))
+        return h.value, m.value, b.value
+
+    def set_fault(self, kind: int, after_n: int):
+        check(lib().moe_lfu_set_fault(self._h, kind, after_n))
+
+    def close(self):
+        if self._h:
+            lib().moe_lfu_destroy(self._h)
+            self._h = C.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def moe_lfu_wait(event, timeout_ms: int):
+    check(lib().moe_lfu_wait(event.cuda_event, timeout_ms))
+
+
+def moe_streamed_workspace_size(T: int, H: int, I: int, Is: int, E: int, k: int) -> int:
+    return lib().moe_streamed_workspace_size(T, H, I, Is, E, k)
+
+
+def moe_streamed_layer_forward(lfu: "MoeLfu", layer: int, h, I: int, Is: int, E: int, k: int, router: moe_qmat,
+                               bias, bias_per_row: int, shared, dev_table, ws, x_out=None, y_out=None, idx_out=None,
+                               main_stream=None, side_stream=None, timeout_ms: int = 5000):
+    T, H = h.shape
+    arr = _qmat3(shared)
+    check(lib().moe_streamed_layer_forward(lfu.handle, layer, ptr(h), T, H, I, Is, E, k, C.byref(router), ptr(bias),
+                                           bias_per_row, arr, ptr(dev_table), ptr(x_out), ptr(y_out), ptr(idx_out),
+                                           ptr(ws), ws.numel() * ws.element_size(), stream_ptr(main_stream),
+                                           stream_ptr(side_stream), timeout_ms))
