@@ -74,13 +74,26 @@ def check_routing(gpu_idx: np.ndarray, logits: np.ndarray, k: int):
     return int(ties.sum())
 
 
+def bf16_half_ulp(ref: np.ndarray) -> np.ndarray:
+    """Half the bf16 spacing at |ref| (8 significant bits)."""
+    a = np.maximum(np.abs(ref), np.finfo(np.float64).tiny)
+    return 0.5 * np.exp2(np.floor(np.log2(a)) - 7)
+
+
 def check_output(y_gpu_bits: np.ndarray, ref: np.ndarray, what: str = "y"):
+    """bf16 output against the fp64 oracle.  The output is bf16, so rounding
+    the exact value to bf16 is not an error of the computation: the max bound
+    is applied on top of half a bf16 unit of the exact value (an element at 6
+    rms already carries up to 2.3e-2 rms of pure rounding); the mean bound
+    includes the rounding."""
     y = O.bf16_to_f64(y_gpu_bits)
     err = np.abs(y - ref)
     rms = float(np.sqrt(np.mean(ref * ref)))
-    mx, mean = float(err.max()) / rms, float(err.mean()) / rms
-    assert mx <= MAX_TOL and mean <= MEAN_TOL, f"{what}: max {mx:.3e} mean {mean:.3e} (x rms)"
-    return mx, mean
+    excess = float(np.max(err - bf16_half_ulp(ref))) / rms
+    mean = float(err.mean()) / rms
+    assert excess <= MAX_TOL and mean <= MEAN_TOL, \
+        f"{what}: max beyond bf16 rounding {excess:.3e}, mean {mean:.3e} (x rms)"
+    return excess, mean
 
 
 def check_close(a: np.ndarray, ref: np.ndarray, max_rel: float, mean_rel: float, what: str):
