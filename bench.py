@@ -144,6 +144,30 @@ def cpu_baseline_oracle(cfg, n_layers: int, stream: int):
     return tok_s, cores, dt
 
 
+def replica_streams(rank: int, n: int) -> list:
+    """Generator stream ids of the n input tokens of replica `rank`: disjoint
+    across ranks (each replica decodes its own token stream)."""
+    base = 1000 + rank * 100000
+    return [base + s for s in range(n)]
+
+
+def max_over_ranks(values, world: int, device):
+    """Element-wise max over ranks of a list of floats (timings): every rank
+    takes part, every rank gets the result."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def whole_job_rate(ms: float, steps: int, world: int) -> float:
+    """Tokens per second of the whole job: every replica decodes `steps`
+    tokens; the job takes the slowest rank's time."""
+    return steps * world / (ms / 1e3)
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -180,8 +204,7 @@ def run_ours(args, rank, world, local_rank):
     stack = M.DecodeStack(layers)
     H = cfg.H
     n_in = args.warmup + args.steps
-    base_stream = 1000 + rank * 100000
-    z = np.concatenate([gen.rows(cfg.seed, base_stream + s, 1, H) for s in range(n_in)])  # [n_in, H]
+    z = np.concatenate([gen.rows(cfg.seed, s, 1, H) for s in replica_streams(rank, n_in)])  # [n_in, H]
     z_dev = torch.from_numpy(z).to(device).view(n_in, 1, H)
     ws = torch.empty(M.moe_decode_workspace_size(1, H, cfg.I, cfg.Is, cfg.E, cfg.k), dtype=torch.uint8,
                      device=device)
@@ -250,16 +273,12 @@ def run_ours(args, rank, world, local_rank):
     ms_e2e = e2.elapsed_time(e3)
     M.moe_sync()
 
-    t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms, ms_e2e = float(t[0]), float(t[1])
+    ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, device)
     del g
     if rank != 0:
         return
-    tokens = args.steps * world
-    value = tokens / (ms / 1e3)
-    e2e_val = tokens / (ms_e2e / 1e3)
+    value = whole_job_rate(ms, args.steps, world)
+    e2e_val = whole_job_rate(ms_e2e, args.steps, world)
     hbm, src = peaks()
     bytes_step = step_bytes(cfg, distinct)
     achieved = bytes_step / (ms / args.steps / 1e3) / 1e9
@@ -307,7 +326,7 @@ def main():
         import torch
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
         run_ours(args, rank, world, local_rank)
