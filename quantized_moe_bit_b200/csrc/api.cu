@@ -356,25 +356,21 @@ int moe_layer_forward(const float* h_in, float* h_out, const uint16_t* x_in, int
 // Shapes the fused batch-1 kernel serves.
 static bool fused_ok(int T, int H, int I, int Is, int E, int k, int bias_per_row, int G) {
   if (!g_decode_fused || T != 1 || bias_per_row) return false;
-  if (H % 64 || H > DF_MAX_H || I % 64 || Is % 64 || E % 8 || E > DF_MAX_E || k > 8) return false;
-  if (k * I + Is > DF_MAX_ACT) return false;
-  if (G <= 0 || (H + G - 1) / G > DF_MAX_ROWS || E > G) return false;
-  const long need = df_staging_need(H, I, Is, k, G);
-  return need >= 0 && need <= DF_RS;
+  return df_fits(H, I, Is, E, k, G);
 }
 
-// CTAs of the fused kernel: one per SM when that many fit at once (cached).
+// CTAs of the fused kernel: one per SM when one CTA with the largest shared
+// memory the kernel may ask for fits on an SM (cached per device).
 static int fused_grid() {
   static int cached[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   if (cached[dev]) return cached[dev];
-  const size_t smem = decode_fused_smem();
   const void* fn = reinterpret_cast<const void*>(k_decode_b1);
-  if (set_smem(fn, smem)) return 0;
+  if (set_smem(fn, DF_SMEM_LIMIT)) return 0;
   int nsm = 0, per = 0;
   if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, DF_THREADS, smem) != cudaSuccess || per < 1) {
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, DF_THREADS, DF_SMEM_LIMIT) != cudaSuccess || per < 1) {
     cudaGetLastError();
     return 0;
   }
@@ -396,9 +392,9 @@ static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, con
   float* logits = reinterpret_cast<float*>(w + align_up(static_cast<size_t>(k * I + Is) * 2));
   unsigned* ctr = reinterpret_cast<unsigned*>(w + align_up(static_cast<size_t>(k * I + Is) * 2) +
                                               align_up(static_cast<size_t>(E) * 4));
-  const size_t smem = decode_fused_smem();
+  const size_t smem = decode_fused_smem(H, I, Is, E, k, G);
   int st;
-  if ((st = set_smem(reinterpret_cast<const void*>(k_decode_b1), smem))) return st;
+  if ((st = set_smem(reinterpret_cast<const void*>(k_decode_b1), DF_SMEM_LIMIT))) return st;
   for (int l0 = 0; l0 < L; l0 += DF_MAX_LAYERS) {
     const int nl = L - l0 < DF_MAX_LAYERS ? L - l0 : DF_MAX_LAYERS;
     static DfArgs args;   // large parameter block; the launch copies it
@@ -425,7 +421,7 @@ static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, con
         d.sq[m] = S.q; d.ss[m] = S.s; d.sb[m] = S.b;
       }
     }
-    if ((st = cuda_check(cudaMemsetAsync(ctr, 0, sizeof(unsigned), s), "zero barrier counter"))) return st;
+    if ((st = cuda_check(cudaMemsetAsync(ctr, 0, 256, s), "zero barrier counter and abort flag"))) return st;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(G, 1, 1);
     cfg.blockDim = dim3(DF_THREADS, 1, 1);

@@ -1,48 +1,68 @@
 // Batch-1 decode of a stack of routed-MoE layers in one persistent kernel.
 //
 // One cooperative launch runs every layer of the step, one CTA per SM (G
-// CTAs).  Work of a layer, split statically over the CTAs (CTA c):
-//   router row c (for c < E), shared-expert gate/up row pairs [c*Is/G, ...),
-//   routed gate/up (slot, row) pairs [c*k*I/G, ...) of the k*I list, and
-//   output rows [c*H/G, ...) (their k routed down rows and shared down row).
+// CTAs of 12 warps).  CTA c owns, in every layer: router row c (c < E), the
+// shared-expert gate/up pairs [c*Is/G, ...), the routed gate/up pairs
+// [c*k*I/G, ...) of the flattened (slot, row) list, and the output rows
+// [c*H/G, ...) with their k routed down rows and their shared down row.
+//
+// Dot products run on the tensor cores (mma.sync m16n8k16, fp16 operands,
+// fp32 accumulate) straight from registers.  A warp takes a tile of 16 weight
+// rows; per quantisation group (64 inputs) each lane loads two 32-bit words
+// of each of its two rows and turns every word into four half2 with LOP3:
+// (w & 0x000F000F) | 0x64006400 = (1024 + q0, 1024 + q4), the 0x00F000F0 mask
+// gives (1024 + 16 q1, 1024 + 16 q5), the same on w >> 8 nibbles 2, 6 and
+// 3, 7.  The activation comes pre-paired to match -- (v0, v4), (v1/16,
+// v5/16), (v2, v6), (v3/16, v7/16) per word -- so 4 mma give the group's
+// sum of (1024 + s q) v / s = sum q v + 1024 sum v' exactly, and the fp32
+// epilogue adds S (dot - 1024 sum v') + B sum v per row and group.  Gate/up
+// tiles give all 8 mma columns the same x; down tiles give column j the
+// activation of slot j, so one tile mixes rows of all k routed experts.
+//
 // Per layer:
-//   A  rms norm of h (every CTA, same order, same result); router logit c and
-//      the shared gate/up rows from L2 (prefetched a layer ahead) with plain
-//      loads -> logits, fp16 activations (global)
+//   A  rms norm of h (every CTA, same result) -> x and its fragments; router
+//      logit c (warp 11) and the shared gate/up pairs from shared memory
+//      staged the layer before -> logits, activations (global)
 //   grid barrier
-//   B  every CTA selects the top k from the logits, then issues every byte of
-//      its routed work at once -- gate/up row pairs and its output rows of the
-//      k down matrices, with their scale/bias windows -- as 1-D bulk copies
-//      (cp.async.bulk) into shared memory, one mbarrier per chunk, so a
-//      layer's 26.8 MB of routed weights is in flight together; warps compute
-//      each chunk as it lands -> fp16 activations
+//   B  top-k by rank over the logits (every CTA); every routed byte of the
+//      CTA -- gate/up rows (padded so fragment loads hit distinct banks), its
+//      output rows of the k down matrices, their scale/bias windows -- goes
+//      out at once as 1-D bulk copies, one mbarrier per 16-row tile; warps
+//      compute each tile as it lands; then the shared down rows are fetched
+//      into the freed area
 //   grid barrier
-//   C  the shared expert's down rows (from L2) are bulk-copied into the freed
-//      gate/up area; all activations are staged in shared memory; per output
-//      row: k routed down dots and the shared down dot, combined in a fixed
-//      order, y = sum_j g_j y_j + ysh; h += y.  The next layer's
-//      routing-independent rows (and slices of the experts with the largest
-//      router bias) are prefetched into L2 here.
+//   C  fragments of all routed and shared activations; down tiles; y = sum_j
+//      g_j y_j + ysh; h += y; the next layer's shared gate/up rows are fetched
 //   grid barrier
 // Grid barriers: named barrier, one atomic per CTA on a counter that grows
 // by G per barrier, named barrier.  Every wait is bounded (about two
 // seconds); a wait that runs out sets the device check word and the thread
 // runs on to the end.
-#include <cooperative_groups.h>
+//
+// The geometry (work split, shared-memory layout, copy lists) is plain C++
+// shared by the host, which sizes shared memory from it and checks it.
 
 namespace moe {
 
 constexpr int DF_THREADS = 384;
 constexpr int DF_WARPS = DF_THREADS / 32;
 constexpr int DF_MAX_LAYERS = 48;
-constexpr int DF_MAX_H = 3072;
-constexpr int DF_CPL = 3;                       // uint4 chunks per lane of a gate/up row (H <= 3072)
-constexpr int DF_MAX_ACT = 8192;                // k*I + Is
-constexpr int DF_MAX_ROWS = 32;                 // output rows per CTA
+constexpr int DF_MAX_H = 3072;            // one 8-element word of h per thread in the norm
 constexpr int DF_MAX_E = 256;
-constexpr int DF_RGC = 10;                      // row pairs per routed gate/up chunk
-constexpr int DF_MAX_CHUNKS = 32;               // routed chunks per CTA and layer (one per lane)
-constexpr int DF_RS = 193536;                   // shared-memory staging for a CTA's routed bytes
+constexpr int DF_MAX_RG_PAIRS = 48;       // routed gate/up pairs per CTA (6 tiles)
+constexpr int DF_MAX_SG_PAIRS = 24;       // shared gate/up pairs per CTA (3 tiles)
+constexpr int DF_MAX_ROWS = 32;           // output rows per CTA
+constexpr int DF_MAX_UNITS = 48;          // warp work units per phase
+constexpr int DF_KS = 5;                  // K parts of a shared gate/up tile (at most)
+constexpr int DF_KR = 4;                  // K parts of a routed gate/up tile (at most)
+constexpr int DF_KD = 2;                  // K parts of a routed down tile (at most)
+constexpr int DF_KSD = 3;                 // K parts of a shared down tile (at most)
+constexpr int DF_SMEM_LIMIT = 232448;     // opt-in shared memory per block
+// mbarriers: routed gate/up tiles 0..5, then
+constexpr int DF_BAR_D = 6, DF_BAR_SD = 7, DF_BAR_SG = 8, DF_BAR_RR = 9, DF_NBARS = 10;
+// copy sources besides routed slots 0..7: shared matrix m array a (q, s, b) at
+// DF_SRC_SHARED + 3m + a, router arrays (q, s, b) at DF_SRC_ROUTER + a
+constexpr int DF_SRC_SHARED = 8, DF_SRC_ROUTER = 17;
 
 struct DfLayer {
   const uint32_t* rq; const uint16_t* rs; const uint16_t* rb;   // router [E, H], 8-bit
@@ -57,14 +77,252 @@ struct DfArgs {
   size_t off[9];                    // blob offsets
   __half* act;                      // workspace: k*I + Is fp16
   float* logits;                    // workspace: [E]
-  unsigned* counter;                // workspace: grid barrier counter (zeroed before launch)
+  unsigned* counter;                // workspace: grid barrier counter; word 32: abort flag (zeroed before launch)
   uint16_t* x_trace; uint16_t* y_trace; int32_t* idx_trace; float* gates_trace;
-  int spec;                         // experts speculatively prefetched per layer
+  int spec;                         // experts speculatively prefetched into L2 per layer
   int prefetch;                     // bit 1: routing-independent rows of the next layer into L2
   unsigned long long* stamps;       // optional phase timestamps [L][G][16] (ns), or null
   DfLayer layer[DF_MAX_LAYERS];
 };
 
+// ------------------------------------------------------------------ geometry
+#ifndef __CUDACC__
+#define DF_HD
+#else
+#define DF_HD __host__ __device__
+#endif
+
+DF_HD constexpr uint32_t df_a16(uint64_t x) { return static_cast<uint32_t>((x + 15) & ~uint64_t(15)); }
+// room for a 16-byte-aligned window over n rows of `per` bytes at any start
+DF_HD constexpr uint32_t df_wres(int n, uint32_t per) { return df_a16(static_cast<uint64_t>(n) * per) + 32u; }
+
+struct DfGeom {
+  int H, I, Is, E, k, G, c;
+  int s0, nsp, r0, np, o0, nrow;    // shared pairs, routed flat pairs, output rows
+  int j0, n0, n1;                   // routed runs: first slot, pairs in it, pairs in the next slot
+  int ntS, ntR, ntD, ntSD;          // 16-row tiles per phase
+  int kS, kR, kD, kSD;              // K parts per tile (no more than the groups)
+  uint32_t rowb;                    // padded gate/up row (H/2 + 16 bytes)
+  uint32_t sbh, sbi, sbs;           // scale row bytes for K = H, I, Is
+  int npmax, nspmax, nrowmax;
+  uint32_t U, D, RR, F, M, total;   // areas: union (RG | SG | SD), routed down, router row, fragments, misc
+  uint32_t dslot;                   // bytes per routed down slot
+
+  DF_HD void init(int H_, int I_, int Is_, int E_, int k_, int G_, int c_) {
+    H = H_; I = I_; Is = Is_; E = E_; k = k_; G = G_; c = c_;
+    const long kI = static_cast<long>(k) * I;
+    s0 = static_cast<int>(static_cast<long>(c) * Is / G);
+    nsp = static_cast<int>(static_cast<long>(c + 1) * Is / G) - s0;
+    r0 = static_cast<int>(c * kI / G);
+    np = static_cast<int>((c + 1) * kI / G) - r0;
+    o0 = static_cast<int>(static_cast<long>(c) * H / G);
+    nrow = static_cast<int>(static_cast<long>(c + 1) * H / G) - o0;
+    j0 = np > 0 ? r0 / I : 0;
+    n0 = np > 0 ? ((j0 + 1) * I - r0 < np ? (j0 + 1) * I - r0 : np) : 0;
+    n1 = np - n0;
+    ntS = (nsp + 7) / 8;
+    ntR = (np + 7) / 8;
+    ntD = (k * nrow + 15) / 16;
+    ntSD = (nrow + 15) / 16;
+    kS = H / 64 < DF_KS ? H / 64 : DF_KS;
+    kR = H / 64 < DF_KR ? H / 64 : DF_KR;
+    kD = I / 64 < DF_KD ? I / 64 : DF_KD;
+    kSD = Is / 64 < DF_KSD ? Is / 64 : DF_KSD;
+    rowb = static_cast<uint32_t>(H / 2 + 16);
+    sbh = static_cast<uint32_t>(H / 64) * 2;
+    sbi = static_cast<uint32_t>(I / 64) * 2;
+    sbs = static_cast<uint32_t>(Is / 64) * 2;
+    npmax = static_cast<int>((kI + G - 1) / G);
+    nspmax = (Is + G - 1) / G;
+    nrowmax = (H + G - 1) / G;
+    // union area: the largest of the three layouts any CTA can have
+    // two runs of n0 + n1 = np pairs: wres(n0) + wres(n1) <= a16(np * sbh) + 80
+    const uint32_t rg = 2u * npmax * rowb + 4u * (df_a16(static_cast<uint64_t>(npmax) * sbh) + 80u);
+    const uint32_t sg = 2u * nspmax * rowb + 4u * df_wres(nspmax, sbh);
+    const uint32_t sd = df_a16(static_cast<uint64_t>(nrowmax) * (Is / 2)) + 2u * df_wres(nrowmax, sbs);
+    uint32_t u = rg > sg ? rg : sg;
+    u = u > sd ? u : sd;
+    U = 0;
+    dslot = df_a16(static_cast<uint64_t>(nrowmax) * (I / 2)) + 2u * df_wres(nrowmax, sbi);
+    D = (U + u + 127u) & ~127u;
+    RR = D + 8u * dslot;
+    const uint32_t rr = static_cast<uint32_t>(H) + 2u * df_wres(1, sbh);
+    F = (RR + rr + 127u) & ~127u;
+    M = (F + frag_bytes() + 127u) & ~127u;
+    total = M + misc_bytes();
+  }
+  DF_HD uint32_t frag_bytes() const {
+    const uint32_t xf = static_cast<uint32_t>(H) * 4 + static_cast<uint32_t>(H / 8) * 16 + static_cast<uint32_t>(H / 64) * 8;
+    const uint32_t af = 8u * astride() + static_cast<uint32_t>(Is / 8) * 16 + 8u * (I / 64) * 8 +
+                        static_cast<uint32_t>(Is / 64) * 8;
+    return xf > af ? xf : af;
+  }
+  DF_HD static constexpr uint32_t misc_bytes() {
+    // logits, sel / selv / selg, red, part, bars
+    return DF_MAX_E * 4 + 8 * 4 * 3 + 16 * 4 + DF_MAX_UNITS * 16 * 4 + DF_NBARS * 8;
+  }
+  // misc sub-offsets
+  DF_HD uint32_t m_lg() const { return M; }
+  DF_HD uint32_t m_sel() const { return M + DF_MAX_E * 4; }
+  DF_HD uint32_t m_selv() const { return m_sel() + 32; }
+  DF_HD uint32_t m_selg() const { return m_sel() + 64; }
+  DF_HD uint32_t m_red() const { return m_sel() + 96; }
+  DF_HD uint32_t m_part() const { return m_red() + 64; }
+  DF_HD uint32_t m_bars() const { return m_part() + DF_MAX_UNITS * 64; }
+  // fragment sub-offsets (phases A, B: x; phase C: activations)
+  DF_HD uint32_t f_xs() const { return F; }
+  DF_HD uint32_t f_xf() const { return F + static_cast<uint32_t>(H) * 4; }
+  DF_HD uint32_t f_xsum() const { return f_xf() + static_cast<uint32_t>(H / 8) * 16; }
+  DF_HD uint32_t astride() const { return static_cast<uint32_t>(I / 8 + 1) * 16; }   // padded: slots on other banks
+  DF_HD uint32_t f_af() const { return F; }
+  DF_HD uint32_t f_sf() const { return F + 8u * astride(); }
+  DF_HD uint32_t f_asum() const { return f_sf() + static_cast<uint32_t>(Is / 8) * 16; }
+  DF_HD uint32_t f_ssum() const { return f_asum() + 8u * (I / 64) * 8; }
+
+  // ---- routed gate/up: pair i (0..np-1), m = 0 gate / 1 up
+  DF_HD uint32_t rg_row(int i, int m) const { return U + (2u * i + m) * rowb; }
+  DF_HD uint32_t rg_win0() const { return U + 2u * np * rowb; }
+  // window of run `run` (0: slot j0, 1: slot j0+1), array a (0 gate.s, 1 gate.b, 2 up.s, 3 up.b)
+  DF_HD uint32_t rg_win(int run, int a) const {
+    return rg_win0() + (run ? 4u * df_wres(n0, sbh) : 0u) + a * df_wres(run ? n1 : n0, sbh);
+  }
+  DF_HD int rg_row0(int run) const { return run ? 0 : r0 - j0 * I; }   // first expert row of the run
+  // byte offset from the (16-byte aligned) blob start of the run's first scale row
+  DF_HD uint64_t rg_src(const size_t* off, int run, int a) const {
+    const int arr = a < 2 ? 1 + a : 2 + a;   // gate.s, gate.b, up.s, up.b
+    return off[arr] + static_cast<uint64_t>(rg_row0(run)) * sbh;
+  }
+  // shared-memory offset of the scale row (a = 0..3) of pair i
+  DF_HD uint32_t rg_scale(const size_t* off, int i, int a) const {
+    const int run = i < n0 ? 0 : 1;
+    const int rin = run ? i - n0 : i;
+    return rg_win(run, a) + static_cast<uint32_t>(rg_src(off, run, a) & 15) + rin * sbh;
+  }
+  // ---- routed down: slot j, row r (0..nrow-1)
+  DF_HD uint32_t d_row(int j, int r) const { return D + j * dslot + r * static_cast<uint32_t>(I / 2); }
+  DF_HD uint32_t d_win(int j, int a) const {   // a = 0 down.s, 1 down.b
+    return D + j * dslot + df_a16(static_cast<uint64_t>(nrowmax) * (I / 2)) + a * df_wres(nrowmax, sbi);
+  }
+  DF_HD uint64_t d_src(const size_t* off, int a) const { return off[7 + a] + static_cast<uint64_t>(o0) * sbi; }
+  DF_HD uint32_t d_scale(const size_t* off, int j, int r, int a) const {
+    return d_win(j, a) + static_cast<uint32_t>(d_src(off, a) & 15) + r * sbi;
+  }
+  // ---- shared gate/up: pair i (0..nsp-1); windows gate.s, gate.b, up.s, up.b
+  DF_HD uint32_t sg_row(int i, int m) const { return U + (2u * i + m) * rowb; }
+  DF_HD uint32_t sg_win(int a) const { return U + 2u * nsp * rowb + a * df_wres(nsp, sbh); }
+  DF_HD uint64_t sg_src() const { return static_cast<uint64_t>(s0) * sbh; }
+  DF_HD uint32_t sg_scale(int i, int a) const { return sg_win(a) + static_cast<uint32_t>(sg_src() & 15) + i * sbh; }
+  // ---- shared down: row r
+  DF_HD uint32_t sd_row(int r) const { return U + r * static_cast<uint32_t>(Is / 2); }
+  DF_HD uint32_t sd_win(int a) const {
+    return U + df_a16(static_cast<uint64_t>(nrowmax) * (Is / 2)) + a * df_wres(nrowmax, sbs);
+  }
+  DF_HD uint64_t sd_src() const { return static_cast<uint64_t>(o0) * sbs; }
+  DF_HD uint32_t sd_scale(int r, int a) const { return sd_win(a) + static_cast<uint32_t>(sd_src() & 15) + r * sbs; }
+  // ---- router row c
+  DF_HD uint32_t rr_win(int a) const { return RR + static_cast<uint32_t>(H) + a * df_wres(1, sbh); }
+  DF_HD uint64_t rr_src() const { return static_cast<uint64_t>(c) * sbh; }
+  DF_HD uint32_t rr_scale(int a) const { return rr_win(a) + static_cast<uint32_t>(rr_src() & 15); }
+};
+
+// One 1-D bulk copy: `bytes` from source `src` (a routed slot, or a shared /
+// router array) at byte offset `src_off` to shared-memory offset `dst`,
+// completing on mbarrier `bar`.
+struct DfCopy {
+  uint32_t dst, bytes;
+  uint64_t src_off;
+  int src, bar;
+};
+
+DF_HD inline DfCopy df_window(uint32_t dst, uint64_t first, int n, uint32_t per, int src, int bar) {
+  DfCopy C;
+  const uint64_t a = first & ~uint64_t(15), e = (first + static_cast<uint64_t>(n) * per + 15) & ~uint64_t(15);
+  C.dst = dst; C.src_off = a; C.bytes = static_cast<uint32_t>(e - a); C.src = src; C.bar = bar;
+  return C;
+}
+DF_HD inline DfCopy df_plain(uint32_t dst, uint64_t src_off, uint32_t bytes, int src, int bar) {
+  DfCopy C;
+  C.dst = dst; C.src_off = src_off; C.bytes = bytes; C.src = src; C.bar = bar;
+  return C;
+}
+
+// routed gate/up: 2*np rows (bar = tile), then 4 windows per run (bar 0)
+DF_HD inline int df_rg_count(const DfGeom& g) { return 2 * g.np + 4 * (g.n0 > 0) + 4 * (g.n1 > 0); }
+DF_HD inline DfCopy df_rg_copy(const DfGeom& g, const size_t* off, int e) {
+  if (e < 2 * g.np) {
+    const int i = e >> 1, m = e & 1;
+    const int p = g.r0 + i, slot = p / g.I, row = p % g.I;
+    return df_plain(g.rg_row(i, m), off[3 * m] + static_cast<uint64_t>(row) * (g.H / 2),
+                    static_cast<uint32_t>(g.H / 2), slot, i / 8);
+  }
+  e -= 2 * g.np;
+  const int run = e / 4, a = e % 4;
+  return df_window(g.rg_win(run, a), g.rg_src(off, run, a), run ? g.n1 : g.n0, g.sbh, g.j0 + run, 0);
+}
+// routed down: per slot the nrow rows, then the two windows
+DF_HD inline int df_d_count(const DfGeom& g) { return g.nrow > 0 ? 3 * g.k : 0; }
+DF_HD inline DfCopy df_d_copy(const DfGeom& g, const size_t* off, int e) {
+  const int j = e / 3, part = e % 3;
+  if (part == 0)
+    return df_plain(g.d_row(j, 0), off[6] + static_cast<uint64_t>(g.o0) * (g.I / 2),
+                    static_cast<uint32_t>(g.nrow) * (g.I / 2), j, DF_BAR_D);
+  return df_window(g.d_win(j, part - 1), g.d_src(off, part - 1), g.nrow, g.sbi, j, DF_BAR_D);
+}
+// shared down (matrix 2): rows, S window, B window
+DF_HD inline int df_sd_count(const DfGeom& g) { return g.nrow > 0 ? 3 : 0; }
+DF_HD inline DfCopy df_sd_copy(const DfGeom& g, int e) {
+  if (e == 0)
+    return df_plain(g.sd_row(0), static_cast<uint64_t>(g.o0) * (g.Is / 2), static_cast<uint32_t>(g.nrow) * (g.Is / 2),
+                    DF_SRC_SHARED + 6, DF_BAR_SD);
+  return df_window(g.sd_win(e - 1), g.sd_src(), g.nrow, g.sbs, DF_SRC_SHARED + 6 + e, DF_BAR_SD);
+}
+// shared gate/up (matrices 0, 1): 2*nsp rows, then gate.s, gate.b, up.s, up.b
+DF_HD inline int df_sg_count(const DfGeom& g) { return g.nsp > 0 ? 2 * g.nsp + 4 : 0; }
+DF_HD inline DfCopy df_sg_copy(const DfGeom& g, int e) {
+  if (e < 2 * g.nsp) {
+    const int i = e >> 1, m = e & 1;
+    return df_plain(g.sg_row(i, m), static_cast<uint64_t>(g.s0 + i) * (g.H / 2), static_cast<uint32_t>(g.H / 2),
+                    DF_SRC_SHARED + 3 * m, DF_BAR_SG);
+  }
+  e -= 2 * g.nsp;
+  const int m = e / 2, a = e % 2;
+  return df_window(g.sg_win(e), g.sg_src(), g.nsp, g.sbh, DF_SRC_SHARED + 3 * m + 1 + a, DF_BAR_SG);
+}
+// router row c: the row, S window, B window
+DF_HD inline int df_rr_count(const DfGeom& g) { return g.c < g.E ? 3 : 0; }
+DF_HD inline DfCopy df_rr_copy(const DfGeom& g, int e) {
+  if (e == 0)
+    return df_plain(g.RR, static_cast<uint64_t>(g.c) * g.H, static_cast<uint32_t>(g.H), DF_SRC_ROUTER, DF_BAR_RR);
+  return df_window(g.rr_win(e - 1), g.rr_src(), 1, g.sbh, DF_SRC_ROUTER + e, DF_BAR_RR);
+}
+
+// Group range [g0, g1) of K part p of `parts` over ng groups.
+DF_HD inline void df_kpart(int ng, int parts, int p, int& g0, int& g1) {
+  g0 = ng * p / parts;
+  g1 = ng * (p + 1) / parts;
+}
+
+// Shared-memory bytes of the kernel for these dims and grid (the layout is
+// the same for every CTA).
+inline size_t decode_fused_smem(int H, int I, int Is, int E, int k, int G) {
+  DfGeom g;
+  g.init(H, I, Is, E, k, G, 0);
+  return g.total;
+}
+
+// Whether every CTA's work fits the kernel's fixed limits.
+inline bool df_fits(int H, int I, int Is, int E, int k, int G) {
+  if (G <= 0 || H % 64 || I % 64 || Is % 64 || H > DF_MAX_H || E > DF_MAX_E || E > G || k > 8) return false;
+  DfGeom g;
+  g.init(H, I, Is, E, k, G, 0);
+  if (g.npmax > DF_MAX_RG_PAIRS || g.npmax > I || g.nspmax > DF_MAX_SG_PAIRS || g.nrowmax > DF_MAX_ROWS) return false;
+  const int tiles_d = (k * g.nrowmax + 15) / 16, tiles_sd = (g.nrowmax + 15) / 16;
+  if (((g.npmax + 7) / 8) * g.kR > DF_MAX_UNITS || ((g.nspmax + 7) / 8) * g.kS > DF_MAX_UNITS) return false;
+  if (tiles_d * g.kD + tiles_sd * g.kSD > DF_MAX_UNITS) return false;
+  return g.total <= static_cast<uint32_t>(DF_SMEM_LIMIT);
+}
+
+#ifdef __CUDACC__
 // ------------------------------------------------------------------ PTX bits
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   unsigned v;
@@ -88,45 +346,17 @@ __device__ __forceinline__ void df_mbar_init(uint32_t bar, uint32_t count) {
 __device__ __forceinline__ void df_mbar_arrive(uint32_t bar) {
   asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ void df_mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
-               "r"(bytes)
-               : "memory");
-}
-// arrive on the mbarrier at the same shared-memory offset in CTA `rank` of the cluster
-__device__ __forceinline__ void df_mbar_arrive_remote(uint32_t bar, uint32_t rank) {
-  asm volatile(
-      "{\n\t.reg .b32 ra;\n\tmapa.shared::cluster.u32 ra, %0, %1;\n\t"
-      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(bar),
-      "r"(rank)
-      : "memory");
-}
-__device__ __forceinline__ void df_st_remote_f32(uint32_t addr, uint32_t rank, float v) {
-  asm volatile(
-      "{\n\t.reg .b32 ra;\n\tmapa.shared::cluster.u32 ra, %0, %1;\n\tst.shared::cluster.f32 [ra], %2;\n\t}" ::"r"(
-          addr),
-      "r"(rank), "f"(v)
-      : "memory");
-}
-// bounded wait on a phase parity; `cluster` acquires at cluster scope
-__device__ __forceinline__ bool df_mbar_wait(uint32_t bar, uint32_t parity, bool cluster = false) {
+// bounded wait on a phase parity
+__device__ __forceinline__ bool df_mbar_wait(uint32_t bar, uint32_t parity) {
   uint64_t t0 = 0;
   for (uint32_t i = 0;; ++i) {
     uint32_t ok;
-    if (cluster)
-      asm volatile(
-          "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-          "selp.u32 %0, 1, 0, p;\n\t}"
-          : "=r"(ok)
-          : "r"(bar), "r"(parity)
-          : "memory");
-    else
-      asm volatile(
-          "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-          "selp.u32 %0, 1, 0, p;\n\t}"
-          : "=r"(ok)
-          : "r"(bar), "r"(parity)
-          : "memory");
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
     if (ok) return true;
     if ((i & 255u) == 0) {
       const uint64_t now = df_clock();
@@ -137,7 +367,9 @@ __device__ __forceinline__ bool df_mbar_wait(uint32_t bar, uint32_t parity, bool
   flag_check(CHECK_WAIT);
   return false;
 }
-__device__ __forceinline__ void df_bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+// raise the barrier's expected bytes, then copy (the copy completes them)
+__device__ __forceinline__ void df_bulk(uint32_t bar, uint32_t dst, const void* src, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                "l"(src), "r"(bytes), "r"(bar)
                : "memory");
@@ -155,156 +387,85 @@ __device__ __forceinline__ void prefetch_l2(const void* p, size_t bytes) {
     a += n;
   }
 }
-__device__ __forceinline__ void prefetch_slice(const void* base, size_t total, int c, int G) {
-  const size_t b0 = total * c / G, b1 = total * (c + 1) / G;
-  prefetch_l2(static_cast<const uint8_t*>(base) + b0, b1 - b0);
-}
 __device__ __forceinline__ uint4 ldcg_v4(const void* p) {
   uint4 r;
   asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
 }
 
-// phase timestamps (when requested): layer l, CTA c, phase p
+// phase timestamps (when requested): layer l, CTA c, point p
 __device__ __forceinline__ void df_stamp(const DfArgs& a, int l, int p) {
   if (a.stamps != nullptr && threadIdx.x == 0)
     a.stamps[(static_cast<size_t>(l) * gridDim.x + blockIdx.x) * 16 + p] = df_clock();
 }
 
+// ------------------------------------------------------------ tensor-core dot
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t nib_lo(uint32_t w) { return (w & 0x000F000Fu) | 0x64006400u; }
+__device__ __forceinline__ uint32_t nib_hi(uint32_t w) { return (w & 0x00F000F0u) | 0x64006400u; }
 
-__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
-
-// 16-byte-aligned window covering rows [r0, r0+n) of a bf16 array with `per`
-// values per row; skew = offset of row r0 inside the window.
-__device__ __forceinline__ void sb_window(const uint16_t* base, int per, int r0, int n, const uint8_t*& src,
-                                          uint32_t& bytes, uint32_t& skew) {
-  const uintptr_t a = reinterpret_cast<uintptr_t>(base) + static_cast<size_t>(r0) * per * 2;
-  const uintptr_t e = a + static_cast<size_t>(n) * per * 2;
-  const uintptr_t a16 = a & ~uintptr_t(15), e16 = (e + 15) & ~uintptr_t(15);
-  src = reinterpret_cast<const uint8_t*>(a16);
-  bytes = static_cast<uint32_t>(e16 - a16);
-  skew = static_cast<uint32_t>(a - a16);
+// One group (64 inputs) of tile rows g (words wa) and g+8 (words wb): lane
+// (g, t) holds words 2t, 2t+1 of the group; f0, f1 are the paired activation
+// of those words in this lane's column.  Fragment rows: a0/a2 row g, a1/a3
+// row g+8; a0/a1 pair with b0, a2/a3 with b1.
+__device__ __forceinline__ void mma_group(float (&d)[4], uint2 wa, uint2 wb, uint4 f0, uint4 f1) {
+  d[0] = d[1] = d[2] = d[3] = 0.f;
+  mma16816(d, nib_lo(wa.x), nib_lo(wb.x), nib_hi(wa.x), nib_hi(wb.x), f0.x, f0.y);
+  const uint32_t ax = wa.x >> 8, bx = wb.x >> 8;
+  mma16816(d, nib_lo(ax), nib_lo(bx), nib_hi(ax), nib_hi(bx), f0.z, f0.w);
+  mma16816(d, nib_lo(wa.y), nib_lo(wb.y), nib_hi(wa.y), nib_hi(wb.y), f1.x, f1.y);
+  const uint32_t ay = wa.y >> 8, by = wb.y >> 8;
+  mma16816(d, nib_lo(ay), nib_lo(by), nib_hi(ay), nib_hi(by), f1.z, f1.w);
 }
 
-enum : int { CH_RG = 0, CH_D = 1, CH_DS = 2, CH_SG = 3, CH_R = 4 };
-
-// One chunk of staged bytes: weight runs (run i at i * qbytes from the chunk
-// start), then scale/bias windows; sk[i] = offset of window i's first row
-// from the chunk start.
-struct DfChunk {
-  const uint8_t* src[6];
-  uint32_t dst[6];
-  uint32_t len[6];
-  int n;
-  uint32_t qbytes, bytes, off;      // off: chunk start inside the staging area
-  uint32_t sk[4];
-  int kind, slot, r0, rows;
-};
-
-__device__ inline DfChunk df_chunk(int kind, int slot, int r0, int rows, int H, int I, int Is, const DfArgs& a,
-                                   const DfLayer& W, const int* sel) {
-  DfChunk C{};
-  C.kind = kind; C.slot = slot; C.r0 = r0; C.rows = rows;
-  const uint8_t* q[2] = {nullptr, nullptr};
-  const uint16_t* sc[4] = {nullptr, nullptr, nullptr, nullptr};
-  int per = 0, nq = 0, ns = 0;
-  if (kind == CH_RG) {
-    const uint8_t* blob = static_cast<const uint8_t*>(W.blobs[sel[slot]]);
-    q[0] = blob + a.off[0] + static_cast<size_t>(r0) * (H / 2);
-    q[1] = blob + a.off[3] + static_cast<size_t>(r0) * (H / 2);
-    C.qbytes = static_cast<uint32_t>(rows) * (H / 2); nq = 2;
-    sc[0] = reinterpret_cast<const uint16_t*>(blob + a.off[1]); sc[1] = reinterpret_cast<const uint16_t*>(blob + a.off[2]);
-    sc[2] = reinterpret_cast<const uint16_t*>(blob + a.off[4]); sc[3] = reinterpret_cast<const uint16_t*>(blob + a.off[5]);
-    ns = 4; per = H / 64;
-  } else if (kind == CH_D) {
-    const uint8_t* blob = static_cast<const uint8_t*>(W.blobs[sel[slot]]);
-    q[0] = blob + a.off[6] + static_cast<size_t>(r0) * (I / 2);
-    C.qbytes = static_cast<uint32_t>(rows) * (I / 2); nq = 1;
-    sc[0] = reinterpret_cast<const uint16_t*>(blob + a.off[7]); sc[1] = reinterpret_cast<const uint16_t*>(blob + a.off[8]);
-    ns = 2; per = I / 64;
-  } else if (kind == CH_DS) {
-    q[0] = reinterpret_cast<const uint8_t*>(W.sq[2]) + static_cast<size_t>(r0) * (Is / 2);
-    C.qbytes = static_cast<uint32_t>(rows) * (Is / 2); nq = 1;
-    sc[0] = W.ss[2]; sc[1] = W.sb[2]; ns = 2; per = Is / 64;
-  } else if (kind == CH_SG) {
-    q[0] = reinterpret_cast<const uint8_t*>(W.sq[0]) + static_cast<size_t>(r0) * (H / 2);
-    q[1] = reinterpret_cast<const uint8_t*>(W.sq[1]) + static_cast<size_t>(r0) * (H / 2);
-    C.qbytes = static_cast<uint32_t>(rows) * (H / 2); nq = 2;
-    sc[0] = W.ss[0]; sc[1] = W.sb[0]; sc[2] = W.ss[1]; sc[3] = W.sb[1]; ns = 4; per = H / 64;
-  } else {   // CH_R: router rows (8-bit, H bytes each)
-    q[0] = reinterpret_cast<const uint8_t*>(W.rq) + static_cast<size_t>(r0) * H;
-    C.qbytes = static_cast<uint32_t>(rows) * H; nq = 1;
-    sc[0] = W.rs; sc[1] = W.rb; ns = 2; per = H / 64;
+// Groups [g0, g1) of this lane's two tile rows: acc += S (dot - sum.x) + B sum.y
+// per group.  qa/qb: the rows' bytes at this lane's offset 8t; sa/ba, sb/bb:
+// their bf16 scale and bias rows; f: this lane's column of paired activation
+// (uint4 per word, 8 words per group) at word 2t; suma/sumb: per group
+// (1024 * sum of paired halves, sum of values) of each row's column; ca/cb:
+// which accumulator of the pair holds the row's column (down tiles).
+template <bool COLS>
+__device__ __forceinline__ void df_rows(const uint8_t* qa, const uint8_t* qb, const uint16_t* sa, const uint16_t* ba,
+                                        const uint16_t* sb, const uint16_t* bb, const uint4* f, const float2* suma,
+                                        const float2* sumb, int ca, int cb, int g0, int g1, float& acc_a,
+                                        float& acc_b) {
+#pragma unroll 2
+  for (int gr = g0; gr < g1; ++gr) {
+    const uint2 wa = *reinterpret_cast<const uint2*>(qa + 32 * gr);
+    const uint2 wb = *reinterpret_cast<const uint2*>(qb + 32 * gr);
+    const uint4 f0 = f[8 * gr], f1 = f[8 * gr + 1];
+    float d[4];
+    mma_group(d, wa, wb, f0, f1);
+    const float2 xa = suma[gr], xb = sumb[gr];
+    const float va = COLS ? (ca ? d[1] : d[0]) : d[0];
+    const float vb = COLS ? (cb ? d[3] : d[2]) : d[2];
+    acc_a += bf16_to_f32(sa[gr]) * (va - xa.x) + bf16_to_f32(ba[gr]) * xa.y;
+    acc_b += bf16_to_f32(sb[gr]) * (vb - xb.x) + bf16_to_f32(bb[gr]) * xb.y;
   }
-  uint32_t o = 0;
-  for (int i = 0; i < nq; ++i) {
-    C.src[C.n] = q[i]; C.dst[C.n] = o; C.len[C.n] = C.qbytes; ++C.n;
-    o += C.qbytes;
-  }
-  for (int i = 0; i < ns; ++i) {
-    const uint8_t* src; uint32_t bytes, skew;
-    sb_window(sc[i], per, r0, rows, src, bytes, skew);
-    C.src[C.n] = src; C.dst[C.n] = o; C.len[C.n] = bytes; ++C.n;
-    C.sk[i] = o + skew;
-    o += bytes;
-  }
-  C.bytes = o;
-  return C;
 }
 
-// Number of routed gate/up chunks of the flattened pair range [r0, r1).
-__device__ inline int df_rg_chunks(int r0, int r1, int I) {
-  if (r1 <= r0) return 0;
-  int n = 0;
-  for (int j = r0 / I; j <= (r1 - 1) / I; ++j) n += ceil_div(min(r1, (j + 1) * I) - max(r0, j * I), DF_RGC);
-  return n;
+// Pair 8 consecutive values into the mma activation word and return its
+// (sum of the stored halves, sum of the values).
+__device__ __forceinline__ uint4 df_pair8(const float v[8], float& off, float& sum) {
+  uint32_t p[4];
+  pair_word4(v, p);
+  const float2 f0 = unpack_half2(p[0]), f1 = unpack_half2(p[1]), f2 = unpack_half2(p[2]), f3 = unpack_half2(p[3]);
+  off = (f0.x + f0.y) + (f1.x + f1.y) + (f2.x + f2.y) + (f3.x + f3.y);
+  sum = (f0.x + f0.y + f2.x + f2.y) + 16.f * (f1.x + f1.y + f3.x + f3.y);
+  return make_uint4(p[0], p[1], p[2], p[3]);
 }
-// Chunk t of them: slot, first row, rows.
-__device__ inline void df_rg_chunk_at(int r0, int r1, int I, int t, int& slot, int& row, int& rows) {
-  for (int j = r0 / I; j <= (r1 - 1) / I; ++j) {
-    const int a = max(r0, j * I), b = min(r1, (j + 1) * I);
-    const int nj = ceil_div(b - a, DF_RGC);
-    if (t < nj) { slot = j; row = a - j * I + t * DF_RGC; rows = min(DF_RGC, b - a - t * DF_RGC); return; }
-    t -= nj;
-  }
-  slot = 0; row = 0; rows = 0;
-}
-
-// One gate/up row pair (rows of K = H nibbles each) against the register x:
-// returns (gate . x, up . x) in every lane.  Weight rows and scale rows may be
-// in shared or global memory.
-__device__ __forceinline__ float2 df_pair(const uint8_t* gq, const uint8_t* uq, const uint16_t* gs,
-                                          const uint16_t* gb, const uint16_t* us, const uint16_t* ub, int nch,
-                                          const uint32_t (&xp)[DF_CPL][16], const float2 (&xst)[DF_CPL],
-                                          bool global) {
-  const int lane = threadIdx.x & 31;
-  uint4 qg[DF_CPL], qu[DF_CPL];
-  float sg[DF_CPL], bg[DF_CPL], su[DF_CPL], bu[DF_CPL];
-#pragma unroll
-  for (int j = 0; j < DF_CPL; ++j) {
-    const int cc = lane + 32 * j;
-    if (cc < nch) {
-      if (global) {
-        qg[j] = ldg_nc_v4(gq + 16 * cc); qu[j] = ldg_nc_v4(uq + 16 * cc);
-        sg[j] = bf16_to_f32(ldg_u16(gs + (cc >> 1))); bg[j] = bf16_to_f32(ldg_u16(gb + (cc >> 1)));
-        su[j] = bf16_to_f32(ldg_u16(us + (cc >> 1))); bu[j] = bf16_to_f32(ldg_u16(ub + (cc >> 1)));
-      } else {
-        qg[j] = *reinterpret_cast<const uint4*>(gq + 16 * cc); qu[j] = *reinterpret_cast<const uint4*>(uq + 16 * cc);
-        sg[j] = bf16_to_f32(gs[cc >> 1]); bg[j] = bf16_to_f32(gb[cc >> 1]);
-        su[j] = bf16_to_f32(us[cc >> 1]); bu[j] = bf16_to_f32(ub[cc >> 1]);
-      }
-    }
-  }
-  float ga = 0.f, ua = 0.f;
-#pragma unroll
-  for (int j = 0; j < DF_CPL; ++j) {
-    const int cc = lane + 32 * j;
-    if (cc < nch) {
-      ga += sg[j] * (dot_chunk4(qg[j], xp[j]) - xst[j].x) + bg[j] * xst[j].y;
-      ua += su[j] * (dot_chunk4(qu[j], xp[j]) - xst[j].x) + bu[j] * xst[j].y;
-    }
-  }
-  return make_float2(warp_sum(ga), warp_sum(ua));
+// sum over the 8 lanes of an aligned lane octet
+__device__ __forceinline__ float oct_sum(float v) {
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  v += __shfl_xor_sync(0xffffffffu, v, 2);
+  v += __shfl_xor_sync(0xffffffffu, v, 4);
+  return v;
 }
 
 // --------------------------------------------------------------- the kernel
@@ -312,40 +473,34 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
   extern __shared__ __align__(16) unsigned char smem[];
   const int H = a.H, I = a.I, Is = a.Is, E = a.E, k = a.k;
   const int G = gridDim.x, c = blockIdx.x;
-  const int kI = k * I, nact = kI + Is;
-  const int s0 = (int)((long)c * Is / G), s1 = (int)((long)(c + 1) * Is / G);
-  const int r0 = (int)((long)c * kI / G), r1 = (int)((long)(c + 1) * kI / G);
-  const int o0 = (int)((long)c * H / G), o1 = (int)((long)(c + 1) * H / G);
-  const int nrow = o1 - o0;
-  const int nrg = df_rg_chunks(r0, r1, I);
-  const int nchunk = nrg + k;                  // routed chunks: gate/up pieces, then one down chunk per slot
+  const int kI = k * I;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nch = H / 32;
+  const int gq = lane >> 2, tq = lane & 3;        // mma fragment row and thread in the row's quad
+  DfGeom g;
+  g.init(H, I, Is, E, k, G, c);
+  const int NGH = H / 64, NGI = I / 64, NGS = Is / 64;
 
-  // shared memory
-  unsigned char* rs = smem;                                            // [DF_RS] routed staging
-  unsigned char* ax = rs + DF_RS;                                      // union: x (phase A) / activations (C)
-  float* xs = reinterpret_cast<float*>(ax);                            // [H]
-  uint4* actP = reinterpret_cast<uint4*>(ax);                          // [nact/8]
-  float2* actS = reinterpret_cast<float2*>(actP + DF_MAX_ACT / 8);     // [nact/8]
-  uint4* xP4 = reinterpret_cast<uint4*>(ax + (DF_MAX_ACT / 8) * 24);   // [4][nch]
-  float2* xS4 = reinterpret_cast<float2*>(xP4 + DF_MAX_H / 8);         // [nch]
-  float* part = reinterpret_cast<float*>(xS4 + DF_MAX_H / 32);         // [MAX_ROWS][9]
-  float* red = part + DF_MAX_ROWS * 9;                                 // [32]
-  int* sel = reinterpret_cast<int*>(red + 32);                         // [8]
-  float* selg = reinterpret_cast<float*>(sel + 8);                     // [8]
-  DfChunk* tab = reinterpret_cast<DfChunk*>(selg + 8);                 // [DF_MAX_CHUNKS + 3]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(tab + DF_MAX_CHUNKS + 3);   // [DF_MAX_CHUNKS + 3]
-  const int IDX_DS = DF_MAX_CHUNKS, IDX_SG = DF_MAX_CHUNKS + 1, IDX_R = DF_MAX_CHUNKS + 2;
-  const uint32_t bar0 = smem_addr(bars);
+  float* lg = reinterpret_cast<float*>(smem + g.m_lg());
+  int* sel = reinterpret_cast<int*>(smem + g.m_sel());
+  float* selv = reinterpret_cast<float*>(smem + g.m_selv());
+  float* selg = reinterpret_cast<float*>(smem + g.m_selg());
+  float* red = reinterpret_cast<float*>(smem + g.m_red());
+  float* part = reinterpret_cast<float*>(smem + g.m_part());
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t bar0 = sbase + g.m_bars();
+  float* xs = reinterpret_cast<float*>(smem + g.f_xs());
+  uint4* xf = reinterpret_cast<uint4*>(smem + g.f_xf());
+  float2* xsum = reinterpret_cast<float2*>(smem + g.f_xsum());
+  uint4* af = reinterpret_cast<uint4*>(smem + g.f_af());
+  uint4* sf = reinterpret_cast<uint4*>(smem + g.f_sf());
+  float2* asum = reinterpret_cast<float2*>(smem + g.f_asum());
+  float2* ssum = reinterpret_cast<float2*>(smem + g.f_ssum());
+  const int astride4 = static_cast<int>(g.astride() / 16);     // uint4 per slot of paired activation
+  const uint16_t* S16 = reinterpret_cast<const uint16_t*>(smem);
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < DF_MAX_CHUNKS + 3; ++i) df_mbar_init(bar0 + 8u * i, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncthreads();
-
+  unsigned* abort_word = a.counter + 32;          // own 128-byte line
   unsigned bar_target = 0;
+  auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
   auto grid_sync = [&]() {
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -360,27 +515,279 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
     }
     __syncthreads();
   };
-  // routing-independent rows of layer l (and likely experts) into L2
-  auto prefetch_layer = [&](int l) {
-    const DfLayer& V = a.layer[l];
-    if (threadIdx.x == 0 && (a.prefetch & 2)) {
-      for (int e = c; e < E; e += G) {
-        prefetch_l2(reinterpret_cast<const uint8_t*>(V.rq) + static_cast<size_t>(e) * H, H);
-        prefetch_l2(V.rs + static_cast<size_t>(e) * (H / 64), (H / 64) * 2);
-        prefetch_l2(V.rb + static_cast<size_t>(e) * (H / 64), (H / 64) * 2);
-      }
-      for (int m = 0; m < 2; ++m) {
-        prefetch_l2(reinterpret_cast<const uint8_t*>(V.sq[m]) + static_cast<size_t>(s0) * (H / 2),
-                    static_cast<size_t>(s1 - s0) * (H / 2));
-        prefetch_l2(V.ss[m] + static_cast<size_t>(s0) * (H / 64), static_cast<size_t>(s1 - s0) * (H / 64) * 2);
-        prefetch_l2(V.sb[m] + static_cast<size_t>(s0) * (H / 64), static_cast<size_t>(s1 - s0) * (H / 64) * 2);
-      }
-      prefetch_l2(reinterpret_cast<const uint8_t*>(V.sq[2]) + static_cast<size_t>(o0) * (Is / 2),
-                  static_cast<size_t>(nrow) * (Is / 2));
-      prefetch_l2(V.ss[2] + static_cast<size_t>(o0) * (Is / 64), static_cast<size_t>(nrow) * (Is / 64) * 2);
-      prefetch_l2(V.sb[2] + static_cast<size_t>(o0) * (Is / 64), static_cast<size_t>(nrow) * (Is / 64) * 2);
+  // source address of a copy in layer W (routed slots through the selection)
+  auto src_ptr = [&](const DfLayer& W, const DfCopy& C) -> const uint8_t* {
+    const uint8_t* b;
+    if (C.src < 8) {
+      int e = sel[C.src];
+      if (e < 0 || e >= E) { flag_check(CHECK_EXPERT_ID); e = 0; }
+      b = static_cast<const uint8_t*>(W.blobs[e]);
+    } else if (C.src < DF_SRC_ROUTER) {
+      const int m = (C.src - DF_SRC_SHARED) / 3, arr = (C.src - DF_SRC_SHARED) % 3;
+      b = arr == 0 ? reinterpret_cast<const uint8_t*>(W.sq[m])
+                   : reinterpret_cast<const uint8_t*>(arr == 1 ? W.ss[m] : W.sb[m]);
+    } else {
+      const int arr = C.src - DF_SRC_ROUTER;
+      b = arr == 0 ? reinterpret_cast<const uint8_t*>(W.rq)
+                   : reinterpret_cast<const uint8_t*>(arr == 1 ? W.rs : W.rb);
     }
-    if (warp == 1 && a.spec > 0 && V.bias != nullptr) {
+    return b + C.src_off;
+  };
+  // warp-wide issue of the shared gate/up and router-row copies of layer W
+  auto issue_sg = [&](const DfLayer& W) {
+    const int n = df_sg_count(g);
+    for (int e = lane; e < n; e += 32) {
+      const DfCopy C = df_sg_copy(g, e);
+      df_bulk(BAR(C.bar), sbase + C.dst, src_ptr(W, C), C.bytes);
+    }
+    __syncwarp();
+    if (lane == 0) df_mbar_arrive(BAR(DF_BAR_SG));
+    __syncwarp();
+  };
+  auto issue_rr = [&](const DfLayer& W) {
+    const int n = df_rr_count(g);
+    for (int e = lane; e < n; e += 32) {
+      const DfCopy C = df_rr_copy(g, e);
+      df_bulk(BAR(C.bar), sbase + C.dst, src_ptr(W, C), C.bytes);
+    }
+    __syncwarp();
+    if (lane == 0) df_mbar_arrive(BAR(DF_BAR_RR));
+    __syncwarp();
+  };
+
+  // --------------------------------------------------------------- set-up
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < DF_NBARS; ++i) df_mbar_init(BAR(i), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // every blob pointer is checked (non-null, 16-byte aligned) before any copy
+  // reads one; a bad one stops every CTA at the same point
+  {
+    const long n = static_cast<long>(a.L) * E;
+    for (long i = static_cast<long>(c) * DF_THREADS + threadIdx.x; i < n; i += static_cast<long>(G) * DF_THREADS) {
+      const uintptr_t p = reinterpret_cast<uintptr_t>(a.layer[i / E].blobs[i % E]);
+      if (p == 0 || (p & 15)) { flag_check(CHECK_EXPERT_ID); atomicOr(abort_word, 1u); }
+    }
+  }
+  grid_sync();
+  if (__ldcg(abort_word) != 0u) return;
+  if (warp == 0) {
+    issue_sg(a.layer[0]);
+    issue_rr(a.layer[0]);
+  }
+
+  for (int l = 0; l < a.L; ++l) {
+    const DfLayer& W = a.layer[l];
+    const uint32_t par = l & 1;
+    df_stamp(a, l, 0);
+    // ------------------------------------------------------ A0: rms norm
+    {
+      const int u = threadIdx.x;            // word u of h: elements 8u .. 8u+7
+      float v[8];
+      float ss = 0.f;
+      if (u < H / 8) {
+        const uint4 p0 = ldcg_v4(a.h + 8 * u), p1 = ldcg_v4(a.h + 8 * u + 4);
+        v[0] = __uint_as_float(p0.x); v[1] = __uint_as_float(p0.y); v[2] = __uint_as_float(p0.z);
+        v[3] = __uint_as_float(p0.w); v[4] = __uint_as_float(p1.x); v[5] = __uint_as_float(p1.y);
+        v[6] = __uint_as_float(p1.z); v[7] = __uint_as_float(p1.w);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) ss = fmaf(v[t], v[t], ss);
+      } else {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) v[t] = 0.f;
+      }
+      ss = warp_sum(ss);
+      if (lane == 0) red[warp] = ss;
+      if (threadIdx.x < 8) sel[threadIdx.x] = -1;
+      __syncthreads();
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < DF_WARPS; ++w) tot += red[w];
+      const float rr = sqrtf(tot / static_cast<float>(H) + 1e-6f);
+      float off = 0.f, sum = 0.f;
+      if (u < H / 8) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const uint16_t b = f32_to_bf16(__fdiv_rn(v[t], rr));
+          v[t] = bf16_to_f32(b);
+          xs[8 * u + t] = v[t];
+          if (c == 0 && a.x_trace) a.x_trace[static_cast<size_t>(l) * H + 8 * u + t] = b;
+        }
+        xf[u] = df_pair8(v, off, sum);
+      }
+      off = oct_sum(off);
+      sum = oct_sum(sum);
+      if (u < H / 8 && (lane & 7) == 0) xsum[u >> 3] = make_float2(1024.f * off, sum);
+      __syncthreads();
+    }
+    df_stamp(a, l, 1);
+
+    // --------------------------- router logit c, shared gate/up pairs
+    if (warp == DF_WARPS - 1) {
+      if (c < E) {
+        df_mbar_wait(BAR(DF_BAR_RR), par);
+        const uint8_t* qrow = smem + g.RR;
+        const uint16_t* S = S16 + g.rr_scale(0) / 2;
+        const uint16_t* B = S16 + g.rr_scale(1) / 2;
+        float acc = 0.f;
+        for (int cc = lane; cc < H / 16; cc += 32) {
+          const uint4 q4 = *reinterpret_cast<const uint4*>(qrow + 16 * cc);
+          const float sc = bf16_to_f32(S[cc >> 2]), bi = bf16_to_f32(B[cc >> 2]);
+          const float* xv = xs + 16 * cc;
+          const uint32_t w[4] = {q4.x, q4.y, q4.z, q4.w};
+          float a0 = 0.f, a1 = 0.f, sm = 0.f;
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const uint32_t p[2] = {pack_half2(xv[4 * m], xv[4 * m + 2]), pack_half2(xv[4 * m + 1], xv[4 * m + 3])};
+            dot_word8(w[m], p, a0, a1);
+            const float2 f0 = unpack_half2(p[0]), f1 = unpack_half2(p[1]);
+            sm += (f0.x + f0.y) + (f1.x + f1.y);
+          }
+          acc += sc * ((a0 + a1) - 1024.f * sm) + bi * sm;
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) a.logits[c] = acc + (W.bias ? W.bias[c] : 0.f);
+      }
+    } else {
+      const int nunits = g.ntS * g.kS;
+      if (nunits > 0) df_mbar_wait(BAR(DF_BAR_SG), par);
+      for (int u = warp; u < nunits; u += DF_WARPS - 1) {
+        const int tile = u / g.kS;
+        int g0, g1;
+        df_kpart(NGH, g.kS, u % g.kS, g0, g1);
+        int i = 8 * tile + gq;
+        if (i >= g.nsp) i = 8 * tile;
+        float acc_a = 0.f, acc_b = 0.f;
+        df_rows<false>(smem + g.sg_row(i, 0) + 8 * tq, smem + g.sg_row(i, 1) + 8 * tq, S16 + g.sg_scale(i, 0) / 2,
+                       S16 + g.sg_scale(i, 1) / 2, S16 + g.sg_scale(i, 2) / 2, S16 + g.sg_scale(i, 3) / 2,
+                       xf + 2 * tq, xsum, xsum, 0, 0, g0, g1, acc_a, acc_b);
+        if (tq == 0) {
+          part[u * 16 + gq] = acc_a;
+          part[u * 16 + 8 + gq] = acc_b;
+        }
+      }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < g.nsp; i += DF_THREADS) {
+      const int tile = i / 8, r = i % 8;
+      float gs = 0.f, us = 0.f;
+      for (int p = 0; p < g.kS; ++p) {
+        gs += part[(tile * g.kS + p) * 16 + r];
+        us += part[(tile * g.kS + p) * 16 + 8 + r];
+      }
+      a.act[kI + g.s0 + i] = __float2half_rn(gelu_tanh(gs) * us);
+    }
+    df_stamp(a, l, 2);
+    grid_sync();
+    df_stamp(a, l, 3);
+
+    // ------------------------------------------------ top-k, routed bytes
+    for (int e = threadIdx.x; e < E; e += DF_THREADS) lg[e] = __ldcg(a.logits + e);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += DF_THREADS) {
+      const float v = lg[e];
+      int rank = 0;
+      for (int f = 0; f < E; ++f) {
+        const float w = lg[f];
+        rank += (w > v || (w == v && f < e)) ? 1 : 0;
+      }
+      if (rank < k) { sel[rank] = e; selv[rank] = v; }
+    }
+    __syncthreads();
+    df_stamp(a, l, 4);
+    if (warp == 0) {
+      if (lane < k) {
+        float den = 0.f;
+        for (int j = 0; j < k; ++j) den += expf(selv[j] - selv[0]);
+        const float gj = expf(selv[lane] - selv[0]) / den;
+        selg[lane] = gj;
+        if (c == 0 && a.idx_trace) a.idx_trace[static_cast<size_t>(l) * k + lane] = sel[lane];
+        if (c == 0 && a.gates_trace) a.gates_trace[static_cast<size_t>(l) * k + lane] = gj;
+      }
+    } else if (warp == 1) {             // routed gate/up rows and windows
+      const int n = df_rg_count(g);
+      for (int e = lane; e < n; e += 32) {
+        const DfCopy C = df_rg_copy(g, a.off, e);
+        df_bulk(BAR(C.bar), sbase + C.dst, src_ptr(W, C), C.bytes);
+      }
+      __syncwarp();
+      if (lane < g.ntR) df_mbar_arrive(BAR(lane));
+      __syncwarp();
+    } else if (warp == 2) {             // routed down rows and windows; the next router row
+      const int n = df_d_count(g);
+      for (int e = lane; e < n; e += 32) {
+        const DfCopy C = df_d_copy(g, a.off, e);
+        df_bulk(BAR(C.bar), sbase + C.dst, src_ptr(W, C), C.bytes);
+      }
+      __syncwarp();
+      if (lane == 0) df_mbar_arrive(BAR(DF_BAR_D));
+      __syncwarp();
+      if (l + 1 < a.L) issue_rr(a.layer[l + 1]);
+    }
+    df_stamp(a, l, 5);
+
+    // ------------------------------------------------------ routed gate/up
+    {
+      const int nunits = g.ntR * g.kR;
+      for (int u = warp; u < nunits; u += DF_WARPS) {
+        const int tile = u / g.kR;
+        int g0, g1;
+        df_kpart(NGH, g.kR, u % g.kR, g0, g1);
+        df_mbar_wait(BAR(tile), par);
+        if (tile != 0) df_mbar_wait(BAR(0), par);      // the scale windows complete on tile 0's barrier
+        int i = 8 * tile + gq;
+        if (i >= g.np) i = 8 * tile;
+        float acc_a = 0.f, acc_b = 0.f;
+        df_rows<false>(smem + g.rg_row(i, 0) + 8 * tq, smem + g.rg_row(i, 1) + 8 * tq,
+                       S16 + g.rg_scale(a.off, i, 0) / 2, S16 + g.rg_scale(a.off, i, 1) / 2,
+                       S16 + g.rg_scale(a.off, i, 2) / 2, S16 + g.rg_scale(a.off, i, 3) / 2, xf + 2 * tq, xsum, xsum,
+                       0, 0, g0, g1, acc_a, acc_b);
+        if (tq == 0) {
+          part[u * 16 + gq] = acc_a;
+          part[u * 16 + 8 + gq] = acc_b;
+        }
+      }
+    }
+    df_stamp(a, l, 6);
+    __syncthreads();                     // the union area is read out
+    if (warp == 0) {                     // shared down rows into it
+      const int n = df_sd_count(g);
+      for (int e = lane; e < n; e += 32) {
+        const DfCopy C = df_sd_copy(g, e);
+        df_bulk(BAR(C.bar), sbase + C.dst, src_ptr(W, C), C.bytes);
+      }
+      __syncwarp();
+      if (lane == 0) df_mbar_arrive(BAR(DF_BAR_SD));
+      __syncwarp();
+    }
+    for (int i = threadIdx.x; i < g.np; i += DF_THREADS) {
+      const int tile = i / 8, r = i % 8;
+      float gs = 0.f, us = 0.f;
+      for (int p = 0; p < g.kR; ++p) {
+        gs += part[(tile * g.kR + p) * 16 + r];
+        us += part[(tile * g.kR + p) * 16 + 8 + r];
+      }
+      a.act[g.r0 + i] = __float2half_rn(gelu_tanh(gs) * us);
+    }
+    df_stamp(a, l, 7);
+    grid_sync();
+    df_stamp(a, l, 8);
+
+    // ------------------------------------------------------------- phase C
+    if (l + 1 < a.L && threadIdx.x == 0 && (a.prefetch & 2)) {
+      const DfLayer& V = a.layer[l + 1];
+      for (int m = 0; m < 2; ++m) {
+        prefetch_l2(reinterpret_cast<const uint8_t*>(V.sq[m]) + static_cast<size_t>(g.s0) * (H / 2),
+                    static_cast<size_t>(g.nsp) * (H / 2));
+        prefetch_l2(V.ss[m] + static_cast<size_t>(g.s0) * (H / 64), static_cast<size_t>(g.nsp) * g.sbh);
+        prefetch_l2(V.sb[m] + static_cast<size_t>(g.s0) * (H / 64), static_cast<size_t>(g.nsp) * g.sbh);
+      }
+      prefetch_l2(reinterpret_cast<const uint8_t*>(V.sq[2]) + static_cast<size_t>(g.o0) * (Is / 2),
+                  static_cast<size_t>(g.nrow) * (Is / 2));
+    }
+    if (l + 1 < a.L && warp == 1 && a.spec > 0 && a.layer[l + 1].bias != nullptr) {
+      // slices of the next layer's experts with the largest router bias
+      const DfLayer& V = a.layer[l + 1];
       unsigned taken = 0;
       int my_id = -1;
       for (int r = 0; r < a.spec && r < 8; ++r) {
@@ -401,371 +808,118 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       }
       if (my_id >= 0 && my_id < E) {
         const size_t bb = a.off[8] + static_cast<size_t>(H) * (I / 64) * 2;
-        prefetch_slice(V.blobs[my_id], bb, c, G);
+        const size_t b0 = bb * c / G, b1 = bb * (c + 1) / G;
+        prefetch_l2(static_cast<const uint8_t*>(V.blobs[my_id]) + b0, b1 - b0);
       }
     }
-  };
-  // warp 0: chunk `idx` at `off` in the staging area, completing on its mbarrier
-  auto issue_chunk = [&](int idx, const DfChunk& C0, uint32_t off) {
-    if (lane == 0) {
-      tab[idx] = C0;
-      tab[idx].off = off;
-      df_mbar_expect_tx(bar0 + 8u * idx, C0.bytes);
-    }
-    __syncwarp();
-    const DfChunk& T = tab[idx];
-    if (lane < T.n) df_bulk_g2s(smem_addr(rs + T.off + T.dst[lane]), T.src[lane], T.len[lane], bar0 + 8u * idx);
-    __syncwarp();
-  };
-  // routing-independent rows of layer l's phase A: shared gate/up rows, router row c
-  auto issue_phase_a = [&](int l) {
-    const DfLayer& V = a.layer[l];
-    DfChunk sg = df_chunk(CH_SG, 0, s0, s1 - s0, H, I, Is, a, V, sel);
-    issue_chunk(IDX_SG, sg, 0u);
-    if (c < E) {
-      DfChunk rc = df_chunk(CH_R, 0, c, 1, H, I, Is, a, V, sel);
-      issue_chunk(IDX_R, rc, (sg.bytes + 127u) & ~127u);
-    }
-  };
-  prefetch_layer(0);
-  if (warp == 0) issue_phase_a(0);
-
-  for (int l = 0; l < a.L; ++l) {
-    const DfLayer& W = a.layer[l];
-    const uint32_t par = l & 1;
-    df_stamp(a, l, 0);
-    // ------------------------------------------------------ A0: rms norm
-    float ss = 0.f;
-    for (int i = threadIdx.x * 4; i < H; i += DF_THREADS * 4) {
-      const uint4 u = ldcg_v4(a.h + i);
-      const float v0 = __uint_as_float(u.x), v1 = __uint_as_float(u.y), v2 = __uint_as_float(u.z),
-                  v3 = __uint_as_float(u.w);
-      xs[i] = v0; xs[i + 1] = v1; xs[i + 2] = v2; xs[i + 3] = v3;
-      ss = fmaf(v0, v0, ss); ss = fmaf(v1, v1, ss); ss = fmaf(v2, v2, ss); ss = fmaf(v3, v3, ss);
-    }
-    ss = warp_sum(ss);
-    if (lane == 0) red[warp] = ss;
-    __syncthreads();
-    if (warp == 0) {
-      float v = lane < DF_WARPS ? red[lane] : 0.f;
-      v = warp_sum(v);
-      if (lane == 0) red[DF_WARPS] = v;
-    }
-    __syncthreads();
-    const float rr = sqrtf(red[DF_WARPS] / static_cast<float>(H) + 1e-6f);
-    for (int i = threadIdx.x; i < H; i += DF_THREADS) {
-      const uint16_t b = f32_to_bf16(__fdiv_rn(xs[i], rr));
-      xs[i] = bf16_to_f32(b);
-      if (c == 0 && a.x_trace) a.x_trace[static_cast<size_t>(l) * H + i] = b;
-    }
-    __syncthreads();
-    for (int w = threadIdx.x; w < H / 8; w += DF_THREADS) {
-      float v[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) v[t] = xs[8 * w + t];
-      uint32_t p[4];
-      pair_word4(v, p);
-      xP4[(w & 3) * nch + (w >> 2)] = make_uint4(p[0], p[1], p[2], p[3]);
-    }
-    __syncthreads();
-    for (int cc = threadIdx.x; cc < nch; cc += DF_THREADS) {
-      float off = 0.f, sum = 0.f;
-      for (int m = 0; m < 4; ++m) {
-        const uint4 u = xP4[m * nch + cc];
-        const float2 f0 = unpack_half2(u.x), f1 = unpack_half2(u.y), f2 = unpack_half2(u.z), f3 = unpack_half2(u.w);
-        off += (f0.x + f0.y) + (f1.x + f1.y) + (f2.x + f2.y) + (f3.x + f3.y);
-        sum += (f0.x + f0.y + f2.x + f2.y) + 16.f * (f1.x + f1.y + f3.x + f3.y);
-      }
-      xS4[cc] = make_float2(1024.f * off, sum);
-    }
-    __syncthreads();
-    uint32_t xp[DF_CPL][16];
-    float2 xst[DF_CPL];
-#pragma unroll
-    for (int j = 0; j < DF_CPL; ++j) {
-      const int cc = lane + 32 * j;
-      if (cc < nch) {
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const uint4 u = xP4[m * nch + cc];
-          xp[j][4 * m + 0] = u.x; xp[j][4 * m + 1] = u.y; xp[j][4 * m + 2] = u.z; xp[j][4 * m + 3] = u.w;
-        }
-        xst[j] = xS4[cc];
-      } else {
-#pragma unroll
-        for (int t = 0; t < 16; ++t) xp[j][t] = 0u;
-        xst[j] = make_float2(0.f, 0.f);
-      }
-    }
-
-    df_stamp(a, l, 1);
-    // --------------------------------- router logit and shared gate/up rows
-    if (warp == DF_WARPS - 1) {
-      if (c < E) {
-        const DfChunk& C = tab[IDX_R];
-        df_mbar_wait(bar0 + 8u * IDX_R, par);
-        const uint8_t* qrow = rs + C.off;
-        const uint16_t* S = reinterpret_cast<const uint16_t*>(rs + C.off + C.sk[0]);
-        const uint16_t* B = reinterpret_cast<const uint16_t*>(rs + C.off + C.sk[1]);
-        float acc = 0.f;
-        for (int cc = lane; cc < H / 16; cc += 32) {
-          const uint4 q4 = *reinterpret_cast<const uint4*>(qrow + 16 * cc);
-          const float sc = bf16_to_f32(S[cc >> 2]), bi = bf16_to_f32(B[cc >> 2]);
-          const float* xv = xs + 16 * cc;
-          const uint32_t w[4] = {q4.x, q4.y, q4.z, q4.w};
-          float a0 = 0.f, a1 = 0.f, sm = 0.f;
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const uint32_t p[2] = {pack_half2(xv[4 * m], xv[4 * m + 2]), pack_half2(xv[4 * m + 1], xv[4 * m + 3])};
-            dot_word8(w[m], p, a0, a1);
-            const float2 f0 = unpack_half2(p[0]), f1 = unpack_half2(p[1]);
-            sm += (f0.x + f0.y) + (f1.x + f1.y);
-          }
-          acc += sc * ((a0 + a1) - 1024.f * sm) + bi * sm;
-        }
-        acc = warp_sum(acc);
-        if (lane == 0) a.logits[c] = acc + (W.bias ? W.bias[c] : 0.f);
-      }
-    } else if (s1 > s0) {
-      const DfChunk& C = tab[IDX_SG];
-      df_mbar_wait(bar0 + 8u * IDX_SG, par);
-      const unsigned char* base = rs + C.off;
-      for (int r = warp; r < s1 - s0; r += DF_WARPS - 1) {
-        const float2 gu = df_pair(base + r * (H / 2), base + C.qbytes + r * (H / 2),
-                                  reinterpret_cast<const uint16_t*>(base + C.sk[0]) + r * (H / 64),
-                                  reinterpret_cast<const uint16_t*>(base + C.sk[1]) + r * (H / 64),
-                                  reinterpret_cast<const uint16_t*>(base + C.sk[2]) + r * (H / 64),
-                                  reinterpret_cast<const uint16_t*>(base + C.sk[3]) + r * (H / 64), nch, xp, xst, false);
-        if (lane == 0) a.act[kI + s0 + r] = __float2half_rn(gelu_tanh(gu.x) * gu.y);
-      }
-    }
-    df_stamp(a, l, 2);
-    grid_sync();
-    df_stamp(a, l, 3);
-
-    // ------------------------------------------------ top-k, issue routed bytes
-    if (warp == 0) {
-      unsigned taken = 0u;
-      float sv[8];
-      int si[8];
-      float lv[DF_MAX_E / 32];            // this lane's logits, read once
-#pragma unroll
-      for (int t = 0; t < DF_MAX_E / 32; ++t) lv[t] = (lane + 32 * t < E) ? __ldcg(a.logits + lane + 32 * t) : 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        sv[j] = 0.f;
-        si[j] = 0;
-        if (j < k) {
-          float bv = -INFINITY;
-          int bi = 0x7fffffff;
-#pragma unroll
-          for (int t = 0; t < DF_MAX_E / 32; ++t) {
-            const int e = lane + 32 * t;
-            if (e >= E || (taken & (1u << t))) continue;
-            const float v = lv[t];
-            if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; }
-          }
-          for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-          }
-          if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-          sv[j] = bv;
-          si[j] = bi;
-        }
-      }
-      float z[8], den = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        z[j] = j < k ? expf(sv[j] - sv[0]) : 0.f;
-        den += z[j];
-      }
-      if (lane < k) {
-        float zl = 0.f;
-        int il = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) if (j == lane) { zl = z[j]; il = si[j]; }
-        sel[lane] = il;
-        selg[lane] = zl / den;
-        if (c == 0 && a.idx_trace) a.idx_trace[static_cast<size_t>(l) * k + lane] = il;
-        if (c == 0 && a.gates_trace) a.gates_trace[static_cast<size_t>(l) * k + lane] = zl / den;
-      }
-      __syncwarp();
-      if (lane == 0) df_stamp(a, l, 4);
-      // chunk `lane`: its bytes, its place in the staging area (exclusive scan)
-      DfChunk C{};
-      if (lane < nchunk) {
-        if (lane < nrg) {
-          int slot, row, rows;
-          df_rg_chunk_at(r0, r1, I, lane, slot, row, rows);
-          C = df_chunk(CH_RG, slot, row, rows, H, I, Is, a, W, sel);
-        } else {
-          C = df_chunk(CH_D, lane - nrg, o0, nrow, H, I, Is, a, W, sel);
-        }
-      }
-      uint32_t sz = lane < nchunk ? C.bytes : 0u, incl = sz;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-      }
-      if (lane < nchunk) {
-        C.off = incl - sz;
-        tab[lane] = C;
-        const uint32_t bar = bar0 + 8u * lane;
-        df_mbar_expect_tx(bar, C.bytes);
-        for (int i = 0; i < C.n; ++i) df_bulk_g2s(smem_addr(rs + C.off + C.dst[i]), C.src[i], C.len[i], bar);
-      }
-    }
-    __syncthreads();
-    df_stamp(a, l, 5);
-
-    // ------------------------------------------------------ routed gate/up
+    // paired activations of the k routed slots and of the shared expert
     {
-      const int npairs = r1 - r0;
-      for (int p = warp; p < npairs; p += DF_WARPS) {
-        const int t = p / DF_RGC;                // chunks hold DF_RGC pairs except at slot ends
-        // find the chunk holding flat pair r0 + p (chunks are in flat order)
-        int ch = 0, first = 0;
-        for (int q = 0; q < nrg; ++q) {
-          const DfChunk& Cq = tab[q];
-          const int f = Cq.slot * I + Cq.r0 - r0;
-          if (p >= f && p < f + Cq.rows) { ch = q; first = f; break; }
+      const int nw = kI / 8 + Is / 8;
+      for (int base = 0; base < nw; base += DF_THREADS) {
+        const int u = base + threadIdx.x;
+        float off = 0.f, sum = 0.f;
+        uint4 p = make_uint4(0u, 0u, 0u, 0u);
+        if (u < nw) {
+          const uint4 raw = ldcg_v4(a.act + 8 * u);
+          const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+          float v[8];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float2 f = unpack_half2(rw[t]);
+            v[2 * t] = f.x;
+            v[2 * t + 1] = f.y;
+          }
+          p = df_pair8(v, off, sum);
         }
-        (void)t;
-        const DfChunk& C = tab[ch];
-        df_mbar_wait(bar0 + 8u * ch, par);
-        const int r = p - first;
-        const unsigned char* base = rs + C.off;
-        const float2 gu = df_pair(base + r * (H / 2), base + C.qbytes + r * (H / 2),
-                                  reinterpret_cast<const uint16_t*>(base + C.sk[0]) + r * (H / 64),
-                                  reinterpret_cast<const uint16_t*>(base + C.sk[1]) + r * (H / 64),
-                                  reinterpret_cast<const uint16_t*>(base + C.sk[2]) + r * (H / 64),
-                                  reinterpret_cast<const uint16_t*>(base + C.sk[3]) + r * (H / 64), nch, xp, xst, false);
-        if (lane == 0) a.act[C.slot * I + C.r0 + r] = __float2half_rn(gelu_tanh(gu.x) * gu.y);
+        off = oct_sum(off);
+        sum = oct_sum(sum);
+        if (u < nw) {
+          if (u < kI / 8) {
+            const int j = u / (I / 8), w = u % (I / 8);
+            af[j * astride4 + w] = p;
+            if ((lane & 7) == 0) asum[j * NGI + w / 8] = make_float2(1024.f * off, sum);
+          } else {
+            const int w = u - kI / 8;
+            sf[w] = p;
+            if ((lane & 7) == 0) ssum[w / 8] = make_float2(1024.f * off, sum);
+          }
+        }
       }
     }
-    df_stamp(a, l, 6);
-    // shared down rows of phase C into the gate/up part of the staging area
-    // (free now) when it is large enough, else after the down chunks
-    const int dsc = IDX_DS;
     __syncthreads();
-    if (warp == 0) {
-      const DfChunk C = df_chunk(CH_DS, 0, o0, nrow, H, I, Is, a, W, sel);
-      const uint32_t rg_bytes = tab[nrg].off;
-      const uint32_t used = tab[nchunk - 1].off + tab[nchunk - 1].bytes;
-      issue_chunk(dsc, C, C.bytes <= rg_bytes ? 0u : ((used + 127u) & ~127u));
-    }
-    df_stamp(a, l, 7);
-    grid_sync();
-    df_stamp(a, l, 8);
-
-    // ------------------------------------------------------------- phase C
-    if (l + 1 < a.L) prefetch_layer(l + 1);
     df_stamp(a, l, 9);
-    for (int w = threadIdx.x; w < nact / 8; w += DF_THREADS) {
-      const uint4 u = ldcg_v4(a.act + 8 * w);
-      float v[8];
-      const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const float2 f = unpack_half2(uw[t]);
-        v[2 * t] = f.x;
-        v[2 * t + 1] = f.y;
+    // down tiles: routed rows rho = j * nrow + r (a tile mixes slots; column j
+    // carries slot j's activation), then the shared rows
+    {
+      const int nd = g.ntD * g.kD, nunits = nd + g.ntSD * g.kSD;
+      const int colslot = gq < k ? gq : 0;
+      for (int u = warp; u < nunits; u += DF_WARPS) {
+        float acc_a = 0.f, acc_b = 0.f;
+        if (u < nd) {
+          const int tile = u / g.kD;
+          int g0, g1;
+          df_kpart(NGI, g.kD, u % g.kD, g0, g1);
+          df_mbar_wait(BAR(DF_BAR_D), par);
+          int ra = 16 * tile + gq, rb = 16 * tile + 8 + gq;
+          const bool va = ra < k * g.nrow, vb = rb < k * g.nrow;
+          if (!va) ra = 0;
+          if (!vb) rb = 0;
+          const int ja = ra / g.nrow, ia = ra % g.nrow, jb = rb / g.nrow, ib = rb % g.nrow;
+          df_rows<true>(smem + g.d_row(ja, ia) + 8 * tq, smem + g.d_row(jb, ib) + 8 * tq,
+                        S16 + g.d_scale(a.off, ja, ia, 0) / 2, S16 + g.d_scale(a.off, ja, ia, 1) / 2,
+                        S16 + g.d_scale(a.off, jb, ib, 0) / 2, S16 + g.d_scale(a.off, jb, ib, 1) / 2,
+                        af + colslot * astride4 + 2 * tq, asum + ja * NGI, asum + jb * NGI, ja & 1, jb & 1, g0, g1,
+                        acc_a, acc_b);
+          if (va && tq == (ja >> 1)) part[u * 16 + gq] = acc_a;
+          if (vb && tq == (jb >> 1)) part[u * 16 + 8 + gq] = acc_b;
+        } else {
+          const int us = u - nd, tile = us / g.kSD;
+          int g0, g1;
+          df_kpart(NGS, g.kSD, us % g.kSD, g0, g1);
+          df_mbar_wait(BAR(DF_BAR_SD), par);
+          int ra = 16 * tile + gq, rb = 16 * tile + 8 + gq;
+          if (ra >= g.nrow) ra = 0;
+          if (rb >= g.nrow) rb = 0;
+          df_rows<false>(smem + g.sd_row(ra) + 8 * tq, smem + g.sd_row(rb) + 8 * tq, S16 + g.sd_scale(ra, 0) / 2,
+                         S16 + g.sd_scale(ra, 1) / 2, S16 + g.sd_scale(rb, 0) / 2, S16 + g.sd_scale(rb, 1) / 2,
+                         sf + 2 * tq, ssum, ssum, 0, 0, g0, g1, acc_a, acc_b);
+          if (tq == 0) {
+            part[u * 16 + gq] = acc_a;
+            part[u * 16 + 8 + gq] = acc_b;
+          }
+        }
       }
-      uint32_t p[4];
-      pair_word4(v, p);
-      actP[w] = make_uint4(p[0], p[1], p[2], p[3]);
-      float off = 0.f;
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const float2 f = unpack_half2(p[t]);
-        off += f.x + f.y;
-      }
-      const float2 f0 = unpack_half2(p[0]), f1 = unpack_half2(p[1]), f2 = unpack_half2(p[2]), f3 = unpack_half2(p[3]);
-      actS[w] = make_float2(1024.f * off, (f0.x + f0.y + f2.x + f2.y) + 16.f * (f1.x + f1.y + f3.x + f3.y));
     }
     __syncthreads();
     df_stamp(a, l, 10);
-    // units (piece u, block of DF_RB rows): u < k routed slot u (K = I),
-    // u == k the shared expert (K = Is); the activation word is loaded once
-    // and applied to the block's rows (independent accumulators)
-    constexpr int DF_RB = 4;
-    const int nblk = (nrow + DF_RB - 1) / DF_RB;
-    for (int un = warp; un < nblk * (k + 1); un += DF_WARPS) {
-      const int u = un % (k + 1), rb = un / (k + 1);
-      const int ch = u < k ? nrg + u : dsc;
-      const DfChunk& C = tab[ch];
-      df_mbar_wait(bar0 + 8u * ch, par);
-      const int K = u < k ? I : Is;
-      const int wbase = u < k ? u * (I / 8) : kI / 8;
-      const int rbeg = rb * DF_RB, nr = min(DF_RB, nrow - rbeg);
-      const unsigned char* base = rs + C.off;
-      const uint8_t* q0 = base + static_cast<size_t>(rbeg) * (K / 2);
-      const uint16_t* S0 = reinterpret_cast<const uint16_t*>(base + C.sk[0]) + rbeg * (K / 64);
-      const uint16_t* B0 = reinterpret_cast<const uint16_t*>(base + C.sk[1]) + rbeg * (K / 64);
-      float acc[DF_RB];
-#pragma unroll
-      for (int t = 0; t < DF_RB; ++t) acc[t] = 0.f;
-      for (int w = lane; w < K / 8; w += 32) {
-        const uint4 pp = actP[wbase + w];
-        const uint32_t p[4] = {pp.x, pp.y, pp.z, pp.w};
-        const float2 st = actS[wbase + w];
-#pragma unroll
-        for (int t = 0; t < DF_RB; ++t) {
-          if (t < nr) {
-            const uint32_t qw = *reinterpret_cast<const uint32_t*>(q0 + t * (K / 2) + 4 * w);
-            float a0 = 0.f, a1 = 0.f;
-            dot_word4(qw, p, a0, a1);
-            acc[t] += bf16_to_f32(S0[t * (K / 64) + (w >> 3)]) * ((a0 + a1) - st.x) +
-                      bf16_to_f32(B0[t * (K / 64) + (w >> 3)]) * st.y;
-          }
+    {
+      const int nd = g.ntD * g.kD;
+      for (int r = threadIdx.x; r < g.nrow; r += DF_THREADS) {
+        float y = 0.f;
+        for (int j = 0; j < k; ++j) {
+          const int rho = j * g.nrow + r, tile = rho / 16, tr = rho % 16;
+          float yj = 0.f;
+          for (int p = 0; p < g.kD; ++p) yj += part[(tile * g.kD + p) * 16 + tr];
+          y = fmaf(selg[j], yj, y);
         }
-      }
-#pragma unroll
-      for (int t = 0; t < DF_RB; ++t) {
-        const float v = warp_sum(acc[t]);
-        if (lane == 0 && t < nr) part[(rbeg + t) * 9 + u] = v;
+        const int ts = r / 16, tr = r % 16;
+        float ysh = 0.f;
+        for (int p = 0; p < g.kSD; ++p) ysh += part[(nd + ts * g.kSD + p) * 16 + tr];
+        y += ysh;
+        const int o = g.o0 + r;
+        a.h[o] = __ldcg(a.h + o) + y;
+        if (a.y_trace) a.y_trace[static_cast<size_t>(l) * H + o] = f32_to_bf16(y);
       }
     }
-    __syncthreads();
     df_stamp(a, l, 11);
-    for (int r = threadIdx.x; r < nrow; r += DF_THREADS) {
-      float y = 0.f;
-      for (int j = 0; j < k; ++j) y = fmaf(selg[j], part[r * 9 + j], y);
-      y += part[r * 9 + k];
-      const int o = o0 + r;
-      a.h[o] = __ldcg(a.h + o) + y;
-      if (a.y_trace) a.y_trace[static_cast<size_t>(l) * H + o] = f32_to_bf16(y);
-    }
-    df_stamp(a, l, 12);
     if (l + 1 < a.L) {
-      __syncthreads();                     // staging area read out
-      if (warp == 0) issue_phase_a(l + 1);
+      if (warp == 0) issue_sg(a.layer[l + 1]);    // the union area was read out before the combine
+      df_stamp(a, l, 12);
+      grid_sync();
     }
     df_stamp(a, l, 13);
-    if (l + 1 < a.L) grid_sync();
-    df_stamp(a, l, 14);
   }
 }
-
-size_t decode_fused_smem() {
-  return static_cast<size_t>(DF_RS) + static_cast<size_t>(DF_MAX_ACT / 8) * 24 + DF_MAX_H / 8 * 16 +
-         DF_MAX_H / 32 * 8 + DF_MAX_ROWS * 9 * 4 + 32 * 4 + 8 * 4 + 8 * 4 +
-         (DF_MAX_CHUNKS + 3) * sizeof(DfChunk) + (DF_MAX_CHUNKS + 3) * 8 + 128;
-}
-
-// Staging bytes a CTA needs for its routed chunks (worst case over CTAs), or
-// -1 if more chunks than DF_MAX_CHUNKS.
-inline long df_staging_need(int H, int I, int Is, int k, int G) {
-  const int pairs = (k * I + G - 1) / G, rows = (H + G - 1) / G;
-  const int nrg = (pairs + DF_RGC - 1) / DF_RGC + 1;
-  if (nrg + k > DF_MAX_CHUNKS) return -1;
-  const long rg = static_cast<long>(pairs) * H + static_cast<long>(nrg) * 4 * (DF_RGC * 2 * (H / 64) + 32);
-  const long d = static_cast<long>(k) * (rows * (I / 2) + 2 * (rows * 2 * (I / 64) + 32));
-  const long ds = static_cast<long>(rows) * (Is / 2) + 2 * (rows * 2 * (Is / 64) + 32);
-  return rg + d + (ds > rg ? ds + 128 : 0);
-}
+#endif  // __CUDACC__
 
 }  // namespace moe
