@@ -52,12 +52,12 @@ constexpr int DF_MAX_E = 256;
 constexpr int DF_MAX_RG_PAIRS = 48;       // routed gate/up pairs per CTA (6 tiles)
 constexpr int DF_MAX_SG_PAIRS = 24;       // shared gate/up pairs per CTA (3 tiles)
 constexpr int DF_MAX_ROWS = 32;           // output rows per CTA
-constexpr int DF_MAX_UNITS = 48;          // warp work units per phase
-constexpr int DF_KS = 5;                  // K parts of a shared gate/up tile (at most)
-constexpr int DF_KR = 4;                  // K parts of a routed gate/up tile (at most)
-constexpr int DF_KD = 2;                  // K parts of a routed down tile (at most)
-constexpr int DF_KSD = 3;                 // K parts of a shared down tile (at most)
+constexpr int DF_MAX_COPIES = 64;         // entries of a CTA's copy table (all five lists)
+constexpr int DF_STRIP = 4;               // quantisation groups a warp holds at once (its strip)
+constexpr int DF_MAX_TILES = 18;          // routed + shared down tiles per CTA
 constexpr int DF_SMEM_LIMIT = 232448;     // opt-in shared memory per block
+constexpr int DF_MAX_ACT = 8 * DF_THREADS * 3;   // k*I + Is fp16 activations (3 words of 8 per thread)
+constexpr int DF_ACT_ROUNDS = 3;
 // mbarriers: routed gate/up tiles 0..5, then
 constexpr int DF_BAR_D = 6, DF_BAR_SD = 7, DF_BAR_SG = 8, DF_BAR_RR = 9, DF_NBARS = 10;
 // copy sources besides routed slots 0..7: shared matrix m array a (q, s, b) at
@@ -101,11 +101,11 @@ struct DfGeom {
   int s0, nsp, r0, np, o0, nrow;    // shared pairs, routed flat pairs, output rows
   int j0, n0, n1;                   // routed runs: first slot, pairs in it, pairs in the next slot
   int ntS, ntR, ntD, ntSD;          // 16-row tiles per phase
-  int kS, kR, kD, kSD;              // K parts per tile (no more than the groups)
-  uint32_t rowb;                    // padded gate/up row (H/2 + 16 bytes)
+  uint32_t rowb;                    // gate/up row bytes (H/2)
   uint32_t sbh, sbi, sbs;           // scale row bytes for K = H, I, Is
   int npmax, nspmax, nrowmax;
-  uint32_t U, D, RR, F, M, total;   // areas: union (RG | SG | SD), routed down, router row, fragments, misc
+  uint32_t U, D, RR, F, M, total;   // areas: union (RG | SD + SG), routed down, router row, fragments, misc
+  uint32_t SGB;                     // shared gate/up inside the union area, after the shared down rows
   uint32_t dslot;                   // bytes per routed down slot
 
   DF_HD void init(int H_, int I_, int Is_, int E_, int k_, int G_, int c_) {
@@ -124,11 +124,7 @@ struct DfGeom {
     ntR = (np + 7) / 8;
     ntD = (k * nrow + 15) / 16;
     ntSD = (nrow + 15) / 16;
-    kS = H / 64 < DF_KS ? H / 64 : DF_KS;
-    kR = H / 64 < DF_KR ? H / 64 : DF_KR;
-    kD = I / 64 < DF_KD ? I / 64 : DF_KD;
-    kSD = Is / 64 < DF_KSD ? Is / 64 : DF_KSD;
-    rowb = static_cast<uint32_t>(H / 2 + 16);
+    rowb = static_cast<uint32_t>(H / 2);
     sbh = static_cast<uint32_t>(H / 64) * 2;
     sbi = static_cast<uint32_t>(I / 64) * 2;
     sbs = static_cast<uint32_t>(Is / 64) * 2;
@@ -138,11 +134,12 @@ struct DfGeom {
     // union area: the largest of the three layouts any CTA can have
     // two runs of n0 + n1 = np pairs: wres(n0) + wres(n1) <= a16(np * sbh) + 80
     const uint32_t rg = 2u * npmax * rowb + 4u * (df_a16(static_cast<uint64_t>(npmax) * sbh) + 80u);
-    const uint32_t sg = 2u * nspmax * rowb + 4u * df_wres(nspmax, sbh);
+    // shared down at the start, the next layer's shared gate/up after it
     const uint32_t sd = df_a16(static_cast<uint64_t>(nrowmax) * (Is / 2)) + 2u * df_wres(nrowmax, sbs);
-    uint32_t u = rg > sg ? rg : sg;
-    u = u > sd ? u : sd;
+    const uint32_t sg = 2u * nspmax * rowb + 4u * df_wres(nspmax, sbh);
     U = 0;
+    SGB = (sd + 127u) & ~127u;
+    const uint32_t u = rg > SGB + sg ? rg : SGB + sg;
     dslot = df_a16(static_cast<uint64_t>(nrowmax) * (I / 2)) + 2u * df_wres(nrowmax, sbi);
     D = (U + u + 127u) & ~127u;
     RR = D + 8u * dslot;
@@ -157,9 +154,30 @@ struct DfGeom {
                         static_cast<uint32_t>(Is / 64) * 8;
     return xf > af ? xf : af;
   }
-  DF_HD static constexpr uint32_t misc_bytes() {
-    // logits, sel / selv / selg, red, part, bars
-    return DF_MAX_E * 4 + 8 * 4 * 3 + 16 * 4 + DF_MAX_UNITS * 16 * 4 + DF_NBARS * 8;
+  // Work split of the dots.  Gate/up: warp w holds groups [w*NGH/nw, ...)
+  // of every tile (nw = 11 in phase A, where warp 11 computes the router
+  // logit, and 12 in phase B).  Down: the routed tiles are split dp ways by
+  // groups and 12/dp ways by tiles; the shared tiles 12 ways by groups.
+  DF_HD int sg_tiles_max() const { return (nspmax + 7) / 8; }
+  DF_HD int rg_tiles_max() const { return (npmax + 7) / 8; }
+  DF_HD int d_tiles_max() const { return (k * nrowmax + 15) / 16; }
+  DF_HD int sd_tiles_max() const { return (nrowmax + 15) / 16; }
+  DF_HD int dp() const { return (I / 64 + DF_STRIP - 1) / DF_STRIP; }
+  // partial-sum slots (16 floats each) of every phase
+  DF_HD int slot_sg(int w, int t) const { return w * sg_tiles_max() + t; }
+  DF_HD int slot_rg(int w, int t) const { return w * rg_tiles_max() + t; }
+  DF_HD int slot_d(int gp, int t) const { return gp * d_tiles_max() + t; }
+  DF_HD int slot_sd(int w, int t) const { return dp() * d_tiles_max() + w * sd_tiles_max() + t; }
+  DF_HD int part_slots() const {
+    const int a = (DF_WARPS - 1) * sg_tiles_max(), b = DF_WARPS * rg_tiles_max();
+    const int c = dp() * d_tiles_max() + DF_WARPS * sd_tiles_max();
+    const int m = a > b ? a : b;
+    return m > c ? m : c;
+  }
+  DF_HD uint32_t misc_bytes() const {
+    // logits, sel / selv / selg, red, bars, blob table, copy table, pair table, part
+    return DF_MAX_E * 4 + 8 * 4 * 3 + 16 * 4 + DF_NBARS * 8 + DF_MAX_E * 8 + DF_MAX_COPIES * 16 +
+           (DF_MAX_RG_PAIRS + DF_MAX_SG_PAIRS) * 16 + static_cast<uint32_t>(part_slots()) * 64;
   }
   // misc sub-offsets
   DF_HD uint32_t m_lg() const { return M; }
@@ -167,8 +185,11 @@ struct DfGeom {
   DF_HD uint32_t m_selv() const { return m_sel() + 32; }
   DF_HD uint32_t m_selg() const { return m_sel() + 64; }
   DF_HD uint32_t m_red() const { return m_sel() + 96; }
-  DF_HD uint32_t m_part() const { return m_red() + 64; }
-  DF_HD uint32_t m_bars() const { return m_part() + DF_MAX_UNITS * 64; }
+  DF_HD uint32_t m_bars() const { return m_red() + 64; }
+  DF_HD uint32_t m_btab() const { return m_bars() + DF_NBARS * 8; }     // this layer's E blob pointers
+  DF_HD uint32_t m_ctab() const { return m_btab() + DF_MAX_E * 8; }      // the CTA's copy lists
+  DF_HD uint32_t m_ptab() const { return m_ctab() + DF_MAX_COPIES * 16; }   // scale rows of every pair
+  DF_HD uint32_t m_part() const { return m_ptab() + (DF_MAX_RG_PAIRS + DF_MAX_SG_PAIRS) * 16; }
   // fragment sub-offsets (phases A, B: x; phase C: activations)
   DF_HD uint32_t f_xs() const { return F; }
   DF_HD uint32_t f_xf() const { return F + static_cast<uint32_t>(H) * 4; }
@@ -180,7 +201,8 @@ struct DfGeom {
   DF_HD uint32_t f_ssum() const { return f_asum() + 8u * (I / 64) * 8; }
 
   // ---- routed gate/up: pair i (0..np-1), m = 0 gate / 1 up
-  DF_HD uint32_t rg_row(int i, int m) const { return U + (2u * i + m) * rowb; }
+  // gate rows of the CTA's pairs one after the other, then the up rows
+  DF_HD uint32_t rg_row(int i, int m) const { return U + (m * static_cast<uint32_t>(np) + i) * rowb; }
   DF_HD uint32_t rg_win0() const { return U + 2u * np * rowb; }
   // window of run `run` (0: slot j0, 1: slot j0+1), array a (0 gate.s, 1 gate.b, 2 up.s, 3 up.b)
   DF_HD uint32_t rg_win(int run, int a) const {
@@ -208,8 +230,8 @@ struct DfGeom {
     return d_win(j, a) + static_cast<uint32_t>(d_src(off, a) & 15) + r * sbi;
   }
   // ---- shared gate/up: pair i (0..nsp-1); windows gate.s, gate.b, up.s, up.b
-  DF_HD uint32_t sg_row(int i, int m) const { return U + (2u * i + m) * rowb; }
-  DF_HD uint32_t sg_win(int a) const { return U + 2u * nsp * rowb + a * df_wres(nsp, sbh); }
+  DF_HD uint32_t sg_row(int i, int m) const { return SGB + (m * static_cast<uint32_t>(nsp) + i) * rowb; }
+  DF_HD uint32_t sg_win(int a) const { return SGB + 2u * nsp * rowb + a * df_wres(nsp, sbh); }
   DF_HD uint64_t sg_src() const { return static_cast<uint64_t>(s0) * sbh; }
   DF_HD uint32_t sg_scale(int i, int a) const { return sg_win(a) + static_cast<uint32_t>(sg_src() & 15) + i * sbh; }
   // ---- shared down: row r
@@ -246,18 +268,45 @@ DF_HD inline DfCopy df_plain(uint32_t dst, uint64_t src_off, uint32_t bytes, int
   return C;
 }
 
-// routed gate/up: 2*np rows (bar = tile), then 4 windows per run (bar 0)
-DF_HD inline int df_rg_count(const DfGeom& g) { return 2 * g.np + 4 * (g.n0 > 0) + 4 * (g.n1 > 0); }
-DF_HD inline DfCopy df_rg_copy(const DfGeom& g, const size_t* off, int e) {
-  if (e < 2 * g.np) {
-    const int i = e >> 1, m = e & 1;
-    const int p = g.r0 + i, slot = p / g.I, row = p % g.I;
-    return df_plain(g.rg_row(i, m), off[3 * m] + static_cast<uint64_t>(row) * (g.H / 2),
-                    static_cast<uint32_t>(g.H / 2), slot, i / 8);
+// routed gate/up: first the 4 scale/bias windows per run (bar 0, so that every
+// tile can start as soon as its rows land), then per tile (8 pairs) and run
+// the gate rows and the up rows of its pairs as two copies (bar = tile)
+DF_HD inline int df_rg_pieces(const DfGeom& g) {
+  int n = 0;
+  for (int t = 0; t < g.ntR; ++t) {
+    const int a = 8 * t, b = 8 * t + 8 < g.np ? 8 * t + 8 : g.np;
+    n += (a < g.n0 && g.n0 < b) ? 2 : 1;
   }
-  e -= 2 * g.np;
-  const int run = e / 4, a = e % 4;
-  return df_window(g.rg_win(run, a), g.rg_src(off, run, a), run ? g.n1 : g.n0, g.sbh, g.j0 + run, 0);
+  return n;
+}
+DF_HD inline int df_rg_count(const DfGeom& g) { return 2 * df_rg_pieces(g) + 4 * (g.n0 > 0) + 4 * (g.n1 > 0); }
+DF_HD inline DfCopy df_rg_copy(const DfGeom& g, const size_t* off, int e) {
+  const int nwin = 4 * (g.n0 > 0) + 4 * (g.n1 > 0);
+  if (e < nwin) {
+    const int run = e / 4, a = e % 4;
+    return df_window(g.rg_win(run, a), g.rg_src(off, run, a), run ? g.n1 : g.n0, g.sbh, g.j0 + run, 0);
+  }
+  e -= nwin;
+  {
+    const int piece = e >> 1, m = e & 1;
+    int t = 0, a = 0, b = 0, seen = 0;
+    for (t = 0; t < g.ntR; ++t) {          // find the piece: tiles in order, a split tile gives two
+      a = 8 * t;
+      b = 8 * t + 8 < g.np ? 8 * t + 8 : g.np;
+      if (a < g.n0 && g.n0 < b) {
+        if (seen == piece) { b = g.n0; break; }
+        if (seen + 1 == piece) { a = g.n0; break; }
+        seen += 2;
+      } else {
+        if (seen == piece) break;
+        seen += 1;
+      }
+    }
+    const int run = a < g.n0 ? 0 : 1;
+    const int row = g.rg_row0(run) + (run ? a - g.n0 : a);
+    return df_plain(g.rg_row(a, m), off[3 * m] + static_cast<uint64_t>(row) * g.rowb, static_cast<uint32_t>(b - a) * g.rowb,
+                    g.j0 + run, t);
+  }
 }
 // routed down: per slot the nrow rows, then the two windows
 DF_HD inline int df_d_count(const DfGeom& g) { return g.nrow > 0 ? 3 * g.k : 0; }
@@ -276,15 +325,13 @@ DF_HD inline DfCopy df_sd_copy(const DfGeom& g, int e) {
                     DF_SRC_SHARED + 6, DF_BAR_SD);
   return df_window(g.sd_win(e - 1), g.sd_src(), g.nrow, g.sbs, DF_SRC_SHARED + 6 + e, DF_BAR_SD);
 }
-// shared gate/up (matrices 0, 1): 2*nsp rows, then gate.s, gate.b, up.s, up.b
-DF_HD inline int df_sg_count(const DfGeom& g) { return g.nsp > 0 ? 2 * g.nsp + 4 : 0; }
+// shared gate/up (matrices 0, 1): the gate rows, the up rows, then gate.s, gate.b, up.s, up.b
+DF_HD inline int df_sg_count(const DfGeom& g) { return g.nsp > 0 ? 6 : 0; }
 DF_HD inline DfCopy df_sg_copy(const DfGeom& g, int e) {
-  if (e < 2 * g.nsp) {
-    const int i = e >> 1, m = e & 1;
-    return df_plain(g.sg_row(i, m), static_cast<uint64_t>(g.s0 + i) * (g.H / 2), static_cast<uint32_t>(g.H / 2),
-                    DF_SRC_SHARED + 3 * m, DF_BAR_SG);
-  }
-  e -= 2 * g.nsp;
+  if (e < 2)
+    return df_plain(g.sg_row(0, e), static_cast<uint64_t>(g.s0) * g.rowb, static_cast<uint32_t>(g.nsp) * g.rowb,
+                    DF_SRC_SHARED + 3 * e, DF_BAR_SG);
+  e -= 2;
   const int m = e / 2, a = e % 2;
   return df_window(g.sg_win(e), g.sg_src(), g.nsp, g.sbh, DF_SRC_SHARED + 3 * m + 1 + a, DF_BAR_SG);
 }
@@ -296,11 +343,26 @@ DF_HD inline DfCopy df_rr_copy(const DfGeom& g, int e) {
   return df_window(g.rr_win(e - 1), g.rr_src(), 1, g.sbh, DF_SRC_ROUTER + e, DF_BAR_RR);
 }
 
-// Group range [g0, g1) of K part p of `parts` over ng groups.
-DF_HD inline void df_kpart(int ng, int parts, int p, int& g0, int& g1) {
-  g0 = ng * p / parts;
-  g1 = ng * (p + 1) / parts;
+// The five copy lists of a CTA in one table: routed gate/up, routed down,
+// shared down, shared gate/up, router row (list i starts at df_list_start(g, i)).
+DF_HD inline int df_list_count(const DfGeom& g, int list) {
+  return list == 0 ? df_rg_count(g) : list == 1 ? df_d_count(g) : list == 2 ? df_sd_count(g)
+       : list == 3 ? df_sg_count(g) : df_rr_count(g);
 }
+DF_HD inline int df_list_start(const DfGeom& g, int list) {
+  int n = 0;
+  for (int i = 0; i < list; ++i) n += df_list_count(g, i);
+  return n;
+}
+DF_HD inline DfCopy df_list_copy(const DfGeom& g, const size_t* off, int list, int e) {
+  return list == 0 ? df_rg_copy(g, off, e) : list == 1 ? df_d_copy(g, off, e) : list == 2 ? df_sd_copy(g, e)
+       : list == 3 ? df_sg_copy(g, e) : df_rr_copy(g, e);
+}
+// table entry: 16 bytes
+struct DfCopyS {
+  uint32_t dst, bytes, src_off;
+  uint16_t src, bar;
+};
 
 // Shared-memory bytes of the kernel for these dims and grid (the layout is
 // the same for every CTA).
@@ -313,12 +375,25 @@ inline size_t decode_fused_smem(int H, int I, int Is, int E, int k, int G) {
 // Whether every CTA's work fits the kernel's fixed limits.
 inline bool df_fits(int H, int I, int Is, int E, int k, int G) {
   if (G <= 0 || H % 64 || I % 64 || Is % 64 || H > DF_MAX_H || E > DF_MAX_E || E > G || k > 8) return false;
+  if (k * I + Is > DF_MAX_ACT) return false;
   DfGeom g;
   g.init(H, I, Is, E, k, G, 0);
   if (g.npmax > DF_MAX_RG_PAIRS || g.npmax > I || g.nspmax > DF_MAX_SG_PAIRS || g.nrowmax > DF_MAX_ROWS) return false;
   const int tiles_d = (k * g.nrowmax + 15) / 16, tiles_sd = (g.nrowmax + 15) / 16;
-  if (((g.npmax + 7) / 8) * g.kR > DF_MAX_UNITS || ((g.nspmax + 7) / 8) * g.kS > DF_MAX_UNITS) return false;
-  if (tiles_d * g.kD + tiles_sd * g.kSD > DF_MAX_UNITS) return false;
+  if (tiles_d + tiles_sd > DF_MAX_TILES) return false;
+  // every CTA's copy lists fit the table; source offsets fit 32 bits
+  if (static_cast<uint64_t>(I) * H * 2 > 0xFFFFFFFFull) return false;
+  for (int c = 0; c < G; ++c) {
+    DfGeom gc;
+    gc.init(H, I, Is, E, k, G, c);
+    int n = 0;
+    for (int i = 0; i < 5; ++i) n += df_list_count(gc, i);
+    if (n > DF_MAX_COPIES) return false;
+  }
+  // strips: gate/up K over 11 warps, routed down over dp (dividing 12) group
+  // parts, shared down over 12 warps; no strip longer than DF_STRIP
+  if ((H / 64 + DF_WARPS - 2) / (DF_WARPS - 1) > DF_STRIP) return false;
+  if (DF_WARPS % g.dp() != 0 || (Is / 64 + DF_WARPS - 1) / DF_WARPS > DF_STRIP) return false;
   return g.total <= static_cast<uint32_t>(DF_SMEM_LIMIT);
 }
 
@@ -351,14 +426,15 @@ __device__ __forceinline__ bool df_mbar_wait(uint32_t bar, uint32_t parity) {
   uint64_t t0 = 0;
   for (uint32_t i = 0;; ++i) {
     uint32_t ok;
+    // the thread sleeps until the phase completes or about 1 us passes
     asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(1000u)
         : "memory");
     if (ok) return true;
-    if ((i & 255u) == 0) {
+    if ((i & 15u) == 0) {
       const uint64_t now = df_clock();
       if (t0 == 0) t0 = now;
       else if (now - t0 > 2000000000ull) break;
@@ -393,10 +469,13 @@ __device__ __forceinline__ uint4 ldcg_v4(const void* p) {
   return r;
 }
 
-// phase timestamps (when requested): layer l, CTA c, point p
+// phase timestamps (when requested): layer l, CTA c, point p; df_stamp by
+// thread 0, df_stamp_here by the calling thread
+__device__ __forceinline__ void df_stamp_here(const DfArgs& a, int l, int p) {
+  if (a.stamps != nullptr) a.stamps[(static_cast<size_t>(l) * gridDim.x + blockIdx.x) * 16 + p] = df_clock();
+}
 __device__ __forceinline__ void df_stamp(const DfArgs& a, int l, int p) {
-  if (a.stamps != nullptr && threadIdx.x == 0)
-    a.stamps[(static_cast<size_t>(l) * gridDim.x + blockIdx.x) * 16 + p] = df_clock();
+  if (threadIdx.x == 0) df_stamp_here(a, l, p);
 }
 
 // ------------------------------------------------------------ tensor-core dot
@@ -415,38 +494,75 @@ __device__ __forceinline__ uint32_t nib_hi(uint32_t w) { return (w & 0x00F000F0u
 // of those words in this lane's column.  Fragment rows: a0/a2 row g, a1/a3
 // row g+8; a0/a1 pair with b0, a2/a3 with b1.
 __device__ __forceinline__ void mma_group(float (&d)[4], uint2 wa, uint2 wb, uint4 f0, uint4 f1) {
+  float e[4] = {0.f, 0.f, 0.f, 0.f};        // second, independent accumulator chain
   d[0] = d[1] = d[2] = d[3] = 0.f;
+  const uint32_t ax = wa.x >> 8, bx = wb.x >> 8, ay = wa.y >> 8, by = wb.y >> 8;
   mma16816(d, nib_lo(wa.x), nib_lo(wb.x), nib_hi(wa.x), nib_hi(wb.x), f0.x, f0.y);
-  const uint32_t ax = wa.x >> 8, bx = wb.x >> 8;
+  mma16816(e, nib_lo(wa.y), nib_lo(wb.y), nib_hi(wa.y), nib_hi(wb.y), f1.x, f1.y);
   mma16816(d, nib_lo(ax), nib_lo(bx), nib_hi(ax), nib_hi(bx), f0.z, f0.w);
-  mma16816(d, nib_lo(wa.y), nib_lo(wb.y), nib_hi(wa.y), nib_hi(wb.y), f1.x, f1.y);
-  const uint32_t ay = wa.y >> 8, by = wb.y >> 8;
-  mma16816(d, nib_lo(ay), nib_lo(by), nib_hi(ay), nib_hi(by), f1.z, f1.w);
+  mma16816(e, nib_lo(ay), nib_lo(by), nib_hi(ay), nib_hi(by), f1.z, f1.w);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] += e[i];
 }
 
-// Groups [g0, g1) of this lane's two tile rows: acc += S (dot - sum.x) + B sum.y
-// per group.  qa/qb: the rows' bytes at this lane's offset 8t; sa/ba, sb/bb:
-// their bf16 scale and bias rows; f: this lane's column of paired activation
-// (uint4 per word, 8 words per group) at word 2t; suma/sumb: per group
-// (1024 * sum of paired halves, sum of values) of each row's column; ca/cb:
-// which accumulator of the pair holds the row's column (down tiles).
-template <bool COLS>
-__device__ __forceinline__ void df_rows(const uint8_t* qa, const uint8_t* qb, const uint16_t* sa, const uint16_t* ba,
-                                        const uint16_t* sb, const uint16_t* bb, const uint4* f, const float2* suma,
-                                        const float2* sumb, int ca, int cb, int g0, int g1, float& acc_a,
-                                        float& acc_b) {
-#pragma unroll 2
-  for (int gr = g0; gr < g1; ++gr) {
-    const uint2 wa = *reinterpret_cast<const uint2*>(qa + 32 * gr);
-    const uint2 wb = *reinterpret_cast<const uint2*>(qb + 32 * gr);
-    const uint4 f0 = f[8 * gr], f1 = f[8 * gr + 1];
-    float d[4];
-    mma_group(d, wa, wb, f0, f1);
-    const float2 xa = suma[gr], xb = sumb[gr];
-    const float va = COLS ? (ca ? d[1] : d[0]) : d[0];
-    const float vb = COLS ? (cb ? d[3] : d[2]) : d[2];
-    acc_a += bf16_to_f32(sa[gr]) * (va - xa.x) + bf16_to_f32(ba[gr]) * xa.y;
-    acc_b += bf16_to_f32(sb[gr]) * (vb - xb.x) + bf16_to_f32(bb[gr]) * xb.y;
+// How the 8 mma columns are used.  BCAST: every column carries the same
+// vector (the result of row g is in accumulator 0/2 of every lane of quad g).
+// SLOT: column j carries slot j's activation (row g's result in column
+// slot(g)).  DIAG: quad g works on group g0 + (s + g) mod ng at step s and
+// column g carries that group of the vector, so the row's result is column
+// g -- rows one whole number of 128-byte lines apart then read distinct banks.
+enum : int { DF_BCAST = 0, DF_SLOT = 1, DF_DIAG = 2 };
+
+// This warp's strip of ng <= DF_STRIP groups (from g0) of one 16-row tile,
+// for the lane's two rows: acc += S (dot - sum.x) + B sum.y per group.
+// qa/qb: the rows' bytes at this lane's offset 8t; sa/ba, sb/bb: their bf16
+// scale and bias rows; fb/xs: the lane's paired activation of the strip and
+// the group sums (1024 * sum of paired halves, sum of values), in step order,
+// held in registers for every tile; suma/sumb: per-row group sums (SLOT);
+// ca/cb: the accumulator of the pair that holds the row's column (SLOT,
+// DIAG); rs: the lane's rotation (DIAG).
+template <int MODE>
+__device__ __forceinline__ void df_strip(const uint8_t* qa, const uint8_t* qb, const uint16_t* sa, const uint16_t* ba,
+                                         const uint16_t* sb, const uint16_t* bb, const uint4 (&fb)[DF_STRIP][2],
+                                         const float2 (&xs)[DF_STRIP], const float2* suma, const float2* sumb,
+                                         int ca, int cb, int g0, int ng, int rs, float& acc_a, float& acc_b) {
+#pragma unroll
+  for (int j = 0; j < DF_STRIP; ++j) {
+    if (j < ng) {
+      int gr = g0 + j;
+      if (MODE == DF_DIAG) {
+        int q = rs + j;
+        if (q >= ng) q -= ng;
+        gr = g0 + q;
+      }
+      const uint2 wa = *reinterpret_cast<const uint2*>(qa + 32 * gr);
+      const uint2 wb = *reinterpret_cast<const uint2*>(qb + 32 * gr);
+      float d[4];
+      mma_group(d, wa, wb, fb[j][0], fb[j][1]);
+      const float2 xa = MODE == DF_SLOT ? suma[gr] : xs[j], xb = MODE == DF_SLOT ? sumb[gr] : xs[j];
+      const float va = MODE == DF_BCAST ? d[0] : (ca ? d[1] : d[0]);
+      const float vb = MODE == DF_BCAST ? d[2] : (cb ? d[3] : d[2]);
+      acc_a += bf16_to_f32(sa[gr]) * (va - xa.x) + bf16_to_f32(ba[gr]) * xa.y;
+      acc_b += bf16_to_f32(sb[gr]) * (vb - xb.x) + bf16_to_f32(bb[gr]) * xb.y;
+    }
+  }
+}
+// Load the strip's activation fragments (column vector f: uint4 per word)
+// and, when given, its group sums into registers, rotated by rs (DIAG).
+__device__ __forceinline__ void df_load_strip(const uint4* f, const float2* sums, int g0, int ng, int rs, int tq,
+                                              uint4 (&fb)[DF_STRIP][2], float2 (&xs)[DF_STRIP]) {
+#pragma unroll
+  for (int j = 0; j < DF_STRIP; ++j) {
+    if (j < ng) {
+      int q = rs + j;
+      if (q >= ng) q -= ng;
+      fb[j][0] = f[8 * (g0 + q) + 2 * tq];
+      fb[j][1] = f[8 * (g0 + q) + 2 * tq + 1];
+      xs[j] = sums ? sums[g0 + q] : make_float2(0.f, 0.f);
+    } else {
+      fb[j][0] = fb[j][1] = make_uint4(0u, 0u, 0u, 0u);
+      xs[j] = make_float2(0.f, 0.f);
+    }
   }
 }
 
@@ -486,6 +602,15 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
   float* selg = reinterpret_cast<float*>(smem + g.m_selg());
   float* red = reinterpret_cast<float*>(smem + g.m_red());
   float* part = reinterpret_cast<float*>(smem + g.m_part());
+  const void** btab = reinterpret_cast<const void**>(smem + g.m_btab());
+  DfCopyS* ctab = reinterpret_cast<DfCopyS*>(smem + g.m_ctab());
+  // per pair: shared-memory offsets of its gate.s, gate.b, up.s, up.b rows
+  // (routed pairs at 0.., shared pairs at DF_MAX_RG_PAIRS..)
+  uint4* ptab = reinterpret_cast<uint4*>(smem + g.m_ptab());
+  int lst[6];                                     // copy-list starts
+  lst[0] = 0;
+#pragma unroll
+  for (int i = 0; i < 5; ++i) lst[i + 1] = lst[i] + df_list_count(g, i);
   const uint32_t sbase = smem_addr(smem);
   const uint32_t bar0 = sbase + g.m_bars();
   float* xs = reinterpret_cast<float*>(smem + g.f_xs());
@@ -509,56 +634,58 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       red_release_gpu(a.counter, 1u);
       const uint64_t t0 = df_clock();
       while (ld_acquire_gpu(a.counter) < bar_target) {
+        __nanosleep(32);
         if (df_clock() - t0 > 2000000000ull) { flag_check(CHECK_WAIT); break; }
       }
       __threadfence();
     }
     __syncthreads();
   };
-  // source address of a copy in layer W (routed slots through the selection)
-  auto src_ptr = [&](const DfLayer& W, const DfCopy& C) -> const uint8_t* {
-    const uint8_t* b;
-    if (C.src < 8) {
-      int e = sel[C.src];
-      if (e < 0 || e >= E) { flag_check(CHECK_EXPERT_ID); e = 0; }
-      b = static_cast<const uint8_t*>(W.blobs[e]);
-    } else if (C.src < DF_SRC_ROUTER) {
-      const int m = (C.src - DF_SRC_SHARED) / 3, arr = (C.src - DF_SRC_SHARED) % 3;
-      b = arr == 0 ? reinterpret_cast<const uint8_t*>(W.sq[m])
-                   : reinterpret_cast<const uint8_t*>(arr == 1 ? W.ss[m] : W.sb[m]);
-    } else {
-      const int arr = C.src - DF_SRC_ROUTER;
-      b = arr == 0 ? reinterpret_cast<const uint8_t*>(W.rq)
-                   : reinterpret_cast<const uint8_t*>(arr == 1 ? W.rs : W.rb);
-    }
-    return b + C.src_off;
-  };
-  // warp-wide issue of the shared gate/up and router-row copies of layer W
-  auto issue_sg = [&](const DfLayer& W) {
-    const int n = df_sg_count(g);
-    for (int e = lane; e < n; e += 32) {
-      const DfCopy C = df_sg_copy(g, e);
-      df_bulk(BAR(C.bar), sbase + C.dst, src_ptr(W, C), C.bytes);
+  // warp-wide: issue copy list `list` of layer W (routed slots through the
+  // selection and the staged blob table), then one arrive on each barrier in [b0, b1)
+  auto issue_list = [&](const DfLayer& W, int list, int b0, int b1) {
+    for (int e = lst[list] + lane; e < lst[list + 1]; e += 32) {
+      const DfCopyS C = ctab[e];
+      const uint8_t* b;
+      if (C.src < 8) {
+        int x = sel[C.src];
+        if (x < 0 || x >= E) { flag_check(CHECK_EXPERT_ID); x = 0; }
+        b = static_cast<const uint8_t*>(btab[x]);
+      } else if (C.src < DF_SRC_ROUTER) {
+        const int m = (C.src - DF_SRC_SHARED) / 3, arr = (C.src - DF_SRC_SHARED) % 3;
+        b = arr == 0 ? reinterpret_cast<const uint8_t*>(W.sq[m])
+                     : reinterpret_cast<const uint8_t*>(arr == 1 ? W.ss[m] : W.sb[m]);
+      } else {
+        const int arr = C.src - DF_SRC_ROUTER;
+        b = arr == 0 ? reinterpret_cast<const uint8_t*>(W.rq)
+                     : reinterpret_cast<const uint8_t*>(arr == 1 ? W.rs : W.rb);
+      }
+      df_bulk(BAR(C.bar), sbase + C.dst, b + C.src_off, C.bytes);
     }
     __syncwarp();
-    if (lane == 0) df_mbar_arrive(BAR(DF_BAR_SG));
+    if (lane < b1 - b0) df_mbar_arrive(BAR(b0 + lane));
     __syncwarp();
   };
-  auto issue_rr = [&](const DfLayer& W) {
-    const int n = df_rr_count(g);
-    for (int e = lane; e < n; e += 32) {
-      const DfCopy C = df_rr_copy(g, e);
-      df_bulk(BAR(C.bar), sbase + C.dst, src_ptr(W, C), C.bytes);
-    }
-    __syncwarp();
-    if (lane == 0) df_mbar_arrive(BAR(DF_BAR_RR));
-    __syncwarp();
-  };
+  auto issue_sg = [&](const DfLayer& W) { issue_list(W, 3, DF_BAR_SG, DF_BAR_SG + 1); };
+  auto issue_rr = [&](const DfLayer& W) { issue_list(W, 4, DF_BAR_RR, DF_BAR_RR + 1); };
 
   // --------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
     for (int i = 0; i < DF_NBARS; ++i) df_mbar_init(BAR(i), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  for (int i = threadIdx.x; i < g.np; i += DF_THREADS)
+    ptab[i] = make_uint4(g.rg_scale(a.off, i, 0), g.rg_scale(a.off, i, 1), g.rg_scale(a.off, i, 2),
+                         g.rg_scale(a.off, i, 3));
+  for (int i = threadIdx.x; i < g.nsp; i += DF_THREADS)
+    ptab[DF_MAX_RG_PAIRS + i] = make_uint4(g.sg_scale(i, 0), g.sg_scale(i, 1), g.sg_scale(i, 2), g.sg_scale(i, 3));
+  // the CTA's copy lists (static: only routed sources change with the selection)
+  for (int e = threadIdx.x; e < lst[5]; e += DF_THREADS) {
+    int list = 0;
+    while (e >= lst[list + 1]) ++list;
+    const DfCopy C = df_list_copy(g, a.off, list, e - lst[list]);
+    ctab[e] = DfCopyS{C.dst, C.bytes, static_cast<uint32_t>(C.src_off), static_cast<uint16_t>(C.src),
+                      static_cast<uint16_t>(C.bar)};
   }
   // every blob pointer is checked (non-null, 16-byte aligned) before any copy
   // reads one; a bad one stops every CTA at the same point
@@ -575,6 +702,10 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
     issue_sg(a.layer[0]);
     issue_rr(a.layer[0]);
   }
+  // blob table and router bias of layer 0 (later layers: staged in phase C)
+  for (int e = threadIdx.x; e < E; e += DF_THREADS) btab[e] = a.layer[0].blobs[e];
+  float bias_c = (c < E && a.layer[0].bias) ? a.layer[0].bias[c] : 0.f;   // used by the router warp
+  __syncthreads();
 
   for (int l = 0; l < a.L; ++l) {
     const DfLayer& W = a.layer[l];
@@ -646,24 +777,27 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
           acc += sc * ((a0 + a1) - 1024.f * sm) + bi * sm;
         }
         acc = warp_sum(acc);
-        if (lane == 0) a.logits[c] = acc + (W.bias ? W.bias[c] : 0.f);
+        if (lane == 0) a.logits[c] = acc + bias_c;
       }
     } else {
-      const int nunits = g.ntS * g.kS;
-      if (nunits > 0) df_mbar_wait(BAR(DF_BAR_SG), par);
-      for (int u = warp; u < nunits; u += DF_WARPS - 1) {
-        const int tile = u / g.kS;
-        int g0, g1;
-        df_kpart(NGH, g.kS, u % g.kS, g0, g1);
+      // warp w < 11: groups [w*NGH/11, (w+1)*NGH/11) of every shared gate/up tile
+      const int s0g = warp * NGH / (DF_WARPS - 1), ng = (warp + 1) * NGH / (DF_WARPS - 1) - s0g;
+      const int rs = ng > 0 ? gq % ng : 0;
+      uint4 fb[DF_STRIP][2];
+      float2 xs2[DF_STRIP];
+      df_load_strip(xf, xsum, s0g, ng, rs, tq, fb, xs2);
+      if (g.ntS > 0) df_mbar_wait(BAR(DF_BAR_SG), par);
+      for (int tile = 0; tile < g.ntS; ++tile) {
         int i = 8 * tile + gq;
         if (i >= g.nsp) i = 8 * tile;
         float acc_a = 0.f, acc_b = 0.f;
-        df_rows<false>(smem + g.sg_row(i, 0) + 8 * tq, smem + g.sg_row(i, 1) + 8 * tq, S16 + g.sg_scale(i, 0) / 2,
-                       S16 + g.sg_scale(i, 1) / 2, S16 + g.sg_scale(i, 2) / 2, S16 + g.sg_scale(i, 3) / 2,
-                       xf + 2 * tq, xsum, xsum, 0, 0, g0, g1, acc_a, acc_b);
-        if (tq == 0) {
-          part[u * 16 + gq] = acc_a;
-          part[u * 16 + 8 + gq] = acc_b;
+        const uint4 sc = ptab[DF_MAX_RG_PAIRS + i];
+        df_strip<DF_DIAG>(smem + g.sg_row(i, 0) + 8 * tq, smem + g.sg_row(i, 1) + 8 * tq, S16 + sc.x / 2,
+                          S16 + sc.y / 2, S16 + sc.z / 2, S16 + sc.w / 2, fb, xs2, nullptr, nullptr, gq & 1, gq & 1,
+                          s0g, ng, rs, acc_a, acc_b);
+        if (tq == (gq >> 1)) {
+          part[g.slot_sg(warp, tile) * 16 + gq] = acc_a;
+          part[g.slot_sg(warp, tile) * 16 + 8 + gq] = acc_b;
         }
       }
     }
@@ -671,9 +805,9 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
     for (int i = threadIdx.x; i < g.nsp; i += DF_THREADS) {
       const int tile = i / 8, r = i % 8;
       float gs = 0.f, us = 0.f;
-      for (int p = 0; p < g.kS; ++p) {
-        gs += part[(tile * g.kS + p) * 16 + r];
-        us += part[(tile * g.kS + p) * 16 + 8 + r];
+      for (int w = 0; w < DF_WARPS - 1; ++w) {
+        gs += part[g.slot_sg(w, tile) * 16 + r];
+        us += part[g.slot_sg(w, tile) * 16 + 8 + r];
       }
       a.act[kI + g.s0 + i] = __float2half_rn(gelu_tanh(gs) * us);
     }
@@ -687,9 +821,13 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
     for (int e = threadIdx.x; e < E; e += DF_THREADS) {
       const float v = lg[e];
       int rank = 0;
-      for (int f = 0; f < E; ++f) {
-        const float w = lg[f];
-        rank += (w > v || (w == v && f < e)) ? 1 : 0;
+      const float4* l4 = reinterpret_cast<const float4*>(lg);
+      for (int f = 0; f < E / 4; ++f) {      // E is a multiple of 8
+        const float4 w = l4[f];
+        rank += (w.x > v || (w.x == v && 4 * f + 0 < e)) ? 1 : 0;
+        rank += (w.y > v || (w.y == v && 4 * f + 1 < e)) ? 1 : 0;
+        rank += (w.z > v || (w.z == v && 4 * f + 2 < e)) ? 1 : 0;
+        rank += (w.w > v || (w.w == v && 4 * f + 3 < e)) ? 1 : 0;
       }
       if (rank < k) { sel[rank] = e; selv[rank] = v; }
     }
@@ -704,68 +842,53 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
         if (c == 0 && a.idx_trace) a.idx_trace[static_cast<size_t>(l) * k + lane] = sel[lane];
         if (c == 0 && a.gates_trace) a.gates_trace[static_cast<size_t>(l) * k + lane] = gj;
       }
-    } else if (warp == 1) {             // routed gate/up rows and windows
-      const int n = df_rg_count(g);
-      for (int e = lane; e < n; e += 32) {
-        const DfCopy C = df_rg_copy(g, a.off, e);
-        df_bulk(BAR(C.bar), sbase + C.dst, src_ptr(W, C), C.bytes);
-      }
-      __syncwarp();
-      if (lane < g.ntR) df_mbar_arrive(BAR(lane));
-      __syncwarp();
-    } else if (warp == 2) {             // routed down rows and windows; the next router row
-      const int n = df_d_count(g);
-      for (int e = lane; e < n; e += 32) {
-        const DfCopy C = df_d_copy(g, a.off, e);
-        df_bulk(BAR(C.bar), sbase + C.dst, src_ptr(W, C), C.bytes);
-      }
-      __syncwarp();
-      if (lane == 0) df_mbar_arrive(BAR(DF_BAR_D));
-      __syncwarp();
+    } else if (warp == DF_WARPS - 1) {  // routed gate/up rows and windows, down rows, the next router row
+      issue_list(W, 0, 0, g.ntR);
+      if (lane == 0) df_stamp_here(a, l, 14);
+      issue_list(W, 1, DF_BAR_D, DF_BAR_D + 1);
       if (l + 1 < a.L) issue_rr(a.layer[l + 1]);
     }
     df_stamp(a, l, 5);
 
     // ------------------------------------------------------ routed gate/up
     {
-      const int nunits = g.ntR * g.kR;
-      for (int u = warp; u < nunits; u += DF_WARPS) {
-        const int tile = u / g.kR;
-        int g0, g1;
-        df_kpart(NGH, g.kR, u % g.kR, g0, g1);
+      // warp w < 11: groups [w*NGH/11, (w+1)*NGH/11) of every routed tile, tile by tile as they land
+      const int s0g = warp * NGH / (DF_WARPS - 1);
+      const int ng = warp < DF_WARPS - 1 ? (warp + 1) * NGH / (DF_WARPS - 1) - s0g : 0;   // warp 11 issues copies
+      const int rs = ng > 0 ? gq % ng : 0;
+      uint4 fb[DF_STRIP][2];
+      float2 xs2[DF_STRIP];
+      df_load_strip(xf, xsum, s0g, ng, rs, tq, fb, xs2);
+      for (int tile = 0; warp < DF_WARPS - 1 && tile < g.ntR; ++tile) {
         df_mbar_wait(BAR(tile), par);
         if (tile != 0) df_mbar_wait(BAR(0), par);      // the scale windows complete on tile 0's barrier
+        if (tile == g.ntR - 1 && threadIdx.x == 0) df_stamp_here(a, l, 15);
         int i = 8 * tile + gq;
         if (i >= g.np) i = 8 * tile;
         float acc_a = 0.f, acc_b = 0.f;
-        df_rows<false>(smem + g.rg_row(i, 0) + 8 * tq, smem + g.rg_row(i, 1) + 8 * tq,
-                       S16 + g.rg_scale(a.off, i, 0) / 2, S16 + g.rg_scale(a.off, i, 1) / 2,
-                       S16 + g.rg_scale(a.off, i, 2) / 2, S16 + g.rg_scale(a.off, i, 3) / 2, xf + 2 * tq, xsum, xsum,
-                       0, 0, g0, g1, acc_a, acc_b);
-        if (tq == 0) {
-          part[u * 16 + gq] = acc_a;
-          part[u * 16 + 8 + gq] = acc_b;
+        const uint4 sc = ptab[i];
+        df_strip<DF_DIAG>(smem + g.rg_row(i, 0) + 8 * tq, smem + g.rg_row(i, 1) + 8 * tq, S16 + sc.x / 2,
+                          S16 + sc.y / 2, S16 + sc.z / 2, S16 + sc.w / 2, fb, xs2, nullptr, nullptr, gq & 1, gq & 1,
+                          s0g, ng, rs, acc_a, acc_b);
+        if (tq == (gq >> 1)) {
+          part[g.slot_rg(warp, tile) * 16 + gq] = acc_a;
+          part[g.slot_rg(warp, tile) * 16 + 8 + gq] = acc_b;
         }
       }
     }
     df_stamp(a, l, 6);
     __syncthreads();                     // the union area is read out
     if (warp == 0) {                     // shared down rows into it
-      const int n = df_sd_count(g);
-      for (int e = lane; e < n; e += 32) {
-        const DfCopy C = df_sd_copy(g, e);
-        df_bulk(BAR(C.bar), sbase + C.dst, src_ptr(W, C), C.bytes);
-      }
-      __syncwarp();
-      if (lane == 0) df_mbar_arrive(BAR(DF_BAR_SD));
-      __syncwarp();
+      issue_list(W, 2, DF_BAR_SD, DF_BAR_SD + 1);
+    } else if (warp == 1) {              // and the next layer's shared gate/up rows after them
+      if (l + 1 < a.L) issue_sg(a.layer[l + 1]);
     }
-    for (int i = threadIdx.x; i < g.np; i += DF_THREADS) {
+    for (int i = threadIdx.x - 64; i >= 0 && i < g.np; i += DF_THREADS - 64) {
       const int tile = i / 8, r = i % 8;
       float gs = 0.f, us = 0.f;
-      for (int p = 0; p < g.kR; ++p) {
-        gs += part[(tile * g.kR + p) * 16 + r];
-        us += part[(tile * g.kR + p) * 16 + 8 + r];
+      for (int w = 0; w < DF_WARPS - 1; ++w) {
+        gs += part[g.slot_rg(w, tile) * 16 + r];
+        us += part[g.slot_rg(w, tile) * 16 + 8 + r];
       }
       a.act[g.r0 + i] = __float2half_rn(gelu_tanh(gs) * us);
     }
@@ -812,15 +935,30 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
         prefetch_l2(static_cast<const uint8_t*>(V.blobs[my_id]) + b0, b1 - b0);
       }
     }
-    // paired activations of the k routed slots and of the shared expert
+    // the next layer's blob table and router bias (this layer's copies are all issued)
+    if (l + 1 < a.L) {
+      for (int e = threadIdx.x; e < E; e += DF_THREADS) btab[e] = a.layer[l + 1].blobs[e];
+      if (warp == DF_WARPS - 1) bias_c = (c < E && a.layer[l + 1].bias) ? a.layer[l + 1].bias[c] : 0.f;
+    }
+    // this CTA's rows of h (only it writes them), read early for the combine
+    const float hpre = threadIdx.x < g.nrow ? __ldcg(a.h + g.o0 + threadIdx.x) : 0.f;
+    // paired activations of the k routed slots and of the shared expert: all
+    // loads first (DF_ACT_ROUNDS words per thread), then pairing
     {
       const int nw = kI / 8 + Is / 8;
-      for (int base = 0; base < nw; base += DF_THREADS) {
-        const int u = base + threadIdx.x;
+      uint4 raws[DF_ACT_ROUNDS];
+#pragma unroll
+      for (int r = 0; r < DF_ACT_ROUNDS; ++r) {
+        const int u = r * DF_THREADS + threadIdx.x;
+        raws[r] = u < nw ? ldcg_v4(a.act + 8 * u) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int r = 0; r < DF_ACT_ROUNDS; ++r) {
+        const int u = r * DF_THREADS + threadIdx.x;
         float off = 0.f, sum = 0.f;
         uint4 p = make_uint4(0u, 0u, 0u, 0u);
         if (u < nw) {
-          const uint4 raw = ldcg_v4(a.act + 8 * u);
+          const uint4 raw = raws[r];
           const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
           float v[8];
 #pragma unroll
@@ -849,43 +987,53 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
     __syncthreads();
     df_stamp(a, l, 9);
     // down tiles: routed rows rho = j * nrow + r (a tile mixes slots; column j
-    // carries slot j's activation), then the shared rows
+    // carries slot j's activation), split dp ways by groups and 12/dp ways by
+    // tiles; then the shared rows, split 12 ways by groups
     {
-      const int nd = g.ntD * g.kD, nunits = nd + g.ntSD * g.kSD;
       const int colslot = gq < k ? gq : 0;
-      for (int u = warp; u < nunits; u += DF_WARPS) {
-        float acc_a = 0.f, acc_b = 0.f;
-        if (u < nd) {
-          const int tile = u / g.kD;
-          int g0, g1;
-          df_kpart(NGI, g.kD, u % g.kD, g0, g1);
-          df_mbar_wait(BAR(DF_BAR_D), par);
-          int ra = 16 * tile + gq, rb = 16 * tile + 8 + gq;
-          const bool va = ra < k * g.nrow, vb = rb < k * g.nrow;
-          if (!va) ra = 0;
-          if (!vb) rb = 0;
-          const int ja = ra / g.nrow, ia = ra % g.nrow, jb = rb / g.nrow, ib = rb % g.nrow;
-          df_rows<true>(smem + g.d_row(ja, ia) + 8 * tq, smem + g.d_row(jb, ib) + 8 * tq,
-                        S16 + g.d_scale(a.off, ja, ia, 0) / 2, S16 + g.d_scale(a.off, ja, ia, 1) / 2,
-                        S16 + g.d_scale(a.off, jb, ib, 0) / 2, S16 + g.d_scale(a.off, jb, ib, 1) / 2,
-                        af + colslot * astride4 + 2 * tq, asum + ja * NGI, asum + jb * NGI, ja & 1, jb & 1, g0, g1,
-                        acc_a, acc_b);
-          if (va && tq == (ja >> 1)) part[u * 16 + gq] = acc_a;
-          if (vb && tq == (jb >> 1)) part[u * 16 + 8 + gq] = acc_b;
-        } else {
-          const int us = u - nd, tile = us / g.kSD;
-          int g0, g1;
-          df_kpart(NGS, g.kSD, us % g.kSD, g0, g1);
-          df_mbar_wait(BAR(DF_BAR_SD), par);
+      {
+        const int dp = g.dp(), tp = DF_WARPS / dp, gp = warp % dp, tw = warp / dp;
+        const int s0g = gp * NGI / dp, ng = (gp + 1) * NGI / dp - s0g;
+        const int t0 = tw * g.ntD / tp, t1 = (tw + 1) * g.ntD / tp;
+        uint4 fb[DF_STRIP][2];
+        float2 xs2[DF_STRIP];
+        df_load_strip(af + colslot * astride4, nullptr, s0g, ng, 0, tq, fb, xs2);
+        if (t1 > t0) df_mbar_wait(BAR(DF_BAR_D), par);
+        const int kn = k * g.nrow;
+        // rows 16 t0 + gq and 16 t0 + 8 + gq as (slot, row), advanced 16 per tile
+        int ja = (16 * t0 + gq) / g.nrow, ia = (16 * t0 + gq) % g.nrow;
+        int jb = (16 * t0 + 8 + gq) / g.nrow, ib = (16 * t0 + 8 + gq) % g.nrow;
+        for (int tile = t0; tile < t1; ++tile) {
+          const bool va = 16 * tile + gq < kn, vb = 16 * tile + 8 + gq < kn;
+          const int xa = va ? ja : 0, ya = va ? ia : 0, xb = vb ? jb : 0, yb = vb ? ib : 0;
+          float acc_a = 0.f, acc_b = 0.f;
+          df_strip<DF_SLOT>(smem + g.d_row(xa, ya) + 8 * tq, smem + g.d_row(xb, yb) + 8 * tq,
+                            S16 + g.d_scale(a.off, xa, ya, 0) / 2, S16 + g.d_scale(a.off, xa, ya, 1) / 2,
+                            S16 + g.d_scale(a.off, xb, yb, 0) / 2, S16 + g.d_scale(a.off, xb, yb, 1) / 2, fb, xs2,
+                            asum + xa * NGI, asum + xb * NGI, xa & 1, xb & 1, s0g, ng, 0, acc_a, acc_b);
+          if (va && tq == (xa >> 1)) part[g.slot_d(gp, tile) * 16 + gq] = acc_a;
+          if (vb && tq == (xb >> 1)) part[g.slot_d(gp, tile) * 16 + 8 + gq] = acc_b;
+          ia += 16; while (ia >= g.nrow) { ia -= g.nrow; ++ja; }
+          ib += 16; while (ib >= g.nrow) { ib -= g.nrow; ++jb; }
+        }
+      }
+      {
+        const int s0g = warp * NGS / DF_WARPS, ng = (warp + 1) * NGS / DF_WARPS - s0g;
+        uint4 fb[DF_STRIP][2];
+        float2 xs2[DF_STRIP];
+        df_load_strip(sf, ssum, s0g, ng, 0, tq, fb, xs2);
+        if (g.ntSD > 0) df_mbar_wait(BAR(DF_BAR_SD), par);
+        for (int tile = 0; tile < g.ntSD; ++tile) {
           int ra = 16 * tile + gq, rb = 16 * tile + 8 + gq;
           if (ra >= g.nrow) ra = 0;
           if (rb >= g.nrow) rb = 0;
-          df_rows<false>(smem + g.sd_row(ra) + 8 * tq, smem + g.sd_row(rb) + 8 * tq, S16 + g.sd_scale(ra, 0) / 2,
-                         S16 + g.sd_scale(ra, 1) / 2, S16 + g.sd_scale(rb, 0) / 2, S16 + g.sd_scale(rb, 1) / 2,
-                         sf + 2 * tq, ssum, ssum, 0, 0, g0, g1, acc_a, acc_b);
+          float acc_a = 0.f, acc_b = 0.f;
+          df_strip<DF_BCAST>(smem + g.sd_row(ra) + 8 * tq, smem + g.sd_row(rb) + 8 * tq, S16 + g.sd_scale(ra, 0) / 2,
+                             S16 + g.sd_scale(ra, 1) / 2, S16 + g.sd_scale(rb, 0) / 2, S16 + g.sd_scale(rb, 1) / 2, fb,
+                             xs2, nullptr, nullptr, 0, 0, s0g, ng, 0, acc_a, acc_b);
           if (tq == 0) {
-            part[u * 16 + gq] = acc_a;
-            part[u * 16 + 8 + gq] = acc_b;
+            part[g.slot_sd(warp, tile) * 16 + gq] = acc_a;
+            part[g.slot_sd(warp, tile) * 16 + 8 + gq] = acc_b;
           }
         }
       }
@@ -893,30 +1041,27 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
     __syncthreads();
     df_stamp(a, l, 10);
     {
-      const int nd = g.ntD * g.kD;
-      for (int r = threadIdx.x; r < g.nrow; r += DF_THREADS) {
+      const int dp = g.dp();
+      for (int r = threadIdx.x; r < g.nrow; r += DF_THREADS) {   // nrow <= DF_THREADS: one row per thread
         float y = 0.f;
         for (int j = 0; j < k; ++j) {
           const int rho = j * g.nrow + r, tile = rho / 16, tr = rho % 16;
           float yj = 0.f;
-          for (int p = 0; p < g.kD; ++p) yj += part[(tile * g.kD + p) * 16 + tr];
+          for (int p = 0; p < dp; ++p) yj += part[g.slot_d(p, tile) * 16 + tr];
           y = fmaf(selg[j], yj, y);
         }
         const int ts = r / 16, tr = r % 16;
         float ysh = 0.f;
-        for (int p = 0; p < g.kSD; ++p) ysh += part[(nd + ts * g.kSD + p) * 16 + tr];
+        for (int w = 0; w < DF_WARPS; ++w) ysh += part[g.slot_sd(w, ts) * 16 + tr];
         y += ysh;
         const int o = g.o0 + r;
-        a.h[o] = __ldcg(a.h + o) + y;
+        a.h[o] = hpre + y;
         if (a.y_trace) a.y_trace[static_cast<size_t>(l) * H + o] = f32_to_bf16(y);
       }
     }
     df_stamp(a, l, 11);
-    if (l + 1 < a.L) {
-      if (warp == 0) issue_sg(a.layer[l + 1]);    // the union area was read out before the combine
-      df_stamp(a, l, 12);
-      grid_sync();
-    }
+    df_stamp(a, l, 12);
+    if (l + 1 < a.L) grid_sync();
     df_stamp(a, l, 13);
   }
 }

@@ -89,7 +89,6 @@ int main(int argc, char** argv) {
     REQUIRE(g.ntR <= DF_BAR_D, "cta %d tiles", c);
     REQUIRE(g.n0 + g.n1 == g.np && g.n1 <= I, "cta %d runs", c);
     // every copy: alignment, inside its source, inside its area
-    struct Group { const char* name; int n; uint32_t lo, hi; };
     auto check_copy = [&](const DfCopy& C, uint32_t lo, uint32_t hi, const char* name) {
       REQUIRE(C.bytes > 0 && C.bytes % 16 == 0 && C.dst % 16 == 0 && C.src_off % 16 == 0,
               "cta %d %s: alignment dst %u bytes %u src %llu", c, name, C.dst, C.bytes,
@@ -131,14 +130,15 @@ int main(int argc, char** argv) {
       REQUIRE(C.bar == DF_BAR_RR, "cta %d rr", c);
       rr.push_back({C.dst, C.dst + C.bytes, "rr"});
     }
-    // copies in flight together
-    std::vector<Range> s1 = rg, s2 = sd, s3 = sg;
+    // copies live together: phase B (routed rows, down rows, the next router
+    // row); from the end of phase B (shared down, the next layer's shared
+    // gate/up, down rows, the next router row)
+    std::vector<Range> s1 = rg, s2 = sd;
     s1.insert(s1.end(), d.begin(), d.end()); s1.insert(s1.end(), rr.begin(), rr.end());
-    s2.insert(s2.end(), d.begin(), d.end()); s2.insert(s2.end(), rr.begin(), rr.end());
-    s3.insert(s3.end(), d.begin(), d.end()); s3.insert(s3.end(), rr.begin(), rr.end());
+    s2.insert(s2.end(), sg.begin(), sg.end()); s2.insert(s2.end(), d.begin(), d.end());
+    s2.insert(s2.end(), rr.begin(), rr.end());
     no_overlap(s1, c, "phase B");
     no_overlap(s2, c, "phase C");
-    no_overlap(s3, c, "next layer");
 
     // reads: the smem byte the kernel reads must hold the source byte it wants
     auto lands = [&](const std::vector<DfCopy>& cs, uint32_t smem, uint32_t n, int src, uint64_t want,
@@ -192,17 +192,26 @@ int main(int argc, char** argv) {
       for (int a = 0; a < 2; ++a)
         lands(crr, g.rr_scale(a), g.sbh, DF_SRC_ROUTER + 1 + a, static_cast<uint64_t>(c) * g.sbh, "rr scale");
     }
-    // K parts cover every group once
-    for (int parts : {g.kS, g.kR}) {
-      int next = 0;
-      for (int p = 0; p < parts; ++p) {
-        int a0, a1;
-        df_kpart(H / 64, parts, p, a0, a1);
-        REQUIRE(a0 == next && a1 > a0, "kpart");
-        next = a1;
+    // the copy table holds every list; list starts agree with the counts
+    {
+      int n = 0;
+      for (int i = 0; i < 5; ++i) {
+        REQUIRE(df_list_start(g, i) == n, "cta %d list start", c);
+        for (int e = 0; e < df_list_count(g, i); ++e)
+          REQUIRE(df_list_copy(g, off, i, e).src_off < (1ull << 32), "cta %d source offset", c);
+        n += df_list_count(g, i);
       }
-      REQUIRE(next == H / 64, "kpart end");
+      REQUIRE(n <= DF_MAX_COPIES, "cta %d: %d copies", c, n);
+      REQUIRE(g.m_ctab() + DF_MAX_COPIES * 16u <= g.m_part() && g.m_ctab() % 16 == 0, "cta %d copy table", c);
     }
+    // partial-sum slots
+    REQUIRE(g.ntS <= g.sg_tiles_max() && g.ntR <= g.rg_tiles_max() && g.ntD <= g.d_tiles_max() &&
+            g.ntSD <= g.sd_tiles_max(), "cta %d tiles beyond the slots", c);
+    REQUIRE(g.slot_sg(DF_WARPS - 2, g.sg_tiles_max() - 1) < g.part_slots() &&
+            g.slot_rg(DF_WARPS - 1, g.rg_tiles_max() - 1) < g.part_slots() &&
+            g.slot_d(g.dp() - 1, g.d_tiles_max() - 1) < g.slot_sd(0, 0) &&
+            g.slot_sd(DF_WARPS - 1, g.sd_tiles_max() - 1) < g.part_slots(), "cta %d partial-sum slots", c);
+    REQUIRE(g.m_part() + g.part_slots() * 64u <= g.total, "cta %d part area", c);
   }
   REQUIRE(pairs == static_cast<long>(k) * I && spairs == Is && rows == H, "coverage %ld %ld %ld", pairs, spairs, rows);
   if (fails) {
