@@ -122,6 +122,133 @@ def load_stack(cfg, device, rank):
     return layers
 
 
+def peaks_tc():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def layer_flops(cfg, T: int) -> float:
+    """Dense FLOPs of one layer on T rows: routed experts (T*k pairs, gate, up
+    and down), shared expert, router."""
+    routed = 2.0 * T * cfg.k * 3 * cfg.I * cfg.H
+    shared = 2.0 * T * 3 * cfg.Is * cfg.H
+    router = 2.0 * T * cfg.E * cfg.H
+    return routed + shared + router
+
+
+def layer_bytes(cfg, distinct: float) -> float:
+    """Weight bytes of one layer touched once: router, shared expert, the distinct routed experts."""
+    router = cfg.E * cfg.H + 2 * 2 * cfg.E * (cfg.H // 64)
+    shared = sum(gen.qmat_bytes(o, i) for o, i in ((cfg.Is, cfg.H), (cfg.Is, cfg.H), (cfg.H, cfg.Is)))
+    return router + shared + distinct * gen.blob_bytes(cfg.H, cfg.I)
+
+
+def run_prefill(M, layers, device, reps: int):
+    """128-row chunk through one layer (the prefill workload's shapes and
+    routing skew); chunk i runs on layer i mod 30 so that weights come from
+    HBM.  One graph replay = one chunk per layer."""
+    import torch
+    cfg = gen.CONFIGS["prefill_1L_128tok"]
+    T, H = cfg.T, cfg.H
+    z = torch.from_numpy(gen.rows(cfg.seed, cfg.row_stream, T, H)).to(device)
+    ws = torch.empty(M.moe_layer_workspace_size(T, H, cfg.I, cfg.Is, cfg.E, cfg.k), dtype=torch.uint8, device=device)
+    ho = torch.empty_like(z)
+    idx = torch.empty((len(layers), T, cfg.k), dtype=torch.int32, device=device)
+
+    def chunk(l):
+        dl = layers[l]
+        M.moe_layer_forward(T, H, cfg.I, cfg.Is, cfg.E, cfg.k, dl.router.c, dl.bias, 0, dl.blob_ptrs, dl.shared_c,
+                            ws, h_in=z, h_out=ho, idx=idx[l])
+    for l in range(len(layers)):
+        chunk(l)
+    torch.cuda.synchronize()
+    M.moe_sync()
+    g = torch.cuda.CUDAGraph()
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        with torch.cuda.graph(g, stream=st):
+            for l in range(len(layers)):
+                chunk(l)
+    torch.cuda.current_stream().wait_stream(st)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    M.moe_sync()
+    n_chunks = reps * len(layers)
+    t = e0.elapsed_time(e1) / 1e3 / n_chunks
+    ids = idx.cpu().numpy()
+    distinct = float(np.mean([len(np.unique(ids[l])) for l in range(len(layers))]))
+    flops, byts = layer_flops(cfg, T), layer_bytes(cfg, distinct)
+    tc, tc_src = peaks_tc()
+    hbm, hbm_src = peaks()
+    del g
+    return {"workload": "prefill_1L_128tok", "value": T / t, "unit": "tokens/s", "us_per_chunk": t * 1e6,
+            "chunks": n_chunks, "distinct_experts_per_chunk": distinct,
+            "tensor": {"achieved_tflops": flops / t / 1e12, "peak": tc, "frac": flops / t / 1e12 / tc,
+                       "peak_source": tc_src, "flops_per_chunk": flops},
+            "hbm": {"achieved_gbs": byts / t / 1e9, "peak": hbm, "frac": byts / t / 1e9 / hbm,
+                    "peak_source": hbm_src, "bytes_per_chunk": byts},
+            "l2": "each chunk on another of 30 layers (8.6 GB of weights per graph replay)"}
+
+
+def run_decode_b64(M, stack, device, reps: int):
+    """64 independent rows per step through the 30 layers (batched-decode
+    workload): one graph replay = one step."""
+    import torch
+    cfg = gen.CONFIGS["decode_30L_b64"]
+    T, H = cfg.T, cfg.H
+    z = torch.from_numpy(gen.rows(cfg.seed, cfg.row_stream, T, H)).to(device)
+    h = torch.empty_like(z)
+    ws = torch.empty(M.moe_decode_workspace_size(T, H, cfg.I, cfg.Is, cfg.E, cfg.k), dtype=torch.uint8, device=device)
+    idx = torch.empty((cfg.layers, T, cfg.k), dtype=torch.int32, device=device)
+
+    def step():
+        h.copy_(z)
+        M.moe_decode_forward(h, cfg.I, cfg.Is, cfg.E, cfg.k, stack, ws, idx_trace=idx)
+    step()
+    torch.cuda.synchronize()
+    M.moe_sync()
+    g = torch.cuda.CUDAGraph()
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        with torch.cuda.graph(g, stream=st):
+            step()
+    torch.cuda.current_stream().wait_stream(st)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    M.moe_sync()
+    t = e0.elapsed_time(e1) / 1e3 / reps
+    ids = idx.cpu().numpy()
+    distinct = float(np.mean([len(np.unique(ids[l])) for l in range(cfg.layers)]))
+    byts = cfg.layers * layer_bytes(cfg, distinct)
+    hbm, hbm_src = peaks()
+    del g
+    return {"workload": "decode_30L_b64", "value": T / t, "unit": "tokens/s", "ms_per_step": t * 1e3, "steps": reps,
+            "distinct_experts_per_layer": distinct,
+            "hbm": {"achieved_gbs": byts / t / 1e9, "peak": hbm, "frac": byts / t / 1e9 / hbm, "peak_source": hbm_src,
+                    "bytes_per_step": byts},
+            "l2": "inputs larger than L2 (every step touches all 30 layers)"}
+
+
 def cpu_baseline_oracle(cfg, n_layers: int, stream: int):
     """Time the fp64 oracle on one token through the first n_layers layers."""
     from oracle import moe_oracle as O
@@ -277,6 +404,10 @@ def run_ours(args, rank, world, local_rank):
     del g
     if rank != 0:
         return
+    extra = {}
+    if not args.no_extra:
+        extra["prefill_128"] = run_prefill(M, layers, device, reps=3)
+        extra["decode_b64"] = run_decode_b64(M, stack, device, reps=5)
     value = whole_job_rate(ms, args.steps, world)
     e2e_val = whole_job_rate(ms_e2e, args.steps, world)
     hbm, src = peaks()
@@ -297,6 +428,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": H * 4, "d2h_bytes_per_step": H * 4},
         "gpu_launches": M.moe_decode_launches(1, cfg.layers) * args.steps,
         "clocks": clocks,
+        **extra,
     }
     if world == 1 and not args.no_cpu_baseline:
         tok_s, cores, dt = cpu_baseline_oracle(cfg, 6, 999)
@@ -312,6 +444,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the prefill and batched-decode lines")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
