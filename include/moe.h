@@ -171,7 +171,11 @@ MOE_API int moe_set_gemv_max_rows(int rows);
 /* A6 — shared expert on every row.
  *   shared  host array of 3 q-matrices: gate [Is,H], up [Is,H], down [H,Is]
  *   ysh     fp32 [T,H] (device)
- *   ws      device workspace of at least moe_shared_workspace_size(T,H,Is) bytes */
+ *   ws      device workspace of at least moe_shared_workspace_size(T,H,Is) bytes
+ * With more rows than the GEMV threshold (moe_set_gemv_max_rows) and
+ * H % 128 == 0, H, Is <= 4096, the shared expert runs on the tensor-core
+ * grouped GEMM as one expert whose bucket holds every row; otherwise on the
+ * GEMV kernels. */
 MOE_API size_t moe_shared_workspace_size(int T, int H, int Is);
 MOE_API int moe_shared_forward(const uint16_t* x, int T, int H, int Is, const moe_qmat* shared,
                        float* ysh, void* ws, size_t ws_bytes, void* stream);

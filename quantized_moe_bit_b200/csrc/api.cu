@@ -229,8 +229,10 @@ int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, int k, con
 }
 
 size_t moe_shared_workspace_size(int T, int H, int Is) {
-  (void)H;
-  return align_up(static_cast<size_t>(T) * Is * sizeof(__half));
+  // fp16 activation [T, Is]; for the tensor-core path also fp16 x [T, H] and
+  // the one-expert bucket list (offsets[2], active[1], n_active, pairs[T])
+  return align_up(static_cast<size_t>(T) * Is * sizeof(__half)) + align_up(static_cast<size_t>(T) * H * sizeof(__half)) +
+         3 * align_up(16) + align_up(static_cast<size_t>(T) * 4);
 }
 
 int moe_shared_forward(const uint16_t* x, int T, int H, int Is, const moe_qmat* sh, float* ysh, void* ws,
@@ -249,6 +251,37 @@ int moe_shared_forward(const uint16_t* x, int T, int H, int Is, const moe_qmat* 
     return fail(MOE_ERR_INVALID_ARG, "moe_shared_forward: workspace too small");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   __half* act = static_cast<__half*>(ws);
+  // several rows: the three matrices on the tensor cores as one expert whose
+  // bucket is every row (same kernel and arithmetic as the routed buckets)
+  if (T > g_gemv_max_rows && H % 128 == 0 && H <= 4096 && Is <= 4096) {
+    char* p = static_cast<char*>(ws) + align_up(static_cast<size_t>(T) * Is * sizeof(__half));
+    __half* xh = reinterpret_cast<__half*>(p);
+    p += align_up(static_cast<size_t>(T) * H * sizeof(__half));
+    int32_t* offsets = reinterpret_cast<int32_t*>(p); p += align_up(16);
+    int32_t* active = reinterpret_cast<int32_t*>(p); p += align_up(16);
+    int32_t* n_active = reinterpret_cast<int32_t*>(p); p += align_up(16);
+    int32_t* pairs = reinterpret_cast<int32_t*>(p);
+    k_one_bucket<<<(T + 255) / 256 < 64 ? (T + 255) / 256 : 64, 256, 0, s>>>(T, offsets, pairs, active, n_active);
+    if ((st = launch_check("k_one_bucket"))) return st;
+    const size_t n8 = static_cast<size_t>(T) * H / 8;
+    k_to_f16<<<static_cast<int>((n8 + 255) / 256 < 1024 ? (n8 + 255) / 256 : 1024), 256, 0, s>>>(x, n8, xh);
+    if ((st = launch_check("k_to_f16(shared)"))) return st;
+    TcArgs ta{};
+    ta.mode = 0; ta.xh = xh; ta.T = T; ta.H = H; ta.I = Is; ta.E = 1; ta.k = 1;
+    ta.blob_ptrs = nullptr;
+    for (int m = 0; m < 3; ++m) {
+      ta.mq[m] = reinterpret_cast<const uint8_t*>(sh[m].q); ta.ms[m] = sh[m].s; ta.mb[m] = sh[m].b;
+    }
+    ta.offsets = offsets; ta.pairs = pairs; ta.active = active; ta.n_active = n_active;
+    ta.max_rows = 0;
+    ta.act_out = act; ta.act_in = act; ta.y_out = ysh;
+    if ((st = set_smem(reinterpret_cast<const void*>(k_expert_tc), TC_SMEM))) return st;
+    k_expert_tc<<<dim3(Is / 64, 1), TC_THREADS, TC_SMEM, s>>>(ta);
+    if ((st = launch_check("k_expert_tc(shared gate/up)"))) return st;
+    ta.mode = 1;
+    k_expert_tc<<<dim3(H / 128, 1), TC_THREADS, TC_SMEM, s>>>(ta);
+    return launch_check("k_expert_tc(shared down)");
+  }
   GateUpArgs g{};
   g.x = x; g.T = T; g.H = H; g.I = Is; g.E = 1; g.k = 1; g.max_rows = 1 << 30;
   g.gq = sh[0].q; g.gs = sh[0].s; g.gb = sh[0].b;

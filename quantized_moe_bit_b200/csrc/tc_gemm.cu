@@ -47,7 +47,10 @@ struct TcArgs {
   const __half* xh;               // mode 0: fp16 [T, H] (the layer input, converted)
   const __half* act_in;           // mode 1: fp16 [T*k, I] (bucket order)
   int T, H, I, E, k;
-  const void* const* blob_ptrs;
+  const void* const* blob_ptrs;   // routed: device [E] blob pointers (matrices at off[]); null: use mq/ms/mb
+  const uint8_t* mq[3];           // one expert given as three q-matrices (gate, up, down), e.g. the shared expert
+  const uint16_t* ms[3];
+  const uint16_t* mb[3];
   const int32_t* offsets;
   const int32_t* pairs;
   const int32_t* active;
@@ -106,6 +109,18 @@ __global__ void k_to_f16(const uint16_t* __restrict__ x, size_t n8, __half* __re
   }
 }
 
+// The bucket list of one expert that serves all T rows: offsets {0, T},
+// active {0}, n_active 1, pairs 0..T-1 (row t, pair width 1).
+__global__ void k_one_bucket(int T, int32_t* offsets, int32_t* pairs, int32_t* active, int32_t* n_active) {
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x) pairs[t] = t;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    offsets[0] = 0;
+    offsets[1] = T;
+    active[0] = 0;
+    *n_active = 1;
+  }
+}
+
 __global__ void __launch_bounds__(TC_THREADS, 1) k_expert_tc(TcArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem =
@@ -127,7 +142,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_expert_tc(TcArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = a.mode == 0 ? a.H : a.I;
   const int nkb = K / TC_BK;
-  const uint8_t* blob = static_cast<const uint8_t*>(a.blob_ptrs[e]);
+  const uint8_t* blob = a.blob_ptrs ? static_cast<const uint8_t*>(a.blob_ptrs[e]) : nullptr;
+  auto mat_q = [&](int mat) { return blob ? blob + a.off[3 * mat] : a.mq[mat]; };
+  auto mat_s = [&](int mat) {
+    return blob ? reinterpret_cast<const uint16_t*>(blob + a.off[3 * mat + 1]) : a.ms[mat];
+  };
+  auto mat_b = [&](int mat) {
+    return blob ? reinterpret_cast<const uint16_t*>(blob + a.off[3 * mat + 2]) : a.mb[mat];
+  };
   const int m0 = blockIdx.x * (a.mode == 0 ? 64 : 128);
 
   const uint32_t bar0 = tc::smem_u32(bars);
@@ -156,7 +178,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_expert_tc(TcArgs a) {
     int grow, mat;
     if (a.mode == 0) { mat = r & 1; grow = m0 + (r >> 1); }
     else { mat = 2; grow = m0 + r; }
-    qrow = blob + a.off[3 * mat] + static_cast<size_t>(grow) * (K / 2);
+    qrow = mat_q(mat) + static_cast<size_t>(grow) * (K / 2);
   }
   // S/B table of the tile: 128 rows x (K/64) groups, packed as S | B << 16
   for (int i = t; i < TC_BM * nkb; i += TC_THREADS) {
@@ -164,8 +186,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_expert_tc(TcArgs a) {
     int grow, mat;
     if (a.mode == 0) { mat = rr & 1; grow = m0 + (rr >> 1); }
     else { mat = 2; grow = m0 + rr; }
-    const uint16_t* sp = reinterpret_cast<const uint16_t*>(blob + a.off[3 * mat + 1]) + static_cast<size_t>(grow) * nkb + gg;
-    const uint16_t* bp = reinterpret_cast<const uint16_t*>(blob + a.off[3 * mat + 2]) + static_cast<size_t>(grow) * nkb + gg;
+    const uint16_t* sp = mat_s(mat) + static_cast<size_t>(grow) * nkb + gg;
+    const uint16_t* bp = mat_b(mat) + static_cast<size_t>(grow) * nkb + gg;
     sSB[rr * TC_MAX_GROUPS + gg] = static_cast<uint32_t>(ldg_u16(sp)) | (static_cast<uint32_t>(ldg_u16(bp)) << 16);
   }
   tc::tc_fence_before();
