@@ -17,6 +17,7 @@ Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -49,6 +50,24 @@ def peaks():
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM, "fallback"
+
+
+# DRAM read + write of the decode kernel measured by ncu on 3 full-size
+# layers of this workload, per layer; valid only for the kernel source the
+# capture was taken on (sha256 prefix of decode_fused.cu).
+DECODE_TRAFFIC = {"source_sha256_prefix": "7ed8f2d9bd6bd613", "bytes_per_layer": 38.8166e6}
+
+
+def decode_traffic(layers: int):
+    src = os.path.join(ROOT, "quantized_moe_bit_b200", "csrc", "decode_fused.cu")
+    try:
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    if sha != DECODE_TRAFFIC["source_sha256_prefix"]:
+        return None
+    return DECODE_TRAFFIC["bytes_per_layer"] * layers
 
 
 def step_bytes(cfg, distinct_per_layer: float) -> float:
@@ -423,7 +442,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "inputs larger than L2 (1.1 GB of weights per step)"},
         "roofline": {"bound": "hbm", "kernel": "k_decode_b1 (one persistent launch per step)",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "peak_source": src, "traffic": None, "bytes_per_step": bytes_step,
+                     "peak_source": src, "traffic": decode_traffic(cfg.layers), "bytes_per_step": bytes_step,
                      "distinct_experts_per_layer": distinct},
         "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": H * 4, "d2h_bytes_per_step": H * 4},
         "gpu_launches": M.moe_decode_launches(1, cfg.layers) * args.steps,
