@@ -133,9 +133,17 @@ MOE_API int moe_bucket(const int32_t* idx, int T, int k, int E, int32_t* offsets
  *   ws         device workspace of at least moe_expert_workspace_size(T,H,I,k) bytes
  * Each expert runs on the decode GEMV kernels (CUDA cores) when its bucket has
  * at most gemv_max_rows rows (moe_set_gemv_max_rows; default 2) and on the
- * tcgen05 grouped GEMM otherwise.  The choice depends only on the bucket's
- * row count.  The activation between the two projections is held in fp16. */
+ * tcgen05 grouped GEMM otherwise.  With a workspace of at least
+ * moe_expert_workspace_size_mma(T,H,I,k) bytes (and the grouped kernel on,
+ * moe_set_grouped_mma), buckets of gemv_max_rows+1 .. 32 rows run on the
+ * grouped mma.sync kernel instead of the tcgen05 GEMM (room for the paired
+ * activation rows).  The choice depends only on the bucket's row count and
+ * the workspace given.  The activation between the projections is fp16. */
 MOE_API size_t moe_expert_workspace_size(int T, int H, int I, int k);
+MOE_API size_t moe_expert_workspace_size_mma(int T, int H, int I, int k);
+/* Grouped mma.sync kernel for buckets of a few rows: 1 on, 0 off (default;
+ * on this B200 it measured slower than the tcgen05 GEMM for 3..32-row buckets). */
+MOE_API int moe_set_grouped_mma(int enable);
 MOE_API int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, int k,
                        const void* const* blob_ptrs, const int32_t* offsets,
                        const int32_t* pairs, const int32_t* active,

@@ -43,6 +43,8 @@ SIGNATURES = {
     "moe_router_topk": (_I, [_P, _I, _I, C.POINTER(moe_qmat), _P, _I, _I, _I, _P, _P, _P, _P]),
     "moe_bucket": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P]),
     "moe_expert_workspace_size": (_Z, [_I, _I, _I, _I]),
+    "moe_expert_workspace_size_mma": (_Z, [_I, _I, _I, _I]),
+    "moe_set_grouped_mma": (_I, [_I]),
     "moe_expert_forward": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _Z, _P]),
     "moe_expert_forward_noalloc": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "moe_set_gemv_max_rows": (_I, [_I]),

@@ -50,6 +50,14 @@ def moe_expert_workspace_size(T: int, H: int, I: int, k: int) -> int:
     return lib().moe_expert_workspace_size(T, H, I, k)
 
 
+def moe_expert_workspace_size_mma(T: int, H: int, I: int, k: int) -> int:
+    return lib().moe_expert_workspace_size_mma(T, H, I, k)
+
+
+def moe_set_grouped_mma(enable: bool):
+    check(lib().moe_set_grouped_mma(1 if enable else 0))
+
+
 def moe_expert_forward(x, I: int, E: int, k: int, blob_ptrs, offsets, pairs, active, n_active, y_pairs,
                        ws, stream=None):
     T, H = x.shape

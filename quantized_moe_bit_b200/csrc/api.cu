@@ -7,11 +7,26 @@
 #include "kernels.cuh"
 #include "tc_gemm.cu"
 #include "decode_fused.cu"
+#include "grouped_mma.cu"
 
 namespace moe {
 
 static thread_local char g_err[512] = "";
 static int g_gemv_max_rows = 2;
+static int g_grouped_mma = 0;            // buckets of 3..32 rows on the grouped mma.sync kernel (off: measured slower)
+
+// CTAs of the persistent grouped kernel: one per SM (cached per device).
+static int grouped_grid() {
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int nsm = 0;
+    if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0) nsm = 148;
+    cached[dev] = nsm;
+  }
+  return cached[dev];
+}
 static int g_decode_fused = 1;
 static int g_decode_spec = 0;
 static int g_decode_prefetch = 0;
@@ -112,6 +127,11 @@ size_t moe_blob_bytes(int H, int I, size_t* offsets9) {
   return 3 * (static_cast<size_t>(I) * H / 2 + static_cast<size_t>(I) * (H / 64) * 4);
 }
 
+int moe_set_grouped_mma(int enable) {
+  g_grouped_mma = enable ? 1 : 0;
+  return MOE_OK;
+}
+
 int moe_set_gemv_max_rows(int rows) {
   if (rows < 0) return fail(MOE_ERR_INVALID_ARG, "gemv_max_rows must be >= 0");
   g_gemv_max_rows = rows;
@@ -163,6 +183,18 @@ size_t moe_expert_workspace_size(int T, int H, int I, int k) {
   return align_up(static_cast<size_t>(T) * k * I * sizeof(__half)) + align_up(static_cast<size_t>(T) * H * sizeof(__half));
 }
 
+// Paired activation rows (x and the gate/up activation) for the grouped
+// mma.sync kernel: fp16 pairs [rows, K] plus fp32 group sums [rows, K/64] x 2.
+static size_t mma_extra_bytes(int T, int H, int I, int k) {
+  const size_t tk = static_cast<size_t>(T) * k;
+  return align_up(static_cast<size_t>(T) * H * 2) + align_up(static_cast<size_t>(T) * (H / 64) * 8) +
+         align_up(tk * I * 2) + align_up(tk * (I / 64) * 8) + align_up(8);   // + the two work counters
+}
+
+size_t moe_expert_workspace_size_mma(int T, int H, int I, int k) {
+  return moe_expert_workspace_size(T, H, I, k) + mma_extra_bytes(T, H, I, k);
+}
+
 int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, int k, const void* const* blob_ptrs,
                        const int32_t* offsets, const int32_t* pairs, const int32_t* active,
                        const int32_t* n_active, float* y_pairs, void* ws, size_t ws_bytes, void* stream) {
@@ -180,9 +212,39 @@ int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, int k, con
   __half* xh = reinterpret_cast<__half*>(static_cast<char*>(ws) + align_up(static_cast<size_t>(T) * k * I * sizeof(__half)));
   const int maxA = T * k < E ? T * k : E;
   // Buckets of at most gemv_max_rows rows go to the GEMV kernels, larger ones
-  // to the tensor-core kernel (shapes it supports: H % 128 == 0, H, I <= 4096).
+  // to the tensor-core kernel (shapes it supports: H % 128 == 0, H, I <= 4096);
+  // with the larger workspace, buckets of up to GM_NMAX rows go to the grouped
+  // mma.sync kernel instead.
   const bool tc = T > g_gemv_max_rows && H % 128 == 0 && H <= 4096 && I <= 4096;
   const int gemv_rows = tc ? g_gemv_max_rows : (1 << 30);
+  const bool mma = tc && g_grouped_mma && grouped_mma_ok(H, I) &&
+                   ws_bytes >= moe_expert_workspace_size_mma(T, H, I, k);
+  const int tc_min = mma ? GM_NMAX : g_gemv_max_rows;     // the tensor-core kernel takes buckets above this
+  char* xw = static_cast<char*>(ws) + moe_expert_workspace_size(T, H, I, k);
+  uint4* xP = reinterpret_cast<uint4*>(xw);
+  float2* xS = reinterpret_cast<float2*>(xw + align_up(static_cast<size_t>(T) * H * 2));
+  uint4* aP = reinterpret_cast<uint4*>(xw + align_up(static_cast<size_t>(T) * H * 2) +
+                                       align_up(static_cast<size_t>(T) * (H / 64) * 8));
+  float2* aS = reinterpret_cast<float2*>(reinterpret_cast<char*>(aP) + align_up(static_cast<size_t>(T) * k * I * 2));
+  unsigned* queues = reinterpret_cast<unsigned*>(reinterpret_cast<char*>(aS) +
+                                                 align_up(static_cast<size_t>(T) * k * (I / 64) * 8));
+  GmArgs gm{};
+  if (mma) {
+    const size_t gsm = grouped_mma_smem(H, I);
+    if ((st = set_smem(reinterpret_cast<const void*>(k_group_mma), gsm))) return st;
+    const long nw = static_cast<long>(T) * (H / 8);
+    k_pair_rows<<<static_cast<int>((nw + 255) / 256 < 1024 ? (nw + 255) / 256 : 1024), 256, 0, s>>>(x, 1, T, H, xP, xS);
+    if ((st = launch_check("k_pair_rows(x)"))) return st;
+    gm.mode = 0; gm.P = xP; gm.S = xS; gm.T = T; gm.H = H; gm.I = I; gm.E = E; gm.k = k;
+    gm.blob_ptrs = blob_ptrs; blob_offsets(H, I, gm.off);
+    gm.offsets = offsets; gm.pairs = pairs; gm.active = active; gm.n_active = n_active;
+    gm.lo = g_gemv_max_rows; gm.hi = GM_NMAX;
+    gm.act_out = static_cast<__half*>(ws); gm.y_out = y_pairs;
+    if ((st = cuda_check(cudaMemsetAsync(queues, 0, 8, s), "zero work counters"))) return st;
+    gm.queue = queues;
+    k_group_mma<<<grouped_grid(), GM_THREADS, gsm, s>>>(gm);
+    if ((st = launch_check("k_group_mma(gate/up)"))) return st;
+  }
 
   GateUpArgs g{};
   g.x = x; g.T = T; g.H = H; g.I = I; g.E = E; g.k = k;
@@ -202,7 +264,7 @@ int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, int k, con
     if ((st = launch_check("k_to_f16"))) return st;
     ta.mode = 0; ta.xh = xh; ta.T = T; ta.H = H; ta.I = I; ta.E = E; ta.k = k;
     ta.blob_ptrs = blob_ptrs; ta.offsets = offsets; ta.pairs = pairs; ta.active = active; ta.n_active = n_active;
-    ta.max_rows = g_gemv_max_rows;
+    ta.max_rows = tc_min;
     blob_offsets(H, I, ta.off);
     ta.act_out = act; ta.act_in = act; ta.y_out = y_pairs;
     if ((st = set_smem(reinterpret_cast<const void*>(k_expert_tc), TC_SMEM))) return st;
@@ -210,6 +272,15 @@ int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, int k, con
     if ((st = launch_check("k_expert_tc(gate/up)"))) return st;
   }
 
+  if (mma) {
+    const long nw = static_cast<long>(T) * k * (I / 8);
+    k_pair_rows<<<static_cast<int>((nw + 255) / 256 < 1024 ? (nw + 255) / 256 : 1024), 256, 0, s>>>(
+        reinterpret_cast<const uint16_t*>(act), 0, T * k, I, aP, aS);
+    if ((st = launch_check("k_pair_rows(act)"))) return st;
+    gm.mode = 1; gm.P = aP; gm.S = aS; gm.queue = queues + 1;
+    k_group_mma<<<grouped_grid(), GM_THREADS, grouped_mma_smem(H, I), s>>>(gm);
+    if ((st = launch_check("k_group_mma(down)"))) return st;
+  }
   DownArgs d{};
   d.act = act; d.T = T; d.H = H; d.I = I; d.E = E; d.k = k;
   d.blob_ptrs = blob_ptrs; d.offsets = offsets; d.pairs = pairs; d.active = active; d.n_active = n_active;
@@ -321,7 +392,7 @@ size_t moe_layer_workspace_size(int T, int H, int I, int Is, int E, int k) {
   n += align_up(4);                                     // n_active
   n += align_up(static_cast<size_t>(T) * k * H * 4);    // y_pairs
   n += align_up(static_cast<size_t>(T) * H * 4);        // ysh
-  n += moe_expert_workspace_size(T, H, I, k);
+  n += moe_expert_workspace_size_mma(T, H, I, k);
   n += moe_shared_workspace_size(T, H, Is);
   return n;
 }
@@ -348,7 +419,7 @@ int moe_layer_forward(const float* h_in, float* h_out, const uint16_t* x_in, int
   int32_t* n_active = reinterpret_cast<int32_t*>(take(4));
   float* y_pairs = reinterpret_cast<float*>(take(static_cast<size_t>(T) * k * H * 4));
   float* ysh = reinterpret_cast<float*>(take(static_cast<size_t>(T) * H * 4));
-  const size_t ews = moe_expert_workspace_size(T, H, I, k);
+  const size_t ews = moe_expert_workspace_size_mma(T, H, I, k);
   void* ew = take(ews);
   const size_t sws = moe_shared_workspace_size(T, H, Is);
   void* sw = take(sws);

@@ -316,7 +316,7 @@ MOE_API int moe_streamed_layer_forward(moe_lfu* h, int layer, float* hres, int T
   int32_t* n_active = reinterpret_cast<int32_t*>(take(4));
   float* y_pairs = reinterpret_cast<float*>(take(static_cast<size_t>(T) * k * H * 4));
   float* ysh = reinterpret_cast<float*>(take(static_cast<size_t>(T) * H * 4));
-  const size_t ews = moe_expert_workspace_size(T, H, I, k);
+  const size_t ews = moe_expert_workspace_size_mma(T, H, I, k);   // the same expert path as moe_layer_forward
   void* ew = take(ews);
   const size_t sws = moe_shared_workspace_size(T, H, Is);
   void* sw = take(sws);

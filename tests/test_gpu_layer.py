@@ -30,8 +30,10 @@ def _bits(t):
     return _np(t.view(torch.int16)).view(np.uint16)
 
 
-def _run_calls(M, hl, dl, z, stream_check=True):
-    """Run A0..A7 through the separate calls; return every intermediate."""
+def _run_calls(M, hl, dl, z, stream_check=True, mma=False):
+    """Run A0..A7 through the separate calls; return every intermediate.
+    mma: give moe_expert_forward the larger workspace that enables the
+    grouped mma.sync kernel for buckets of 3..32 rows."""
     c = hl.cfg
     T = z.shape[0]
     dev = "cuda"
@@ -48,7 +50,8 @@ def _run_calls(M, hl, dl, z, stream_check=True):
     n_active = torch.empty(1, dtype=torch.int32, device=dev)
     M.moe_bucket(idx, c.E, offs, pairs, active, n_active)
     yp = torch.empty((T * c.k, c.H), dtype=torch.float32, device=dev)
-    ws = torch.empty(M.moe_expert_workspace_size(T, c.H, c.I, c.k), dtype=torch.uint8, device=dev)
+    wsz = (M.moe_expert_workspace_size_mma if mma else M.moe_expert_workspace_size)(T, c.H, c.I, c.k)
+    ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
     M.moe_expert_forward(x, c.I, c.E, c.k, dl.blob_ptrs, offs, pairs, active, n_active, yp, ws)
     ysh = torch.empty((T, c.H), dtype=torch.float32, device=dev)
     wss = torch.empty(M.moe_shared_workspace_size(T, c.H, c.Is), dtype=torch.uint8, device=dev)
@@ -108,7 +111,7 @@ def test_layer_forward_matches_calls_and_is_deterministic(M):
     hl = HostLayer(cfg, 0)
     dl = hl.upload()
     z = gen.rows(cfg.seed, 1000, cfg.T, cfg.H)
-    g = _run_calls(M, hl, dl, z)
+    g = _run_calls(M, hl, dl, z, mma=True)      # the layer call's workspace enables the grouped kernel too
     c = cfg
     outs = []
     for _ in range(2):
@@ -174,3 +177,39 @@ def test_prefill_128_full(M, gemv_rows, max_rows):
     z = gen.rows(cfg.seed, 1000, cfg.T, cfg.H, accept=gap_ok_predicate(hl))
     g = _run_calls(M, hl, hl.upload(), z)
     _check_all(hl, z, g)
+
+
+@pytest.fixture
+def grouped(M):
+    M.moe_set_grouped_mma(True)
+    yield
+    M.moe_set_grouped_mma(False)
+
+
+@pytest.mark.parametrize("T", [9, 37, 130])
+def test_grouped_mma_tiny(M, grouped, T):
+    """Buckets of 3..32 rows on the grouped mma.sync kernel (T = 130 also
+    sends buckets above 32 rows to the tensor-core GEMM)."""
+    cfg = tiny_config("prefill_1L_128tok", T=T)
+    hl = HostLayer(cfg, 0)
+    z = gen.rows(cfg.seed, 1000, T, cfg.H, accept=gap_ok_predicate(hl))
+    g = _run_calls(M, hl, hl.upload(), z, mma=True)
+    _check_all(hl, z, g)
+
+
+def test_grouped_mma_prefill_128_full(M):
+    """The 128-row prefill chunk at full size with the grouped kernel (most
+    of its ~88 buckets have 3..32 rows), and the same chunk without it."""
+    cfg = CONFIGS["prefill_1L_128tok"]
+    hl = HostLayer(cfg, 0)
+    dl = hl.upload()
+    z = gen.rows(cfg.seed, 1000, cfg.T, cfg.H, accept=gap_ok_predicate(hl))
+    try:
+        M.moe_set_grouped_mma(True)
+        g = _run_calls(M, hl, dl, z, mma=True)
+    finally:
+        M.moe_set_grouped_mma(False)
+    _check_all(hl, z, g)
+    g2 = _run_calls(M, hl, dl, z, mma=True)
+    _check_all(hl, z, g2)
+    assert np.array_equal(g["idx"], g2["idx"])
