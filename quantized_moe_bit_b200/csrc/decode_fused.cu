@@ -547,6 +547,38 @@ __device__ __forceinline__ void df_strip(const uint8_t* qa, const uint8_t* qb, c
     }
   }
 }
+// DIAG strip with the lane's rotated group indices precomputed (gr[j] =
+// g0 + (rs + j) mod ng); FULL: the strip holds DF_STRIP groups (no guards).
+template <bool FULL>
+__device__ __forceinline__ void df_strip_diag(const uint8_t* qa, const uint8_t* qb, const uint16_t* sa,
+                                              const uint16_t* ba, const uint16_t* sb, const uint16_t* bb,
+                                              const uint4 (&fb)[DF_STRIP][2], const float2 (&xs)[DF_STRIP],
+                                              const int (&gr)[DF_STRIP], int odd, int ng, float& acc_a,
+                                              float& acc_b) {
+#pragma unroll
+  for (int j = 0; j < DF_STRIP; ++j) {
+    if (FULL || j < ng) {
+      const uint2 wa = *reinterpret_cast<const uint2*>(qa + 32 * gr[j]);
+      const uint2 wb = *reinterpret_cast<const uint2*>(qb + 32 * gr[j]);
+      float d[4];
+      mma_group(d, wa, wb, fb[j][0], fb[j][1]);
+      const float va = odd ? d[1] : d[0];
+      const float vb = odd ? d[3] : d[2];
+      acc_a += bf16_to_f32(sa[gr[j]]) * (va - xs[j].x) + bf16_to_f32(ba[gr[j]]) * xs[j].y;
+      acc_b += bf16_to_f32(sb[gr[j]]) * (vb - xs[j].x) + bf16_to_f32(bb[gr[j]]) * xs[j].y;
+    }
+  }
+}
+// The lane's rotated group indices of a DIAG strip.
+__device__ __forceinline__ void df_strip_groups(int g0, int ng, int rs, int (&gr)[DF_STRIP]) {
+#pragma unroll
+  for (int j = 0; j < DF_STRIP; ++j) {
+    int q = rs + j;
+    if (ng > 0) q %= ng;
+    gr[j] = g0 + q;
+  }
+}
+
 // Load the strip's activation fragments (column vector f: uint4 per word)
 // and, when given, its group sums into registers, rotated by rs (DIAG).
 __device__ __forceinline__ void df_load_strip(const uint4* f, const float2* sums, int g0, int ng, int rs, int tq,
@@ -786,15 +818,16 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       uint4 fb[DF_STRIP][2];
       float2 xs2[DF_STRIP];
       df_load_strip(xf, xsum, s0g, ng, rs, tq, fb, xs2);
+      int grs[DF_STRIP];
+      df_strip_groups(s0g, ng, rs, grs);
       if (g.ntS > 0) df_mbar_wait(BAR(DF_BAR_SG), par);
       for (int tile = 0; tile < g.ntS; ++tile) {
         int i = 8 * tile + gq;
         if (i >= g.nsp) i = 8 * tile;
         float acc_a = 0.f, acc_b = 0.f;
         const uint4 sc = ptab[DF_MAX_RG_PAIRS + i];
-        df_strip<DF_DIAG>(smem + g.sg_row(i, 0) + 8 * tq, smem + g.sg_row(i, 1) + 8 * tq, S16 + sc.x / 2,
-                          S16 + sc.y / 2, S16 + sc.z / 2, S16 + sc.w / 2, fb, xs2, nullptr, nullptr, gq & 1, gq & 1,
-                          s0g, ng, rs, acc_a, acc_b);
+        df_strip_diag<false>(smem + g.sg_row(i, 0) + 8 * tq, smem + g.sg_row(i, 1) + 8 * tq, S16 + sc.x / 2,
+                               S16 + sc.y / 2, S16 + sc.z / 2, S16 + sc.w / 2, fb, xs2, grs, gq & 1, ng, acc_a, acc_b);
         if (tq == (gq >> 1)) {
           part[g.slot_sg(warp, tile) * 16 + gq] = acc_a;
           part[g.slot_sg(warp, tile) * 16 + 8 + gq] = acc_b;
@@ -859,6 +892,8 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       uint4 fb[DF_STRIP][2];
       float2 xs2[DF_STRIP];
       df_load_strip(xf, xsum, s0g, ng, rs, tq, fb, xs2);
+      int grs[DF_STRIP];
+      df_strip_groups(s0g, ng, rs, grs);
       for (int tile = 0; warp < DF_WARPS - 1 && tile < g.ntR; ++tile) {
         df_mbar_wait(BAR(tile), par);
         if (tile != 0) df_mbar_wait(BAR(0), par);      // the scale windows complete on tile 0's barrier
@@ -867,9 +902,8 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
         if (i >= g.np) i = 8 * tile;
         float acc_a = 0.f, acc_b = 0.f;
         const uint4 sc = ptab[i];
-        df_strip<DF_DIAG>(smem + g.rg_row(i, 0) + 8 * tq, smem + g.rg_row(i, 1) + 8 * tq, S16 + sc.x / 2,
-                          S16 + sc.y / 2, S16 + sc.z / 2, S16 + sc.w / 2, fb, xs2, nullptr, nullptr, gq & 1, gq & 1,
-                          s0g, ng, rs, acc_a, acc_b);
+        df_strip_diag<false>(smem + g.rg_row(i, 0) + 8 * tq, smem + g.rg_row(i, 1) + 8 * tq, S16 + sc.x / 2,
+                               S16 + sc.y / 2, S16 + sc.z / 2, S16 + sc.w / 2, fb, xs2, grs, gq & 1, ng, acc_a, acc_b);
         if (tq == (gq >> 1)) {
           part[g.slot_rg(warp, tile) * 16 + gq] = acc_a;
           part[g.slot_rg(warp, tile) * 16 + 8 + gq] = acc_b;
@@ -941,7 +975,9 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       if (warp == DF_WARPS - 1) bias_c = (c < E && a.layer[l + 1].bias) ? a.layer[l + 1].bias[c] : 0.f;
     }
     // this CTA's rows of h (only it writes them), read early for the combine
-    const float hpre = threadIdx.x < g.nrow ? __ldcg(a.h + g.o0 + threadIdx.x) : 0.f;
+    float hpre = 0.f;
+    if (threadIdx.x < g.nrow)      // issued here (volatile: not moved to its use in the combine)
+      asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(hpre) : "l"(a.h + g.o0 + threadIdx.x));
     // paired activations of the k routed slots and of the shared expert: all
     // loads first (DF_ACT_ROUNDS words per thread), then pairing
     {
