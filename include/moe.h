@@ -205,7 +205,13 @@ MOE_API int moe_combine(const float* y_pairs, const float* gates, const float* y
  *   y        bf16 [T,H] (device) or NULL: the layer output
  *   idx, gates  int32/fp32 [T,k] (device) or NULL: the routing used
  *   blob_ptrs   device array [E] of blob pointers
- *   ws       device workspace of at least moe_layer_workspace_size(...) bytes */
+ *   ws       device workspace of at least moe_layer_workspace_size(...) bytes
+ * With more rows than the GEMV threshold, independent parts of the layer
+ * (the shared expert; the experts whose buckets take the GEMV kernels) run on
+ * two library-owned streams per device, forked from `stream` and joined back
+ * into it with events before the combine, so they overlap the tensor-core
+ * experts (also inside a captured graph).  The streams are created by the
+ * first such call on a device (make it outside graph capture). */
 MOE_API size_t moe_layer_workspace_size(int T, int H, int I, int Is, int E, int k);
 MOE_API int moe_layer_forward(const float* h_in, float* h_out, const uint16_t* x_in, int T, int H,
                       int I, int Is, int E, int k, const moe_qmat* router,

@@ -1,5 +1,6 @@
 // C-ABI of libmoe: argument checks, workspace carving and kernel launches.
 #include <cstdarg>
+#include <mutex>
 #include <cstdio>
 #include <cstring>
 
@@ -14,6 +15,37 @@ namespace moe {
 static thread_local char g_err[512] = "";
 static int g_gemv_max_rows = 2;
 static int g_grouped_mma = 0;            // buckets of 3..32 rows on the grouped mma.sync kernel (off: measured slower)
+
+// Two library-owned streams per device for independent parts of a call (the
+// shared expert, the GEMV buckets), forked from and joined back into the
+// caller's stream with events, so a captured graph gets the same branches.
+// Created on first use, kept until exit; the fork-launch-join sequence of a
+// call holds g_fork_mu so that concurrent host threads do not mix events.
+struct SideStreams {
+  cudaStream_t st[2] = {nullptr, nullptr};
+  cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
+};
+static std::recursive_mutex g_fork_mu;
+static SideStreams* side_streams() {
+  static SideStreams per_dev[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  SideStreams& S = per_dev[dev];
+  if (!S.st[0]) {
+    for (int i = 0; i < 2; ++i)
+      if (cudaStreamCreateWithFlags(&S.st[i], cudaStreamNonBlocking) != cudaSuccess) { cudaGetLastError(); return nullptr; }
+    for (int i = 0; i < 4; ++i)
+      if (cudaEventCreateWithFlags(&S.ev[i], cudaEventDisableTiming) != cudaSuccess) { cudaGetLastError(); return nullptr; }
+  }
+  return &S;
+}
+int cuda_check(cudaError_t e, const char* what);
+// `to` waits for the work issued so far on `from` (event ev)
+static int stream_after(cudaStream_t to, cudaStream_t from, cudaEvent_t ev) {
+  int st = cuda_check(cudaEventRecord(ev, from), "cudaEventRecord");
+  if (st) return st;
+  return cuda_check(cudaStreamWaitEvent(to, ev, 0), "cudaStreamWaitEvent");
+}
 
 // CTAs of the persistent grouped kernel: one per SM (cached per device).
 static int grouped_grid() {
@@ -246,6 +278,16 @@ int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, int k, con
     if ((st = launch_check("k_group_mma(gate/up)"))) return st;
   }
 
+  // with the tensor-core path, the GEMV buckets (disjoint rows of act and
+  // y_pairs) run on a side stream alongside it
+  std::unique_lock<std::recursive_mutex> fork_lock(g_fork_mu, std::defer_lock);
+  SideStreams* side = tc ? side_streams() : nullptr;
+  cudaStream_t gs = s;
+  if (side) {
+    fork_lock.lock();
+    gs = side->st[1];
+    if ((st = stream_after(gs, s, side->ev[2]))) return st;
+  }
   GateUpArgs g{};
   g.x = x; g.T = T; g.H = H; g.I = I; g.E = E; g.k = k;
   g.blob_ptrs = blob_ptrs; g.offsets = offsets; g.pairs = pairs; g.active = active; g.n_active = n_active;
@@ -254,7 +296,7 @@ int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, int k, con
   g.act = act;
   size_t sm = gemv_smem(H);
   if ((st = set_smem(reinterpret_cast<const void*>(k_gateup_gemv), sm))) return st;
-  k_gateup_gemv<<<dim3((I + GEMV_ROWS - 1) / GEMV_ROWS, maxA), 256, sm, s>>>(g);
+  k_gateup_gemv<<<dim3((I + GEMV_ROWS - 1) / GEMV_ROWS, maxA), 256, sm, gs>>>(g);
   if ((st = launch_check("k_gateup_gemv"))) return st;
 
   TcArgs ta{};
@@ -289,13 +331,14 @@ int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, int k, con
   d.y = y_pairs;
   sm = gemv_smem(I);
   if ((st = set_smem(reinterpret_cast<const void*>(k_down_gemv), sm))) return st;
-  k_down_gemv<<<dim3((H + GEMV_ROWS - 1) / GEMV_ROWS, maxA), 256, sm, s>>>(d);
+  k_down_gemv<<<dim3((H + GEMV_ROWS - 1) / GEMV_ROWS, maxA), 256, sm, gs>>>(d);
   if ((st = launch_check("k_down_gemv"))) return st;
   if (tc) {
     ta.mode = 1;
     k_expert_tc<<<dim3(H / 128, maxA), TC_THREADS, TC_SMEM, s>>>(ta);
     if ((st = launch_check("k_expert_tc(down)"))) return st;
   }
+  if (side && (st = stream_after(s, gs, side->ev[3]))) return st;     // join
   return MOE_OK;
 }
 
@@ -433,12 +476,23 @@ int moe_layer_forward(const float* h_in, float* h_out, const uint16_t* x_in, int
   if (x_out && (st = cuda_check(cudaMemcpyAsync(x_out, xin, static_cast<size_t>(T) * H * 2,
                                                 cudaMemcpyDeviceToDevice, s), "copy x_out")))
     return st;
+  // the shared expert needs only x: it runs on a side stream alongside the
+  // router, the buckets and the routed experts (several rows only)
+  std::unique_lock<std::recursive_mutex> fork_lock(g_fork_mu, std::defer_lock);
+  SideStreams* side = T > g_gemv_max_rows ? side_streams() : nullptr;
+  cudaStream_t shs = s;
+  if (side) {
+    fork_lock.lock();
+    shs = side->st[0];
+    if ((st = stream_after(shs, s, side->ev[0]))) return st;
+  }
+  if ((st = moe_shared_forward(xin, T, H, Is, shared, ysh, sw, sws, shs))) return st;
   if ((st = moe_router_topk(xin, T, H, router, bias, bias_per_row, E, k, idx, gates, nullptr, stream))) return st;
   if ((st = moe_bucket(idx, T, k, E, offsets, pairs, active, n_active, stream))) return st;
-  if ((st = moe_shared_forward(xin, T, H, Is, shared, ysh, sw, sws, stream))) return st;
   if ((st = moe_expert_forward(xin, T, H, I, E, k, blob_ptrs, offsets, pairs, active, n_active, y_pairs, ew, ews,
                                stream)))
     return st;
+  if (side && (st = stream_after(s, shs, side->ev[1]))) return st;   // join before the combine
   float* resid = nullptr;
   if (h_out) {
     if (h_out != h_in &&
