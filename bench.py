@@ -268,6 +268,89 @@ def run_decode_b64(M, stack, device, reps: int):
             "l2": "inputs larger than L2 (every step touches all 30 layers)"}
 
 
+def run_streamed_lfu(M, device):
+    """Streamed workload: 1024-token prompt in chunks of 128 through 30 layers,
+    then 128 decode steps, routed experts in pinned host memory, 16 HBM slots
+    per layer (misses copied host -> device on a side stream while the shared
+    expert runs).  Prefill and decode timed separately (CUDA events; the LFU
+    plan of every layer step needs the routing on the host)."""
+    import torch
+    from quantized_moe_bit_b200.weights import blob_table, upload_qmat
+    c = gen.CONFIGS["streamed_30L_lfu"]
+    stride = gen.synth.default_blob_stride(c.H, c.I)
+    host = torch.empty((c.layers, c.E, stride), dtype=torch.uint8, pin_memory=True)
+    hv = host.numpy()
+    routers, shared = [], []
+    for l in range(c.layers):
+        gen.layer_blobs(c.seed, l, c.E, c.H, c.I, stride, out=hv[l], threads=16)
+        routers.append(upload_qmat(gen.router_weights(c.seed, l, c.E, c.H), device))
+        shared.append([upload_qmat(m, device) for m in gen.shared_weights(c.seed, l, c.H, c.Is)])
+    pool = torch.empty((c.layers, c.n_slots, stride), dtype=torch.uint8, device=device)
+    tables = torch.zeros((c.layers, c.E), dtype=torch.int64, device=device)
+    base = host.data_ptr()
+    host_ptrs = [base + (l * c.E + e) * stride for l in range(c.layers) for e in range(c.E)]
+    n_tok = c.prompt_tokens + c.decode_steps
+    sets = [gen.forced_routing(c.seed, l, n_tok, c.E, c.k) for l in range(c.layers)]
+    biases = {}
+
+    def bias(l, t0, T):
+        key = (l, t0, T)
+        if key not in biases:
+            biases[key] = torch.from_numpy(gen.forced_bias(sets[l][t0:t0 + T], c.E)).to(device)
+        return biases[key]
+    prompt = gen.rows(c.seed, 3000, c.prompt_tokens, c.H)
+    dec = [gen.rows(c.seed, 4000 + d, 1, c.H) for d in range(c.decode_steps)]
+    units = [(torch.from_numpy(prompt[i:i + c.T]).to(device), i) for i in range(0, c.prompt_tokens, c.T)]
+    units += [(torch.from_numpy(dec[d]).to(device), c.prompt_tokens + d) for d in range(c.decode_steps)]
+    for l in range(c.layers):                   # biases built before the timed region
+        for z, t0 in units:
+            bias(l, t0, z.shape[0])
+    lfu = M.MoeLfu(c.layers, c.E, c.n_slots, gen.blob_bytes(c.H, c.I), host_ptrs, pool, stride)
+    side = torch.cuda.Stream(device=device)
+    main = torch.cuda.current_stream()
+    ws = {T: torch.empty(M.moe_streamed_workspace_size(T, c.H, c.I, c.Is, c.E, c.k), dtype=torch.uint8,
+                         device=device) for T in (c.T, 1)}
+
+    def run(us):
+        for z, t0 in us:
+            T = z.shape[0]
+            h = z.clone()
+            for l in range(c.layers):
+                M.moe_streamed_layer_forward(lfu, l, h, c.I, c.Is, c.E, c.k, routers[l].c, bias(l, t0, T), 1,
+                                             [m.c for m in shared[l]], tables[l], ws[T], main_stream=main,
+                                             side_stream=side)
+    n_pre = c.prompt_tokens // c.T
+    torch.cuda.synchronize()
+    e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    e0.record()
+    run(units[:n_pre])
+    e1.record()
+    run(units[n_pre:])
+    e2.record()
+    torch.cuda.synchronize()
+    M.moe_sync()
+    t_pre, t_dec = e0.elapsed_time(e1) / 1e3, e1.elapsed_time(e2) / 1e3
+    hits, misses, nbytes = lfu.stats()
+    lfu.close()
+    # pinned host -> device copy bandwidth of this box, for context
+    buf = host.view(-1)[: 256 << 20]
+    dst = torch.empty(buf.numel(), dtype=torch.uint8, device=device)
+    dst.copy_(buf, non_blocking=True)
+    torch.cuda.synchronize()
+    e3, e4 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e3.record()
+    dst.copy_(buf, non_blocking=True)
+    e4.record()
+    torch.cuda.synchronize()
+    h2d = buf.numel() / (e3.elapsed_time(e4) / 1e3) / 1e9
+    return {"workload": "streamed_30L_lfu", "prefill_tokens_per_s": c.prompt_tokens / t_pre,
+            "decode_tokens_per_s": c.decode_steps / t_dec, "prefill_s": t_pre, "decode_s": t_dec,
+            "hits": hits, "misses": misses, "h2d_bytes": nbytes,
+            "h2d_gbs_while_streaming": nbytes / (t_pre + t_dec) / 1e9, "pinned_h2d_copy_gbs": h2d,
+            "slots_per_layer": c.n_slots,
+            "note": "bitwise equality with the all-resident run and the LFU log are checked by the GPU tests"}
+
+
 def cpu_baseline_oracle(cfg, n_layers: int, stream: int):
     """Time the fp64 oracle on one token through the first n_layers layers."""
     from oracle import moe_oracle as O
@@ -427,6 +510,7 @@ def run_ours(args, rank, world, local_rank):
     if not args.no_extra:
         extra["prefill_128"] = run_prefill(M, layers, device, reps=3)
         extra["decode_b64"] = run_decode_b64(M, stack, device, reps=5)
+        extra["streamed_lfu"] = run_streamed_lfu(M, device)
     value = whole_job_rate(ms, args.steps, world)
     e2e_val = whole_job_rate(ms_e2e, args.steps, world)
     hbm, src = peaks()
