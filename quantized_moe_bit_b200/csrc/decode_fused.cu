@@ -60,6 +60,7 @@ constexpr int DF_MAX_ACT = 8 * DF_THREADS * 3;   // k*I + Is fp16 activations (3
 constexpr int DF_ACT_ROUNDS = 3;
 // mbarriers: routed gate/up tiles 0..5, then
 constexpr int DF_BAR_D = 6, DF_BAR_SD = 7, DF_BAR_SG = 8, DF_BAR_RR = 9, DF_NBARS = 10;
+constexpr int DF_TX_BYTES = (DF_NBARS * 4 + 15) & ~15;   // one u32 per barrier, 16-byte rounded
 // copy sources besides routed slots 0..7: shared matrix m array a (q, s, b) at
 // DF_SRC_SHARED + 3m + a, router arrays (q, s, b) at DF_SRC_ROUTER + a
 constexpr int DF_SRC_SHARED = 8, DF_SRC_ROUTER = 17;
@@ -176,7 +177,7 @@ struct DfGeom {
   }
   DF_HD uint32_t misc_bytes() const {
     // logits, sel / selv / selg, red, bars, blob table, copy table, pair table, part
-    return DF_MAX_E * 4 + 8 * 4 * 3 + 16 * 4 + DF_NBARS * 8 + DF_MAX_E * 8 + DF_MAX_COPIES * 16 +
+    return DF_MAX_E * 4 + 8 * 4 * 3 + 16 * 4 + DF_NBARS * 8 + DF_TX_BYTES + DF_MAX_E * 8 + DF_MAX_COPIES * 16 +
            (DF_MAX_RG_PAIRS + DF_MAX_SG_PAIRS) * 16 + static_cast<uint32_t>(part_slots()) * 64;
   }
   // misc sub-offsets
@@ -186,7 +187,8 @@ struct DfGeom {
   DF_HD uint32_t m_selg() const { return m_sel() + 64; }
   DF_HD uint32_t m_red() const { return m_sel() + 96; }
   DF_HD uint32_t m_bars() const { return m_red() + 64; }
-  DF_HD uint32_t m_btab() const { return m_bars() + DF_NBARS * 8; }     // this layer's E blob pointers
+  DF_HD uint32_t m_tx() const { return m_bars() + DF_NBARS * 8; }       // bytes each barrier's copies bring
+  DF_HD uint32_t m_btab() const { return m_tx() + DF_TX_BYTES; }         // this layer's E blob pointers
   DF_HD uint32_t m_ctab() const { return m_btab() + DF_MAX_E * 8; }      // the CTA's copy lists
   DF_HD uint32_t m_ptab() const { return m_ctab() + DF_MAX_COPIES * 16; }   // scale rows of every pair
   DF_HD uint32_t m_part() const { return m_ptab() + (DF_MAX_RG_PAIRS + DF_MAX_SG_PAIRS) * 16; }
@@ -421,6 +423,12 @@ __device__ __forceinline__ void df_mbar_init(uint32_t bar, uint32_t count) {
 __device__ __forceinline__ void df_mbar_arrive(uint32_t bar) {
   asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar) : "memory");
 }
+// the single arrival of a phase, announcing the bytes its copies will bring
+__device__ __forceinline__ void df_mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
+               "r"(bytes)
+               : "memory");
+}
 // bounded wait on a phase parity
 __device__ __forceinline__ bool df_mbar_wait(uint32_t bar, uint32_t parity) {
   uint64_t t0 = 0;
@@ -443,12 +451,18 @@ __device__ __forceinline__ bool df_mbar_wait(uint32_t bar, uint32_t parity) {
   flag_check(CHECK_WAIT);
   return false;
 }
-// raise the barrier's expected bytes, then copy (the copy completes them)
+// One 1-D bulk copy completing `bytes` of transaction count on mbarrier
+// `bar`; the count was announced beforehand by df_mbar_arrive_tx.
 __device__ __forceinline__ void df_bulk(uint32_t bar, uint32_t dst, const void* src, uint32_t bytes) {
-  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                "l"(src), "r"(bytes), "r"(bar)
                : "memory");
+}
+// The same, announcing its own bytes first (for barriers whose arrival
+// comes after the copies, by df_mbar_arrive).
+__device__ __forceinline__ void df_bulk_tx(uint32_t bar, uint32_t dst, const void* src, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+  df_bulk(bar, dst, src, bytes);
 }
 // L2 prefetch of the 16-byte-aligned window around [p, p + bytes).  Arrays
 // handed to this kernel are 16-byte aligned with sizes that are multiples of
@@ -636,6 +650,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
   float* part = reinterpret_cast<float*>(smem + g.m_part());
   const void** btab = reinterpret_cast<const void**>(smem + g.m_btab());
   DfCopyS* ctab = reinterpret_cast<DfCopyS*>(smem + g.m_ctab());
+  uint32_t* txb = reinterpret_cast<uint32_t*>(smem + g.m_tx());
   // per pair: shared-memory offsets of its gate.s, gate.b, up.s, up.b rows
   // (routed pairs at 0.., shared pairs at DF_MAX_RG_PAIRS..)
   uint4* ptab = reinterpret_cast<uint4*>(smem + g.m_ptab());
@@ -658,12 +673,17 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
   unsigned* abort_word = a.counter + 32;          // own 128-byte line
   unsigned bar_target = 0;
   auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
-  auto grid_sync = [&]() {
+  // grid barrier, split: one thread of every CTA arrives once its CTA's
+  // results for the other CTAs are written; grid_wait (all threads) returns
+  // once every CTA has arrived.  grid_sync = both, for the whole CTA.
+  auto grid_arrive = [&]() {
+    __threadfence();
+    red_release_gpu(a.counter, 1u);
+  };
+  auto grid_wait = [&]() {
     __syncthreads();
     if (threadIdx.x == 0) {
-      __threadfence();
       bar_target += static_cast<unsigned>(G);
-      red_release_gpu(a.counter, 1u);
       const uint64_t t0 = df_clock();
       while (ld_acquire_gpu(a.counter) < bar_target) {
         __nanosleep(32);
@@ -673,9 +693,17 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
     }
     __syncthreads();
   };
-  // warp-wide: issue copy list `list` of layer W (routed slots through the
-  // selection and the staged blob table), then one arrive on each barrier in [b0, b1)
+  auto grid_sync = [&]() {
+    __syncthreads();
+    if (threadIdx.x == 0) grid_arrive();
+    grid_wait();
+  };
+  // warp-wide: one arrive on each barrier in [b0, b1) with the bytes its
+  // copies bring, then copy list `list` of layer W (routed slots through the
+  // selection and the staged blob table)
   auto issue_list = [&](const DfLayer& W, int list, int b0, int b1) {
+    if (lane < b1 - b0) df_mbar_arrive_tx(BAR(b0 + lane), txb[b0 + lane]);
+    __syncwarp();
     for (int e = lst[list] + lane; e < lst[list + 1]; e += 32) {
       const DfCopyS C = ctab[e];
       const uint8_t* b;
@@ -694,8 +722,6 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       }
       df_bulk(BAR(C.bar), sbase + C.dst, b + C.src_off, C.bytes);
     }
-    __syncwarp();
-    if (lane < b1 - b0) df_mbar_arrive(BAR(b0 + lane));
     __syncwarp();
   };
   auto issue_sg = [&](const DfLayer& W) { issue_list(W, 3, DF_BAR_SG, DF_BAR_SG + 1); };
@@ -718,6 +744,12 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
     const DfCopy C = df_list_copy(g, a.off, list, e - lst[list]);
     ctab[e] = DfCopyS{C.dst, C.bytes, static_cast<uint32_t>(C.src_off), static_cast<uint16_t>(C.src),
                       static_cast<uint16_t>(C.bar)};
+  }
+  __syncthreads();
+  if (threadIdx.x < DF_NBARS) {          // static too: the byte counts do not depend on the selection
+    uint32_t t = 0;
+    for (int e = 0; e < lst[5]; ++e) t += ctab[e].bar == threadIdx.x ? ctab[e].bytes : 0u;
+    txb[threadIdx.x] = t;
   }
   // every blob pointer is checked (non-null, 16-byte aligned) before any copy
   // reads one; a bad one stops every CTA at the same point
@@ -786,6 +818,8 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
     df_stamp(a, l, 1);
 
     // --------------------------- router logit c, shared gate/up pairs
+    // (the router warp arrives at the grid barrier as soon as the logit is
+    // written; the shared pairs are computed while the other CTAs get there)
     if (warp == DF_WARPS - 1) {
       if (c < E) {
         df_mbar_wait(BAR(DF_BAR_RR), par);
@@ -811,6 +845,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
         acc = warp_sum(acc);
         if (lane == 0) a.logits[c] = acc + bias_c;
       }
+      if (lane == 0) grid_arrive();      // the logit is all other CTAs need from this one
     } else {
       // warp w < 11: groups [w*NGH/11, (w+1)*NGH/11) of every shared gate/up tile
       const int s0g = warp * NGH / (DF_WARPS - 1), ng = (warp + 1) * NGH / (DF_WARPS - 1) - s0g;
@@ -845,7 +880,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       a.act[kI + g.s0 + i] = __float2half_rn(gelu_tanh(gs) * us);
     }
     df_stamp(a, l, 2);
-    grid_sync();
+    grid_wait();                         // these act values are read after the next barrier
     df_stamp(a, l, 3);
 
     // ------------------------------------------------ top-k, routed bytes

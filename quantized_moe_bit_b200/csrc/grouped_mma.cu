@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_group_mma(const __grid_consta
         d = g.win(w);
         bytes = static_cast<uint32_t>(g.winrows) * g.sb;
       }
-      df_bulk(bar, dst + d, src, bytes);
+      df_bulk_tx(bar, dst + d, src, bytes);
     }
     __syncwarp();
     if (lane == 0) df_mbar_arrive(bar);

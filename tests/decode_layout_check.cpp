@@ -202,6 +202,20 @@ int main(int argc, char** argv) {
         n += df_list_count(g, i);
       }
       REQUIRE(n <= DF_MAX_COPIES, "cta %d: %d copies", c, n);
+      // every barrier is fed by one list only, which arrives on it with the
+      // byte total (the mbarrier transaction count is below 2^20)
+      const int lo[5] = {0, DF_BAR_D, DF_BAR_SD, DF_BAR_SG, DF_BAR_RR};
+      const int hi[5] = {g.ntR, DF_BAR_D + 1, DF_BAR_SD + 1, DF_BAR_SG + 1, DF_BAR_RR + 1};
+      uint64_t tx[DF_NBARS] = {};
+      for (int i = 0; i < 5; ++i)
+        for (int e = 0; e < df_list_count(g, i); ++e) {
+          const DfCopy C = df_list_copy(g, off, i, e);
+          REQUIRE(C.bar >= lo[i] && C.bar < hi[i], "cta %d list %d barrier %d", c, i, C.bar);
+          tx[C.bar] += C.bytes;
+        }
+      for (int b = 0; b < DF_NBARS; ++b) REQUIRE(tx[b] < (1u << 20), "cta %d barrier %d: %llu bytes", c, b,
+                                                 (unsigned long long)tx[b]);
+      REQUIRE(g.m_tx() % 16 == 0 && g.m_btab() % 16 == 0, "cta %d tx table", c);
       REQUIRE(g.m_ctab() + DF_MAX_COPIES * 16u <= g.m_part() && g.m_ctab() % 16 == 0, "cta %d copy table", c);
     }
     // partial-sum slots
