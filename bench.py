@@ -519,7 +519,7 @@ def run_ours(args, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f16xf16->f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": "u4xs16->s32,f32", "data": "synthetic",
         "config": {"workload": "decode_30L_b1", "layers": cfg.layers, "batch": 1, "H": cfg.H, "E": cfg.E,
                    "k": cfg.k, "I": cfg.I, "Is": cfg.Is, "weights": "4-bit affine g64 experts, 8-bit router",
                    "routing": "Zipf(1.1) per-layer bias", "parallelism": f"replicas x{world}",

@@ -519,6 +519,37 @@ __device__ __forceinline__ void mma_group(float (&d)[4], uint2 wa, uint2 wb, uin
   for (int i = 0; i < 4; ++i) d[i] += e[i];
 }
 
+// m16n8k32 integer mma: A u8 (4-bit codes), B s8 (one activation digit),
+// s32 accumulators.
+__device__ __forceinline__ void imma16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// One group (64 inputs) of tile rows g (words wa) and g+8 (words wb) in
+// integer form.  Lane (g, t) holds words 2t, 2t+1 of the group (inputs
+// 16t .. 16t+15); the low nibbles of a word (inputs 2i of its eight) are the
+// u8 operands of k-slots 4t+i, its high nibbles (inputs 2i+1) those of
+// k-slots 16+4t+i -- one mask (and one shift) per four codes.  fh, fl: the
+// high and low int8 digits of the matching activations in this lane's
+// column, as {word 2t even inputs, word 2t odd inputs, word 2t+1 even, odd}.
+// d = 256 (codes . high digits) + (codes . low digits), exact in s32.
+__device__ __forceinline__ void mma_group_q(int (&d)[4], uint2 wa, uint2 wb, uint4 fh, uint4 fl) {
+  constexpr uint32_t M = 0x0F0F0F0Fu;
+  int e[4] = {0, 0, 0, 0};
+  d[0] = d[1] = d[2] = d[3] = 0;
+  const uint32_t lax = wa.x & M, hax = (wa.x >> 4) & M, lbx = wb.x & M, hbx = (wb.x >> 4) & M;
+  const uint32_t lay = wa.y & M, hay = (wa.y >> 4) & M, lby = wb.y & M, hby = (wb.y >> 4) & M;
+  imma16832(d, lax, lbx, hax, hbx, fh.x, fh.y);
+  imma16832(e, lax, lbx, hax, hbx, fl.x, fl.y);
+  imma16832(d, lay, lby, hay, hby, fh.z, fh.w);
+  imma16832(e, lay, lby, hay, hby, fl.z, fl.w);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] = d[i] * 256 + e[i];
+}
+
 // How the 8 mma columns are used.  BCAST: every column carries the same
 // vector (the result of row g is in accumulator 0/2 of every lane of quad g).
 // SLOT: column j carries slot j's activation (row g's result in column
@@ -528,11 +559,12 @@ __device__ __forceinline__ void mma_group(float (&d)[4], uint2 wa, uint2 wb, uin
 enum : int { DF_BCAST = 0, DF_SLOT = 1, DF_DIAG = 2 };
 
 // This warp's strip of ng <= DF_STRIP groups (from g0) of one 16-row tile,
-// for the lane's two rows: acc += S (dot - sum.x) + B sum.y per group.
+// for the lane's two rows: acc += S (step * idot) + B sum per group, idot
+// the integer dot of the codes with the activation's fixed-point values.
 // qa/qb: the rows' bytes at this lane's offset 8t; sa/ba, sb/bb: their bf16
-// scale and bias rows; fb/xs: the lane's paired activation of the strip and
-// the group sums (1024 * sum of paired halves, sum of values), in step order,
-// held in registers for every tile; suma/sumb: per-row group sums (SLOT);
+// scale and bias rows; fb/xs: the lane's activation digits of the strip and
+// the groups' (step, sum of values), in step order, held in registers for
+// every tile; suma/sumb: per-row group (step, sum) (SLOT);
 // ca/cb: the accumulator of the pair that holds the row's column (SLOT,
 // DIAG); rs: the lane's rotation (DIAG).
 template <int MODE>
@@ -551,13 +583,13 @@ __device__ __forceinline__ void df_strip(const uint8_t* qa, const uint8_t* qb, c
       }
       const uint2 wa = *reinterpret_cast<const uint2*>(qa + 32 * gr);
       const uint2 wb = *reinterpret_cast<const uint2*>(qb + 32 * gr);
-      float d[4];
-      mma_group(d, wa, wb, fb[j][0], fb[j][1]);
+      int d[4];
+      mma_group_q(d, wa, wb, fb[j][0], fb[j][1]);
       const float2 xa = MODE == DF_SLOT ? suma[gr] : xs[j], xb = MODE == DF_SLOT ? sumb[gr] : xs[j];
-      const float va = MODE == DF_BCAST ? d[0] : (ca ? d[1] : d[0]);
-      const float vb = MODE == DF_BCAST ? d[2] : (cb ? d[3] : d[2]);
-      acc_a += bf16_to_f32(sa[gr]) * (va - xa.x) + bf16_to_f32(ba[gr]) * xa.y;
-      acc_b += bf16_to_f32(sb[gr]) * (vb - xb.x) + bf16_to_f32(bb[gr]) * xb.y;
+      const float va = __int2float_rn(MODE == DF_BCAST ? d[0] : (ca ? d[1] : d[0]));
+      const float vb = __int2float_rn(MODE == DF_BCAST ? d[2] : (cb ? d[3] : d[2]));
+      acc_a += bf16_to_f32(sa[gr]) * (xa.x * va) + bf16_to_f32(ba[gr]) * xa.y;
+      acc_b += bf16_to_f32(sb[gr]) * (xb.x * vb) + bf16_to_f32(bb[gr]) * xb.y;
     }
   }
 }
@@ -574,12 +606,12 @@ __device__ __forceinline__ void df_strip_diag(const uint8_t* qa, const uint8_t* 
     if (FULL || j < ng) {
       const uint2 wa = *reinterpret_cast<const uint2*>(qa + 32 * gr[j]);
       const uint2 wb = *reinterpret_cast<const uint2*>(qb + 32 * gr[j]);
-      float d[4];
-      mma_group(d, wa, wb, fb[j][0], fb[j][1]);
-      const float va = odd ? d[1] : d[0];
-      const float vb = odd ? d[3] : d[2];
-      acc_a += bf16_to_f32(sa[gr[j]]) * (va - xs[j].x) + bf16_to_f32(ba[gr[j]]) * xs[j].y;
-      acc_b += bf16_to_f32(sb[gr[j]]) * (vb - xs[j].x) + bf16_to_f32(bb[gr[j]]) * xs[j].y;
+      int d[4];
+      mma_group_q(d, wa, wb, fb[j][0], fb[j][1]);
+      const float va = __int2float_rn(odd ? d[1] : d[0]);
+      const float vb = __int2float_rn(odd ? d[3] : d[2]);
+      acc_a += bf16_to_f32(sa[gr[j]]) * (xs[j].x * va) + bf16_to_f32(ba[gr[j]]) * xs[j].y;
+      acc_b += bf16_to_f32(sb[gr[j]]) * (xs[j].x * vb) + bf16_to_f32(bb[gr[j]]) * xs[j].y;
     }
   }
 }
@@ -593,8 +625,9 @@ __device__ __forceinline__ void df_strip_groups(int g0, int ng, int rs, int (&gr
   }
 }
 
-// Load the strip's activation fragments (column vector f: uint4 per word)
-// and, when given, its group sums into registers, rotated by rs (DIAG).
+// Load the strip's activation digits (vector f: per group, per lane t the
+// high digits at entry 2t and the low digits at 2t+1) and, when given, the
+// groups' (step, sum) into registers, rotated by rs (DIAG).
 __device__ __forceinline__ void df_load_strip(const uint4* f, const float2* sums, int g0, int ng, int rs, int tq,
                                               uint4 (&fb)[DF_STRIP][2], float2 (&xs)[DF_STRIP]) {
 #pragma unroll
@@ -628,6 +661,49 @@ __device__ __forceinline__ float oct_sum(float v) {
   v += __shfl_xor_sync(0xffffffffu, v, 2);
   v += __shfl_xor_sync(0xffffffffu, v, 4);
   return v;
+}
+__device__ __forceinline__ float oct_max(float v) {
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+  return v;
+}
+// largest fixed-point magnitude: 127 * 256 + 127, so both digits are int8
+constexpr float DF_QMAX = 32639.f;
+// Fixed-point form of one group of 64 activations, 8 per lane of an aligned
+// octet (all 32 lanes call it): v ~ step * (256 hi + lo) with step = max|v| /
+// DF_QMAX and hi, lo int8 (round to nearest).  Returns the lane's high and
+// low digits as {inputs 0,2,4,6; inputs 1,3,5,7} words and the group's
+// (step, sum of the values).
+__device__ __forceinline__ void df_quant8(const float v[8], uint2& hi, uint2& lo, float2& ss) {
+  float m = 0.f, s = 0.f;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    m = fmaxf(m, fabsf(v[t]));
+    s += v[t];
+  }
+  m = oct_max(m);
+  s = oct_sum(s);
+  const float inv = m > 0.f ? DF_QMAX / m : 0.f;
+  uint32_t h[2] = {0u, 0u}, l[2] = {0u, 0u};
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    const int q = __float2int_rn(v[t] * inv);
+    const int dl = ((q + 128) & 255) - 128;
+    const int dh = (q - dl) >> 8;
+    h[t & 1] |= static_cast<uint32_t>(dh & 255) << (8 * (t >> 1));
+    l[t & 1] |= static_cast<uint32_t>(dl & 255) << (8 * (t >> 1));
+  }
+  hi = make_uint2(h[0], h[1]);
+  lo = make_uint2(l[0], l[1]);
+  ss = make_float2(m / DF_QMAX, s);
+}
+// Store word u's digits (8 consecutive inputs) into the digit vector f:
+// group u / 8, lane t = (u % 8) / 2, word 2t + (u & 1) of the group.
+__device__ __forceinline__ void df_store_digits(uint4* f, int u, uint2 hi, uint2 lo) {
+  uint2* f2 = reinterpret_cast<uint2*>(f);
+  f2[2 * (u & ~1) + (u & 1)] = hi;
+  f2[2 * (u & ~1) + 2 + (u & 1)] = lo;
 }
 
 // --------------------------------------------------------------- the kernel
@@ -799,7 +875,6 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
 #pragma unroll
       for (int w = 0; w < DF_WARPS; ++w) tot += red[w];
       const float rr = sqrtf(tot / static_cast<float>(H) + 1e-6f);
-      float off = 0.f, sum = 0.f;
       if (u < H / 8) {
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
@@ -808,11 +883,14 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
           xs[8 * u + t] = v[t];
           if (c == 0 && a.x_trace) a.x_trace[static_cast<size_t>(l) * H + 8 * u + t] = b;
         }
-        xf[u] = df_pair8(v, off, sum);
       }
-      off = oct_sum(off);
-      sum = oct_sum(sum);
-      if (u < H / 8 && (lane & 7) == 0) xsum[u >> 3] = make_float2(1024.f * off, sum);
+      uint2 dh, dl;
+      float2 gs;
+      df_quant8(v, dh, dl, gs);
+      if (u < H / 8) {
+        df_store_digits(xf, u, dh, dl);
+        if ((lane & 7) == 0) xsum[u >> 3] = gs;
+      }
       __syncthreads();
     }
     df_stamp(a, l, 1);
@@ -1013,8 +1091,8 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
     float hpre = 0.f;
     if (threadIdx.x < g.nrow)      // issued here (volatile: not moved to its use in the combine)
       asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(hpre) : "l"(a.h + g.o0 + threadIdx.x));
-    // paired activations of the k routed slots and of the shared expert: all
-    // loads first (DF_ACT_ROUNDS words per thread), then pairing
+    // fixed-point digits of the k routed slots' activations and of the shared
+    // expert's: all loads first (DF_ACT_ROUNDS words per thread), then digits
     {
       const int nw = kI / 8 + Is / 8;
       uint4 raws[DF_ACT_ROUNDS];
@@ -1026,31 +1104,27 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
 #pragma unroll
       for (int r = 0; r < DF_ACT_ROUNDS; ++r) {
         const int u = r * DF_THREADS + threadIdx.x;
-        float off = 0.f, sum = 0.f;
-        uint4 p = make_uint4(0u, 0u, 0u, 0u);
-        if (u < nw) {
-          const uint4 raw = raws[r];
-          const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
-          float v[8];
+        const uint4 raw = raws[r];             // zero beyond nw
+        const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+        float v[8];
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const float2 f = unpack_half2(rw[t]);
-            v[2 * t] = f.x;
-            v[2 * t + 1] = f.y;
-          }
-          p = df_pair8(v, off, sum);
+        for (int t = 0; t < 4; ++t) {
+          const float2 f = unpack_half2(rw[t]);
+          v[2 * t] = f.x;
+          v[2 * t + 1] = f.y;
         }
-        off = oct_sum(off);
-        sum = oct_sum(sum);
+        uint2 dh, dl;
+        float2 ss;
+        df_quant8(v, dh, dl, ss);              // an octet is one group (I, Is: multiples of 64)
         if (u < nw) {
           if (u < kI / 8) {
             const int j = u / (I / 8), w = u % (I / 8);
-            af[j * astride4 + w] = p;
-            if ((lane & 7) == 0) asum[j * NGI + w / 8] = make_float2(1024.f * off, sum);
+            df_store_digits(af + j * astride4, w, dh, dl);
+            if ((lane & 7) == 0) asum[j * NGI + w / 8] = ss;
           } else {
             const int w = u - kI / 8;
-            sf[w] = p;
-            if ((lane & 7) == 0) ssum[w / 8] = make_float2(1024.f * off, sum);
+            df_store_digits(sf, w, dh, dl);
+            if ((lane & 7) == 0) ssum[w / 8] = ss;
           }
         }
       }
