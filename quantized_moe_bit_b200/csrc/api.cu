@@ -537,7 +537,7 @@ static int fused_grid() {
 }
 
 static size_t fused_ws(int I, int Is, int E, int k) {
-  return align_up(static_cast<size_t>(k * I + Is) * 2) + align_up(static_cast<size_t>(E) * 4) + 256;
+  return align_up(static_cast<size_t>(k * I + Is) * 2) + align_up(static_cast<size_t>(E) * 8) + 256;
 }
 
 static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, const moe_qmat* routers,
@@ -547,9 +547,10 @@ static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, con
   if (!aligned16(h)) return fail(MOE_ERR_INVALID_ARG, "moe_decode_forward: h must be 16-byte aligned");
   char* w = static_cast<char*>(ws);
   __half* act = reinterpret_cast<__half*>(w);
-  float* logits = reinterpret_cast<float*>(w + align_up(static_cast<size_t>(k * I + Is) * 2));
+  unsigned long long* logits =
+      reinterpret_cast<unsigned long long*>(w + align_up(static_cast<size_t>(k * I + Is) * 2));   // tagged
   unsigned* ctr = reinterpret_cast<unsigned*>(w + align_up(static_cast<size_t>(k * I + Is) * 2) +
-                                              align_up(static_cast<size_t>(E) * 4));
+                                              align_up(static_cast<size_t>(E) * 8));
   const size_t smem = decode_fused_smem(H, I, Is, E, k, G);
   int st;
   if ((st = set_smem(reinterpret_cast<const void*>(k_decode_b1), DF_SMEM_LIMIT))) return st;

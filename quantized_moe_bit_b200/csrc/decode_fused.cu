@@ -51,7 +51,8 @@ constexpr int DF_MAX_H = 3072;            // one 8-element word of h per thread 
 constexpr int DF_MAX_E = 256;
 constexpr int DF_MAX_RG_PAIRS = 48;       // routed gate/up pairs per CTA (6 tiles)
 constexpr int DF_MAX_SG_PAIRS = 24;       // shared gate/up pairs per CTA (3 tiles)
-constexpr int DF_MAX_ROWS = 32;           // output rows per CTA
+constexpr int DF_MAX_ROWS = 32;           // output rows per CTA (<= DF_MAX_E: staged in the logit area)
+static_assert(DF_MAX_ROWS <= DF_MAX_E, "the combine stages h rows in the logit area");
 constexpr int DF_MAX_COPIES = 64;         // entries of a CTA's copy table (all five lists)
 constexpr int DF_STRIP = 4;               // quantisation groups a warp holds at once (its strip)
 constexpr int DF_MAX_TILES = 18;          // routed + shared down tiles per CTA
@@ -77,7 +78,10 @@ struct DfArgs {
   int H, I, Is, E, k, L;
   size_t off[9];                    // blob offsets
   __half* act;                      // workspace: k*I + Is fp16
-  float* logits;                    // workspace: [E]
+  // router logits, each word tagged with the layer that wrote it ((l + 1)
+  // << 32 | fp32 bits; zeroed by the kernel at start-up): the top-k polls
+  // them instead of waiting at a grid barrier
+  unsigned long long* logits;       // workspace: [E]
   unsigned* counter;                // workspace: grid barrier counter; word 32: abort flag (zeroed before launch)
   uint16_t* x_trace; uint16_t* y_trace; int32_t* idx_trace; float* gates_trace;
   int spec;                         // experts speculatively prefetched into L2 per layer
@@ -409,6 +413,16 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
 __device__ __forceinline__ void red_release_gpu(unsigned* p, unsigned v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+// tagged words: release stores, relaxed polls closed by an acquire fence
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ uint64_t df_clock() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -749,17 +763,12 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
   unsigned* abort_word = a.counter + 32;          // own 128-byte line
   unsigned bar_target = 0;
   auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
-  // grid barrier, split: one thread of every CTA arrives once its CTA's
-  // results for the other CTAs are written; grid_wait (all threads) returns
-  // once every CTA has arrived.  grid_sync = both, for the whole CTA.
-  auto grid_arrive = [&]() {
-    __threadfence();
-    red_release_gpu(a.counter, 1u);
-  };
-  auto grid_wait = [&]() {
+  auto grid_sync = [&]() {
     __syncthreads();
     if (threadIdx.x == 0) {
+      __threadfence();
       bar_target += static_cast<unsigned>(G);
+      red_release_gpu(a.counter, 1u);
       const uint64_t t0 = df_clock();
       while (ld_acquire_gpu(a.counter) < bar_target) {
         __nanosleep(32);
@@ -768,11 +777,6 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       __threadfence();
     }
     __syncthreads();
-  };
-  auto grid_sync = [&]() {
-    __syncthreads();
-    if (threadIdx.x == 0) grid_arrive();
-    grid_wait();
   };
   // warp-wide: one arrive on each barrier in [b0, b1) with the bytes its
   // copies bring, then copy list `list` of layer W (routed slots through the
@@ -836,6 +840,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       if (p == 0 || (p & 15)) { flag_check(CHECK_EXPERT_ID); atomicOr(abort_word, 1u); }
     }
   }
+  for (int e = c * DF_THREADS + threadIdx.x; e < E; e += G * DF_THREADS) a.logits[e] = 0ull;   // untagged
   grid_sync();
   if (__ldcg(abort_word) != 0u) return;
   if (warp == 0) {
@@ -896,8 +901,8 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
     df_stamp(a, l, 1);
 
     // --------------------------- router logit c, shared gate/up pairs
-    // (the router warp arrives at the grid barrier as soon as the logit is
-    // written; the shared pairs are computed while the other CTAs get there)
+    // (the logit goes out as soon as it is computed; the shared pairs are
+    // computed while the other CTAs' logits arrive)
     if (warp == DF_WARPS - 1) {
       if (c < E) {
         df_mbar_wait(BAR(DF_BAR_RR), par);
@@ -921,9 +926,9 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
           acc += sc * ((a0 + a1) - 1024.f * sm) + bi * sm;
         }
         acc = warp_sum(acc);
-        if (lane == 0) a.logits[c] = acc + bias_c;
+        if (lane == 0)
+          st_release_u64(a.logits + c, (static_cast<unsigned long long>(l + 1) << 32) | __float_as_uint(acc + bias_c));
       }
-      if (lane == 0) grid_arrive();      // the logit is all other CTAs need from this one
     } else {
       // warp w < 11: groups [w*NGH/11, (w+1)*NGH/11) of every shared gate/up tile
       const int s0g = warp * NGH / (DF_WARPS - 1), ng = (warp + 1) * NGH / (DF_WARPS - 1) - s0g;
@@ -958,12 +963,23 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       a.act[kI + g.s0 + i] = __float2half_rn(gelu_tanh(gs) * us);
     }
     df_stamp(a, l, 2);
-    grid_wait();                         // these act values are read after the next barrier
-    df_stamp(a, l, 3);
-
     // ------------------------------------------------ top-k, routed bytes
-    for (int e = threadIdx.x; e < E; e += DF_THREADS) lg[e] = __ldcg(a.logits + e);
+    // every logit of layer l (tag l + 1).  Logits of layer l + 1 are written
+    // only after the next grid barrier, when every CTA has read these.
+    for (int e = threadIdx.x; e < E; e += DF_THREADS) {
+      unsigned long long v = ld_relaxed_u64(a.logits + e);
+      uint64_t t0 = 0;
+      while (static_cast<uint32_t>(v >> 32) != static_cast<uint32_t>(l + 1)) {
+        if (t0 == 0) t0 = df_clock();
+        else if (df_clock() - t0 > 2000000000ull) { flag_check(CHECK_WAIT); break; }
+        __nanosleep(20);
+        v = ld_relaxed_u64(a.logits + e);
+      }
+      fence_acq_rel_gpu();
+      lg[e] = __uint_as_float(static_cast<uint32_t>(v));
+    }
     __syncthreads();
+    df_stamp(a, l, 3);
     for (int e = threadIdx.x; e < E; e += DF_THREADS) {
       const float v = lg[e];
       int rank = 0;
@@ -1183,25 +1199,30 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
         }
       }
     }
+    if (threadIdx.x < g.nrow) lg[threadIdx.x] = hpre;   // the logits are read (nrow <= DF_MAX_E)
     __syncthreads();
     df_stamp(a, l, 10);
     {
-      const int dp = g.dp();
-      for (int r = threadIdx.x; r < g.nrow; r += DF_THREADS) {   // nrow <= DF_THREADS: one row per thread
+      // warp w combines rows w, w + 12, ...: the row's k * dp routed partials
+      // (times their gates) and its DF_WARPS shared partials over the lanes,
+      // then one warp sum
+      const int dp = g.dp(), nr = k * dp, nq = nr + DF_WARPS;
+      for (int r = warp; r < g.nrow; r += DF_WARPS) {
         float y = 0.f;
-        for (int j = 0; j < k; ++j) {
-          const int rho = j * g.nrow + r, tile = rho / 16, tr = rho % 16;
-          float yj = 0.f;
-          for (int p = 0; p < dp; ++p) yj += part[g.slot_d(p, tile) * 16 + tr];
-          y = fmaf(selg[j], yj, y);
+        for (int q = lane; q < nq; q += 32) {
+          if (q < nr) {
+            const int j = q / dp, p = q - j * dp, rho = j * g.nrow + r;
+            y = fmaf(selg[j], part[g.slot_d(p, rho / 16) * 16 + rho % 16], y);
+          } else {
+            y += part[g.slot_sd(q - nr, r / 16) * 16 + r % 16];
+          }
         }
-        const int ts = r / 16, tr = r % 16;
-        float ysh = 0.f;
-        for (int w = 0; w < DF_WARPS; ++w) ysh += part[g.slot_sd(w, ts) * 16 + tr];
-        y += ysh;
-        const int o = g.o0 + r;
-        a.h[o] = hpre + y;
-        if (a.y_trace) a.y_trace[static_cast<size_t>(l) * H + o] = f32_to_bf16(y);
+        y = warp_sum(y);
+        if (lane == 0) {
+          const int o = g.o0 + r;
+          a.h[o] = lg[r] + y;
+          if (a.y_trace) a.y_trace[static_cast<size_t>(l) * H + o] = f32_to_bf16(y);
+        }
       }
     }
     df_stamp(a, l, 11);
