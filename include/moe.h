@@ -248,12 +248,13 @@ MOE_API int moe_set_decode_prefetch(int flags);
 /* Phase timestamps of the fused batch-1 kernel (a tracing aid): when
  * `stamps` (device, [L][G][16] uint64, G = moe_decode_grid()) is non-NULL,
  * thread 0 of every CTA writes %globaltimer (ns) at the phase boundaries of
- * each layer: 0 start, 1 norm done, 2 router/shared gate-up done, 3 after the
- * first grid barrier, 4 top-k done, 5 routed copies issued, 6 routed gate/up
- * done, 7 shared-down copies issued, 8 after the second grid barrier, 9 L2
- * prefetch issued, 10 activations staged, 11 down dots done, 12 combine done,
- * 13 next layer's copies issued, 14 after the third grid barrier.  NULL turns
- * it off (default). */
+ * each layer: 0 start, 1 norm done, 2 router logit sent and shared gate/up
+ * done, 3 every router logit received, 4 top-k done, 5 gates done, 6 routed
+ * gate/up done, 7 activations written and down copies issued, 8 after the
+ * first grid barrier, 9 activations staged, 10 down dots done, 11 and 12
+ * combine done, 13 after the second grid barrier; the copy-issuing thread
+ * writes 14 (routed copies issued) and 15 (last routed tile landed).  NULL
+ * turns it off (default). */
 MOE_API int moe_set_decode_profile(unsigned long long* stamps);
 /* CTAs of the fused batch-1 kernel on the current device (0: not available). */
 MOE_API int moe_decode_grid(void);
