@@ -784,6 +784,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
   auto issue_list = [&](const DfLayer& W, int list, int b0, int b1) {
     if (lane < b1 - b0) df_mbar_arrive_tx(BAR(b0 + lane), txb[b0 + lane]);
     __syncwarp();
+#pragma unroll 1
     for (int e = lst[list] + lane; e < lst[list + 1]; e += 32) {
       const DfCopyS C = ctab[e];
       const uint8_t* b;
@@ -1117,7 +1118,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
         const int u = r * DF_THREADS + threadIdx.x;
         raws[r] = u < nw ? ldcg_v4(a.act + 8 * u) : make_uint4(0u, 0u, 0u, 0u);
       }
-#pragma unroll
+#pragma unroll 1                             // rolled: one copy of the digit code
       for (int r = 0; r < DF_ACT_ROUNDS; ++r) {
         const int u = r * DF_THREADS + threadIdx.x;
         const uint4 raw = raws[r];             // zero beyond nw
@@ -1206,16 +1207,23 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
       // warp w combines rows w, w + 12, ...: the row's k * dp routed partials
       // (times their gates) and its DF_WARPS shared partials over the lanes,
       // then one warp sum
-      const int dp = g.dp(), nr = k * dp, nq = nr + DF_WARPS;
+      const int dp = g.dp(), nr = k * dp, nq = nr + DF_WARPS, dtm = g.d_tiles_max(), stm = g.sd_tiles_max();
       for (int r = warp; r < g.nrow; r += DF_WARPS) {
         float y = 0.f;
+#pragma unroll 1
         for (int q = lane; q < nq; q += 32) {
-          if (q < nr) {
-            const int j = q / dp, p = q - j * dp, rho = j * g.nrow + r;
-            y = fmaf(selg[j], part[g.slot_d(p, rho / 16) * 16 + rho % 16], y);
-          } else {
-            y += part[g.slot_sd(q - nr, r / 16) * 16 + r % 16];
+          int slot, row;
+          float gate = 1.f;
+          if (q < nr) {                    // slot_d(p, tile) = p * dtm + tile
+            const int j = q / dp, rho = j * g.nrow + r;
+            slot = (q - j * dp) * dtm + (rho >> 4);
+            row = rho & 15;
+            gate = selg[j];
+          } else {                         // slot_sd(w, tile) = dp * dtm + w * stm + tile
+            slot = dp * dtm + (q - nr) * stm + (r >> 4);
+            row = r & 15;
           }
+          y = fmaf(gate, part[slot * 16 + row], y);
         }
         y = warp_sum(y);
         if (lane == 0) {
