@@ -48,3 +48,94 @@ def test_host_argument_checks():
     assert L.moe_bucket(None, 1, 9, 128, None, None, None, None, None) == 1   # k > 8
     assert L.moe_set_gemv_max_rows(-1) == 1
     assert L.moe_blob_bytes(100, 64, None) == 0
+
+
+# A host address that is 16-byte aligned and non-NULL.  Every call below
+# fails its argument checks (or returns early for T = 0 / L = 0) before any
+# pointer is dereferenced or any CUDA call is made, so nothing ever reads
+# through it; the exact status each one expects also shows that no call got
+# as far as the CUDA runtime (which would answer MOE_ERR_CUDA).
+_FAKE = 0x10000
+_INVALID, _OK = 1, 0
+
+
+def _q(out, inn, bits):
+    from quantized_moe_bit_b200._lib import moe_qmat
+    return moe_qmat(_FAKE, _FAKE, _FAKE, out, inn, bits)
+
+
+def test_router_and_bucket_argument_checks():
+    from quantized_moe_bit_b200 import _lib
+    L = _lib.lib()
+    r = _q(128, 2816, 8)
+    f = _FAKE
+    assert L.moe_router_topk(f, 1, 2800, C.byref(r), None, 0, 128, 8, f, f, None, None) == _INVALID  # H % 64
+    assert L.moe_router_topk(f, 1, 2816, C.byref(r), None, 0, 100, 8, f, f, None, None) == _INVALID  # E % 8
+    assert L.moe_router_topk(f, 1, 2816, C.byref(r), None, 0, 128, 9, f, f, None, None) == _INVALID  # k > 8
+    assert L.moe_router_topk(None, 1, 2816, C.byref(r), None, 0, 128, 8, f, f, None, None) == _INVALID
+    r4 = _q(128, 2816, 4)
+    assert L.moe_router_topk(f, 1, 2816, C.byref(r4), None, 0, 128, 8, f, f, None, None) == _INVALID  # 4-bit
+    rs = _q(64, 2816, 8)
+    assert L.moe_router_topk(f, 1, 2816, C.byref(rs), None, 0, 128, 8, f, f, None, None) == _INVALID  # [E, H]
+    assert L.moe_router_topk(f + 2, 1, 2816, C.byref(r), None, 0, 128, 8, f, f, None, None) == _INVALID  # align
+    assert L.moe_router_topk(f, 0, 2816, C.byref(r), None, 0, 128, 8, f, f, None, None) == _OK        # T = 0
+    assert L.moe_bucket(f, 1, 8, 100, f, f, f, f, None) == _INVALID                                  # E % 8
+    assert L.moe_bucket(f, 20000, 8, 128, f, f, f, f, None) == 5             # T*k cap: MOE_ERR_UNSUPPORTED
+    assert L.moe_bucket(None, 1, 8, 128, f, f, f, f, None) == _INVALID
+
+
+def test_expert_shared_combine_argument_checks():
+    from quantized_moe_bit_b200 import _lib
+    L = _lib.lib()
+    f = _FAKE
+    T, H, I, Is, E, k = 4, 2816, 704, 2112, 128, 8
+    ews = L.moe_expert_workspace_size(T, H, I, k)
+    assert ews > 0 and L.moe_expert_workspace_size(T + 1, H, I, k) >= ews
+    assert L.moe_expert_workspace_size_mma(T, H, I, k) >= ews
+    args = [f, T, H, I, E, k, f, f, f, f, f, f, f]
+    assert L.moe_expert_forward(*args, ews - 1, None) == _INVALID                       # workspace
+    assert b"workspace" in L.moe_last_error_string()
+    assert L.moe_expert_forward(f + 2, *args[1:], ews, None) == _INVALID                # alignment
+    assert L.moe_expert_forward(*args[:6], None, *args[7:], ews, None) == _INVALID       # NULL blobs
+    assert L.moe_expert_forward(f, T, H, 700, E, k, *args[6:], ews, None) == _INVALID   # I % 64
+    assert L.moe_expert_forward(f, 0, H, I, E, k, *args[6:], 0, None) == _OK            # T = 0
+    sh = (_lib.moe_qmat * 3)(_q(Is, H, 4), _q(Is, H, 4), _q(H, Is, 4))
+    sws = L.moe_shared_workspace_size(T, H, Is)
+    assert sws > 0
+    assert L.moe_shared_forward(f, T, H, Is, sh, f, f, sws - 1, None) == _INVALID       # workspace
+    bad = (_lib.moe_qmat * 3)(_q(Is, H, 4), _q(Is, H, 8), _q(H, Is, 4))
+    assert L.moe_shared_forward(f, T, H, Is, bad, f, f, sws, None) == _INVALID          # 8-bit up
+    shape = (_lib.moe_qmat * 3)(_q(Is, H, 4), _q(Is, H, 4), _q(Is, H, 4))
+    assert L.moe_shared_forward(f, T, H, Is, shape, f, f, sws, None) == _INVALID        # down is [H, Is]
+    assert L.moe_combine(f, f, f, T, H, 9, f, None, None) == _INVALID                   # k > 8
+    assert L.moe_combine(None, f, f, T, H, k, f, None, None) == _INVALID
+    assert L.moe_combine(f, f, f, 0, H, k, f, None, None) == _OK
+
+
+def test_layer_and_decode_argument_checks():
+    from quantized_moe_bit_b200 import _lib
+    L = _lib.lib()
+    f = _FAKE
+    T, H, I, Is, E, k = 2, 2816, 704, 2112, 128, 8
+    r = _q(E, H, 8)
+    sh = (_lib.moe_qmat * 3)(_q(Is, H, 4), _q(Is, H, 4), _q(H, Is, 4))
+    lws = L.moe_layer_workspace_size(T, H, I, Is, E, k)
+    assert lws >= L.moe_expert_workspace_size_mma(T, H, I, k) + L.moe_shared_workspace_size(T, H, Is)
+    tail = [T, H, I, Is, E, k, C.byref(r), None, 0, f, sh, None, None, None, None]
+    assert L.moe_layer_forward(None, None, None, *tail, f, lws, None) == _INVALID       # no input
+    assert L.moe_layer_forward(None, f, f, *tail, f, lws, None) == _INVALID             # h_out without h_in
+    assert L.moe_layer_forward(f, f, None, *tail, f, lws - 1, None) == _INVALID         # workspace
+    dws = L.moe_decode_workspace_size(1, H, I, Is, E, k)
+    assert dws >= L.moe_layer_workspace_size(1, H, I, Is, E, k)
+    routers = (_lib.moe_qmat * 2)(r, r)
+    shared = (_lib.moe_qmat * 6)(*(list(sh) * 2))
+    blobs = (C.c_void_p * 2)(f, f)
+    d = [1, H, I, Is, E, k]
+    assert L.moe_decode_forward(f, *d, -1, routers, None, 0, blobs, shared, None, None, None, None, f, dws,
+                                None) == _INVALID                                        # L < 0
+    assert L.moe_decode_forward(f, *d, 2, routers, None, 0, blobs, shared, None, None, None, None, f, dws - 1,
+                                None) == _INVALID                                        # workspace
+    assert L.moe_decode_forward(None, *d, 2, routers, None, 0, blobs, shared, None, None, None, None, f, dws,
+                                None) == _INVALID                                        # NULL h
+    assert L.moe_decode_forward(f, *d, 0, routers, None, 0, blobs, shared, None, None, None, None, f, dws,
+                                None) == _OK                                             # L = 0
