@@ -35,7 +35,7 @@ import numpy as np  # noqa: E402
 import gen  # noqa: E402
 
 CFG = gen.CONFIGS["decode_30L_b1"]
-METRIC = "MoE tokens/s (30-layer decode b=1)"
+METRIC = "MoE tokens/s (30-layer decode b=1; 128-tok prefill) and % of HBM/TC roofline"
 FALLBACK_HBM = 6650.0
 
 
@@ -166,13 +166,14 @@ def layer_bytes(cfg, distinct: float) -> float:
     return router + shared + distinct * gen.blob_bytes(cfg.H, cfg.I)
 
 
-def run_prefill(M, layers, device, reps: int):
-    """128-row chunk through one layer (the prefill workload's shapes and
-    routing skew); chunk i runs on layer i mod 30 so that weights come from
-    HBM.  One graph replay = one chunk per layer."""
+def run_prefill(M, layers, device, reps: int, T: int = 128):
+    """T-row prefill chunks through one layer (the prefill workload's shapes,
+    input stream and routing skew); chunk i runs on layer i mod 30 so that
+    weights come from HBM.  One graph replay = one chunk per layer."""
     import torch
-    cfg = gen.CONFIGS["prefill_1L_128tok"]
-    T, H = cfg.T, cfg.H
+    from dataclasses import replace
+    cfg = replace(gen.CONFIGS["prefill_1L_128tok"], T=T)
+    H = cfg.H
     z = torch.from_numpy(gen.rows(cfg.seed, cfg.row_stream, T, H)).to(device)
     ws = torch.empty(M.moe_layer_workspace_size(T, H, cfg.I, cfg.Is, cfg.E, cfg.k), dtype=torch.uint8, device=device)
     ho = torch.empty_like(z)
@@ -209,16 +210,20 @@ def run_prefill(M, layers, device, reps: int):
     ids = idx.cpu().numpy()
     distinct = float(np.mean([len(np.unique(ids[l])) for l in range(len(layers))]))
     flops, byts = layer_flops(cfg, T), layer_bytes(cfg, distinct)
+    gemm_flops = 2.0 * T * (cfg.k * 3 * cfg.I * cfg.H + 3 * cfg.Is * cfg.H)
     tc, tc_src = peaks_tc()
     hbm, hbm_src = peaks()
     del g
-    return {"workload": "prefill_1L_128tok", "value": T / t, "unit": "tokens/s", "us_per_chunk": t * 1e6,
-            "chunks": n_chunks, "distinct_experts_per_chunk": distinct,
+    t_hbm, t_tc = byts / (hbm * 1e9), gemm_flops / (tc * 1e12)
+    return {"workload": f"prefill_1L_{T}tok", "value": T / t, "unit": "tokens/s", "us_per_chunk": t * 1e6,
+            "rows_per_chunk": T, "chunks": n_chunks, "distinct_experts_per_chunk": distinct,
             "tensor": {"achieved_tflops": flops / t / 1e12, "peak": tc, "frac": flops / t / 1e12 / tc,
                        "peak_source": tc_src, "flops_per_chunk": flops},
             "hbm": {"achieved_gbs": byts / t / 1e9, "peak": hbm, "frac": byts / t / 1e9 / hbm,
                     "peak_source": hbm_src, "bytes_per_chunk": byts},
-            "l2": "each chunk on another of 30 layers (8.6 GB of weights per graph replay)"}
+            "binding_roofline": {"bound": "hbm" if t_hbm >= t_tc else "tensor",
+                                 "frac": max(t_hbm, t_tc) / t, "ideal_us": max(t_hbm, t_tc) * 1e6},
+            "l2": "each chunk on another of 30 layers (weights of 30 layers per graph replay)"}
 
 
 def run_decode_b64(M, stack, device, reps: int):
@@ -351,26 +356,86 @@ def run_streamed_lfu(M, device):
             "note": "bitwise equality with the all-resident run and the LFU log are checked by the GPU tests"}
 
 
-def cpu_baseline_oracle(cfg, n_layers: int, stream: int):
-    """Time the fp64 oracle on one token through the first n_layers layers."""
-    from oracle import moe_oracle as O
+class OracleLayers:
+    """Host weights of the first layers of a workload for the oracle, built
+    before any timer starts; a routed expert's weights are generated the
+    first time it is asked for and kept (a warm-up pass asks for them)."""
+
+    def __init__(self, cfg, n_layers: int):
+        self.cfg, self.cache = cfg, {}
+        self.layers = []
+        for l in range(n_layers):
+            self.layers.append((gen.router_weights(cfg.seed, l, cfg.E, cfg.H),
+                                gen.zipf_bias(cfg.seed, l, cfg.E) if cfg.zipf else None,
+                                self._expert_fn(l), gen.shared_weights(cfg.seed, l, cfg.H, cfg.Is)))
+
+    def _expert_fn(self, l):
+        def f(e):
+            if (l, e) not in self.cache:
+                self.cache[(l, e)] = gen.expert_weights(self.cfg.seed, l, e, self.cfg.H, self.cfg.I)
+            return self.cache[(l, e)]
+        return f
+
+    def generate_all(self):
+        for l, (_, _, f, _) in enumerate(self.layers):
+            for e in range(self.cfg.E):
+                f(e)
+
+
+def oracle_cores():
     try:
         from threadpoolctl import threadpool_info
-        cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+        return max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
     except Exception:
-        cores = os.cpu_count()
-    z = gen.rows(cfg.seed, stream, 1, cfg.H).astype(np.float64)
-    layers = []
-    for l in range(n_layers):
-        layers.append((gen.router_weights(cfg.seed, l, cfg.E, cfg.H),
-                       gen.zipf_bias(cfg.seed, l, cfg.E) if cfg.zipf else None,
-                       (lambda l_: (lambda e: gen.expert_weights(cfg.seed, l_, e, cfg.H, cfg.I)))(l),
-                       gen.shared_weights(cfg.seed, l, cfg.H, cfg.Is)))
+        return os.cpu_count()
+
+
+def time_oracle(fn, one_core: bool):
+    """Wall time of fn() on the host: all cores (numpy's BLAS threads) or one."""
+    if one_core:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(1):
+            t0 = time.perf_counter()
+            fn()
+            return time.perf_counter() - t0
     t0 = time.perf_counter()
-    O.stack_forward(z, layers, cfg.k, cfg.E)
-    dt = time.perf_counter() - t0
-    tok_s = 1.0 / (dt * cfg.layers / n_layers)
-    return tok_s, cores, dt
+    fn()
+    return time.perf_counter() - t0
+
+
+def cpu_baseline_oracle(n_layers: int = 3):
+    """The fp64 oracle on the host cores, weights generated before the timer:
+    one token of the 30-layer batch-1 workload through its first n_layers
+    layers (scaled to tokens/s of the 30-layer step), the single-layer token
+    and the 128-row prefill chunk; each on all cores and on one core."""
+    from oracle import moe_oracle as O
+    cfg = CFG
+    ol = OracleLayers(cfg, n_layers)
+    z = gen.rows(cfg.seed, 999, 1, cfg.H).astype(np.float64)
+    run = lambda: O.stack_forward(z, ol.layers, cfg.k, cfg.E)
+    run()                                   # warm-up: generates the routed experts this token touches
+    t_all = time_oracle(run, False)
+    t_one = time_oracle(run, True)
+    c0 = gen.CONFIGS["single_layer_1tok"]
+    o0 = OracleLayers(c0, 1)
+    z0 = gen.rows(c0.seed, 1000, 1, c0.H).astype(np.float64)
+    r0 = lambda: O.stack_forward(z0, o0.layers, c0.k, c0.E)
+    r0()
+    c2 = gen.CONFIGS["prefill_1L_128tok"]
+    o2 = OracleLayers(c2, 1)
+    z2 = gen.rows(c2.seed, c2.row_stream, c2.T, c2.H).astype(np.float64)
+    r2 = lambda: O.stack_forward(z2, o2.layers, c2.k, c2.E)
+    r2()
+    t0a, t0o = time_oracle(r0, False), time_oracle(r0, True)
+    t2a, t2o = time_oracle(r2, False), time_oracle(r2, True)
+    scale = cfg.layers / n_layers
+    return {"value": 1.0 / (t_all * scale), "unit": "tokens/s", "cores": oracle_cores(), "kind": "oracle",
+            "one_core": {"value": 1.0 / (t_one * scale), "cores": 1},
+            "sample": (f"one token of decode_30L_b1 through its first {n_layers} of 30 layers ({t_all:.2f} s on "
+                       f"all cores, {t_one:.2f} s on one), scaled by 30/{n_layers}; weights generated before the "
+                       f"timer (a warm-up pass generates the experts the token routes to)"),
+            "single_layer_1tok": {"s_all_cores": t0a, "s_one_core": t0o, "tokens_per_s": 1.0 / t0a},
+            "prefill_1L_128tok": {"s_all_cores": t2a, "s_one_core": t2o, "tokens_per_s": c2.T / t2a}}
 
 
 def replica_streams(rank: int, n: int) -> list:
@@ -398,25 +463,35 @@ def whole_job_rate(ms: float, steps: int, world: int) -> float:
 
 
 def run_reference(args, rank, world):
+    """The oracle as it stands, on the host cores (rank 0 only): each step is
+    one fresh token of the 30-layer batch-1 workload through its first
+    REF_LAYERS layers; every routed expert of those layers is generated
+    before the first timed step.  value = tokens/s of the whole 30-layer step
+    (the sample's layers / 30 tokens per step time)."""
     if rank != 0:
         return
-    per_step_layers = 1
+    from oracle import moe_oracle as O
+    cfg = CFG
+    n_layers = 3
+    ol = OracleLayers(cfg, n_layers)
+    ol.generate_all()
     times = []
-    cores = None
     for i in range(args.warmup + args.steps):
-        tok_s, cores, dt = cpu_baseline_oracle(CFG, per_step_layers, 1000 + i)
+        z = gen.rows(cfg.seed, 1000 + i, 1, cfg.H).astype(np.float64)
+        dt = time_oracle(lambda: O.stack_forward(z, ol.layers, cfg.k, cfg.E), False)
         if i >= args.warmup:
             times.append(dt)
-    tot = sum(times)
-    value = args.steps / (tot * CFG.layers / per_step_layers)
-    sample = (f"each step: one token through the first {per_step_layers} of 30 layers (oracle, fp64 numpy, "
-              f"expert weights generated inside the timed call), time scaled by 30/{per_step_layers}")
+    ms = 1e3 * sum(times) / args.steps
+    value = (n_layers / cfg.layers) / (ms / 1e3)
+    sample = (f"each step: one token through the first {n_layers} of the 30 layers (fp64 numpy oracle, all its "
+              f"experts generated before the first step), i.e. {n_layers}/30 of a token")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps * CFG.layers / per_step_layers,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "decode_30L_b1", "layers": 30, "batch": 1, "H": CFG.H, "E": CFG.E, "k": CFG.k,
-                       "I": CFG.I, "Is": CFG.Is},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "config": {"workload": "decode_30L_b1", "layers": 30, "batch": 1, "H": cfg.H, "E": cfg.E, "k": cfg.k,
+                       "I": cfg.I, "Is": cfg.Is},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle_cores(), "kind": "oracle",
+                             "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -485,30 +560,53 @@ def run_ours(args, rank, world, local_rank):
     idx_last = idx_tr.cpu().numpy()
     distinct = float(np.mean([len(set(idx_last[l, 0].tolist())) for l in range(cfg.layers)]))
 
-    # end to end through the public call: pinned host input -> step -> host result
+    # end to end through the public call, one token at a time: the row is
+    # copied in from pinned host memory, moe_decode_forward runs (an eager
+    # C-ABI call: argument checks and launch inside the timed region), the
+    # residual row is copied back and the host waits for it
     zh = torch.from_numpy(z[args.warmup:]).pin_memory().view(args.steps, 1, H)
     out_h = torch.empty((args.steps, 1, H), dtype=torch.float32).pin_memory()
+    cur = torch.cuda.current_stream()
     torch.cuda.synchronize()
     barrier()
     e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2.record()
     for i in range(args.steps):
         h.copy_(zh[i], non_blocking=True)
-        g.replay()
+        step()
         out_h[i].copy_(h, non_blocking=True)
+        cur.synchronize()
     e3.record()
     torch.cuda.synchronize()
     barrier()
     ms_e2e = e2.elapsed_time(e3)
+    # the same with the step replayed from a CUDA graph and no host wait
+    # between tokens (copies and steps queued back to back)
+    e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e4.record()
+    for i in range(args.steps):
+        h.copy_(zh[i], non_blocking=True)
+        g.replay()
+        out_h[i].copy_(h, non_blocking=True)
+    e5.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms_pipe = e4.elapsed_time(e5)
     M.moe_sync()
 
-    ms, ms_e2e = max_over_ranks([ms, ms_e2e], world, device)
+    ms, ms_e2e, ms_pipe = max_over_ranks([ms, ms_e2e, ms_pipe], world, device)
     del g
     if rank != 0:
         return
     extra = {}
     if not args.no_extra:
-        extra["prefill_128"] = run_prefill(M, layers, device, reps=3)
+        extra["prefill_128"] = run_prefill(M, layers, device, reps=3, T=128)
+        sweep = [run_prefill(M, layers, device, reps=2, T=T) for T in (256, 512, 1024)]
+        extra["prefill_1L_1024tok"] = sweep[-1]
+        extra["prefill_chunk_sweep"] = [{"rows": r["rows_per_chunk"], "us_per_chunk": r["us_per_chunk"],
+                                         "tokens_per_s": r["value"], "tensor_frac": r["tensor"]["frac"],
+                                         "hbm_frac": r["hbm"]["frac"]}
+                                        for r in [extra["prefill_128"]] + sweep]
         extra["decode_b64"] = run_decode_b64(M, stack, device, reps=5)
         extra["streamed_lfu"] = run_streamed_lfu(M, device)
     value = whole_job_rate(ms, args.steps, world)
@@ -528,15 +626,18 @@ def run_ours(args, rank, world, local_rank):
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "peak_source": src, "traffic": decode_traffic(cfg.layers), "bytes_per_step": bytes_step,
                      "distinct_experts_per_layer": distinct},
-        "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": H * 4, "d2h_bytes_per_step": H * 4},
+        "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": H * 4, "d2h_bytes_per_step": H * 4,
+                "mode": "one token per call: pinned row copied in, eager moe_decode_forward, row copied out, "
+                        "host waits for it"},
+        "e2e_pipelined": {"value": whole_job_rate(ms_pipe, args.steps, world), "unit": "tokens/s",
+                          "h2d_bytes_per_step": H * 4, "d2h_bytes_per_step": H * 4,
+                          "mode": "graph replay per token, copies in and out queued, no host wait between tokens"},
         "gpu_launches": M.moe_decode_launches(1, cfg.layers) * args.steps,
         "clocks": clocks,
         **extra,
     }
     if world == 1 and not args.no_cpu_baseline:
-        tok_s, cores, dt = cpu_baseline_oracle(cfg, 6, 999)
-        line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                                "sample": f"one token through the first 6 of 30 layers ({dt:.1f} s), scaled by 5"}
+        line["cpu_baseline"] = cpu_baseline_oracle()
     print(json.dumps(line), flush=True)
 
 

@@ -97,11 +97,26 @@ MOE_API int moe_sync(void* stream);
  * offsets of gate.q gate.s gate.b up.q up.s up.b down.q down.s down.b. */
 MOE_API size_t moe_blob_bytes(int H, int I, size_t* offsets9);
 
-/* A0 — layer-input RMS norm.  h fp32 [T,H] (device) -> x bf16 [T,H] (device):
- * x = bf16_rn(h / sqrt(mean(h^2) + eps)), sum of squares in fp32, fixed order. */
+/* A0 — layer-input RMS norm.
+ * Source: "drumih/turbo-fieldfare" (paperfeed.app), section "How it works":
+ * each decode step walks the 30 transformer layers, so every layer's MoE input
+ * is the running hidden state.  The pages do not give the norm; this library
+ * defines it as an RMS norm with eps and no learned weight, the output rounded
+ * to bf16 (the layer input of every routed-MoE call below).
+ *   h  fp32 [T,H] (device, read)     x  bf16 [T,H] (device, written)
+ * x = bf16_rn(h / sqrt(mean(h^2) + eps)), sum of squares in fp32, fixed order.
+ * Errors: MOE_ERR_INVALID_ARG (T < 0, H not a positive multiple of 64, NULL or
+ * misaligned pointer) before any launch; T = 0 is a no-op. */
 MOE_API int moe_rmsnorm(const float* h, int T, int H, float eps, uint16_t* x, void* stream);
 
 /* A1 + A2 — router and top-k.
+ * Sources: "TurboFieldfare: Gemma 4 26B on an 8 GB MacBook, in ~2 GB of RAM"
+ * (blog-mushroom.pages.dev), section "Why 26B Fits in 2 GB": the router picks
+ * 8 of 128 experts per token in each layer; "TurboFieldfareとは｜26BのGemma 4
+ * を約2GBのRAMで動かすSwift製ランタイムの実像" (ai-heartland.com), section
+ * "TurboFieldfareとは：エキスパートをSSDに置いたままMoEを走らせる": the router
+ * projection alone is 8-bit MLX affine (group 64, bf16 scale and bias).  The
+ * softmax over the k selected logits is this library's definition.
  *   x       bf16 [T,H] (device)
  *   router  8-bit q-matrix [E,H] (host struct of device pointers)
  *   bias    fp32 [E] (bias_per_row = 0) or [T,E] (bias_per_row = 1) or NULL (device)
@@ -110,60 +125,80 @@ MOE_API int moe_rmsnorm(const float* h, int T, int H, float eps, uint16_t* x, vo
  *   gates   fp32 [T,k] (device): softmax over the k selected logits
  *   logits_opt fp32 [T,E] (device) or NULL: logits including the bias
  * Logits are accumulated in fp32.  Runs as clusters of 8 CTAs per block of
- * rows; the top-k reads the logits through distributed shared memory. */
+ * rows; the top-k reads the logits through distributed shared memory.
+ * Errors: MOE_ERR_INVALID_ARG (dims, NULL pointer, router not 8-bit [E,H],
+ * misaligned x or router codes), MOE_ERR_UNSUPPORTED (H, E too large for the
+ * kernel's shared memory); nothing is launched on an error. */
 MOE_API int moe_router_topk(const uint16_t* x, int T, int H, const moe_qmat* router,
                     const float* bias, int bias_per_row, int E, int k,
                     int32_t* idx, float* gates, float* logits_opt, void* stream);
 
 /* A3 — bucketing (stable counting sort of the T*k pairs by expert).
+ * Source: "TurboFieldfare: Gemma 4 26B on an 8 GB MacBook, in ~2 GB of RAM"
+ * (blog-mushroom.pages.dev), section "Why 26B Fits in 2 GB": prefill chunks of
+ * up to 128 tokens let one expert blob serve every row of the chunk routed to
+ * it; the buckets are those row groups.
  *   idx      int32 [T,k] (device)
  *   offsets  int32 [E+1] (device): bucket e is pairs[offsets[e] .. offsets[e+1])
  *   pairs    int32 [T*k] (device): value t*k + j, t then j ascending inside a bucket
  *   active   int32 [E]   (device): experts with a non-empty bucket, ascending
  *   n_active int32 [1]   (device)
- * Requires T*k <= 65536.  Out-of-range ids are skipped and flagged. */
+ * Requires T*k <= 65536 (else MOE_ERR_UNSUPPORTED).  Out-of-range ids are
+ * skipped and flagged (MOE_ERR_DEVICE_CHECK at the next moe_sync). */
 MOE_API int moe_bucket(const int32_t* idx, int T, int k, int E, int32_t* offsets,
                int32_t* pairs, int32_t* active, int32_t* n_active, void* stream);
 
+/* Per-call path flags (bit set; 0 lets the library choose).  A flag changes
+ * which kernels run, never the definition of the result; paths agree within
+ * the output tolerance, not bit for bit. */
+enum {
+  MOE_FLAG_GEMV = 1,      /* every expert bucket and the shared expert on the CUDA-core GEMV kernels */
+  MOE_FLAG_TC = 2,        /* every bucket (one row included) on the tensor-core grouped GEMM */
+  MOE_FLAG_LAYERED = 4    /* moe_decode_forward at T = 1: the per-layer calls, not the persistent kernel */
+};
+
 /* A4 + A5 — routed experts for every pair.
+ * Sources: "TurboFieldfareとは｜26BのGemma 4を約2GBのRAMで動かすSwift製ランタイム
+ * の実像" (ai-heartland.com), section "TurboFieldfareとは：エキスパートをSSDに
+ * 置いたままMoEを走らせる": routed experts are MLX affine 4-bit, group 64, bf16
+ * scale and bias; "TurboFieldfare: Gemma 4 26B on an 8 GB MacBook, in ~2 GB
+ * of RAM" (blog-mushroom.pages.dev), section "Why 26B Fits in 2 GB": each
+ * expert is one ~3.3 MB blob.  The expert itself (gelu_tanh(W_g x) * W_u x,
+ * then W_d) is this library's definition.
  *   x          bf16 [T,H] (device)
  *   blob_ptrs  device array [E] of device pointers to expert blobs
  *   offsets, pairs, active, n_active   from moe_bucket (device)
  *   y_pairs    fp32 [T*k, H] (device): row t*k + j = expert idx[t,j] applied to x[t]
  *   ws         device workspace of at least moe_expert_workspace_size(T,H,I,k) bytes
- * Each expert runs on the decode GEMV kernels (CUDA cores) when its bucket has
- * at most gemv_max_rows rows (moe_set_gemv_max_rows; default 2) and on the
- * tcgen05 grouped GEMM otherwise.  With a workspace of at least
- * moe_expert_workspace_size_mma(T,H,I,k) bytes (and the grouped kernel on,
- * moe_set_grouped_mma), buckets of gemv_max_rows+1 .. 32 rows run on the
- * grouped mma.sync kernel instead of the tcgen05 GEMM (room for the paired
- * activation rows).  The choice depends only on the bucket's row count and
- * the workspace given.  The activation between the projections is fp16. */
+ *   flags      MOE_FLAG_* (0: the library's choice)
+ * Path: with flags 0, T <= 2 runs the decode GEMV kernels (CUDA cores) and
+ * larger T the tcgen05 grouped GEMM; MOE_FLAG_GEMV / MOE_FLAG_TC force one.
+ * The choice depends on T and flags only, never on the data.  The
+ * activation between the projections is fp16.
+ * Errors: MOE_ERR_INVALID_ARG (dims, NULL or misaligned pointer, workspace too
+ * small) before any launch; T = 0 is a no-op. */
 MOE_API size_t moe_expert_workspace_size(int T, int H, int I, int k);
-MOE_API size_t moe_expert_workspace_size_mma(int T, int H, int I, int k);
-/* Grouped mma.sync kernel for buckets of a few rows: 1 on, 0 off (default;
- * on this B200 it measured slower than the tcgen05 GEMM for 3..32-row buckets). */
-MOE_API int moe_set_grouped_mma(int enable);
 MOE_API int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, int k,
                        const void* const* blob_ptrs, const int32_t* offsets,
                        const int32_t* pairs, const int32_t* active,
                        const int32_t* n_active, float* y_pairs,
-                       void* ws, size_t ws_bytes, void* stream);
+                       void* ws, size_t ws_bytes, int flags, void* stream);
 /* moe_expert_forward without a workspace argument, for callers that cannot
  * allocate device memory where they run the experts (inside a CUDA graph
  * being captured, under a memory pool that must not be re-entered, or in an
  * embedder whose device memory is reserved up front).  The pages describe no
  * counterpart of this call; it is a convenience of this library.
- *   Arguments and results are those of moe_expert_forward.
+ *   Arguments and results are those of moe_expert_forward with flags 0.
  *   Scratch: a static device array of MOE_NOALLOC_SCRATCH_BYTES (4 MiB) in
  *   the library image, one per GPU that loads the library, kept until exit.
- *   It must hold moe_expert_workspace_size(T,H,I,k) bytes (T*k*I fp16
- *   values plus a T*H fp16 copy of x; at H = 2816, I = 704, k = 8 that is
- *   T <= 248); larger requests return
+ *   It must hold moe_expert_workspace_size(T,H,I,k) bytes (at H = 2816,
+ *   I = 704, k = 8 that is T <= 70); larger requests return
  *   MOE_ERR_INVALID_ARG and launch nothing.
- *   The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress) and caches it; make that first call before any
- *   stream capture.
+ *   Argument checks (sizes, NULL and misaligned pointers) come before any
+ *   CUDA call.  Every call then looks up the array's device address on the
+ *   current device (cudaGetSymbolAddress), so the address stays right after a
+ *   device reset; the first call on a device may load the library's device
+ *   code, so make it before any stream capture.
  *   Every call on a device shares the one array and leaves its contents
  *   behind; two calls whose kernels overlap on the GPU (different streams,
  *   no ordering between them) race on it.  Nothing in it needs to start at
@@ -173,28 +208,42 @@ MOE_API int moe_expert_forward_noalloc(const uint16_t* x, int T, int H, int I, i
                                        const void* const* blob_ptrs, const int32_t* offsets,
                                        const int32_t* pairs, const int32_t* active,
                                        const int32_t* n_active, float* y_pairs, void* stream);
-/* Bucket-size threshold between the GEMV and the tensor-core path (>= 0). */
-MOE_API int moe_set_gemv_max_rows(int rows);
 
 /* A6 — shared expert on every row.
+ * Sources: "TurboFieldfare: Gemma 4 26B on an 8 GB MacBook, in ~2 GB of RAM"
+ * (blog-mushroom.pages.dev), section "Why 26B Fits in 2 GB": the shared-expert
+ * branch runs while the routed blobs are fetched; "TurboFieldfareとは｜26Bの
+ * Gemma 4を約2GBのRAMで動かすSwift製ランタイムの実像" (ai-heartland.com),
+ * section "TurboFieldfareとは：エキスパートをSSDに置いたままMoEを走らせる": the
+ * shared expert is 4-bit like the routed ones.  Ungated (added as is) by this
+ * library's definition.
  *   shared  host array of 3 q-matrices: gate [Is,H], up [Is,H], down [H,Is]
  *   ysh     fp32 [T,H] (device)
  *   ws      device workspace of at least moe_shared_workspace_size(T,H,Is) bytes
- * With more rows than the GEMV threshold (moe_set_gemv_max_rows) and
- * H % 128 == 0, H, Is <= 4096, the shared expert runs on the tensor-core
- * grouped GEMM as one expert whose bucket holds every row; otherwise on the
- * GEMV kernels. */
+ *   flags   MOE_FLAG_* (path as in moe_expert_forward: one expert whose
+ *           bucket holds every row)
+ * Errors: MOE_ERR_INVALID_ARG (dims, a matrix not 4-bit of the stated shape,
+ * NULL or misaligned pointer, workspace too small) before any launch. */
 MOE_API size_t moe_shared_workspace_size(int T, int H, int Is);
 MOE_API int moe_shared_forward(const uint16_t* x, int T, int H, int Is, const moe_qmat* shared,
-                       float* ysh, void* ws, size_t ws_bytes, void* stream);
+                       float* ysh, void* ws, size_t ws_bytes, int flags, void* stream);
 
-/* A7 — combine.  y[t] = sum_{j=0..k-1} gates[t,j] * y_pairs[t*k+j] + ysh[t],
+/* A7 — combine.
+ * Source: "TurboFieldfare: Gemma 4 26B on an 8 GB MacBook, in ~2 GB of RAM"
+ * (blog-mushroom.pages.dev), section "Why 26B Fits in 2 GB": the routed and
+ * the shared-expert outputs are merged.  The merge is this library's
+ * definition: the gate-weighted sum of the k routed outputs plus the shared one,
+ *   y[t] = sum_{j=0..k-1} gates[t,j] * y_pairs[t*k+j] + ysh[t],
  * summed in fp32 in that order; y bf16 [T,H] (device, may be NULL);
- * residual_inout fp32 [T,H] (device) or NULL: residual += the fp32 sum. */
+ * residual_inout fp32 [T,H] (device) or NULL: residual += the fp32 sum.
+ * Errors: MOE_ERR_INVALID_ARG (T < 0, k outside 1..8, NULL y_pairs or gates). */
 MOE_API int moe_combine(const float* y_pairs, const float* gates, const float* ysh,
                 int T, int H, int k, uint16_t* y, float* residual_inout, void* stream);
 
-/* One whole layer, A0 (optional) to A7, through the calls above.
+/* One whole layer, A0 (optional) to A7: the calls above in order on `stream`.
+ * Source: "drumih/turbo-fieldfare" (paperfeed.app), section "How it works":
+ * per layer the router runs from resident weights, the routed experts the
+ * step needs are applied and the shared-expert compute overlaps their fetch.
  *   h_in     fp32 [T,H] (device) residual stream or NULL; when x_in is NULL the
  *            layer input is its RMS norm (A0, eps = 1e-6)
  *   h_out    fp32 [T,H] (device) or NULL: receives h_in + y (fp32, before the
@@ -206,21 +255,23 @@ MOE_API int moe_combine(const float* y_pairs, const float* gates, const float* y
  *   idx, gates  int32/fp32 [T,k] (device) or NULL: the routing used
  *   blob_ptrs   device array [E] of blob pointers
  *   ws       device workspace of at least moe_layer_workspace_size(...) bytes
- * With more rows than the GEMV threshold, independent parts of the layer
- * (the shared expert; the experts whose buckets take the GEMV kernels) run on
- * two library-owned streams per device, forked from `stream` and joined back
- * into it with events before the combine, so they overlap the tensor-core
- * experts (also inside a captured graph).  The streams are created by the
- * first such call on a device (make it outside graph capture). */
+ *   flags    MOE_FLAG_* for the routed and the shared experts
+ * On the tensor-core path the routed buckets and the shared expert share one
+ * persistent launch per projection (gate/up, then down), so the shared
+ * expert's weights stream while the routed experts compute.
+ * Errors: as the calls it makes; h_out without h_in, or neither h_in nor
+ * x_in, is MOE_ERR_INVALID_ARG. */
 MOE_API size_t moe_layer_workspace_size(int T, int H, int I, int Is, int E, int k);
 MOE_API int moe_layer_forward(const float* h_in, float* h_out, const uint16_t* x_in, int T, int H,
                       int I, int Is, int E, int k, const moe_qmat* router,
                       const float* bias, int bias_per_row, const void* const* blob_ptrs,
                       const moe_qmat* shared, uint16_t* x_out, uint16_t* y,
-                      int32_t* idx, float* gates, void* ws, size_t ws_bytes, void* stream);
+                      int32_t* idx, float* gates, void* ws, size_t ws_bytes, int flags, void* stream);
 
 /* A whole decode/prefill step through L stacked layers (A0 .. A7 per layer,
- * residual add between layers): for l = 0 .. L-1
+ * residual add between layers).
+ * Source: "drumih/turbo-fieldfare" (paperfeed.app), section "How it works":
+ * each decode step walks the 30 transformer layers.  For l = 0 .. L-1:
  *   x_l = rmsnorm(h); h += layer_l(x_l)
  *   h          fp32 [T,H] (device), updated in place (the step input on entry,
  *              the residual stream after the last layer on return)
@@ -232,40 +283,31 @@ MOE_API int moe_layer_forward(const float* h_in, float* h_out, const uint16_t* x
  *   x_trace, y_trace   bf16 [L,T,H] (device) or NULL: every layer's input/output
  *   idx_trace, gates_trace  int32/fp32 [L,T,k] (device) or NULL
  *   ws         device workspace of at least moe_decode_workspace_size(...) bytes
- * Layers run in order on `stream`. */
+ *   flags      MOE_FLAG_*
+ * Batch-1 steps (T = 1, per-expert or no bias) run as one persistent kernel
+ * per up to 48 layers (one CTA per SM, cooperative launch) unless
+ * MOE_FLAG_LAYERED is set; other shapes run moe_layer_forward per layer.
+ * Layers run in order on `stream`.
+ * Errors: MOE_ERR_INVALID_ARG (dims, L < 0, NULL arrays, workspace too small)
+ * before any launch. */
 MOE_API size_t moe_decode_workspace_size(int T, int H, int I, int Is, int E, int k);
-/* Batch-1 steps (T = 1, per-expert or no bias) run as one persistent kernel
- * per up to 48 layers (one CTA per SM, cooperative launch); other shapes run
- * the per-layer calls.  enable = 0 forces the per-layer path.  spec_experts
- * (0..8, default 0): per layer, the experts with the largest router bias are
- * prefetched into L2 while the layer waits for its routing (their bytes are
- * read again, from L2, only if they are chosen). */
-MOE_API int moe_set_decode_fused(int enable, int spec_experts);
-/* L2 prefetch policy of the fused batch-1 kernel (bit flags, default 0):
- * 2 = prefetch the next layer's routing-independent rows ahead of time;
- * 1 is reserved (no effect). */
-MOE_API int moe_set_decode_prefetch(int flags);
-/* Phase timestamps of the fused batch-1 kernel (a tracing aid): when
- * `stamps` (device, [L][G][16] uint64, G = moe_decode_grid()) is non-NULL,
- * thread 0 of every CTA writes %globaltimer (ns) at the phase boundaries of
- * each layer: 0 start, 1 norm done, 2 router logit sent and shared gate/up
- * done, 3 every router logit received, 4 top-k done, 5 gates done, 6 routed
- * gate/up done, 7 activations written and down copies issued, 8 after the
- * first grid barrier, 9 activations staged, 10 down dots done, 11 and 12
- * combine done, 13 after the second grid barrier; the copy-issuing thread
- * writes 14 (routed copies issued) and 15 (last routed tile landed).  NULL
- * turns it off (default). */
+/* Phase timestamps of the persistent batch-1 kernel (a tracing aid that never
+ * changes results).  Applies to moe_decode_forward calls made later by the
+ * calling thread: when `stamps` (device, [L][G][16] uint64, G =
+ * moe_decode_grid()) is non-NULL, thread 0 of every CTA writes %globaltimer
+ * (ns) at the phase boundaries of each layer (the points are listed in the
+ * kernel's source).  NULL turns it off (default). */
 MOE_API int moe_set_decode_profile(unsigned long long* stamps);
-/* CTAs of the fused batch-1 kernel on the current device (0: not available). */
+/* CTAs of the persistent batch-1 kernel on the current device (0: not available). */
 MOE_API int moe_decode_grid(void);
-/* Number of kernels one moe_decode_forward(T, L) call launches. */
-MOE_API int moe_decode_launches(int T, int L);
+/* Number of kernels one moe_decode_forward(T, L, flags) call launches. */
+MOE_API int moe_decode_launches(int T, int L, int flags);
 MOE_API int moe_decode_forward(float* h, int T, int H, int I, int Is, int E, int k, int L,
                                const moe_qmat* routers, const float* const* biases,
                                int bias_per_row, const void* const* const* blob_tables,
                                const moe_qmat* shared, uint16_t* x_trace, uint16_t* y_trace,
                                int32_t* idx_trace, float* gates_trace, void* ws,
-                               size_t ws_bytes, void* stream);
+                               size_t ws_bytes, int flags, void* stream);
 
 /* ------------------------------------------------------------------------
  * Per-layer LFU expert-slot cache (routed experts streamed from pinned host
@@ -300,7 +342,14 @@ MOE_API int moe_lfu_plan(moe_lfu* h, int layer, const int32_t* ids, int n, int32
  * each missed blob into its slot (one cudaMemcpyAsync per miss), update the
  * layer's device pointer table dev_table [E] for the step's ids, and record
  * `done_event`; the caller's compute stream waits on done_event before the
- * expert kernels.  Host waits are bounded by timeout_ms (MOE_ERR_TIMEOUT). */
+ * expert kernels.  Host waits are bounded by timeout_ms (MOE_ERR_TIMEOUT).
+ * A step is all or nothing for the cache state: when any part of it fails
+ * (a copy that cannot be issued, a wait that runs out) the layer's state and
+ * log are restored to what they were before the call and the error is
+ * returned; slots that copies issued by the failed call overwrite are marked,
+ * and the next step that hits the expert such a slot holds copies its blob
+ * again (logged as the hit the policy makes it).  Repeating the failed call
+ * therefore plans exactly as the first attempt would have. */
 MOE_API int moe_lfu_step(moe_lfu* h, int layer, const int32_t* ids, int n, void* side_stream,
                          void* wait_event, void* done_event, void** dev_table, int timeout_ms);
 /* Poll an event until it completes or timeout_ms passes (MOE_ERR_TIMEOUT). */
@@ -309,8 +358,8 @@ MOE_API int moe_lfu_wait(void* event, int timeout_ms);
  * slot); up to cap_records are copied into buf (may be NULL). */
 MOE_API int moe_lfu_get_log(moe_lfu* h, int32_t* buf, size_t cap_records, size_t* n_records);
 MOE_API int moe_lfu_stats(moe_lfu* h, int64_t* hits, int64_t* misses, int64_t* bytes_copied);
-/* Test hook: after `after_n` copies, every further copy fails (kind 1) or is
- * delayed by 50 ms on the host (kind 2); kind 0 clears it. */
+/* Test hook: after `after_n` copies, every further copy fails before it is
+ * issued (kind 1) or is delayed by 50 ms on the host (kind 2); kind 0 clears it. */
 MOE_API int moe_lfu_set_fault(moe_lfu* h, int kind, int after_n);
 MOE_API int moe_lfu_destroy(moe_lfu* h);
 
@@ -323,16 +372,24 @@ MOE_API int moe_lfu_destroy(moe_lfu* h);
  * chunk's distinct experts, resident ones first, each group ascending, k per
  * step); per step moe_lfu_step stages the blobs and main_stream runs the
  * expert kernels for that step's experts through dev_table; then the combine
- * adds y into hres.  The per-pair arithmetic is that of moe_layer_forward,
- * so the result equals the all-resident layer bit for bit.
+ * adds y into hres.  The per-pair arithmetic is that of moe_layer_forward
+ * with the same flags, so the result equals the all-resident layer bit for bit.
+ * Source: "TurboFieldfare: Gemma 4 26B on an 8 GB MacBook, in ~2 GB of RAM"
+ * (blog-mushroom.pages.dev), section "Why 26B Fits in 2 GB" (hits reuse the
+ * resident blob, misses fetch it, the shared expert runs meanwhile).
  *   dev_table  device [E] pointer table of this layer (updated per step)
- *   ws         device workspace >= moe_streamed_workspace_size(...) */
+ *   ws         device workspace >= moe_streamed_workspace_size(...)
+ *   flags      MOE_FLAG_* as in moe_layer_forward
+ * All the steps of one call form one transaction of the cache (see
+ * moe_lfu_step): if the call fails after planning, the layer's cache state
+ * and log are as before the call and hres is unchanged, so the caller may
+ * repeat the call. */
 MOE_API size_t moe_streamed_workspace_size(int T, int H, int I, int Is, int E, int k);
 MOE_API int moe_streamed_layer_forward(moe_lfu* h, int layer, float* hres, int T, int H, int I, int Is,
                                        int E, int k, const moe_qmat* router, const float* bias,
                                        int bias_per_row, const moe_qmat* shared, void** dev_table,
                                        uint16_t* x_out, uint16_t* y_out, int32_t* idx_out, void* ws,
-                                       size_t ws_bytes, void* main_stream, void* side_stream,
+                                       size_t ws_bytes, int flags, void* main_stream, void* side_stream,
                                        int timeout_ms);
 
 #ifdef __cplusplus

@@ -15,6 +15,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libmoe.so")
 
 MOE_OK = 0
+# per-call path flags (include/moe.h)
+MOE_FLAG_GEMV, MOE_FLAG_TC, MOE_FLAG_LAYERED = 1, 2, 4
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_CUDA", 3: "MOE_ERR_TIMEOUT",
           4: "MOE_ERR_DEVICE_CHECK", 5: "MOE_ERR_UNSUPPORTED"}
 
@@ -43,25 +45,20 @@ SIGNATURES = {
     "moe_router_topk": (_I, [_P, _I, _I, C.POINTER(moe_qmat), _P, _I, _I, _I, _P, _P, _P, _P]),
     "moe_bucket": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P]),
     "moe_expert_workspace_size": (_Z, [_I, _I, _I, _I]),
-    "moe_expert_workspace_size_mma": (_Z, [_I, _I, _I, _I]),
-    "moe_set_grouped_mma": (_I, [_I]),
-    "moe_expert_forward": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _Z, _P]),
+    "moe_expert_forward": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _Z, _I, _P]),
     "moe_expert_forward_noalloc": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
-    "moe_set_gemv_max_rows": (_I, [_I]),
     "moe_shared_workspace_size": (_Z, [_I, _I, _I]),
-    "moe_shared_forward": (_I, [_P, _I, _I, _I, C.POINTER(moe_qmat), _P, _P, _Z, _P]),
+    "moe_shared_forward": (_I, [_P, _I, _I, _I, C.POINTER(moe_qmat), _P, _P, _Z, _I, _P]),
     "moe_combine": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _P]),
     "moe_layer_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
     "moe_layer_forward": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, C.POINTER(moe_qmat), _P, _I, _P,
-                               C.POINTER(moe_qmat), _P, _P, _P, _P, _P, _Z, _P]),
+                               C.POINTER(moe_qmat), _P, _P, _P, _P, _P, _Z, _I, _P]),
     "moe_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
-    "moe_decode_launches": (_I, [_I, _I]),
-    "moe_set_decode_fused": (_I, [_I, _I]),
+    "moe_decode_launches": (_I, [_I, _I, _I]),
     "moe_set_decode_profile": (_I, [_P]),
-    "moe_set_decode_prefetch": (_I, [_I]),
     "moe_decode_grid": (_I, []),
     "moe_decode_forward": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, C.POINTER(moe_qmat), C.POINTER(C.c_void_p), _I,
-                                C.POINTER(C.c_void_p), C.POINTER(moe_qmat), _P, _P, _P, _P, _P, _Z, _P]),
+                                C.POINTER(C.c_void_p), C.POINTER(moe_qmat), _P, _P, _P, _P, _P, _Z, _I, _P]),
     "moe_lfu_create": (_I, [_I, _I, _I, _Z, _P, _P, _Z, C.POINTER(C.c_void_p)]),
     "moe_lfu_plan": (_I, [_P, _I, _P, _I, _P, _P]),
     "moe_lfu_step": (_I, [_P, _I, _P, _I, _P, _P, _P, _P, _I]),
@@ -72,7 +69,7 @@ SIGNATURES = {
     "moe_lfu_destroy": (_I, [_P]),
     "moe_streamed_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
     "moe_streamed_layer_forward": (_I, [_P, _I, _P, _I, _I, _I, _I, _I, _I, C.POINTER(moe_qmat), _P, _I,
-                                        C.POINTER(moe_qmat), _P, _P, _P, _P, _P, _Z, _P, _P, _I]),
+                                        C.POINTER(moe_qmat), _P, _P, _P, _P, _P, _Z, _I, _P, _P, _I]),
 }
 
 

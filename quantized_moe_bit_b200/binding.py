@@ -7,7 +7,7 @@ from __future__ import annotations
 
 import ctypes as C
 
-from ._lib import check, lib, moe_qmat, ptr, stream_ptr
+from ._lib import MOE_FLAG_GEMV, MOE_FLAG_LAYERED, MOE_FLAG_TC, check, lib, moe_qmat, ptr, stream_ptr  # noqa: F401
 
 
 def moe_version() -> int:
@@ -22,10 +22,6 @@ def moe_blob_bytes(H: int, I: int):
     offs = (C.c_size_t * 9)()
     n = lib().moe_blob_bytes(H, I, offs)
     return n, list(offs)
-
-
-def moe_set_gemv_max_rows(rows: int):
-    check(lib().moe_set_gemv_max_rows(rows))
 
 
 def moe_rmsnorm(h, x, eps: float = 1e-6, stream=None):
@@ -50,20 +46,12 @@ def moe_expert_workspace_size(T: int, H: int, I: int, k: int) -> int:
     return lib().moe_expert_workspace_size(T, H, I, k)
 
 
-def moe_expert_workspace_size_mma(T: int, H: int, I: int, k: int) -> int:
-    return lib().moe_expert_workspace_size_mma(T, H, I, k)
-
-
-def moe_set_grouped_mma(enable: bool):
-    check(lib().moe_set_grouped_mma(1 if enable else 0))
-
-
 def moe_expert_forward(x, I: int, E: int, k: int, blob_ptrs, offsets, pairs, active, n_active, y_pairs,
-                       ws, stream=None):
+                       ws, flags: int = 0, stream=None):
     T, H = x.shape
     check(lib().moe_expert_forward(ptr(x), T, H, I, E, k, ptr(blob_ptrs), ptr(offsets), ptr(pairs),
                                    ptr(active), ptr(n_active), ptr(y_pairs), ptr(ws), ws.numel() * ws.element_size(),
-                                   stream_ptr(stream)))
+                                   flags, stream_ptr(stream)))
 
 
 def moe_expert_forward_noalloc(x, I: int, E: int, k: int, blob_ptrs, offsets, pairs, active, n_active,
@@ -84,11 +72,11 @@ def _qmat3(shared):
     return arr
 
 
-def moe_shared_forward(x, Is: int, shared, ysh, ws, stream=None):
+def moe_shared_forward(x, Is: int, shared, ysh, ws, flags: int = 0, stream=None):
     T, H = x.shape
     arr = _qmat3(shared)
     check(lib().moe_shared_forward(ptr(x), T, H, Is, arr, ptr(ysh), ptr(ws), ws.numel() * ws.element_size(),
-                                   stream_ptr(stream)))
+                                   flags, stream_ptr(stream)))
 
 
 def moe_combine(y_pairs, gates, ysh, y=None, residual=None, stream=None):
@@ -104,31 +92,23 @@ def moe_layer_workspace_size(T: int, H: int, I: int, Is: int, E: int, k: int) ->
 
 def moe_layer_forward(T: int, H: int, I: int, Is: int, E: int, k: int, router: moe_qmat, bias,
                       bias_per_row: int, blob_ptrs, shared, ws, h_in=None, h_out=None, x_in=None,
-                      x_out=None, y=None, idx=None, gates=None, stream=None):
+                      x_out=None, y=None, idx=None, gates=None, flags: int = 0, stream=None):
     arr = _qmat3(shared)
     check(lib().moe_layer_forward(ptr(h_in), ptr(h_out), ptr(x_in), T, H, I, Is, E, k, C.byref(router),
                                   ptr(bias), bias_per_row, ptr(blob_ptrs), arr, ptr(x_out), ptr(y), ptr(idx),
-                                  ptr(gates), ptr(ws), ws.numel() * ws.element_size(), stream_ptr(stream)))
-
-
-def moe_set_decode_fused(enable: bool, spec_experts: int = 0):
-    check(lib().moe_set_decode_fused(1 if enable else 0, spec_experts))
+                                  ptr(gates), ptr(ws), ws.numel() * ws.element_size(), flags, stream_ptr(stream)))
 
 
 def moe_set_decode_profile(stamps=None):
     check(lib().moe_set_decode_profile(ptr(stamps)))
 
 
-def moe_set_decode_prefetch(flags: int):
-    check(lib().moe_set_decode_prefetch(flags))
-
-
 def moe_decode_grid() -> int:
     return lib().moe_decode_grid()
 
 
-def moe_decode_launches(T: int, L: int) -> int:
-    return lib().moe_decode_launches(T, L)
+def moe_decode_launches(T: int, L: int, flags: int = 0) -> int:
+    return lib().moe_decode_launches(T, L, flags)
 
 
 def moe_decode_workspace_size(T: int, H: int, I: int, Is: int, E: int, k: int) -> int:
@@ -154,12 +134,12 @@ class DecodeStack:
 
 
 def moe_decode_forward(h, I: int, Is: int, E: int, k: int, stack: "DecodeStack", ws, x_trace=None,
-                       y_trace=None, idx_trace=None, gates_trace=None, stream=None):
+                       y_trace=None, idx_trace=None, gates_trace=None, flags: int = 0, stream=None):
     T, H = h.shape
     check(lib().moe_decode_forward(ptr(h), T, H, I, Is, E, k, stack.L, stack.routers, stack.biases,
                                    stack.bias_per_row, stack.tables, stack.shared, ptr(x_trace), ptr(y_trace),
                                    ptr(idx_trace), ptr(gates_trace), ptr(ws), ws.numel() * ws.element_size(),
-                                   stream_ptr(stream)))
+                                   flags, stream_ptr(stream)))
 
 
 # ------------------------------------------------------------------ LFU cache
@@ -233,10 +213,10 @@ def moe_streamed_workspace_size(T: int, H: int, I: int, Is: int, E: int, k: int)
 
 def moe_streamed_layer_forward(lfu: "MoeLfu", layer: int, h, I: int, Is: int, E: int, k: int, router: moe_qmat,
                                bias, bias_per_row: int, shared, dev_table, ws, x_out=None, y_out=None, idx_out=None,
-                               main_stream=None, side_stream=None, timeout_ms: int = 5000):
+                               flags: int = 0, main_stream=None, side_stream=None, timeout_ms: int = 5000):
     T, H = h.shape
     arr = _qmat3(shared)
     check(lib().moe_streamed_layer_forward(lfu.handle, layer, ptr(h), T, H, I, Is, E, k, C.byref(router), ptr(bias),
                                            bias_per_row, arr, ptr(dev_table), ptr(x_out), ptr(y_out), ptr(idx_out),
-                                           ptr(ws), ws.numel() * ws.element_size(), stream_ptr(main_stream),
+                                           ptr(ws), ws.numel() * ws.element_size(), flags, stream_ptr(main_stream),
                                            stream_ptr(side_stream), timeout_ms))

@@ -6,63 +6,14 @@
 
 #include "gemv.cuh"
 #include "kernels.cuh"
-#include "tc_gemm.cu"
+#include "moe_gemm.cu"
 #include "decode_fused.cu"
-#include "grouped_mma.cu"
 
 namespace moe {
 
 static thread_local char g_err[512] = "";
-static int g_gemv_max_rows = 2;
-static int g_grouped_mma = 0;            // buckets of 3..32 rows on the grouped mma.sync kernel (off: measured slower)
-
-// Two library-owned streams per device for independent parts of a call (the
-// shared expert, the GEMV buckets), forked from and joined back into the
-// caller's stream with events, so a captured graph gets the same branches.
-// Created on first use, kept until exit; the fork-launch-join sequence of a
-// call holds g_fork_mu so that concurrent host threads do not mix events.
-struct SideStreams {
-  cudaStream_t st[2] = {nullptr, nullptr};
-  cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
-};
-static std::recursive_mutex g_fork_mu;
-static SideStreams* side_streams() {
-  static SideStreams per_dev[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  SideStreams& S = per_dev[dev];
-  if (!S.st[0]) {
-    for (int i = 0; i < 2; ++i)
-      if (cudaStreamCreateWithFlags(&S.st[i], cudaStreamNonBlocking) != cudaSuccess) { cudaGetLastError(); return nullptr; }
-    for (int i = 0; i < 4; ++i)
-      if (cudaEventCreateWithFlags(&S.ev[i], cudaEventDisableTiming) != cudaSuccess) { cudaGetLastError(); return nullptr; }
-  }
-  return &S;
-}
-int cuda_check(cudaError_t e, const char* what);
-// `to` waits for the work issued so far on `from` (event ev)
-static int stream_after(cudaStream_t to, cudaStream_t from, cudaEvent_t ev) {
-  int st = cuda_check(cudaEventRecord(ev, from), "cudaEventRecord");
-  if (st) return st;
-  return cuda_check(cudaStreamWaitEvent(to, ev, 0), "cudaStreamWaitEvent");
-}
-
-// CTAs of the persistent grouped kernel: one per SM (cached per device).
-static int grouped_grid() {
-  static int cached[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
-    int nsm = 0;
-    if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0) nsm = 148;
-    cached[dev] = nsm;
-  }
-  return cached[dev];
-}
-static int g_decode_fused = 1;
-static int g_decode_spec = 0;
-static int g_decode_prefetch = 0;
-static unsigned long long* g_decode_stamps = nullptr;
+// phase timestamps of the persistent batch-1 kernel for this thread's calls (tracing aid)
+static thread_local unsigned long long* g_decode_stamps = nullptr;
 
 int fail(int code, const char* fmt, ...) {
   va_list ap;
@@ -102,6 +53,14 @@ static int check_dims(int T, int H, int I, int E, int k) {
   return MOE_OK;
 }
 
+static int check_flags(int flags) {
+  if (flags & ~(MOE_FLAG_GEMV | MOE_FLAG_TC | MOE_FLAG_LAYERED))
+    return fail(MOE_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+  if ((flags & MOE_FLAG_GEMV) && (flags & MOE_FLAG_TC))
+    return fail(MOE_ERR_INVALID_ARG, "MOE_FLAG_GEMV and MOE_FLAG_TC exclude each other");
+  return MOE_OK;
+}
+
 // Raise a kernel's dynamic shared-memory limit once per (device, kernel);
 // later calls (also inside stream capture) find it done and make no API call.
 static int set_smem(const void* fn, size_t bytes) {
@@ -109,6 +68,8 @@ static int set_smem(const void* fn, size_t bytes) {
   struct Entry { const void* fn; int dev; size_t bytes; };
   static Entry table[64];
   static int n = 0;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
   for (int i = 0; i < n; ++i)
@@ -125,6 +86,267 @@ static int set_smem(const void* fn, size_t bytes) {
 
 static size_t gemv_smem(int K) {
   return GEMV_RG * staged_row_bytes(K) + static_cast<size_t>(GEMV_RG) * (K / 8) * sizeof(float2);
+}
+
+// SMs of the current device (cached per device): the persistent grids.
+static int sm_count() {
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int nsm = 0;
+    if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0) nsm = 148;
+    cached[dev] = nsm;
+  }
+  return cached[dev];
+}
+
+// ------------------------------------------------------- tensor maps (TMA)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// The GM_NBOX activation tensor maps of one fp16 matrix [rows, cols]
+// (row-major): boxes of 64 columns (128 bytes, 128-byte swizzle) by
+// 16, 32, 64 or 128 rows; rows beyond the matrix read as zero.
+static int make_act_maps(CUtensorMap* maps, const void* base, int rows, int cols) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  for (int i = 0; i < GM_NBOX; ++i) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(gm_box_rows(i))};
+    const cuuint32_t es[2] = {1u, 1u};
+    const CUresult r = enc(&maps[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                           es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  }
+  return MOE_OK;
+}
+
+// The tensor map of a matrix's packed codes: uint8 [rows, row_bytes]
+// (row-major), boxes of 128 bytes (256 4-bit values) by box_rows rows,
+// 128-byte swizzle; bytes beyond a row's end read as zero.
+static int make_code_map(CUtensorMap* map, const void* base, int rows, int row_bytes, int box_rows) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t es[2] = {1u, 1u};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled (codes) failed (%d)", static_cast<int>(r));
+  return MOE_OK;
+}
+
+// ------------------------------------------------------- expert path
+// Which kernels serve the experts of a T-row call: the GEMV kernels for T <= 2
+// (or MOE_FLAG_GEMV), the grouped GEMM otherwise (or MOE_FLAG_TC), when the
+// shapes fit it.
+static bool gemm_shapes_ok(int T, int H, int I, int Is, int E, int k) {
+  if (H % GM_BM || H > GM_MAX_G * 64 || I > GM_MAX_G * 64 || Is > GM_MAX_G * 64) return false;
+  const long P = static_cast<long>(T) * k;
+  const long chunks = (E < P ? E : P) + (P + GM_NMAX - 1) / GM_NMAX + (T + GM_NMAX - 1) / GM_NMAX;
+  return P < (1L << 24) && chunks <= GM_MAX_CHUNKS;
+}
+static bool use_gemm(int T, int H, int I, int Is, int E, int k, int flags) {
+  if (flags & MOE_FLAG_GEMV) return false;
+  if (!(flags & MOE_FLAG_TC) && T <= 2) return false;
+  return gemm_shapes_ok(T, H, I, Is, E, k);
+}
+
+// Workspace carving of the expert calls (every region 256-byte aligned).
+struct ExpertWs {      // routed experts
+  GmPlan* plan;
+  CUtensorMap* maps;   // [GM_MAX_CTAS][GM_MAP_RING][2] per-CTA patched code maps (grouped GEMM only)
+  __half* act;         // [T*k, I] bucket order
+  __half* xs;          // [T*k, H] the layer input gathered into bucket order (grouped GEMM only)
+};
+constexpr size_t GM_RING_BYTES = static_cast<size_t>(GM_MAX_CTAS) * GM_MAP_RING * 2 * sizeof(CUtensorMap);
+static size_t expert_ws_bytes(int T, int H, int I, int k) {
+  const size_t P = static_cast<size_t>(T) * k;
+  return align_up(sizeof(GmPlan)) + align_up(GM_RING_BYTES) + align_up(P * I * 2) + align_up(P * H * 2);
+}
+static ExpertWs carve_expert(void* ws, int T, int H, int I, int k) {
+  const size_t P = static_cast<size_t>(T) * k;
+  char* p = static_cast<char*>(ws);
+  ExpertWs w;
+  w.plan = reinterpret_cast<GmPlan*>(p); p += align_up(sizeof(GmPlan));
+  w.maps = reinterpret_cast<CUtensorMap*>(p); p += align_up(GM_RING_BYTES);
+  w.act = reinterpret_cast<__half*>(p); p += align_up(P * I * 2);
+  w.xs = reinterpret_cast<__half*>(p);
+  (void)H;
+  return w;
+}
+struct SharedWs {
+  GmPlan* plan;
+  __half* act;         // [T, Is]
+  __half* xh;          // [T, H] the layer input as fp16 (grouped GEMM only)
+};
+static size_t shared_ws_bytes(int T, int H, int Is) {
+  return align_up(sizeof(GmPlan)) + align_up(static_cast<size_t>(T) * Is * 2) + align_up(static_cast<size_t>(T) * H * 2);
+}
+static SharedWs carve_shared(void* ws, int T, int H, int Is) {
+  char* p = static_cast<char*>(ws);
+  SharedWs w;
+  w.plan = reinterpret_cast<GmPlan*>(p); p += align_up(sizeof(GmPlan));
+  w.act = reinterpret_cast<__half*>(p); p += align_up(static_cast<size_t>(T) * Is * 2);
+  w.xh = reinterpret_cast<__half*>(p);
+  (void)H;
+  return w;
+}
+
+// The grouped GEMM over a routed segment (rt != null) and/or the shared
+// expert (sh != null) of one T-row step: prep, gate/up, down.
+struct RoutedIn {
+  const void* const* blob_ptrs; const int32_t* offsets; const int32_t* pairs; const int32_t* active;
+  const int32_t* n_active; float* y_pairs; int I, E, k;
+};
+struct SharedIn {
+  const moe_qmat* m; float* ysh; int Is;
+};
+static int run_gemm(const uint16_t* x, int T, int H, const RoutedIn* rt, const SharedIn* sh, GmPlan* plan,
+                    CUtensorMap* map_ring, __half* act_r, __half* xs, __half* act_s, __half* xh, cudaStream_t s) {
+  int st;
+  const int k = rt ? rt->k : 1;
+  const long P = rt ? static_cast<long>(T) * k : 0;
+  {
+    const long work = (P + (sh ? T : 0)) * (H / 8);
+    int blocks = static_cast<int>((work + 255) / 256);
+    blocks = blocks < 1 ? 1 : (blocks > 4 * sm_count() ? 4 * sm_count() : blocks);
+    k_gm_prep<<<blocks, 256, 0, s>>>(x, T, H, k, rt ? rt->offsets : nullptr, rt ? rt->pairs : nullptr,
+                                     rt ? rt->active : nullptr, rt ? rt->n_active : nullptr, rt ? rt->E : 0,
+                                     rt ? 1 : 0, sh ? T : 0, xs, sh ? xh : nullptr, plan);
+    if ((st = launch_check("k_gm_prep"))) return st;
+  }
+  if ((st = set_smem(reinterpret_cast<const void*>(k_moe_gemm), GM_SMEM))) return st;
+  static thread_local GemmArgs g;       // large parameter block (tensor maps); the launch copies it
+  memset(&g, 0, sizeof(g));
+  g.H = H;
+  g.plan = plan;
+  if (rt) {
+    g.I = rt->I; g.E = rt->E; g.k = rt->k;
+    g.blob_ptrs = rt->blob_ptrs; g.pairs = rt->pairs; g.P = static_cast<int>(P);
+    blob_offsets(H, rt->I, g.off);
+    g.act_r = act_r; g.y_r = rt->y_pairs;
+  }
+  if (sh) {
+    g.Is = sh->Is; g.Ts = T;
+    for (int m = 0; m < 3; ++m) {
+      g.sq[m] = reinterpret_cast<const uint8_t*>(sh->m[m].q); g.ss[m] = sh->m[m].s; g.sb[m] = sh->m[m].b;
+    }
+    g.act_s = act_s; g.y_s = sh->ysh;
+  } else {
+    g.Is = 64;   // unused (no shared chunks); keeps the m-tile count well defined
+  }
+  if (!rt) g.I = 64;
+  const int grid = sm_count() < GM_MAX_CTAS ? sm_count() : GM_MAX_CTAS;
+  g.map_ring = map_ring;
+  for (int phase = 0; phase < 2; ++phase) {
+    g.phase = phase;
+    // code maps: the routed template (any valid address; replaced per item)
+    // and the shared expert's matrices
+    const int box_rows = phase == 0 ? 64 : GM_BM;
+    if (rt && (st = make_code_map(&g.tmR, map_ring, phase == 0 ? rt->I : H, phase == 0 ? H / 2 : rt->I / 2, box_rows)))
+      return st;
+    if (sh) {
+      if (phase == 0) {
+        if ((st = make_code_map(&g.tmS[0], sh->m[0].q, sh->Is, H / 2, box_rows))) return st;
+        if ((st = make_code_map(&g.tmS[1], sh->m[1].q, sh->Is, H / 2, box_rows))) return st;
+      } else if ((st = make_code_map(&g.tmS[0], sh->m[2].q, H, sh->Is / 2, box_rows))) {
+        return st;
+      }
+    }
+    if (rt && (st = make_act_maps(g.tmB[1], phase == 0 ? static_cast<const void*>(xs) : act_r, static_cast<int>(P),
+                                  phase == 0 ? H : rt->I)))
+      return st;
+    if (sh && (st = make_act_maps(g.tmB[0], phase == 0 ? static_cast<const void*>(xh) : act_s, T,
+                                  phase == 0 ? H : sh->Is)))
+      return st;
+    k_moe_gemm<<<grid, GM_THREADS, GM_SMEM, s>>>(g);
+    if ((st = launch_check(phase == 0 ? "k_moe_gemm(gate/up)" : "k_moe_gemm(down)"))) return st;
+  }
+  return MOE_OK;
+}
+
+static int check_shared_mats(const moe_qmat* sh, int H, int Is) {
+  for (int m = 0; m < 3; ++m) {
+    const int out = m < 2 ? Is : H, in = m < 2 ? H : Is;
+    if (!sh[m].q || !sh[m].s || !sh[m].b || sh[m].bits != 4 || sh[m].out != out || sh[m].in != in)
+      return fail(MOE_ERR_INVALID_ARG, "shared expert: matrix %d must be 4-bit [%d, %d]", m, out, in);
+    if (!aligned16(sh[m].q) || !aligned16(sh[m].s) || !aligned16(sh[m].b))
+      return fail(MOE_ERR_INVALID_ARG, "shared expert: matrix %d arrays must be 16-byte aligned", m);
+  }
+  return MOE_OK;
+}
+
+// GEMV path of the routed experts (every bucket): gate/up + GeGLU, then down.
+static int run_routed_gemv(const uint16_t* x, int T, int H, int I, int E, int k, const void* const* blob_ptrs,
+                           const int32_t* offsets, const int32_t* pairs, const int32_t* active,
+                           const int32_t* n_active, float* y_pairs, __half* act, cudaStream_t s) {
+  int st;
+  const int maxA = T * k < E ? T * k : E;
+  GateUpArgs g{};
+  g.x = x; g.T = T; g.H = H; g.I = I; g.E = E; g.k = k;
+  g.blob_ptrs = blob_ptrs; g.offsets = offsets; g.pairs = pairs; g.active = active; g.n_active = n_active;
+  g.max_rows = 1 << 30;
+  blob_offsets(H, I, g.off);
+  g.act = act;
+  size_t sm = gemv_smem(H);
+  if ((st = set_smem(reinterpret_cast<const void*>(k_gateup_gemv), sm))) return st;
+  k_gateup_gemv<<<dim3((I + GEMV_ROWS - 1) / GEMV_ROWS, maxA), 256, sm, s>>>(g);
+  if ((st = launch_check("k_gateup_gemv"))) return st;
+  DownArgs d{};
+  d.act = act; d.T = T; d.H = H; d.I = I; d.E = E; d.k = k;
+  d.blob_ptrs = blob_ptrs; d.offsets = offsets; d.pairs = pairs; d.active = active; d.n_active = n_active;
+  d.max_rows = 1 << 30;
+  blob_offsets(H, I, d.off);
+  d.y = y_pairs;
+  sm = gemv_smem(I);
+  if ((st = set_smem(reinterpret_cast<const void*>(k_down_gemv), sm))) return st;
+  k_down_gemv<<<dim3((H + GEMV_ROWS - 1) / GEMV_ROWS, maxA), 256, sm, s>>>(d);
+  return launch_check("k_down_gemv");
+}
+
+// GEMV path of the shared expert.
+static int run_shared_gemv(const uint16_t* x, int T, int H, int Is, const moe_qmat* sh, float* ysh, __half* act,
+                           cudaStream_t s) {
+  int st;
+  GateUpArgs g{};
+  g.x = x; g.T = T; g.H = H; g.I = Is; g.E = 1; g.k = 1; g.max_rows = 1 << 30;
+  g.gq = sh[0].q; g.gs = sh[0].s; g.gb = sh[0].b;
+  g.uq = sh[1].q; g.us = sh[1].s; g.ub = sh[1].b;
+  g.act = act;
+  size_t sm = gemv_smem(H);
+  if ((st = set_smem(reinterpret_cast<const void*>(k_gateup_gemv), sm))) return st;
+  k_gateup_gemv<<<dim3((Is + GEMV_ROWS - 1) / GEMV_ROWS, 1), 256, sm, s>>>(g);
+  if ((st = launch_check("k_gateup_gemv(shared)"))) return st;
+  DownArgs d{};
+  d.act = act; d.T = T; d.H = H; d.I = Is; d.E = 1; d.k = 1; d.max_rows = 1 << 30;
+  d.dq = sh[2].q; d.ds = sh[2].s; d.db = sh[2].b;
+  d.y = ysh;
+  sm = gemv_smem(Is);
+  if ((st = set_smem(reinterpret_cast<const void*>(k_down_gemv), sm))) return st;
+  k_down_gemv<<<dim3((H + GEMV_ROWS - 1) / GEMV_ROWS, 1), 256, sm, s>>>(d);
+  return launch_check("k_down_gemv(shared)");
 }
 
 }  // namespace moe
@@ -157,17 +379,6 @@ size_t moe_blob_bytes(int H, int I, size_t* offsets9) {
   blob_offsets(H, I, off);
   if (offsets9) memcpy(offsets9, off, sizeof(off));
   return 3 * (static_cast<size_t>(I) * H / 2 + static_cast<size_t>(I) * (H / 64) * 4);
-}
-
-int moe_set_grouped_mma(int enable) {
-  g_grouped_mma = enable ? 1 : 0;
-  return MOE_OK;
-}
-
-int moe_set_gemv_max_rows(int rows) {
-  if (rows < 0) return fail(MOE_ERR_INVALID_ARG, "gemv_max_rows must be >= 0");
-  g_gemv_max_rows = rows;
-  return MOE_OK;
 }
 
 int moe_rmsnorm(const float* h, int T, int H, float eps, uint16_t* x, void* stream) {
@@ -211,27 +422,16 @@ int moe_bucket(const int32_t* idx, int T, int k, int E, int32_t* offsets, int32_
 }
 
 size_t moe_expert_workspace_size(int T, int H, int I, int k) {
-  // fp16 activation between the projections + fp16 copy of x for the tensor-core path
-  return align_up(static_cast<size_t>(T) * k * I * sizeof(__half)) + align_up(static_cast<size_t>(T) * H * sizeof(__half));
-}
-
-// Paired activation rows (x and the gate/up activation) for the grouped
-// mma.sync kernel: fp16 pairs [rows, K] plus fp32 group sums [rows, K/64] x 2.
-static size_t mma_extra_bytes(int T, int H, int I, int k) {
-  const size_t tk = static_cast<size_t>(T) * k;
-  return align_up(static_cast<size_t>(T) * H * 2) + align_up(static_cast<size_t>(T) * (H / 64) * 8) +
-         align_up(tk * I * 2) + align_up(tk * (I / 64) * 8) + align_up(8);   // + the two work counters
-}
-
-size_t moe_expert_workspace_size_mma(int T, int H, int I, int k) {
-  return moe_expert_workspace_size(T, H, I, k) + mma_extra_bytes(T, H, I, k);
+  if (T < 0 || H <= 0 || I <= 0 || k <= 0) return 0;
+  return expert_ws_bytes(T, H, I, k);
 }
 
 int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, int k, const void* const* blob_ptrs,
                        const int32_t* offsets, const int32_t* pairs, const int32_t* active,
-                       const int32_t* n_active, float* y_pairs, void* ws, size_t ws_bytes, void* stream) {
+                       const int32_t* n_active, float* y_pairs, void* ws, size_t ws_bytes, int flags, void* stream) {
   int st = check_dims(T, H, I, E, k);
   if (st) return st;
+  if ((st = check_flags(flags))) return st;
   if (T == 0) return MOE_OK;
   if (!x || !blob_ptrs || !offsets || !pairs || !active || !n_active || !y_pairs || !ws)
     return fail(MOE_ERR_INVALID_ARG, "moe_expert_forward: NULL pointer");
@@ -240,179 +440,40 @@ int moe_expert_forward(const uint16_t* x, int T, int H, int I, int E, int k, con
   if (!aligned16(x) || !aligned16(ws) || !aligned16(y_pairs))
     return fail(MOE_ERR_INVALID_ARG, "moe_expert_forward: misaligned pointer");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  __half* act = static_cast<__half*>(ws);
-  __half* xh = reinterpret_cast<__half*>(static_cast<char*>(ws) + align_up(static_cast<size_t>(T) * k * I * sizeof(__half)));
-  const int maxA = T * k < E ? T * k : E;
-  // Buckets of at most gemv_max_rows rows go to the GEMV kernels, larger ones
-  // to the tensor-core kernel (shapes it supports: H % 128 == 0, H, I <= 4096);
-  // with the larger workspace, buckets of up to GM_NMAX rows go to the grouped
-  // mma.sync kernel instead.
-  const bool tc = T > g_gemv_max_rows && H % 128 == 0 && H <= 4096 && I <= 4096;
-  const int gemv_rows = tc ? g_gemv_max_rows : (1 << 30);
-  const bool mma = tc && g_grouped_mma && grouped_mma_ok(H, I) &&
-                   ws_bytes >= moe_expert_workspace_size_mma(T, H, I, k);
-  const int tc_min = mma ? GM_NMAX : g_gemv_max_rows;     // the tensor-core kernel takes buckets above this
-  char* xw = static_cast<char*>(ws) + moe_expert_workspace_size(T, H, I, k);
-  uint4* xP = reinterpret_cast<uint4*>(xw);
-  float2* xS = reinterpret_cast<float2*>(xw + align_up(static_cast<size_t>(T) * H * 2));
-  uint4* aP = reinterpret_cast<uint4*>(xw + align_up(static_cast<size_t>(T) * H * 2) +
-                                       align_up(static_cast<size_t>(T) * (H / 64) * 8));
-  float2* aS = reinterpret_cast<float2*>(reinterpret_cast<char*>(aP) + align_up(static_cast<size_t>(T) * k * I * 2));
-  unsigned* queues = reinterpret_cast<unsigned*>(reinterpret_cast<char*>(aS) +
-                                                 align_up(static_cast<size_t>(T) * k * (I / 64) * 8));
-  GmArgs gm{};
-  if (mma) {
-    const size_t gsm = grouped_mma_smem(H, I);
-    if ((st = set_smem(reinterpret_cast<const void*>(k_group_mma), gsm))) return st;
-    const long nw = static_cast<long>(T) * (H / 8);
-    k_pair_rows<<<static_cast<int>((nw + 255) / 256 < 1024 ? (nw + 255) / 256 : 1024), 256, 0, s>>>(x, 1, T, H, xP, xS);
-    if ((st = launch_check("k_pair_rows(x)"))) return st;
-    gm.mode = 0; gm.P = xP; gm.S = xS; gm.T = T; gm.H = H; gm.I = I; gm.E = E; gm.k = k;
-    gm.blob_ptrs = blob_ptrs; blob_offsets(H, I, gm.off);
-    gm.offsets = offsets; gm.pairs = pairs; gm.active = active; gm.n_active = n_active;
-    gm.lo = g_gemv_max_rows; gm.hi = GM_NMAX;
-    gm.act_out = static_cast<__half*>(ws); gm.y_out = y_pairs;
-    if ((st = cuda_check(cudaMemsetAsync(queues, 0, 8, s), "zero work counters"))) return st;
-    gm.queue = queues;
-    k_group_mma<<<grouped_grid(), GM_THREADS, gsm, s>>>(gm);
-    if ((st = launch_check("k_group_mma(gate/up)"))) return st;
+  ExpertWs w = carve_expert(ws, T, H, I, k);
+  if (!use_gemm(T, H, I, 64, E, k, flags)) {
+    if (flags & MOE_FLAG_TC) return fail(MOE_ERR_UNSUPPORTED, "moe_expert_forward: shapes outside the grouped GEMM");
+    return run_routed_gemv(x, T, H, I, E, k, blob_ptrs, offsets, pairs, active, n_active, y_pairs, w.act, s);
   }
-
-  // with the tensor-core path, the GEMV buckets (disjoint rows of act and
-  // y_pairs) run on a side stream alongside it
-  std::unique_lock<std::recursive_mutex> fork_lock(g_fork_mu, std::defer_lock);
-  SideStreams* side = tc ? side_streams() : nullptr;
-  cudaStream_t gs = s;
-  if (side) {
-    fork_lock.lock();
-    gs = side->st[1];
-    if ((st = stream_after(gs, s, side->ev[2]))) return st;
-  }
-  GateUpArgs g{};
-  g.x = x; g.T = T; g.H = H; g.I = I; g.E = E; g.k = k;
-  g.blob_ptrs = blob_ptrs; g.offsets = offsets; g.pairs = pairs; g.active = active; g.n_active = n_active;
-  g.max_rows = gemv_rows;
-  blob_offsets(H, I, g.off);
-  g.act = act;
-  size_t sm = gemv_smem(H);
-  if ((st = set_smem(reinterpret_cast<const void*>(k_gateup_gemv), sm))) return st;
-  k_gateup_gemv<<<dim3((I + GEMV_ROWS - 1) / GEMV_ROWS, maxA), 256, sm, gs>>>(g);
-  if ((st = launch_check("k_gateup_gemv"))) return st;
-
-  TcArgs ta{};
-  if (tc) {
-    const size_t n8 = static_cast<size_t>(T) * H / 8;
-    k_to_f16<<<static_cast<int>((n8 + 255) / 256 < 1024 ? (n8 + 255) / 256 : 1024), 256, 0, s>>>(x, n8, xh);
-    if ((st = launch_check("k_to_f16"))) return st;
-    ta.mode = 0; ta.xh = xh; ta.T = T; ta.H = H; ta.I = I; ta.E = E; ta.k = k;
-    ta.blob_ptrs = blob_ptrs; ta.offsets = offsets; ta.pairs = pairs; ta.active = active; ta.n_active = n_active;
-    ta.max_rows = tc_min;
-    blob_offsets(H, I, ta.off);
-    ta.act_out = act; ta.act_in = act; ta.y_out = y_pairs;
-    if ((st = set_smem(reinterpret_cast<const void*>(k_expert_tc), TC_SMEM))) return st;
-    k_expert_tc<<<dim3(I / 64, maxA), TC_THREADS, TC_SMEM, s>>>(ta);
-    if ((st = launch_check("k_expert_tc(gate/up)"))) return st;
-  }
-
-  if (mma) {
-    const long nw = static_cast<long>(T) * k * (I / 8);
-    k_pair_rows<<<static_cast<int>((nw + 255) / 256 < 1024 ? (nw + 255) / 256 : 1024), 256, 0, s>>>(
-        reinterpret_cast<const uint16_t*>(act), 0, T * k, I, aP, aS);
-    if ((st = launch_check("k_pair_rows(act)"))) return st;
-    gm.mode = 1; gm.P = aP; gm.S = aS; gm.queue = queues + 1;
-    k_group_mma<<<grouped_grid(), GM_THREADS, grouped_mma_smem(H, I), s>>>(gm);
-    if ((st = launch_check("k_group_mma(down)"))) return st;
-  }
-  DownArgs d{};
-  d.act = act; d.T = T; d.H = H; d.I = I; d.E = E; d.k = k;
-  d.blob_ptrs = blob_ptrs; d.offsets = offsets; d.pairs = pairs; d.active = active; d.n_active = n_active;
-  d.max_rows = gemv_rows;
-  blob_offsets(H, I, d.off);
-  d.y = y_pairs;
-  sm = gemv_smem(I);
-  if ((st = set_smem(reinterpret_cast<const void*>(k_down_gemv), sm))) return st;
-  k_down_gemv<<<dim3((H + GEMV_ROWS - 1) / GEMV_ROWS, maxA), 256, sm, gs>>>(d);
-  if ((st = launch_check("k_down_gemv"))) return st;
-  if (tc) {
-    ta.mode = 1;
-    k_expert_tc<<<dim3(H / 128, maxA), TC_THREADS, TC_SMEM, s>>>(ta);
-    if ((st = launch_check("k_expert_tc(down)"))) return st;
-  }
-  if (side && (st = stream_after(s, gs, side->ev[3]))) return st;     // join
-  return MOE_OK;
+  RoutedIn rt{blob_ptrs, offsets, pairs, active, n_active, y_pairs, I, E, k};
+  return run_gemm(x, T, H, &rt, nullptr, w.plan, w.maps, w.act, w.xs, nullptr, nullptr, s);
 }
 
 size_t moe_shared_workspace_size(int T, int H, int Is) {
-  // fp16 activation [T, Is]; for the tensor-core path also fp16 x [T, H] and
-  // the one-expert bucket list (offsets[2], active[1], n_active, pairs[T])
-  return align_up(static_cast<size_t>(T) * Is * sizeof(__half)) + align_up(static_cast<size_t>(T) * H * sizeof(__half)) +
-         3 * align_up(16) + align_up(static_cast<size_t>(T) * 4);
+  if (T < 0 || H <= 0 || Is <= 0) return 0;
+  return shared_ws_bytes(T, H, Is);
 }
 
 int moe_shared_forward(const uint16_t* x, int T, int H, int Is, const moe_qmat* sh, float* ysh, void* ws,
-                       size_t ws_bytes, void* stream) {
+                       size_t ws_bytes, int flags, void* stream) {
   int st = check_dims(T, H, Is, 8, 1);
   if (st) return st;
+  if ((st = check_flags(flags))) return st;
   if (T == 0) return MOE_OK;
   if (!x || !sh || !ysh || !ws) return fail(MOE_ERR_INVALID_ARG, "moe_shared_forward: NULL pointer");
-  for (int m = 0; m < 3; ++m) {
-    const int out = m < 2 ? Is : H, in = m < 2 ? H : Is;
-    if (!sh[m].q || !sh[m].s || !sh[m].b || sh[m].bits != 4 || sh[m].out != out || sh[m].in != in)
-      return fail(MOE_ERR_INVALID_ARG, "moe_shared_forward: matrix %d must be 4-bit [%d, %d]", m, out, in);
-    if (!aligned16(sh[m].q)) return fail(MOE_ERR_INVALID_ARG, "moe_shared_forward: misaligned weights");
-  }
+  if ((st = check_shared_mats(sh, H, Is))) return st;
   if (ws_bytes < moe_shared_workspace_size(T, H, Is))
     return fail(MOE_ERR_INVALID_ARG, "moe_shared_forward: workspace too small");
+  if (!aligned16(x) || !aligned16(ws) || !aligned16(ysh))
+    return fail(MOE_ERR_INVALID_ARG, "moe_shared_forward: misaligned pointer");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  __half* act = static_cast<__half*>(ws);
-  // several rows: the three matrices on the tensor cores as one expert whose
-  // bucket is every row (same kernel and arithmetic as the routed buckets)
-  if (T > g_gemv_max_rows && H % 128 == 0 && H <= 4096 && Is <= 4096) {
-    char* p = static_cast<char*>(ws) + align_up(static_cast<size_t>(T) * Is * sizeof(__half));
-    __half* xh = reinterpret_cast<__half*>(p);
-    p += align_up(static_cast<size_t>(T) * H * sizeof(__half));
-    int32_t* offsets = reinterpret_cast<int32_t*>(p); p += align_up(16);
-    int32_t* active = reinterpret_cast<int32_t*>(p); p += align_up(16);
-    int32_t* n_active = reinterpret_cast<int32_t*>(p); p += align_up(16);
-    int32_t* pairs = reinterpret_cast<int32_t*>(p);
-    k_one_bucket<<<(T + 255) / 256 < 64 ? (T + 255) / 256 : 64, 256, 0, s>>>(T, offsets, pairs, active, n_active);
-    if ((st = launch_check("k_one_bucket"))) return st;
-    const size_t n8 = static_cast<size_t>(T) * H / 8;
-    k_to_f16<<<static_cast<int>((n8 + 255) / 256 < 1024 ? (n8 + 255) / 256 : 1024), 256, 0, s>>>(x, n8, xh);
-    if ((st = launch_check("k_to_f16(shared)"))) return st;
-    TcArgs ta{};
-    ta.mode = 0; ta.xh = xh; ta.T = T; ta.H = H; ta.I = Is; ta.E = 1; ta.k = 1;
-    ta.blob_ptrs = nullptr;
-    for (int m = 0; m < 3; ++m) {
-      ta.mq[m] = reinterpret_cast<const uint8_t*>(sh[m].q); ta.ms[m] = sh[m].s; ta.mb[m] = sh[m].b;
-    }
-    ta.offsets = offsets; ta.pairs = pairs; ta.active = active; ta.n_active = n_active;
-    ta.max_rows = 0;
-    ta.act_out = act; ta.act_in = act; ta.y_out = ysh;
-    if ((st = set_smem(reinterpret_cast<const void*>(k_expert_tc), TC_SMEM))) return st;
-    k_expert_tc<<<dim3(Is / 64, 1), TC_THREADS, TC_SMEM, s>>>(ta);
-    if ((st = launch_check("k_expert_tc(shared gate/up)"))) return st;
-    ta.mode = 1;
-    k_expert_tc<<<dim3(H / 128, 1), TC_THREADS, TC_SMEM, s>>>(ta);
-    return launch_check("k_expert_tc(shared down)");
+  SharedWs w = carve_shared(ws, T, H, Is);
+  if (!use_gemm(T, H, 64, Is, 8, 1, flags)) {
+    if (flags & MOE_FLAG_TC) return fail(MOE_ERR_UNSUPPORTED, "moe_shared_forward: shapes outside the grouped GEMM");
+    return run_shared_gemv(x, T, H, Is, sh, ysh, w.act, s);
   }
-  GateUpArgs g{};
-  g.x = x; g.T = T; g.H = H; g.I = Is; g.E = 1; g.k = 1; g.max_rows = 1 << 30;
-  g.gq = sh[0].q; g.gs = sh[0].s; g.gb = sh[0].b;
-  g.uq = sh[1].q; g.us = sh[1].s; g.ub = sh[1].b;
-  g.act = act;
-  size_t sm = gemv_smem(H);
-  if ((st = set_smem(reinterpret_cast<const void*>(k_gateup_gemv), sm))) return st;
-  k_gateup_gemv<<<dim3((Is + GEMV_ROWS - 1) / GEMV_ROWS, 1), 256, sm, s>>>(g);
-  if ((st = launch_check("k_gateup_gemv(shared)"))) return st;
-  DownArgs d{};
-  d.act = act; d.T = T; d.H = H; d.I = Is; d.E = 1; d.k = 1; d.max_rows = 1 << 30;
-  d.dq = sh[2].q; d.ds = sh[2].s; d.db = sh[2].b;
-  d.y = ysh;
-  sm = gemv_smem(Is);
-  if ((st = set_smem(reinterpret_cast<const void*>(k_down_gemv), sm))) return st;
-  k_down_gemv<<<dim3((H + GEMV_ROWS - 1) / GEMV_ROWS, 1), 256, sm, s>>>(d);
-  return launch_check("k_down_gemv(shared)");
+  SharedIn si{sh, ysh, Is};
+  return run_gemm(x, T, H, nullptr, &si, w.plan, nullptr, nullptr, nullptr, w.act, w.xh, s);
 }
 
 int moe_combine(const float* y_pairs, const float* gates, const float* ysh, int T, int H, int k, uint16_t* y,
@@ -425,7 +486,13 @@ int moe_combine(const float* y_pairs, const float* gates, const float* ysh, int 
   return launch_check("k_combine");
 }
 
-size_t moe_layer_workspace_size(int T, int H, int I, int Is, int E, int k) {
+// Workspace of one layer: routing buffers, y_pairs, ysh, then the expert and
+// shared-expert regions (the grouped GEMM's plan is the expert region's).
+struct LayerWs {
+  uint16_t* x; int32_t* idx; float* gates; int32_t* offsets; int32_t* pairs; int32_t* active; int32_t* n_active;
+  float* y_pairs; float* ysh; void* ew; size_t ews; void* sw; size_t sws;
+};
+static size_t layer_ws_bytes(int T, int H, int I, int Is, int E, int k) {
   size_t n = 0;
   n += align_up(static_cast<size_t>(T) * H * 2);        // x
   n += align_up(static_cast<size_t>(T) * k * 4) * 2;    // idx, gates
@@ -435,64 +502,79 @@ size_t moe_layer_workspace_size(int T, int H, int I, int Is, int E, int k) {
   n += align_up(4);                                     // n_active
   n += align_up(static_cast<size_t>(T) * k * H * 4);    // y_pairs
   n += align_up(static_cast<size_t>(T) * H * 4);        // ysh
-  n += moe_expert_workspace_size_mma(T, H, I, k);
-  n += moe_shared_workspace_size(T, H, Is);
+  n += expert_ws_bytes(T, H, I, k);
+  n += shared_ws_bytes(T, H, Is);
   return n;
+}
+static LayerWs carve_layer(void* ws, int T, int H, int I, int Is, int E, int k) {
+  char* p = static_cast<char*>(ws);
+  auto take = [&](size_t n) { char* q = p; p += align_up(n); return q; };
+  LayerWs w;
+  w.x = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(T) * H * 2));
+  w.idx = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * k * 4));
+  w.gates = reinterpret_cast<float*>(take(static_cast<size_t>(T) * k * 4));
+  w.offsets = reinterpret_cast<int32_t*>(take(static_cast<size_t>(E + 1) * 4));
+  w.pairs = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * k * 4));
+  w.active = reinterpret_cast<int32_t*>(take(static_cast<size_t>(E) * 4));
+  w.n_active = reinterpret_cast<int32_t*>(take(4));
+  w.y_pairs = reinterpret_cast<float*>(take(static_cast<size_t>(T) * k * H * 4));
+  w.ysh = reinterpret_cast<float*>(take(static_cast<size_t>(T) * H * 4));
+  w.ews = expert_ws_bytes(T, H, I, k);
+  w.ew = p; p += w.ews;
+  w.sws = shared_ws_bytes(T, H, Is);
+  w.sw = p;
+  return w;
+}
+
+size_t moe_layer_workspace_size(int T, int H, int I, int Is, int E, int k) {
+  if (T < 0 || H <= 0 || I <= 0 || Is <= 0 || E <= 0 || k <= 0) return 0;
+  return layer_ws_bytes(T, H, I, Is, E, k);
 }
 
 int moe_layer_forward(const float* h_in, float* h_out, const uint16_t* x_in, int T, int H, int I, int Is, int E,
                       int k, const moe_qmat* router, const float* bias, int bias_per_row,
                       const void* const* blob_ptrs, const moe_qmat* shared, uint16_t* x_out, uint16_t* y,
-                      int32_t* idx_out, float* gates_out, void* ws, size_t ws_bytes, void* stream) {
+                      int32_t* idx_out, float* gates_out, void* ws, size_t ws_bytes, int flags, void* stream) {
   int st = check_dims(T, H, I, E, k);
   if (st) return st;
+  if ((st = check_dims(T, H, Is, E, k))) return st;
+  if ((st = check_flags(flags))) return st;
   if (T == 0) return MOE_OK;
   if (!x_in && !h_in) return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward: need h_in or x_in");
   if (h_out && !h_in) return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward: h_out needs h_in");
-  if (!ws || ws_bytes < moe_layer_workspace_size(T, H, I, Is, E, k))
-    return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward: workspace too small");
-  char* p = static_cast<char*>(ws);
-  auto take = [&](size_t n) { char* q = p; p += align_up(n); return q; };
-  uint16_t* x = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(T) * H * 2));
-  int32_t* idx = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * k * 4));
-  float* gates = reinterpret_cast<float*>(take(static_cast<size_t>(T) * k * 4));
-  int32_t* offsets = reinterpret_cast<int32_t*>(take(static_cast<size_t>(E + 1) * 4));
-  int32_t* pairs = reinterpret_cast<int32_t*>(take(static_cast<size_t>(T) * k * 4));
-  int32_t* active = reinterpret_cast<int32_t*>(take(static_cast<size_t>(E) * 4));
-  int32_t* n_active = reinterpret_cast<int32_t*>(take(4));
-  float* y_pairs = reinterpret_cast<float*>(take(static_cast<size_t>(T) * k * H * 4));
-  float* ysh = reinterpret_cast<float*>(take(static_cast<size_t>(T) * H * 4));
-  const size_t ews = moe_expert_workspace_size_mma(T, H, I, k);
-  void* ew = take(ews);
-  const size_t sws = moe_shared_workspace_size(T, H, Is);
-  void* sw = take(sws);
+  if (!blob_ptrs || !shared || !router) return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward: NULL pointer");
+  if (!ws || !aligned16(ws) || ws_bytes < moe_layer_workspace_size(T, H, I, Is, E, k))
+    return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward: workspace too small or misaligned");
+  if ((st = check_shared_mats(shared, H, Is))) return st;
+  LayerWs w = carve_layer(ws, T, H, I, Is, E, k);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   const uint16_t* xin = x_in;
   if (!xin) {
-    if ((st = moe_rmsnorm(h_in, T, H, 1e-6f, x, stream))) return st;
-    xin = x;
+    if ((st = moe_rmsnorm(h_in, T, H, 1e-6f, w.x, stream))) return st;
+    xin = w.x;
   }
   if (x_out && (st = cuda_check(cudaMemcpyAsync(x_out, xin, static_cast<size_t>(T) * H * 2,
                                                 cudaMemcpyDeviceToDevice, s), "copy x_out")))
     return st;
-  // the shared expert needs only x: it runs on a side stream alongside the
-  // router, the buckets and the routed experts (several rows only)
-  std::unique_lock<std::recursive_mutex> fork_lock(g_fork_mu, std::defer_lock);
-  SideStreams* side = T > g_gemv_max_rows ? side_streams() : nullptr;
-  cudaStream_t shs = s;
-  if (side) {
-    fork_lock.lock();
-    shs = side->st[0];
-    if ((st = stream_after(shs, s, side->ev[0]))) return st;
+  if ((st = moe_router_topk(xin, T, H, router, bias, bias_per_row, E, k, w.idx, w.gates, nullptr, stream))) return st;
+  if ((st = moe_bucket(w.idx, T, k, E, w.offsets, w.pairs, w.active, w.n_active, stream))) return st;
+  const bool gemm = use_gemm(T, H, I, Is, E, k, flags);
+  if (!gemm && (flags & MOE_FLAG_TC)) return fail(MOE_ERR_UNSUPPORTED, "moe_layer_forward: shapes outside the grouped GEMM");
+  if (gemm) {
+    // routed buckets and the shared expert in one persistent launch per projection
+    if (!aligned16(xin)) return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward: misaligned x_in");
+    ExpertWs ew = carve_expert(w.ew, T, H, I, k);
+    SharedWs sw = carve_shared(w.sw, T, H, Is);
+    RoutedIn rt{blob_ptrs, w.offsets, w.pairs, w.active, w.n_active, w.y_pairs, I, E, k};
+    SharedIn si{shared, w.ysh, Is};
+    if ((st = run_gemm(xin, T, H, &rt, &si, ew.plan, ew.maps, ew.act, ew.xs, sw.act, sw.xh, s))) return st;
+  } else {
+    if ((st = moe_shared_forward(xin, T, H, Is, shared, w.ysh, w.sw, w.sws, flags, stream))) return st;
+    if ((st = moe_expert_forward(xin, T, H, I, E, k, blob_ptrs, w.offsets, w.pairs, w.active, w.n_active, w.y_pairs,
+                                 w.ew, w.ews, flags, stream)))
+      return st;
   }
-  if ((st = moe_shared_forward(xin, T, H, Is, shared, ysh, sw, sws, shs))) return st;
-  if ((st = moe_router_topk(xin, T, H, router, bias, bias_per_row, E, k, idx, gates, nullptr, stream))) return st;
-  if ((st = moe_bucket(idx, T, k, E, offsets, pairs, active, n_active, stream))) return st;
-  if ((st = moe_expert_forward(xin, T, H, I, E, k, blob_ptrs, offsets, pairs, active, n_active, y_pairs, ew, ews,
-                               stream)))
-    return st;
-  if (side && (st = stream_after(s, shs, side->ev[1]))) return st;   // join before the combine
   float* resid = nullptr;
   if (h_out) {
     if (h_out != h_in &&
@@ -501,19 +583,19 @@ int moe_layer_forward(const float* h_in, float* h_out, const uint16_t* x_in, int
       return st;
     resid = h_out;
   }
-  if ((st = moe_combine(y_pairs, gates, ysh, T, H, k, y, resid, stream))) return st;
-  if (idx_out && (st = cuda_check(cudaMemcpyAsync(idx_out, idx, static_cast<size_t>(T) * k * 4,
+  if ((st = moe_combine(w.y_pairs, w.gates, w.ysh, T, H, k, y, resid, stream))) return st;
+  if (idx_out && (st = cuda_check(cudaMemcpyAsync(idx_out, w.idx, static_cast<size_t>(T) * k * 4,
                                                   cudaMemcpyDeviceToDevice, s), "copy idx")))
     return st;
-  if (gates_out && (st = cuda_check(cudaMemcpyAsync(gates_out, gates, static_cast<size_t>(T) * k * 4,
+  if (gates_out && (st = cuda_check(cudaMemcpyAsync(gates_out, w.gates, static_cast<size_t>(T) * k * 4,
                                                     cudaMemcpyDeviceToDevice, s), "copy gates")))
     return st;
   return MOE_OK;
 }
 
 // Shapes the fused batch-1 kernel serves.
-static bool fused_ok(int T, int H, int I, int Is, int E, int k, int bias_per_row, int G) {
-  if (!g_decode_fused || T != 1 || bias_per_row) return false;
+static bool fused_ok(int T, int H, int I, int Is, int E, int k, int bias_per_row, int G, int flags) {
+  if ((flags & MOE_FLAG_LAYERED) || T != 1 || bias_per_row) return false;
   return df_fits(H, I, Is, E, k, G);
 }
 
@@ -566,8 +648,6 @@ static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, con
     args.y_trace = y_trace ? y_trace + l0 * TH : nullptr;
     args.idx_trace = idx_trace ? idx_trace + l0 * Tk : nullptr;
     args.gates_trace = gates_trace ? gates_trace + l0 * Tk : nullptr;
-    args.spec = g_decode_spec;
-    args.prefetch = g_decode_prefetch;
     args.stamps = g_decode_stamps ? g_decode_stamps + static_cast<size_t>(l0) * G * 16 : nullptr;
     for (int l = 0; l < nl; ++l) {
       const moe_qmat& R = routers[l0 + l];
@@ -603,29 +683,19 @@ int moe_set_decode_profile(unsigned long long* stamps) {
 
 int moe_decode_grid(void) { return fused_grid(); }
 
-int moe_set_decode_prefetch(int flags) {
-  if (flags < 0 || flags > 3) return fail(MOE_ERR_INVALID_ARG, "prefetch flags must be in [0, 3]");
-  g_decode_prefetch = flags;
-  return MOE_OK;
-}
-
-int moe_set_decode_fused(int enable, int spec_experts) {
-  if (spec_experts < 0 || spec_experts > 8) return fail(MOE_ERR_INVALID_ARG, "spec_experts must be in [0, 8]");
-  g_decode_fused = enable ? 1 : 0;
-  g_decode_spec = spec_experts;
-  return MOE_OK;
-}
-
-int moe_decode_launches(int T, int L) {
+int moe_decode_launches(int T, int L, int flags) {
   if (T <= 0 || L <= 0) return 0;
-  // fused batch-1 path: one kernel per DF_MAX_LAYERS layers; otherwise rmsnorm,
-  // router, bucket, shared gate/up, shared down, expert gate/up, expert down and
-  // combine per layer (plus the tensor-core kernels for multi-row buckets)
-  if (T == 1 && g_decode_fused) return (L + DF_MAX_LAYERS - 1) / DF_MAX_LAYERS;
-  return 8 * L;
+  // persistent batch-1 path: one kernel per DF_MAX_LAYERS layers.  Otherwise
+  // per layer: rmsnorm, router, bucket, then either the grouped GEMM (prep,
+  // gate/up, down) or the GEMV kernels (shared gate/up and down, routed
+  // gate/up and down), and the combine.
+  if (T == 1 && !(flags & MOE_FLAG_LAYERED)) return (L + DF_MAX_LAYERS - 1) / DF_MAX_LAYERS;
+  const bool gemm = !(flags & MOE_FLAG_GEMV) && (T > 2 || (flags & MOE_FLAG_TC));
+  return (gemm ? 7 : 8) * L;
 }
 
 size_t moe_decode_workspace_size(int T, int H, int I, int Is, int E, int k) {
+  if (T < 0 || H <= 0 || I <= 0 || Is <= 0 || E <= 0 || k <= 0) return 0;
   const size_t layered = moe_layer_workspace_size(T, H, I, Is, E, k);
   const size_t fused = fused_ws(I, Is, E, k);
   return layered > fused ? layered : fused;
@@ -634,16 +704,17 @@ size_t moe_decode_workspace_size(int T, int H, int I, int Is, int E, int k) {
 int moe_decode_forward(float* h, int T, int H, int I, int Is, int E, int k, int L, const moe_qmat* routers,
                        const float* const* biases, int bias_per_row, const void* const* const* blob_tables,
                        const moe_qmat* shared, uint16_t* x_trace, uint16_t* y_trace, int32_t* idx_trace,
-                       float* gates_trace, void* ws, size_t ws_bytes, void* stream) {
+                       float* gates_trace, void* ws, size_t ws_bytes, int flags, void* stream) {
   int st = check_dims(T, H, I, E, k);
   if (st) return st;
+  if ((st = check_flags(flags))) return st;
   if (L < 0) return fail(MOE_ERR_INVALID_ARG, "moe_decode_forward: L < 0");
   if (T == 0 || L == 0) return MOE_OK;
   if (!h || !routers || !blob_tables || !shared) return fail(MOE_ERR_INVALID_ARG, "moe_decode_forward: NULL pointer");
   if (ws_bytes < moe_decode_workspace_size(T, H, I, Is, E, k))
     return fail(MOE_ERR_INVALID_ARG, "moe_decode_forward: workspace too small");
-  const int G = (T == 1 && g_decode_fused) ? fused_grid() : 0;
-  if (fused_ok(T, H, I, Is, E, k, bias_per_row, G))
+  const int G = (T == 1 && !(flags & MOE_FLAG_LAYERED)) ? fused_grid() : 0;
+  if (fused_ok(T, H, I, Is, E, k, bias_per_row, G, flags))
     return launch_fused(h, H, I, Is, E, k, L, routers, biases, blob_tables, shared, x_trace, y_trace, idx_trace,
                         gates_trace, ws, G, static_cast<cudaStream_t>(stream));
   const size_t TH = static_cast<size_t>(T) * H, Tk = static_cast<size_t>(T) * k;
@@ -652,7 +723,7 @@ int moe_decode_forward(float* h, int T, int H, int I, int Is, int E, int k, int 
     st = moe_layer_forward(h, h, nullptr, T, H, I, Is, E, k, &routers[l], b, bias_per_row, blob_tables[l],
                            &shared[3 * l], x_trace ? x_trace + l * TH : nullptr, y_trace ? y_trace + l * TH : nullptr,
                            idx_trace ? idx_trace + l * Tk : nullptr, gates_trace ? gates_trace + l * Tk : nullptr, ws,
-                           ws_bytes, stream);
+                           ws_bytes, flags, stream);
     if (st) return st;
   }
   return MOE_OK;

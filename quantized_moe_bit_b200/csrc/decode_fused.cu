@@ -6,18 +6,18 @@
 // [c*k*I/G, ...) of the flattened (slot, row) list, and the output rows
 // [c*H/G, ...) with their k routed down rows and their shared down row.
 //
-// Dot products run on the tensor cores (mma.sync m16n8k16, fp16 operands,
-// fp32 accumulate) straight from registers.  A warp takes a tile of 16 weight
-// rows; per quantisation group (64 inputs) each lane loads two 32-bit words
-// of each of its two rows and turns every word into four half2 with LOP3:
-// (w & 0x000F000F) | 0x64006400 = (1024 + q0, 1024 + q4), the 0x00F000F0 mask
-// gives (1024 + 16 q1, 1024 + 16 q5), the same on w >> 8 nibbles 2, 6 and
-// 3, 7.  The activation comes pre-paired to match -- (v0, v4), (v1/16,
-// v5/16), (v2, v6), (v3/16, v7/16) per word -- so 4 mma give the group's
-// sum of (1024 + s q) v / s = sum q v + 1024 sum v' exactly, and the fp32
-// epilogue adds S (dot - 1024 sum v') + B sum v per row and group.  Gate/up
-// tiles give all 8 mma columns the same x; down tiles give column j the
-// activation of slot j, so one tile mixes rows of all k routed experts.
+// Dot products run on the tensor cores as exact integer mma.sync m16n8k32
+// (u8 x s8 -> s32) straight from registers.  A warp takes a tile of 16
+// weight rows; per quantisation group (64 inputs) each lane loads two 32-bit
+// words of each of its two rows; one mask gives the four low nibbles of a
+// word as u8 bytes, a shift and the mask the four high nibbles.  The
+// activation of every group is 16-bit fixed point (step = max |v| / 32639,
+// split into a high and a low int8 digit), laid out to match, so four mmas
+// give the group's exact integer dot d = 256 (q . high) + (q . low) and the
+// fp32 epilogue adds S step d + B sum v per row and group.  Gate/up tiles
+// give all 8 mma columns the same x (rotated by group so that rows 1,408 B
+// apart read distinct banks); down tiles give column j the activation of
+// slot j, so one tile mixes rows of all k routed experts.
 //
 // Per layer:
 //   A  rms norm of h (every CTA, same result) -> x and its fragments; router
@@ -84,8 +84,6 @@ struct DfArgs {
   unsigned long long* logits;       // workspace: [E]
   unsigned* counter;                // workspace: grid barrier counter; word 32: abort flag (zeroed before launch)
   uint16_t* x_trace; uint16_t* y_trace; int32_t* idx_trace; float* gates_trace;
-  int spec;                         // experts speculatively prefetched into L2 per layer
-  int prefetch;                     // bit 1: routing-independent rows of the next layer into L2
   unsigned long long* stamps;       // optional phase timestamps [L][G][16] (ns), or null
   DfLayer layer[DF_MAX_LAYERS];
 };
@@ -478,19 +476,6 @@ __device__ __forceinline__ void df_bulk_tx(uint32_t bar, uint32_t dst, const voi
   asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
   df_bulk(bar, dst, src, bytes);
 }
-// L2 prefetch of the 16-byte-aligned window around [p, p + bytes).  Arrays
-// handed to this kernel are 16-byte aligned with sizes that are multiples of
-// 16, so the window stays inside them.
-__device__ __forceinline__ void prefetch_l2(const void* p, size_t bytes) {
-  if (bytes == 0) return;
-  uintptr_t a = reinterpret_cast<uintptr_t>(p) & ~uintptr_t(15);
-  const uintptr_t e = (reinterpret_cast<uintptr_t>(p) + bytes + 15) & ~uintptr_t(15);
-  while (a < e) {
-    const uint32_t n = static_cast<uint32_t>((e - a) < 65536 ? (e - a) : 65536);
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(n) : "memory");
-    a += n;
-  }
-}
 __device__ __forceinline__ uint4 ldcg_v4(const void* p) {
   uint4 r;
   asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
@@ -507,32 +492,6 @@ __device__ __forceinline__ void df_stamp(const DfArgs& a, int l, int p) {
 }
 
 // ------------------------------------------------------------ tensor-core dot
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ uint32_t nib_lo(uint32_t w) { return (w & 0x000F000Fu) | 0x64006400u; }
-__device__ __forceinline__ uint32_t nib_hi(uint32_t w) { return (w & 0x00F000F0u) | 0x64006400u; }
-
-// One group (64 inputs) of tile rows g (words wa) and g+8 (words wb): lane
-// (g, t) holds words 2t, 2t+1 of the group; f0, f1 are the paired activation
-// of those words in this lane's column.  Fragment rows: a0/a2 row g, a1/a3
-// row g+8; a0/a1 pair with b0, a2/a3 with b1.
-__device__ __forceinline__ void mma_group(float (&d)[4], uint2 wa, uint2 wb, uint4 f0, uint4 f1) {
-  float e[4] = {0.f, 0.f, 0.f, 0.f};        // second, independent accumulator chain
-  d[0] = d[1] = d[2] = d[3] = 0.f;
-  const uint32_t ax = wa.x >> 8, bx = wb.x >> 8, ay = wa.y >> 8, by = wb.y >> 8;
-  mma16816(d, nib_lo(wa.x), nib_lo(wb.x), nib_hi(wa.x), nib_hi(wb.x), f0.x, f0.y);
-  mma16816(e, nib_lo(wa.y), nib_lo(wb.y), nib_hi(wa.y), nib_hi(wb.y), f1.x, f1.y);
-  mma16816(d, nib_lo(ax), nib_lo(bx), nib_hi(ax), nib_hi(bx), f0.z, f0.w);
-  mma16816(e, nib_lo(ay), nib_lo(by), nib_hi(ay), nib_hi(by), f1.z, f1.w);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) d[i] += e[i];
-}
-
 // m16n8k32 integer mma: A u8 (4-bit codes), B s8 (one activation digit),
 // s32 accumulators.
 __device__ __forceinline__ void imma16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -1061,44 +1020,6 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
     df_stamp(a, l, 8);
 
     // ------------------------------------------------------------- phase C
-    if (l + 1 < a.L && threadIdx.x == 0 && (a.prefetch & 2)) {
-      const DfLayer& V = a.layer[l + 1];
-      for (int m = 0; m < 2; ++m) {
-        prefetch_l2(reinterpret_cast<const uint8_t*>(V.sq[m]) + static_cast<size_t>(g.s0) * (H / 2),
-                    static_cast<size_t>(g.nsp) * (H / 2));
-        prefetch_l2(V.ss[m] + static_cast<size_t>(g.s0) * (H / 64), static_cast<size_t>(g.nsp) * g.sbh);
-        prefetch_l2(V.sb[m] + static_cast<size_t>(g.s0) * (H / 64), static_cast<size_t>(g.nsp) * g.sbh);
-      }
-      prefetch_l2(reinterpret_cast<const uint8_t*>(V.sq[2]) + static_cast<size_t>(g.o0) * (Is / 2),
-                  static_cast<size_t>(g.nrow) * (Is / 2));
-    }
-    if (l + 1 < a.L && warp == 1 && a.spec > 0 && a.layer[l + 1].bias != nullptr) {
-      // slices of the next layer's experts with the largest router bias
-      const DfLayer& V = a.layer[l + 1];
-      unsigned taken = 0;
-      int my_id = -1;
-      for (int r = 0; r < a.spec && r < 8; ++r) {
-        float v = -INFINITY;
-        int id = 0x7fffffff;
-        for (int t = 0, e = lane; e < E; ++t, e += 32) {
-          if (taken & (1u << t)) continue;
-          const float b = V.bias[e];
-          if (b > v || (b == v && e < id)) { v = b; id = e; }
-        }
-        for (int o = 16; o > 0; o >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, v, o);
-          const int oi = __shfl_xor_sync(0xffffffffu, id, o);
-          if (ov > v || (ov == v && oi < id)) { v = ov; id = oi; }
-        }
-        if ((id & 31) == lane) taken |= 1u << (id >> 5);
-        if (lane == r) my_id = id;
-      }
-      if (my_id >= 0 && my_id < E) {
-        const size_t bb = a.off[8] + static_cast<size_t>(H) * (I / 64) * 2;
-        const size_t b0 = bb * c / G, b1 = bb * (c + 1) / G;
-        prefetch_l2(static_cast<const uint8_t*>(V.blobs[my_id]) + b0, b1 - b0);
-      }
-    }
     // the next layer's blob table and router bias (this layer's copies are all issued)
     if (l + 1 < a.L) {
       for (int e = threadIdx.x; e < E; e += DF_THREADS) btab[e] = a.layer[l + 1].blobs[e];

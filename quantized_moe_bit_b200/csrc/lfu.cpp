@@ -46,6 +46,22 @@ struct moe_lfu {
   int fault_kind = 0, fault_after = -1;
   long copies = 0;
   int64_t bytes_copied = 0;
+  // A slot whose bytes do not hold the expert that expert[] names: a call that
+  // failed after issuing copies was rolled back (its plan undone) while the
+  // copies it had issued still overwrite their slots.  The next hit on such a
+  // slot copies the blob again.
+  std::vector<char> dirty;                    // [L*S]
+  // Transaction of one call (moe_lfu_step, or a whole streamed layer call that
+  // makes several steps): the layer's state as it was before the call, and
+  // the slots that copies issued during the call write.  A failure restores
+  // the state, so that repeating the call plans exactly as the first attempt.
+  int txn_depth = 0, txn_layer = -1;
+  std::vector<int32_t> snap_expert, snap_count;
+  std::vector<int64_t> snap_last;
+  int64_t snap_tick = 0;
+  int32_t snap_steps = 0;
+  size_t snap_log = 0;
+  std::vector<int32_t> txn_written;
   // streamed layer forward: per-layer "slots read" events, pinned staging
   std::vector<cudaEvent_t> consumed;          // [L] recorded after the expert kernels of a layer
   cudaEvent_t done = nullptr, idx_ready = nullptr, stage_free = nullptr;
@@ -68,6 +84,42 @@ int victim(moe_lfu* h, int layer, const std::vector<char>& used) {
     if (h->count[a] < h->count[b] || (h->count[a] == h->count[b] && h->last[a] < h->last[b])) best = s;
   }
   return best;
+}
+
+void txn_begin(moe_lfu* h, int layer) {
+  if (h->txn_depth++ > 0) return;
+  const size_t b = static_cast<size_t>(layer) * h->S;
+  h->txn_layer = layer;
+  h->snap_expert.assign(h->expert.begin() + b, h->expert.begin() + b + h->S);
+  h->snap_count.assign(h->count.begin() + b, h->count.begin() + b + h->S);
+  h->snap_last.assign(h->last.begin() + b, h->last.begin() + b + h->S);
+  h->snap_tick = h->tick;
+  h->snap_steps = h->steps[layer];
+  h->snap_log = h->log.size();
+  h->txn_written.clear();
+}
+
+void txn_commit(moe_lfu* h) {
+  if (h->txn_depth > 0) --h->txn_depth;
+}
+
+// Undo the plan of the current transaction (every step of it) and mark the
+// slots its issued copies overwrite.  Returns `status` for the caller to pass on.
+int txn_rollback(moe_lfu* h, int status) {
+  if (h->txn_depth == 0) return status;
+  const int layer = h->txn_layer;
+  const size_t b = static_cast<size_t>(layer) * h->S;
+  std::copy(h->snap_expert.begin(), h->snap_expert.end(), h->expert.begin() + b);
+  std::copy(h->snap_count.begin(), h->snap_count.end(), h->count.begin() + b);
+  std::copy(h->snap_last.begin(), h->snap_last.end(), h->last.begin() + b);
+  h->tick = h->snap_tick;
+  h->steps[layer] = h->snap_steps;
+  h->log.resize(h->snap_log);
+  if (!h->dirty.empty())
+    for (int32_t s : h->txn_written) h->dirty[b + s] = 1;
+  h->txn_written.clear();
+  h->txn_depth = 0;
+  return status;
 }
 
 // Plan one step: slots_out[i] / hit_out[i] for ids[i].  Updates the state and the log.
@@ -152,6 +204,7 @@ MOE_API int moe_lfu_create(int n_layers, int n_experts, int n_slots, size_t blob
   h->count.assign(static_cast<size_t>(n_layers) * n_slots, 0);
   h->last.assign(static_cast<size_t>(n_layers) * n_slots, 0);
   h->steps.assign(n_layers, 0);
+  if (slot_pool) h->dirty.assign(static_cast<size_t>(n_layers) * n_slots, 0);
   if (slot_pool) {
     h->mirror.assign(n_layers, nullptr);
     h->mirror_ev.assign(n_layers, nullptr);
@@ -201,38 +254,50 @@ MOE_API int moe_lfu_step(moe_lfu* h, int layer, const int32_t* ids, int n, void*
   if (!h || !h->pool) return moe::fail(MOE_ERR_INVALID_ARG, "lfu_step: handle has no slot pool");
   if (n > 0 && !ids) return moe::fail(MOE_ERR_INVALID_ARG, "lfu_step: NULL ids");
   if (!dev_table || !done_event) return moe::fail(MOE_ERR_INVALID_ARG, "lfu_step: NULL table or event");
+  if (layer < 0 || layer >= h->L) return moe::fail(MOE_ERR_INVALID_ARG, "lfu_step: layer %d out of range", layer);
+  if (h->txn_depth > 0 && h->txn_layer != layer)
+    return moe::fail(MOE_ERR_INVALID_ARG, "lfu_step: layer %d inside a call on layer %d", layer, h->txn_layer);
   cudaStream_t s = static_cast<cudaStream_t>(side_stream);
   std::vector<int32_t> slots(n), hit(n, 0);
+  txn_begin(h, layer);
   int st = plan(h, layer, ids, n, slots.data(), hit.data());
-  if (st) return st;
+  if (st) return txn_rollback(h, st);
   // slots are overwritten only after the kernels that read them are done
   if (wait_event_ && (st = moe::cuda_check(cudaStreamWaitEvent(s, static_cast<cudaEvent_t>(wait_event_), 0),
                                            "lfu_step: wait")))
-    return st;
+    return txn_rollback(h, st);
+  const size_t base = static_cast<size_t>(layer) * h->S;
   for (int i = 0; i < n; ++i) {
-    unsigned char* slot = h->pool + (static_cast<size_t>(layer) * h->S + slots[i]) * h->slot_stride;
-    if (!hit[i]) {
+    unsigned char* slot = h->pool + (base + slots[i]) * h->slot_stride;
+    // a miss, or a hit on a slot that a rolled-back call overwrote
+    if (!hit[i] || h->dirty[base + slots[i]]) {
       ++h->copies;
       if (h->fault_kind == MOE_LFU_FAULT_COPY_FAILS && h->fault_after >= 0 && h->copies > h->fault_after)
-        return moe::fail(MOE_ERR_CUDA, "lfu_step: injected copy failure (copy %ld)", h->copies);
+        return txn_rollback(h, moe::fail(MOE_ERR_CUDA, "lfu_step: injected copy failure (copy %ld)", h->copies));
       if (h->fault_kind == MOE_LFU_FAULT_SLOW_COPY && h->fault_after >= 0 && h->copies > h->fault_after)
         std::this_thread::sleep_for(std::chrono::milliseconds(50));
       const void* src = h->host_blobs[static_cast<size_t>(layer) * h->E + ids[i]];
       if ((st = moe::cuda_check(cudaMemcpyAsync(slot, src, h->blob_bytes, cudaMemcpyHostToDevice, s),
                                 "lfu_step: copy")))
-        return st;
+        return txn_rollback(h, st);
+      h->txn_written.push_back(slots[i]);
+      h->dirty[base + slots[i]] = 0;
       h->bytes_copied += static_cast<int64_t>(h->blob_bytes);
     }
   }
   // the pinned table mirror may still feed the previous copy of this layer's table
-  if ((st = wait_event(h->mirror_ev[layer], timeout_ms))) return st;
+  if ((st = wait_event(h->mirror_ev[layer], timeout_ms))) return txn_rollback(h, st);
   for (int i = 0; i < n; ++i)
-    h->mirror[layer][ids[i]] = h->pool + (static_cast<size_t>(layer) * h->S + slots[i]) * h->slot_stride;
+    h->mirror[layer][ids[i]] = h->pool + (base + slots[i]) * h->slot_stride;
   if ((st = moe::cuda_check(cudaMemcpyAsync(dev_table, h->mirror[layer], sizeof(void*) * h->E,
                                             cudaMemcpyHostToDevice, s), "lfu_step: table")))
-    return st;
-  if ((st = moe::cuda_check(cudaEventRecord(h->mirror_ev[layer], s), "lfu_step: record"))) return st;
-  return moe::cuda_check(cudaEventRecord(static_cast<cudaEvent_t>(done_event), s), "lfu_step: done event");
+    return txn_rollback(h, st);
+  if ((st = moe::cuda_check(cudaEventRecord(h->mirror_ev[layer], s), "lfu_step: record")))
+    return txn_rollback(h, st);
+  if ((st = moe::cuda_check(cudaEventRecord(static_cast<cudaEvent_t>(done_event), s), "lfu_step: done event")))
+    return txn_rollback(h, st);
+  txn_commit(h);
+  return MOE_OK;
 }
 
 MOE_API int moe_lfu_wait(void* event, int timeout_ms) {
@@ -294,7 +359,7 @@ MOE_API size_t moe_streamed_workspace_size(int T, int H, int I, int Is, int E, i
 MOE_API int moe_streamed_layer_forward(moe_lfu* h, int layer, float* hres, int T, int H, int I, int Is, int E, int k,
                                        const moe_qmat* router, const float* bias, int bias_per_row,
                                        const moe_qmat* shared, void** dev_table, uint16_t* x_out, uint16_t* y_out,
-                                       int32_t* idx_out, void* ws, size_t ws_bytes, void* main_stream,
+                                       int32_t* idx_out, void* ws, size_t ws_bytes, int flags, void* main_stream,
                                        void* side_stream, int timeout_ms) {
   if (!h || !h->pool) return moe::fail(MOE_ERR_INVALID_ARG, "streamed: handle has no slot pool");
   if (!hres || !dev_table || !ws || T < 0 || k < 1 || k > 8 || E != h->E || layer < 0 || layer >= h->L)
@@ -316,7 +381,7 @@ MOE_API int moe_streamed_layer_forward(moe_lfu* h, int layer, float* hres, int T
   int32_t* n_active = reinterpret_cast<int32_t*>(take(4));
   float* y_pairs = reinterpret_cast<float*>(take(static_cast<size_t>(T) * k * H * 4));
   float* ysh = reinterpret_cast<float*>(take(static_cast<size_t>(T) * H * 4));
-  const size_t ews = moe_expert_workspace_size_mma(T, H, I, k);   // the same expert path as moe_layer_forward
+  const size_t ews = moe_expert_workspace_size(T, H, I, k);
   void* ew = take(ews);
   const size_t sws = moe_shared_workspace_size(T, H, Is);
   void* sw = take(sws);
@@ -338,7 +403,7 @@ MOE_API int moe_streamed_layer_forward(moe_lfu* h, int layer, float* hres, int T
                             "streamed: idx to host")))
     return st;
   if ((st = moe::cuda_check(cudaEventRecord(h->idx_ready, ms), "streamed: record"))) return st;
-  if ((st = moe_shared_forward(x, T, H, Is, shared, ysh, sw, sws, ms))) return st;
+  if ((st = moe_shared_forward(x, T, H, Is, shared, ysh, sw, sws, flags, ms))) return st;
   if ((st = wait_event(h->idx_ready, timeout_ms))) return st;
   // steps: one token's ids in selection order, or the chunk's distinct experts,
   // resident ones first (ascending), then the rest (ascending), k at a time
@@ -361,24 +426,35 @@ MOE_API int moe_streamed_layer_forward(moe_lfu* h, int layer, float* hres, int T
   }
   // the pinned active-list staging of the previous call must have been consumed
   if ((st = wait_event(h->stage_free, timeout_ms))) return st;
+  // every step of this call is one transaction: a failure in any of them
+  // undoes the plan of all of them (a repeated call then plans the same way)
+  txn_begin(h, layer);
+  // a failed call still marks its pinned staging (the active lists already
+  // queued for copying) so that the next call waits before reusing it
+  auto abort_call = [&](int status) {
+    cudaEventRecord(h->stage_free, ms);
+    return txn_rollback(h, status);
+  };
   for (size_t g = 0; g < steps.size(); ++g) {
     const auto& ids = steps[g];
     const int n = static_cast<int>(ids.size());
     if ((st = moe_lfu_step(h, layer, ids.data(), n, side_stream, h->consumed[layer], h->done, dev_table, timeout_ms)))
-      return st;
-    if ((st = moe::cuda_check(cudaStreamWaitEvent(ms, h->done, 0), "streamed: wait copies"))) return st;
+      return abort_call(st);
+    if ((st = moe::cuda_check(cudaStreamWaitEvent(ms, h->done, 0), "streamed: wait copies"))) return abort_call(st);
     int32_t* pa = h->pin_act + g * (E + 1);
     pa[0] = n;
     for (int i = 0; i < n; ++i) pa[1 + i] = ids[i];
     int32_t* da = dev_act + g * (E + 1);
     if ((st = moe::cuda_check(cudaMemcpyAsync(da, pa, sizeof(int32_t) * (n + 1), cudaMemcpyHostToDevice, ms),
                               "streamed: active list")))
-      return st;
+      return abort_call(st);
     if ((st = moe_expert_forward(x, T, H, I, E, k, const_cast<const void* const*>(dev_table), offsets, pairs, da + 1,
-                                 da, y_pairs, ew, ews, ms)))
-      return st;
-    if ((st = moe::cuda_check(cudaEventRecord(h->consumed[layer], ms), "streamed: record consumed"))) return st;
+                                 da, y_pairs, ew, ews, flags, ms)))
+      return abort_call(st);
+    if ((st = moe::cuda_check(cudaEventRecord(h->consumed[layer], ms), "streamed: record consumed")))
+      return abort_call(st);
   }
+  txn_commit(h);
   if ((st = moe::cuda_check(cudaEventRecord(h->stage_free, ms), "streamed: record staging"))) return st;
   if ((st = moe_combine(y_pairs, gates, ysh, T, H, k, y_out, hres, ms))) return st;
   if (x_out && (st = moe::cuda_check(cudaMemcpyAsync(x_out, x, static_cast<size_t>(T) * H * 2,

@@ -1,5 +1,6 @@
 // Thin wrappers over the sm_100a PTX used by the tensor-core kernels:
-// mbarriers, proxy fences, TMEM allocation, tcgen05.mma / commit / ld.
+// mbarriers, proxy fences, bulk and tensor (TMA) copies, TMEM allocation,
+// tcgen05.mma / commit / ld.
 #pragma once
 #include "common.cuh"
 
@@ -26,6 +27,52 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
   return t;
+}
+
+// The single arrival of a phase that also announces the bytes its copies bring.
+__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
+               "r"(bytes)
+               : "memory");
+}
+
+// One 1-D bulk copy global -> shared completing `bytes` of transaction count
+// on mbarrier `bar` (addresses 16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// One 2-D tiled tensor copy (TMA) global -> shared of the box at element
+// coordinates (x, y) of the tensor map (a kernel parameter), completing on `bar`.
+// No cluster multicast.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// Tensor maps patched on the device (a grouped GEMM whose operands' addresses
+// are known only on the device): the global address field of a 128-byte map
+// staged in shared memory is replaced, the map is copied to global memory
+// with a release fence between the generic and the tensor-map proxies, and
+// the thread that will use it acquires it before its first copy.
+__device__ __forceinline__ void tmap_replace_addr(uint32_t smem_map, const void* addr) {
+  asm volatile("tensormap.replace.tile.global_address.shared::cta.b1024.b64 [%0], %1;" ::"r"(smem_map), "l"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void tmap_publish(void* gmem_map, uint32_t smem_map) {   // whole warp
+  asm volatile(
+      "tensormap.cp_fenceproxy.global.shared::cta.tensormap::generic.release.gpu.sync.aligned [%0], [%1], 128;" ::"l"(
+          gmem_map),
+      "r"(smem_map)
+      : "memory");
+}
+__device__ __forceinline__ void tmap_acquire(const void* gmem_map) {
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(gmem_map) : "memory");
 }
 
 // Wait for the phase with the given parity to complete.  Gives up after about

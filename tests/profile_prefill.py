@@ -1,10 +1,11 @@
-"""One 128-row prefill chunk through one layer, for profiling the grouped
-expert GEMM on the tensor cores.
+"""Prefill chunks through one layer, for profiling the grouped expert GEMM
+on the tensor cores.
 
-    python -m tests.profile_prefill --reps 3
+    python -m tests.profile_prefill --reps 3 [--rows 128]
 
 Uploads layer 0 of the prefill workload and runs the layer call `reps` times
-(not a test; collected by no test runner)."""
+on `rows` rows of the prefill workload's input stream (not a test; collected
+by no test runner)."""
 import argparse
 import os
 import sys
@@ -19,8 +20,10 @@ def main():
     from tests._support import HostLayer
     ap = argparse.ArgumentParser()
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--rows", type=int, default=128)
     args = ap.parse_args()
-    cfg = gen.CONFIGS["prefill_1L_128tok"]
+    from dataclasses import replace
+    cfg = replace(gen.CONFIGS["prefill_1L_128tok"], T=args.rows)
     dl = HostLayer(cfg, 0).upload()
     T, H = cfg.T, cfg.H
     z = torch.from_numpy(gen.rows(cfg.seed, cfg.row_stream, T, H)).cuda()

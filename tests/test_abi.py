@@ -46,7 +46,6 @@ def test_host_argument_checks():
     assert L.moe_rmsnorm(None, 1, 100, 1e-6, None, None) == 1       # H % 64
     assert b"H" in L.moe_last_error_string()
     assert L.moe_bucket(None, 1, 9, 128, None, None, None, None, None) == 1   # k > 8
-    assert L.moe_set_gemv_max_rows(-1) == 1
     assert L.moe_blob_bytes(100, 64, None) == 0
 
 
@@ -91,22 +90,26 @@ def test_expert_shared_combine_argument_checks():
     T, H, I, Is, E, k = 4, 2816, 704, 2112, 128, 8
     ews = L.moe_expert_workspace_size(T, H, I, k)
     assert ews > 0 and L.moe_expert_workspace_size(T + 1, H, I, k) >= ews
-    assert L.moe_expert_workspace_size_mma(T, H, I, k) >= ews
     args = [f, T, H, I, E, k, f, f, f, f, f, f, f]
-    assert L.moe_expert_forward(*args, ews - 1, None) == _INVALID                       # workspace
+    assert L.moe_expert_forward(*args, ews - 1, 0, None) == _INVALID                    # workspace
     assert b"workspace" in L.moe_last_error_string()
-    assert L.moe_expert_forward(f + 2, *args[1:], ews, None) == _INVALID                # alignment
-    assert L.moe_expert_forward(*args[:6], None, *args[7:], ews, None) == _INVALID       # NULL blobs
-    assert L.moe_expert_forward(f, T, H, 700, E, k, *args[6:], ews, None) == _INVALID   # I % 64
-    assert L.moe_expert_forward(f, 0, H, I, E, k, *args[6:], 0, None) == _OK            # T = 0
+    assert L.moe_expert_forward(f + 2, *args[1:], ews, 0, None) == _INVALID             # alignment
+    assert L.moe_expert_forward(*args[:6], None, *args[7:], ews, 0, None) == _INVALID    # NULL blobs
+    assert L.moe_expert_forward(f, T, H, 700, E, k, *args[6:], ews, 0, None) == _INVALID  # I % 64
+    assert L.moe_expert_forward(*args, ews, 8, None) == _INVALID                        # unknown flag bit
+    assert L.moe_expert_forward(*args, ews, 3, None) == _INVALID                        # GEMV and TC together
+    assert L.moe_expert_forward(f, 0, H, I, E, k, *args[6:], 0, 0, None) == _OK         # T = 0
     sh = (_lib.moe_qmat * 3)(_q(Is, H, 4), _q(Is, H, 4), _q(H, Is, 4))
     sws = L.moe_shared_workspace_size(T, H, Is)
     assert sws > 0
-    assert L.moe_shared_forward(f, T, H, Is, sh, f, f, sws - 1, None) == _INVALID       # workspace
+    assert L.moe_shared_forward(f, T, H, Is, sh, f, f, sws - 1, 0, None) == _INVALID    # workspace
     bad = (_lib.moe_qmat * 3)(_q(Is, H, 4), _q(Is, H, 8), _q(H, Is, 4))
-    assert L.moe_shared_forward(f, T, H, Is, bad, f, f, sws, None) == _INVALID          # 8-bit up
+    assert L.moe_shared_forward(f, T, H, Is, bad, f, f, sws, 0, None) == _INVALID       # 8-bit up
     shape = (_lib.moe_qmat * 3)(_q(Is, H, 4), _q(Is, H, 4), _q(Is, H, 4))
-    assert L.moe_shared_forward(f, T, H, Is, shape, f, f, sws, None) == _INVALID        # down is [H, Is]
+    assert L.moe_shared_forward(f, T, H, Is, shape, f, f, sws, 0, None) == _INVALID     # down is [H, Is]
+    mis = (_lib.moe_qmat * 3)(_q(Is, H, 4), _q(Is, H, 4), _q(H, Is, 4))
+    mis[1].s = f + 8
+    assert L.moe_shared_forward(f, T, H, Is, mis, f, f, sws, 0, None) == _INVALID       # misaligned scales
     assert L.moe_combine(f, f, f, T, H, 9, f, None, None) == _INVALID                   # k > 8
     assert L.moe_combine(None, f, f, T, H, k, f, None, None) == _INVALID
     assert L.moe_combine(f, f, f, 0, H, k, f, None, None) == _OK
@@ -120,11 +123,12 @@ def test_layer_and_decode_argument_checks():
     r = _q(E, H, 8)
     sh = (_lib.moe_qmat * 3)(_q(Is, H, 4), _q(Is, H, 4), _q(H, Is, 4))
     lws = L.moe_layer_workspace_size(T, H, I, Is, E, k)
-    assert lws >= L.moe_expert_workspace_size_mma(T, H, I, k) + L.moe_shared_workspace_size(T, H, Is)
+    assert lws >= L.moe_expert_workspace_size(T, H, I, k) + L.moe_shared_workspace_size(T, H, Is)
     tail = [T, H, I, Is, E, k, C.byref(r), None, 0, f, sh, None, None, None, None]
-    assert L.moe_layer_forward(None, None, None, *tail, f, lws, None) == _INVALID       # no input
-    assert L.moe_layer_forward(None, f, f, *tail, f, lws, None) == _INVALID             # h_out without h_in
-    assert L.moe_layer_forward(f, f, None, *tail, f, lws - 1, None) == _INVALID         # workspace
+    assert L.moe_layer_forward(None, None, None, *tail, f, lws, 0, None) == _INVALID    # no input
+    assert L.moe_layer_forward(None, f, f, *tail, f, lws, 0, None) == _INVALID          # h_out without h_in
+    assert L.moe_layer_forward(f, f, None, *tail, f, lws - 1, 0, None) == _INVALID      # workspace
+    assert L.moe_layer_forward(f, f, None, *tail, f, lws, 16, None) == _INVALID         # unknown flag bit
     dws = L.moe_decode_workspace_size(1, H, I, Is, E, k)
     assert dws >= L.moe_layer_workspace_size(1, H, I, Is, E, k)
     routers = (_lib.moe_qmat * 2)(r, r)
@@ -132,10 +136,33 @@ def test_layer_and_decode_argument_checks():
     blobs = (C.c_void_p * 2)(f, f)
     d = [1, H, I, Is, E, k]
     assert L.moe_decode_forward(f, *d, -1, routers, None, 0, blobs, shared, None, None, None, None, f, dws,
-                                None) == _INVALID                                        # L < 0
+                                0, None) == _INVALID                                     # L < 0
     assert L.moe_decode_forward(f, *d, 2, routers, None, 0, blobs, shared, None, None, None, None, f, dws - 1,
-                                None) == _INVALID                                        # workspace
+                                0, None) == _INVALID                                     # workspace
     assert L.moe_decode_forward(None, *d, 2, routers, None, 0, blobs, shared, None, None, None, None, f, dws,
-                                None) == _INVALID                                        # NULL h
+                                0, None) == _INVALID                                     # NULL h
     assert L.moe_decode_forward(f, *d, 0, routers, None, 0, blobs, shared, None, None, None, None, f, dws,
-                                None) == _OK                                             # L = 0
+                                0, None) == _OK                                          # L = 0
+    assert L.moe_decode_launches(1, 30, 0) == 1 and L.moe_decode_launches(1, 30, 4) == 240
+    assert L.moe_decode_launches(64, 30, 0) == 210 and L.moe_decode_launches(64, 30, 1) == 240
+
+
+def test_noalloc_argument_checks_come_before_any_cuda_call():
+    """Every rejected request of the no-allocation entry point is rejected by
+    its own checks (MOE_ERR_INVALID_ARG), before the scratch lookup or any
+    other CUDA call (which, without a GPU, would answer MOE_ERR_CUDA)."""
+    from quantized_moe_bit_b200 import _lib
+    L = _lib.lib()
+    f = _FAKE
+    H, I, E, k = 2816, 704, 128, 8
+    limit = 4 * 1024 * 1024
+    T_max = max(T for T in range(1, 400) if L.moe_expert_workspace_size(T, H, I, k) <= limit)
+    rest = [f, f, f, f, f, f]
+    assert L.moe_expert_forward_noalloc(f, T_max + 1, H, I, E, k, *rest, None) == _INVALID   # beyond the scratch
+    assert b"static scratch" in L.moe_last_error_string()
+    assert L.moe_expert_forward_noalloc(None, T_max, H, I, E, k, *rest, None) == _INVALID    # NULL x
+    assert L.moe_expert_forward_noalloc(f, 4, H, I, E, k, None, *rest[1:], None) == _INVALID  # NULL blob table
+    assert L.moe_expert_forward_noalloc(f, 4, H, I, E, k, *rest[:5], None, None) == _INVALID  # NULL y_pairs
+    assert L.moe_expert_forward_noalloc(f + 4, 4, H, I, E, k, *rest, None) == _INVALID        # misaligned x
+    assert L.moe_expert_forward_noalloc(f, 4, H, 100, E, k, *rest, None) == _INVALID          # I % 64
+    assert L.moe_expert_forward_noalloc(f, 0, H, I, E, k, *rest, None) == _OK                 # T = 0

@@ -9,6 +9,8 @@ import pytest
 import torch
 
 import gen
+from dataclasses import replace
+
 from gen import tiny_config, CONFIGS
 from oracle import moe_oracle as O
 from tests._support import HostLayer, check_close, check_output, check_routing, gap_ok_predicate
@@ -30,10 +32,9 @@ def _bits(t):
     return _np(t.view(torch.int16)).view(np.uint16)
 
 
-def _run_calls(M, hl, dl, z, stream_check=True, mma=False):
-    """Run A0..A7 through the separate calls; return every intermediate.
-    mma: give moe_expert_forward the larger workspace that enables the
-    grouped mma.sync kernel for buckets of 3..32 rows."""
+def _run_calls(M, hl, dl, z, flags=0):
+    """Run A0..A7 through the separate calls (expert path per `flags`);
+    return every intermediate."""
     c = hl.cfg
     T = z.shape[0]
     dev = "cuda"
@@ -50,12 +51,11 @@ def _run_calls(M, hl, dl, z, stream_check=True, mma=False):
     n_active = torch.empty(1, dtype=torch.int32, device=dev)
     M.moe_bucket(idx, c.E, offs, pairs, active, n_active)
     yp = torch.empty((T * c.k, c.H), dtype=torch.float32, device=dev)
-    wsz = (M.moe_expert_workspace_size_mma if mma else M.moe_expert_workspace_size)(T, c.H, c.I, c.k)
-    ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
-    M.moe_expert_forward(x, c.I, c.E, c.k, dl.blob_ptrs, offs, pairs, active, n_active, yp, ws)
+    ws = torch.empty(M.moe_expert_workspace_size(T, c.H, c.I, c.k), dtype=torch.uint8, device=dev)
+    M.moe_expert_forward(x, c.I, c.E, c.k, dl.blob_ptrs, offs, pairs, active, n_active, yp, ws, flags=flags)
     ysh = torch.empty((T, c.H), dtype=torch.float32, device=dev)
     wss = torch.empty(M.moe_shared_workspace_size(T, c.H, c.Is), dtype=torch.uint8, device=dev)
-    M.moe_shared_forward(x, c.Is, dl.shared_c, ysh, wss)
+    M.moe_shared_forward(x, c.Is, dl.shared_c, ysh, wss, flags=flags)
     y = torch.empty((T, c.H), dtype=torch.int16, device=dev)
     resid = h.clone()
     M.moe_combine(yp, gates, ysh, y, resid)
@@ -106,12 +106,16 @@ def test_calls_single_layer_full(M):
     _check_all(hl, z, g)
 
 
-def test_layer_forward_matches_calls_and_is_deterministic(M):
-    cfg = tiny_config("prefill_1L_128tok", T=19)
+@pytest.mark.parametrize("T", [2, 19, 150])
+def test_layer_forward_matches_calls_and_is_deterministic(M, T):
+    """The whole-layer call (routed buckets and shared expert in one grouped
+    launch per projection when T > 2) equals the separate calls bit for bit,
+    and repeats bit for bit."""
+    cfg = tiny_config("prefill_1L_128tok", T=T)
     hl = HostLayer(cfg, 0)
     dl = hl.upload()
     z = gen.rows(cfg.seed, 1000, cfg.T, cfg.H)
-    g = _run_calls(M, hl, dl, z, mma=True)      # the layer call's workspace enables the grouped kernel too
+    g = _run_calls(M, hl, dl, z)
     c = cfg
     outs = []
     for _ in range(2):
@@ -147,69 +151,57 @@ def test_empty_and_invalid(M):
     M.moe_sync()
 
 
-@pytest.fixture
-def gemv_rows(M):
-    def set_(n):
-        M.moe_set_gemv_max_rows(n)
-    yield set_
-    M.moe_set_gemv_max_rows(2)
-
-
-@pytest.mark.parametrize("max_rows", [0, 2, 1 << 30])
-@pytest.mark.parametrize("T", [37, 130])
-def test_expert_paths_tiny(M, gemv_rows, T, max_rows):
-    """Tensor-core path (buckets > max_rows) and GEMV path against the oracle;
-    T = 130 gives buckets above 128 rows (two N tiles on the tensor cores)."""
-    gemv_rows(max_rows)
+@pytest.mark.parametrize("flags", [0, 1, 2])
+@pytest.mark.parametrize("T", [1, 3, 37, 130])
+def test_expert_paths_tiny(M, T, flags):
+    """GEMV (flag 1), grouped tensor-core GEMM (flag 2) and the library's
+    choice (0) against the oracle.  T = 1 on the GEMM pads one-row buckets to
+    16 MMA columns; T = 130 gives buckets above 128 rows (several chunks)."""
     cfg = tiny_config("prefill_1L_128tok", T=T)
     hl = HostLayer(cfg, 0)
     z = gen.rows(cfg.seed, 1000, T, cfg.H, accept=gap_ok_predicate(hl))
-    g = _run_calls(M, hl, hl.upload(), z)
+    g = _run_calls(M, hl, hl.upload(), z, flags=flags)
     _check_all(hl, z, g)
 
 
-@pytest.mark.parametrize("max_rows", [2, 1 << 30])
-def test_prefill_128_full(M, gemv_rows, max_rows):
-    """The 128-row prefill chunk at full size (H=2816, E=128, I=704)."""
-    gemv_rows(max_rows)
+@pytest.mark.parametrize("flags", [0, 1])
+def test_prefill_128_full(M, flags):
+    """The 128-row prefill chunk at full size (H=2816, E=128, I=704) on the
+    grouped GEMM (0) and on the GEMV kernels (1)."""
     cfg = CONFIGS["prefill_1L_128tok"]
     hl = HostLayer(cfg, 0)
     z = gen.rows(cfg.seed, 1000, cfg.T, cfg.H, accept=gap_ok_predicate(hl))
-    g = _run_calls(M, hl, hl.upload(), z)
+    g = _run_calls(M, hl, hl.upload(), z, flags=flags)
     _check_all(hl, z, g)
 
 
-@pytest.fixture
-def grouped(M):
-    M.moe_set_grouped_mma(True)
-    yield
-    M.moe_set_grouped_mma(False)
-
-
-@pytest.mark.parametrize("T", [9, 37, 130])
-def test_grouped_mma_tiny(M, grouped, T):
-    """Buckets of 3..32 rows on the grouped mma.sync kernel (T = 130 also
-    sends buckets above 32 rows to the tensor-core GEMM)."""
-    cfg = tiny_config("prefill_1L_128tok", T=T)
-    hl = HostLayer(cfg, 0)
-    z = gen.rows(cfg.seed, 1000, T, cfg.H, accept=gap_ok_predicate(hl))
-    g = _run_calls(M, hl, hl.upload(), z, mma=True)
-    _check_all(hl, z, g)
-
-
-def test_grouped_mma_prefill_128_full(M):
-    """The 128-row prefill chunk at full size with the grouped kernel (most
-    of its ~88 buckets have 3..32 rows), and the same chunk without it."""
-    cfg = CONFIGS["prefill_1L_128tok"]
+def test_prefill_large_chunk_full(M):
+    """Large prefill chunk (512 rows of the prefill workload's shapes and
+    routing skew) through the whole-layer call: routing, buckets and every
+    output row against the oracle; the largest buckets span several
+    128-row chunks of the grouped GEMM."""
+    cfg = replace(CONFIGS["prefill_1L_128tok"], T=512)
+    c = cfg
     hl = HostLayer(cfg, 0)
     dl = hl.upload()
-    z = gen.rows(cfg.seed, 1000, cfg.T, cfg.H, accept=gap_ok_predicate(hl))
-    try:
-        M.moe_set_grouped_mma(True)
-        g = _run_calls(M, hl, dl, z, mma=True)
-    finally:
-        M.moe_set_grouped_mma(False)
-    _check_all(hl, z, g)
-    g2 = _run_calls(M, hl, dl, z, mma=True)
-    _check_all(hl, z, g2)
-    assert np.array_equal(g["idx"], g2["idx"])
+    z = gen.rows(c.seed, 2000, c.T, c.H, accept=gap_ok_predicate(hl))
+    h = torch.from_numpy(z).cuda()
+    ho = torch.empty_like(h)
+    x = torch.empty((c.T, c.H), dtype=torch.int16, device="cuda")
+    y = torch.empty((c.T, c.H), dtype=torch.int16, device="cuda")
+    idx = torch.empty((c.T, c.k), dtype=torch.int32, device="cuda")
+    gates = torch.empty((c.T, c.k), dtype=torch.float32, device="cuda")
+    ws = torch.empty(M.moe_layer_workspace_size(c.T, c.H, c.I, c.Is, c.E, c.k), dtype=torch.uint8, device="cuda")
+    M.moe_layer_forward(c.T, c.H, c.I, c.Is, c.E, c.k, dl.router.c, dl.bias, 0, dl.blob_ptrs, dl.shared_c, ws,
+                        h_in=h, h_out=ho, x_out=x, y=y, idx=idx, gates=gates)
+    M.moe_sync()
+    xg = O.bf16_to_f64(_bits(x))
+    lg = O.router_logits(xg, hl.router, hl.bias)
+    gi = _np(idx)
+    check_routing(gi, lg, c.k)
+    off, _, active = O.buckets(gi, c.E)
+    assert int(np.diff(off).max()) > 128                       # several chunks for the top expert
+    assert np.abs(_np(gates) - O.softmax_gates(lg, gi)).max() < 2e-6
+    r = O.layer_forward(xg, hl.router, hl.bias, hl.expert, hl.shared, c.k, c.E, idx=gi)
+    check_output(_bits(y), r["out"], "y (512 rows)")
+    check_close(_np(ho), z.astype(np.float64) + r["out"], 2e-3, 2e-4, "h + y (512 rows)")

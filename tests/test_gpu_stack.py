@@ -21,18 +21,18 @@ from tests._support import HostStack, check_close, check_output, check_routing, 
 pytestmark = pytest.mark.gpu
 
 
-def _run_stack(M, cfg, layers, z, traces=True):
+def _run_stack(M, cfg, layers, z, traces=True, flags=0):
     T, H, L = z.shape[0], cfg.H, cfg.layers
     stack = M.DecodeStack(layers)
     h = torch.from_numpy(z).cuda()
     ws = torch.empty(M.moe_decode_workspace_size(T, H, cfg.I, cfg.Is, cfg.E, cfg.k), dtype=torch.uint8, device="cuda")
     if traces == "idx":          # only the routing trace, as the benchmark asks
         it = torch.empty((L, T, cfg.k), dtype=torch.int32, device="cuda")
-        M.moe_decode_forward(h, cfg.I, cfg.Is, cfg.E, cfg.k, stack, ws, idx_trace=it)
+        M.moe_decode_forward(h, cfg.I, cfg.Is, cfg.E, cfg.k, stack, ws, idx_trace=it, flags=flags)
         M.moe_sync()
         return dict(h=h.cpu().numpy(), idx=it.cpu().numpy())
     if not traces:
-        M.moe_decode_forward(h, cfg.I, cfg.Is, cfg.E, cfg.k, stack, ws)
+        M.moe_decode_forward(h, cfg.I, cfg.Is, cfg.E, cfg.k, stack, ws, flags=flags)
         M.moe_sync()
         return dict(h=h.cpu().numpy())
     xt = torch.empty((L, T, H), dtype=torch.int16, device="cuda")
@@ -40,7 +40,7 @@ def _run_stack(M, cfg, layers, z, traces=True):
     it = torch.empty((L, T, cfg.k), dtype=torch.int32, device="cuda")
     gt = torch.empty((L, T, cfg.k), dtype=torch.float32, device="cuda")
     M.moe_decode_forward(h, cfg.I, cfg.Is, cfg.E, cfg.k, stack, ws, x_trace=xt, y_trace=yt, idx_trace=it,
-                         gates_trace=gt)
+                         gates_trace=gt, flags=flags)
     M.moe_sync()
     u16 = lambda t: t.cpu().numpy().view(np.uint16)
     return dict(h=h.cpu().numpy(), x=u16(xt), y=u16(yt), idx=it.cpu().numpy(), gates=gt.cpu().numpy())
@@ -92,59 +92,57 @@ def test_stack_tiny_all_layers(M):
 
 
 def test_decode_30L_b1_full(M):
-    """30 layers, batch 1, all resident (12.9 GB): two steps, every layer checked."""
+    """30 layers, batch 1, all resident (12.9 GB): 8 consecutive steps through
+    the persistent kernel (its barrier counter, tagged logits and phase skew
+    carry across steps), every layer of every step checked, residual chain
+    included; then the same kernel with no traces gives the same residual."""
     cfg = CONFIGS["decode_30L_b1"]
     layers = upload_stack(cfg)
     hs = HostStack(cfg)
-    for step in (0, 1):
+    for step in range(8):
         z = gen.rows(cfg.seed, cfg.row_stream + step, 1, cfg.H)
         g = _run_stack(M, cfg, layers, z)
         _check_stack(cfg, hs, z, g, set(range(cfg.layers)))
+        if step == 7:
+            g2 = _run_stack(M, cfg, layers, z, traces=False)
+            assert np.array_equal(g2["h"], g["h"])
 
 
 def test_decode_30L_b64_full(M):
-    """30 layers, 64 rows per step: one step, layers 0, 14 and 29 checked against
-    the oracle, the residual stream checked at every layer."""
+    """30 layers, 64 rows per step: one step, every layer checked against the
+    oracle (teacher-forced on the GPU's layer inputs) and the residual stream
+    checked at every layer."""
     cfg = CONFIGS["decode_30L_b64"]
     layers = upload_stack(cfg)
     z = gen.rows(cfg.seed, cfg.row_stream, cfg.T, cfg.H)
     g = _run_stack(M, cfg, layers, z)
-    _check_stack(cfg, HostStack(cfg), z, g, {0, 14, 29}, chain=False)
+    _check_stack(cfg, HostStack(cfg), z, g, set(range(cfg.layers)), chain=True)
 
 
-@pytest.mark.parametrize("spec", [0, 2])
-def test_stack_tiny_b1_fused_and_layered(M, spec):
-    """Batch 1: the persistent fused kernel and the per-layer path, both against
-    the oracle on every layer; the fused result does not depend on the
-    speculative prefetch setting and is bitwise repeatable."""
+def test_stack_tiny_b1_fused_and_layered(M):
+    """Batch 1: the persistent kernel and the per-layer path
+    (MOE_FLAG_LAYERED), both against the oracle on every layer; the
+    persistent kernel's result is bitwise repeatable and does not depend on
+    which traces are taken."""
     cfg = tiny_config("decode_30L_b1", layers=5, T=1)
     layers = upload_stack(cfg)
     hs = HostStack(cfg)
     z = gen.rows(cfg.seed, 1000, 1, cfg.H)
-    try:
-        M.moe_set_decode_fused(True, spec)
-        gf = _run_stack(M, cfg, layers, z)
-        gf2 = _run_stack(M, cfg, layers, z)
-        M.moe_set_decode_fused(False, spec)
-        gl = _run_stack(M, cfg, layers, z)
-    finally:
-        M.moe_set_decode_fused(True, 0)
+    gf = _run_stack(M, cfg, layers, z)
+    gf2 = _run_stack(M, cfg, layers, z)
+    gl = _run_stack(M, cfg, layers, z, flags=M.MOE_FLAG_LAYERED)
     for g in (gf, gl):
         _check_stack(cfg, hs, z, g, set(range(cfg.layers)))
     for key in ("h", "x", "y", "idx", "gates"):
         assert np.array_equal(gf[key], gf2[key]), key
     assert np.array_equal(gf["idx"], gl["idx"])
-    # traces are optional, each on its own; the result does not depend on them
-    M.moe_set_decode_fused(True, spec)
-    try:
-        g_none = _run_stack(M, cfg, layers, z, traces=False)
-        g_idx = _run_stack(M, cfg, layers, z, traces="idx")
-    finally:
-        M.moe_set_decode_fused(True, 0)
+    g_none = _run_stack(M, cfg, layers, z, traces=False)
+    g_idx = _run_stack(M, cfg, layers, z, traces="idx")
     assert np.array_equal(g_none["h"], gf["h"]) and np.array_equal(g_idx["h"], gf["h"])
     assert np.array_equal(g_idx["idx"], gf["idx"])
 
 
 def test_fused_launch_count(M):
     assert M.moe_decode_launches(1, 30) == 1
-    assert M.moe_decode_launches(2, 30) == 240
+    assert M.moe_decode_launches(1, 30, M.MOE_FLAG_LAYERED) == 240
+    assert M.moe_decode_launches(64, 30) == 210

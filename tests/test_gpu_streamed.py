@@ -84,11 +84,13 @@ def run_resident(M, S, units):
     return outs
 
 
-def run_streamed(M, S, units, lfu, side):
+def run_streamed(M, S, units, lfu, side, on_error=None):
+    """Streamed run; on_error(unit, layer, exc) may clear an injected fault
+    and return True to repeat the failed layer call."""
     c = S.cfg
     outs = []
     main = torch.cuda.current_stream()
-    for z, t0 in units:
+    for u, (z, t0) in enumerate(units):
         T = z.shape[0]
         h = torch.from_numpy(z).cuda()
         ws = torch.empty(M.moe_streamed_workspace_size(T, c.H, c.I, c.Is, c.E, c.k), dtype=torch.uint8, device="cuda")
@@ -97,9 +99,15 @@ def run_streamed(M, S, units, lfu, side):
             y = torch.empty((T, c.H), dtype=torch.int16, device="cuda")
             x = torch.empty((T, c.H), dtype=torch.int16, device="cuda")
             idx = torch.empty((T, c.k), dtype=torch.int32, device="cuda")
-            M.moe_streamed_layer_forward(lfu, l, h, c.I, c.Is, c.E, c.k, S.routers[l].c, S.bias(l, t0, T), 1,
-                                         [m.c for m in S.shared[l]], S.slot_tables[l], ws, x_out=x, y_out=y,
-                                         idx_out=idx, main_stream=main, side_stream=side)
+            while True:
+                try:
+                    M.moe_streamed_layer_forward(lfu, l, h, c.I, c.Is, c.E, c.k, S.routers[l].c, S.bias(l, t0, T),
+                                                 1, [m.c for m in S.shared[l]], S.slot_tables[l], ws, x_out=x,
+                                                 y_out=y, idx_out=idx, main_stream=main, side_stream=side)
+                    break
+                except M.MoeError as exc:
+                    if on_error is None or not on_error(u, l, exc):
+                        raise
             ys.append(y); idxs.append(idx); xs.append(x)
         M.moe_sync()
         outs.append(dict(h=h.cpu().numpy(), y=[t.cpu().numpy() for t in ys], idx=[t.cpu().numpy() for t in idxs],
@@ -200,3 +208,48 @@ def test_lfu_host_faults(M):
     s.synchronize()
     M.moe_lfu_wait(ev, 1000)
     M.moe_sync()
+
+
+def test_lfu_copy_failure_mid_chunk_then_retry(M):
+    """A copy that fails in the middle of a prefill chunk's layer call rolls
+    the layer's cache state back; repeating the call and carrying on gives
+    output bitwise equal to the all-resident run and an access log equal to
+    the simulator's (the failed attempt leaves no record)."""
+    cfg = replace(tiny_config("streamed_30L_lfu"), layers=3, T=24, prompt_tokens=72, decode_steps=4, n_slots=6)
+    S = Streamed(M, cfg)
+    units = S.inputs()
+    ref = run_resident(M, S, units)
+    # misses per (unit, layer) of the policy on this routing, from the simulator
+    sim = LFUSim(cfg.layers, cfg.n_slots)
+    misses = {}
+    for u, o in enumerate(ref):
+        for l in range(cfg.layers):
+            n0 = len(sim.log)
+            idx = o["idx"][l]
+            steps = [[int(e) for e in idx[0]]] if idx.shape[0] == 1 else \
+                sim.chunk_steps(l, np.unique(idx).tolist(), cfg.k)
+            for ids in steps:
+                sim.step(l, ids)
+            misses[(u, l)] = sum(1 for r in sim.log[n0:] if r[3] == 0)
+    # fail the 3rd miss of unit 1 (a prefill chunk), layer 1
+    before = sum(misses[(u, l)] for u in range(1) for l in range(cfg.layers)) + misses[(1, 0)]
+    assert misses[(1, 1)] >= 4
+    lfu = M.MoeLfu(cfg.layers, cfg.E, cfg.n_slots, gen.blob_bytes(cfg.H, cfg.I), S.host_ptrs, S.pool, S.stride)
+    lfu.set_fault(1, before + 2)
+    failures = []
+
+    def on_error(u, l, exc):
+        assert exc.status == 2 and "injected" in str(exc)
+        failures.append((u, l))
+        lfu.set_fault(0, 0)
+        return True
+    got = run_streamed(M, S, units, lfu, torch.cuda.Stream(), on_error=on_error)
+    assert failures == [(1, 1)]
+    for a, b in zip(ref, got):
+        assert np.array_equal(a["h"], b["h"])
+        for l in range(cfg.layers):
+            assert np.array_equal(a["y"][l], b["y"][l]) and np.array_equal(a["idx"][l], b["idx"][l])
+    assert lfu.log() == simulate(S, got).log
+    hits, n_miss, nbytes = lfu.stats()
+    assert n_miss * gen.blob_bytes(cfg.H, cfg.I) <= nbytes      # the failed attempt's copies are extra
+    lfu.close()

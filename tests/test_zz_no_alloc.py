@@ -3,9 +3,11 @@ cannot allocate device memory (no workspace argument; its scratch is a static
 array inside the library).
 
 Checked through the C-ABI against moe_expert_forward with a caller workspace,
-on two calls in a row with different inputs, and for the size limit.  This
-file is collected last so that a run stopping at the first failure has
-already run every other test.
+on two calls in a row with different inputs, and for the size limit.  Both
+calls run the same kernels on the same inputs and differ only in where the
+scratch lives, and every kernel on the path is deterministic, so the outputs
+must be equal bit for bit.  This file is collected last so that a run
+stopping at the first failure has already run every other test.
 """
 from dataclasses import replace
 
@@ -15,7 +17,7 @@ import torch
 
 import gen
 from gen import tiny_config, CONFIGS
-from tests._support import HostLayer, check_close
+from tests._support import HostLayer
 
 pytestmark = pytest.mark.gpu
 
@@ -37,7 +39,7 @@ def _buckets(M, hl, dl, z):
     return x, offs, pairs, active, n_active
 
 
-@pytest.mark.parametrize("which,T", [("tiny", 37), ("full", 16)])
+@pytest.mark.parametrize("which,T", [("tiny", 37), ("full", 16), ("full", 70)])
 def test_noalloc_matches_workspace_entry_on_two_calls(which, T):
     import quantized_moe_bit_b200 as M
     cfg = tiny_config("prefill_1L_128tok", T=T) if which == "tiny" else replace(CONFIGS["prefill_1L_128tok"], T=T)
@@ -53,15 +55,14 @@ def test_noalloc_matches_workspace_entry_on_two_calls(which, T):
         y = torch.full((T * c.k, c.H), float("nan"), dtype=torch.float32, device="cuda")
         M.moe_expert_forward_noalloc(x, c.I, c.E, c.k, dl.blob_ptrs, offs, pairs, active, n_active, y)
         M.moe_sync()
-        a, b = y.cpu().numpy().astype(np.float64), y_ref.cpu().numpy().astype(np.float64)
-        assert np.isfinite(a).all(), f"call {call}: unwritten rows"
-        check_close(a, b, 2e-3, 2e-4, f"noalloc call {call}")
+        assert torch.isfinite(y).all(), f"call {call}: unwritten rows"
+        assert torch.equal(y, y_ref), f"call {call}: differs from the workspace entry point"
 
 
 def test_noalloc_rejects_requests_beyond_the_static_scratch():
     import quantized_moe_bit_b200 as M
     c = CONFIGS["prefill_1L_128tok"]
-    T = 400                                  # 400 * 8 * 704 * 2 bytes > 4 MiB
+    T = 71                                   # 71 rows need more than the 4 MiB scratch
     x = torch.empty((T, c.H), dtype=torch.int16, device="cuda")
     dummy = torch.empty(1024, dtype=torch.int32, device="cuda")
     y = torch.empty((1,), dtype=torch.float32, device="cuda")
