@@ -20,16 +20,22 @@
 //   warps 0-3   epilogue: TMEM -> registers -> GeGLU / fp32 rows to global
 //   warp 4      raw producer: per item its scale/bias rows (4 or 2 bulk
 //               copies into a double buffer), then its packed 4-bit codes,
-//               256 K-values of 128 rows per ring slot as 2-D TMA tiles (a
+//               256 K-values of 128 rows (one stage) per ring slot as 2-D TMA tiles (a
 //               routed expert's tensor maps are a template whose address
 //               the warp patches per item into a small ring in global memory)
-//   warp 5      B producer: per atom the bucket rows' fp16 activations as
-//               one 2-D TMA tile (128-byte swizzle)
-//   warp 6      MMA issuer: 4 x tcgen05.mma (M=128, N, K=16) per atom into
-//               one of two TMEM accumulators (the epilogue of an item
-//               overlaps the next item's MMAs)
-//   warps 7-14  dequant: w = S q + B in half2 arithmetic (q exact, w rounded
-//               once to fp16) from a raw slot into an A atom of the ring
+//   warp 5      B producer: per stage the bucket rows' fp16 activations as
+//               one 2-D TMA tile per atom (128-byte swizzle)
+//   warps 6-9   MMA issuers: 4 x tcgen05.mma (M=128, N, K=16) per atom, A
+//               from TMEM, B from shared memory, into one of two TMEM
+//               accumulator sets (the epilogue of an item overlaps the next
+//               item's MMAs); the 4 MMAs of an atom go to up to 4 issuers
+//               and accumulator chains, since a single thread issues about
+//               one tcgen05.mma per 100 cycles whatever N is
+//   warps 10-25 dequant (two groups of 8): w = S q + B in half2 arithmetic (q exact, w rounded
+//               once to fp16) from a raw slot straight into an A atom of a
+//               ring in TMEM (tcgen05.st): the fp16 operand, 4x the bytes of
+//               the codes, never passes through shared memory, whose
+//               bandwidth it would otherwise exhaust
 // Every mbarrier wait is bounded; a wait that runs out sets the device check
 // word and a CTA-wide abort flag, after which every role stops issuing work,
 // the copies in flight are waited for (bounded) and TMEM is freed.
@@ -40,14 +46,24 @@
 namespace moe {
 
 constexpr int GM_BM = 128;                   // weight rows per item (MMA M)
-constexpr int GM_BK = 64;                    // K per atom
-constexpr int GM_APR = 4;                    // atoms per raw slot
+constexpr int GM_BK = 64;                    // K per atom (one quantisation group)
+// The pipeline moves in stages of GM_APS atoms (K = 256): one raw slot of
+// codes, one A stage in TMEM, one B stage of activation tiles.  Every
+// barrier wait and release covers a whole stage: a single thread pays a few
+// hundred cycles per tcgen05 instruction or mbarrier round trip, which per
+// atom would cost more than the atom's data takes to arrive.
+constexpr int GM_APS = 4;                    // atoms per stage
 constexpr int GM_RAW_SLOT = GM_BM * 128;     // 128 rows x 128 B of codes (256 K values), 128-byte swizzle
-constexpr int GM_RS = 4;                     // raw slots
-constexpr int GM_AS = 3;                     // dequantised A atoms
-constexpr int GM_BS = 3;                     // activation (B) tiles
+constexpr int GM_RS = 3;                     // raw slots
+constexpr int GM_ST = 2;                     // A stages (TMEM) and B stages (shared memory)
 constexpr int GM_NMAX = 128;                 // bucket rows per chunk (MMA N; TMEM columns per accumulator)
-constexpr int GM_ATOM = 128 * 128;           // 16 KB: 128 rows x 128 B
+constexpr int GM_ACOLS = GM_BK / 2;          // TMEM columns of one A atom (two fp16 per 32-bit column)
+constexpr int GM_TMEM_COLS = 512;            // 2 accumulators of GM_NMAX columns, then the A stages
+static_assert(2 * GM_NMAX + GM_ST * GM_APS * GM_ACOLS <= GM_TMEM_COLS, "TMEM budget");
+// accumulator chains of an item with Np (padded) rows: 4 up to 32, 2 at 64, 1 at 128
+__device__ __forceinline__ int gm_chains(int Np) { return Np <= 32 ? 4 : Np <= 64 ? 2 : 1; }
+constexpr int GM_BSLOT = GM_NMAX * 128;      // one atom's activation tile: up to GM_NMAX rows x 128 B
+constexpr int GM_BSTAGE = GM_APS * GM_BSLOT;
 constexpr int GM_MAX_G = 48;                 // quantisation groups per weight row (K <= 3072)
 constexpr int GM_SC_BUF = 4 * (64 * GM_MAX_G * 2 + 16) + 64;   // scale/bias rows of one item (24,704 B)
 static_assert(GM_SC_BUF % 128 == 0, "scale buffers keep the maps after them 128-byte aligned");
@@ -60,17 +76,30 @@ constexpr int GM_MAX_CTAS = 160;             // grid cap (one CTA per SM)
 // patched under a copy still in flight.
 constexpr int GM_MAP_RING = 6;
 static_assert(GM_MAP_RING > GM_RS + 1, "tensor-map ring vs raw ring");
-constexpr int GM_EPI_WARPS = 4, GM_RAW_WARP = 4, GM_B_WARP = 5, GM_MMA_WARP = 6, GM_DQ_WARP0 = 7, GM_DQ_WARPS = 8;
+// MMA issue: one thread issues about one tcgen05.mma per 100 cycles whatever
+// N is, so small-N items are issue-bound; GM_MMA_WARPS warps issue in
+// parallel, each into its own accumulator chain of the item (up to 4 chains
+// of 128 / chains TMEM columns; the epilogue adds them).
+// Dequant: 2 groups of 8 warps; in every stage group g takes the atoms g,
+// g + 2 (an atom's dequant is a latency-bound chain of about 400 cycles, so
+// two run at once).  In a group two warps share each TMEM sub-partition
+// (warp w writes TMEM lanes 32 (w % 4) ..), each taking half of every atom
+// row (4 code words).  Both groups take part in every stage's barriers.
+constexpr int GM_EPI_WARPS = 4, GM_RAW_WARP = 4, GM_B_WARP = 5, GM_MMA_WARP = 6, GM_MMA_WARPS = 4;
+constexpr int GM_DQ_WARP0 = GM_MMA_WARP + GM_MMA_WARPS, GM_DQ_GROUPS = 2, GM_DQ_WARPS = 8 * GM_DQ_GROUPS;
 constexpr int GM_THREADS = (GM_DQ_WARP0 + GM_DQ_WARPS) * 32;
-// barriers: raw full/empty [RS], a full/empty [AS], b full/empty [BS], sc full/empty [2], acc full/empty [2], final
-constexpr int GM_NBARS = 2 * GM_RS + 2 * GM_AS + 2 * GM_BS + 4 + 4 + 1;
-constexpr size_t GM_SMEM = 1024 + static_cast<size_t>(GM_AS) * GM_ATOM + static_cast<size_t>(GM_BS) * GM_ATOM +
+// barriers: raw full/empty [RS], a full [ST], stage empty [ST], b full [ST], sc full/empty [2],
+// acc full/empty [2], final
+constexpr int GM_NBARS = 2 * GM_RS + 3 * GM_ST + 4 + 4 + 1;
+constexpr size_t GM_SMEM = 1024 + static_cast<size_t>(GM_ST) * GM_BSTAGE +
                            static_cast<size_t>(GM_RS) * GM_RAW_SLOT + 2 * GM_SC_BUF + 256 + GM_NBARS * 8 + 64;
 static_assert(GM_SC_BUF % 128 == 0 && GM_RAW_SLOT % 1024 == 0, "copy destinations: swizzle atoms 1024-byte, maps 128-byte aligned");
 static_assert(GM_SMEM <= 232448, "shared memory of the grouped GEMM");
 
-// Box heights of the activation tensor maps (rows of the TMA tile).
-constexpr int GM_NBOX = 4;
+// Box heights of the activation tensor maps (rows of the TMA tile): 16, 32, .. GM_NMAX.
+constexpr int GM_NBOX = GM_NMAX == 128 ? 4 : GM_NMAX == 64 ? 3 : GM_NMAX == 32 ? 2 : 1;
+static_assert((16 << (GM_NBOX - 1)) == GM_NMAX, "GM_NMAX is 16, 32, 64 or 128");
+static_assert(GM_BSLOT % 1024 == 0, "activation tiles are 1024-byte aligned swizzle atoms");
 __host__ __device__ constexpr int gm_box_rows(int i) { return 16 << i; }
 
 // A chunk: up to GM_NMAX consecutive rows of one expert's bucket.
@@ -119,9 +148,17 @@ __device__ __forceinline__ uint32_t gm_sw128(int r, int c) {
 __device__ __forceinline__ __half2 gm_h2(uint32_t v) { return *reinterpret_cast<__half2*>(&v); }
 __device__ __forceinline__ uint32_t gm_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 
-// 8 nibbles of one word -> 8 fp16 weights S*q + B in element order.  Each
-// nibble becomes the fp16 1024 + q (or 1024 + 16 q) by OR-ing it into the
-// exponent pattern 0x6400, minus 1024 (exact); then one fma rounds S*q + B.
+// K order inside every block of 8 K values, for both MMA operands: stored
+// position p holds element kperm(p) = {0, 4, 1, 5, 2, 6, 3, 7}[p] of the block,
+// i.e. element e sits at position 2 (e % 4) + e / 4.  The nibble masks below
+// produce the weights in exactly this order (q0 q4 | q1 q5 | q2 q6 | q3 q7),
+// so the activations are written in it too (gather and GeGLU epilogue) and
+// the sum over K is unchanged.
+__host__ __device__ __forceinline__ int gm_kpos(int e) { return ((e & 7) & 3) * 2 + ((e & 7) >> 2) + (e & ~7); }
+
+// 8 nibbles of one word -> 8 fp16 weights S*q + B in the permuted K order.
+// Each nibble becomes the fp16 1024 + q (or 1024 + 16 q) by OR-ing it into
+// the exponent pattern 0x6400, minus 1024 (exact); then one fma rounds S*q + B.
 __device__ __forceinline__ uint4 gm_dequant_word(uint32_t w, __half2 s2, __half2 b2) {
   const __half2 k1024 = __floats2half2_rn(1024.f, 1024.f);
   const __half2 k16 = __floats2half2_rn(0.0625f, 0.0625f);
@@ -131,21 +168,39 @@ __device__ __forceinline__ uint4 gm_dequant_word(uint32_t w, __half2 s2, __half2
   const __half2 q15 = __hfma2(gm_h2((w & 0x00F000F0u) | 0x64006400u), k16, k64);  // q1, q5
   const __half2 q26 = __hsub2(gm_h2((w8 & 0x000F000Fu) | 0x64006400u), k1024);   // q2, q6
   const __half2 q37 = __hfma2(gm_h2((w8 & 0x00F000F0u) | 0x64006400u), k16, k64); // q3, q7
-  const uint32_t a = gm_u32(__hfma2(q04, s2, b2)), b = gm_u32(__hfma2(q15, s2, b2));
-  const uint32_t c = gm_u32(__hfma2(q26, s2, b2)), d = gm_u32(__hfma2(q37, s2, b2));
   uint4 o;
-  o.x = __byte_perm(a, b, 0x5410);   // w0 w1
-  o.y = __byte_perm(c, d, 0x5410);   // w2 w3
-  o.z = __byte_perm(a, b, 0x7632);   // w4 w5
-  o.w = __byte_perm(c, d, 0x7632);   // w6 w7
+  o.x = gm_u32(__hfma2(q04, s2, b2));
+  o.y = gm_u32(__hfma2(q15, s2, b2));
+  o.z = gm_u32(__hfma2(q26, s2, b2));
+  o.w = gm_u32(__hfma2(q37, s2, b2));
   return o;
+}
+
+__device__ __forceinline__ uint4 gm_lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint2 gm_lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t gm_lds_u16(uint32_t a) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void gm_sts128(uint32_t a, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
 // ------------------------------------------------------------------ prep
 // Block 0 writes the chunk list (shared chunks first, then the routed
 // buckets in active order, each cut into chunks of at most GM_NMAX rows);
 // every block gathers the layer input into bucket order as fp16
-// (xs[pos] = x[pairs[pos] / k]) and, when xh is given, writes x as fp16.
+// (xs[pos] = x[pairs[pos] / k]) and, when xh is given, writes x as fp16;
+// both in the permuted K order of gm_kpos.
 __global__ void __launch_bounds__(256) k_gm_prep(const uint16_t* __restrict__ x, int T, int H, int k,
                                                  const int32_t* __restrict__ offsets,
                                                  const int32_t* __restrict__ pairs,
@@ -224,10 +279,15 @@ __global__ void __launch_bounds__(256) k_gm_prep(const uint16_t* __restrict__ x,
     uint4 o = make_uint4(0u, 0u, 0u, 0u);
     if (t >= 0) {
       const uint4 u = *reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H + 8 * w);
-      o.x = pack_half2(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u));
-      o.y = pack_half2(__uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
-      o.z = pack_half2(__uint_as_float(u.z << 16), __uint_as_float(u.z & 0xFFFF0000u));
-      o.w = pack_half2(__uint_as_float(u.w << 16), __uint_as_float(u.w & 0xFFFF0000u));
+      // elements e0..e7 of the block in the permuted K order e0 e4 | e1 e5 | e2 e6 | e3 e7
+      const float e0 = __uint_as_float(u.x << 16), e1 = __uint_as_float(u.x & 0xFFFF0000u);
+      const float e2 = __uint_as_float(u.y << 16), e3 = __uint_as_float(u.y & 0xFFFF0000u);
+      const float e4 = __uint_as_float(u.z << 16), e5 = __uint_as_float(u.z & 0xFFFF0000u);
+      const float e6 = __uint_as_float(u.w << 16), e7 = __uint_as_float(u.w & 0xFFFF0000u);
+      o.x = pack_half2(e0, e4);
+      o.y = pack_half2(e1, e5);
+      o.z = pack_half2(e2, e6);
+      o.w = pack_half2(e3, e7);
     }
     *reinterpret_cast<uint4*>(dst) = o;
   }
@@ -287,26 +347,30 @@ __device__ __forceinline__ uint32_t gm_region_bytes(int phase, int G) {
   return static_cast<uint32_t>((phase == 0 ? 64 : 128) * G * 2 + 16);
 }
 
-// Bounded mbarrier wait that also gives up when another role of the CTA
-// has aborted (abort flag in shared memory).
+// One try_wait that lets the hardware suspend the thread until the phase
+// completes or about `ns` nanoseconds pass: waiting warps then do not take
+// issue slots from the dequant warps that share their sub-partition.
+__device__ __forceinline__ bool gm_try(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded mbarrier wait (about two seconds) that also gives up when another
+// role of the CTA has aborted (abort flag in shared memory).
 __device__ __forceinline__ bool gm_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-  uint64_t t0 = 0;
-  for (uint32_t i = 0;; ++i) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    if (ok) return true;
-    if ((i & 63u) == 0) {
-      if (*abort_flag) return false;
-      const uint64_t now = tc::globaltimer_ns();
-      if (t0 == 0) t0 = now;
-      else if (now - t0 > 2000000000ull) break;
-    }
+  if (gm_try(bar, parity, 0u)) return true;
+  const uint64_t t0 = tc::globaltimer_ns();
+  for (;;) {
+    if (gm_try(bar, parity, 20000u)) return true;
+    if (*abort_flag) return false;
+    if (tc::globaltimer_ns() - t0 > 2000000000ull) break;
   }
   flag_check(CHECK_WAIT);
   *abort_flag = 1;
@@ -316,22 +380,11 @@ __device__ __forceinline__ bool gm_wait(uint32_t bar, uint32_t parity, volatile 
 // Bounded wait that ignores the abort flag (used on the way out, for copies
 // already in flight and the last MMAs).
 __device__ __forceinline__ void gm_wait_drain(uint32_t bar, uint32_t parity) {
-  uint64_t t0 = 0;
-  for (uint32_t i = 0;; ++i) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    if (ok) return;
-    if ((i & 63u) == 0) {
-      const uint64_t now = tc::globaltimer_ns();
-      if (t0 == 0) t0 = now;
-      else if (now - t0 > 2000000000ull) { flag_check(CHECK_WAIT); return; }
-    }
+  if (gm_try(bar, parity, 0u)) return;
+  const uint64_t t0 = tc::globaltimer_ns();
+  for (;;) {
+    if (gm_try(bar, parity, 20000u)) return;
+    if (tc::globaltimer_ns() - t0 > 2000000000ull) { flag_check(CHECK_WAIT); return; }
   }
 }
 
@@ -340,9 +393,8 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
   extern __shared__ __align__(1024) unsigned char gm_smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(gm_smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* sA = smem;                                      // [AS][16 KB], 1024-aligned
-  unsigned char* sB = sA + GM_AS * GM_ATOM;                      // [BS][16 KB], 1024-aligned
-  unsigned char* sRaw = sB + GM_BS * GM_ATOM;                    // [RS][128 rows x 128 B], swizzled
+  unsigned char* sB = smem;                                      // [ST][GM_APS][GM_BSLOT], 1024-aligned
+  unsigned char* sRaw = sB + GM_ST * GM_BSTAGE;                  // [RS][128 rows x 128 B], swizzled
   unsigned char* sSC = sRaw + GM_RS * GM_RAW_SLOT;               // [2][GM_SC_BUF]
   unsigned char* sMap = sSC + 2 * GM_SC_BUF;                     // [2][128 B] tensor maps being patched
   uint64_t* bars = reinterpret_cast<uint64_t*>(sMap + 256);
@@ -354,10 +406,9 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
   auto raw_full = [&](int s) { return bar0 + 8u * s; };
   auto raw_empty = [&](int s) { return bar0 + 8u * (GM_RS + s); };
   auto a_full = [&](int s) { return bar0 + 8u * (2 * GM_RS + s); };
-  auto a_empty = [&](int s) { return bar0 + 8u * (2 * GM_RS + GM_AS + s); };
-  auto b_full = [&](int s) { return bar0 + 8u * (2 * GM_RS + 2 * GM_AS + s); };
-  auto b_empty = [&](int s) { return bar0 + 8u * (2 * GM_RS + 2 * GM_AS + GM_BS + s); };
-  const uint32_t barx = bar0 + 8u * (2 * GM_RS + 2 * GM_AS + 2 * GM_BS);
+  auto st_empty = [&](int s) { return bar0 + 8u * (2 * GM_RS + GM_ST + s); };   // A and B stage s free
+  auto b_full = [&](int s) { return bar0 + 8u * (2 * GM_RS + 2 * GM_ST + s); };
+  const uint32_t barx = bar0 + 8u * (2 * GM_RS + 3 * GM_ST);
   auto sc_full = [&](int s) { return barx + 8u * s; };
   auto sc_empty = [&](int s) { return barx + 8u * (2 + s); };
   auto acc_full = [&](int s) { return barx + 8u * (4 + s); };
@@ -366,20 +417,25 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < GM_RS; ++s) { tc::mbar_init(raw_full(s), 1); tc::mbar_init(raw_empty(s), GM_DQ_WARPS); }
-    for (int s = 0; s < GM_AS; ++s) { tc::mbar_init(a_full(s), GM_DQ_WARPS); tc::mbar_init(a_empty(s), 1); }
-    for (int s = 0; s < GM_BS; ++s) { tc::mbar_init(b_full(s), 1); tc::mbar_init(b_empty(s), 1); }
+    // a stage: every dequant warp arrives once when its atoms are in TMEM;
+    // every MMA issuer commits once when its MMAs of the stage are done
+    for (int s = 0; s < GM_ST; ++s) {
+      tc::mbar_init(a_full(s), GM_DQ_WARPS);
+      tc::mbar_init(st_empty(s), GM_MMA_WARPS);
+      tc::mbar_init(b_full(s), 1);
+    }
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(sc_full(s), 1);
       tc::mbar_init(sc_empty(s), GM_DQ_WARPS);
-      tc::mbar_init(acc_full(s), 1);
+      tc::mbar_init(acc_full(s), GM_MMA_WARPS);
       tc::mbar_init(acc_empty(s), GM_EPI_WARPS);
     }
-    tc::mbar_init(final_bar, 1);
+    tc::mbar_init(final_bar, GM_MMA_WARPS);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
   if (warp == 0) {
-    tc::tmem_alloc(tc::smem_u32(tmem_slot), 2 * GM_NMAX);
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), GM_TMEM_COLS);
     tc::tmem_relinquish();
   }
   tc::tc_fence_before();
@@ -432,7 +488,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
         }
         ++sc_issued;
       }
-      const int nraw = (it.nkb + GM_APR - 1) / GM_APR;
+      const int nraw = (it.nkb + GM_APS - 1) / GM_APS;
       const CUtensorMap* map0 = &a.tmS[0];
       const CUtensorMap* map1 = &a.tmS[1];
       for (int j = 0; j < nraw; ++j, ++rs) {
@@ -477,7 +533,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
     for (uint32_t q = sc_issued > 2 ? sc_issued - 2 : 0; q < sc_issued; ++q) gm_wait_drain(sc_full(q & 1), (q >> 1) & 1);
   } else if (warp == GM_B_WARP) {
     // ---------------------------------------------------- activation tiles
-    uint32_t bs = 0;
+    uint32_t ss = 0;                                       // stages issued
     bool ok = true;
     for (int item = blockIdx.x; item < n_items && ok; item += G) {
       const GmItem it = gm_item(a, n_sh, item);
@@ -486,44 +542,59 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
       while (bi < GM_NBOX - 1 && gm_box_rows(bi) < Np) ++bi;
       const uint32_t bbytes = static_cast<uint32_t>(gm_box_rows(bi)) * 128u;
       const CUtensorMap* tm = &a.tmB[it.seg][bi];
-      for (int kb = 0; kb < it.nkb; ++kb, ++bs) {
-        const int slot = bs % GM_BS;
-        if (bs >= GM_BS && !(ok = gm_wait(b_empty(slot), ((bs / GM_BS) - 1) & 1, abort_flag))) break;
+      const int nst = (it.nkb + GM_APS - 1) / GM_APS;
+      for (int jst = 0; jst < nst; ++jst, ++ss) {
+        const int slot = ss % GM_ST;
+        if (ss >= GM_ST && !(ok = gm_wait(st_empty(slot), ((ss / GM_ST) - 1) & 1, abort_flag))) break;
+        const int na = min(GM_APS, it.nkb - GM_APS * jst);
         if (lane == 0) {
-          tc::mbar_arrive_tx(b_full(slot), bbytes);
-          tc::tma_load_2d(tc::smem_u32(sB + slot * GM_ATOM), tm, kb * GM_BK, it.row0, b_full(slot));
+          tc::mbar_arrive_tx(b_full(slot), na * bbytes);
+          for (int aa = 0; aa < na; ++aa)
+            tc::tma_load_2d(tc::smem_u32(sB + slot * GM_BSTAGE + aa * GM_BSLOT), tm, (GM_APS * jst + aa) * GM_BK,
+                            it.row0, b_full(slot));
         }
         __syncwarp();
       }
     }
-    for (uint32_t q = bs > GM_BS ? bs - GM_BS : 0; q < bs; ++q) gm_wait_drain(b_full(q % GM_BS), (q / GM_BS) & 1);
-  } else if (warp == GM_MMA_WARP) {
-    // ----------------------------------------------------------- MMA issuer
-    uint32_t as = 0;
+    for (uint32_t q = ss > GM_ST ? ss - GM_ST : 0; q < ss; ++q) gm_wait_drain(b_full(q % GM_ST), (q / GM_ST) & 1);
+  } else if (warp >= GM_MMA_WARP && warp < GM_MMA_WARP + GM_MMA_WARPS) {
+    // ---------------------------------------------------------- MMA issuers
+    // issuer j < C (C chains for the item) issues MMAs kk = j, j + C, .. of
+    // every atom into chain j (TMEM columns acc * GM_NMAX + j * GM_NMAX / C).
+    // Every issuer, active or not, waits for every stage and item and
+    // commits once per stage (st_empty) and once per item (acc_full): the
+    // barriers count GM_MMA_WARPS arrivals, and no issuer runs ahead of the
+    // rings (a parity wait is only unambiguous within one phase).
+    const int j = warp - GM_MMA_WARP;
+    uint32_t ss = 0;
     int il = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < n_items && ok; item += G, ++il) {
       const GmItem it = gm_item(a, n_sh, item);
+      const int Np = (it.N + 15) & ~15;
+      const int C = gm_chains(Np);
       const int acc = il & 1;
       if (il >= 2 && !(ok = gm_wait(acc_empty(acc), ((il >> 1) - 1) & 1, abort_flag))) break;
       tc::tc_fence_after();
-      const int Np = (it.N + 15) & ~15;
       const uint32_t idesc = tc::idesc_f16_f32(GM_BM, Np);
-      const uint32_t dcol = tmem + static_cast<uint32_t>(acc * GM_NMAX);
-      for (int kb = 0; kb < it.nkb; ++kb, ++as) {
-        const int sa = as % GM_AS, sbb = as % GM_BS;
-        if (!(ok = gm_wait(a_full(sa), (as / GM_AS) & 1, abort_flag))) break;
-        if (!(ok = gm_wait(b_full(sbb), (as / GM_BS) & 1, abort_flag))) break;
+      const uint32_t dcol = tmem + static_cast<uint32_t>(acc * GM_NMAX + (j % C) * (GM_NMAX / C));
+      const int nst = (it.nkb + GM_APS - 1) / GM_APS;
+      for (int jst = 0; jst < nst; ++jst, ++ss) {
+        const int slot = ss % GM_ST;
+        if (!(ok = gm_wait(a_full(slot), (ss / GM_ST) & 1, abort_flag))) break;
+        if (!(ok = gm_wait(b_full(slot), (ss / GM_ST) & 1, abort_flag))) break;
         tc::tc_fence_after();
         if (lane == 0) {
-          const uint32_t aBase = tc::smem_u32(sA + sa * GM_ATOM);
-          const uint32_t bBase = tc::smem_u32(sB + sbb * GM_ATOM);
-#pragma unroll
-          for (int kk = 0; kk < GM_BK / 16; ++kk)
-            tc::umma_f16(dcol, tc::sdesc_k_sw128(aBase + kk * 32), tc::sdesc_k_sw128(bBase + kk * 32), idesc,
-                         (kb > 0 || kk > 0) ? 1u : 0u);
-          tc::umma_commit(a_empty(sa));
-          tc::umma_commit(b_empty(sbb));
+          if (j < C) {
+            const int na = min(GM_APS, it.nkb - GM_APS * jst);
+            const uint32_t aT = tmem + static_cast<uint32_t>(2 * GM_NMAX + slot * GM_APS * GM_ACOLS);
+            const uint32_t bBase = tc::smem_u32(sB + slot * GM_BSTAGE);
+            for (int aa = 0; aa < na; ++aa)
+              for (int kk = j; kk < GM_BK / 16; kk += C)   // K = 16: 8 TMEM columns of A, 32 bytes of each B row
+                tc::umma_f16_ta(dcol, aT + aa * GM_ACOLS + kk * 8, tc::sdesc_k_sw128(bBase + aa * GM_BSLOT + kk * 32),
+                                idesc, (jst > 0 || aa > 0 || kk > j) ? 1u : 0u);
+          }
+          tc::umma_commit(st_empty(slot));
         }
         __syncwarp();
       }
@@ -536,11 +607,15 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
     gm_wait_drain(final_bar, 0);
   } else if (warp >= GM_DQ_WARP0) {
     // -------------------------------------------------------------- dequant
-    const int t = threadIdx.x - GM_DQ_WARP0 * 32;      // 0..255
-    const int r = t >> 1, h = t & 1;                     // A row, half of the atom's 64 K values
+    const int dw = warp - GM_DQ_WARP0;
+    const int grp = dw >> 3;                             // dequant group: atoms grp, grp + 2 of every stage
+    const int r = 32 * (warp & 3) + lane;                // A row = this thread's TMEM lane
+    const int h = (dw >> 2) & 1;                         // half h of the row's 8 code words
     // code-tile row of A row r: phase 0 gate row i at tile row i, up row i at 64 + i
     const int R = a.phase == 0 ? (r & 1) * 64 + (r >> 1) : r;
-    uint32_t rs = 0, as = 0;
+    const uint32_t sRaw_u = tc::smem_u32(sRaw);
+    const uint32_t tA = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + static_cast<uint32_t>(2 * GM_NMAX + 16 * h);
+    uint32_t ss = 0;                                     // stages (= raw slots) consumed
     int il = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < n_items && ok; item += G, ++il) {
@@ -549,36 +624,46 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
       if (!(ok = gm_wait(sc_full(sb), (il >> 1) & 1, abort_flag))) break;
       const int Gq = it.nkb;
       const uint32_t reg = gm_region_bytes(a.phase, Gq);
-      const unsigned char* scb = sSC + sb * GM_SC_BUF;
-      const uint16_t *sS, *sBv;
+      const uint32_t scb = tc::smem_u32(sSC + sb * GM_SC_BUF);
+      uint32_t sS_u, sB_u;                                 // this row's scale and bias rows (bf16 per group)
       if (a.phase == 0) {
         const int m = r & 1, i = r >> 1;
-        sS = reinterpret_cast<const uint16_t*>(scb + (2 * m) * reg) + i * Gq;
-        sBv = reinterpret_cast<const uint16_t*>(scb + (2 * m + 1) * reg) + i * Gq;
+        sS_u = scb + (2 * m) * reg + 2 * i * Gq;
+        sB_u = scb + (2 * m + 1) * reg + 2 * i * Gq;
       } else {
-        sS = reinterpret_cast<const uint16_t*>(scb) + r * Gq;
-        sBv = reinterpret_cast<const uint16_t*>(scb + reg) + r * Gq;
+        sS_u = scb + 2 * r * Gq;
+        sB_u = scb + reg + 2 * r * Gq;
       }
-      for (int kb = 0; kb < it.nkb; ++kb, ++as) {
-        const int aa = kb % GM_APR;
-        if (aa == 0 && !(ok = gm_wait(raw_full(rs % GM_RS), (rs / GM_RS) & 1, abort_flag))) break;
-        const int sa = as % GM_AS;
-        if (as >= GM_AS && !(ok = gm_wait(a_empty(sa), ((as / GM_AS) - 1) & 1, abort_flag))) break;
-        const uint4 qq = *reinterpret_cast<const uint4*>(sRaw + (rs % GM_RS) * GM_RAW_SLOT +
-                                                         gm_sw128(R, 2 * aa + h));
-        const float sf = bf16_to_f32(sS[kb]), bf = bf16_to_f32(sBv[kb]);
-        const __half2 s2 = __floats2half2_rn(sf, sf), b2 = __floats2half2_rn(bf, bf);
-        unsigned char* atom = sA + sa * GM_ATOM;
-        *reinterpret_cast<uint4*>(atom + gm_sw128(r, 4 * h + 0)) = gm_dequant_word(qq.x, s2, b2);
-        *reinterpret_cast<uint4*>(atom + gm_sw128(r, 4 * h + 1)) = gm_dequant_word(qq.y, s2, b2);
-        *reinterpret_cast<uint4*>(atom + gm_sw128(r, 4 * h + 2)) = gm_dequant_word(qq.z, s2, b2);
-        *reinterpret_cast<uint4*>(atom + gm_sw128(r, 4 * h + 3)) = gm_dequant_word(qq.w, s2, b2);
-        tc::fence_proxy_async_smem();
+      const int nst = (it.nkb + GM_APS - 1) / GM_APS;
+      for (int jst = 0; jst < nst; ++jst, ++ss) {
+        const int rslot = ss % GM_RS, slot = ss % GM_ST;
+        if (!(ok = gm_wait(raw_full(rslot), (ss / GM_RS) & 1, abort_flag))) break;
+        if (ss >= GM_ST && !(ok = gm_wait(st_empty(slot), ((ss / GM_ST) - 1) & 1, abort_flag))) break;
+        const int na = min(GM_APS, it.nkb - GM_APS * jst);
+        const uint32_t raw = sRaw_u + rslot * GM_RAW_SLOT;
+        for (int aa = grp; aa < na; aa += GM_DQ_GROUPS) {
+          const int kb = GM_APS * jst + aa;
+          // this thread's 4 code words of the atom row (16 bytes at 32 aa + 16 h)
+          const uint4 v = gm_lds128(raw + gm_sw128(R, 2 * aa + h));
+          const float sf = bf16_to_f32(static_cast<uint16_t>(gm_lds_u16(sS_u + 2 * kb)));
+          const float bf = bf16_to_f32(static_cast<uint16_t>(gm_lds_u16(sB_u + 2 * kb)));
+          const __half2 s2 = __floats2half2_rn(sf, sf), b2 = __floats2half2_rn(bf, bf);
+          uint32_t wv[16];
+          const uint32_t qw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 o = gm_dequant_word(qw[q], s2, b2);
+            wv[4 * q + 0] = o.x; wv[4 * q + 1] = o.y; wv[4 * q + 2] = o.z; wv[4 * q + 3] = o.w;
+          }
+          // 32 K values = 16 TMEM columns of this lane in the atom's A slot
+          tc::tmem_st16(tA + static_cast<uint32_t>((slot * GM_APS + aa) * GM_ACOLS), wv);
+        }
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(a_full(sa));
-        if (aa == GM_APR - 1 || kb == it.nkb - 1) {
-          if (lane == 0) tc::mbar_arrive(raw_empty(rs % GM_RS));
-          ++rs;
+        if (lane == 0) {
+          tc::mbar_arrive(a_full(slot));
+          tc::mbar_arrive(raw_empty(rslot));
         }
       }
       if (!ok) break;
@@ -598,9 +683,16 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
       const int Np = (it.N + 15) & ~15;
       const int row = 32 * warp + lane;             // TMEM lane = A row
       const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * warp) << 16) + static_cast<uint32_t>(acc * GM_NMAX);
+      const int C = gm_chains(Np);
       for (int nc = 0; nc < Np; nc += 16) {
         float v[16];
         tc::tmem_ld16(taddr + nc, v);
+        for (int c = 1; c < C; ++c) {        // add the item's other accumulator chains
+          float w2[16];
+          tc::tmem_ld16(taddr + static_cast<uint32_t>(c * (GM_NMAX / C)) + nc, w2);
+#pragma unroll
+          for (int q = 0; q < 16; ++q) v[q] += w2[q];
+        }
         if (a.phase == 0) {
           const int Iw = it.seg ? a.I : a.Is;
           __half* out = it.seg ? a.act_r : a.act_s;
@@ -610,7 +702,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
             const float u = __shfl_xor_sync(0xffffffffu, v[j], 1);
             const int n = nc + j;
             if ((lane & 1) == 0 && n < it.N)
-              out[static_cast<size_t>(it.row0 + n) * Iw + i] = __float2half_rn(gelu_tanh(v[j]) * u);
+              out[static_cast<size_t>(it.row0 + n) * Iw + gm_kpos(i)] = __float2half_rn(gelu_tanh(v[j]) * u);
           }
         } else {
           const int o = GM_BM * it.mt + row;
@@ -640,7 +732,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
-  if (warp == 0) tc::tmem_dealloc(tmem, 2 * GM_NMAX);
+  if (warp == 0) tc::tmem_dealloc(tmem, GM_TMEM_COLS);
 }
 
 }  // namespace moe
