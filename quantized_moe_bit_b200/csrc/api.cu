@@ -627,6 +627,14 @@ static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, con
                         uint16_t* x_trace, uint16_t* y_trace, int32_t* idx_trace, float* gates_trace, void* ws,
                         int G, cudaStream_t s) {
   if (!aligned16(h)) return fail(MOE_ERR_INVALID_ARG, "moe_decode_forward: h must be 16-byte aligned");
+  for (int l = 0; l < L; ++l) {
+    const moe_qmat& R = routers[l];
+    if (!R.q || !R.s || !R.b || R.bits != 8 || R.out != E || R.in != H || !aligned16(R.q) || !aligned16(R.s) ||
+        !aligned16(R.b))
+      return fail(MOE_ERR_INVALID_ARG, "moe_decode_forward: router %d must be 8-bit [E, H] with 16-byte aligned arrays", l);
+    int st = check_shared_mats(shared + 3 * l, H, Is);
+    if (st) return st;
+  }
   char* w = static_cast<char*>(ws);
   __half* act = reinterpret_cast<__half*>(w);
   unsigned long long* logits =
@@ -638,7 +646,7 @@ static int launch_fused(float* h, int H, int I, int Is, int E, int k, int L, con
   if ((st = set_smem(reinterpret_cast<const void*>(k_decode_b1), DF_SMEM_LIMIT))) return st;
   for (int l0 = 0; l0 < L; l0 += DF_MAX_LAYERS) {
     const int nl = L - l0 < DF_MAX_LAYERS ? L - l0 : DF_MAX_LAYERS;
-    static DfArgs args;   // large parameter block; the launch copies it
+    static thread_local DfArgs args;   // large parameter block; the launch copies it
     memset(&args, 0, sizeof(args));
     args.h = h; args.H = H; args.I = I; args.Is = Is; args.E = E; args.k = k; args.L = nl;
     blob_offsets(H, I, args.off);

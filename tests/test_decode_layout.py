@@ -26,6 +26,7 @@ def checker(tmp_path_factory):
     (2816, 704, 2112, 128, 8, 148),     # the 30-layer decode workload on 148 SMs
     (2816, 704, 2112, 128, 8, 160),
     (256, 128, 192, 16, 4, 148),        # the tiny test configuration
+    (192, 128, 192, 16, 4, 148),        # an odd number of 64-groups along H
     (512, 192, 320, 32, 8, 100),
     (2048, 512, 1024, 64, 6, 148),
 ])
