@@ -229,9 +229,9 @@ static int run_gemm(const uint16_t* x, int T, int H, const RoutedIn* rt, const S
   const int k = rt ? rt->k : 1;
   const long P = rt ? static_cast<long>(T) * k : 0;
   {
-    const long work = (P + (sh ? T : 0)) * (H / 8);
-    int blocks = static_cast<int>((work + 255) / 256);
-    blocks = blocks < 1 ? 1 : (blocks > 4 * sm_count() ? 4 * sm_count() : blocks);
+    const long rows = P + (sh ? T : 0);     // one row per block and step
+    int blocks = static_cast<int>(rows < 4L * sm_count() ? rows : 4L * sm_count());
+    blocks = blocks < 1 ? 1 : blocks;
     k_gm_prep<<<blocks, 256, 0, s>>>(x, T, H, k, rt ? rt->offsets : nullptr, rt ? rt->pairs : nullptr,
                                      rt ? rt->active : nullptr, rt ? rt->n_active : nullptr, rt ? rt->E : 0,
                                      rt ? 1 : 0, sh ? T : 0, xs, sh ? xh : nullptr, plan);
@@ -405,7 +405,7 @@ int moe_router_topk(const uint16_t* x, int T, int H, const moe_qmat* router, con
   st = set_smem(reinterpret_cast<const void*>(k_router_topk), smem);
   if (st) return st;
   const int nblk = (T + ROUTER_TB - 1) / ROUTER_TB;
-  k_router_topk<<<nblk * 8, 256, smem, static_cast<cudaStream_t>(stream)>>>(
+  k_router_topk<<<nblk * 8, ROUTER_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
       x, T, H, router->q, router->s, router->b, bias, bias_per_row, E, k, idx, gates, logits_opt);
   return launch_check("k_router_topk");
 }
@@ -416,8 +416,10 @@ int moe_bucket(const int32_t* idx, int T, int k, int E, int32_t* offsets, int32_
   if (st) return st;
   if (static_cast<long>(T) * k > 65536) return fail(MOE_ERR_UNSUPPORTED, "moe_bucket: T*k > 65536");
   if (!idx || !offsets || !pairs || !active || !n_active) return fail(MOE_ERR_INVALID_ARG, "moe_bucket: NULL pointer");
-  k_bucket<<<1, 256, 2 * E * sizeof(int), static_cast<cudaStream_t>(stream)>>>(idx, T * k, E, offsets, pairs,
-                                                                              active, n_active);
+  const size_t bsm = (BUCKET_THREADS / 32 + 1) * static_cast<size_t>(E) * sizeof(int);   // per-warp histograms
+  if (bsm > 48 * 1024 && (st = set_smem(reinterpret_cast<const void*>(k_bucket), bsm))) return st;
+  k_bucket<<<1, BUCKET_THREADS, bsm, static_cast<cudaStream_t>(stream)>>>(idx, T * k, E, offsets, pairs, active,
+                                                                         n_active);
   return launch_check("k_bucket");
 }
 
@@ -481,8 +483,14 @@ int moe_combine(const float* y_pairs, const float* gates, const float* ysh, int 
   if (T < 0 || H <= 0 || k < 1 || k > 8) return fail(MOE_ERR_INVALID_ARG, "moe_combine: bad T/H/k");
   if (T == 0) return MOE_OK;
   if (!y_pairs || !gates) return fail(MOE_ERR_INVALID_ARG, "moe_combine: NULL pointer");
-  k_combine<<<dim3((H + 255) / 256, T), 256, 0, static_cast<cudaStream_t>(stream)>>>(y_pairs, gates, ysh, H, k, y,
-                                                                                 residual_inout);
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const bool vec = H % 4 == 0 && aligned16(y_pairs) && (!ysh || aligned16(ysh)) && (!residual_inout || aligned16(residual_inout)) &&
+                   (reinterpret_cast<uintptr_t>(y) & 7) == 0;
+  if (vec) {
+    k_combine4<<<dim3((H / 4 + 255) / 256, T), 256, 0, cs>>>(y_pairs, gates, ysh, H, k, y, residual_inout);
+    return launch_check("k_combine4");
+  }
+  k_combine<<<dim3((H + 255) / 256, T), 256, 0, cs>>>(y_pairs, gates, ysh, H, k, y, residual_inout);
   return launch_check("k_combine");
 }
 

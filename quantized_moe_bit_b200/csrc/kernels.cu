@@ -35,15 +35,17 @@ __global__ void k_rmsnorm(const float* __restrict__ h, int H, float eps, uint16_
 
 // --------------------------------------------------------------------- A1+A2
 // Cluster of 8 CTAs per block of ROUTER_TB rows.  CTA rank r computes the
-// logits of experts [r*E/8, (r+1)*E/8) for those rows and writes them into
-// rank 0's shared memory; after the cluster barrier rank 0 selects the top k
-// per row (one warp per row) and applies the softmax.
+// logits of experts [r*E/8, (r+1)*E/8) for those rows (one warp per expert)
+// and writes them into rank 0's shared memory; after the cluster barrier
+// rank 0 selects the top k per row (one warp per row) and applies the softmax.
 //
 // x is staged as "byte-paired" half2: word m of a row holds elements 4m..4m+3
 // as P0 = (v0, v2), P1 = (v1, v3), stored word-pair-major per 16-element
 // chunk so lane c reads consecutive bytes.  Chunk stats per 16 elements:
-// (1024 * sum of stored halves, plain sum).
-__global__ void __cluster_dims__(8, 1, 1) __launch_bounds__(256)
+// (1024 * sum of stored halves, plain sum).  Every load of a thread's batch
+// (x words; a lane's router chunks with their scale and bias) is issued
+// before any of it is used, so a warp waits one memory latency per batch.
+__global__ void __cluster_dims__(8, 1, 1) __launch_bounds__(ROUTER_THREADS)
 k_router_topk(const uint16_t* __restrict__ x, int T, int H, const uint32_t* __restrict__ rq,
               const uint16_t* __restrict__ rs, const uint16_t* __restrict__ rb,
               const float* __restrict__ bias, int bias_per_row, int E, int k,
@@ -59,27 +61,41 @@ k_router_topk(const uint16_t* __restrict__ x, int T, int H, const uint32_t* __re
   unsigned char* xs = smem + ROUTER_TB * E * sizeof(float);
   const size_t row_bytes = static_cast<size_t>(nch) * 4 * sizeof(uint2) + nch * sizeof(float2);
 
-  // stage x rows
-  for (int i = threadIdx.x; i < nrows * nch; i += blockDim.x) {
-    const int r = i / nch, c = i - r * nch;
-    const uint16_t* src = x + static_cast<size_t>(row0 + r) * H + 16 * c;
-    uint2* P = reinterpret_cast<uint2*>(xs + r * row_bytes);
-    float2* st = reinterpret_cast<float2*>(xs + r * row_bytes + static_cast<size_t>(nch) * 4 * sizeof(uint2));
-    float off = 0.f, sum = 0.f;
-    const uint4 u0 = *reinterpret_cast<const uint4*>(src);
-    const uint4 u1 = *reinterpret_cast<const uint4*>(src + 8);
-    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+  // stage x rows, ROUTER_XB items per thread per batch
+  const int nitems = nrows * nch;
+  for (int i0 = threadIdx.x; i0 < nitems; i0 += blockDim.x * ROUTER_XB) {
+    uint4 u[ROUTER_XB][2];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {          // word m covers elements 4m..4m+3
-      const float v0 = __uint_as_float(w[2 * m] << 16), v1 = __uint_as_float(w[2 * m] & 0xFFFF0000u);
-      const float v2 = __uint_as_float(w[2 * m + 1] << 16), v3 = __uint_as_float(w[2 * m + 1] & 0xFFFF0000u);
-      const uint32_t p0 = pack_half2(v0, v2), p1 = pack_half2(v1, v3);
-      P[m * nch + c] = make_uint2(p0, p1);
-      const float2 f0 = unpack_half2(p0), f1 = unpack_half2(p1);
-      off += (f0.x + f0.y) + (f1.x + f1.y);
+    for (int j = 0; j < ROUTER_XB; ++j) {
+      const int i = i0 + j * static_cast<int>(blockDim.x);
+      if (i < nitems) {
+        const int r = i / nch, c = i - r * nch;
+        const uint16_t* src = x + static_cast<size_t>(row0 + r) * H + 16 * c;
+        u[j][0] = *reinterpret_cast<const uint4*>(src);
+        u[j][1] = *reinterpret_cast<const uint4*>(src + 8);
+      }
     }
-    sum = off;
-    st[c] = make_float2(1024.f * off, sum);
+#pragma unroll
+    for (int j = 0; j < ROUTER_XB; ++j) {
+      const int i = i0 + j * static_cast<int>(blockDim.x);
+      if (i < nitems) {
+        const int r = i / nch, c = i - r * nch;
+        uint2* P = reinterpret_cast<uint2*>(xs + r * row_bytes);
+        float2* st = reinterpret_cast<float2*>(xs + r * row_bytes + static_cast<size_t>(nch) * 4 * sizeof(uint2));
+        float off = 0.f;
+        const uint32_t w[8] = {u[j][0].x, u[j][0].y, u[j][0].z, u[j][0].w, u[j][1].x, u[j][1].y, u[j][1].z, u[j][1].w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {          // word m covers elements 4m..4m+3
+          const float v0 = __uint_as_float(w[2 * m] << 16), v1 = __uint_as_float(w[2 * m] & 0xFFFF0000u);
+          const float v2 = __uint_as_float(w[2 * m + 1] << 16), v3 = __uint_as_float(w[2 * m + 1] & 0xFFFF0000u);
+          const uint32_t p0 = pack_half2(v0, v2), p1 = pack_half2(v1, v3);
+          P[m * nch + c] = make_uint2(p0, p1);
+          const float2 f0 = unpack_half2(p0), f1 = unpack_half2(p1);
+          off += (f0.x + f0.y) + (f1.x + f1.y);
+        }
+        st[c] = make_float2(1024.f * off, off);
+      }
+    }
   }
   __syncthreads();
 
@@ -93,23 +109,39 @@ k_router_topk(const uint16_t* __restrict__ x, int T, int H, const uint32_t* __re
     float acc[ROUTER_TB];
 #pragma unroll
     for (int r = 0; r < ROUTER_TB; ++r) acc[r] = 0.f;
-    for (int c = lane; c < nch; c += 32) {
-      const uint4 q = ldg_nc_v4(qrow + static_cast<size_t>(c) * 16);
-      const float sc = bf16_to_f32(ldg_u16(rs + static_cast<size_t>(e) * (H / 64) + (c >> 2)));
-      const float bi = bf16_to_f32(ldg_u16(rb + static_cast<size_t>(e) * (H / 64) + (c >> 2)));
+    // the lane's chunks c = lane, lane + 32, ... in order, ROUTER_CB at a time
+    for (int c0 = lane; c0 < nch; c0 += 32 * ROUTER_CB) {
+      uint4 q[ROUTER_CB];
+      float sc[ROUTER_CB], bi[ROUTER_CB];
 #pragma unroll
-      for (int r = 0; r < ROUTER_TB; ++r) {
-        if (r < nrows) {
-          const uint2* P = reinterpret_cast<const uint2*>(xs + r * row_bytes);
-          const float2* st = reinterpret_cast<const float2*>(xs + r * row_bytes + static_cast<size_t>(nch) * 4 * sizeof(uint2));
-          float a0 = 0.f, a1 = 0.f;
-          uint2 p;
-          p = P[0 * nch + c]; { uint32_t pp[2] = {p.x, p.y}; dot_word8(q.x, pp, a0, a1); }
-          p = P[1 * nch + c]; { uint32_t pp[2] = {p.x, p.y}; dot_word8(q.y, pp, a0, a1); }
-          p = P[2 * nch + c]; { uint32_t pp[2] = {p.x, p.y}; dot_word8(q.z, pp, a0, a1); }
-          p = P[3 * nch + c]; { uint32_t pp[2] = {p.x, p.y}; dot_word8(q.w, pp, a0, a1); }
-          const float2 s2 = st[c];
-          acc[r] += sc * ((a0 + a1) - s2.x) + bi * s2.y;
+      for (int b = 0; b < ROUTER_CB; ++b) {
+        const int c = c0 + 32 * b;
+        if (c < nch) {
+          q[b] = ldg_nc_v4(qrow + static_cast<size_t>(c) * 16);
+          sc[b] = bf16_to_f32(ldg_u16(rs + static_cast<size_t>(e) * (H / 64) + (c >> 2)));
+          bi[b] = bf16_to_f32(ldg_u16(rb + static_cast<size_t>(e) * (H / 64) + (c >> 2)));
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < ROUTER_CB; ++b) {
+        const int c = c0 + 32 * b;
+        if (c < nch) {
+#pragma unroll
+          for (int r = 0; r < ROUTER_TB; ++r) {
+            if (r < nrows) {
+              const uint2* P = reinterpret_cast<const uint2*>(xs + r * row_bytes);
+              const float2* st =
+                  reinterpret_cast<const float2*>(xs + r * row_bytes + static_cast<size_t>(nch) * 4 * sizeof(uint2));
+              float a0 = 0.f, a1 = 0.f;
+              uint2 p;
+              p = P[0 * nch + c]; { uint32_t pp[2] = {p.x, p.y}; dot_word8(q[b].x, pp, a0, a1); }
+              p = P[1 * nch + c]; { uint32_t pp[2] = {p.x, p.y}; dot_word8(q[b].y, pp, a0, a1); }
+              p = P[2 * nch + c]; { uint32_t pp[2] = {p.x, p.y}; dot_word8(q[b].z, pp, a0, a1); }
+              p = P[3 * nch + c]; { uint32_t pp[2] = {p.x, p.y}; dot_word8(q[b].w, pp, a0, a1); }
+              const float2 s2 = st[c];
+              acc[r] += sc[b] * ((a0 + a1) - s2.x) + bi[b] * s2.y;
+            }
+          }
         }
       }
     }
@@ -166,29 +198,54 @@ k_router_topk(const uint16_t* __restrict__ x, int T, int H, const uint32_t* __re
 }
 
 // ------------------------------------------------------------------------ A3
-// One block.  Counts with shared atomics (order-free), exclusive scan, then a
-// single warp places the pairs chunk by chunk in index order (stable).
-__global__ void k_bucket(const int32_t* __restrict__ idx, int n, int E, int32_t* __restrict__ offsets,
-                         int32_t* __restrict__ pairs, int32_t* __restrict__ active,
-                         int32_t* __restrict__ n_active) {
+// One block of BUCKET_THREADS.  Warp w owns the pairs [w n / W, (w+1) n / W)
+// (W warps): it counts them per expert (order-free shared atomics into its
+// own histogram row), then, after an exclusive scan over (expert, warp),
+// places them in index order from its own start offsets -- so the pairs of
+// every expert come out in index order (stable) with all warps placing at
+// once.  Pair indices are loaded BUCKET_B chunks of 32 at a time.
+__global__ void __launch_bounds__(BUCKET_THREADS)
+k_bucket(const int32_t* __restrict__ idx, int n, int E, int32_t* __restrict__ offsets,
+         int32_t* __restrict__ pairs, int32_t* __restrict__ active, int32_t* __restrict__ n_active) {
   extern __shared__ int sh[];
-  int* cnt = sh;          // [E]
-  int* cur = sh + E;      // [E]
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  constexpr int W = BUCKET_THREADS / 32;
+  int* hist = sh;           // [W][E]: counts, then start offsets
+  int* tot = sh + W * E;    // [E]: counts, then expert offsets
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < W * E; i += BUCKET_THREADS) hist[i] = 0;
   __syncthreads();
-  for (int p = threadIdx.x; p < n; p += blockDim.x) {
-    const int e = idx[p];
-    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
-    else flag_check(CHECK_EXPERT_ID);
+  const int p0 = static_cast<int>(static_cast<long>(n) * warp / W);
+  const int p1 = static_cast<int>(static_cast<long>(n) * (warp + 1) / W);
+  int* h = hist + warp * E;
+  for (int q0 = p0; q0 < p1; q0 += 32 * BUCKET_B) {
+    int ev[BUCKET_B];
+#pragma unroll
+    for (int b = 0; b < BUCKET_B; ++b) {
+      const int p = q0 + 32 * b + lane;
+      ev[b] = p < p1 ? idx[p] : -1;
+    }
+#pragma unroll
+    for (int b = 0; b < BUCKET_B; ++b) {
+      const int p = q0 + 32 * b + lane;
+      if (p < p1) {
+        if (ev[b] >= 0 && ev[b] < E) atomicAdd(&h[ev[b]], 1);
+        else flag_check(CHECK_EXPERT_ID);
+      }
+    }
   }
   __syncthreads();
-  if (threadIdx.x < 32) {
-    // warp scan over E in chunks of 32
-    const int lane = threadIdx.x;
+  for (int e = threadIdx.x; e < E; e += BUCKET_THREADS) {
+    int c = 0;
+    for (int w = 0; w < W; ++w) c += hist[w * E + e];
+    tot[e] = c;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // warp scan over E in chunks of 32: expert offsets and the active list
     int base = 0, abase = 0;
     for (int e0 = 0; e0 < E; e0 += 32) {
       const int e = e0 + lane;
-      const int v = e < E ? cnt[e] : 0;
+      const int v = e < E ? tot[e] : 0;
       const int a = v > 0 ? 1 : 0;
       int incl = v, ainc = a;
 #pragma unroll
@@ -199,7 +256,7 @@ __global__ void k_bucket(const int32_t* __restrict__ idx, int n, int E, int32_t*
       }
       if (e < E) {
         offsets[e] = base + incl - v;
-        cur[e] = base + incl - v;
+        tot[e] = base + incl - v;
         if (a) active[abase + ainc - 1] = e;
       }
       base += __shfl_sync(0xffffffffu, incl, 31);
@@ -209,18 +266,33 @@ __global__ void k_bucket(const int32_t* __restrict__ idx, int n, int E, int32_t*
       offsets[E] = base;
       *n_active = abase;
     }
-    __syncwarp();
-    for (int p0 = 0; p0 < n; p0 += 32) {
-      const int p = p0 + lane;
-      const int e = p < n ? idx[p] : -1;
-      const bool ok = (e >= 0 && e < E);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += BUCKET_THREADS) {
+    int s = tot[e];
+    for (int w = 0; w < W; ++w) {
+      const int c = hist[w * E + e];
+      hist[w * E + e] = s;
+      s += c;
+    }
+  }
+  __syncthreads();
+  for (int q0 = p0; q0 < p1; q0 += 32 * BUCKET_B) {
+    int ev[BUCKET_B];
+#pragma unroll
+    for (int b = 0; b < BUCKET_B; ++b) {
+      const int p = q0 + 32 * b + lane;
+      ev[b] = p < p1 ? idx[p] : -1;
+    }
+#pragma unroll
+    for (int b = 0; b < BUCKET_B; ++b) {
+      const int p = q0 + 32 * b + lane;
+      const int e = ev[b];
+      const bool ok = p < p1 && e >= 0 && e < E;
       const unsigned m = __match_any_sync(0xffffffffu, ok ? e : -1);
-      if (ok) {
-        const int rk = __popc(m & ((1u << lane) - 1u));
-        pairs[cur[e] + rk] = p;
-      }
+      if (ok) pairs[h[e] + __popc(m & ((1u << lane) - 1u))] = p;
       __syncwarp();
-      if (ok && (__ffs(m) - 1) == lane) cur[e] += __popc(m);
+      if (ok && (__ffs(m) - 1) == lane) h[e] += __popc(m);
       __syncwarp();
     }
   }
@@ -350,6 +422,52 @@ __global__ void k_combine(const float* __restrict__ yp, const float* __restrict_
   if (ysh != nullptr) acc += ysh[static_cast<size_t>(t) * H + c];
   if (y != nullptr) y[static_cast<size_t>(t) * H + c] = f32_to_bf16(acc);
   if (resid != nullptr) resid[static_cast<size_t>(t) * H + c] += acc;
+}
+
+// The same sum four columns per thread (16-byte aligned arrays, H % 4 == 0):
+// the k pair rows are loaded before the fma chain, which runs in the same
+// order (j = 0 .. k-1, then the shared row), so the result is bit-identical.
+__global__ void __launch_bounds__(256)
+k_combine4(const float* __restrict__ yp, const float* __restrict__ gates, const float* __restrict__ ysh, int H,
+           int k, uint16_t* __restrict__ y, float* __restrict__ resid) {
+  const int t = blockIdx.y;
+  const int c = 4 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (c >= H) return;
+  float g[8];
+  float4 v[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j < k) {
+      g[j] = gates[static_cast<size_t>(t) * k + j];
+      v[j] = *reinterpret_cast<const float4*>(yp + (static_cast<size_t>(t) * k + j) * H + c);
+    }
+  }
+  const float4 sh = ysh != nullptr ? *reinterpret_cast<const float4*>(ysh + static_cast<size_t>(t) * H + c)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j < k) {
+      a0 = fmaf(g[j], v[j].x, a0);
+      a1 = fmaf(g[j], v[j].y, a1);
+      a2 = fmaf(g[j], v[j].z, a2);
+      a3 = fmaf(g[j], v[j].w, a3);
+    }
+  }
+  if (ysh != nullptr) {
+    a0 += sh.x; a1 += sh.y; a2 += sh.z; a3 += sh.w;
+  }
+  const size_t o = static_cast<size_t>(t) * H + c;
+  if (y != nullptr) {
+    const uint2 pk = make_uint2(static_cast<uint32_t>(f32_to_bf16(a0)) | (static_cast<uint32_t>(f32_to_bf16(a1)) << 16),
+                                static_cast<uint32_t>(f32_to_bf16(a2)) | (static_cast<uint32_t>(f32_to_bf16(a3)) << 16));
+    *reinterpret_cast<uint2*>(y + o) = pk;
+  }
+  if (resid != nullptr) {
+    float4 r = *reinterpret_cast<float4*>(resid + o);
+    r.x += a0; r.y += a1; r.z += a2; r.w += a3;
+    *reinterpret_cast<float4*>(resid + o) = r;
+  }
 }
 
 }  // namespace moe

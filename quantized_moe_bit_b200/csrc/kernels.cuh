@@ -5,6 +5,11 @@
 namespace moe {
 
 constexpr int ROUTER_TB = 8;     // rows per router cluster
+constexpr int ROUTER_THREADS = 512;   // threads per router CTA (one warp per expert of the CTA's E/8)
+constexpr int ROUTER_XB = 4;     // x chunks a router thread loads before staging them
+constexpr int ROUTER_CB = 8;     // router chunks a lane loads before using them
+constexpr int BUCKET_THREADS = 512;   // one block; each warp buckets a contiguous run of pairs
+constexpr int BUCKET_B = 8;      // chunks of 32 pair indices a bucket warp loads at once
 constexpr int GEMV_RG = 4;       // bucket rows staged at once by the GEMV kernels
 constexpr int GEMV_ROWS = 32;    // output rows per GEMV block
 
@@ -49,6 +54,8 @@ __global__ void k_gateup_gemv(GateUpArgs a);
 __global__ void k_down_gemv(DownArgs a);
 __global__ void k_combine(const float* yp, const float* gates, const float* ysh, int H, int k,
                           uint16_t* y, float* resid);
+__global__ void k_combine4(const float* yp, const float* gates, const float* ysh, int H, int k,
+                           uint16_t* y, float* resid);
 
 inline size_t router_smem_bytes(int H, int E) {
   const int nch = H / 16;

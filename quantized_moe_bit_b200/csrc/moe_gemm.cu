@@ -60,14 +60,16 @@ constexpr int GM_NMAX = 128;                 // bucket rows per chunk (MMA N; TM
 constexpr int GM_ACOLS = GM_BK / 2;          // TMEM columns of one A atom (two fp16 per 32-bit column)
 constexpr int GM_TMEM_COLS = 512;            // 2 accumulators of GM_NMAX columns, then the A stages
 static_assert(2 * GM_NMAX + GM_ST * GM_APS * GM_ACOLS <= GM_TMEM_COLS, "TMEM budget");
-// accumulator chains of an item with Np (padded) rows: 4 up to 32, 2 at 64, 1 at 128
-__device__ __forceinline__ int gm_chains(int Np) { return Np <= 32 ? 4 : Np <= 64 ? 2 : 1; }
+// accumulator chains of an item with Np (padded) rows: as many (up to 4) as
+// fit side by side in one accumulator of GM_NMAX columns
+__device__ __forceinline__ int gm_chains(int Np) { return Np <= GM_NMAX / 4 ? 4 : Np <= GM_NMAX / 2 ? 2 : 1; }
 constexpr int GM_BSLOT = GM_NMAX * 128;      // one atom's activation tile: up to GM_NMAX rows x 128 B
 constexpr int GM_BSTAGE = GM_APS * GM_BSLOT;
 constexpr int GM_MAX_G = 48;                 // quantisation groups per weight row (K <= 3072)
 constexpr int GM_SC_BUF = 4 * (64 * GM_MAX_G * 2 + 16) + 64;   // scale/bias rows of one item (24,704 B)
 static_assert(GM_SC_BUF % 128 == 0, "scale buffers keep the maps after them 128-byte aligned");
 constexpr int GM_MAX_CHUNKS = 512;
+constexpr int GM_PREP_W = (GM_MAX_G * 64 / 8 + 255) / 256;   // 16-byte words of a row per prep thread
 constexpr int GM_MAX_CTAS = 160;             // grid cap (one CTA per SM)
 // Per-CTA tensor-map sets (gate and up, or down) in global memory.  An
 // item's set is patched after the wait that frees its first raw slot, which
@@ -196,8 +198,10 @@ __device__ __forceinline__ void gm_sts128(uint32_t a, uint4 v) {
 }
 
 // ------------------------------------------------------------------ prep
-// Block 0 writes the chunk list (shared chunks first, then the routed
-// buckets in active order, each cut into chunks of at most GM_NMAX rows);
+// Block 0 writes the chunk list: shared chunks first, then the routed
+// buckets cut into chunks of at most GM_NMAX rows, largest chunks first (a
+// counting sort by size; the order within a size is free), so that the
+// grid's serpentine walk over the items balances the CTAs;
 // every block gathers the layer input into bucket order as fp16
 // (xs[pos] = x[pairs[pos] / k]) and, when xh is given, writes x as fp16;
 // both in the permuted K order of gm_kpos.
@@ -209,43 +213,47 @@ __global__ void __launch_bounds__(256) k_gm_prep(const uint16_t* __restrict__ x,
                                                  int shared_rows, __half* __restrict__ xs, __half* __restrict__ xh,
                                                  GmPlan* __restrict__ plan) {
   if (blockIdx.x == 0) {
+    __shared__ int s_cnt[GM_NMAX + 1];     // routed chunks per size, then the next slot of each size
     const int nsh = (shared_rows + GM_NMAX - 1) / GM_NMAX;
     for (int c = threadIdx.x; c < nsh; c += blockDim.x) {
       const int n0 = c * GM_NMAX, n = min(GM_NMAX, shared_rows - n0);
       plan->chunk[c] = make_uint2(0u, static_cast<uint32_t>(n0) | (static_cast<uint32_t>(n) << 24));
     }
+    for (int i = threadIdx.x; i <= GM_NMAX; i += blockDim.x) s_cnt[i] = 0;
     int na = routed ? *n_active : 0;
     if (na < 0 || na > E) { if (threadIdx.x == 0) flag_check(CHECK_EXPERT_ID); na = 0; }
-    // one warp: 32 experts per round, chunk counts scanned across the warp
+    auto bucket = [&](int a, int& e, int& pos0, int& cnt) {
+      e = active[a];
+      pos0 = 0;
+      cnt = 0;
+      if (e < 0 || e >= E) { flag_check(CHECK_EXPERT_ID); e = 0; }
+      else { pos0 = offsets[e]; cnt = offsets[e + 1] - pos0; }
+      if (cnt < 0) cnt = 0;
+    };
+    __syncthreads();
+    for (int a = threadIdx.x; a < na; a += blockDim.x) {      // chunks per size
+      int e, pos0, cnt;
+      bucket(a, e, pos0, cnt);
+      if (cnt / GM_NMAX) atomicAdd(&s_cnt[GM_NMAX], cnt / GM_NMAX);
+      if (cnt % GM_NMAX) atomicAdd(&s_cnt[cnt % GM_NMAX], 1);
+    }
+    __syncthreads();
     if (threadIdx.x < 32) {
+      // first slot of every size, the largest chunks first (a warp scan over
+      // sizes GM_NMAX .. 1, 32 at a time)
       const int lane = threadIdx.x;
       int base = nsh;
-      for (int a0 = 0; a0 < na; a0 += 32) {
-        const int a = a0 + lane;
-        int e = 0, pos0 = 0, cnt = 0;
-        if (a < na) {
-          e = active[a];
-          if (e < 0 || e >= E) { flag_check(CHECK_EXPERT_ID); e = 0; }
-          else { pos0 = offsets[e]; cnt = offsets[e + 1] - pos0; }
-          if (cnt < 0) cnt = 0;
-        }
-        const int nch = (cnt + GM_NMAX - 1) / GM_NMAX;
-        int incl = nch;
+      for (int n0 = GM_NMAX; n0 >= 1; n0 -= 32) {
+        const int n = n0 - lane;
+        const int v = n >= 1 ? s_cnt[n] : 0;
+        int incl = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += v;
+          const int t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
         }
-        const int total = __shfl_sync(0xffffffffu, incl, 31);
-        for (int c = 0; c < nch; ++c) {
-          const int slot = base + incl - nch + c;
-          if (slot < GM_MAX_CHUNKS) {
-            const int n0 = c * GM_NMAX, n = min(GM_NMAX, cnt - n0);
-            plan->chunk[slot] = make_uint2(static_cast<uint32_t>(e) | 0x80000000u,
-                                           static_cast<uint32_t>(pos0 + n0) | (static_cast<uint32_t>(n) << 24));
-          }
-        }
-        base += total;
+        if (n >= 1) s_cnt[n] = base + incl - v;
+        base += __shfl_sync(0xffffffffu, incl, 31);
       }
       if (lane == 0) {
         int nr = base - nsh;
@@ -254,42 +262,61 @@ __global__ void __launch_bounds__(256) k_gm_prep(const uint16_t* __restrict__ x,
         plan->n_chunks[1] = nr;
       }
     }
+    __syncthreads();
+    for (int a = threadIdx.x; a < na; a += blockDim.x) {      // every chunk into the next slot of its size
+      int e, pos0, cnt;
+      bucket(a, e, pos0, cnt);
+      for (int n0 = 0; n0 < cnt; n0 += GM_NMAX) {
+        const int n = min(GM_NMAX, cnt - n0);
+        const int slot = atomicAdd(&s_cnt[n], 1);
+        if (slot < GM_MAX_CHUNKS)
+          plan->chunk[slot] = make_uint2(static_cast<uint32_t>(e) | 0x80000000u,
+                                         static_cast<uint32_t>(pos0 + n0) | (static_cast<uint32_t>(n) << 24));
+      }
+    }
   }
-  // gather: 8 values (16 bytes) per thread and step
+  // gather, a row per block and step (the row's source looked up once): 8
+  // values (16 bytes) per thread, all of a thread's loads of the row first
   const int w8 = H / 8;
-  const long P = routed ? static_cast<long>(T) * k : 0;
-  const long nxs = P * w8, nxh = xh ? static_cast<long>(T) * w8 : 0;
-  for (long i = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; i < nxs + nxh;
-       i += static_cast<long>(gridDim.x) * blockDim.x) {
-    long row, w;
+  const int P = routed ? T * k : 0;
+  const int nrow = P + (xh ? T : 0);
+  for (int row = blockIdx.x; row < nrow; row += gridDim.x) {
     int t;
     __half* dst;
-    if (i < nxs) {
-      row = i / w8; w = i - row * w8;
+    if (row < P) {
       const int p = pairs[row];
       t = p / k;
-      if (p < 0 || t >= T) { flag_check(CHECK_PAIR_ID); t = -1; }
-      dst = xs + row * H + 8 * w;
+      if (p < 0 || t >= T) { if (threadIdx.x == 0) flag_check(CHECK_PAIR_ID); t = -1; }
+      dst = xs + static_cast<size_t>(row) * H;
     } else {
-      const long j = i - nxs;
-      row = j / w8; w = j - row * w8;
-      t = static_cast<int>(row);
-      dst = xh + row * H + 8 * w;
+      t = row - P;
+      dst = xh + static_cast<size_t>(t) * H;
     }
-    uint4 o = make_uint4(0u, 0u, 0u, 0u);
-    if (t >= 0) {
-      const uint4 u = *reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H + 8 * w);
-      // elements e0..e7 of the block in the permuted K order e0 e4 | e1 e5 | e2 e6 | e3 e7
-      const float e0 = __uint_as_float(u.x << 16), e1 = __uint_as_float(u.x & 0xFFFF0000u);
-      const float e2 = __uint_as_float(u.y << 16), e3 = __uint_as_float(u.y & 0xFFFF0000u);
-      const float e4 = __uint_as_float(u.z << 16), e5 = __uint_as_float(u.z & 0xFFFF0000u);
-      const float e6 = __uint_as_float(u.w << 16), e7 = __uint_as_float(u.w & 0xFFFF0000u);
-      o.x = pack_half2(e0, e4);
-      o.y = pack_half2(e1, e5);
-      o.z = pack_half2(e2, e6);
-      o.w = pack_half2(e3, e7);
+    uint4 u[GM_PREP_W];
+#pragma unroll
+    for (int j = 0; j < GM_PREP_W; ++j) {
+      const int w = threadIdx.x + j * 256;
+      u[j] = (t >= 0 && w < w8) ? *reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H + 8 * w)
+                                : make_uint4(0u, 0u, 0u, 0u);
     }
-    *reinterpret_cast<uint4*>(dst) = o;
+#pragma unroll
+    for (int j = 0; j < GM_PREP_W; ++j) {
+      const int w = threadIdx.x + j * 256;
+      if (w < w8) {
+        // elements e0..e7 of the block in the permuted K order e0 e4 | e1 e5 | e2 e6 | e3 e7
+        const uint4 v = u[j];
+        const float e0 = __uint_as_float(v.x << 16), e1 = __uint_as_float(v.x & 0xFFFF0000u);
+        const float e2 = __uint_as_float(v.y << 16), e3 = __uint_as_float(v.y & 0xFFFF0000u);
+        const float e4 = __uint_as_float(v.z << 16), e5 = __uint_as_float(v.z & 0xFFFF0000u);
+        const float e6 = __uint_as_float(v.w << 16), e7 = __uint_as_float(v.w & 0xFFFF0000u);
+        uint4 o;
+        o.x = pack_half2(e0, e4);
+        o.y = pack_half2(e1, e5);
+        o.z = pack_half2(e2, e6);
+        o.w = pack_half2(e3, e7);
+        *reinterpret_cast<uint4*>(dst + 8 * w) = o;
+      }
+    }
   }
 }
 
@@ -319,6 +346,14 @@ __device__ __forceinline__ GmItem gm_item(const GemmArgs& a, int n_sh, int item)
   it.K = a.phase == 0 ? a.H : (it.seg ? a.I : a.Is);
   it.nkb = it.K / GM_BK;
   return it;
+}
+
+// The items of a launch go out in rounds of G (the grid): round r gives item
+// r G + c to CTA c in even rounds and to CTA G - 1 - c in odd ones.  With the
+// chunks sorted by size (cost) this serpentine evens out the CTAs' totals;
+// every role of a CTA walks the same sequence.
+__device__ __forceinline__ int gm_item_at(int r, int G) {
+  return r * G + ((r & 1) ? G - 1 - static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x));
 }
 
 // Matrix m (0 gate, 1 up, 2 down) of the item's expert: codes, scales, biases.
@@ -454,7 +489,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
     uint32_t rs = 0, sc_issued = 0;
     int il = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < n_items && ok; item += G, ++il) {
+    for (int rd = 0, item = gm_item_at(0, G); item < n_items && ok; item = gm_item_at(++rd, G), ++il) {
       const GmItem it = gm_item(a, n_sh, item);
       if (!gm_blob_ok(a, it)) {
         if (lane == 0) { flag_check(CHECK_EXPERT_ID); *abort_flag = 1; }
@@ -535,7 +570,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
     // ---------------------------------------------------- activation tiles
     uint32_t ss = 0;                                       // stages issued
     bool ok = true;
-    for (int item = blockIdx.x; item < n_items && ok; item += G) {
+    for (int rd = 0, item = gm_item_at(0, G); item < n_items && ok; item = gm_item_at(++rd, G)) {
       const GmItem it = gm_item(a, n_sh, item);
       const int Np = (it.N + 15) & ~15;
       int bi = 0;
@@ -569,7 +604,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
     uint32_t ss = 0;
     int il = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < n_items && ok; item += G, ++il) {
+    for (int rd = 0, item = gm_item_at(0, G); item < n_items && ok; item = gm_item_at(++rd, G), ++il) {
       const GmItem it = gm_item(a, n_sh, item);
       const int Np = (it.N + 15) & ~15;
       const int C = gm_chains(Np);
@@ -618,7 +653,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
     uint32_t ss = 0;                                     // stages (= raw slots) consumed
     int il = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < n_items && ok; item += G, ++il) {
+    for (int rd = 0, item = gm_item_at(0, G); item < n_items && ok; item = gm_item_at(++rd, G), ++il) {
       const GmItem it = gm_item(a, n_sh, item);
       const int sb = il & 1;
       if (!(ok = gm_wait(sc_full(sb), (il >> 1) & 1, abort_flag))) break;
@@ -674,7 +709,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
     // ------------------------------------------------------------- epilogue
     int il = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < n_items && ok; item += G, ++il) {
+    for (int rd = 0, item = gm_item_at(0, G); item < n_items && ok; item = gm_item_at(++rd, G), ++il) {
       const GmItem it = gm_item(a, n_sh, item);
       const int acc = il & 1;
       ok = __all_sync(0xffffffffu, gm_wait(acc_full(acc), (il >> 1) & 1, abort_flag));
