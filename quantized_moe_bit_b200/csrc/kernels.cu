@@ -34,17 +34,37 @@ __global__ void k_rmsnorm(const float* __restrict__ h, int H, float eps, uint16_
 }
 
 // --------------------------------------------------------------------- A1+A2
-// Cluster of 8 CTAs per block of ROUTER_TB rows.  CTA rank r computes the
-// logits of experts [r*E/8, (r+1)*E/8) for those rows (one warp per expert)
-// and writes them into rank 0's shared memory; after the cluster barrier
-// rank 0 selects the top k per row (one warp per row) and applies the softmax.
+// Cluster of 8 CTAs per block of ROUTER_TB rows (tokens).  CTA rank r owns
+// experts [r*E/8, (r+1)*E/8): its logits for those rows come from the tensor
+// cores (mma.sync m16n8k16, fp16 operands, fp32 accumulate) and go into rank
+// 0's shared memory; after the cluster barrier rank 0 selects the top k per
+// row (one warp per row) and applies the softmax.
 //
-// x is staged as "byte-paired" half2: word m of a row holds elements 4m..4m+3
-// as P0 = (v0, v2), P1 = (v1, v3), stored word-pair-major per 16-element
-// chunk so lane c reads consecutive bytes.  Chunk stats per 16 elements:
-// (1024 * sum of stored halves, plain sum).  Every load of a thread's batch
-// (x words; a lane's router chunks with their scale and bias) is issued
-// before any of it is used, so a warp waits one memory latency per batch.
+// Operands.  x is staged as "byte-paired" half2: word m of a chunk of 16
+// elements (elements 4m..4m+3) holds P0 = (v0, v2), P1 = (v1, v3).  A lane
+// (g, t) of an mma reads 16 code bytes of expert row g (and g+8): chunk
+// 4 grp + t of the quantisation group; in k-step j it uses the bytes of word
+// j, the even ones (1024 + b made exact fp16, minus 1024) as k-slots 2t, 2t+1
+// and the odd ones as 2t+8, 2t+9 -- the order P0 / P1 of word j of the same
+// chunk give the B fragment, so every product pairs a code with its own x
+// value.  The four k-steps of a group (64 inputs) give the exact-product fp32
+// dot d; then logit += S d + B sum(x of the group).
+// Warps split the CTA's experts in m-tiles of 16 and the groups in slices;
+// the slices' partial logits are added in slice order.
+__device__ __forceinline__ void mma_16816_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// (1024 + b) as fp16 for bytes 0 and 2 (odd = false) or 1 and 3 of w, minus 1024: exact b
+__device__ __forceinline__ uint32_t router_pair(uint32_t w, bool odd) {
+  const uint32_t h = ((odd ? w >> 8 : w) & 0x00FF00FFu) | 0x64006400u;
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&h), __floats2half2_rn(1024.f, 1024.f));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
 __global__ void __cluster_dims__(8, 1, 1) __launch_bounds__(ROUTER_THREADS)
 k_router_topk(const uint16_t* __restrict__ x, int T, int H, const uint32_t* __restrict__ rq,
               const uint16_t* __restrict__ rs, const uint16_t* __restrict__ rb,
@@ -55,20 +75,25 @@ k_router_topk(const uint16_t* __restrict__ x, int T, int H, const uint32_t* __re
   const int rank = static_cast<int>(cluster.block_rank());
   const int row0 = (blockIdx.x / 8) * ROUTER_TB;
   const int nrows = min(ROUTER_TB, T - row0);
-  const int nch = H / 16;                      // 16-element chunks (one uint4 of 8-bit codes)
-  // smem: logits [TB][E] | per row: P uint2 [nch*4] (word-major), st float2 [nch]
-  float* lg = reinterpret_cast<float*>(smem);
-  unsigned char* xs = smem + ROUTER_TB * E * sizeof(float);
-  const size_t row_bytes = static_cast<size_t>(nch) * 4 * sizeof(uint2) + nch * sizeof(float2);
+  const int nch = H / 16, NG = H / 64;
+  const RouterSmem L = router_smem_layout(H, E);
+  float* lg = reinterpret_cast<float*>(smem + L.lg);           // [TB][E] (rank 0's is the cluster's)
+  unsigned char* xs = smem + L.xs;                             // per row: P uint2 [4][nch]
+  float* xg = reinterpret_cast<float*>(smem + L.xg);           // [TB][NG] group sums of the staged x
+  float* part = reinterpret_cast<float*>(smem + L.part);       // [8 warps][TB][16] partial logits
+  const size_t row_bytes = L.row_bytes;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+  const int nwarp = blockDim.x >> 5;
 
-  // stage x rows, ROUTER_XB items per thread per batch
-  const int nitems = nrows * nch;
+  // stage x rows (zeros past the last row), ROUTER_XB chunks per thread per batch
+  const int nitems = ROUTER_TB * nch;
   for (int i0 = threadIdx.x; i0 < nitems; i0 += blockDim.x * ROUTER_XB) {
     uint4 u[ROUTER_XB][2];
 #pragma unroll
     for (int j = 0; j < ROUTER_XB; ++j) {
       const int i = i0 + j * static_cast<int>(blockDim.x);
-      if (i < nitems) {
+      u[j][0] = u[j][1] = make_uint4(0u, 0u, 0u, 0u);
+      if (i < nitems && i / nch < nrows) {
         const int r = i / nch, c = i - r * nch;
         const uint16_t* src = x + static_cast<size_t>(row0 + r) * H + 16 * c;
         u[j][0] = *reinterpret_cast<const uint4*>(src);
@@ -78,11 +103,10 @@ k_router_topk(const uint16_t* __restrict__ x, int T, int H, const uint32_t* __re
 #pragma unroll
     for (int j = 0; j < ROUTER_XB; ++j) {
       const int i = i0 + j * static_cast<int>(blockDim.x);
+      float sum = 0.f;
       if (i < nitems) {
         const int r = i / nch, c = i - r * nch;
         uint2* P = reinterpret_cast<uint2*>(xs + r * row_bytes);
-        float2* st = reinterpret_cast<float2*>(xs + r * row_bytes + static_cast<size_t>(nch) * 4 * sizeof(uint2));
-        float off = 0.f;
         const uint32_t w[8] = {u[j][0].x, u[j][0].y, u[j][0].z, u[j][0].w, u[j][1].x, u[j][1].y, u[j][1].z, u[j][1].w};
 #pragma unroll
         for (int m = 0; m < 4; ++m) {          // word m covers elements 4m..4m+3
@@ -91,68 +115,109 @@ k_router_topk(const uint16_t* __restrict__ x, int T, int H, const uint32_t* __re
           const uint32_t p0 = pack_half2(v0, v2), p1 = pack_half2(v1, v3);
           P[m * nch + c] = make_uint2(p0, p1);
           const float2 f0 = unpack_half2(p0), f1 = unpack_half2(p1);
-          off += (f0.x + f0.y) + (f1.x + f1.y);
+          sum += (f0.x + f0.y) + (f1.x + f1.y);
         }
-        st[c] = make_float2(1024.f * off, off);
       }
+      // a group's four chunks are items 4q .. 4q+3 of a row (nch % 4 == 0),
+      // held by four consecutive lanes: their sums meet in the first
+      sum += __shfl_down_sync(0xffffffffu, sum, 1);
+      sum += __shfl_down_sync(0xffffffffu, sum, 2);
+      if (i < nitems && (i % nch) % 4 == 0) xg[(i / nch) * NG + (i % nch) / 4] = sum;
     }
   }
   __syncthreads();
 
-  float* lg0 = cluster.map_shared_rank(lg, 0);
+  // this warp: m-tile mt of the CTA's experts, group slice ks
   const int epc = E / 8;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarp = blockDim.x >> 5;
-  const int hb = H / 4;                       // bytes... words per router row
-  for (int el = warp; el < epc; el += nwarp) {
-    const int e = rank * epc + el;
-    const uint8_t* qrow = reinterpret_cast<const uint8_t*>(rq + static_cast<size_t>(e) * hb);
-    float acc[ROUTER_TB];
+  const int nmt = (epc + 15) / 16, nks = 8 / nmt;
+  const int mt = warp % nmt, ks = warp / nmt;
+  if (ks < nks) {
+    const int g0 = ks * NG / nks, g1 = (ks + 1) * NG / nks;
+    const int ea = mt * 16 + gq, eb = ea + 8;               // the lane's two experts (CTA-local)
+    const bool oka = ea < epc, okb = eb < epc;
+    const int Ea = rank * epc + ea, Eb = rank * epc + eb;
+    const uint8_t* qa = reinterpret_cast<const uint8_t*>(rq) + static_cast<size_t>(oka ? Ea : 0) * H + 16 * tq;
+    const uint8_t* qb = reinterpret_cast<const uint8_t*>(rq) + static_cast<size_t>(okb ? Eb : 0) * H + 16 * tq;
+    const uint16_t* sa = rs + static_cast<size_t>(oka ? Ea : 0) * NG;
+    const uint16_t* ba = rb + static_cast<size_t>(oka ? Ea : 0) * NG;
+    const uint16_t* sb = rs + static_cast<size_t>(okb ? Eb : 0) * NG;
+    const uint16_t* bb = rb + static_cast<size_t>(okb ? Eb : 0) * NG;
+    float acc[2][4];
 #pragma unroll
-    for (int r = 0; r < ROUTER_TB; ++r) acc[r] = 0.f;
-    // the lane's chunks c = lane, lane + 32, ... in order, ROUTER_CB at a time
-    for (int c0 = lane; c0 < nch; c0 += 32 * ROUTER_CB) {
-      uint4 q[ROUTER_CB];
-      float sc[ROUTER_CB], bi[ROUTER_CB];
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int b = 0; b < ROUTER_CB; ++b) {
-        const int c = c0 + 32 * b;
-        if (c < nch) {
-          q[b] = ldg_nc_v4(qrow + static_cast<size_t>(c) * 16);
-          sc[b] = bf16_to_f32(ldg_u16(rs + static_cast<size_t>(e) * (H / 64) + (c >> 2)));
-          bi[b] = bf16_to_f32(ldg_u16(rb + static_cast<size_t>(e) * (H / 64) + (c >> 2)));
+      for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
+    for (int gb = g0; gb < g1; gb += ROUTER_GB) {
+      uint4 wa[ROUTER_GB], wb[ROUTER_GB];
+      float s4[ROUTER_GB][4];
+#pragma unroll
+      for (int u = 0; u < ROUTER_GB; ++u) {     // the batch's codes and scales first
+        const int g = gb + u;
+        if (g < g1) {
+          wa[u] = oka ? ldg_nc_v4(qa + 64 * static_cast<size_t>(g)) : make_uint4(0u, 0u, 0u, 0u);
+          wb[u] = okb ? ldg_nc_v4(qb + 64 * static_cast<size_t>(g)) : make_uint4(0u, 0u, 0u, 0u);
+          s4[u][0] = oka ? bf16_to_f32(ldg_u16(sa + g)) : 0.f;
+          s4[u][1] = oka ? bf16_to_f32(ldg_u16(ba + g)) : 0.f;
+          s4[u][2] = okb ? bf16_to_f32(ldg_u16(sb + g)) : 0.f;
+          s4[u][3] = okb ? bf16_to_f32(ldg_u16(bb + g)) : 0.f;
         }
       }
 #pragma unroll
-      for (int b = 0; b < ROUTER_CB; ++b) {
-        const int c = c0 + 32 * b;
-        if (c < nch) {
+      for (int u = 0; u < ROUTER_GB; ++u) {
+        const int g = gb + u;
+        if (g < g1) {
+          float d[2][4];
 #pragma unroll
-          for (int r = 0; r < ROUTER_TB; ++r) {
-            if (r < nrows) {
-              const uint2* P = reinterpret_cast<const uint2*>(xs + r * row_bytes);
-              const float2* st =
-                  reinterpret_cast<const float2*>(xs + r * row_bytes + static_cast<size_t>(nch) * 4 * sizeof(uint2));
-              float a0 = 0.f, a1 = 0.f;
-              uint2 p;
-              p = P[0 * nch + c]; { uint32_t pp[2] = {p.x, p.y}; dot_word8(q[b].x, pp, a0, a1); }
-              p = P[1 * nch + c]; { uint32_t pp[2] = {p.x, p.y}; dot_word8(q[b].y, pp, a0, a1); }
-              p = P[2 * nch + c]; { uint32_t pp[2] = {p.x, p.y}; dot_word8(q[b].z, pp, a0, a1); }
-              p = P[3 * nch + c]; { uint32_t pp[2] = {p.x, p.y}; dot_word8(q[b].w, pp, a0, a1); }
-              const float2 s2 = st[c];
-              acc[r] += sc[b] * ((a0 + a1) - s2.x) + bi[b] * s2.y;
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d[nt][i] = 0.f;
+          const uint32_t qwa[4] = {wa[u].x, wa[u].y, wa[u].z, wa[u].w};
+          const uint32_t qwb[4] = {wb[u].x, wb[u].y, wb[u].z, wb[u].w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t af[4] = {router_pair(qwa[j], false), router_pair(qwb[j], false),
+                                    router_pair(qwa[j], true), router_pair(qwb[j], true)};
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+              const uint2 P = reinterpret_cast<const uint2*>(xs + (nt * 8 + gq) * row_bytes)[j * nch + 4 * g + tq];
+              mma_16816_f16(d[nt], af, P.x, P.y);
             }
+          }
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const float xa = xg[(nt * 8 + 2 * tq) * NG + g], xb = xg[(nt * 8 + 2 * tq + 1) * NG + g];
+            acc[nt][0] += s4[u][0] * d[nt][0] + s4[u][1] * xa;
+            acc[nt][1] += s4[u][0] * d[nt][1] + s4[u][1] * xb;
+            acc[nt][2] += s4[u][2] * d[nt][2] + s4[u][3] * xa;
+            acc[nt][3] += s4[u][2] * d[nt][3] + s4[u][3] * xb;
           }
         }
       }
     }
+    // partial logits of (row, expert) into the warp's slot
+    float* pw = part + warp * (ROUTER_TB * 16);
 #pragma unroll
-    for (int r = 0; r < ROUTER_TB; ++r) {
-      const float v = warp_sum(acc[r]);
-      if (lane == 0 && r < nrows) {
-        float bb = 0.f;
-        if (bias != nullptr) bb = bias_per_row ? bias[static_cast<size_t>(row0 + r) * E + e] : bias[e];
-        lg0[r * E + e] = v + bb;
-      }
+    for (int nt = 0; nt < 2; ++nt) {
+      const int ra = nt * 8 + 2 * tq;
+      pw[ra * 16 + gq] = acc[nt][0];
+      pw[(ra + 1) * 16 + gq] = acc[nt][1];
+      pw[ra * 16 + gq + 8] = acc[nt][2];
+      pw[(ra + 1) * 16 + gq + 8] = acc[nt][3];
+    }
+  }
+  __syncthreads();
+  // the slices' sums, in slice order, plus the bias, into rank 0's logits
+  float* lg0 = cluster.map_shared_rank(lg, 0);
+  for (int i = threadIdx.x; i < nmt * ROUTER_TB * 16; i += blockDim.x) {
+    const int m = i / (ROUTER_TB * 16), rem = i - m * (ROUTER_TB * 16), r = rem / 16, el = rem % 16;
+    const int e_loc = m * 16 + el;
+    if (r < nrows && e_loc < epc) {
+      float v = 0.f;
+      for (int q = 0; q < nks; ++q) v += part[(q * nmt + m) * (ROUTER_TB * 16) + r * 16 + el];
+      const int e = rank * epc + e_loc;
+      float bbv = 0.f;
+      if (bias != nullptr) bbv = bias_per_row ? bias[static_cast<size_t>(row0 + r) * E + e] : bias[e];
+      lg0[r * E + e] = v + bbv;
     }
   }
   cluster.sync();

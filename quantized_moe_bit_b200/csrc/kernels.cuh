@@ -4,10 +4,10 @@
 
 namespace moe {
 
-constexpr int ROUTER_TB = 8;     // rows per router cluster
-constexpr int ROUTER_THREADS = 512;   // threads per router CTA (one warp per expert of the CTA's E/8)
+constexpr int ROUTER_TB = 16;    // rows per router cluster (two mma n-tiles)
+constexpr int ROUTER_THREADS = 256;   // 8 warps: m-tiles of 16 experts x slices of the groups
 constexpr int ROUTER_XB = 4;     // x chunks a router thread loads before staging them
-constexpr int ROUTER_CB = 8;     // router chunks a lane loads before using them
+constexpr int ROUTER_GB = 3;     // groups of codes and scales a router lane loads before using them
 constexpr int BUCKET_THREADS = 512;   // one block; each warp buckets a contiguous run of pairs
 constexpr int BUCKET_B = 8;      // chunks of 32 pair indices a bucket warp loads at once
 constexpr int GEMV_RG = 4;       // bucket rows staged at once by the GEMV kernels
@@ -57,10 +57,24 @@ __global__ void k_combine(const float* yp, const float* gates, const float* ysh,
 __global__ void k_combine4(const float* yp, const float* gates, const float* ysh, int H, int k,
                            uint16_t* y, float* resid);
 
-inline size_t router_smem_bytes(int H, int E) {
-  const int nch = H / 16;
-  return ROUTER_TB * E * sizeof(float) +
-         ROUTER_TB * (static_cast<size_t>(nch) * 4 * 8 + nch * 8);
+// Shared memory of the router kernel: logits [TB][E] | staged x, per row the
+// byte-paired words [4][H/16] (rows 32 bytes apart modulo 128, so the eight
+// rows an mma reads fall in distinct banks) | group sums [TB][H/64] |
+// partial logits [8 warps][TB][16].
+struct RouterSmem {
+  size_t lg, xs, row_bytes, xg, part, total;
+};
+__host__ __device__ inline RouterSmem router_smem_layout(int H, int E) {
+  RouterSmem L;
+  const size_t nch = static_cast<size_t>(H) / 16;
+  L.lg = 0;
+  L.xs = (static_cast<size_t>(ROUTER_TB) * E * sizeof(float) + 127) & ~size_t(127);
+  L.row_bytes = nch * 4 * 8 + 32;
+  L.xg = L.xs + ROUTER_TB * L.row_bytes;
+  L.part = (L.xg + static_cast<size_t>(ROUTER_TB) * (H / 64) * sizeof(float) + 15) & ~size_t(15);
+  L.total = L.part + static_cast<size_t>(ROUTER_THREADS / 32) * ROUTER_TB * 16 * sizeof(float);
+  return L;
 }
+inline size_t router_smem_bytes(int H, int E) { return router_smem_layout(H, E).total; }
 
 }  // namespace moe
