@@ -77,6 +77,7 @@ k_router_topk(const uint16_t* __restrict__ x, int T, int H, const uint32_t* __re
   const int nrows = min(ROUTER_TB, T - row0);
   const int nch = H / 16, NG = H / 64;
   const RouterSmem L = router_smem_layout(H, E);
+  cluster.barrier_arrive();       // waited on before the first write into rank 0's shared memory
   float* lg = reinterpret_cast<float*>(smem + L.lg);           // [TB][E] (rank 0's is the cluster's)
   unsigned char* xs = smem + L.xs;                             // per row: P uint2 [4][nch]
   float* xg = reinterpret_cast<float*>(smem + L.xg);           // [TB][NG] group sums of the staged x
@@ -84,6 +85,39 @@ k_router_topk(const uint16_t* __restrict__ x, int T, int H, const uint32_t* __re
   const size_t row_bytes = L.row_bytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
   const int nwarp = blockDim.x >> 5;
+
+  // this warp: m-tile mt of the CTA's experts, group slice ks; its first
+  // batch of codes and scales is requested before x is staged
+  const int epc = E / 8;
+  const int nmt = (epc + 15) / 16, nks = (ROUTER_THREADS / 32) / nmt;
+  const int mt = warp % nmt, ks = warp / nmt;
+  const bool active_w = ks < nks;
+  const int g0 = active_w ? ks * NG / nks : 0, g1 = active_w ? (ks + 1) * NG / nks : 0;
+  const int ea = mt * 16 + gq, eb = ea + 8;               // the lane's two experts (CTA-local)
+  const bool oka = ea < epc, okb = eb < epc;
+  const int Ea = rank * epc + ea, Eb = rank * epc + eb;
+  const uint8_t* qa = reinterpret_cast<const uint8_t*>(rq) + static_cast<size_t>(oka ? Ea : 0) * H + 16 * tq;
+  const uint8_t* qb = reinterpret_cast<const uint8_t*>(rq) + static_cast<size_t>(okb ? Eb : 0) * H + 16 * tq;
+  const uint16_t* sa = rs + static_cast<size_t>(oka ? Ea : 0) * NG;
+  const uint16_t* ba = rb + static_cast<size_t>(oka ? Ea : 0) * NG;
+  const uint16_t* sb = rs + static_cast<size_t>(okb ? Eb : 0) * NG;
+  const uint16_t* bb = rb + static_cast<size_t>(okb ? Eb : 0) * NG;
+  uint4 wa[ROUTER_GB], wb[ROUTER_GB];
+  float s4[ROUTER_GB][4];
+  auto load_batch = [&](int gb) {
+#pragma unroll
+    for (int u = 0; u < ROUTER_GB; ++u) {
+      const int g = gb + u;
+      const bool in = g < g1;
+      wa[u] = (in && oka) ? ldg_nc_v4(qa + 64 * static_cast<size_t>(g)) : make_uint4(0u, 0u, 0u, 0u);
+      wb[u] = (in && okb) ? ldg_nc_v4(qb + 64 * static_cast<size_t>(g)) : make_uint4(0u, 0u, 0u, 0u);
+      s4[u][0] = (in && oka) ? bf16_to_f32(ldg_u16(sa + g)) : 0.f;
+      s4[u][1] = (in && oka) ? bf16_to_f32(ldg_u16(ba + g)) : 0.f;
+      s4[u][2] = (in && okb) ? bf16_to_f32(ldg_u16(sb + g)) : 0.f;
+      s4[u][3] = (in && okb) ? bf16_to_f32(ldg_u16(bb + g)) : 0.f;
+    }
+  };
+  load_batch(g0);
 
   // stage x rows (zeros past the last row), ROUTER_XB chunks per thread per batch
   const int nitems = ROUTER_TB * nch;
@@ -127,41 +161,14 @@ k_router_topk(const uint16_t* __restrict__ x, int T, int H, const uint32_t* __re
   }
   __syncthreads();
 
-  // this warp: m-tile mt of the CTA's experts, group slice ks
-  const int epc = E / 8;
-  const int nmt = (epc + 15) / 16, nks = 8 / nmt;
-  const int mt = warp % nmt, ks = warp / nmt;
-  if (ks < nks) {
-    const int g0 = ks * NG / nks, g1 = (ks + 1) * NG / nks;
-    const int ea = mt * 16 + gq, eb = ea + 8;               // the lane's two experts (CTA-local)
-    const bool oka = ea < epc, okb = eb < epc;
-    const int Ea = rank * epc + ea, Eb = rank * epc + eb;
-    const uint8_t* qa = reinterpret_cast<const uint8_t*>(rq) + static_cast<size_t>(oka ? Ea : 0) * H + 16 * tq;
-    const uint8_t* qb = reinterpret_cast<const uint8_t*>(rq) + static_cast<size_t>(okb ? Eb : 0) * H + 16 * tq;
-    const uint16_t* sa = rs + static_cast<size_t>(oka ? Ea : 0) * NG;
-    const uint16_t* ba = rb + static_cast<size_t>(oka ? Ea : 0) * NG;
-    const uint16_t* sb = rs + static_cast<size_t>(okb ? Eb : 0) * NG;
-    const uint16_t* bb = rb + static_cast<size_t>(okb ? Eb : 0) * NG;
+  if (active_w) {
     float acc[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
     for (int gb = g0; gb < g1; gb += ROUTER_GB) {
-      uint4 wa[ROUTER_GB], wb[ROUTER_GB];
-      float s4[ROUTER_GB][4];
-#pragma unroll
-      for (int u = 0; u < ROUTER_GB; ++u) {     // the batch's codes and scales first
-        const int g = gb + u;
-        if (g < g1) {
-          wa[u] = oka ? ldg_nc_v4(qa + 64 * static_cast<size_t>(g)) : make_uint4(0u, 0u, 0u, 0u);
-          wb[u] = okb ? ldg_nc_v4(qb + 64 * static_cast<size_t>(g)) : make_uint4(0u, 0u, 0u, 0u);
-          s4[u][0] = oka ? bf16_to_f32(ldg_u16(sa + g)) : 0.f;
-          s4[u][1] = oka ? bf16_to_f32(ldg_u16(ba + g)) : 0.f;
-          s4[u][2] = okb ? bf16_to_f32(ldg_u16(sb + g)) : 0.f;
-          s4[u][3] = okb ? bf16_to_f32(ldg_u16(bb + g)) : 0.f;
-        }
-      }
+      if (gb != g0) load_batch(gb);            // the first batch came before the staging
 #pragma unroll
       for (int u = 0; u < ROUTER_GB; ++u) {
         const int g = gb + u;
@@ -207,6 +214,8 @@ k_router_topk(const uint16_t* __restrict__ x, int T, int H, const uint32_t* __re
   }
   __syncthreads();
   // the slices' sums, in slice order, plus the bias, into rank 0's logits
+  // (every CTA of the cluster has started: the arrive above)
+  cluster.barrier_wait();
   float* lg0 = cluster.map_shared_rank(lg, 0);
   for (int i = threadIdx.x; i < nmt * ROUTER_TB * 16; i += blockDim.x) {
     const int m = i / (ROUTER_TB * 16), rem = i - m * (ROUTER_TB * 16), r = rem / 16, el = rem % 16;

@@ -5,8 +5,8 @@
 namespace moe {
 
 constexpr int ROUTER_TB = 16;    // rows per router cluster (two mma n-tiles)
-constexpr int ROUTER_THREADS = 256;   // 8 warps: m-tiles of 16 experts x slices of the groups
-constexpr int ROUTER_XB = 4;     // x chunks a router thread loads before staging them
+constexpr int ROUTER_THREADS = 512;   // 16 warps: m-tiles of 16 experts x slices of the groups
+constexpr int ROUTER_XB = 6;     // x chunks a router thread loads before staging them
 constexpr int ROUTER_GB = 3;     // groups of codes and scales a router lane loads before using them
 constexpr int BUCKET_THREADS = 512;   // one block; each warp buckets a contiguous run of pairs
 constexpr int BUCKET_B = 8;      // chunks of 32 pair indices a bucket warp loads at once
@@ -60,7 +60,7 @@ __global__ void k_combine4(const float* yp, const float* gates, const float* ysh
 // Shared memory of the router kernel: logits [TB][E] | staged x, per row the
 // byte-paired words [4][H/16] (rows 32 bytes apart modulo 128, so the eight
 // rows an mma reads fall in distinct banks) | group sums [TB][H/64] |
-// partial logits [8 warps][TB][16].
+// partial logits [ROUTER_THREADS / 32 warps][TB][16].
 struct RouterSmem {
   size_t lg, xs, row_bytes, xg, part, total;
 };
