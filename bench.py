@@ -55,7 +55,7 @@ def peaks():
 # DRAM read + write of the decode kernel measured by ncu on 3 full-size
 # layers of this workload, per layer; valid only for the kernel source the
 # capture was taken on (sha256 prefix of decode_fused.cu).
-DECODE_TRAFFIC = {"source_sha256_prefix": "c5c566c3e0dbf8e3", "bytes_per_layer": 38.7148e6}
+DECODE_TRAFFIC = {"source_sha256_prefix": "c5c566c3e0dbf8e3", "bytes_per_layer": 38.9716e6}
 
 
 def decode_traffic(layers: int):
@@ -278,7 +278,10 @@ def run_streamed_lfu(M, device):
     then 128 decode steps, routed experts in pinned host memory, 16 HBM slots
     per layer (misses copied host -> device on a side stream while the shared
     expert runs).  Prefill and decode timed separately (CUDA events; the LFU
-    plan of every layer step needs the routing on the host)."""
+    plan of every layer step needs the routing on the host).  A/B of the
+    lookahead prefetch: off and on (2 experts per layer call), each on a fresh
+    cache, alternately twice; the top-level figures are the first run with
+    the prefetch off."""
     import torch
     from quantized_moe_bit_b200.weights import blob_table, upload_qmat
     c = gen.CONFIGS["streamed_30L_lfu"]
@@ -310,33 +313,45 @@ def run_streamed_lfu(M, device):
     for l in range(c.layers):                   # biases built before the timed region
         for z, t0 in units:
             bias(l, t0, z.shape[0])
-    lfu = M.MoeLfu(c.layers, c.E, c.n_slots, gen.blob_bytes(c.H, c.I), host_ptrs, pool, stride)
     side = torch.cuda.Stream(device=device)
     main = torch.cuda.current_stream()
     ws = {T: torch.empty(M.moe_streamed_workspace_size(T, c.H, c.I, c.Is, c.E, c.k), dtype=torch.uint8,
                          device=device) for T in (c.T, 1)}
-
-    def run(us):
-        for z, t0 in us:
-            T = z.shape[0]
-            h = z.clone()
-            for l in range(c.layers):
-                M.moe_streamed_layer_forward(lfu, l, h, c.I, c.Is, c.E, c.k, routers[l].c, bias(l, t0, T), 1,
-                                             [m.c for m in shared[l]], tables[l], ws[T], main_stream=main,
-                                             side_stream=side)
     n_pre = c.prompt_tokens // c.T
-    torch.cuda.synchronize()
-    e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-    e0.record()
-    run(units[:n_pre])
-    e1.record()
-    run(units[n_pre:])
-    e2.record()
-    torch.cuda.synchronize()
-    M.moe_sync()
-    t_pre, t_dec = e0.elapsed_time(e1) / 1e3, e1.elapsed_time(e2) / 1e3
-    hits, misses, nbytes = lfu.stats()
-    lfu.close()
+
+    def arm(prefetch: int):
+        """One run of the workload on a fresh cache (lookahead prefetch of
+        `prefetch` experts per layer call, 0: off)."""
+        lfu = M.MoeLfu(c.layers, c.E, c.n_slots, gen.blob_bytes(c.H, c.I), host_ptrs, pool, stride)
+        lfu.set_prefetch(prefetch)
+
+        def run(us):
+            for z, t0 in us:
+                T = z.shape[0]
+                h = z.clone()
+                for l in range(c.layers):
+                    M.moe_streamed_layer_forward(lfu, l, h, c.I, c.Is, c.E, c.k, routers[l].c, bias(l, t0, T), 1,
+                                                 [m.c for m in shared[l]], tables[l], ws[T], main_stream=main,
+                                                 side_stream=side)
+        torch.cuda.synchronize()
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record()
+        run(units[:n_pre])
+        e1.record()
+        run(units[n_pre:])
+        e2.record()
+        torch.cuda.synchronize()
+        M.moe_sync()
+        t_pre, t_dec = e0.elapsed_time(e1) / 1e3, e1.elapsed_time(e2) / 1e3
+        hits, misses, nbytes = lfu.stats()
+        staged = sum(1 for r in lfu.log() if r[3] == 2)
+        lfu.close()
+        return {"prefetch_per_call": prefetch, "prefill_tokens_per_s": c.prompt_tokens / t_pre,
+                "decode_tokens_per_s": c.decode_steps / t_dec, "prefill_s": t_pre, "decode_s": t_dec,
+                "hits": hits, "misses": misses, "prefetched": staged, "h2d_bytes": nbytes,
+                "h2d_gbs_while_streaming": nbytes / (t_pre + t_dec) / 1e9}
+    runs = [arm(p) for p in (0, 2, 0, 2)]           # the two arms alternately, twice
+    base = runs[0]
     # pinned host -> device copy bandwidth of this box, for context
     buf = host.view(-1)[: 256 << 20]
     dst = torch.empty(buf.numel(), dtype=torch.uint8, device=device)
@@ -348,11 +363,10 @@ def run_streamed_lfu(M, device):
     e4.record()
     torch.cuda.synchronize()
     h2d = buf.numel() / (e3.elapsed_time(e4) / 1e3) / 1e9
-    return {"workload": "streamed_30L_lfu", "prefill_tokens_per_s": c.prompt_tokens / t_pre,
-            "decode_tokens_per_s": c.decode_steps / t_dec, "prefill_s": t_pre, "decode_s": t_dec,
-            "hits": hits, "misses": misses, "h2d_bytes": nbytes,
-            "h2d_gbs_while_streaming": nbytes / (t_pre + t_dec) / 1e9, "pinned_h2d_copy_gbs": h2d,
-            "slots_per_layer": c.n_slots,
+    return {"workload": "streamed_30L_lfu", **{k: base[k] for k in base if k != "prefetch_per_call"},
+            "pinned_h2d_copy_gbs": h2d, "slots_per_layer": c.n_slots,
+            "prefetch_ab": {"arms": "lookahead prefetch off (0) and on (2 experts per layer call), run alternately",
+                            "runs": runs},
             "note": "bitwise equality with the all-resident run and the LFU log are checked by the GPU tests"}
 
 

@@ -361,6 +361,23 @@ MOE_API int moe_lfu_stats(moe_lfu* h, int64_t* hits, int64_t* misses, int64_t* b
 /* Test hook: after `after_n` copies, every further copy fails before it is
  * issued (kind 1) or is delayed by 50 ms on the host (kind 2); kind 0 clears it. */
 MOE_API int moe_lfu_set_fault(moe_lfu* h, int kind, int after_n);
+/* Lookahead prefetch (f2; off by default): after each moe_streamed_layer_forward
+ * call on a layer, stage up to per_call (0 .. n_slots) experts of that layer
+ * ahead of their next use -- the non-resident experts accessed most often so
+ * far in the run (ties to the lower id), each into the slot a miss would
+ * take, only while that slot is empty or its resident's count is below the
+ * candidate's access total; a prefetched expert enters with count 0, is one
+ * more step of the layer and is logged with hit = 2 (moe_lfu_stats counts
+ * such records neither as hits nor as misses).  The copies follow the
+ * call's expert kernels on the side stream and belong to the call's
+ * transaction.  The pages report speculative expert reads as measured and
+ * rejected: "TurboFieldfareとは｜…の実像" (ai-heartland.com), section
+ * "103件の実験記録が教える「効いたのに採用しなかった最適化」".
+ * moe_lfu_plan_prefetch plans one such prefetch without copying (state and
+ * log updated; ids_out / slots_out of capacity per_call; *n_out = count). */
+MOE_API int moe_lfu_set_prefetch(moe_lfu* h, int per_call);
+MOE_API int moe_lfu_plan_prefetch(moe_lfu* h, int layer, int per_call, int32_t* ids_out, int32_t* slots_out,
+                                  int* n_out);
 MOE_API int moe_lfu_destroy(moe_lfu* h);
 
 /* One routed-MoE layer whose routed experts are streamed through the LFU

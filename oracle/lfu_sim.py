@@ -22,6 +22,16 @@ more than that; the policy below is this library's reading of it:
 
 Every access is logged as (layer, step, expert, hit, slot); `step` counts
 the steps of that layer from 0.
+
+Lookahead prefetch (an option of this library, not of the pages, which
+report speculative reads as tried and rejected): `prefetch(layer, P)` stages
+up to P experts of a layer -- the non-resident ones with the most accesses so
+far in the run (hits and misses; ties to the lower id), each into the slot a
+miss would take (the victim rule above, slots taken by this prefetch
+excluded), stopping at the first candidate whose victim slot holds an expert
+with count >= the candidate's access total.  A prefetched expert enters with
+count 0 and the tick advances; the prefetch is one more step of the layer
+and each staged expert is logged with hit = 2.
 """
 from __future__ import annotations
 
@@ -35,6 +45,7 @@ class LFUSim:
         self.steps = [0] * n_layers
         self.tick = 0
         self.log = []
+        self.freq = [dict() for _ in range(n_layers)]   # accesses per expert over the run
 
     def resident(self, layer: int):
         return {e for e in self.expert[layer] if e >= 0}
@@ -56,6 +67,8 @@ class LFUSim:
         where = {}
         hits = [e for e in ids if self.slot_of(layer, e) >= 0]
         misses = [e for e in ids if self.slot_of(layer, e) < 0]
+        for e in hits + misses:
+            self.freq[layer][e] = self.freq[layer].get(e, 0) + 1
         for e in hits:
             s = self.slot_of(layer, e)
             self.tick += 1
@@ -88,6 +101,31 @@ class LFUSim:
             if best is None or key < best:
                 best = key
         return best[2]
+
+    def prefetch(self, layer: int, P: int):
+        """One lookahead prefetch of up to P experts; returns [(expert, slot)]."""
+        if P <= 0:
+            return []
+        res = self.resident(layer)
+        fr = self.freq[layer]
+        cand = sorted((e for e in fr if fr[e] > 0 and e not in res), key=lambda e: (-fr[e], e))
+        st = self.steps[layer]
+        self.steps[layer] += 1
+        used, out = set(), []
+        for e in cand:
+            if len(out) == P:
+                break
+            s = self._victim(layer, used)
+            if self.expert[layer][s] >= 0 and self.count[layer][s] >= fr[e]:
+                break
+            self.tick += 1
+            self.expert[layer][s] = e
+            self.count[layer][s] = 0
+            self.last[layer][s] = self.tick
+            used.add(s)
+            out.append((e, s))
+            self.log.append((layer, st, e, 2, s))
+        return out
 
     def chunk_steps(self, layer: int, distinct, width: int):
         """Order a chunk's distinct experts into steps (resident first)."""

@@ -66,6 +66,8 @@ SIGNATURES = {
     "moe_lfu_get_log": (_I, [_P, _P, _Z, C.POINTER(C.c_size_t)]),
     "moe_lfu_stats": (_I, [_P, C.POINTER(C.c_int64), C.POINTER(C.c_int64), C.POINTER(C.c_int64)]),
     "moe_lfu_set_fault": (_I, [_P, _I, _I]),
+    "moe_lfu_set_prefetch": (_I, [_P, _I]),
+    "moe_lfu_plan_prefetch": (_I, [_P, _I, _I, _P, _P, C.POINTER(C.c_int)]),
     "moe_lfu_destroy": (_I, [_P]),
     "moe_streamed_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
     "moe_streamed_layer_forward": (_I, [_P, _I, _P, _I, _I, _I, _I, _I, _I, C.POINTER(moe_qmat), _P, _I,

@@ -191,6 +191,16 @@ class MoeLfu:
     def set_fault(self, kind: int, after_n: int):
         check(lib().moe_lfu_set_fault(self._h, kind, after_n))
 
+    def set_prefetch(self, per_call: int):
+        check(lib().moe_lfu_set_prefetch(self._h, per_call))
+
+    def plan_prefetch(self, layer: int, per_call: int):
+        ids = (C.c_int32 * max(per_call, 1))()
+        slots = (C.c_int32 * max(per_call, 1))()
+        n = C.c_int()
+        check(lib().moe_lfu_plan_prefetch(self._h, layer, per_call, ids, slots, C.byref(n)))
+        return list(ids)[:n.value], list(slots)[:n.value]
+
     def close(self):
         if self._h:
             lib().moe_lfu_destroy(self._h)

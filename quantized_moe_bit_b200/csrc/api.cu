@@ -478,20 +478,27 @@ int moe_shared_forward(const uint16_t* x, int T, int H, int Is, const moe_qmat* 
   return run_gemm(x, T, H, nullptr, &si, w.plan, nullptr, nullptr, nullptr, w.act, w.xh, s);
 }
 
+// The combine with the residual add read from resid_in and written to
+// resid_out (the same array for the in-place form).
+static int launch_combine(const float* y_pairs, const float* gates, const float* ysh, int T, int H, int k, uint16_t* y,
+                          const float* resid_in, float* resid_out, cudaStream_t cs) {
+  const bool vec = H % 4 == 0 && aligned16(y_pairs) && (!ysh || aligned16(ysh)) &&
+                   (!resid_out || (aligned16(resid_out) && aligned16(resid_in))) && (reinterpret_cast<uintptr_t>(y) & 7) == 0;
+  if (vec) {
+    k_combine4<<<dim3((H / 4 + 255) / 256, T), 256, 0, cs>>>(y_pairs, gates, ysh, H, k, y, resid_in, resid_out);
+    return launch_check("k_combine4");
+  }
+  k_combine<<<dim3((H + 255) / 256, T), 256, 0, cs>>>(y_pairs, gates, ysh, H, k, y, resid_in, resid_out);
+  return launch_check("k_combine");
+}
+
 int moe_combine(const float* y_pairs, const float* gates, const float* ysh, int T, int H, int k, uint16_t* y,
                 float* residual_inout, void* stream) {
   if (T < 0 || H <= 0 || k < 1 || k > 8) return fail(MOE_ERR_INVALID_ARG, "moe_combine: bad T/H/k");
   if (T == 0) return MOE_OK;
   if (!y_pairs || !gates) return fail(MOE_ERR_INVALID_ARG, "moe_combine: NULL pointer");
-  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  const bool vec = H % 4 == 0 && aligned16(y_pairs) && (!ysh || aligned16(ysh)) && (!residual_inout || aligned16(residual_inout)) &&
-                   (reinterpret_cast<uintptr_t>(y) & 7) == 0;
-  if (vec) {
-    k_combine4<<<dim3((H / 4 + 255) / 256, T), 256, 0, cs>>>(y_pairs, gates, ysh, H, k, y, residual_inout);
-    return launch_check("k_combine4");
-  }
-  k_combine<<<dim3((H + 255) / 256, T), 256, 0, cs>>>(y_pairs, gates, ysh, H, k, y, residual_inout);
-  return launch_check("k_combine");
+  return launch_combine(y_pairs, gates, ysh, T, H, k, y, residual_inout, residual_inout,
+                        static_cast<cudaStream_t>(stream));
 }
 
 // Workspace of one layer: routing buffers, y_pairs, ysh, then the expert and
@@ -583,15 +590,8 @@ int moe_layer_forward(const float* h_in, float* h_out, const uint16_t* x_in, int
                                  w.ew, w.ews, flags, stream)))
       return st;
   }
-  float* resid = nullptr;
-  if (h_out) {
-    if (h_out != h_in &&
-        (st = cuda_check(cudaMemcpyAsync(h_out, h_in, static_cast<size_t>(T) * H * 4, cudaMemcpyDeviceToDevice, s),
-                         "copy h")))
-      return st;
-    resid = h_out;
-  }
-  if ((st = moe_combine(w.y_pairs, w.gates, w.ysh, T, H, k, y, resid, stream))) return st;
+  // h_out = h_in + the layer's output (the combine reads one and writes the other)
+  if ((st = launch_combine(w.y_pairs, w.gates, w.ysh, T, H, k, y, h_out ? h_in : nullptr, h_out, s))) return st;
   if (idx_out && (st = cuda_check(cudaMemcpyAsync(idx_out, w.idx, static_cast<size_t>(T) * k * 4,
                                                   cudaMemcpyDeviceToDevice, s), "copy idx")))
     return st;

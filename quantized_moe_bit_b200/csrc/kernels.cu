@@ -485,7 +485,7 @@ k_down_gemv(DownArgs a) {
 // ------------------------------------------------------------------------ A7
 __global__ void k_combine(const float* __restrict__ yp, const float* __restrict__ gates,
                           const float* __restrict__ ysh, int H, int k, uint16_t* __restrict__ y,
-                          float* __restrict__ resid) {
+                          const float* resid_in, float* resid_out) {
   const int t = blockIdx.y;
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= H) return;
@@ -495,15 +495,17 @@ __global__ void k_combine(const float* __restrict__ yp, const float* __restrict_
   for (int j = 0; j < k; ++j) acc = fmaf(g[j], yp[(static_cast<size_t>(t) * k + j) * H + c], acc);
   if (ysh != nullptr) acc += ysh[static_cast<size_t>(t) * H + c];
   if (y != nullptr) y[static_cast<size_t>(t) * H + c] = f32_to_bf16(acc);
-  if (resid != nullptr) resid[static_cast<size_t>(t) * H + c] += acc;
+  if (resid_out != nullptr) resid_out[static_cast<size_t>(t) * H + c] = resid_in[static_cast<size_t>(t) * H + c] + acc;
 }
 
+// (resid_out = resid_in + the sum: the residual add, in place when the two
+// are the same array.)
 // The same sum four columns per thread (16-byte aligned arrays, H % 4 == 0):
 // the k pair rows are loaded before the fma chain, which runs in the same
 // order (j = 0 .. k-1, then the shared row), so the result is bit-identical.
 __global__ void __launch_bounds__(256)
 k_combine4(const float* __restrict__ yp, const float* __restrict__ gates, const float* __restrict__ ysh, int H,
-           int k, uint16_t* __restrict__ y, float* __restrict__ resid) {
+           int k, uint16_t* __restrict__ y, const float* resid_in, float* resid_out) {
   const int t = blockIdx.y;
   const int c = 4 * (blockIdx.x * blockDim.x + threadIdx.x);
   if (c >= H) return;
@@ -537,10 +539,10 @@ k_combine4(const float* __restrict__ yp, const float* __restrict__ gates, const 
                                 static_cast<uint32_t>(f32_to_bf16(a2)) | (static_cast<uint32_t>(f32_to_bf16(a3)) << 16));
     *reinterpret_cast<uint2*>(y + o) = pk;
   }
-  if (resid != nullptr) {
-    float4 r = *reinterpret_cast<float4*>(resid + o);
+  if (resid_out != nullptr) {
+    float4 r = *reinterpret_cast<const float4*>(resid_in + o);
     r.x += a0; r.y += a1; r.z += a2; r.w += a3;
-    *reinterpret_cast<float4*>(resid + o) = r;
+    *reinterpret_cast<float4*>(resid_out + o) = r;
   }
 }
 

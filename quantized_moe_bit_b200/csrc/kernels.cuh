@@ -53,9 +53,9 @@ __global__ void k_bucket(const int32_t* idx, int n, int E, int32_t* offsets, int
 __global__ void k_gateup_gemv(GateUpArgs a);
 __global__ void k_down_gemv(DownArgs a);
 __global__ void k_combine(const float* yp, const float* gates, const float* ysh, int H, int k,
-                          uint16_t* y, float* resid);
+                          uint16_t* y, const float* resid_in, float* resid_out);
 __global__ void k_combine4(const float* yp, const float* gates, const float* ysh, int H, int k,
-                           uint16_t* y, float* resid);
+                           uint16_t* y, const float* resid_in, float* resid_out);
 
 // Shared memory of the router kernel: logits [TB][E] | staged x, per row the
 // byte-paired words [4][H/16] (rows 32 bytes apart modulo 128, so the eight

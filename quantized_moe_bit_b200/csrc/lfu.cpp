@@ -13,6 +13,14 @@
 // misses, each in the step's order; a global tick advances per access; a miss
 // fills the lowest empty slot, else evicts, among slots not used by the
 // current step, the smallest (count, last tick, slot index).
+//
+// Optional lookahead prefetch (off unless set): after a streamed layer call,
+// up to P experts of that layer are staged ahead of their next use -- the
+// non-resident ones accessed most often so far in the run (ties to the lower
+// id), each into the slot a miss would take, and only while that slot is
+// empty or its resident's count is below the candidate's access total.  A
+// prefetched expert enters with count 0; it is one more step of the layer
+// and is logged with hit = 2.
 #include <chrono>
 #include <cstdint>
 #include <cstdio>
@@ -37,6 +45,8 @@ struct moe_lfu {
   const void* const* host_blobs = nullptr;    // [L*E] pinned host pointers (null: plan only)
   unsigned char* pool = nullptr;              // device, L*S*slot_stride
   std::vector<int32_t> expert, count, steps;  // [L*S], [L*S], [L]
+  std::vector<int32_t> freq;                  // [L*E] accesses per expert over the run (prefetch ranking)
+  int prefetch_n = 0;                         // experts prefetched per streamed layer call (0: off)
   std::vector<int64_t> last;                  // [L*S]
   int64_t tick = 0;
   std::vector<int32_t> log;                   // records of 5
@@ -56,7 +66,7 @@ struct moe_lfu {
   // the slots that copies issued during the call write.  A failure restores
   // the state, so that repeating the call plans exactly as the first attempt.
   int txn_depth = 0, txn_layer = -1;
-  std::vector<int32_t> snap_expert, snap_count;
+  std::vector<int32_t> snap_expert, snap_count, snap_freq;
   std::vector<int64_t> snap_last;
   int64_t snap_tick = 0;
   int32_t snap_steps = 0;
@@ -93,6 +103,8 @@ void txn_begin(moe_lfu* h, int layer) {
   h->snap_expert.assign(h->expert.begin() + b, h->expert.begin() + b + h->S);
   h->snap_count.assign(h->count.begin() + b, h->count.begin() + b + h->S);
   h->snap_last.assign(h->last.begin() + b, h->last.begin() + b + h->S);
+  const size_t fb = static_cast<size_t>(layer) * h->E;
+  h->snap_freq.assign(h->freq.begin() + fb, h->freq.begin() + fb + h->E);
   h->snap_tick = h->tick;
   h->snap_steps = h->steps[layer];
   h->snap_log = h->log.size();
@@ -112,6 +124,7 @@ int txn_rollback(moe_lfu* h, int status) {
   std::copy(h->snap_expert.begin(), h->snap_expert.end(), h->expert.begin() + b);
   std::copy(h->snap_count.begin(), h->snap_count.end(), h->count.begin() + b);
   std::copy(h->snap_last.begin(), h->snap_last.end(), h->last.begin() + b);
+  std::copy(h->snap_freq.begin(), h->snap_freq.end(), h->freq.begin() + static_cast<size_t>(layer) * h->E);
   h->tick = h->snap_tick;
   h->steps[layer] = h->snap_steps;
   h->log.resize(h->snap_log);
@@ -159,12 +172,47 @@ int plan(moe_lfu* h, int layer, const int32_t* ids, int n, int32_t* slots_out, i
       }
       h->tick += 1;
       h->last[base + s] = h->tick;
+      h->freq[static_cast<size_t>(layer) * h->E + e] += 1;
       used[s] = 1;
       slots_out[i] = s;
       hit_out[i] = hit;
       const int32_t rec[5] = {layer, st, e, hit, s};
       h->log.insert(h->log.end(), rec, rec + 5);
     }
+  }
+  return MOE_OK;
+}
+
+// Plan a lookahead prefetch of up to P experts of `layer` (the policy in the
+// file header): ids_out / slots_out get the chosen experts and their slots.
+int plan_prefetch(moe_lfu* h, int layer, int P, std::vector<int32_t>& ids_out, std::vector<int32_t>& slots_out) {
+  ids_out.clear();
+  slots_out.clear();
+  if (P <= 0) return MOE_OK;
+  const size_t base = static_cast<size_t>(layer) * h->S, fb = static_cast<size_t>(layer) * h->E;
+  std::vector<char> res(h->E, 0);
+  for (int s = 0; s < h->S; ++s)
+    if (h->expert[base + s] >= 0) res[h->expert[base + s]] = 1;
+  std::vector<int32_t> cand;
+  for (int e = 0; e < h->E; ++e)
+    if (!res[e] && h->freq[fb + e] > 0) cand.push_back(e);
+  std::stable_sort(cand.begin(), cand.end(), [&](int32_t a, int32_t b) { return h->freq[fb + a] > h->freq[fb + b]; });
+  const int st = h->steps[layer]++;
+  std::vector<char> used(h->S, 0);
+  for (size_t i = 0; i < cand.size() && static_cast<int>(ids_out.size()) < P; ++i) {
+    const int e = cand[i];
+    const int s = victim(h, layer, used);
+    if (s < 0) break;
+    if (h->expert[base + s] >= 0 && h->count[base + s] >= h->freq[fb + e]) break;   // no colder resident
+    h->expert[base + s] = e;
+    h->count[base + s] = 0;
+    h->tick += 1;
+    h->last[base + s] = h->tick;
+    used[s] = 1;
+    ids_out.push_back(e);
+    slots_out.push_back(s);
+    const int32_t rec[5] = {layer, st, e, 2, s};
+    h->log.insert(h->log.end(), rec, rec + 5);
   }
   return MOE_OK;
 }
@@ -204,6 +252,7 @@ MOE_API int moe_lfu_create(int n_layers, int n_experts, int n_slots, size_t blob
   h->count.assign(static_cast<size_t>(n_layers) * n_slots, 0);
   h->last.assign(static_cast<size_t>(n_layers) * n_slots, 0);
   h->steps.assign(n_layers, 0);
+  h->freq.assign(static_cast<size_t>(n_layers) * n_experts, 0);
   if (slot_pool) h->dirty.assign(static_cast<size_t>(n_layers) * n_slots, 0);
   if (slot_pool) {
     h->mirror.assign(n_layers, nullptr);
@@ -316,7 +365,10 @@ MOE_API int moe_lfu_get_log(moe_lfu* h, int32_t* buf, size_t cap_records, size_t
 MOE_API int moe_lfu_stats(moe_lfu* h, int64_t* hits, int64_t* misses, int64_t* bytes_copied) {
   if (!h) return moe::fail(MOE_ERR_INVALID_ARG, "lfu_stats: NULL");
   int64_t nh = 0, nm = 0;
-  for (size_t i = 0; i + 4 < h->log.size(); i += 5) (h->log[i + 3] ? nh : nm) += 1;
+  for (size_t i = 0; i + 4 < h->log.size(); i += 5) {      // prefetch records (hit = 2) are neither
+    if (h->log[i + 3] == 1) ++nh;
+    else if (h->log[i + 3] == 0) ++nm;
+  }
   if (hits) *hits = nh;
   if (misses) *misses = nm;
   if (bytes_copied) *bytes_copied = h->bytes_copied;
@@ -327,6 +379,25 @@ MOE_API int moe_lfu_set_fault(moe_lfu* h, int kind, int after_n) {
   if (!h || kind < 0 || kind > 2) return moe::fail(MOE_ERR_INVALID_ARG, "lfu_set_fault: bad arguments");
   h->fault_kind = kind;
   h->fault_after = after_n;
+  return MOE_OK;
+}
+
+MOE_API int moe_lfu_set_prefetch(moe_lfu* h, int per_call) {
+  if (!h || per_call < 0 || per_call > h->S) return moe::fail(MOE_ERR_INVALID_ARG, "lfu_set_prefetch: bad arguments");
+  h->prefetch_n = per_call;
+  return MOE_OK;
+}
+
+MOE_API int moe_lfu_plan_prefetch(moe_lfu* h, int layer, int per_call, int32_t* ids_out, int32_t* slots_out,
+                                  int* n_out) {
+  if (!h || !n_out || (per_call > 0 && (!ids_out || !slots_out)))
+    return moe::fail(MOE_ERR_INVALID_ARG, "lfu_plan_prefetch: NULL");
+  if (layer < 0 || layer >= h->L || per_call < 0 || per_call > h->S)
+    return moe::fail(MOE_ERR_INVALID_ARG, "lfu_plan_prefetch: bad arguments");
+  std::vector<int32_t> ids, slots;
+  plan_prefetch(h, layer, per_call, ids, slots);
+  for (size_t i = 0; i < ids.size(); ++i) { ids_out[i] = ids[i]; slots_out[i] = slots[i]; }
+  *n_out = static_cast<int>(ids.size());
   return MOE_OK;
 }
 
@@ -453,6 +524,31 @@ MOE_API int moe_streamed_layer_forward(moe_lfu* h, int layer, float* hres, int T
       return abort_call(st);
     if ((st = moe::cuda_check(cudaEventRecord(h->consumed[layer], ms), "streamed: record consumed")))
       return abort_call(st);
+  }
+  // lookahead prefetch (part of the call's transaction): the copies follow
+  // the call's expert kernels on the side stream, since a victim slot may be
+  // one they read
+  if (h->prefetch_n > 0) {
+    std::vector<int32_t> pids, pslots;
+    plan_prefetch(h, layer, h->prefetch_n, pids, pslots);
+    if (!pids.empty() &&
+        (st = moe::cuda_check(cudaStreamWaitEvent(static_cast<cudaStream_t>(side_stream), h->consumed[layer], 0),
+                              "streamed: prefetch wait")))
+      return abort_call(st);
+    const size_t base = static_cast<size_t>(layer) * h->S;
+    for (size_t i = 0; i < pids.size(); ++i) {
+      ++h->copies;
+      if (h->fault_kind == MOE_LFU_FAULT_COPY_FAILS && h->fault_after >= 0 && h->copies > h->fault_after)
+        return abort_call(moe::fail(MOE_ERR_CUDA, "streamed: injected copy failure (copy %ld)", h->copies));
+      unsigned char* slot = h->pool + (base + pslots[i]) * h->slot_stride;
+      const void* src = h->host_blobs[static_cast<size_t>(layer) * h->E + pids[i]];
+      if ((st = moe::cuda_check(cudaMemcpyAsync(slot, src, h->blob_bytes, cudaMemcpyHostToDevice,
+                                                static_cast<cudaStream_t>(side_stream)), "streamed: prefetch copy")))
+        return abort_call(st);
+      h->txn_written.push_back(pslots[i]);
+      h->dirty[base + pslots[i]] = 0;
+      h->bytes_copied += static_cast<int64_t>(h->blob_bytes);
+    }
   }
   txn_commit(h);
   if ((st = moe::cuda_check(cudaEventRecord(h->stage_free, ms), "streamed: record staging"))) return st;

@@ -115,7 +115,7 @@ def run_streamed(M, S, units, lfu, side, on_error=None):
     return outs
 
 
-def simulate(S, outs):
+def simulate(S, outs, prefetch: int = 0):
     c = S.cfg
     sim = LFUSim(c.layers, c.n_slots)
     for o in outs:
@@ -126,6 +126,7 @@ def simulate(S, outs):
             else:
                 for ids in sim.chunk_steps(l, np.unique(idx).tolist(), c.k):
                     sim.step(l, ids)
+            sim.prefetch(l, prefetch)            # after every layer call (nothing at 0)
     return sim
 
 
@@ -144,38 +145,45 @@ def check_against_oracle(S, outs, units, samples):
         check_output(outs[u]["y"][l].view(np.uint16), r["out"], f"unit {u} layer {l}")
 
 
-def _run_all(M, cfg, samples):
+def _run_all(M, cfg, samples, prefetch: int = 0):
     S = Streamed(M, cfg)
     units = S.inputs()
     ref = run_resident(M, S, units)
     lfu = M.MoeLfu(cfg.layers, cfg.E, cfg.n_slots, gen.blob_bytes(cfg.H, cfg.I), S.host_ptrs, S.pool,
                    S.stride)
+    lfu.set_prefetch(prefetch)
     side = torch.cuda.Stream()
     got = run_streamed(M, S, units, lfu, side)
     for a, b in zip(ref, got):
         assert np.array_equal(a["h"], b["h"])
         for l in range(cfg.layers):
             assert np.array_equal(a["y"][l], b["y"][l]) and np.array_equal(a["idx"][l], b["idx"][l])
-    sim = simulate(S, got)
+    sim = simulate(S, got, prefetch)
     assert lfu.log() == sim.log
     hits, misses, nbytes = lfu.stats()
-    assert misses * gen.blob_bytes(cfg.H, cfg.I) == nbytes and hits > 0
+    staged = sum(1 for r in sim.log if r[3] == 2)
+    assert (misses + staged) * gen.blob_bytes(cfg.H, cfg.I) == nbytes and hits > 0
+    assert (staged > 0) == (prefetch > 0)
     check_against_oracle(S, got, units, samples)
     lfu.close()
     return hits, misses
 
 
-def test_streamed_tiny(M):
+@pytest.mark.parametrize("prefetch", [0, 2])
+def test_streamed_tiny(M, prefetch):
     cfg = replace(tiny_config("streamed_30L_lfu"), layers=4, T=24, prompt_tokens=48, decode_steps=6, n_slots=6)
-    _run_all(M, cfg, samples=[(0, 0), (1, 3), (2, 1), (7, 2)])
+    _run_all(M, cfg, samples=[(0, 0), (1, 3), (2, 1), (7, 2)], prefetch=prefetch)
 
 
-def test_streamed_full(M):
+@pytest.mark.parametrize("prefetch", [0, 2])
+def test_streamed_full(M, prefetch):
     """1024-token prompt in chunks of 128 through 30 layers, then 128 decode
-    steps, routed experts in pinned host memory, 16 slots per layer."""
+    steps, routed experts in pinned host memory, 16 slots per layer (with and
+    without the lookahead prefetch of 2 experts per layer call)."""
     cfg = CONFIGS["streamed_30L_lfu"]
-    hits, misses = _run_all(M, cfg, samples=[(0, 0), (3, 17), (7, 29), (8, 5), (100, 12), (135, 29)])
-    print(f"streamed_30L_lfu: hits {hits} misses {misses}")
+    hits, misses = _run_all(M, cfg, samples=[(0, 0), (3, 17), (7, 29), (8, 5), (100, 12), (135, 29)],
+                            prefetch=prefetch)
+    print(f"streamed_30L_lfu prefetch {prefetch}: hits {hits} misses {misses}")
 
 
 def test_lfu_host_faults(M):

@@ -46,9 +46,15 @@ def test_random_streams_match_simulator(M, seed):
             slots, hits = lf.plan(layer, ids)
             where = sim.step(layer, ids)
             assert slots == [where[e] for e in ids]
+        if rng.random() < 0.25:
+            # a lookahead prefetch of up to P experts of the layer
+            P = int(rng.integers(1, 4))
+            ids, slots = lf.plan_prefetch(layer, P)
+            assert list(zip(ids, slots)) == sim.prefetch(layer, P)
     assert lf.log() == sim.log
+    assert any(r[3] == 2 for r in sim.log)
     h, m, _ = lf.stats()
-    assert h + m == len(sim.log) and h == sum(r[3] for r in sim.log)
+    assert h == sum(1 for r in sim.log if r[3] == 1) and m == sum(1 for r in sim.log if r[3] == 0)
 
 
 def test_invalid_steps(M):

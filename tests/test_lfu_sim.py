@@ -68,3 +68,33 @@ def test_chunk_steps_resident_first():
     sim = LFUSim(1, 4)
     sim.step(0, [3, 9])
     assert sim.chunk_steps(0, [1, 9, 3, 12, 5, 9], 2) == [[3, 9], [1, 5], [12]]
+
+
+def test_hand_traced_prefetch():
+    # 2 slots, one id per step; traced by hand:
+    #  [1] -> s0 (c1, t1); [2] -> s1 (c1, t2); [1] hit s0 (c2, t3);
+    #  [3]: victims s0 (2, t3), s1 (1, t2) -> s1 (c1, t4);
+    #  [2]: victims s0 (2, t3), s1 (1, t4) -> s1 (c1, t5);
+    #  [3]: -> s1 (c1, t6).  Access totals: 1: 2, 2: 2, 3: 2.
+    #  prefetch(1): candidates (not resident) [2]; victim s1 (count 1 < 2)
+    #               -> 2 into s1 with count 0 (t7), step 6;
+    #  prefetch(1): candidates [3]; victim s1 (count 0 < 2) -> 3 into s1 (t8), step 7;
+    #  [2]: a miss again: victims s0 (2, t3), s1 (0, t8) -> s1 (t9), step 8.
+    sim = LFUSim(1, 2)
+    for ids in ([1], [2], [1], [3], [2], [3]):
+        sim.step(0, ids)
+    assert sim.prefetch(0, 1) == [(2, 1)]
+    assert sim.prefetch(0, 1) == [(3, 1)]
+    sim.step(0, [2])
+    assert sim.log[6:] == [(0, 6, 2, 2, 1), (0, 7, 3, 2, 1), (0, 8, 2, 0, 1)]
+
+
+def test_prefetch_keeps_hotter_residents():
+    # 1 slot: expert 2 resident with count 3; expert 1 accessed once: its
+    # victim (count 3) is not colder, so nothing is staged (the step still counts)
+    sim = LFUSim(1, 1)
+    for ids in ([1], [2], [2], [2]):
+        sim.step(0, ids)
+    assert sim.prefetch(0, 1) == []
+    assert sim.steps[0] == 5 and len(sim.log) == 4
+    assert sim.prefetch(0, 0) == [] and sim.steps[0] == 5     # P = 0: no step
