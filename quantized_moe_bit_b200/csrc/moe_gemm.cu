@@ -87,9 +87,13 @@ static_assert(GM_MAP_RING > GM_RS + 1, "tensor-map ring vs raw ring");
 // two run at once).  In a group two warps share each TMEM sub-partition
 // (warp w writes TMEM lanes 32 (w % 4) ..), each taking half of every atom
 // row (4 code words).  Both groups take part in every stage's barriers.
-constexpr int GM_EPI_WARPS = 4, GM_RAW_WARP = 4, GM_B_WARP = 5, GM_MMA_WARP = 6, GM_MMA_WARPS = 4;
+// Epilogue: 8 warps, two per TMEM sub-partition (warps 0-3 and the four
+// consecutive warps from GM_EPI_WARP1; warp w reads TMEM lanes 32 (w % 4) ..),
+// each pair taking the item's 16-column blocks alternately.
+constexpr int GM_RAW_WARP = 4, GM_B_WARP = 5, GM_MMA_WARP = 6, GM_MMA_WARPS = 4;
 constexpr int GM_DQ_WARP0 = GM_MMA_WARP + GM_MMA_WARPS, GM_DQ_GROUPS = 2, GM_DQ_WARPS = 8 * GM_DQ_GROUPS;
-constexpr int GM_THREADS = (GM_DQ_WARP0 + GM_DQ_WARPS) * 32;
+constexpr int GM_EPI_WARP1 = GM_DQ_WARP0 + GM_DQ_WARPS, GM_EPI_WARPS = 8;
+constexpr int GM_THREADS = (GM_EPI_WARP1 + 4) * 32;
 // barriers: raw full/empty [RS], a full [ST], stage empty [ST], b full [ST], sc full/empty [2],
 // acc full/empty [2], final
 constexpr int GM_NBARS = 2 * GM_RS + 3 * GM_ST + 4 + 4 + 1;
@@ -640,7 +644,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
     if (lane == 0) tc::umma_commit(final_bar);
     __syncwarp();
     gm_wait_drain(final_bar, 0);
-  } else if (warp >= GM_DQ_WARP0) {
+  } else if (warp >= GM_DQ_WARP0 && warp < GM_DQ_WARP0 + GM_DQ_WARPS) {
     // -------------------------------------------------------------- dequant
     const int dw = warp - GM_DQ_WARP0;
     const int grp = dw >> 3;                             // dequant group: atoms grp, grp + 2 of every stage
@@ -705,8 +709,10 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(sc_empty(sb));
     }
-  } else if (warp < GM_EPI_WARPS) {
+  } else if (warp < 4 || warp >= GM_EPI_WARP1) {
     // ------------------------------------------------------------- epilogue
+    const int wq = warp & 3;                        // TMEM sub-partition (lanes 32 wq ..)
+    const int half = warp >= GM_EPI_WARP1 ? 1 : 0;  // which 16-column blocks: 2 b + half
     int il = 0;
     bool ok = true;
     for (int rd = 0, item = gm_item_at(0, G); item < n_items && ok; item = gm_item_at(++rd, G), ++il) {
@@ -716,10 +722,10 @@ __global__ void __launch_bounds__(GM_THREADS, 1) k_moe_gemm(const __grid_constan
       if (!ok) break;
       tc::tc_fence_after();
       const int Np = (it.N + 15) & ~15;
-      const int row = 32 * warp + lane;             // TMEM lane = A row
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * warp) << 16) + static_cast<uint32_t>(acc * GM_NMAX);
+      const int row = 32 * wq + lane;               // TMEM lane = A row
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * wq) << 16) + static_cast<uint32_t>(acc * GM_NMAX);
       const int C = gm_chains(Np);
-      for (int nc = 0; nc < Np; nc += 16) {
+      for (int nc = 16 * half; nc < Np; nc += 32) {
         float v[16];
         tc::tmem_ld16(taddr + nc, v);
         for (int c = 1; c < C; ++c) {        // add the item's other accumulator chains
