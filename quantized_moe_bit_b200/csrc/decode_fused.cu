@@ -174,9 +174,8 @@ struct DfGeom {
   DF_HD int part_slots() const {
     const int a = (DF_WARPS - 1) * sg_tiles_max(), b = DF_WARPS * rg_tiles_max();
     const int c = dp() * d_tiles_max() + DF_WARPS * sd_tiles_max();
-    const int r = DF_THREADS * 4 / 64;              // the top-k's partial ranks: one int per thread
-    const int m = a > b ? a : b, n = m > c ? m : c;
-    return n > r ? n : r;
+    const int m = a > b ? a : b;
+    return m > c ? m : c;
   }
   DF_HD uint32_t misc_bytes() const {
     // logits, sel / selv / selg, red, bars, blob table, copy table, pair table, part
@@ -941,35 +940,18 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
     }
     __syncthreads();
     df_stamp(a, l, 3);
-    {
-      // rank of every logit (the number above it; an exact tie goes to the
-      // lower id) over all threads: thread (p, e) counts over the p-th of
-      // P = DF_THREADS / E slices of the logits into the partial-sum area
-      // (free between the shared activations and the routed tiles), then
-      // thread e adds its P partials; ranks 0 .. k-1 are the selection
-      int* rk = reinterpret_cast<int*>(part);
-      const int P = DF_THREADS / E, nq = E / 4;      // E is a multiple of 8
-      if (threadIdx.x < P * E) {
-        const int e = threadIdx.x % E, p = threadIdx.x / E;
-        const float v = lg[e];
-        int rank = 0;
-        const float4* l4 = reinterpret_cast<const float4*>(lg);
-        for (int f = p * nq / P; f < (p + 1) * nq / P; ++f) {
-          const float4 w = l4[f];
-          rank += (w.x > v || (w.x == v && 4 * f + 0 < e)) ? 1 : 0;
-          rank += (w.y > v || (w.y == v && 4 * f + 1 < e)) ? 1 : 0;
-          rank += (w.z > v || (w.z == v && 4 * f + 2 < e)) ? 1 : 0;
-          rank += (w.w > v || (w.w == v && 4 * f + 3 < e)) ? 1 : 0;
-        }
-        rk[p * E + e] = rank;
+    for (int e = threadIdx.x; e < E; e += DF_THREADS) {
+      const float v = lg[e];
+      int rank = 0;
+      const float4* l4 = reinterpret_cast<const float4*>(lg);
+      for (int f = 0; f < E / 4; ++f) {      // E is a multiple of 8
+        const float4 w = l4[f];
+        rank += (w.x > v || (w.x == v && 4 * f + 0 < e)) ? 1 : 0;
+        rank += (w.y > v || (w.y == v && 4 * f + 1 < e)) ? 1 : 0;
+        rank += (w.z > v || (w.z == v && 4 * f + 2 < e)) ? 1 : 0;
+        rank += (w.w > v || (w.w == v && 4 * f + 3 < e)) ? 1 : 0;
       }
-      __syncthreads();
-      if (threadIdx.x < E) {
-        const int e = threadIdx.x;
-        int rank = 0;
-        for (int p = 0; p < P; ++p) rank += rk[p * E + e];
-        if (rank < k) { sel[rank] = e; selv[rank] = lg[e]; }
-      }
+      if (rank < k) { sel[rank] = e; selv[rank] = v; }
     }
     __syncthreads();
     df_stamp(a, l, 4);

@@ -226,9 +226,6 @@ int main(int argc, char** argv) {
             g.slot_d(g.dp() - 1, g.d_tiles_max() - 1) < g.slot_sd(0, 0) &&
             g.slot_sd(DF_WARPS - 1, g.sd_tiles_max() - 1) < g.part_slots(), "cta %d partial-sum slots", c);
     REQUIRE(g.m_part() + g.part_slots() * 64u <= g.total, "cta %d part area", c);
-    // the top-k's partial ranks: (DF_THREADS / E) * E ints in the part area
-    REQUIRE((DF_THREADS / E) * E * 4 <= g.part_slots() * 64 && DF_THREADS / E >= 1 && E % 8 == 0,
-            "cta %d top-k partial ranks", c);
   }
   REQUIRE(pairs == static_cast<long>(k) * I && spairs == Is && rows == H, "coverage %ld %ld %ld", pairs, spairs, rows);
   if (fails) {
