@@ -409,6 +409,87 @@ MOE_API int moe_streamed_layer_forward(moe_lfu* h, int layer, float* hres, int T
                                        size_t ws_bytes, int flags, void* main_stream, void* side_stream,
                                        int timeout_ms);
 
+/* ---------------------------------------------------------------------------
+ * Expert parallelism (one process per GPU, G ranks).  The pages run the
+ * layer on one device; splitting its routed experts over ranks is this
+ * library's extension of the same computation.  Per token only its top-k
+ * routed experts are applied ("drumih/turbo-fieldfare" (paperfeed.app),
+ * section "Why this is interesting"), each from its own 4-bit blob
+ * ("TurboFieldfare: Gemma 4 26B on an 8 GB MacBook, in ~2 GB of RAM"
+ * (blog-mushroom.pages.dev), section "Why 26B Fits in 2 GB"), so the experts
+ * split into disjoint sets: rank d owns experts [d E/G, (d+1) E/G), and a
+ * (token, slot) pair is computed where its expert lives.  Each rank keeps its
+ * own tokens, router, shared expert and combine; results equal the one-GPU
+ * layer's within the output tolerance (the grouped GEMM sees other bucket
+ * sizes).
+ *
+ * Per layer, on each rank: norm, router, moe_bucket; all ranks' bucket
+ * offsets gathered into all_offsets (int32 [G][E+1], rank r's row r, e.g. by
+ * an all-gather); moe_ep_dispatch; a barrier across ranks; moe_ep_recv_plan
+ * and moe_expert_forward over the received rows (k = 1, E/G experts);
+ * moe_ep_return; a barrier; moe_combine of the rank's own y_pairs.
+ *
+ * Receiver layout: rank d's received rows are ordered by its experts, then
+ * by source rank, then by the source's bucket order.  With
+ * cnt(s,e) = all_offsets[s][e+1] - all_offsets[s][e], slot i of source s's
+ * bucket e lands on row base(e) + before(s,e) + (i - all_offsets[s][e]) of
+ * rank e/(E/G), where base(e) sums cnt over all sources and the experts of
+ * that rank below e, and before(s,e) sums cnt(s',e) over s' < s.
+ *
+ * Peer tables are host arrays of G device pointers, entry r being rank r's
+ * buffer as this process maps it (its own buffer for r = this rank, an
+ * moe_ipc_open mapping for the others); each must be 16-byte aligned.
+ * Requirements: 1 <= G <= 8, E/G a whole multiple of 8, 0 <= rank < G.
+ * Rows past a receiver's capacity are skipped and flagged (check word bit 8,
+ * MOE_ERR_DEVICE_CHECK at the next moe_sync).  Errors otherwise as the other
+ * calls: MOE_ERR_INVALID_ARG before any launch.
+ * --------------------------------------------------------------------------- */
+
+/* Dispatch (source rank `rank`): for each bucketed slot i < all_offsets[rank][E]
+ * with pair p = pairs[i], copies x row p / k (bf16 [H]) to row
+ * base(e) + before(rank,e) + (i - off[e]) of recv_x[e/(E/G)] (bf16 [cap_rows, H])
+ * and writes (rank, p) to the same row of recv_meta[...] (int32 [cap_rows, 2]),
+ * e = idx[p].
+ *   x        bf16 [T,H] (device): the layer input
+ *   idx      int32 [T,k] (device) routing; pairs: from moe_bucket (device)
+ *   all_offsets  int32 [G][E+1] (device)
+ *   recv_x, recv_meta  host arrays [G] of peer device pointers
+ * Ends with a system-scope fence, so the stores are visible to the peers once
+ * the kernel has completed. */
+MOE_API int moe_ep_dispatch(const uint16_t* x, int T, int H, int k, int E, int G, int rank,
+                            const int32_t* idx, const int32_t* pairs, const int32_t* all_offsets,
+                            void* const* recv_x, void* const* recv_meta, int cap_rows, void* stream);
+
+/* Receiver plan (rank `rank`): offsets int32 [E/G + 1] = base(rank*E/G + j)
+ * clamped to cap_rows (offsets[E/G] = rows received), pairs int32 [cap_rows]
+ * = the identity over the rows received, active int32 [E/G] = the local
+ * experts with rows, ascending, and n_active int32 [1] (all device): the
+ * inputs of moe_expert_forward over recv_x with T = cap_rows, k = 1,
+ * E = E/G and this rank's blob table. */
+MOE_API int moe_ep_recv_plan(const int32_t* all_offsets, int G, int E, int rank, int cap_rows,
+                             int32_t* offsets, int32_t* pairs, int32_t* active, int32_t* n_active,
+                             void* stream);
+
+/* Return (receiver rank `rank`): row r < offsets[E/G] of y_rows (fp32
+ * [cap_rows, H], the expert outputs over the received rows) goes to row p of
+ * y_pairs[s] (fp32 [n_pair_slots, H] on rank s), (s, p) = recv_meta[r].
+ * Ends with a system-scope fence like the dispatch. */
+MOE_API int moe_ep_return(const float* y_rows, int H, int E, int G, int rank, const void* recv_meta,
+                          const int32_t* offsets, int n_pair_slots, int cap_rows, void* const* y_pairs,
+                          void* stream);
+
+/* Device buffers that other processes may map: moe_device_alloc returns a
+ * whole allocation of `bytes` (cudaMalloc) whose handle moe_ipc_get_handle
+ * writes into moe_ipc_handle_bytes() bytes; another process on the same node
+ * maps it with moe_ipc_open (peer access enabled on first use) and unmaps it
+ * with moe_ipc_close.  A process cannot open its own handle. */
+MOE_API int moe_device_alloc(size_t bytes, void** ptr);
+MOE_API int moe_device_free(void* ptr);
+MOE_API int moe_ipc_handle_bytes(void);
+MOE_API int moe_ipc_get_handle(const void* ptr, void* handle_out);
+MOE_API int moe_ipc_open(const void* handle, void** ptr);
+MOE_API int moe_ipc_close(void* ptr);
+
 #ifdef __cplusplus
 }
 #endif

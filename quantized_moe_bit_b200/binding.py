@@ -230,3 +230,55 @@ def moe_streamed_layer_forward(lfu: "MoeLfu", layer: int, h, I: int, Is: int, E:
                                            bias_per_row, arr, ptr(dev_table), ptr(x_out), ptr(y_out), ptr(idx_out),
                                            ptr(ws), ws.numel() * ws.element_size(), flags, stream_ptr(main_stream),
                                            stream_ptr(side_stream), timeout_ms))
+
+
+# --------------------------------------------------------------- expert parallelism
+def _peer_table(ptrs):
+    """Host array of device pointers (ints or tensors) for a peer table."""
+    return (C.c_void_p * len(ptrs))(*[ptr(p) for p in ptrs])
+
+
+def moe_ep_dispatch(x, k: int, E: int, G: int, rank: int, idx, pairs, all_offsets, recv_x, recv_meta,
+                    cap_rows: int, stream=None):
+    T, H = x.shape
+    check(lib().moe_ep_dispatch(ptr(x), T, H, k, E, G, rank, ptr(idx), ptr(pairs), ptr(all_offsets),
+                                _peer_table(recv_x), _peer_table(recv_meta), cap_rows, stream_ptr(stream)))
+
+
+def moe_ep_recv_plan(all_offsets, G: int, E: int, rank: int, cap_rows: int, offsets, pairs, active, n_active,
+                     stream=None):
+    check(lib().moe_ep_recv_plan(ptr(all_offsets), G, E, rank, cap_rows, ptr(offsets), ptr(pairs), ptr(active),
+                                 ptr(n_active), stream_ptr(stream)))
+
+
+def moe_ep_return(y_rows, E: int, G: int, rank: int, recv_meta, offsets, n_pair_slots: int, y_pairs,
+                  stream=None):
+    cap_rows, H = y_rows.shape
+    check(lib().moe_ep_return(ptr(y_rows), H, E, G, rank, ptr(recv_meta), ptr(offsets), n_pair_slots, cap_rows,
+                              _peer_table(y_pairs), stream_ptr(stream)))
+
+
+def moe_device_alloc(nbytes: int) -> int:
+    p = C.c_void_p()
+    check(lib().moe_device_alloc(nbytes, C.byref(p)))
+    return p.value
+
+
+def moe_device_free(p: int):
+    check(lib().moe_device_free(p))
+
+
+def moe_ipc_get_handle(p: int) -> bytes:
+    buf = C.create_string_buffer(lib().moe_ipc_handle_bytes())
+    check(lib().moe_ipc_get_handle(p, buf))
+    return buf.raw
+
+
+def moe_ipc_open(handle: bytes) -> int:
+    p = C.c_void_p()
+    check(lib().moe_ipc_open(C.c_char_p(handle), C.byref(p)))
+    return p.value
+
+
+def moe_ipc_close(p: int):
+    check(lib().moe_ipc_close(p))

@@ -368,7 +368,7 @@ int moe_sync(void* stream) {
   if (w != 0) {
     unsigned int z = 0;
     cudaMemcpyToSymbol(g_check_word, &z, sizeof(z));
-    return fail(MOE_ERR_DEVICE_CHECK, "device check word 0x%x (1: expert id, 2: pair id, 4: wait)", w);
+    return fail(MOE_ERR_DEVICE_CHECK, "device check word 0x%x (1: expert id, 2: pair id, 4: wait, 8: expert-parallel row past capacity)", w);
   }
   return MOE_OK;
 }

@@ -13,7 +13,7 @@ namespace moe {
 // access and sets a bit here; moe_sync() reads and clears it.
 __device__ unsigned int g_check_word = 0;  // defined once: libmoe is one CUDA translation unit
 
-enum : unsigned { CHECK_EXPERT_ID = 1u, CHECK_PAIR_ID = 2u, CHECK_WAIT = 4u };
+enum : unsigned { CHECK_EXPERT_ID = 1u, CHECK_PAIR_ID = 2u, CHECK_WAIT = 4u, CHECK_EP_ROW = 8u };
 
 __device__ __forceinline__ void flag_check(unsigned bit) { atomicOr(&g_check_word, bit); }
 

@@ -3,3 +3,4 @@
 #include "kernels.cu"
 #include "api.cu"
 #include "expert_noalloc.cu"
+#include "ep.cu"

@@ -1,0 +1,170 @@
+"""The expert-parallel layer schedule (quantized_moe_bit_b200.ep) across two
+gloo ranks on the CPU.
+
+The product's schedule (`ep_layer_forward`) and collectives (`EpComm`) run
+unchanged; each rank's steps are host stand-ins computed with the oracle, and
+the peers' buffers are shared-memory CPU tensors that the ranks store into
+directly, as the kernels store into peer GPU memory.  The stand-ins place rows
+by the receiver layout as the C-ABI header defines it.  Two layers in a row
+(buffers reused across layers), and the result of every rank equals the
+one-process oracle layer on that rank's tokens.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import gen
+from gen import tiny_config
+from oracle import moe_oracle as O
+
+CFG = tiny_config("prefill_1L_128tok", T=5)
+WORLD = 2
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+class HostEpRank:
+    """Oracle stand-in of EpRank's steps on host buffers."""
+
+    def __init__(self, G, rank, cfg, recv_x, recv_meta, y_pairs):
+        self.G, self.rank, self.c = G, rank, cfg
+        self.El = cfg.E // G
+        self.recv_x, self.recv_meta, self.y_pairs = recv_x, recv_meta, y_pairs
+        self.offsets = torch.zeros(cfg.E + 1, dtype=torch.int32)
+        self.all_off = torch.zeros((G, cfg.E + 1), dtype=torch.int32)
+        self.layer = None
+
+    def set_layer(self, l):
+        c = self.c
+        self.layer = l
+        self.router = gen.router_weights(c.seed, l, c.E, c.H)
+        self.bias = gen.zipf_bias(c.seed, l, c.E) if c.zipf else None
+        self.shared = gen.shared_weights(c.seed, l, c.H, c.Is)
+
+    def front(self, h, flags=0):
+        c = self.c
+        _, self.x = O.rmsnorm(h.numpy())
+        lg = O.router_logits(self.x, self.router, self.bias)
+        self.idx = O.top_k(lg, c.k)
+        self.gates = O.softmax_gates(lg, self.idx)
+        off, self.pairs, _ = O.buckets(self.idx, c.E)
+        self.offsets.copy_(torch.from_numpy(off))
+        self.ysh = O.mlp(self.x, *self.shared)
+
+    def _row(self, s, e, i):
+        """Receiver row of slot i of source s's bucket e (the header's layout)."""
+        A = self.all_off.numpy().astype(np.int64)
+        cnt = A[:, 1:] - A[:, :-1]
+        d0 = (e // self.El) * self.El
+        base = int(cnt[:, d0:e].sum())
+        before = int(cnt[:s, e].sum())
+        return base + before + (i - int(A[s, e]))
+
+    def dispatch(self):
+        c = self.c
+        n = int(self.offsets[c.E])
+        for i in range(n):
+            p = int(self.pairs[i])
+            e = int(self.idx.reshape(-1)[p])
+            d = e // self.El
+            r = self._row(self.rank, e, i)
+            self.recv_x[d][r] = torch.from_numpy(self.x[p // c.k])
+            self.recv_meta[d][r] = torch.tensor([self.rank, p], dtype=torch.int32)
+
+    def experts(self, flags=0):
+        c = self.c
+        A = self.all_off.numpy().astype(np.int64)
+        cnt = A[:, 1:] - A[:, :-1]
+        d = self.rank
+        mine = cnt[:, d * self.El:(d + 1) * self.El].sum(axis=0)
+        loff = np.concatenate([[0], np.cumsum(mine)])
+        rx = self.recv_x[d].numpy()
+        meta = self.recv_meta[d].numpy()
+        for j in range(self.El):
+            a, b = int(loff[j]), int(loff[j + 1])
+            if a == b:
+                continue
+            e = d * self.El + j
+            # every row of the expert's range came from a pair routed to e
+            for r in range(a, b):
+                s, p = meta[r]
+                assert s in range(self.G)
+            y = O.mlp(rx[a:b], *gen.expert_weights(c.seed, self.layer, e, c.H, c.I))
+            for r in range(a, b):
+                s, p = meta[r]
+                self.y_pairs[s][p] = torch.from_numpy(y[r - a])
+
+    def combine(self, h):
+        out = O.combine(self.y_pairs[self.rank].numpy(), self.gates, self.ysh)
+        h += torch.from_numpy(out)
+
+
+def _worker(rank, world, port, recv_x, recv_meta, y_pairs, q):
+    import datetime
+    import torch.distributed as dist
+    from quantized_moe_bit_b200 import ep
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        c = CFG
+        comm = ep.EpComm()
+        r = HostEpRank(world, rank, c, recv_x, recv_meta, y_pairs)
+        z = gen.rows(c.seed, 1000 + rank, c.T, c.H).astype(np.float64)
+        h = torch.from_numpy(z.copy())
+        want = z.copy()
+        for l in range(2):
+            r.set_layer(l)
+            ep.ep_layer_forward([r], comm, [h])
+            _, x = O.rmsnorm(want)
+            res = O.layer_forward(x, r.router, r.bias, lambda e, l=l: gen.expert_weights(c.seed, l, e, c.H, c.I),
+                                  r.shared, c.k, c.E)
+            want = want + res["out"]
+        q.put((rank, float(np.abs(h.numpy() - want).max()), float(np.abs(want).max())))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_two_layers_match_oracle():
+    c = CFG
+    cap = WORLD * c.T * c.k
+    recv_x = [torch.zeros((cap, c.H), dtype=torch.float64).share_memory_() for _ in range(WORLD)]
+    recv_meta = [torch.full((cap, 2), -1, dtype=torch.int32).share_memory_() for _ in range(WORLD)]
+    y_pairs = [torch.zeros((c.T * c.k, c.H), dtype=torch.float64).share_memory_() for _ in range(WORLD)]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_worker, args=(r, WORLD, port, recv_x, recv_meta, y_pairs, q)) for r in range(WORLD)]
+    for p in ps:
+        p.start()
+    got = {}
+    for _ in range(WORLD):
+        rank, err, scale = q.get(timeout=180)
+        got[rank] = (err, scale)
+    for p in ps:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, (err, scale) in got.items():
+        assert err <= 1e-12 * scale, (rank, err, scale)
+    # both ranks received rows of the other (the exchange was exercised)
+    for d in range(WORLD):
+        srcs = set(recv_meta[d][:, 0].tolist()) - {-1}
+        assert srcs == {0, 1}, (d, srcs)
+
+
+def test_rank_shapes_rejected_before_any_allocation():
+    from quantized_moe_bit_b200 import ep
+    with pytest.raises(ValueError):
+        ep.EpRank(3, 0, 4, 256, 128, 192, 16, 4, layer=None)      # 16 experts do not split over 3 ranks
+    with pytest.raises(ValueError):
+        ep.EpRank(4, 0, 4, 256, 128, 192, 16, 4, layer=None)      # 4 experts per rank: not a multiple of 8
