@@ -425,9 +425,10 @@ MOE_API int moe_streamed_layer_forward(moe_lfu* h, int layer, float* hres, int T
  *
  * Per layer, on each rank: norm, router, moe_bucket; all ranks' bucket
  * offsets gathered into all_offsets (int32 [G][E+1], rank r's row r, e.g. by
- * an all-gather); moe_ep_dispatch; a barrier across ranks; moe_ep_recv_plan
- * and moe_expert_forward over the received rows (k = 1, E/G experts);
- * moe_ep_return; a barrier; moe_combine of the rank's own y_pairs.
+ * an all-gather); moe_ep_dispatch (which also writes the rank's receiver
+ * plan); a barrier across ranks; moe_expert_forward over the received rows
+ * (k = 1, E/G experts); moe_ep_return; a barrier; moe_combine of the rank's
+ * own y_pairs.
  *
  * Receiver layout: rank d's received rows are ordered by its experts, then
  * by source rank, then by the source's bucket order.  With
@@ -449,31 +450,30 @@ MOE_API int moe_streamed_layer_forward(moe_lfu* h, int layer, float* hres, int T
  * with pair p = pairs[i], copies x row p / k (bf16 [H]) to row
  * base(e) + before(rank,e) + (i - off[e]) of recv_x[e/(E/G)] (bf16 [cap_rows, H])
  * and writes (rank, p) to the same row of recv_meta[...] (int32 [cap_rows, 2]),
- * e = idx[p].
+ * e = idx[p].  The same launch writes this rank's receiver plan (device):
+ * plan_offsets int32 [E/G + 1] = base(rank*E/G + j) clamped to cap_rows
+ * (plan_offsets[E/G] = rows received), plan_pairs int32 [cap_rows] = the
+ * identity over the rows received, plan_active int32 [E/G] = the local
+ * experts with rows, ascending, plan_n_active int32 [1]: the inputs of
+ * moe_expert_forward over recv_x with T = cap_rows, k = 1, E = E/G and this
+ * rank's blob table, once every rank's dispatch has completed.
  *   x        bf16 [T,H] (device): the layer input
  *   idx      int32 [T,k] (device) routing; pairs: from moe_bucket (device)
  *   all_offsets  int32 [G][E+1] (device)
  *   recv_x, recv_meta  host arrays [G] of peer device pointers
- * Ends with a system-scope fence, so the stores are visible to the peers once
- * the kernel has completed. */
+ * T = 0 still launches (the plan covers what the other ranks send).  The
+ * stores are complete when the kernel is; a barrier across ranks ordered
+ * after it on the stream makes them safe to read on the peers. */
 MOE_API int moe_ep_dispatch(const uint16_t* x, int T, int H, int k, int E, int G, int rank,
                             const int32_t* idx, const int32_t* pairs, const int32_t* all_offsets,
-                            void* const* recv_x, void* const* recv_meta, int cap_rows, void* stream);
-
-/* Receiver plan (rank `rank`): offsets int32 [E/G + 1] = base(rank*E/G + j)
- * clamped to cap_rows (offsets[E/G] = rows received), pairs int32 [cap_rows]
- * = the identity over the rows received, active int32 [E/G] = the local
- * experts with rows, ascending, and n_active int32 [1] (all device): the
- * inputs of moe_expert_forward over recv_x with T = cap_rows, k = 1,
- * E = E/G and this rank's blob table. */
-MOE_API int moe_ep_recv_plan(const int32_t* all_offsets, int G, int E, int rank, int cap_rows,
-                             int32_t* offsets, int32_t* pairs, int32_t* active, int32_t* n_active,
-                             void* stream);
+                            void* const* recv_x, void* const* recv_meta, int cap_rows,
+                            int32_t* plan_offsets, int32_t* plan_pairs, int32_t* plan_active,
+                            int32_t* plan_n_active, void* stream);
 
 /* Return (receiver rank `rank`): row r < offsets[E/G] of y_rows (fp32
  * [cap_rows, H], the expert outputs over the received rows) goes to row p of
  * y_pairs[s] (fp32 [n_pair_slots, H] on rank s), (s, p) = recv_meta[r].
- * Ends with a system-scope fence like the dispatch. */
+ * Completion as for the dispatch. */
 MOE_API int moe_ep_return(const float* y_rows, int H, int E, int G, int rank, const void* recv_meta,
                           const int32_t* offsets, int n_pair_slots, int cap_rows, void* const* y_pairs,
                           void* stream);

@@ -73,8 +73,7 @@ SIGNATURES = {
     "moe_streamed_layer_forward": (_I, [_P, _I, _P, _I, _I, _I, _I, _I, _I, C.POINTER(moe_qmat), _P, _I,
                                         C.POINTER(moe_qmat), _P, _P, _P, _P, _P, _Z, _I, _P, _P, _I]),
     "moe_ep_dispatch": (_I, [_P, _I, _I, _I, _I, _I, _I, _P, _P, _P, C.POINTER(C.c_void_p),
-                             C.POINTER(C.c_void_p), _I, _P]),
-    "moe_ep_recv_plan": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
+                             C.POINTER(C.c_void_p), _I, _P, _P, _P, _P, _P]),
     "moe_ep_return": (_I, [_P, _I, _I, _I, _I, _P, _P, _I, _I, C.POINTER(C.c_void_p), _P]),
     "moe_device_alloc": (_I, [_Z, C.POINTER(C.c_void_p)]),
     "moe_device_free": (_I, [_P]),

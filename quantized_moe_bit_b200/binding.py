@@ -239,16 +239,11 @@ def _peer_table(ptrs):
 
 
 def moe_ep_dispatch(x, k: int, E: int, G: int, rank: int, idx, pairs, all_offsets, recv_x, recv_meta,
-                    cap_rows: int, stream=None):
+                    cap_rows: int, plan_offsets, plan_pairs, plan_active, plan_n_active, stream=None):
     T, H = x.shape
     check(lib().moe_ep_dispatch(ptr(x), T, H, k, E, G, rank, ptr(idx), ptr(pairs), ptr(all_offsets),
-                                _peer_table(recv_x), _peer_table(recv_meta), cap_rows, stream_ptr(stream)))
-
-
-def moe_ep_recv_plan(all_offsets, G: int, E: int, rank: int, cap_rows: int, offsets, pairs, active, n_active,
-                     stream=None):
-    check(lib().moe_ep_recv_plan(ptr(all_offsets), G, E, rank, cap_rows, ptr(offsets), ptr(pairs), ptr(active),
-                                 ptr(n_active), stream_ptr(stream)))
+                                _peer_table(recv_x), _peer_table(recv_meta), cap_rows, ptr(plan_offsets),
+                                ptr(plan_pairs), ptr(plan_active), ptr(plan_n_active), stream_ptr(stream)))
 
 
 def moe_ep_return(y_rows, E: int, G: int, rank: int, recv_meta, offsets, n_pair_slots: int, y_pairs,

@@ -3,7 +3,10 @@
 // router, its shared expert and its combine.  Per layer two exchanges move
 // rows between ranks, each a kernel that stores straight into the peers'
 // buffers (NVLink peer mappings, or this GPU's own memory for the rank
-// itself), with no host round trip:
+// itself), with no host round trip.  The stores are complete when the kernel
+// is (the end of a grid flushes its writes system-wide, as for mapped host
+// memory), so a stream-ordered barrier across ranks after the kernel is what
+// orders them before any peer reads them; no fence inside the kernel:
 //   dispatch  the layer input row of every (token, slot) pair goes to the
 //             owner of the pair's expert, at a row computed on the device
 //             from every rank's bucket offsets;
@@ -73,45 +76,127 @@ __device__ int ep_block_exscan(int* v, int n, int* sc) {
 
 // tot[e] = sum over ranks of cnt(r, e) for e in [e0, e0 + n), and, when
 // before is non-NULL, before[e - e0] = sum over r < s of cnt(r, e) - off_s[e].
-__device__ void ep_counts(const int32_t* all_off, int G, int E, int s, int e0, int n, int* tot, int* before) {
+// A thread's loads of all ranks are issued together (one memory latency).
+__device__ void ep_counts(const int32_t* __restrict__ all_off, int G, int E, int s, int e0, int n, int* tot,
+                          int* before) {
   for (int j = threadIdx.x; j < n; j += blockDim.x) {
     const int e = e0 + j;
+    int lo[EP_MAX_G], hi[EP_MAX_G];
+#pragma unroll
+    for (int r = 0; r < EP_MAX_G; ++r) {
+      lo[r] = r < G ? __ldg(all_off + r * (E + 1) + e) : 0;
+      hi[r] = r < G ? __ldg(all_off + r * (E + 1) + e + 1) : 0;
+    }
     int t = 0, b = 0;
-    for (int r = 0; r < G; ++r) {
-      const int c = all_off[r * (E + 1) + e + 1] - all_off[r * (E + 1) + e];
-      t += c;
-      if (r < s) b += c;
+#pragma unroll
+    for (int r = 0; r < EP_MAX_G; ++r) {
+      t += hi[r] - lo[r];
+      if (r < s) b += hi[r] - lo[r];
     }
     tot[j] = t;
-    if (before) before[j] = b - all_off[s * (E + 1) + e];
+    if (before) before[j] = b - __ldg(all_off + s * (E + 1) + e);
   }
   __syncthreads();
 }
 
+constexpr int EP_NV = 12;   // 16-byte vectors per lane in one warp copy step (a 6 KB bf16 row)
+
+// One warp's copy step of vectors [b, b + 32 EP_NV) of a row: all loads of the
+// step are issued before its stores.
+__device__ __forceinline__ void ep_load(uint4 (&u)[EP_NV], const uint4* __restrict__ src, int n16, int b, int lane) {
+#pragma unroll
+  for (int j = 0; j < EP_NV; ++j) {
+    const int v = b + lane + 32 * j;
+    if (v < n16) u[j] = __ldg(src + v);
+  }
+}
+__device__ __forceinline__ void ep_store(uint4* dst, const uint4 (&u)[EP_NV], int n16, int b, int lane) {
+#pragma unroll
+  for (int j = 0; j < EP_NV; ++j) {
+    const int v = b + lane + 32 * j;
+    if (v < n16) dst[v] = u[j];
+  }
+}
+
+// Receiver plan of rank d, by one CTA: its bucket offsets [El + 1] over the
+// rows it receives (clamped to the capacity), the identity pair list of
+// those rows and the non-empty local experts ascending with their count --
+// the inputs of the grouped expert GEMM with k = 1.  sm: 2 (El + 1) +
+// EP_THREADS / 32 + 1 ints.
+__device__ void ep_recv_plan_block(const int32_t* __restrict__ all_off, int G, int E, int d, int cap_rows,
+                                   int32_t* __restrict__ offsets, int32_t* __restrict__ pairs,
+                                   int32_t* __restrict__ active, int32_t* __restrict__ n_active, int* sm) {
+  const int El = E / G;
+  int* tot = sm;
+  int* flg = sm + El + 1;
+  int* sc = sm + 2 * (El + 1);
+  ep_counts(all_off, G, E, d, d * El, El, tot, nullptr);
+  for (int j = threadIdx.x; j < El; j += blockDim.x) flg[j] = tot[j] > 0;
+  __syncthreads();
+  const int R = ep_block_exscan(tot, El, sc);
+  const int na = ep_block_exscan(flg, El, sc);
+  for (int j = threadIdx.x; j < El; j += blockDim.x) {
+    offsets[j] = tot[j] < cap_rows ? tot[j] : cap_rows;
+    const int nxt = j + 1 < El ? flg[j + 1] : na;
+    if (nxt > flg[j]) active[flg[j]] = j;
+  }
+  if (threadIdx.x == 0) {
+    offsets[El] = R < cap_rows ? R : cap_rows;
+    n_active[0] = na;
+    if (R > cap_rows) flag_check(CHECK_EP_ROW);   // rows past the capacity were not stored
+  }
+  const int rows = R < cap_rows ? R : cap_rows;
+  for (int r = threadIdx.x; r < rows; r += blockDim.x) pairs[r] = r;
+}
+
 // Source rank s: every bucketed slot's layer input row (bf16 [H]) and its
-// (source, pair index) go to the owner of its expert.  One warp per slot.
+// (source, pair index) go to the owner of its expert, one warp per slot.  A
+// warp's first row is loaded before the CTA builds its row table (the load
+// does not depend on it).  The grid's last block writes rank s's own
+// receiver plan meanwhile.
+// sm: 2 (E + 1) + EP_THREADS / 32 + 1 ints.
 __global__ void __launch_bounds__(EP_THREADS) k_ep_dispatch(const uint16_t* __restrict__ x, int H, int k,
                                                             const int32_t* __restrict__ idx,
                                                             const int32_t* __restrict__ pairs,
                                                             const int32_t* __restrict__ all_off, int G, int E, int s,
-                                                            EpPeers recv_x, EpPeers recv_meta, int cap_rows) {
+                                                            EpPeers recv_x, EpPeers recv_meta, int cap_rows,
+                                                            int n_slots, int32_t* plan_offsets, int32_t* plan_pairs,
+                                                            int32_t* plan_active, int32_t* plan_n_active) {
   extern __shared__ int ep_sm[];
-  int* tot = ep_sm;              // [E] -> base (segmented scan, each owner's range from 0)
-  int* pos0 = ep_sm + E;         // [E] before(s, e) - off_s[e]
-  int* sc = ep_sm + 2 * E;
+  int* tot = ep_sm;              // [E] -> the scan of the totals
+  int* pos0 = ep_sm + E + 1;     // [E] row of slot i of bucket e = pos0[e] + i
+  int* sc = ep_sm + 2 * (E + 1);
   const int El = E / G;
-  ep_counts(all_off, G, E, s, 0, E, tot, pos0);
-  // base(e): the scan over all experts minus its value at the owner's first expert
-  int* scan = tot;
-  ep_block_exscan(scan, E, sc);
-  for (int e = threadIdx.x; e < E; e += blockDim.x) pos0[e] += scan[e] - scan[(e / El) * El];
-  __syncthreads();
-  const int n = all_off[s * (E + 1) + E];
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
-  const int nv = H / 8;                      // 16-byte vectors per row
-  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < n; i += gridDim.x * wpb) {
-    const int p = pairs[i];
+  const int nv = H / 8;          // 16-byte vectors per row
+  int n = all_off[s * (E + 1) + E];
+  if (n < 0 || n > n_slots) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) flag_check(CHECK_PAIR_ID);
+    n = n < 0 ? 0 : n_slots;
+  }
+  if (blockIdx.x == gridDim.x - 1) {   // the plan block copies nothing
+    ep_recv_plan_block(all_off, G, E, s, cap_rows, plan_offsets, plan_pairs, plan_active, plan_n_active, ep_sm);
+    return;
+  }
+  const int ncopy = gridDim.x - 1;    // copying blocks
+  int i = blockIdx.x * wpb + (threadIdx.x >> 5);
+  uint4 u[EP_NV];
+  int p0 = -1;
+  if (i < n) {
+    p0 = pairs[i];
+    if (p0 >= 0 && p0 < n_slots) ep_load(u, reinterpret_cast<const uint4*>(x + static_cast<size_t>(p0 / k) * H), nv, 0, lane);
+  }
+  ep_counts(all_off, G, E, s, 0, E, tot, pos0);
+  ep_block_exscan(tot, E, sc);   // base(e) = tot[e] - tot[first expert of e's owner]
+  for (int e = threadIdx.x; e < E; e += blockDim.x) pos0[e] += tot[e] - tot[(e / El) * El];
+  __syncthreads();
+  for (bool first = true; i < n; i += ncopy * wpb, first = false) {
+    const int p = first ? p0 : pairs[i];
+    if (p < 0 || p >= n_slots) {
+      if (lane == 0) flag_check(CHECK_PAIR_ID);
+      continue;
+    }
     const int e = idx[p];
     if (e < 0 || e >= E) {
       if (lane == 0) flag_check(CHECK_EXPERT_ID);
@@ -125,43 +210,17 @@ __global__ void __launch_bounds__(EP_THREADS) k_ep_dispatch(const uint16_t* __re
     }
     const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(p / k) * H);
     uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(recv_x.p[d]) + static_cast<size_t>(row) * H);
-    for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
+    int b = 0;
+    if (first) {
+      ep_store(dst, u, nv, 0, lane);
+      b = 32 * EP_NV;
+    }
+    for (; b < nv; b += 32 * EP_NV) {
+      ep_load(u, src, nv, b, lane);
+      ep_store(dst, u, nv, b, lane);
+    }
     if (lane == 0) static_cast<int2*>(recv_meta.p[d])[row] = make_int2(s, p);
   }
-  __threadfence_system();
-}
-
-// Receiver rank d: its bucket offsets [El + 1] over the rows it received,
-// the identity pair list of those rows, and the non-empty experts ascending
-// with their count -- the inputs of the grouped expert GEMM with k = 1.
-__global__ void __launch_bounds__(EP_THREADS) k_ep_recv_plan(const int32_t* __restrict__ all_off, int G, int E,
-                                                             int d, int cap_rows, int32_t* __restrict__ offsets,
-                                                             int32_t* __restrict__ pairs, int32_t* __restrict__ active,
-                                                             int32_t* __restrict__ n_active) {
-  extern __shared__ int ep_sm[];
-  const int El = E / G;
-  int* tot = ep_sm;              // [El + 1]
-  int* flg = ep_sm + El + 1;     // [El + 1]
-  int* sc = ep_sm + 2 * (El + 1);
-  ep_counts(all_off, G, E, d, d * El, El, tot, nullptr);
-  for (int j = threadIdx.x; j < El; j += blockDim.x) flg[j] = tot[j] > 0;
-  __syncthreads();
-  const int R = ep_block_exscan(tot, El, sc);
-  const int na = ep_block_exscan(flg, El, sc);
-  // offsets clamped to the capacity (rows past it were not stored; the
-  // check word reports it)
-  for (int j = threadIdx.x; j < El; j += blockDim.x) {
-    offsets[j] = tot[j] < cap_rows ? tot[j] : cap_rows;
-    const int nxt = j + 1 < El ? flg[j + 1] : na;
-    if (nxt > flg[j]) active[flg[j]] = j;
-  }
-  if (threadIdx.x == 0) {
-    offsets[El] = R < cap_rows ? R : cap_rows;
-    n_active[0] = na;
-    if (R > cap_rows) flag_check(CHECK_EP_ROW);
-  }
-  const int rows = R < cap_rows ? R : cap_rows;
-  for (int r = threadIdx.x; r < rows; r += blockDim.x) pairs[r] = r;
 }
 
 // Receiver rank d: expert output row r (fp32 [H]) goes back to its source
@@ -183,9 +242,12 @@ __global__ void __launch_bounds__(EP_THREADS) k_ep_return(const float* __restric
     }
     const uint4* src = reinterpret_cast<const uint4*>(y_rows + static_cast<size_t>(r) * H);
     uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(y_pairs.p[m.x]) + static_cast<size_t>(m.y) * H);
-    for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
+    uint4 u[EP_NV];
+    for (int b = 0; b < nv; b += 32 * EP_NV) {
+      ep_load(u, src, nv, b, lane);
+      ep_store(dst, u, nv, b, lane);
+    }
   }
-  __threadfence_system();
 }
 
 }  // namespace moe
@@ -216,37 +278,29 @@ extern "C" {
 
 int moe_ep_dispatch(const uint16_t* x, int T, int H, int k, int E, int G, int rank, const int32_t* idx,
                     const int32_t* pairs, const int32_t* all_offsets, void* const* recv_x, void* const* recv_meta,
-                    int cap_rows, void* stream) {
+                    int cap_rows, int32_t* plan_offsets, int32_t* plan_pairs, int32_t* plan_active,
+                    int32_t* plan_n_active, void* stream) {
   int st = ep_check(T, H, k, E, G, rank, "moe_ep_dispatch");
   if (st) return st;
   if (cap_rows < 0) return fail(MOE_ERR_INVALID_ARG, "moe_ep_dispatch: cap_rows < 0");
   if (!x || !idx || !pairs || !all_offsets) return fail(MOE_ERR_INVALID_ARG, "moe_ep_dispatch: NULL pointer");
+  if (!plan_offsets || !plan_pairs || !plan_active || !plan_n_active)
+    return fail(MOE_ERR_INVALID_ARG, "moe_ep_dispatch: NULL plan output");
   if (!aligned16(x)) return fail(MOE_ERR_INVALID_ARG, "moe_ep_dispatch: misaligned x");
   EpPeers px, pm;
   if ((st = ep_peers(recv_x, G, &px, "moe_ep_dispatch"))) return st;
   if ((st = ep_peers(recv_meta, G, &pm, "moe_ep_dispatch"))) return st;
-  if (T == 0) return MOE_OK;
+  // T = 0 still launches: the rank's receiver plan covers the rows other
+  // ranks send it
   const int slots = T * k, wpb = EP_THREADS / 32;
   int grid = (slots + wpb - 1) / wpb;
   if (grid > 4 * 148) grid = 4 * 148;
-  const size_t smem = (2 * static_cast<size_t>(E) + EP_THREADS / 32 + 1) * sizeof(int);
-  k_ep_dispatch<<<grid, EP_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(x, H, k, idx, pairs, all_offsets, G, E,
-                                                                                rank, px, pm, cap_rows);
+  grid += 1;                            // the plan block
+  const size_t smem = (2 * static_cast<size_t>(E + 1) + EP_THREADS / 32 + 1) * sizeof(int);
+  k_ep_dispatch<<<grid, EP_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(
+      x, H, k, idx, pairs, all_offsets, G, E, rank, px, pm, cap_rows, slots, plan_offsets, plan_pairs, plan_active,
+      plan_n_active);
   return launch_check("k_ep_dispatch");
-}
-
-int moe_ep_recv_plan(const int32_t* all_offsets, int G, int E, int rank, int cap_rows, int32_t* offsets,
-                     int32_t* pairs, int32_t* active, int32_t* n_active, void* stream) {
-  int st = ep_check(0, 64, 1, E, G, rank, "moe_ep_recv_plan");
-  if (st) return st;
-  if (cap_rows < 0) return fail(MOE_ERR_INVALID_ARG, "moe_ep_recv_plan: cap_rows < 0");
-  if (!all_offsets || !offsets || !pairs || !active || !n_active)
-    return fail(MOE_ERR_INVALID_ARG, "moe_ep_recv_plan: NULL pointer");
-  const int El = E / G;
-  const size_t smem = (2 * static_cast<size_t>(El + 1) + EP_THREADS / 32 + 1) * sizeof(int);
-  k_ep_recv_plan<<<1, EP_THREADS, smem, static_cast<cudaStream_t>(stream)>>>(all_offsets, G, E, rank, cap_rows,
-                                                                             offsets, pairs, active, n_active);
-  return launch_check("k_ep_recv_plan");
 }
 
 int moe_ep_return(const float* y_rows, int H, int E, int G, int rank, const void* recv_meta, const int32_t* offsets,

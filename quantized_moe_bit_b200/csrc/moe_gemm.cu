@@ -282,7 +282,10 @@ __global__ void __launch_bounds__(256) k_gm_prep(const uint16_t* __restrict__ x,
   // gather, a row per block and step (the row's source looked up once): 8
   // values (16 bytes) per thread, all of a thread's loads of the row first
   const int w8 = H / 8;
-  const int P = routed ? T * k : 0;
+  // routed rows: the bucketed pairs only; pair slots past offsets[E] belong
+  // to no chunk (a caller may size T for more rows than it bucketed)
+  int P = routed ? offsets[E] : 0;
+  if (P < 0 || P > T * k) P = routed ? T * k : 0;
   const int nrow = P + (xh ? T : 0);
   for (int row = blockIdx.x; row < nrow; row += gridDim.x) {
     int t;

@@ -7,8 +7,9 @@ Per layer (`ep_layer_forward`):
     front      moe_rmsnorm, moe_router_topk, moe_bucket, moe_shared_forward
     gather     every rank's bucket offsets into all_offsets [G, E+1]
     dispatch   moe_ep_dispatch: input rows stored into the owners' recv_x
+               (and the rank's own receiver plan written)
     barrier
-    experts    moe_ep_recv_plan, moe_expert_forward (k = 1, E/G experts),
+    experts    moe_expert_forward (k = 1, E/G experts) over the received rows,
                moe_ep_return: output rows stored into the sources' y_pairs
     barrier
     combine    moe_combine into the rank's residual stream
@@ -141,11 +142,10 @@ class EpRank:
 
     def dispatch(self):
         B.moe_ep_dispatch(self.x, self.k, self.E, self.G, self.rank, self.idx, self.pairs, self.all_off,
-                          self.peer_recv_x, self.peer_recv_meta, self.cap)
+                          self.peer_recv_x, self.peer_recv_meta, self.cap, self.loff, self.rpairs, self.ractive,
+                          self.rn)
 
     def experts(self, flags: int = 0):
-        B.moe_ep_recv_plan(self.all_off, self.G, self.E, self.rank, self.cap, self.loff, self.rpairs, self.ractive,
-                           self.rn)
         B.moe_expert_forward(self.recv_x[:self.cap], self.I, self.El, 1, self.local_blobs, self.loff, self.rpairs,
                              self.ractive, self.rn, self.y_rows, self.ws_e, flags=flags)
         B.moe_ep_return(self.y_rows[:self.cap], self.E, self.G, self.rank, self.recv_meta, self.loff, self.T * self.k,

@@ -175,7 +175,7 @@ def test_expert_parallel_argument_checks():
     T, H, k, E = 4, 2816, 8, 128
     peers = lambda n, bad=None: (C.c_void_p * 8)(*[(bad if i == 0 and bad is not None else f) for i in range(n)])  # noqa: E731
     ok2 = peers(2)
-    d = lambda *a: L.moe_ep_dispatch(*a)  # noqa: E731
+    d = lambda *a: L.moe_ep_dispatch(*a[:-1], f, f, f, f, None)  # noqa: E731  (plan outputs, stream)
     assert d(f, T, H, k, E, 0, 0, f, f, f, ok2, ok2, 64, None) == _INVALID               # G = 0
     assert d(f, T, H, k, E, 9, 0, f, f, f, peers(8), peers(8), 64, None) == _INVALID      # G > 8
     assert d(f, T, H, k, 24, 2, 0, f, f, f, ok2, ok2, 64, None) == _INVALID              # E/G = 12
@@ -185,9 +185,7 @@ def test_expert_parallel_argument_checks():
     assert d(f + 2, T, H, k, E, 2, 0, f, f, f, ok2, ok2, 64, None) == _INVALID           # misaligned x
     assert d(f, T, H, k, E, 2, 0, f, f, f, None, ok2, 64, None) == _INVALID              # no table
     assert d(f, T, H, k, E, 2, 0, f, f, f, ok2, ok2, -1, None) == _INVALID               # capacity
-    assert d(f, 0, H, k, E, 2, 1, f, f, f, ok2, ok2, 0, None) == _OK                     # T = 0
-    assert L.moe_ep_recv_plan(f, 2, E, 5, 64, f, f, f, f, None) == _INVALID              # rank >= G
-    assert L.moe_ep_recv_plan(f, 2, E, 1, 64, None, f, f, f, None) == _INVALID
+    assert L.moe_ep_dispatch(f, T, H, k, E, 2, 0, f, f, f, ok2, ok2, 64, None, f, f, f, None) == _INVALID  # plan
     assert L.moe_ep_return(f, H, E, 2, 0, f, f, 32, 64, peers(2, 0), None) == _INVALID   # NULL peer
     assert L.moe_ep_return(f, H, E, 2, 0, f + 4, f, 32, 64, ok2, None) == _INVALID       # meta alignment
     assert L.moe_ep_return(f, H, E, 2, 0, f, f, 32, 0, ok2, None) == _OK                 # nothing received

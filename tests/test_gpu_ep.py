@@ -66,7 +66,7 @@ def _run_layers(M, cfg, G, layers, z_by_rank, bias_override=None):
             lg = O.router_logits(x, hls[l].router, hls[l].bias)
             check_routing(idx, lg, c.k)
             ref = O.layer_forward(x, hls[l].router, hls[l].bias, hls[l].expert, hls[l].shared, c.k, c.E, idx=idx)
-            check_close(_np(r.gates), ref["gates"], 2e-6, 2e-6, f"gates l{l} r{g}")
+            assert np.abs(_np(r.gates) - ref["gates"]).max() < 2e-6, f"gates l{l} r{g}"
             check_output(_bits(r.y), ref["out"], f"y l{l} r{g}")
             check_close(_np(hs[g]), before[g] + ref["out"], 2e-3, 2e-4, f"h l{l} r{g}")
         # every pair of every rank was received exactly once
@@ -82,7 +82,9 @@ def test_ep_local_ranks_tiny(M, G):
     zs = [gen.rows(cfg.seed, 1000 + g, cfg.T, cfg.H) for g in range(G)]
     rec = _run_layers(M, cfg, G, 2, zs)
     if G > 1:
-        assert all(n > 0 for n in rec[0])
+        # several owners received rows (with the Zipf routing skew some of
+        # the 8-expert ranges may stay empty)
+        assert sum(n > 0 for n in rec[0]) >= 2
 
 
 @pytest.mark.parametrize("G,T", [(4, 16), (8, 16)])
