@@ -309,19 +309,26 @@ def run_streamed_lfu(M, device):
     prompt = gen.rows(c.seed, 3000, c.prompt_tokens, c.H)
     dec = [gen.rows(c.seed, 4000 + d, 1, c.H) for d in range(c.decode_steps)]
     units = [(torch.from_numpy(prompt[i:i + c.T]).to(device), i) for i in range(0, c.prompt_tokens, c.T)]
-    units += [(torch.from_numpy(dec[d]).to(device), c.prompt_tokens + d) for d in range(c.decode_steps)]
+    dec_units = [(torch.from_numpy(dec[d]).to(device), c.prompt_tokens + d) for d in range(c.decode_steps)]
+    units += dec_units
+    # layer-major prompt: the whole prompt as one call per layer (each layer's
+    # distinct experts staged about once), the same decode steps after it
+    units_lm = [(torch.from_numpy(prompt).to(device), 0)] + dec_units
     for l in range(c.layers):                   # biases built before the timed region
-        for z, t0 in units:
+        for z, t0 in units + units_lm[:1]:
             bias(l, t0, z.shape[0])
     side = torch.cuda.Stream(device=device)
     main = torch.cuda.current_stream()
     ws = {T: torch.empty(M.moe_streamed_workspace_size(T, c.H, c.I, c.Is, c.E, c.k), dtype=torch.uint8,
-                         device=device) for T in (c.T, 1)}
-    n_pre = c.prompt_tokens // c.T
+                         device=device) for T in (c.T, 1, c.prompt_tokens)}
 
-    def arm(prefetch: int):
+    def arm(prefetch: int, layer_major: bool = False):
         """One run of the workload on a fresh cache (lookahead prefetch of
-        `prefetch` experts per layer call, 0: off)."""
+        `prefetch` experts per layer call, 0: off; the prompt in chunks of
+        128 rows, each through all layers, or layer-major: the whole prompt
+        through each layer in one call)."""
+        us_all = units_lm if layer_major else units
+        n_pre = 1 if layer_major else c.prompt_tokens // c.T
         lfu = M.MoeLfu(c.layers, c.E, c.n_slots, gen.blob_bytes(c.H, c.I), host_ptrs, pool, stride)
         lfu.set_prefetch(prefetch)
 
@@ -336,9 +343,9 @@ def run_streamed_lfu(M, device):
         torch.cuda.synchronize()
         e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
         e0.record()
-        run(units[:n_pre])
+        run(us_all[:n_pre])
         e1.record()
-        run(units[n_pre:])
+        run(us_all[n_pre:])
         e2.record()
         torch.cuda.synchronize()
         M.moe_sync()
@@ -346,11 +353,13 @@ def run_streamed_lfu(M, device):
         hits, misses, nbytes = lfu.stats()
         staged = sum(1 for r in lfu.log() if r[3] == 2)
         lfu.close()
-        return {"prefetch_per_call": prefetch, "prefill_tokens_per_s": c.prompt_tokens / t_pre,
+        return {"prefetch_per_call": prefetch, "prompt": "layer-major" if layer_major else f"chunks of {c.T}",
+                "prefill_tokens_per_s": c.prompt_tokens / t_pre,
                 "decode_tokens_per_s": c.decode_steps / t_dec, "prefill_s": t_pre, "decode_s": t_dec,
                 "hits": hits, "misses": misses, "prefetched": staged, "h2d_bytes": nbytes,
                 "h2d_gbs_while_streaming": nbytes / (t_pre + t_dec) / 1e9}
     runs = [arm(p) for p in (0, 2, 0, 2)]           # the two arms alternately, twice
+    lm = [arm(0, True), arm(0, True)]
     base = runs[0]
     # pinned host -> device copy bandwidth of this machine, for context
     buf = host.view(-1)[: 256 << 20]
@@ -367,6 +376,9 @@ def run_streamed_lfu(M, device):
             "pinned_h2d_copy_gbs": h2d, "slots_per_layer": c.n_slots,
             "prefetch_ab": {"arms": "lookahead prefetch off (0) and on (2 experts per layer call), run alternately",
                             "runs": runs},
+            "layer_major": {"prompt": f"all {c.prompt_tokens} prompt rows through each layer in one call "
+                                      "(layer-major), then the same decode steps; prefetch off",
+                            "runs": lm},
             "note": "bitwise equality with the all-resident run and the LFU log are checked by the GPU tests"}
 
 

@@ -186,6 +186,25 @@ def test_streamed_full(M, prefetch):
     print(f"streamed_30L_lfu prefetch {prefetch}: hits {hits} misses {misses}")
 
 
+def test_streamed_layer_major_tiny(M):
+    """The whole prompt through each layer in one call (layer-major): equal
+    to the all-resident run of the same units bit for bit, the log equal to
+    the simulator's, and fewer misses than the same prompt in chunks."""
+    chunked = replace(tiny_config("streamed_30L_lfu"), layers=4, T=12, prompt_tokens=48, decode_steps=6, n_slots=6)
+    _, miss_chunked = _run_all(M, chunked, samples=[(0, 0)])
+    cfg = replace(chunked, T=48)
+    hits, misses = _run_all(M, cfg, samples=[(0, 0), (0, 3), (1, 2), (6, 1)])
+    assert misses < miss_chunked
+
+
+def test_streamed_layer_major_full(M):
+    """The full streamed workload with its 1024-token prompt through each of
+    the 30 layers in one call, then the 128 decode steps."""
+    cfg = replace(CONFIGS["streamed_30L_lfu"], T=1024)
+    hits, misses = _run_all(M, cfg, samples=[(1, 0), (60, 17), (128, 29)])
+    print(f"streamed_30L_lfu layer-major prompt: hits {hits} misses {misses}")
+
+
 def test_lfu_host_faults(M):
     cfg = replace(tiny_config("streamed_30L_lfu"), layers=2, T=8, prompt_tokens=8, decode_steps=0, n_slots=4)
     S = Streamed(M, cfg)
