@@ -75,6 +75,18 @@ struct moe_lfu {
   // streamed layer forward: per-layer "slots read" events, pinned staging
   std::vector<cudaEvent_t> consumed;          // [L] recorded after the expert kernels of a layer
   cudaEvent_t done = nullptr, idx_ready = nullptr, stage_free = nullptr;
+  // The kernels that last read each slot (streamed layer forward): read_ev is
+  // a ring of events recorded on the main stream after a step's expert
+  // kernels, read_seq counts the steps recorded, slot_read[l*S+s] is the
+  // read_seq of the last step that read slot s (-1: not known, wait for all
+  // of the layer's kernels).  A copy into a slot waits only for that event;
+  // an event re-recorded by a later step only makes the wait longer.
+  static constexpr int READ_RING = 64;
+  std::vector<cudaEvent_t> read_ev;           // [READ_RING]
+  int64_t read_seq = 0;
+  int64_t read_done = 0;                      // every step below this one is known complete
+  cudaStream_t read_stream = nullptr;         // the stream the read events were recorded on
+  std::vector<int64_t> slot_read;             // [L*S]
   int32_t* pin_idx = nullptr;                 // pinned [cap_rows * 8]
   int32_t* pin_act = nullptr;                 // pinned [groups * (E + 1)]
   int cap_rows = 0;
@@ -130,6 +142,8 @@ int txn_rollback(moe_lfu* h, int status) {
   h->log.resize(h->snap_log);
   if (!h->dirty.empty())
     for (int32_t s : h->txn_written) h->dirty[b + s] = 1;
+  if (!h->slot_read.empty())
+    for (int s = 0; s < h->S; ++s) h->slot_read[b + s] = -1;
   h->txn_written.clear();
   h->txn_depth = 0;
   return status;
@@ -276,6 +290,10 @@ MOE_API int moe_lfu_create(int n_layers, int n_experts, int n_slots, size_t blob
     ok = ok && cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming) == cudaSuccess;
     ok = ok && cudaEventCreateWithFlags(&h->idx_ready, cudaEventDisableTiming) == cudaSuccess;
     ok = ok && cudaEventCreateWithFlags(&h->stage_free, cudaEventDisableTiming) == cudaSuccess;
+    h->read_ev.assign(moe_lfu::READ_RING, nullptr);
+    for (int i = 0; i < moe_lfu::READ_RING && ok; ++i)
+      ok = cudaEventCreateWithFlags(&h->read_ev[i], cudaEventDisableTiming) == cudaSuccess;
+    h->slot_read.assign(static_cast<size_t>(n_layers) * n_slots, -1);
     void* p = nullptr;
     ok = ok && cudaHostAlloc(&p, sizeof(int32_t) * (n_experts + 1) * (n_experts + 1), 0) == cudaSuccess;
     h->pin_act = static_cast<int32_t*>(p);
@@ -298,8 +316,14 @@ MOE_API int moe_lfu_plan(moe_lfu* h, int layer, const int32_t* ids, int n, int32
   return st;
 }
 
-MOE_API int moe_lfu_step(moe_lfu* h, int layer, const int32_t* ids, int n, void* side_stream, void* wait_event_,
-                         void* done_event, void** dev_table, int timeout_ms) {
+namespace {
+
+// One step.  per_slot = false: every copy waits for wait_event (the public
+// call).  per_slot = true (the streamed layer forward): a copy waits only for
+// the kernels that last read its slot, and the device table copy (read by the
+// previous step's kernels) waits for wait_event.  slots_out: the step's slots.
+int lfu_step_impl(moe_lfu* h, int layer, const int32_t* ids, int n, void* side_stream, void* wait_event_,
+                  bool per_slot, void* done_event, void** dev_table, int timeout_ms, int32_t* slots_out) {
   if (!h || !h->pool) return moe::fail(MOE_ERR_INVALID_ARG, "lfu_step: handle has no slot pool");
   if (n > 0 && !ids) return moe::fail(MOE_ERR_INVALID_ARG, "lfu_step: NULL ids");
   if (!dev_table || !done_event) return moe::fail(MOE_ERR_INVALID_ARG, "lfu_step: NULL table or event");
@@ -307,19 +331,38 @@ MOE_API int moe_lfu_step(moe_lfu* h, int layer, const int32_t* ids, int n, void*
   if (h->txn_depth > 0 && h->txn_layer != layer)
     return moe::fail(MOE_ERR_INVALID_ARG, "lfu_step: layer %d inside a call on layer %d", layer, h->txn_layer);
   cudaStream_t s = static_cast<cudaStream_t>(side_stream);
+  cudaEvent_t wait_all = static_cast<cudaEvent_t>(wait_event_);
   std::vector<int32_t> slots(n), hit(n, 0);
   txn_begin(h, layer);
   int st = plan(h, layer, ids, n, slots.data(), hit.data());
   if (st) return txn_rollback(h, st);
-  // slots are overwritten only after the kernels that read them are done
-  if (wait_event_ && (st = moe::cuda_check(cudaStreamWaitEvent(s, static_cast<cudaEvent_t>(wait_event_), 0),
-                                           "lfu_step: wait")))
-    return txn_rollback(h, st);
   const size_t base = static_cast<size_t>(layer) * h->S;
+  auto needs_copy = [&](int i) { return !hit[i] || h->dirty[base + slots[i]]; };
+  // slots are overwritten only after the kernels that read them are done
+  if (!per_slot || h->slot_read.empty()) {
+    if (wait_all && (st = moe::cuda_check(cudaStreamWaitEvent(s, wait_all, 0), "lfu_step: wait")))
+      return txn_rollback(h, st);
+  } else {
+    std::vector<char> waited(moe_lfu::READ_RING, 0);
+    bool all = false;
+    for (int i = 0; i < n && !all; ++i) {
+      if (!needs_copy(i)) continue;
+      const int64_t q = h->slot_read[base + slots[i]];
+      if (q < 0) { all = true; break; }
+      if (q < h->read_done) continue;         // its kernels have finished
+      const int r = static_cast<int>(q % moe_lfu::READ_RING);
+      if (waited[r]) continue;
+      waited[r] = 1;
+      if ((st = moe::cuda_check(cudaStreamWaitEvent(s, h->read_ev[r], 0), "lfu_step: wait slot reader")))
+        return txn_rollback(h, st);
+    }
+    if (all && wait_all && (st = moe::cuda_check(cudaStreamWaitEvent(s, wait_all, 0), "lfu_step: wait")))
+      return txn_rollback(h, st);
+  }
   for (int i = 0; i < n; ++i) {
     unsigned char* slot = h->pool + (base + slots[i]) * h->slot_stride;
     // a miss, or a hit on a slot that a rolled-back call overwrote
-    if (!hit[i] || h->dirty[base + slots[i]]) {
+    if (needs_copy(i)) {
       ++h->copies;
       if (h->fault_kind == MOE_LFU_FAULT_COPY_FAILS && h->fault_after >= 0 && h->copies > h->fault_after)
         return txn_rollback(h, moe::fail(MOE_ERR_CUDA, "lfu_step: injected copy failure (copy %ld)", h->copies));
@@ -334,6 +377,9 @@ MOE_API int moe_lfu_step(moe_lfu* h, int layer, const int32_t* ids, int n, void*
       h->bytes_copied += static_cast<int64_t>(h->blob_bytes);
     }
   }
+  // the device table is read by the previous step's kernels
+  if (per_slot && wait_all && (st = moe::cuda_check(cudaStreamWaitEvent(s, wait_all, 0), "lfu_step: wait table")))
+    return txn_rollback(h, st);
   // the pinned table mirror may still feed the previous copy of this layer's table
   if ((st = wait_event(h->mirror_ev[layer], timeout_ms))) return txn_rollback(h, st);
   for (int i = 0; i < n; ++i)
@@ -345,8 +391,23 @@ MOE_API int moe_lfu_step(moe_lfu* h, int layer, const int32_t* ids, int n, void*
     return txn_rollback(h, st);
   if ((st = moe::cuda_check(cudaEventRecord(static_cast<cudaEvent_t>(done_event), s), "lfu_step: done event")))
     return txn_rollback(h, st);
+  if (slots_out)
+    for (int i = 0; i < n; ++i) slots_out[i] = slots[i];
   txn_commit(h);
   return MOE_OK;
+}
+
+}  // namespace
+
+MOE_API int moe_lfu_step(moe_lfu* h, int layer, const int32_t* ids, int n, void* side_stream, void* wait_event_,
+                         void* done_event, void** dev_table, int timeout_ms) {
+  std::vector<int32_t> sl(n > 0 ? n : 0);
+  const int st = lfu_step_impl(h, layer, ids, n, side_stream, wait_event_, false, done_event, dev_table, timeout_ms,
+                               sl.data());
+  // the caller's kernels read these slots, ordered by the caller's own events
+  if (st == MOE_OK && !h->slot_read.empty())
+    for (int i = 0; i < n; ++i) h->slot_read[static_cast<size_t>(layer) * h->S + sl[i]] = -1;
+  return st;
 }
 
 MOE_API int moe_lfu_wait(void* event, int timeout_ms) {
@@ -405,6 +466,7 @@ MOE_API int moe_lfu_destroy(moe_lfu* h) {
   if (!h) return MOE_OK;
   for (cudaEvent_t e : h->consumed) if (e) { cudaEventSynchronize(e); cudaEventDestroy(e); }
   for (cudaEvent_t e : {h->done, h->idx_ready, h->stage_free}) if (e) { cudaEventSynchronize(e); cudaEventDestroy(e); }
+  for (cudaEvent_t e : h->read_ev) if (e) { cudaEventSynchronize(e); cudaEventDestroy(e); }
   if (h->pin_idx) cudaFreeHost(h->pin_idx);
   if (h->pin_act) cudaFreeHost(h->pin_act);
   for (size_t l = 0; l < h->mirror.size(); ++l) {
@@ -476,6 +538,15 @@ MOE_API int moe_streamed_layer_forward(moe_lfu* h, int layer, float* hres, int T
   if ((st = moe::cuda_check(cudaEventRecord(h->idx_ready, ms), "streamed: record"))) return st;
   if ((st = moe_shared_forward(x, T, H, Is, shared, ysh, sw, sws, flags, ms))) return st;
   if ((st = wait_event(h->idx_ready, timeout_ms))) return st;
+  // the routing follows every earlier step's kernels on the main stream, when
+  // they were issued on this same stream; readers recorded on another stream
+  // are forgotten (their slots then wait for the layer's last kernels)
+  if (ms == h->read_stream) {
+    h->read_done = h->read_seq;
+  } else {
+    h->read_stream = ms;
+    std::fill(h->slot_read.begin(), h->slot_read.end(), -1);
+  }
   // steps: one token's ids in selection order, or the chunk's distinct experts,
   // resident ones first (ascending), then the rest (ascending), k at a time
   std::vector<std::vector<int32_t>> steps;
@@ -509,7 +580,9 @@ MOE_API int moe_streamed_layer_forward(moe_lfu* h, int layer, float* hres, int T
   for (size_t g = 0; g < steps.size(); ++g) {
     const auto& ids = steps[g];
     const int n = static_cast<int>(ids.size());
-    if ((st = moe_lfu_step(h, layer, ids.data(), n, side_stream, h->consumed[layer], h->done, dev_table, timeout_ms)))
+    std::vector<int32_t> sl(n);
+    if ((st = lfu_step_impl(h, layer, ids.data(), n, side_stream, h->consumed[layer], true, h->done, dev_table,
+                            timeout_ms, sl.data())))
       return abort_call(st);
     if ((st = moe::cuda_check(cudaStreamWaitEvent(ms, h->done, 0), "streamed: wait copies"))) return abort_call(st);
     int32_t* pa = h->pin_act + g * (E + 1);
@@ -524,6 +597,15 @@ MOE_API int moe_streamed_layer_forward(moe_lfu* h, int layer, float* hres, int T
       return abort_call(st);
     if ((st = moe::cuda_check(cudaEventRecord(h->consumed[layer], ms), "streamed: record consumed")))
       return abort_call(st);
+    // this step's kernels read its slots; the last step's event is never
+    // waited for (the next call's routing wait covers it), so it is not
+    // recorded
+    const int r = static_cast<int>(h->read_seq % moe_lfu::READ_RING);
+    if (g + 1 < steps.size() &&
+        (st = moe::cuda_check(cudaEventRecord(h->read_ev[r], ms), "streamed: record slot readers")))
+      return abort_call(st);
+    for (int i = 0; i < n; ++i) h->slot_read[static_cast<size_t>(layer) * h->S + sl[i]] = h->read_seq;
+    ++h->read_seq;
   }
   // lookahead prefetch (part of the call's transaction): the copies follow
   // the call's expert kernels on the side stream, since a victim slot may be
