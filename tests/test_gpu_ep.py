@@ -138,3 +138,41 @@ def test_ep_process_group_one_rank(M):
         r.close()
     finally:
         dist.destroy_process_group()
+
+
+def test_ep_layer_replays_from_a_cuda_graph(M):
+    """The whole expert-parallel layer of 2 local ranks captured in one CUDA
+    graph (no host synchronisation inside) replays bit for bit like the
+    eager calls."""
+    from quantized_moe_bit_b200 import ep
+    G = 2
+    cfg = tiny_config("prefill_1L_128tok", T=6)
+    hl = HostLayer(cfg, 0)
+    dl = hl.upload()
+    ranks = [ep.EpRank(G, r, cfg.T, cfg.H, cfg.I, cfg.Is, cfg.E, cfg.k, dl) for r in range(G)]
+    comm = ep.LocalRanks(ranks)
+    zs = [torch.from_numpy(gen.rows(cfg.seed, 1000 + g, cfg.T, cfg.H)).cuda() for g in range(G)]
+    hs = [z.clone() for z in zs]
+    ep.ep_layer_forward(ranks, comm, hs)
+    M.moe_sync()
+    want = [(_np(h), _bits(r.y)) for h, r in zip(hs, ranks)]
+    hs_g = [z.clone() for z in zs]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):                       # warm-up outside the capture
+        ep.ep_layer_forward(ranks, comm, hs_g)
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        ep.ep_layer_forward(ranks, comm, hs_g)
+    for _ in range(2):
+        for h, z in zip(hs_g, zs):
+            h.copy_(z)
+        graph.replay()
+        torch.cuda.synchronize()
+        M.moe_sync()
+        for (h_w, y_w), h, r in zip(want, hs_g, ranks):
+            assert np.array_equal(_np(h), h_w) and np.array_equal(_bits(r.y), y_w)
+    del graph
+    for r in ranks:
+        r.close()
