@@ -174,8 +174,8 @@ class EpComm:
 
     def barrier(self):
         # stream-ordered on NCCL: later kernels on the stream start after
-        # every rank's earlier ones have finished
-        dist.all_reduce(self._one, group=self.group)
+        # every rank's earlier ones have finished (MAX keeps the word at 1)
+        dist.all_reduce(self._one, op=dist.ReduceOp.MAX, group=self.group)
 
     def exchange_handles(self, rank: EpRank):
         out = [None] * self.world
