@@ -491,14 +491,16 @@ def whole_job_rate(ms: float, steps: int, world: int) -> float:
 def run_reference(args, rank, world):
     """The oracle as it stands, on the host cores (rank 0 only): each step is
     one fresh token of the 30-layer batch-1 workload through its first
-    REF_LAYERS layers; every routed expert of those layers is generated
-    before the first timed step.  value = tokens/s of the whole 30-layer step
-    (the sample's layers / 30 tokens per step time)."""
+    layers (3, or fewer for long runs); every routed expert of those layers
+    is generated before the first timed step.  value = tokens/s of the whole
+    30-layer step (the sample's layers / 30 tokens per step time)."""
     if rank != 0:
         return
     from oracle import moe_oracle as O
     cfg = CFG
-    n_layers = 3
+    # layers per step: 3, fewer when many steps are asked for, so that the
+    # whole run stays near two minutes (about 0.6 s of oracle per layer)
+    n_layers = max(1, min(3, int(120.0 / (0.6 * max(1, args.steps + args.warmup)))))
     ol = OracleLayers(cfg, n_layers)
     ol.generate_all()
     times = []
