@@ -4,10 +4,12 @@ Rank d owns routed experts [d E/G, (d+1) E/G); every rank keeps its own
 tokens and runs its own norm, router, bucketing, shared expert and combine.
 Per layer (`ep_layer_forward`):
 
-    front      moe_rmsnorm, moe_router_topk, moe_bucket, moe_shared_forward
+    front      moe_rmsnorm, moe_router_topk, moe_bucket
     gather     every rank's bucket offsets into all_offsets [G, E+1]
     dispatch   moe_ep_dispatch: input rows stored into the owners' recv_x
                (and the rank's own receiver plan written)
+    shared     moe_shared_forward (before the barrier: a rank's shared expert
+               runs while slower ranks still dispatch)
     barrier
     experts    moe_expert_forward (k = 1, E/G experts) over the received rows,
                moe_ep_return: output rows stored into the sources' y_pairs
@@ -138,7 +140,9 @@ class EpRank:
         B.moe_rmsnorm(h, self.x)
         B.moe_router_topk(self.x, L.router.c, L.bias, 0, self.E, self.k, self.idx, self.gates)
         B.moe_bucket(self.idx, self.E, self.offsets, self.pairs, self.active, self.n_active)
-        B.moe_shared_forward(self.x, self.Is, L.shared_c, self.ysh, self.ws_s, flags=flags)
+
+    def shared(self, flags: int = 0):
+        B.moe_shared_forward(self.x, self.Is, self.layer.shared_c, self.ysh, self.ws_s, flags=flags)
 
     def dispatch(self):
         B.moe_ep_dispatch(self.x, self.k, self.E, self.G, self.rank, self.idx, self.pairs, self.all_off,
@@ -222,6 +226,8 @@ def ep_layer_forward(ranks: Sequence[EpRank], comm, hs: Sequence[torch.Tensor], 
     comm.gather_offsets(ranks)
     for r in ranks:
         r.dispatch()
+    for r in ranks:
+        r.shared(flags)
     comm.barrier()
     for r in ranks:
         r.experts(flags)

@@ -53,7 +53,7 @@ def main():
         torch.cuda._sleep(20_000_000)
         for r, h in zip(ranks, hh):
             e0, e1 = ev(), ev()
-            e0.record(); r.front(h); e1.record()
+            e0.record(); r.front(h); r.shared(); e1.record()
             spans["front"].append((e0, e1))
         comm.gather_offsets(ranks)
         for r in ranks:

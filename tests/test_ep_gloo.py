@@ -49,7 +49,7 @@ class HostEpRank:
         self.layer = l
         self.router = gen.router_weights(c.seed, l, c.E, c.H)
         self.bias = gen.zipf_bias(c.seed, l, c.E) if c.zipf else None
-        self.shared = gen.shared_weights(c.seed, l, c.H, c.Is)
+        self.shared_w = gen.shared_weights(c.seed, l, c.H, c.Is)
 
     def front(self, h, flags=0):
         c = self.c
@@ -59,7 +59,9 @@ class HostEpRank:
         self.gates = O.softmax_gates(lg, self.idx)
         off, self.pairs, _ = O.buckets(self.idx, c.E)
         self.offsets.copy_(torch.from_numpy(off))
-        self.ysh = O.mlp(self.x, *self.shared)
+
+    def shared(self, flags=0):
+        self.ysh = O.mlp(self.x, *self.shared_w)
 
     def _row(self, s, e, i):
         """Receiver row of slot i of source s's bucket e (the header's layout)."""
@@ -128,7 +130,7 @@ def _worker(rank, world, port, recv_x, recv_meta, y_pairs, q):
             ep.ep_layer_forward([r], comm, [h])
             _, x = O.rmsnorm(want)
             res = O.layer_forward(x, r.router, r.bias, lambda e, l=l: gen.expert_weights(c.seed, l, e, c.H, c.I),
-                                  r.shared, c.k, c.E)
+                                  r.shared_w, c.k, c.E)
             want = want + res["out"]
         q.put((rank, float(np.abs(h.numpy() - want).max()), float(np.abs(want).max())))
     finally:
