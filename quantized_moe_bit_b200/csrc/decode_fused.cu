@@ -722,10 +722,13 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
   unsigned* abort_word = a.counter + 32;          // own 128-byte line
   unsigned bar_target = 0;
   auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  // The CTA barrier orders every thread's writes before thread 0's release
+  // add, and thread 0's acquire poll before every thread's reads after the
+  // second CTA barrier; release and acquire are cumulative, so no separate
+  // fences (the data crossing CTAs is read through L2).
   auto grid_sync = [&]() {
     __syncthreads();
     if (threadIdx.x == 0) {
-      __threadfence();
       bar_target += static_cast<unsigned>(G);
       red_release_gpu(a.counter, 1u);
       const uint64_t t0 = df_clock();
@@ -733,7 +736,6 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
         __nanosleep(32);
         if (df_clock() - t0 > 2000000000ull) { flag_check(CHECK_WAIT); break; }
       }
-      __threadfence();
     }
     __syncthreads();
   };
