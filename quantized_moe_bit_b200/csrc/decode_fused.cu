@@ -411,16 +411,17 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
 __device__ __forceinline__ void red_release_gpu(unsigned* p, unsigned v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
-// tagged words: release stores, relaxed polls closed by an acquire fence
-__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
-  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+// tagged words: the 64-bit word carries its value and its layer tag and no
+// other data travels with it, so relaxed stores and relaxed polls suffice
+// (one single-copy-atomic word; a reader that sees the tag has the value)
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
   unsigned long long v;
   asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
-__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ uint64_t df_clock() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -889,7 +890,7 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
         }
         acc = warp_sum(acc);
         if (lane == 0)
-          st_release_u64(a.logits + c, (static_cast<unsigned long long>(l + 1) << 32) | __float_as_uint(acc + bias_c));
+          st_relaxed_u64(a.logits + c, (static_cast<unsigned long long>(l + 1) << 32) | __float_as_uint(acc + bias_c));
       }
     } else {
       // warp w < 11: groups [w*NGH/11, (w+1)*NGH/11) of every shared gate/up tile
@@ -937,7 +938,6 @@ __global__ void __launch_bounds__(DF_THREADS, 1) k_decode_b1(const __grid_consta
         __nanosleep(20);
         v = ld_relaxed_u64(a.logits + e);
       }
-      fence_acq_rel_gpu();
       lg[e] = __uint_as_float(static_cast<uint32_t>(v));
     }
     __syncthreads();
