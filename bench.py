@@ -55,7 +55,7 @@ def peaks():
 # DRAM read + write of the decode kernel measured by ncu on 3 full-size
 # layers of this workload, per layer; valid only for the kernel source the
 # capture was taken on (sha256 prefix of decode_fused.cu).
-DECODE_TRAFFIC = {"source_sha256_prefix": "96c47764376e60a3", "bytes_per_layer": 39.0954e6}
+DECODE_TRAFFIC = {"source_sha256_prefix": "0b3e112df90c7b80", "bytes_per_layer": 38.7517e6}
 
 
 def decode_traffic(layers: int):
