@@ -588,26 +588,44 @@ def run_ours(args, rank, world, local_rank):
     idx_last = idx_tr.cpu().numpy()
     distinct = float(np.mean([len(set(idx_last[l, 0].tolist())) for l in range(cfg.layers)]))
 
-    # end to end through the public call, one token at a time: the row is
-    # copied in from pinned host memory, moe_decode_forward runs (an eager
-    # C-ABI call: argument checks and launch inside the timed region), the
-    # residual row is copied back and the host waits for it
+    # end to end through the public C-ABI, one token at a time from host
+    # memory to host memory: moe_decode_session_step copies the row in, runs
+    # the 30 layers, copies the row out and waits for it (one C call per
+    # token; events on the session's stream bracket the whole loop)
     zh = torch.from_numpy(z[args.warmup:]).pin_memory().view(args.steps, 1, H)
     out_h = torch.empty((args.steps, 1, H), dtype=torch.float32).pin_memory()
-    cur = torch.cuda.current_stream()
+    h_sess = torch.empty((1, H), dtype=torch.float32, device=device)
+    sess = M.DecodeSession(h_sess, cfg.I, cfg.Is, cfg.E, cfg.k, stack, ws)
+    sstream = torch.cuda.ExternalStream(sess.stream, device=device)
+    for i in range(3):
+        sess.step(zh[i].data_ptr(), out_h[i].data_ptr())
     torch.cuda.synchronize()
     barrier()
     e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2.record()
+    e2.record(sstream)
+    for i in range(args.steps):
+        sess.step(zh[i].data_ptr(), out_h[i].data_ptr())
+    e3.record(sstream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = e2.elapsed_time(e3)
+    sess.close()
+    # the same through the eager moe_decode_forward call with torch copies of
+    # the row and a host wait per token (argument checks and launch inside)
+    cur = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    barrier()
+    e6, e7 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e6.record()
     for i in range(args.steps):
         h.copy_(zh[i], non_blocking=True)
         step()
         out_h[i].copy_(h, non_blocking=True)
         cur.synchronize()
-    e3.record()
+    e7.record()
     torch.cuda.synchronize()
     barrier()
-    ms_e2e = e2.elapsed_time(e3)
+    ms_eager = e6.elapsed_time(e7)
     # the same with the step replayed from a CUDA graph and no host wait
     # between tokens (copies and steps queued back to back)
     e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -622,7 +640,7 @@ def run_ours(args, rank, world, local_rank):
     ms_pipe = e4.elapsed_time(e5)
     M.moe_sync()
 
-    ms, ms_e2e, ms_pipe = max_over_ranks([ms, ms_e2e, ms_pipe], world, device)
+    ms, ms_e2e, ms_pipe, ms_eager = max_over_ranks([ms, ms_e2e, ms_pipe, ms_eager], world, device)
     del g
     if rank != 0:
         return
@@ -655,8 +673,12 @@ def run_ours(args, rank, world, local_rank):
                      "peak_source": src, "traffic": decode_traffic(cfg.layers), "bytes_per_step": bytes_step,
                      "distinct_experts_per_layer": distinct},
         "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": H * 4, "d2h_bytes_per_step": H * 4,
-                "mode": "one token per call: pinned row copied in, eager moe_decode_forward, row copied out, "
-                        "host waits for it"},
+                "mode": "one token per C-ABI call (moe_decode_session_step): host row copied in, 30 layers, row "
+                        "copied out, host waits for it"},
+        "e2e_eager": {"value": whole_job_rate(ms_eager, args.steps, world), "unit": "tokens/s",
+                      "h2d_bytes_per_step": H * 4, "d2h_bytes_per_step": H * 4,
+                      "mode": "one token per eager moe_decode_forward call with torch copies of the row in and "
+                              "out and a host wait"},
         "e2e_pipelined": {"value": whole_job_rate(ms_pipe, args.steps, world), "unit": "tokens/s",
                           "h2d_bytes_per_step": H * 4, "d2h_bytes_per_step": H * 4,
                           "mode": "graph replay per token, copies in and out queued, no host wait between tokens"},

@@ -309,6 +309,35 @@ MOE_API int moe_decode_forward(float* h, int T, int H, int I, int Is, int E, int
                                int32_t* idx_trace, float* gates_trace, void* ws,
                                size_t ws_bytes, int flags, void* stream);
 
+/* Decode session: one batch-1 step per call from host memory to host memory,
+ * the way a server calls the layer stack token by token.  Created once with
+ * the arguments of moe_decode_forward (T = 1; checked once, here); every
+ * step copies the token's residual row in, runs the L layers, copies the row
+ * out and waits for it.  The copies and the launches are one CUDA graph
+ * (instantiated at creation on the session's own stream) between two
+ * pinned staging rows of the session.
+ *   h_dev     fp32 [1,H] (device): the row the layers update (owned by the caller)
+ *   routers .. ws, flags   as moe_decode_forward (they must stay valid for
+ *             the session's life; the graph holds their addresses)
+ *   out       receives the session handle
+ * moe_decode_session_step:
+ *   h_in      fp32 [H] host (any host memory): the step's input row
+ *   h_out     fp32 [H] host: the residual row after the L layers (may equal h_in)
+ *   returns after the row is back; a device check (bounded waits, ids) is
+ *   reported by the next moe_sync
+ * moe_decode_session_stream: the session's CUDA stream (for events).
+ * Errors: creation fails with the codes of moe_decode_forward, before any
+ * launch; a step fails with MOE_ERR_CUDA. */
+typedef struct moe_decode_session moe_decode_session;
+MOE_API int moe_decode_session_create(float* h_dev, int H, int I, int Is, int E, int k, int L,
+                                      const moe_qmat* routers, const float* const* biases,
+                                      int bias_per_row, const void* const* const* blob_tables,
+                                      const moe_qmat* shared, void* ws, size_t ws_bytes, int flags,
+                                      moe_decode_session** out);
+MOE_API int moe_decode_session_step(moe_decode_session* s, const float* h_in, float* h_out);
+MOE_API void* moe_decode_session_stream(moe_decode_session* s);
+MOE_API int moe_decode_session_destroy(moe_decode_session* s);
+
 /* ------------------------------------------------------------------------
  * Per-layer LFU expert-slot cache (routed experts streamed from pinned host
  * memory).  "TurboFieldfare: Gemma 4 26B on an 8 GB MacBook, in ~2 GB of

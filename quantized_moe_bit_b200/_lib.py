@@ -59,6 +59,12 @@ SIGNATURES = {
     "moe_decode_grid": (_I, []),
     "moe_decode_forward": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, C.POINTER(moe_qmat), C.POINTER(C.c_void_p), _I,
                                 C.POINTER(C.c_void_p), C.POINTER(moe_qmat), _P, _P, _P, _P, _P, _Z, _I, _P]),
+    "moe_decode_session_create": (_I, [_P, _I, _I, _I, _I, _I, _I, C.POINTER(moe_qmat), C.POINTER(C.c_void_p), _I,
+                                       C.POINTER(C.c_void_p), C.POINTER(moe_qmat), _P, _Z, _I,
+                                       C.POINTER(C.c_void_p)]),
+    "moe_decode_session_step": (_I, [_P, _P, _P]),
+    "moe_decode_session_stream": (_P, [_P]),
+    "moe_decode_session_destroy": (_I, [_P]),
     "moe_lfu_create": (_I, [_I, _I, _I, _Z, _P, _P, _Z, C.POINTER(C.c_void_p)]),
     "moe_lfu_plan": (_I, [_P, _I, _P, _I, _P, _P]),
     "moe_lfu_step": (_I, [_P, _I, _P, _I, _P, _P, _P, _P, _I]),

@@ -142,6 +142,43 @@ def moe_decode_forward(h, I: int, Is: int, E: int, k: int, stack: "DecodeStack",
                                    flags, stream_ptr(stream)))
 
 
+class DecodeSession:
+    """moe_decode_session_*: batch-1 steps from host rows to host rows (the
+    arguments marshalled once; a step is one C call)."""
+
+    def __init__(self, h_dev, I: int, Is: int, E: int, k: int, stack: "DecodeStack", ws, flags: int = 0):
+        H = h_dev.shape[-1]
+        self._refs = (h_dev, stack, ws)
+        hnd = C.c_void_p()
+        check(lib().moe_decode_session_create(ptr(h_dev), H, I, Is, E, k, stack.L, stack.routers, stack.biases,
+                                              stack.bias_per_row, stack.tables, stack.shared, ptr(ws),
+                                              ws.numel() * ws.element_size(), flags, C.byref(hnd)))
+        self._h = hnd.value
+        self._step = lib().moe_decode_session_step
+
+    @property
+    def stream(self) -> int:
+        return lib().moe_decode_session_stream(self._h)
+
+    def step(self, h_in, h_out):
+        """h_in, h_out: host addresses (ints) or CPU tensors of H fp32."""
+        st = self._step(self._h, h_in if isinstance(h_in, int) else h_in.data_ptr(),
+                        h_out if isinstance(h_out, int) else h_out.data_ptr())
+        if st:
+            check(st)
+
+    def close(self):
+        if self._h:
+            check(lib().moe_decode_session_destroy(self._h))
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
 # ------------------------------------------------------------------ LFU cache
 class MoeLfu:
     """Handle of the per-layer LFU expert-slot cache (moe_lfu_* calls)."""

@@ -745,4 +745,98 @@ int moe_decode_forward(float* h, int T, int H, int I, int Is, int E, int k, int 
   return MOE_OK;
 }
 
+// ------------------------------------------------------------ decode session
+struct moe_decode_session {
+  int H = 0;
+  cudaStream_t stream = nullptr;
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  float* pin_in = nullptr;
+  float* pin_out = nullptr;
+};
+
+int moe_decode_session_destroy(moe_decode_session* s) {
+  if (!s) return MOE_OK;
+  if (s->stream) cudaStreamSynchronize(s->stream);
+  if (s->exec) cudaGraphExecDestroy(s->exec);
+  if (s->graph) cudaGraphDestroy(s->graph);
+  if (s->pin_in) cudaFreeHost(s->pin_in);
+  if (s->pin_out) cudaFreeHost(s->pin_out);
+  if (s->stream) cudaStreamDestroy(s->stream);
+  delete s;
+  return MOE_OK;
+}
+
+int moe_decode_session_create(float* h_dev, int H, int I, int Is, int E, int k, int L, const moe_qmat* routers,
+                              const float* const* biases, int bias_per_row, const void* const* const* blob_tables,
+                              const moe_qmat* shared, void* ws, size_t ws_bytes, int flags, moe_decode_session** out) {
+  if (!out) return fail(MOE_ERR_INVALID_ARG, "moe_decode_session_create: NULL out");
+  *out = nullptr;
+  int st = check_dims(1, H, I, E, k);
+  if (st) return st;
+  if ((st = check_dims(1, H, Is, E, k))) return st;
+  if ((st = check_flags(flags))) return st;
+  if (L <= 0) return fail(MOE_ERR_INVALID_ARG, "moe_decode_session_create: L must be > 0");
+  if (!h_dev || !routers || !blob_tables || !shared || !ws)
+    return fail(MOE_ERR_INVALID_ARG, "moe_decode_session_create: NULL pointer");
+  if (!aligned16(h_dev)) return fail(MOE_ERR_INVALID_ARG, "moe_decode_session_create: h_dev must be 16-byte aligned");
+  if (ws_bytes < moe_decode_workspace_size(1, H, I, Is, E, k))
+    return fail(MOE_ERR_INVALID_ARG, "moe_decode_session_create: workspace too small");
+  for (int l = 0; l < L; ++l) {
+    const moe_qmat& R = routers[l];
+    if (!R.q || !R.s || !R.b || R.bits != 8 || R.out != E || R.in != H)
+      return fail(MOE_ERR_INVALID_ARG, "moe_decode_session_create: router %d must be 8-bit [E, H]", l);
+    if ((st = check_shared_mats(shared + 3 * l, H, Is))) return st;
+  }
+  moe_decode_session* s = new moe_decode_session();
+  s->H = H;
+  const size_t nb = static_cast<size_t>(H) * sizeof(float);
+  if ((st = cuda_check(cudaStreamCreateWithFlags(&s->stream, cudaStreamNonBlocking), "session stream")) ||
+      (st = cuda_check(cudaHostAlloc(reinterpret_cast<void**>(&s->pin_in), nb, cudaHostAllocDefault), "session pinned")) ||
+      (st = cuda_check(cudaHostAlloc(reinterpret_cast<void**>(&s->pin_out), nb, cudaHostAllocDefault), "session pinned"))) {
+    moe_decode_session_destroy(s);
+    return st;
+  }
+  // the kernels load their code and attributes before the capture
+  if ((st = moe_decode_forward(h_dev, 1, H, I, Is, E, k, L, routers, biases, bias_per_row, blob_tables, shared,
+                               nullptr, nullptr, nullptr, nullptr, ws, ws_bytes, flags, s->stream)) ||
+      (st = cuda_check(cudaStreamSynchronize(s->stream), "session warm-up"))) {
+    moe_decode_session_destroy(s);
+    return st;
+  }
+  if ((st = cuda_check(cudaStreamBeginCapture(s->stream, cudaStreamCaptureModeThreadLocal), "session capture"))) {
+    moe_decode_session_destroy(s);
+    return st;
+  }
+  int cst = cuda_check(cudaMemcpyAsync(h_dev, s->pin_in, nb, cudaMemcpyHostToDevice, s->stream), "session copy in");
+  if (!cst)
+    cst = moe_decode_forward(h_dev, 1, H, I, Is, E, k, L, routers, biases, bias_per_row, blob_tables, shared,
+                             nullptr, nullptr, nullptr, nullptr, ws, ws_bytes, flags, s->stream);
+  if (!cst) cst = cuda_check(cudaMemcpyAsync(s->pin_out, h_dev, nb, cudaMemcpyDeviceToHost, s->stream), "session copy out");
+  st = cuda_check(cudaStreamEndCapture(s->stream, &s->graph), "session end capture");
+  if (cst || st) {
+    moe_decode_session_destroy(s);
+    return cst ? cst : st;
+  }
+  if ((st = cuda_check(cudaGraphInstantiate(&s->exec, s->graph, 0), "session instantiate"))) {
+    moe_decode_session_destroy(s);
+    return st;
+  }
+  *out = s;
+  return MOE_OK;
+}
+
+int moe_decode_session_step(moe_decode_session* s, const float* h_in, float* h_out) {
+  if (!s || !s->exec || !h_in || !h_out) return fail(MOE_ERR_INVALID_ARG, "moe_decode_session_step: NULL pointer");
+  const size_t nb = static_cast<size_t>(s->H) * sizeof(float);
+  memcpy(s->pin_in, h_in, nb);
+  int st = cuda_check(cudaGraphLaunch(s->exec, s->stream), "session step launch");
+  if (st) return st;
+  if ((st = cuda_check(cudaStreamSynchronize(s->stream), "session step"))) return st;
+  memcpy(h_out, s->pin_out, nb);
+  return MOE_OK;
+}
+
+void* moe_decode_session_stream(moe_decode_session* s) { return s ? static_cast<void*>(s->stream) : nullptr; }
+
 }  // extern "C"

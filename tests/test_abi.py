@@ -192,3 +192,26 @@ def test_expert_parallel_argument_checks():
     assert L.moe_ipc_handle_bytes() == 64
     assert L.moe_ipc_open(None, None) == _INVALID
     assert L.moe_device_alloc(0, C.byref(C.c_void_p())) == _INVALID
+
+
+def test_decode_session_argument_checks():
+    from quantized_moe_bit_b200 import _lib
+    L = _lib.lib()
+    f = _FAKE
+    H, I, Is, E, k = 2816, 704, 2112, 128, 8
+    r = _q(E, H, 8)
+    routers = (_lib.moe_qmat * 1)(r)
+    sh = (_lib.moe_qmat * 3)(_q(Is, H, 4), _q(Is, H, 4), _q(H, Is, 4))
+    blobs = (C.c_void_p * 1)(f)
+    out = C.c_void_p()
+    dws = L.moe_decode_workspace_size(1, H, I, Is, E, k)
+    args = [f, H, I, Is, E, k, 1, routers, None, 0, blobs, sh, f, dws, 0]
+    assert L.moe_decode_session_create(*args, None) == _INVALID                          # no out
+    assert L.moe_decode_session_create(*args[:6], 0, *args[7:], C.byref(out)) == _INVALID  # L = 0
+    assert L.moe_decode_session_create(*args[:13], dws - 1, 0, C.byref(out)) == _INVALID  # workspace
+    assert L.moe_decode_session_create(f + 4, *args[1:], C.byref(out)) == _INVALID        # misaligned h
+    bad = (_lib.moe_qmat * 1)(_q(E, H, 4))
+    assert L.moe_decode_session_create(*args[:7], bad, *args[8:], C.byref(out)) == _INVALID  # 4-bit router
+    assert out.value is None
+    assert L.moe_decode_session_step(None, f, f) == _INVALID
+    assert L.moe_decode_session_destroy(None) == _OK

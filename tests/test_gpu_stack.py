@@ -106,6 +106,9 @@ def test_decode_30L_b1_full(M):
         if step == 7:
             g2 = _run_stack(M, cfg, layers, z, traces=False)
             assert np.array_equal(g2["h"], g["h"])
+    # the decode session (host row in, host row out, one C call per step)
+    # gives the same residual rows as the kernel above, step after step
+    _check_session(M, cfg, layers, steps=3)
 
 
 def test_decode_30L_b64_full(M):
@@ -140,6 +143,30 @@ def test_stack_tiny_b1_fused_and_layered(M):
     g_idx = _run_stack(M, cfg, layers, z, traces="idx")
     assert np.array_equal(g_none["h"], gf["h"]) and np.array_equal(g_idx["h"], gf["h"])
     assert np.array_equal(g_idx["idx"], gf["idx"])
+
+
+def _check_session(M, cfg, layers, steps):
+    import quantized_moe_bit_b200 as MM
+    stack = MM.DecodeStack(layers)
+    ws = torch.empty(M.moe_decode_workspace_size(1, cfg.H, cfg.I, cfg.Is, cfg.E, cfg.k), dtype=torch.uint8,
+                     device="cuda")
+    h_dev = torch.empty((1, cfg.H), dtype=torch.float32, device="cuda")
+    sess = MM.DecodeSession(h_dev, cfg.I, cfg.Is, cfg.E, cfg.k, stack, ws)
+    out = torch.empty(cfg.H, dtype=torch.float32).pin_memory()
+    for step in range(steps):
+        z = gen.rows(cfg.seed, cfg.row_stream + 100 + step, 1, cfg.H)
+        zin = torch.from_numpy(z[0].copy())
+        sess.step(zin, out)
+        h = torch.from_numpy(z).cuda()
+        M.moe_decode_forward(h, cfg.I, cfg.Is, cfg.E, cfg.k, stack, ws)
+        M.moe_sync()
+        assert np.array_equal(out.numpy(), h.cpu().numpy()[0]), step
+    sess.close()
+
+
+def test_decode_session_tiny(M):
+    cfg = tiny_config("decode_30L_b1", layers=4, T=1)
+    _check_session(M, cfg, upload_stack(cfg), steps=4)
 
 
 def test_fused_launch_count(M):
