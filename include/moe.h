@@ -326,6 +326,8 @@ MOE_API int moe_decode_forward(float* h, int T, int H, int I, int Is, int E, int
  *   returns after the row is back; a device check (bounded waits, ids) is
  *   reported by the next moe_sync
  * moe_decode_session_stream: the session's CUDA stream (for events).
+ * A session is used by one thread at a time (its staging rows are shared
+ * by its steps); creation runs one warm-up step on a zeroed h_dev.
  * Errors: creation fails with the codes of moe_decode_forward, before any
  * launch; a step fails with MOE_ERR_CUDA. */
 typedef struct moe_decode_session moe_decode_session;

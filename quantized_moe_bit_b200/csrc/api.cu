@@ -797,8 +797,10 @@ int moe_decode_session_create(float* h_dev, int H, int I, int Is, int E, int k, 
     moe_decode_session_destroy(s);
     return st;
   }
-  // the kernels load their code and attributes before the capture
-  if ((st = moe_decode_forward(h_dev, 1, H, I, Is, E, k, L, routers, biases, bias_per_row, blob_tables, shared,
+  // the kernels load their code and attributes before the capture (on a
+  // zero row: whatever h_dev held, the warm-up then routes validly)
+  if ((st = cuda_check(cudaMemsetAsync(h_dev, 0, nb, s->stream), "session zero row")) ||
+      (st = moe_decode_forward(h_dev, 1, H, I, Is, E, k, L, routers, biases, bias_per_row, blob_tables, shared,
                                nullptr, nullptr, nullptr, nullptr, ws, ws_bytes, flags, s->stream)) ||
       (st = cuda_check(cudaStreamSynchronize(s->stream), "session warm-up"))) {
     moe_decode_session_destroy(s);
