@@ -215,3 +215,19 @@ def test_decode_session_argument_checks():
     assert out.value is None
     assert L.moe_decode_session_step(None, f, f) == _INVALID
     assert L.moe_decode_session_destroy(None) == _OK
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/moe.h compiles as C99 with warnings as errors (the boundary
+    carries no C++ or torch types)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        import pytest
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "moe.h"\nint main(void) { return moe_version() > 0 ? 0 : 1; }\n')
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-I",
+                        os.path.join(ROOT, "include"), str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
