@@ -176,3 +176,26 @@ def test_ep_layer_replays_from_a_cuda_graph(M):
     del graph
     for r in ranks:
         r.close()
+
+
+def test_ep_exportable_buffers_one_rank(M):
+    """A rank whose receive buffers are whole device allocations exportable
+    by CUDA IPC (moe_device_alloc): the layer runs on them, their IPC
+    handles are produced, and close() frees them."""
+    from quantized_moe_bit_b200 import ep
+    cfg = tiny_config("prefill_1L_128tok", T=4, E=64)
+    hl = HostLayer(cfg, 0)
+    dl = hl.upload()
+    r = ep.EpRank(1, 0, cfg.T, cfg.H, cfg.I, cfg.Is, cfg.E, cfg.k, dl, exportable=True)
+    handles = r.ipc_handles()
+    assert len(handles) == 3 and all(len(h) == 64 for h in handles)
+    comm = ep.LocalRanks([r])
+    z = gen.rows(cfg.seed, 1000, cfg.T, cfg.H)
+    h = torch.from_numpy(z).cuda()
+    ep.ep_layer_forward([r], comm, [h])
+    M.moe_sync()
+    x = O.bf16_to_f64(_bits(r.x))
+    ref = O.layer_forward(x, hl.router, hl.bias, hl.expert, hl.shared, cfg.k, cfg.E, idx=_np(r.idx))
+    check_output(_bits(r.y), ref["out"], "y")
+    r.close()
+    assert r._raw == []
