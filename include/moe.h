@@ -310,7 +310,10 @@ MOE_API int moe_decode_forward(float* h, int T, int H, int I, int Is, int E, int
                                size_t ws_bytes, int flags, void* stream);
 
 /* Decode session: one batch-1 step per call from host memory to host memory,
- * the way a server calls the layer stack token by token.  Created once with
+ * the way a server calls the layer stack token by token.
+ * Source: "drumih/turbo-fieldfare" (paperfeed.app), section "How it works":
+ * each decode step walks the 30 layers; the step is moe_decode_forward's
+ * (T = 1), the session only holds its arguments and the row copies.  Created once with
  * the arguments of moe_decode_forward (T = 1; checked once, here); every
  * step copies the token's residual row in, runs the L layers, copies the row
  * out and waits for it.  The copies and the launches are one CUDA graph
