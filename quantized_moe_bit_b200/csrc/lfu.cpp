@@ -231,15 +231,20 @@ int plan_prefetch(moe_lfu* h, int layer, int P, std::vector<int32_t>& ids_out, s
   return MOE_OK;
 }
 
+// Bounded host wait for an event: polled without sleeping for the first
+// millisecond (the waits on the layer path -- routing, table copies -- end
+// within tens of microseconds, and a sleep of the thread overshoots by the
+// scheduler's timer slack), then with 20 us sleeps until timeout_ms.
 int wait_event(cudaEvent_t ev, int timeout_ms) {
   const auto t0 = std::chrono::steady_clock::now();
   while (true) {
     const cudaError_t e = cudaEventQuery(ev);
     if (e == cudaSuccess) return MOE_OK;
     if (e != cudaErrorNotReady) return moe::cuda_check(e, "lfu: event query");
-    if (std::chrono::steady_clock::now() - t0 > std::chrono::milliseconds(timeout_ms))
+    const auto waited = std::chrono::steady_clock::now() - t0;
+    if (waited > std::chrono::milliseconds(timeout_ms))
       return moe::fail(MOE_ERR_TIMEOUT, "lfu: wait ran out after %d ms", timeout_ms);
-    std::this_thread::sleep_for(std::chrono::microseconds(20));
+    if (waited > std::chrono::milliseconds(1)) std::this_thread::sleep_for(std::chrono::microseconds(20));
   }
 }
 
